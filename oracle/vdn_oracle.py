@@ -1,0 +1,363 @@
+"""Plain fp64 CPU oracle for the Video DeltaNet hybrid attention core.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
+and the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may
+import this module.  The product path (the CUDA library and its Python
+binding) never calls it and shares no code with it.
+
+Every function computes the method *as the pages define it*, in float64, with
+NumPy's ``solve`` / ``@`` as the only library steps, so that a reader can
+check it against the pages by eye.  Nothing is blocked, fused or reordered.
+
+Sources (web pages on "Video DeltaNet: A Video-Native Hybrid Attention for
+Livestream Video Generation", arXiv 2609.20744):
+
+* [P1] PaperDaily digest "伯克利与Impossible视频生成:14.3秒视频6.70秒去噪"
+  (longzhangge.com), sections 二 (local window + anchors), 三 (bidirectional
+  states, half-text init, gates, RMSNorm), 四 (frame-wise joint write).
+* [P2] shd-paper.top abstract page of arXiv 2609.20744.
+* [P4] deepmagic.app post "生成比播放還快：Video DeltaNet 用 11 秒產出 14 秒
+  768p 影片", section "用兩條分支取代一條" (closed form, 4-way anchors).
+* [P5] aimodeling.com news "video-deltanet-h3-hybrid-attention", section
+  "The VDN split" (frame-wise (I+A) solve, non-expansive, saturation).
+* The page at juejin.cn (per-frame-independent kernel, K=3 window, optical
+  flow gate) contradicts the four others and is NOT followed.
+
+Readings taken where the pages are silent (each one is listed with its
+reason in the design notes of the repository):
+
+* alpha enters as the inherited state S_bar = alpha_t * S_{t-1};
+* both scan directions use the same alpha_t, beta, k, v of frame t;
+* anchor frames are an identity step of either scan (no write, no decay);
+* an anchor query frame reads S_init_f + S_init_b (its softmax already
+  sees every frame); ``anchor_read="chunk"`` gives the other reading;
+* the window is clipped at the sequence ends;
+* softmax scale defaults to 1/sqrt(d_k); RMSNorm is over d_v with eps;
+* gates are elementwise sigmoid(logit) over [.., d_v];
+* the output keeps the two gated branches apart on a size-2 axis
+  (slot 0 = softmax, slot 1 = linear), or sums them (out_mode=1).
+
+Parity: every function here is pinned by ``tests/test_oracle_pins.py``
+against closed forms, invariants, an independent least-squares route, brute
+force on tiny inputs, library routines and the pages' printed densities.
+The end-to-end output has no printed worked example on the pages (no page
+prints one), so the end-to-end *value* is pinned only through its parts.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+F64 = np.float64
+
+
+# ---------------------------------------------------------------------------
+# configuration
+# ---------------------------------------------------------------------------
+@dataclass(frozen=True)
+class Cfg:
+    """Problem sizes and switches.  Layouts used throughout:
+
+    q, k, v, gate_sm, gate_lin : [B, T, N, H, d]
+    beta : [B, T, N, H]     alpha : [B, T, H]
+    text_k, text_v : [B, L, H, d]   text_beta : [B, L, H]
+    """
+    B: int
+    T: int
+    N: int
+    H: int
+    d_k: int
+    d_v: int
+    L: int = 0
+    chunk: int = 5
+    anchors: int = 4          # 0 = none, 4 = 4-way first/last-frame anchors
+    softmax_scale: float = 0.0  # <= 0 -> 1/sqrt(d_k)
+    rms_eps: float = 1e-6
+    out_mode: int = 0         # 0 = [.., 2, d_v] slots, 1 = summed [.., d_v]
+
+    @property
+    def scale(self) -> float:
+        return self.softmax_scale if self.softmax_scale > 0 else 1.0 / np.sqrt(self.d_k)
+
+
+# ---------------------------------------------------------------------------
+# the hybrid mask  ([P1] 二; [P4] 用兩條分支取代一條; [P5] The VDN split)
+# ---------------------------------------------------------------------------
+def num_chunks(T: int, chunk: int) -> int:
+    """Chunks of `chunk` consecutive latent frames; a short last chunk if
+    T is not a multiple of the chunk size."""
+    return -(-T // chunk)
+
+
+def anchor_frames(T: int, anchors: int) -> tuple:
+    """The boundary anchors are the first and the last latent frame."""
+    if anchors == 0:
+        return ()
+    return tuple(sorted({0, T - 1}))
+
+
+def frame_mask(T: int, chunk: int = 5, anchors: int = 4) -> np.ndarray:
+    """allowed[tq, tk]: may a query in frame tq attend by softmax to a key in
+    frame tk?  A query chunk sees itself and its two neighbour chunks; every
+    frame sees the anchor frames and the anchor frames see every frame."""
+    c = np.arange(T) // chunk
+    allowed = np.abs(c[:, None] - c[None, :]) <= 1
+    for a in anchor_frames(T, anchors):
+        allowed[:, a] = True
+        allowed[a, :] = True
+    return allowed
+
+
+def token_mask(T: int, N: int, chunk: int = 5, anchors: int = 4) -> np.ndarray:
+    """The frame mask expanded to tokens (frame-major, N tokens per frame)."""
+    return np.kron(frame_mask(T, chunk, anchors), np.ones((N, N), dtype=bool)).astype(bool)
+
+
+def mask_density(T: int, chunk: int = 5, anchors: int = 4) -> float:
+    """Fraction of (query, key) video pairs kept on the softmax path."""
+    return float(frame_mask(T, chunk, anchors).mean())
+
+
+def window_frames(t: int, T: int, chunk: int = 5) -> tuple:
+    """[lo, hi): the frames of the query chunk and its two neighbours,
+    clipped to the sequence."""
+    c = t // chunk
+    return max(0, chunk * (c - 1)), min(T, chunk * (c + 2))
+
+
+# ---------------------------------------------------------------------------
+# Video Delta Attention  ([P1] 四; [P4] closed form; [P5] The VDN split)
+# ---------------------------------------------------------------------------
+def gram_write(K: np.ndarray, V: np.ndarray, beta: np.ndarray):
+    """A = sum_i beta_i k_i k_i^T  (d_k x d_k), the beta-weighted key Gram
+    matrix, and B = sum_i beta_i v_i k_i^T  (d_v x d_k), the value-key write
+    matrix, over the n tokens of one frame.  K [n, d_k], V [n, d_v], beta [n]."""
+    K = np.asarray(K, F64)
+    V = np.asarray(V, F64)
+    Kb = K * np.asarray(beta, F64)[:, None]
+    return K.T @ Kb, V.T @ Kb
+
+
+def vda_update(S_bar: np.ndarray, K: np.ndarray, V: np.ndarray, beta: np.ndarray) -> np.ndarray:
+    """The frame-wise joint write: the S that minimises
+        ||S - S_bar||_F^2 + sum_i beta_i ||S k_i - v_i||^2
+    over all tokens of the frame at once, i.e. the closed form
+        S = (S_bar + B)(I + A)^{-1}.
+    (I + A) is symmetric, so S^T solves (I + A) S^T = (S_bar + B)^T."""
+    A, Bw = gram_write(K, V, beta)
+    G = np.eye(A.shape[0]) + A
+    return np.linalg.solve(G, (np.asarray(S_bar, F64) + Bw).T).T
+
+
+def frame_map(K: np.ndarray, V: np.ndarray, beta: np.ndarray):
+    """The frame update written as an affine map of the inherited state:
+    S = S_bar M + C with M = (I + A)^{-1} and C = B M (the same closed form,
+    expanded).  Returned for intermediate-value checks."""
+    A, Bw = gram_write(K, V, beta)
+    M = np.linalg.solve(np.eye(A.shape[0]) + A, np.eye(A.shape[0]))
+    return M, Bw @ M
+
+
+def text_state(text_k: np.ndarray, text_v: np.ndarray, text_beta: np.ndarray, d_v: int, d_k: int) -> np.ndarray:
+    """Text is pre-written by one joint solve from the zero state over the L
+    text tokens ([P1] 三: the prompt is written into both states, half each).
+    Returns the full text state S_x; each direction starts from S_x / 2."""
+    if text_k is None or len(text_k) == 0:
+        return np.zeros((d_v, d_k))
+    return vda_update(np.zeros((d_v, d_k)), text_k, text_v, text_beta)
+
+
+def forward_states(S0, k, v, beta, alpha, anchors: int = 4) -> np.ndarray:
+    """Forward scan for one (batch, head).  k [T, N, d_k], v [T, N, d_v],
+    beta [T, N], alpha [T].  F[t] is the state that covers frames < t
+    (F[0] = S0); at a non-anchor frame the inherited state is alpha_t F[t]
+    and the frame is written jointly; anchor frames are not written."""
+    T = k.shape[0]
+    anc = set(anchor_frames(T, anchors))
+    F = np.empty((T + 1,) + np.shape(S0))
+    F[0] = S0
+    for t in range(T):
+        if t in anc:
+            F[t + 1] = F[t]
+        else:
+            F[t + 1] = vda_update(alpha[t] * F[t], k[t], v[t], beta[t])
+    return F
+
+
+def backward_states(S0, k, v, beta, alpha, anchors: int = 4) -> np.ndarray:
+    """Backward scan: G[t] covers frames >= t (G[T] = S0), built from the
+    last frame down with the same per-frame update."""
+    T = k.shape[0]
+    anc = set(anchor_frames(T, anchors))
+    G = np.empty((T + 1,) + np.shape(S0))
+    G[T] = S0
+    for t in range(T - 1, -1, -1):
+        if t in anc:
+            G[t] = G[t + 1]
+        else:
+            G[t] = vda_update(alpha[t] * G[t + 1], k[t], v[t], beta[t])
+    return G
+
+
+def read_state(F, G, t: int, T: int, chunk: int = 5, anchors: int = 4, anchor_read: str = "text"):
+    """The state a query in frame t reads: the forward state over the frames
+    before its window plus the backward state over the frames after it
+    ([P1] 三; [P4] the two regions do not overlap).  An anchor query frame
+    reads the two half-text initial states (anchor_read="text"), or its chunk
+    window like any other frame (anchor_read="chunk")."""
+    if anchor_read == "text" and t in anchor_frames(T, anchors):
+        return F[0] + G[T]
+    lo, hi = window_frames(t, T, chunk)
+    return F[lo] + G[hi]
+
+
+def read_table(F, G, T: int, chunk: int = 5, anchors: int = 4):
+    """Per query chunk c the summed read state, plus one entry (index C) for
+    the anchor query frames.  Returned for intermediate-value checks."""
+    C = num_chunks(T, chunk)
+    R = np.empty((C + 1,) + F.shape[1:])
+    for c in range(C):
+        lo, hi = window_frames(c * chunk, T, chunk)
+        R[c] = F[lo] + G[hi]
+    R[C] = F[0] + G[T]
+    return R
+
+
+def sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-np.asarray(x, F64)))
+
+
+def rms_gate(o, g, eps: float, weight=None):
+    """Linear-branch epilogue ([P1] 三): RMS-normalise over d_v, then the
+    content-dependent sigmoid gate.  o, g [..., d_v]."""
+    o = np.asarray(o, F64)
+    r = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    if weight is not None:
+        r = r * np.asarray(weight, F64)
+    return sigmoid(g) * r
+
+
+# ---------------------------------------------------------------------------
+# softmax branch  ([P1] 二; [P4]; [P5])
+# ---------------------------------------------------------------------------
+def softmax_attend(q, keys, vals, scale: float):
+    """Plain softmax attention of queries q [n, d_k] over keys [m, d_k]."""
+    s = scale * (np.asarray(q, F64) @ np.asarray(keys, F64).T)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ np.asarray(vals, F64)
+
+
+def softmax_frame(q_t, k_bh, v_bh, t: int, T: int, chunk: int, anchors: int, scale: float):
+    """Softmax output for the queries of frame t of one (batch, head):
+    keys are the tokens of every frame the frame mask allows."""
+    allowed = np.nonzero(frame_mask(T, chunk, anchors)[t])[0]
+    keys = k_bh[allowed].reshape(-1, k_bh.shape[-1])
+    vals = v_bh[allowed].reshape(-1, v_bh.shape[-1])
+    return softmax_attend(q_t, keys, vals, scale)
+
+
+def softmax_dense_masked(q_bh, k_bh, v_bh, T, N, chunk, anchors, scale):
+    """Dense attention over all T*N video tokens with the explicit token mask
+    (masked logits = -inf).  Only for small sizes."""
+    Q = np.asarray(q_bh, F64).reshape(T * N, -1)
+    K = np.asarray(k_bh, F64).reshape(T * N, -1)
+    V = np.asarray(v_bh, F64).reshape(T * N, -1)
+    s = scale * (Q @ K.T)
+    s = np.where(token_mask(T, N, chunk, anchors), s, -np.inf)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return (p @ V).reshape(T, N, -1)
+
+
+# ---------------------------------------------------------------------------
+# the whole core
+# ---------------------------------------------------------------------------
+def head_states(inp: dict, cfg: Cfg, b: int, h: int):
+    """F, G (forward / backward states for every frame boundary) of one
+    (batch, head), both started from half the text state."""
+    if cfg.L > 0 and inp.get("text_k") is not None:
+        Sx = text_state(inp["text_k"][b, :, h], inp["text_v"][b, :, h], inp["text_beta"][b, :, h],
+                        cfg.d_v, cfg.d_k)
+    elif inp.get("init_state") is not None:
+        Sx = np.asarray(inp["init_state"][b, h], F64)
+    else:
+        Sx = np.zeros((cfg.d_v, cfg.d_k))
+    S0 = 0.5 * Sx
+    k = inp["k"][b, :, :, h]
+    v = inp["v"][b, :, :, h]
+    beta = inp["beta"][b, :, :, h]
+    alpha = inp["alpha"][b, :, h]
+    F = forward_states(S0, k, v, beta, alpha, cfg.anchors)
+    G = backward_states(S0, k, v, beta, alpha, cfg.anchors)
+    return F, G
+
+
+def hybrid_attn(inp: dict, cfg: Cfg, anchor_read: str = "text", softmax: str = "frames") -> np.ndarray:
+    """The video-to-video hybrid attention core for every token.
+
+    Returns Y [B, T, N, H, 2, d_v] (slot 0 = gated softmax branch, slot 1 =
+    gated, RMS-normalised linear branch) or, with out_mode=1, their sum
+    [B, T, N, H, d_v].  softmax="dense" uses the explicit token mask."""
+    B, T, N, H, dv = cfg.B, cfg.T, cfg.N, cfg.H, cfg.d_v
+    Y = np.zeros((B, T, N, H, 2, dv))
+    w = inp.get("rms_weight")
+    for b in range(B):
+        for h in range(H):
+            F, G = head_states(inp, cfg, b, h)
+            q_bh = np.asarray(inp["q"][b, :, :, h], F64)
+            k_bh = np.asarray(inp["k"][b, :, :, h], F64)
+            v_bh = np.asarray(inp["v"][b, :, :, h], F64)
+            wh = None if w is None else w[h]
+            if softmax == "dense":
+                osm = softmax_dense_masked(q_bh, k_bh, v_bh, T, N, cfg.chunk, cfg.anchors, cfg.scale)
+            for t in range(T):
+                R = read_state(F, G, t, T, cfg.chunk, cfg.anchors, anchor_read)
+                o_lin = q_bh[t] @ R.T                      # o = R q per token
+                Y[b, t, :, h, 1] = rms_gate(o_lin, inp["gate_lin"][b, t, :, h], cfg.rms_eps, wh)
+                o = osm[t] if softmax == "dense" else softmax_frame(
+                    q_bh[t], k_bh, v_bh, t, T, cfg.chunk, cfg.anchors, cfg.scale)
+                Y[b, t, :, h, 0] = sigmoid(inp["gate_sm"][b, t, :, h]) * o
+    if cfg.out_mode == 1:
+        return Y.sum(axis=4)
+    return Y
+
+
+def hybrid_attn_rows(inp: dict, cfg: Cfg, rows, anchor_read: str = "text") -> np.ndarray:
+    """The same core evaluated only at the listed (b, t, n, h) positions.
+    Returns [len(rows), 2, d_v] (softmax slot, linear slot), unsummed."""
+    rows = [tuple(int(x) for x in r) for r in rows]
+    states = {}
+    out = np.zeros((len(rows), 2, cfg.d_v))
+    w = inp.get("rms_weight")
+    for i, (b, t, n, h) in enumerate(rows):
+        if (b, h) not in states:
+            states[(b, h)] = head_states(inp, cfg, b, h)
+        F, G = states[(b, h)]
+        q = np.asarray(inp["q"][b, t, n, h], F64)
+        R = read_state(F, G, t, cfg.T, cfg.chunk, cfg.anchors, anchor_read)
+        out[i, 1] = rms_gate(R @ q, inp["gate_lin"][b, t, n, h], cfg.rms_eps, None if w is None else w[h])
+        k_bh = inp["k"][b, :, :, h]
+        v_bh = inp["v"][b, :, :, h]
+        o = softmax_frame(q[None], k_bh, v_bh, t, cfg.T, cfg.chunk, cfg.anchors, cfg.scale)[0]
+        out[i, 0] = sigmoid(inp["gate_sm"][b, t, n, h]) * o
+    return out
+
+
+def vda_intermediates(inp: dict, cfg: Cfg, b: int, h: int):
+    """Per-frame maps (M_t, C_t), the text state S_x and the per-chunk read
+    table R of one (batch, head), for checking a kernel stage by stage."""
+    T = cfg.T
+    Ms = np.zeros((T, cfg.d_k, cfg.d_k))
+    Cs = np.zeros((T, cfg.d_v, cfg.d_k))
+    anc = set(anchor_frames(T, cfg.anchors))
+    for t in range(T):
+        if t in anc:
+            continue
+        Ms[t], Cs[t] = frame_map(inp["k"][b, t, :, h], inp["v"][b, t, :, h], inp["beta"][b, t, :, h])
+    F, G = head_states(inp, cfg, b, h)
+    return {"M": Ms, "C": Cs, "S_init": F[0], "F": F, "G": G,
+            "R": read_table(F, G, T, cfg.chunk, cfg.anchors)}

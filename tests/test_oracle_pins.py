@@ -1,0 +1,373 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these re-types an oracle formula: each checks the oracle against an
+independent route (the objective itself, a stacked least-squares solve, the
+token-space Woodbury form, the classic delta rule, a combinatorial count,
+library routines, brute force) or an invariant the pages state.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import vdn_oracle as O
+from video_diffusion_hybrid_b200.synth import Shape, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(1234)
+
+
+def _frame(n, dk, dv, seed=0, unit=True):
+    r = np.random.default_rng(seed)
+    K = r.standard_normal((n, dk))
+    if unit:
+        K /= np.linalg.norm(K, axis=1, keepdims=True)
+    V = r.standard_normal((n, dv))
+    beta = 1 / (1 + np.exp(-r.standard_normal(n)))
+    Sbar = r.standard_normal((dv, dk))
+    return Sbar, K, V, beta
+
+
+def _objective(S, Sbar, K, V, beta):
+    """||S - S_bar||^2 + sum_i beta_i ||S k_i - v_i||^2, written token by
+    token ([P1] section 四; deepmagic post, closed form paragraph)."""
+    f = np.sum((S - Sbar) ** 2)
+    for i in range(K.shape[0]):
+        r = S @ K[i] - V[i]
+        f += beta[i] * (r @ r)
+    return f
+
+
+# ---------------------------------------------------------------- mask ----
+def _golden_rows():
+    rows = {}
+    with open(os.path.join(GOLDEN, "mask_density.txt")) as fh:
+        for line in fh:
+            if line.strip() and not line.startswith("#"):
+                q, T, ch, an, val, _src = line.split()
+                rows[q] = (int(T), int(ch), int(an), float(val))
+    return rows
+
+
+def test_density_matches_page_value():
+    T, ch, an, val = _golden_rows()["density"]
+    assert round(100 * O.mask_density(T, ch, an), 2) == pytest.approx(val, abs=1e-9)
+
+
+def test_anchor_overhead_matches_page_value():
+    T, ch, an, val = _golden_rows()["anchor_overhead"]
+    extra = 100 * (O.mask_density(T, ch, an) - O.mask_density(T, ch, 0))
+    assert abs(extra - val) < 0.01
+
+
+@pytest.mark.parametrize("T", [15, 20, 30, 45, 90, 180])
+def test_mask_count_closed_form(T):
+    """Allowed frame pairs counted combinatorially for T = 5C, C >= 3:
+    25 (3C - 2) window pairs, plus the 4T - 4 anchor row/column pairs, minus
+    the 38 of those already inside the window."""
+    C = T // 5
+    window = 25 * (3 * C - 2)
+    assert O.frame_mask(T, 5, 0).sum() == window
+    assert O.frame_mask(T, 5, 4).sum() == window + (4 * T - 4) - 38
+
+
+def test_token_mask_is_frame_mask_blocks():
+    T, N = 12, 3
+    M = O.token_mask(T, N, 5, 4)
+    Fm = O.frame_mask(T, 5, 4)
+    for i in range(T * N):
+        for j in range(T * N):
+            assert M[i, j] == Fm[i // N, j // N]
+
+
+# ---------------------------------------------------------- VDA update ----
+@pytest.mark.parametrize("n,dk,dv", [(1, 8, 8), (7, 8, 5), (40, 16, 16), (3, 32, 32)])
+def test_update_minimises_objective(n, dk, dv):
+    """At the minimiser of a quadratic, f(S + D) - f(S) equals the quadratic
+    form ||D||^2 + sum beta_i ||D k_i||^2 for every perturbation D."""
+    Sbar, K, V, beta = _frame(n, dk, dv, seed=n)
+    S = O.vda_update(Sbar, K, V, beta)
+    f0 = _objective(S, Sbar, K, V, beta)
+    for s in range(4):
+        D = np.random.default_rng(s).standard_normal(S.shape) * 1e-2
+        quad = np.sum(D ** 2) + sum(beta[i] * np.sum((D @ K[i]) ** 2) for i in range(n))
+        assert _objective(S + D, Sbar, K, V, beta) - f0 == pytest.approx(quad, rel=1e-8, abs=1e-14)
+
+
+def test_update_equals_stacked_least_squares():
+    """The objective is an ordinary least-squares problem per row of S:
+    rows [I ; sqrt(beta_i) k_i^T] against targets [s_bar ; sqrt(beta_i) v_i]."""
+    Sbar, K, V, beta = _frame(50, 12, 9, seed=3)
+    S = O.vda_update(Sbar, K, V, beta)
+    sb = np.sqrt(beta)[:, None]
+    Amat = np.vstack([np.eye(12), sb * K])
+    for r in range(9):
+        rhs = np.concatenate([Sbar[r], sb[:, 0] * V[:, r]])
+        x, *_ = np.linalg.lstsq(Amat, rhs, rcond=None)
+        np.testing.assert_allclose(S[r], x, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("n,d", [(5, 16), (60, 16), (33, 32)])
+def test_update_matches_token_space_woodbury(n, d):
+    """S = S_bar + W^T K with W = (D^-1 + K K^T)^-1 (V - K S_bar^T), D = diag(beta):
+    the same minimiser reached through an n x n solve instead of d x d."""
+    Sbar, K, V, beta = _frame(n, d, d, seed=n + d)
+    W = np.linalg.solve(np.diag(1 / beta) + K @ K.T, V - K @ Sbar.T)
+    np.testing.assert_allclose(O.vda_update(Sbar, K, V, beta), Sbar + W.T @ K, rtol=0, atol=1e-10)
+
+
+def test_single_token_is_classic_delta_rule():
+    """One token per frame: S = S_bar + beta' (v - S_bar k) k^T with the
+    effective strength beta' = beta / (1 + beta ||k||^2) (the token-wise
+    delta rule that VDA generalises, aimodeling news 'The VDN split')."""
+    for s in range(5):
+        Sbar, K, V, beta = _frame(1, 16, 12, seed=100 + s, unit=(s % 2 == 0))
+        k, v, b = K[0], V[0], beta[0]
+        want = Sbar + (b / (1 + b * k @ k)) * np.outer(v - Sbar @ k, k)
+        np.testing.assert_allclose(O.vda_update(Sbar, K, V, beta), want, rtol=0, atol=1e-12)
+
+
+def test_inherited_map_is_non_expansive():
+    """S_bar -> S_bar (I + A)^-1 never amplifies the inherited state
+    ([P1] section 四; deepmagic post; aimodeling news)."""
+    for s in range(6):
+        _, K, V, beta = _frame(30 + 20 * s, 16, 16, seed=200 + s)
+        M, _ = O.frame_map(K, V, beta)
+        assert np.linalg.norm(M, 2) <= 1 + 1e-12
+        X = np.random.default_rng(s).standard_normal((16, 16))
+        assert np.linalg.norm(X @ M) <= np.linalg.norm(X) * (1 + 1e-12)
+        # the inherited part of the update is exactly that map
+        np.testing.assert_allclose(O.vda_update(X, K, V, beta) - O.vda_update(0 * X, K, V, beta), X @ M,
+                                   rtol=0, atol=1e-11)
+
+
+def test_evidence_saturates_below_one():
+    """n copies of one unit key written from zero give S k = n b / (1 + n b) v:
+    a hundred patches push the weight toward, never past, one.  Orthogonal
+    keys each keep b / (1 + b) (aimodeling news 'The VDN split')."""
+    d, b = 16, 0.7
+    k = np.zeros(d); k[3] = 1.0
+    v = np.random.default_rng(0).standard_normal(d)
+    for n in (1, 2, 10, 100):
+        S = O.vda_update(np.zeros((d, d)), np.tile(k, (n, 1)), np.tile(v, (n, 1)), np.full(n, b))
+        w = n * b / (1 + n * b)
+        np.testing.assert_allclose(S @ k, w * v, rtol=0, atol=1e-12)
+        assert w < 1
+    K = np.eye(d)[:5]
+    V = np.random.default_rng(1).standard_normal((5, d))
+    S = O.vda_update(np.zeros((d, d)), K, V, np.full(5, b))
+    for i in range(5):
+        np.testing.assert_allclose(S @ K[i], b / (1 + b) * V[i], rtol=0, atol=1e-12)
+
+
+def test_update_independent_of_token_order():
+    """The joint frame write does not depend on an order of the tokens
+    ([P1] section 四: no artificial scan order inside a frame)."""
+    Sbar, K, V, beta = _frame(64, 16, 16, seed=9)
+    p = np.random.default_rng(2).permutation(64)
+    np.testing.assert_allclose(O.vda_update(Sbar, K, V, beta), O.vda_update(Sbar, K[p], V[p], beta[p]),
+                               rtol=0, atol=1e-12)
+
+
+def test_frame_map_expands_update():
+    Sbar, K, V, beta = _frame(20, 8, 6, seed=5)
+    M, C = O.frame_map(K, V, beta)
+    np.testing.assert_allclose(Sbar @ M + C, O.vda_update(Sbar, K, V, beta), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(M, M.T, rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- scan ----
+def _scan_inputs(T, N, d, seed):
+    r = np.random.default_rng(seed)
+    k = r.standard_normal((T, N, d)); k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = r.standard_normal((T, N, d))
+    beta = 1 / (1 + np.exp(-r.standard_normal((T, N))))
+    alpha = 1 / (1 + np.exp(-(2 + 0.5 * r.standard_normal(T))))
+    S0 = r.standard_normal((d, d))
+    return S0, k, v, beta, alpha
+
+
+def test_backward_scan_is_forward_scan_reversed():
+    S0, k, v, beta, alpha = _scan_inputs(17, 6, 8, 1)
+    G = O.backward_states(S0, k, v, beta, alpha, anchors=4)
+    F = O.forward_states(S0, k[::-1], v[::-1], beta[::-1], alpha[::-1], anchors=4)
+    np.testing.assert_allclose(G[::-1], F, rtol=0, atol=1e-12)
+
+
+def test_zero_decay_forgets_history():
+    S0, k, v, beta, alpha = _scan_inputs(8, 5, 8, 2)
+    F = O.forward_states(S0, k, v, beta, np.zeros(8), anchors=0)
+    for t in range(8):
+        np.testing.assert_allclose(F[t + 1], O.vda_update(np.zeros((8, 8)), k[t], v[t], beta[t]), atol=1e-13)
+
+
+def test_scan_equals_least_squares_chain():
+    """Each forward step, computed by the stacked least-squares route from the
+    previous step's state decayed by alpha, reproduces the scan."""
+    S0, k, v, beta, alpha = _scan_inputs(12, 4, 6, 3)
+    F = O.forward_states(S0, k, v, beta, alpha, anchors=4)
+    S = S0.copy()
+    for t in range(12):
+        if t not in (0, 11):
+            Sb = alpha[t] * S
+            sb = np.sqrt(beta[t])[:, None]
+            Amat = np.vstack([np.eye(6), sb * k[t]])
+            S = np.stack([np.linalg.lstsq(Amat, np.concatenate([Sb[r], sb[:, 0] * v[t][:, r]]), rcond=None)[0]
+                          for r in range(6)])
+        np.testing.assert_allclose(F[t + 1], S, rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("T,anchors", [(30, 4), (23, 4), (35, 0), (10, 4), (7, 4)])
+def test_read_regions_cover_each_frame_once(T, anchors):
+    """Tag every frame with its own orthogonal key/value (one token, alpha=1):
+    the diagonal of a state then shows which frames it holds.  For every query
+    frame, forward reads + backward reads + the softmax key frames cover every
+    frame exactly once, and anchor frames are never written
+    ([P1] section 三: the regions do not overlap; anchors are not re-written)."""
+    d = T
+    k = np.eye(d)[:T, None, :]
+    v = np.eye(d)[:T, None, :]
+    beta = np.ones((T, 1))
+    alpha = np.ones(T)
+    S0 = np.zeros((d, d))
+    F = O.forward_states(S0, k, v, beta, alpha, anchors)
+    G = O.backward_states(S0, k, v, beta, alpha, anchors)
+    fm = O.frame_mask(T, 5, anchors)
+    anc = set(O.anchor_frames(T, anchors))
+    for t in range(T):
+        R = O.read_state(F, G, t, T, 5, anchors)
+        held = np.diag(R)
+        np.testing.assert_allclose(held[held > 1e-9], 0.5, atol=1e-12)  # beta/(1+beta) with beta=1
+        lin = set(np.nonzero(held > 1e-9)[0])
+        soft = set(np.nonzero(fm[t])[0])
+        assert not (lin & soft)
+        assert not (lin & anc)
+        assert lin | soft == set(range(T))
+
+
+def test_half_text_reads_sum_to_one_text_read():
+    """With no video written into a query's states (T=10: two chunks, all in
+    window), its linear read is exactly the text state applied once
+    ([P1] section 三; deepmagic post: each direction starts from half)."""
+    shp = Shape(B=1, T=10, N=16, H=2, d_k=32, d_v=32, L=8)
+    inp = make_inputs(shp, seed=0)
+    cfg = O.Cfg(B=1, T=10, N=16, H=2, d_k=32, d_v=32, L=8)
+    Y = O.hybrid_attn(inp, cfg)
+    for h in range(2):
+        Sx = O.vda_update(np.zeros((32, 32)), inp["text_k"][0, :, h], inp["text_v"][0, :, h], inp["text_beta"][0, :, h])
+        o = inp["q"][0, :, :, h].astype(np.float64) @ Sx.T
+        want = O.rms_gate(o, inp["gate_lin"][0, :, :, h], 1e-6)
+        np.testing.assert_allclose(Y[0, :, :, h, 1], want, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------- softmax ----
+def _torch_sdpa(q, k, v, mask, scale):
+    qt, kt, vt = (torch.from_numpy(np.asarray(x, np.float64))[None] for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(mask)[None],
+                                                           scale=scale)
+    return out[0].numpy()
+
+
+@pytest.mark.parametrize("T,N,anchors,scale", [(10, 4, 4, None), (23, 3, 4, None), (30, 2, 0, 10.0),
+                                               (20, 5, 4, 10.0)])
+def test_windowed_softmax_equals_dense_masked_attention(T, N, anchors, scale):
+    """The windowed + anchor softmax the oracle uses equals dense attention
+    under the explicit hybrid token mask, computed by torch's SDPA."""
+    r = np.random.default_rng(T)
+    d = 8
+    q, k, v = (r.standard_normal((T, N, d)) for _ in range(3))
+    sc = scale or 1 / np.sqrt(d)
+    want = _torch_sdpa(q.reshape(T * N, d), k.reshape(T * N, d), v.reshape(T * N, d),
+                       O.token_mask(T, N, 5, anchors), sc).reshape(T, N, d)
+    dense = O.softmax_dense_masked(q, k, v, T, N, 5, anchors, sc)
+    np.testing.assert_allclose(dense, want, rtol=0, atol=1e-12)
+    for t in range(T):
+        np.testing.assert_allclose(O.softmax_frame(q[t], k, v, t, T, 5, anchors, sc), want[t], rtol=0, atol=1e-12)
+
+
+def test_softmax_brute_force_tiny():
+    """Pair-by-pair softmax with explicit exponentials on a tiny case."""
+    T, N, d = 11, 2, 4
+    r = np.random.default_rng(7)
+    q, k, v = (r.standard_normal((T, N, d)) for _ in range(3))
+    sc = 0.9
+    for tq in range(T):
+        for n in range(N):
+            num = np.zeros(d); den = 0.0
+            for tk in range(T):
+                cq, ck = tq // 5, tk // 5
+                if abs(cq - ck) <= 1 or tk in (0, T - 1) or tq in (0, T - 1):
+                    for m in range(N):
+                        e = np.exp(sc * q[tq, n] @ k[tk, m])
+                        num += e * v[tk, m]; den += e
+            got = O.softmax_frame(q[tq, n:n + 1], k, v, tq, T, 5, 4, sc)[0]
+            np.testing.assert_allclose(got, num / den, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------ norm and gates ----
+def test_rms_gate_matches_library():
+    r = np.random.default_rng(3)
+    o = r.standard_normal((7, 32)); g = r.standard_normal((7, 32)); w = r.standard_normal(32)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(o), (32,), torch.from_numpy(w), eps=1e-6)
+    ref = torch.sigmoid(torch.from_numpy(g)) * ref
+    np.testing.assert_allclose(O.rms_gate(o, g, 1e-6, w), ref.numpy(), rtol=1e-13, atol=1e-14)
+
+
+# ------------------------------------------------------------ end to end --
+def _cfg(shp, **kw):
+    return O.Cfg(B=shp.B, T=shp.T, N=shp.N, H=shp.H, d_k=shp.d_k, d_v=shp.d_v, L=shp.L, **kw)
+
+
+def test_rows_route_equals_full_route():
+    shp = Shape(B=2, T=30, N=4, H=2, d_k=8, d_v=8, L=5)
+    inp = make_inputs(shp, seed=11)
+    cfg = _cfg(shp)
+    Y = O.hybrid_attn(inp, cfg)
+    Yd = O.hybrid_attn(inp, cfg, softmax="dense")
+    np.testing.assert_allclose(Y, Yd, rtol=0, atol=1e-12)
+    rows = [(b, t, n, h) for b in range(2) for t in (0, 4, 5, 13, 24, 29) for n in (0, 3) for h in range(2)]
+    got = O.hybrid_attn_rows(inp, cfg, rows)
+    for i, (b, t, n, h) in enumerate(rows):
+        np.testing.assert_allclose(got[i], Y[b, t, n, h], rtol=0, atol=1e-12)
+    Ys = O.hybrid_attn(inp, _cfg(shp, out_mode=1))
+    np.testing.assert_allclose(Ys, Y.sum(axis=4), rtol=0, atol=1e-12)
+
+
+def test_intermediates_reassemble_states():
+    """The per-frame affine maps (M_t, C_t) chained from S_init reproduce the
+    definitional forward scan, and the read table matches read_state."""
+    shp = Shape(B=1, T=20, N=6, H=1, d_k=8, d_v=8, L=4)
+    inp = make_inputs(shp, seed=5)
+    cfg = _cfg(shp)
+    it = O.vda_intermediates(inp, cfg, 0, 0)
+    S = it["S_init"].copy()
+    for t in range(20):
+        if t not in (0, 19):
+            S = inp["alpha"][0, t, 0] * S @ it["M"][t] + it["C"][t]
+        np.testing.assert_allclose(S, it["F"][t + 1], rtol=0, atol=1e-11)
+    for t in range(20):
+        c = 4 if t in (0, 19) else t // 5
+        np.testing.assert_allclose(it["R"][c], O.read_state(it["F"], it["G"], t, 20), rtol=0, atol=0)
+
+
+# ------------------------------------------- planted mistakes must fail ---
+def test_pins_catch_dropped_inherited_term(monkeypatch):
+    orig = O.vda_update
+    monkeypatch.setattr(O, "vda_update", lambda Sbar, K, V, b: orig(0 * np.asarray(Sbar), K, V, b))
+    with pytest.raises(AssertionError):
+        test_single_token_is_classic_delta_rule()
+
+
+def test_pins_catch_shifted_read_window(monkeypatch):
+    monkeypatch.setattr(O, "window_frames", lambda t, T, chunk=5: (max(0, chunk * (t // chunk)),
+                                                                   min(T, chunk * (t // chunk + 2))))
+    with pytest.raises(AssertionError):
+        test_read_regions_cover_each_frame_once(30, 4)
+
+
+def test_pins_catch_transposed_write(monkeypatch):
+    orig = O.gram_write
+    monkeypatch.setattr(O, "gram_write", lambda K, V, b: (orig(K, V, b)[0], orig(K, V, b)[1].T))
+    with pytest.raises(AssertionError):
+        test_update_matches_token_space_woodbury(5, 16)
