@@ -1,0 +1,352 @@
+#!/usr/bin/env python
+"""Throughput of the Video DeltaNet hybrid attention core on B200.
+
+One step = one pass of the whole core (text solve, per-frame Gram/solve,
+bidirectional scan, windowed softmax, state read + epilogue) over one batch
+of synthetic input of the named workload (default: the 768p single-block
+stand-in, T=90, N=1008, H=24, d=128, L=512, bf16).  Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 it runs under torchrun, one rank per GPU; every rank processes its
+own independent problem (weak scaling, no collective on the data path) and
+the time is the max over ranks.  ``--impl reference`` times the fp64 CPU
+oracle on the host cores instead (rank 0 only), on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "video tokens/s per hybrid-attn layer on 1 B200; % tensor-pipe / HBM roofline"
+UNIT = "video tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="768p")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- oracle --
+def oracle_sample(workload, n_na_tokens=128, n_a_tokens=64, head=0, seed_offset=0):
+    """Time the fp64 oracle on a bounded sample of one head of the workload:
+    the full bidirectional VDA chain of that head, both branches for
+    `n_na_tokens` queries of a non-anchor frame and `n_a_tokens` queries of an
+    anchor frame.  Extrapolates per-token costs to the whole layer (all heads,
+    all frames).  Returns (tokens/s, seconds of CPU work, description)."""
+    from oracle import vdn_oracle as O
+    from video_diffusion_hybrid_b200.synth import Shape, make_inputs
+    s = workload.shape
+    one = Shape(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
+    inp = make_inputs(one, workload.seed + seed_offset, workload.dtype)
+    cfg = O.Cfg(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
+    t0 = time.perf_counter()
+    F, G = O.head_states(inp, cfg, 0, 0)
+    t_chain = time.perf_counter() - t0
+    q = inp["q"][0, :, :, 0].astype(np.float64)
+    k, v = inp["k"][0, :, :, 0], inp["v"][0, :, :, 0]
+
+    def frame_cost(t, n):
+        t1 = time.perf_counter()
+        R = O.read_state(F, G, t, s.T, cfg.chunk, cfg.anchors)
+        O.rms_gate(q[t, :n] @ R.T, inp["gate_lin"][0, t, :n, 0], cfg.rms_eps)
+        o = O.softmax_frame(q[t, :n], k, v, t, s.T, cfg.chunk, cfg.anchors, cfg.scale)
+        O.sigmoid(inp["gate_sm"][0, t, :n, 0]) * o
+        return (time.perf_counter() - t1) / n
+
+    c_na = frame_cost(s.T // 2, min(n_na_tokens, s.N))
+    c_a = frame_cost(0, min(n_a_tokens, s.N))
+    n_anchor = 2
+    per_head = t_chain + (s.T - n_anchor) * s.N * c_na + n_anchor * s.N * c_a
+    layer = per_head * s.H * s.B
+    work = t_chain + min(n_na_tokens, s.N) * c_na + min(n_a_tokens, s.N) * c_a
+    desc = (f"head {head} of {workload.name}: full VDA chain over {s.T} frames + both branches for "
+            f"{min(n_na_tokens, s.N)} queries of a non-anchor frame and {min(n_a_tokens, s.N)} of an anchor "
+            f"frame; per-token costs extrapolated to {s.B}x{s.H} heads x {s.T * s.N} tokens")
+    return s.B * s.T * s.N / layer, work, desc
+
+
+def host_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    w = WORKLOADS[args.workload]
+    vals, times = [], []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        val, _work, desc = oracle_sample(w, n_na_tokens=32, n_a_tokens=8)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            vals.append(val)
+            times.append(dt)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.shape.B, "T": w.shape.T, "N": w.shape.N, "H": w.shape.H,
+                   "d": w.shape.d_k, "L": w.shape.L, "inputs": w.dtype},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- ours ----
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_traffic(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (matching hash); else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(key)
+    if not d:
+        return None
+    src = open(os.path.join(ROOT, "video_diffusion_hybrid_b200", "csrc", kernel_file), "rb").read()
+    if hashlib.sha256(src).hexdigest()[:16] != d.get("source_sha256_16"):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from video_diffusion_hybrid_b200 import _lib as L
+    from video_diffusion_hybrid_b200.api import HybridAttention, cfg_for
+    from video_diffusion_hybrid_b200.roofline import softmax_flops
+    from video_diffusion_hybrid_b200.synth import make_inputs_torch
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    L.lib()  # fail loudly if the extension is missing
+
+    w = WORKLOADS[args.workload]
+    s = w.shape
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, work, desc = oracle_sample(w)
+        cpu = {"value": val, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc,
+               "sample_cpu_seconds": round(work, 2)}
+
+    t = make_inputs_torch(s, w.seed + 17 * rank, w.dtype, dev)
+    cfg = cfg_for(s, w.dtype)
+    ha = HybridAttention(cfg, dev)
+    stream = torch.cuda.current_stream(dev)
+    pre = L.STAGE_TEXT | L.STAGE_SOLVE | L.STAGE_SCAN
+    launches_per_step = 5 if (s.L > 0) else 4
+    K, W = args.steps, args.warmup
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def step(i=None):
+        ha(t, stages=pre)
+        if i is not None:
+            ev[i][0].record(stream)
+        ha(t, stages=L.STAGE_SOFTMAX)
+        if i is not None:
+            ev[i][1].record(stream)
+        ha(t, stages=L.STAGE_READ)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(dev)
+    st, where = L.vdn_hybrid_device_status(cfg, ha.args(t))
+    if st != L.VDN_OK:
+        raise SystemExit(f"device status {st} at kernel tag {where}")
+
+    props = torch.cuda.get_device_properties(dev)
+    clk = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if rank == 0:
+        clk.start()
+        time.sleep(0.3)
+    start.record(stream)
+    for i in range(K):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop() if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end) / K
+    sm_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        x = torch.tensor([ms, sm_ms], device=dev)
+        dist.all_reduce(x, op=dist.ReduceOp.MAX)
+        ms, sm_ms = x.tolist()
+
+    # end to end: pinned host inputs -> device, the call, the whole output back
+    e2e = None
+    if not args.no_e2e:
+        host = {k: v.cpu().pin_memory() for k, v in t.items()}
+        yh = torch.empty(ha.y.shape, dtype=ha.y.dtype, pin_memory=True)
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = yh.numel() * yh.element_size()
+
+        def e2e_step():
+            for k, v in host.items():
+                t[k].copy_(v, non_blocking=True)
+            ha(t)
+            yh.copy_(ha.y, non_blocking=True)
+
+        for _ in range(max(1, W)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = s0.elapsed_time(s1) / K
+        if world > 1:
+            x = torch.tensor([ems], device=dev)
+            dist.all_reduce(x, op=dist.ReduceOp.MAX)
+            ems = x.item()
+        e2e = {"value": world * w.tokens / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        flops = softmax_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.chunk, cfg.anchors)
+        achieved = flops / (sm_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        impl = L.vdn_hybrid_stage_impl(cfg, L.STAGE_SOFTMAX)
+        line = {
+            "metric": METRIC, "value": world * w.tokens / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": s.B, "T": s.T, "N": s.N, "H": s.H, "d": s.d_k, "L": s.L,
+                       "chunk": 5, "anchors": 4, "state": "fp32", "accumulate": "fp32",
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "inputs exceed L2 (2.8 GB of q/k/v/gates per step at 768p)"},
+            "roofline": {"kernel": "window_softmax" + ("_tcgen05" if impl == 1 else "_simt"), "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"bf16_tflops_sustained ({src})", "ms_per_launch": sm_ms,
+                         "flops_per_launch": flops,
+                         "traffic": kernel_traffic("vdn_softmax_tc.cu" if impl == 1 else "vdn_simt.cu",
+                                                   "window_softmax")},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * K,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,162 @@
+/*
+ * vdn_hybrid.h -- C ABI of the Video DeltaNet hybrid attention core on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes (sources: the PaperDaily digest "伯克利与Impossible视频生成:
+ * 14.3秒视频6.70秒去噪", sections 二, 三 and 四; the deepmagic.app post
+ * "生成比播放還快", section "用兩條分支取代一條"; the aimodeling.com news
+ * "video-deltanet-h3-hybrid-attention", section "The VDN split"):
+ *
+ *   Video Delta Attention (linear branch).  For every non-anchor frame t and
+ *   head, over the N tokens of the frame,
+ *       A_t = sum_i beta_i k_i k_i^T,   B_t = sum_i beta_i v_i k_i^T,
+ *       S_t = (alpha_t S_{t-1} + B_t) (I + A_t)^{-1},
+ *   run forward (frames 0..T-1) and backward (T-1..0), both started from half
+ *   of the text state S_x = B_x (I + A_x)^{-1} (one joint solve over the L text
+ *   tokens).  The first and last frame (the anchors) are not written.  A query
+ *   in chunk c = floor(t / 5) reads the forward state over frames < 5(c-1) plus
+ *   the backward state over frames >= 5(c+2): o_lin = R q.  Anchor query frames
+ *   read the two initial states (S_x).  Then
+ *       y_lin = sigmoid(g_lin) * o_lin / sqrt(mean(o_lin^2) + eps) [* w].
+ *
+ *   Windowed softmax.  A query in chunk c attends to the keys of chunks
+ *   c-1, c, c+1 (clipped at the ends), every query sees the anchor frames and
+ *   anchor queries see every frame:  y_sm = sigmoid(g_sm) * softmax(s q K^T) V.
+ *
+ * Conventions for every entry point:
+ *   - Ownership: the library allocates nothing.  The caller owns every input,
+ *     the output and the workspace; all data pointers are DEVICE pointers on the
+ *     current CUDA device, all struct pointers are HOST pointers read during the
+ *     call only.
+ *   - Asynchrony: work is enqueued on `stream` (NULL = legacy default stream)
+ *     and the call returns without synchronising.
+ *   - Errors: arguments are validated before any launch; a status other than
+ *     VDN_OK from validation means nothing was enqueued.  A launch failure is
+ *     VDN_ERR_CUDA (the CUDA error is left for cudaGetLastError).
+ *   - Aliasing: inputs are read-only; `y` and `workspace` must not overlap any
+ *     input or each other.
+ *   - Layouts are dense, row-major, innermost dimension last, no padding.
+ */
+#ifndef VDN_HYBRID_H
+#define VDN_HYBRID_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so that the header needs no CUDA headers. */
+typedef struct CUstream_st *vdn_stream_t;
+
+typedef enum {
+  VDN_OK = 0,
+  VDN_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad enum, misaligned pointer */
+  VDN_ERR_UNSUPPORTED = 2, /* a valid configuration this build does not implement (d, chunk) */
+  VDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than vdn_hybrid_attn_workspace_size */
+  VDN_ERR_CUDA = 4,        /* a CUDA call or launch failed */
+  VDN_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (see vdn_hybrid_device_status) */
+} vdn_status;
+
+typedef enum {
+  VDN_F32 = 0,  /* q, k, v, gates, text k/v in float32; exact mode (SIMT fp32 arithmetic) */
+  VDN_BF16 = 1  /* the same tensors in bfloat16; fp32 accumulation and fp32 state */
+} vdn_dtype;
+
+typedef struct {
+  int B;        /* batch (independent problems)                                   >= 1 */
+  int T;        /* latent frames                                                  >= 2 */
+  int N;        /* spatial tokens per frame                                       >= 1 */
+  int H;        /* heads                                                          >= 1 */
+  int d_k;      /* key/query head dim: 32, 64 or 128                                   */
+  int d_v;      /* value head dim; must equal d_k in this build                        */
+  int L;        /* text tokens; 0 = no text (states start from init_state or zero)     */
+  int chunk;    /* latent frames per chunk; must be 5                                  */
+  int anchors;  /* 0 = no anchors, 4 = 4-way first/last-frame anchors                   */
+  int dtype;    /* vdn_dtype                                                           */
+  float softmax_scale; /* <= 0 selects 1/sqrt(d_k)                                    */
+  float rms_eps;       /* <= 0 selects 1e-6                                            */
+  int out_mode;        /* 0: y[B,T,N,H,2,d_v], slot 0 = softmax, slot 1 = linear;
+                          1: y[B,T,N,H,d_v] = sum of the two gated branches           */
+  int y_dtype;         /* vdn_dtype of y: VDN_F32 (default, also in bf16 mode) or
+                          VDN_BF16 (rounded to nearest even on store)                  */
+} vdn_hybrid_cfg;
+
+typedef struct {
+  const void *q, *k, *v;           /* [B,T,N,H,d_k] ([..,d_v] for v), dtype              */
+  const float *beta;               /* [B,T,N,H]   write strengths (> 0)                  */
+  const float *alpha;              /* [B,T,H]     decay gates in [0, 1]                  */
+  const void *gate_sm, *gate_lin;  /* [B,T,N,H,d_v] gate logits, dtype                   */
+  const void *text_k, *text_v;     /* [B,L,H,d_k] / [B,L,H,d_v], dtype; NULL iff L == 0   */
+  const float *text_beta;          /* [B,L,H];  NULL iff L == 0                           */
+  const float *init_state;         /* [B,H,d_v,d_k] full text state S_x used instead of a
+                                      text solve (each direction starts from S_x / 2);
+                                      only allowed with L == 0; NULL = zero state          */
+  const float *rms_weight;         /* [H,d_v] RMSNorm weight, NULL = ones                 */
+  void *y;                         /* output, cfg.y_dtype, shape per cfg.out_mode         */
+  void *workspace;                 /* device scratch, 256-byte aligned                   */
+  size_t workspace_bytes;
+} vdn_hybrid_args;
+
+/* Pipeline stages; vdn_hybrid_attn_fwd runs VDN_STAGE_ALL in this order. */
+enum {
+  VDN_STAGE_TEXT = 1u,   /* text solve (or init_state copy) -> half text state       */
+  VDN_STAGE_SOLVE = 2u,  /* per-frame Gram/write + SPD solve -> M_t, C_t              */
+  VDN_STAGE_SCAN = 4u,   /* forward/backward state scans -> chunk-boundary states     */
+  VDN_STAGE_SOFTMAX = 8u,/* windowed softmax + gate -> y slot 0 (or y)                */
+  VDN_STAGE_READ = 16u,  /* state read + RMSNorm + gate -> y slot 1 (or y += )        */
+  VDN_STAGE_ALL = 31u
+};
+
+/* Byte offsets of the intermediate values inside the workspace (all float32,
+ * dense).  C = ceil(T / chunk).  Stable across calls with the same cfg, so that
+ * a caller can inspect the stages.
+ *   status     : uint32 device status words (VDN_ERR_TIMEOUT flags)
+ *   half_text  : [B,H,d_v,d_k]        S_x / 2, the start state of both scans
+ *   frame_M    : [B,T,H,d_k,d_k]      (I + A_t)^{-1}        (anchor frames unset)
+ *   frame_C    : [B,T,H,d_v,d_k]      B_t (I + A_t)^{-1}    (anchor frames unset)
+ *   fwd_snap   : [B,H,C+1,d_v,d_k]    forward state over frames < min(5j, T)
+ *   bwd_snap   : [B,H,C+1,d_v,d_k]    backward state over frames >= min(5j, T)
+ *   read_table : [B,H,C+1,d_v,d_k]    R[c] = fwd_snap[max(c-1,0)] + bwd_snap[min(c+2,C)],
+ *                                     R[C] = half_text * 2 (anchor query frames)        */
+typedef struct {
+  size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, total;
+} vdn_workspace_layout;
+
+/* Bytes of workspace the configuration needs; 0 if cfg is invalid. */
+size_t vdn_hybrid_attn_workspace_size(const vdn_hybrid_cfg *cfg);
+
+/* Fill *out with the workspace layout of cfg.  Errors: VDN_ERR_INVALID_ARG,
+ * VDN_ERR_UNSUPPORTED. */
+vdn_status vdn_hybrid_workspace_layout(const vdn_hybrid_cfg *cfg, vdn_workspace_layout *out);
+
+/* The whole hybrid attention core: all stages, in order, on `stream`. */
+vdn_status vdn_hybrid_attn_fwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
+                               vdn_stream_t stream);
+
+/* A subset of the stages (bitwise OR of VDN_STAGE_*), in pipeline order.
+ * Each stage reads what the earlier stages left in the workspace; running a
+ * stage whose inputs were never produced gives unspecified (but in-bounds)
+ * results.  Used to time and check the stages one by one. */
+vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
+                                      unsigned stages, vdn_stream_t stream);
+
+/* Reads the device status words left by the most recent call on this
+ * workspace (every fwd / fwd_stages call clears them first; synchronises `stream`).
+ * Returns VDN_OK or VDN_ERR_TIMEOUT; *where (if not NULL) gets the kernel tag
+ * that gave up. */
+vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
+                                    vdn_stream_t stream, unsigned *where);
+
+/* Which implementation a stage uses for cfg: 0 = SIMT fp32, 1 = tcgen05 tensor
+ * cores (TMA + TMEM), -1 = stage not supported for cfg. */
+int vdn_hybrid_stage_impl(const vdn_hybrid_cfg *cfg, unsigned stage);
+
+/* Static description of a status code. */
+const char *vdn_status_string(vdn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VDN_HYBRID_H */

@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+the header declares, sizes its workspace, and rejects bad arguments before
+touching the GPU (no compute call here: these run without a device)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from video_diffusion_hybrid_b200 import _lib as L
+from video_diffusion_hybrid_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build()
+    return L.lib()
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(vdn_\w+)\s*\(", src, flags=re.M))
+    return names
+
+
+def test_exports_every_declared_symbol():
+    declared = _declared()
+    assert declared == set(L.EXPORTED)
+    lib = L.lib()
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def _cfg(**kw):
+    base = dict(B=1, T=90, N=1008, H=24, d_k=128, d_v=128, L=512, dtype=L.VDN_BF16)
+    base.update(kw)
+    return L.HybridCfg(**base)
+
+
+def test_workspace_size_and_layout():
+    cfg = _cfg()
+    size = L.vdn_hybrid_attn_workspace_size(cfg)
+    lay = L.vdn_hybrid_workspace_layout(cfg)
+    assert lay["total"] == size
+    dd = 128 * 128 * 4
+    assert lay["frame_C"] - lay["frame_M"] >= 90 * 24 * dd
+    assert lay["read_table"] - lay["bwd_snap"] >= 24 * 19 * dd
+    offs = [lay[k] for k in ("status", "half_text", "frame_M", "frame_C", "fwd_snap", "bwd_snap", "read_table",
+                             "total")]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=1), L.VDN_ERR_INVALID_ARG), (dict(N=0), L.VDN_ERR_INVALID_ARG), (dict(anchors=2), L.VDN_ERR_INVALID_ARG),
+    (dict(dtype=7), L.VDN_ERR_INVALID_ARG), (dict(out_mode=3), L.VDN_ERR_INVALID_ARG),
+    (dict(L=-1), L.VDN_ERR_INVALID_ARG), (dict(chunk=0), L.VDN_ERR_INVALID_ARG),
+    (dict(d_k=48, d_v=48), L.VDN_ERR_UNSUPPORTED), (dict(d_v=64), L.VDN_ERR_UNSUPPORTED),
+    (dict(chunk=4), L.VDN_ERR_UNSUPPORTED), (dict(B=3000, H=24), L.VDN_ERR_UNSUPPORTED),
+])
+def test_bad_config_rejected(kw, status):
+    cfg = _cfg(**kw)
+    assert L.vdn_hybrid_attn_workspace_size(cfg) == 0
+    with pytest.raises(L.VdnError) as e:
+        L.vdn_hybrid_workspace_layout(cfg)
+    assert e.value.status == status
+
+
+def _fake_args(cfg, **over):
+    """Aligned but never dereferenced pointer values: every test below fails
+    validation before a launch."""
+    p = 1 << 20
+    a = dict(q=p, k=p, v=p, beta=p, alpha=p, gate_sm=p, gate_lin=p, y=p, workspace=p,
+             workspace_bytes=L.vdn_hybrid_attn_workspace_size(cfg), text_k=p, text_v=p, text_beta=p)
+    a.update(over)
+    return L.make_args(**a)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), L.VDN_ERR_INVALID_ARG), (dict(y=None), L.VDN_ERR_INVALID_ARG),
+    (dict(k=(1 << 20) + 2), L.VDN_ERR_INVALID_ARG), (dict(text_k=None), L.VDN_ERR_INVALID_ARG),
+    (dict(init_state=1 << 20), L.VDN_ERR_INVALID_ARG), (dict(workspace=None), L.VDN_ERR_WORKSPACE),
+    (dict(workspace=(1 << 20) + 16), L.VDN_ERR_WORKSPACE), (dict(workspace_bytes=1024), L.VDN_ERR_WORKSPACE),
+])
+def test_bad_args_rejected_before_launch(over, status):
+    cfg = _cfg()
+    args = _fake_args(cfg, **over)
+    assert L.vdn_hybrid_attn_fwd(cfg, args, stream=0, check=False) == status
+    assert L.vdn_hybrid_attn_fwd_stages(cfg, args, L.STAGE_SOFTMAX, stream=0, check=False) == status
+
+
+def test_text_pointers_forbidden_without_text():
+    cfg = _cfg(L=0)
+    assert L.vdn_hybrid_attn_fwd(cfg, _fake_args(cfg), stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+
+
+def test_bad_stage_mask_rejected():
+    cfg = _cfg()
+    for mask in (0, 32, 0xFFFF):
+        assert L.vdn_hybrid_attn_fwd_stages(cfg, _fake_args(cfg), mask, stream=0, check=False) == \
+            L.VDN_ERR_INVALID_ARG
+
+
+def test_null_struct_pointers():
+    lib = L.lib()
+    assert lib.vdn_hybrid_attn_fwd(None, None, None) == L.VDN_ERR_INVALID_ARG
+    assert lib.vdn_hybrid_attn_workspace_size(None) == 0
+    c = _cfg().c()
+    assert lib.vdn_hybrid_attn_fwd(C.byref(c), None, None) == L.VDN_ERR_INVALID_ARG
+
+
+def test_status_strings_and_stage_impl():
+    for s in range(6):
+        assert L.status_string(s) and L.status_string(s) != "unknown status"
+    assert L.status_string(99) == "unknown status"
+    cfg = _cfg()
+    for st in (L.STAGE_TEXT, L.STAGE_SOLVE, L.STAGE_SCAN, L.STAGE_READ, L.STAGE_SOFTMAX):
+        assert L.vdn_hybrid_stage_impl(cfg, st) in (0, 1)
+    assert L.vdn_hybrid_stage_impl(cfg, 3) == -1
+    assert L.vdn_hybrid_stage_impl(_cfg(d_k=256, d_v=256), L.STAGE_SOLVE) == -1

@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.
+
+Bar (element by element, per output slot): max |y_gpu - y_oracle| <= tol *
+RMS(y_oracle slot), tol = 1e-4 in fp32 mode and 2e-2 in bf16-input /
+fp32-accumulate mode.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vdn_oracle as O
+from video_diffusion_hybrid_b200 import _lib as L
+from video_diffusion_hybrid_b200.api import HybridAttention, cfg_for, to_torch
+from video_diffusion_hybrid_b200.build import build
+from video_diffusion_hybrid_b200.synth import Shape, make_inputs
+from video_diffusion_hybrid_b200.workloads import WORKLOADS
+
+pytestmark = pytest.mark.gpu
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built(cuda_ok):
+    build()
+
+
+def ocfg(cfg: L.HybridCfg) -> O.Cfg:
+    return O.Cfg(B=cfg.B, T=cfg.T, N=cfg.N, H=cfg.H, d_k=cfg.d_k, d_v=cfg.d_v, L=cfg.L, chunk=cfg.chunk,
+                 anchors=cfg.anchors, softmax_scale=cfg.softmax_scale, rms_eps=cfg.rms_eps or 1e-6,
+                 out_mode=cfg.out_mode)
+
+
+def run(shape: Shape, dtype: str, seed: int, extra=None, drop_text=False, **kw):
+    inp = make_inputs(shape, seed, dtype)
+    if drop_text:
+        for k in ("text_k", "text_v", "text_beta", "text_k_bits", "text_v_bits"):
+            inp.pop(k, None)
+    if extra:
+        inp.update(extra)
+    cfg = cfg_for(shape, dtype, **kw)
+    if drop_text:
+        cfg.L = 0
+    t = to_torch(inp, dtype, "cuda")
+    ha = HybridAttention(cfg)
+    y = ha(t)
+    torch.cuda.synchronize()
+    st, where = L.vdn_hybrid_device_status(cfg, ha.args(t))
+    assert st == L.VDN_OK, where
+    return inp, cfg, ha, t, y.float().cpu().numpy().astype(np.float64)
+
+
+def rel_err(got, ref, store_bf16=False):
+    """max |got - ref| / RMS(ref).  A slot that is exactly zero in the oracle
+    (no state to read) must be exactly zero.  With a bf16-stored output the
+    rounding of the store itself (at most 2^-9 |y| per element, half an ulp)
+    is taken off before the comparison."""
+    rms = np.sqrt(np.mean(ref ** 2))
+    diff = np.abs(got - ref)
+    if store_bf16:
+        diff = np.maximum(diff - 2.0 ** -9 * np.abs(ref) * (1 + 2.0 ** -8), 0.0)
+    if rms == 0:
+        return 0.0 if np.max(diff) == 0 else float("inf")
+    return float(np.max(diff) / rms)
+
+
+def check(got, ref, cfg, dtype):
+    tol = TOL[dtype]
+    sb = cfg.y_dtype == L.VDN_BF16
+    if cfg.out_mode == 0:
+        for s, name in ((0, "softmax"), (1, "linear")):
+            e = rel_err(got[..., s, :], ref[..., s, :], sb)
+            assert e <= tol, f"{name} slot: max err {e:.3g} x RMS > {tol}"
+    else:
+        e = rel_err(got, ref, sb)
+        assert e <= tol, f"summed output: max err {e:.3g} x RMS > {tol}"
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_scan", "small"])
+def test_workload_full_parity(name):
+    w = WORKLOADS[name]
+    inp, cfg, _, _, y = run(w.shape, w.dtype, w.seed)
+    check(y, O.hybrid_attn(inp, ocfg(cfg)), cfg, w.dtype)
+
+
+CASES = {
+    "d128": (Shape(1, 15, 40, 2, 128, 128, 16), {}),
+    "d64_ragged_N": (Shape(1, 20, 17, 3, 64, 64, 5), {}),
+    "no_anchors": (Shape(1, 25, 12, 2, 32, 32, 4), dict(anchors=0)),
+    "partial_chunk_T23": (Shape(1, 23, 9, 2, 64, 64, 3), {}),
+    "T2_all_anchor": (Shape(1, 2, 33, 2, 32, 32, 3), {}),
+    "T7": (Shape(1, 7, 20, 1, 64, 64, 0), {}),
+    "batch2": (Shape(2, 15, 24, 2, 64, 64, 6), {}),
+    "scale10": (Shape(1, 20, 16, 2, 64, 64, 8), dict(softmax_scale=10.0)),
+    "summed_out": (Shape(1, 20, 16, 2, 64, 64, 8), dict(out_mode=1)),
+    "eps": (Shape(1, 10, 8, 2, 32, 32, 4), dict(rms_eps=0.5)),
+    "y_bf16": (Shape(1, 20, 24, 2, 64, 64, 8), dict(y_dtype=L.VDN_BF16)),
+    "y_bf16_summed": (Shape(1, 20, 24, 2, 64, 64, 8), dict(y_dtype=L.VDN_BF16, out_mode=1)),
+}
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_edge_case_parity(case, dtype):
+    shape, kw = CASES[case]
+    inp, cfg, _, _, y = run(shape, dtype, 7, **kw)
+    check(y, O.hybrid_attn(inp, ocfg(cfg)), cfg, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_init_state_and_rms_weight(dtype):
+    shape = Shape(1, 20, 16, 2, 64, 64, 0)
+    r = np.random.default_rng(5)
+    extra = {"init_state": r.standard_normal((1, 2, 64, 64)).astype(np.float32) * 0.3,
+             "rms_weight": (1 + 0.5 * r.standard_normal((2, 64))).astype(np.float32)}
+    inp, cfg, _, _, y = run(shape, dtype, 9, extra=extra, drop_text=True)
+    check(y, O.hybrid_attn(inp, ocfg(cfg)), cfg, dtype)
+
+
+def test_zero_text_state():
+    inp, cfg, _, _, y = run(Shape(1, 20, 8, 2, 32, 32, 0), "f32", 3, drop_text=True)
+    check(y, O.hybrid_attn(inp, ocfg(cfg)), cfg, "f32")
+
+
+def test_intermediates_match_oracle():
+    """Stage outputs in the workspace: text state, (M_t, C_t), snapshots, R."""
+    w = WORKLOADS["tiny_scan"]
+    inp, cfg, ha, _, _ = run(w.shape, "f32", w.seed)
+    it = {k: v.double().cpu().numpy() for k, v in ha.intermediates().items()}
+    oc = ocfg(cfg)
+    for h in range(cfg.H):
+        ref = O.vda_intermediates(inp, oc, 0, h)
+        scale = np.sqrt(np.mean(ref["R"] ** 2))
+        np.testing.assert_allclose(it["half_text"][0, h], ref["S_init"], atol=1e-5 * scale)
+        for t in range(1, cfg.T - 1):
+            np.testing.assert_allclose(it["M"][0, t, h], ref["M"][t], atol=1e-5)
+            np.testing.assert_allclose(it["C"][0, t, h], ref["C"][t], atol=1e-5 * np.abs(ref["C"][t]).max())
+        for j in range(cfg.C + 1):
+            fj = min(5 * j, cfg.T)
+            np.testing.assert_allclose(it["fwd_snap"][0, h, j], ref["F"][fj], atol=1e-5 * scale)
+            np.testing.assert_allclose(it["bwd_snap"][0, h, j], ref["G"][fj], atol=1e-5 * scale)
+        np.testing.assert_allclose(it["R"][0, h], ref["R"], atol=1e-5 * scale)
+
+
+def test_stages_compose_to_full_call_and_are_deterministic():
+    w = WORKLOADS["small"]
+    inp, cfg, ha, t, y = run(w.shape, w.dtype, w.seed)
+    y2 = ha(t).float().cpu().numpy()
+    assert np.array_equal(y, y2)
+    ha.y.zero_()
+    for st in (L.STAGE_TEXT, L.STAGE_SOLVE, L.STAGE_SCAN, L.STAGE_SOFTMAX, L.STAGE_READ):
+        ha(t, stages=st)
+    torch.cuda.synchronize()
+    assert np.array_equal(y, ha.y.float().cpu().numpy())
+
+
+def _sample_rows(cfg, heads, per_head, rng):
+    T, N = cfg.T, cfg.N
+    rows = []
+    for b in range(cfg.B):
+        for h in heads:
+            frames = [0, 1, 4, 5, 9, 10, T // 2, T - 6, T - 5, T - 2, T - 1]
+            for t in frames:
+                for n in (0, N - 1, int(rng.integers(N))):
+                    rows.append((b, t, n, h))
+            for _ in range(per_head):
+                rows.append((b, int(rng.integers(T)), int(rng.integers(N)), h))
+    return rows
+
+
+@pytest.mark.parametrize("name", ["768p"])
+def test_full_size_sampled_parity(name):
+    """At the benchmark's size and launch configuration (inputs drawn on the
+    device): sampled outputs against the oracle evaluated position by
+    position on two heads."""
+    from video_diffusion_hybrid_b200.synth import head_slice, make_inputs_torch
+    w = WORKLOADS[name]
+    t = make_inputs_torch(w.shape, w.seed, w.dtype, "cuda")
+    cfg = cfg_for(w.shape, w.dtype)
+    ha = HybridAttention(cfg)
+    y = ha(t)
+    torch.cuda.synchronize()
+    assert L.vdn_hybrid_device_status(cfg, ha.args(t))[0] == L.VDN_OK
+    assert bool(torch.isfinite(y).all())
+    rng = np.random.default_rng(0)
+    s = w.shape
+    for h in (0, s.H - 1):
+        inp = head_slice(t, 0, h)
+        oc = O.Cfg(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
+        rows = _sample_rows(oc, heads=(0,), per_head=24, rng=rng)
+        ref = O.hybrid_attn_rows(inp, oc, rows)
+        idx = torch.tensor([(t_, n) for (_, t_, n, _) in rows], device=y.device)
+        got = y[0, idx[:, 0], idx[:, 1], h].float().cpu().numpy()
+        for sl in (0, 1):
+            rms = np.sqrt(np.mean(ref[:, sl] ** 2))
+            err = np.max(np.abs(got[:, sl] - ref[:, sl])) / rms
+            assert err <= TOL[w.dtype], (h, sl, err)

@@ -1,0 +1,179 @@
+"""ctypes binding of ``libvdn_hybrid.so`` (the C ABI in ``include/vdn_hybrid.h``).
+
+Argument marshalling only: every step of the hybrid attention core runs in
+the library's CUDA kernels.  Names follow the C entry points.  Torch is used
+for device memory and streams; the functions accept torch tensors and pass
+their device pointers.  There is no fallback: if the library is missing the
+first call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass, fields
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libvdn_hybrid.so")
+
+VDN_OK, VDN_ERR_INVALID_ARG, VDN_ERR_UNSUPPORTED, VDN_ERR_WORKSPACE, VDN_ERR_CUDA, VDN_ERR_TIMEOUT = range(6)
+VDN_F32, VDN_BF16 = 0, 1
+STAGE_TEXT, STAGE_SOLVE, STAGE_SCAN, STAGE_SOFTMAX, STAGE_READ = 1, 2, 4, 8, 16
+STAGE_ALL = 31
+
+EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
+            "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
+            "vdn_status_string")
+
+
+class VdnCfg(C.Structure):
+    _fields_ = [("B", C.c_int), ("T", C.c_int), ("N", C.c_int), ("H", C.c_int), ("d_k", C.c_int),
+                ("d_v", C.c_int), ("L", C.c_int), ("chunk", C.c_int), ("anchors", C.c_int),
+                ("dtype", C.c_int), ("softmax_scale", C.c_float), ("rms_eps", C.c_float),
+                ("out_mode", C.c_int), ("y_dtype", C.c_int)]
+
+
+class VdnArgs(C.Structure):
+    _fields_ = [("q", C.c_void_p), ("k", C.c_void_p), ("v", C.c_void_p), ("beta", C.c_void_p),
+                ("alpha", C.c_void_p), ("gate_sm", C.c_void_p), ("gate_lin", C.c_void_p),
+                ("text_k", C.c_void_p), ("text_v", C.c_void_p), ("text_beta", C.c_void_p),
+                ("init_state", C.c_void_p), ("rms_weight", C.c_void_p), ("y", C.c_void_p),
+                ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t)]
+
+
+class VdnLayout(C.Structure):
+    _fields_ = [(n, C.c_size_t) for n in ("status", "half_text", "frame_M", "frame_C", "fwd_snap",
+                                          "bwd_snap", "read_table", "total")]
+
+
+@dataclass
+class HybridCfg:
+    """Mirror of ``vdn_hybrid_cfg``."""
+    B: int
+    T: int
+    N: int
+    H: int
+    d_k: int
+    d_v: int
+    L: int = 0
+    chunk: int = 5
+    anchors: int = 4
+    dtype: int = VDN_F32
+    softmax_scale: float = 0.0
+    rms_eps: float = 0.0
+    out_mode: int = 0
+    y_dtype: int = VDN_F32
+
+    def c(self) -> VdnCfg:
+        return VdnCfg(**{f.name: getattr(self, f.name) for f in fields(self)})
+
+    @property
+    def C(self) -> int:
+        return -(-self.T // self.chunk)
+
+
+class VdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run video_diffusion_hybrid_b200/build.py "
+                               "(there is no CPU fallback)")
+        L = C.CDLL(LIB_PATH)
+        L.vdn_hybrid_attn_workspace_size.restype = C.c_size_t
+        L.vdn_hybrid_attn_workspace_size.argtypes = [C.POINTER(VdnCfg)]
+        L.vdn_hybrid_workspace_layout.restype = C.c_int
+        L.vdn_hybrid_workspace_layout.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnLayout)]
+        L.vdn_hybrid_attn_fwd.restype = C.c_int
+        L.vdn_hybrid_attn_fwd.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
+        L.vdn_hybrid_attn_fwd_stages.restype = C.c_int
+        L.vdn_hybrid_attn_fwd_stages.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_uint, C.c_void_p]
+        L.vdn_hybrid_device_status.restype = C.c_int
+        L.vdn_hybrid_device_status.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p,
+                                               C.POINTER(C.c_uint)]
+        L.vdn_hybrid_stage_impl.restype = C.c_int
+        L.vdn_hybrid_stage_impl.argtypes = [C.POINTER(VdnCfg), C.c_uint]
+        L.vdn_status_string.restype = C.c_char_p
+        L.vdn_status_string.argtypes = [C.c_int]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().vdn_status_string(status).decode()
+
+
+def vdn_hybrid_attn_workspace_size(cfg: HybridCfg) -> int:
+    c = cfg.c()
+    return int(lib().vdn_hybrid_attn_workspace_size(C.byref(c)))
+
+
+def vdn_hybrid_workspace_layout(cfg: HybridCfg) -> dict:
+    c, out = cfg.c(), VdnLayout()
+    st = lib().vdn_hybrid_workspace_layout(C.byref(c), C.byref(out))
+    if st != VDN_OK:
+        raise VdnError(st, "vdn_hybrid_workspace_layout")
+    return {n: int(getattr(out, n)) for n, _ in VdnLayout._fields_}
+
+
+def vdn_hybrid_stage_impl(cfg: HybridCfg, stage: int) -> int:
+    c = cfg.c()
+    return int(lib().vdn_hybrid_stage_impl(C.byref(c), stage))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def make_args(q, k, v, beta, alpha, gate_sm, gate_lin, y, workspace, workspace_bytes=None,
+              text_k=None, text_v=None, text_beta=None, init_state=None, rms_weight=None) -> VdnArgs:
+    """Build a ``vdn_hybrid_args`` from torch tensors (or raw integer device
+    pointers).  The caller keeps the tensors alive for the call."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return VdnArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate_sm), _ptr(gate_lin),
+                   _ptr(text_k), _ptr(text_v), _ptr(text_beta), _ptr(init_state), _ptr(rms_weight),
+                   _ptr(y), _ptr(workspace), int(workspace_bytes))
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def vdn_hybrid_attn_fwd(cfg: HybridCfg, args: VdnArgs, stream=None, check: bool = True) -> int:
+    c = cfg.c()
+    st = lib().vdn_hybrid_attn_fwd(C.byref(c), C.byref(args), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_hybrid_attn_fwd")
+    return st
+
+
+def vdn_hybrid_attn_fwd_stages(cfg: HybridCfg, args: VdnArgs, stages: int, stream=None, check: bool = True) -> int:
+    c = cfg.c()
+    st = lib().vdn_hybrid_attn_fwd_stages(C.byref(c), C.byref(args), stages, _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_hybrid_attn_fwd_stages")
+    return st
+
+
+def vdn_hybrid_device_status(cfg: HybridCfg, args: VdnArgs, stream=None) -> tuple:
+    c, where = cfg.c(), C.c_uint(0)
+    st = lib().vdn_hybrid_device_status(C.byref(c), C.byref(args), _stream_handle(stream), C.byref(where))
+    return st, int(where.value)

@@ -1,0 +1,88 @@
+"""Torch-facing helpers over the C ABI: device placement of the inputs and a
+small callable that owns nothing but a workspace and an output buffer.
+
+Every byte of compute runs in ``libvdn_hybrid.so``; torch provides device
+memory and the current stream.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import _lib as L
+from .synth import Shape
+
+TENSOR_NAMES = ("q", "k", "v", "beta", "alpha", "gate_sm", "gate_lin", "text_k", "text_v", "text_beta",
+                "init_state", "rms_weight")
+
+
+def cfg_for(shape: Shape, dtype: str, **kw) -> L.HybridCfg:
+    return L.HybridCfg(B=shape.B, T=shape.T, N=shape.N, H=shape.H, d_k=shape.d_k, d_v=shape.d_v, L=shape.L,
+                       dtype=L.VDN_BF16 if dtype == "bf16" else L.VDN_F32, **kw)
+
+
+def to_torch(inp: dict, dtype: str, device="cuda", pin: bool = False) -> dict:
+    """Move the synthetic inputs to `device` in their storage types (bf16
+    tensors from their exact bit patterns).  With device="cpu" and pin=True
+    the result lives in pinned host memory."""
+    out = {}
+    for name in TENSOR_NAMES:
+        if name not in inp:
+            continue
+        if dtype == "bf16" and name + "_bits" in inp:
+            t = torch.from_numpy(np.ascontiguousarray(inp[name + "_bits"]).view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(np.ascontiguousarray(inp[name], dtype=np.float32))
+        if pin:
+            t = t.pin_memory()
+        out[name] = t.to(device) if device != "cpu" else t
+    return out
+
+
+def output_shape(cfg: L.HybridCfg) -> tuple:
+    base = (cfg.B, cfg.T, cfg.N, cfg.H)
+    return base + ((2, cfg.d_v) if cfg.out_mode == 0 else (cfg.d_v,))
+
+
+class HybridAttention:
+    """Calls ``vdn_hybrid_attn_fwd`` on torch tensors.  Workspace and output
+    are allocated once (by torch) and reused."""
+
+    def __init__(self, cfg: L.HybridCfg, device="cuda"):
+        self.cfg = cfg
+        self.ws_bytes = L.vdn_hybrid_attn_workspace_size(cfg)
+        if self.ws_bytes == 0:
+            raise L.VdnError(L.VDN_ERR_INVALID_ARG, "vdn_hybrid_attn_workspace_size")
+        self.device = torch.device(device)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        tdt = torch.bfloat16 if cfg.y_dtype == L.VDN_BF16 else torch.float32
+        self.y = torch.empty(output_shape(cfg), dtype=tdt, device=self.device)
+
+    def args(self, t: dict) -> L.VdnArgs:
+        return L.make_args(t["q"], t["k"], t["v"], t["beta"], t["alpha"], t["gate_sm"], t["gate_lin"], self.y,
+                           self.workspace, self.ws_bytes, text_k=t.get("text_k"), text_v=t.get("text_v"),
+                           text_beta=t.get("text_beta"), init_state=t.get("init_state"),
+                           rms_weight=t.get("rms_weight"))
+
+    def __call__(self, t: dict, stages: int = L.STAGE_ALL, stream=None) -> torch.Tensor:
+        a = self.args(t)
+        if stages == L.STAGE_ALL:
+            L.vdn_hybrid_attn_fwd(self.cfg, a, stream)
+        else:
+            L.vdn_hybrid_attn_fwd_stages(self.cfg, a, stages, stream)
+        return self.y
+
+    def intermediates(self) -> dict:
+        """Views of the workspace's intermediate values (float32)."""
+        lay = L.vdn_hybrid_workspace_layout(self.cfg)
+        c = self.cfg
+        C = c.C
+        f = lambda off, shape: self.workspace[off:off + 4 * int(np.prod(shape))].view(torch.float32).view(*shape)
+        return {
+            "half_text": f(lay["half_text"], (c.B, c.H, c.d_v, c.d_k)),
+            "M": f(lay["frame_M"], (c.B, c.T, c.H, c.d_k, c.d_k)),
+            "C": f(lay["frame_C"], (c.B, c.T, c.H, c.d_v, c.d_k)),
+            "fwd_snap": f(lay["fwd_snap"], (c.B, c.H, C + 1, c.d_v, c.d_k)),
+            "bwd_snap": f(lay["bwd_snap"], (c.B, c.H, C + 1, c.d_v, c.d_k)),
+            "R": f(lay["read_table"], (c.B, c.H, C + 1, c.d_v, c.d_k)),
+        }

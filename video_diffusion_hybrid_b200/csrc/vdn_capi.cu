@@ -1,0 +1,215 @@
+// C ABI entry points: argument validation, workspace layout, stage dispatch.
+#include <cstdint>
+#include <cstring>
+
+#include "vdn_internal.h"
+
+namespace vdn {
+
+cudaError_t launch_softmax_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+bool softmax_tc_supported(const Dims& d);
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+vdn_status check_cfg(const vdn_hybrid_cfg* c) {
+  if (!c) return VDN_ERR_INVALID_ARG;
+  if (c->B < 1 || c->T < 2 || c->N < 1 || c->H < 1 || c->L < 0) return VDN_ERR_INVALID_ARG;
+  if (c->d_k < 1 || c->d_v < 1 || c->chunk < 1) return VDN_ERR_INVALID_ARG;
+  if (c->anchors != 0 && c->anchors != 4) return VDN_ERR_INVALID_ARG;
+  if (c->dtype != VDN_F32 && c->dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
+  if (c->out_mode != 0 && c->out_mode != 1) return VDN_ERR_INVALID_ARG;
+  if (c->y_dtype != VDN_F32 && c->y_dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
+  if (!(c->softmax_scale == c->softmax_scale) || !(c->rms_eps == c->rms_eps)) return VDN_ERR_INVALID_ARG;
+  if (c->d_k != 32 && c->d_k != 64 && c->d_k != 128) return VDN_ERR_UNSUPPORTED;
+  if (c->d_v != c->d_k) return VDN_ERR_UNSUPPORTED;
+  if (c->chunk != 5) return VDN_ERR_UNSUPPORTED;
+  // grid limits of the launches (gridDim.y / gridDim.z <= 65535)
+  if ((long long)c->B * c->H > 65535) return VDN_ERR_UNSUPPORTED;
+  if (c->T / c->chunk + 3 > 65535) return VDN_ERR_UNSUPPORTED;
+  // element counts must fit comfortably in int64 index arithmetic
+  const double tokens = (double)c->B * c->T * c->N * c->H * (double)c->d_k;
+  if (tokens * 2.0 > 9.0e18) return VDN_ERR_UNSUPPORTED;
+  return VDN_OK;
+}
+
+Dims make_dims(const vdn_hybrid_cfg* c) {
+  Dims d;
+  d.B = c->B; d.T = c->T; d.N = c->N; d.H = c->H; d.dk = c->d_k; d.dv = c->d_v; d.L = c->L;
+  d.chunk = c->chunk; d.anchors = c->anchors; d.C = (c->T + c->chunk - 1) / c->chunk;
+  d.scale = c->softmax_scale > 0.f ? c->softmax_scale : 1.0f / sqrtf((float)c->d_k);
+  d.eps = c->rms_eps > 0.f ? c->rms_eps : 1e-6f;
+  d.out_mode = c->out_mode;
+  d.bf16 = c->dtype == VDN_BF16;
+  d.out_bf16 = c->y_dtype == VDN_BF16;
+  return d;
+}
+
+void layout_of(const vdn_hybrid_cfg* c, vdn_workspace_layout* L) {
+  const size_t C = (size_t)((c->T + c->chunk - 1) / c->chunk);
+  const size_t dd = (size_t)c->d_v * c->d_k * sizeof(float);
+  const size_t bh = (size_t)c->B * c->H;
+  size_t off = 0;
+  L->status = off;     off += up(kAlign);
+  L->half_text = off;  off += up(bh * dd);
+  L->frame_M = off;    off += up(bh * (size_t)c->T * (size_t)c->d_k * c->d_k * sizeof(float));
+  L->frame_C = off;    off += up(bh * (size_t)c->T * dd);
+  L->fwd_snap = off;   off += up(bh * (C + 1) * dd);
+  L->bwd_snap = off;   off += up(bh * (C + 1) * dd);
+  L->read_table = off; off += up(bh * (C + 1) * dd);
+  L->total = off;
+}
+
+vdn_status check_args(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a, unsigned stages) {
+  if (!a) return VDN_ERR_INVALID_ARG;
+  if ((stages & ~(unsigned)VDN_STAGE_ALL) != 0 || stages == 0) return VDN_ERR_INVALID_ARG;
+  const void* req[] = {a->q, a->k, a->v, a->beta, a->alpha, a->gate_sm, a->gate_lin, a->y};
+  for (const void* p : req)
+    if (!p || !aligned(p, 16)) return VDN_ERR_INVALID_ARG;
+  if (c->L > 0) {
+    if (!a->text_k || !a->text_v || !a->text_beta || a->init_state) return VDN_ERR_INVALID_ARG;
+    if (!aligned(a->text_k, 16) || !aligned(a->text_v, 16) || !aligned(a->text_beta, 4))
+      return VDN_ERR_INVALID_ARG;
+  } else if (a->text_k || a->text_v || a->text_beta) {
+    return VDN_ERR_INVALID_ARG;
+  }
+  if (a->init_state && !aligned(a->init_state, 16)) return VDN_ERR_INVALID_ARG;
+  if (a->rms_weight && !aligned(a->rms_weight, 4)) return VDN_ERR_INVALID_ARG;
+  vdn_workspace_layout L;
+  layout_of(c, &L);
+  if (!a->workspace || !aligned(a->workspace, kAlign) || a->workspace_bytes < L.total) return VDN_ERR_WORKSPACE;
+  return VDN_OK;
+}
+
+Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
+  vdn_workspace_layout L;
+  layout_of(c, &L);
+  char* base = static_cast<char*>(a->workspace);
+  Work w;
+  w.status = reinterpret_cast<uint32_t*>(base + L.status);
+  w.half_text = reinterpret_cast<float*>(base + L.half_text);
+  w.M = reinterpret_cast<float*>(base + L.frame_M);
+  w.Cm = reinterpret_cast<float*>(base + L.frame_C);
+  w.fsnap = reinterpret_cast<float*>(base + L.fwd_snap);
+  w.bsnap = reinterpret_cast<float*>(base + L.bwd_snap);
+  w.R = reinterpret_cast<float*>(base + L.read_table);
+  return w;
+}
+
+Inputs inputs_of(const vdn_hybrid_args* a) {
+  Inputs in;
+  in.q = a->q; in.k = a->k; in.v = a->v; in.beta = a->beta; in.alpha = a->alpha;
+  in.gate_sm = a->gate_sm; in.gate_lin = a->gate_lin;
+  in.text_k = a->text_k; in.text_v = a->text_v; in.text_beta = a->text_beta;
+  in.init_state = a->init_state; in.rms_weight = a->rms_weight; in.y = a->y;
+  return in;
+}
+
+}  // namespace
+}  // namespace vdn
+
+using namespace vdn;
+
+extern "C" {
+
+size_t vdn_hybrid_attn_workspace_size(const vdn_hybrid_cfg* cfg) {
+  if (check_cfg(cfg) != VDN_OK) return 0;
+  vdn_workspace_layout L;
+  layout_of(cfg, &L);
+  return L.total;
+}
+
+vdn_status vdn_hybrid_workspace_layout(const vdn_hybrid_cfg* cfg, vdn_workspace_layout* out) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!out) return VDN_ERR_INVALID_ARG;
+  layout_of(cfg, out);
+  return VDN_OK;
+}
+
+int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
+  if (check_cfg(cfg) != VDN_OK) return -1;
+  Dims d = make_dims(cfg);
+  switch (stage) {
+    case VDN_STAGE_TEXT:
+    case VDN_STAGE_SOLVE:
+    case VDN_STAGE_SCAN:
+    case VDN_STAGE_READ:
+      return 0;
+    case VDN_STAGE_SOFTMAX:
+      return softmax_tc_supported(d) ? 1 : 0;
+    default:
+      return -1;
+  }
+}
+
+vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, unsigned stages,
+                                      vdn_stream_t stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  st = check_args(cfg, args, stages);
+  if (st != VDN_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const Dims d = make_dims(cfg);
+  const Work w = work_of(cfg, args);
+  const Inputs in = inputs_of(args);
+  cudaError_t e = cudaSuccess;
+  if (cudaMemsetAsync(w.status, 0, 256, s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (stages & VDN_STAGE_TEXT) {
+    if ((e = launch_text(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+  }
+  if (stages & VDN_STAGE_SOLVE) {
+    if ((e = launch_solve_simt(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+  }
+  if (stages & VDN_STAGE_SCAN) {
+    if ((e = launch_scan_simt(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+  }
+  if (stages & VDN_STAGE_SOFTMAX) {
+    e = softmax_tc_supported(d) ? launch_softmax_tc(d, in, w, s) : launch_softmax_simt(d, in, w, s);
+    if (e != cudaSuccess) return VDN_ERR_CUDA;
+  }
+  if (stages & VDN_STAGE_READ) {
+    if ((e = launch_read_simt(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+  }
+  return VDN_OK;
+}
+
+vdn_status vdn_hybrid_attn_fwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, vdn_stream_t stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  st = check_args(cfg, args, VDN_STAGE_ALL);
+  if (st != VDN_OK) return st;
+  return vdn_hybrid_attn_fwd_stages(cfg, args, VDN_STAGE_ALL, stream);
+}
+
+vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, vdn_stream_t stream,
+                                    unsigned* where) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!args || !args->workspace) return VDN_ERR_INVALID_ARG;
+  const Work w = work_of(cfg, args);
+  uint32_t host[2] = {0, 0};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host, w.status, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (where) *where = host[1];
+  return host[0] ? VDN_ERR_TIMEOUT : VDN_OK;
+}
+
+const char* vdn_status_string(vdn_status s) {
+  switch (s) {
+    case VDN_OK: return "ok";
+    case VDN_ERR_INVALID_ARG: return "invalid argument";
+    case VDN_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case VDN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case VDN_ERR_CUDA: return "CUDA error";
+    case VDN_ERR_TIMEOUT: return "a bounded device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/vdn_hybrid.h"
+
+namespace vdn {
+
+// Problem description handed to every kernel (by value).
+struct Dims {
+  int B, T, N, H, dk, dv, L, chunk, anchors, C;
+  float scale, eps;
+  int out_mode;
+  int bf16;      // inputs stored as bf16
+  int out_bf16;  // y stored as bf16
+};
+
+// Device-side status words at the head of the workspace.
+enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3 };
+
+struct Work {
+  uint32_t* status;
+  float* half_text;  // [B,H,dv,dk]
+  float* M;          // [B,T,H,dk,dk]
+  float* Cm;         // [B,T,H,dv,dk]
+  float* fsnap;      // [B,H,C+1,dv,dk]
+  float* bsnap;      // [B,H,C+1,dv,dk]
+  float* R;          // [B,H,C+1,dv,dk]
+};
+
+struct Inputs {
+  const void *q, *k, *v;
+  const float *beta, *alpha;
+  const void *gate_sm, *gate_lin;
+  const void *text_k, *text_v;
+  const float *text_beta, *init_state, *rms_weight;
+  void* y;
+};
+
+__host__ __device__ inline bool is_anchor(const Dims& d, int t) {
+  return d.anchors != 0 && (t == 0 || t == d.T - 1);
+}
+
+// Launchers (return cudaGetLastError after the launch).
+cudaError_t launch_text(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_solve_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_read_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_softmax_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+
+}  // namespace vdn

@@ -1,0 +1,47 @@
+"""Algorithmic work of the hybrid attention core, for roofline fractions.
+
+These are counts of what the method must compute or move at minimum
+(independent of any kernel's blocking), used by the benchmark:
+
+* softmax: 4 * d * (allowed query-key token pairs) per head -- QK^T and PV,
+  one multiply-add (2 flops) each per pair and dimension;
+* Gram/write: 2 * N * (d_k^2 + d_v d_k) per non-anchor frame-head;
+* read: 2 * d_k * d_v per query token and head;
+* bytes: each input read once and each output written once.
+"""
+from __future__ import annotations
+
+
+def allowed_frame_pairs(T: int, chunk: int = 5, anchors: int = 4) -> int:
+    """Number of (query frame, key frame) pairs on the softmax path."""
+    total = 0
+    for tq in range(T):
+        if anchors and tq in (0, T - 1):
+            total += T
+            continue
+        c = tq // chunk
+        lo, hi = max(0, (c - 1) * chunk), min(T, (c + 2) * chunk)
+        n = hi - lo
+        if anchors:
+            n += (1 if lo > 0 else 0) + (1 if hi < T and T - 1 >= hi else 0)
+        total += n
+    return total
+
+
+def softmax_flops(B, T, N, H, d, chunk=5, anchors=4) -> float:
+    return 4.0 * d * allowed_frame_pairs(T, chunk, anchors) * N * N * H * B
+
+
+def gram_flops(B, T, N, H, d, anchors=4) -> float:
+    frames = T - (2 if anchors and T >= 2 else 0)
+    return 2.0 * N * (2 * d * d) * frames * H * B
+
+
+def read_flops(B, T, N, H, d) -> float:
+    return 2.0 * d * d * B * T * N * H
+
+
+def softmax_bytes(B, T, N, H, d, elem=2, out_slot_bytes=None) -> float:
+    """q, k, v, gate_sm read once; y softmax slot written once."""
+    tok = B * T * N * H * d
+    return tok * elem * 4 + tok * (out_slot_bytes or elem)

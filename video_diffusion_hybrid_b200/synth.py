@@ -15,6 +15,12 @@ Recipe (per batch element b, its own PCG64 stream seeded ``seed * 1000 + b``):
 
 In bf16 mode every bf16-stored tensor is rounded to bf16 (round to nearest
 even) here, and the *rounded* values are what both paths see.
+
+``make_inputs`` draws on the host (NumPy PCG64) and suits the sizes the
+oracle evaluates in full.  ``make_inputs_torch`` draws the same recipe with
+torch's seeded generator directly on a device (its stream differs from
+PCG64's), for the full-size workloads; ``head_slice`` then copies one
+(batch, head) of those tensors back to the host for the oracle.
 """
 from __future__ import annotations
 
@@ -37,10 +43,10 @@ class Shape:
 
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
-    """float32 -> nearest-even bf16, returned as uint16 bit patterns."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    """float32 -> nearest-even bf16, returned as uint16 bit patterns
+    (finite inputs; the carry cannot overflow 32 bits below the NaN range)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return u.astype(np.uint16)
 
 
@@ -92,3 +98,56 @@ def make_inputs(shape: Shape, seed: int, dtype: str = "f32") -> dict:
     elif dtype != "f32":
         raise ValueError(f"unknown dtype {dtype!r}")
     return inp
+
+
+def make_inputs_torch(shape: Shape, seed: int, dtype: str = "bf16", device="cuda") -> dict:
+    """The same recipe drawn with a seeded ``torch.Generator`` on `device`.
+    Returns torch tensors in their storage types (bf16-stored tensors already
+    rounded; beta/alpha/text_beta float32), with a leading batch axis."""
+    import torch
+    st = torch.bfloat16 if dtype == "bf16" else torch.float32
+    T, N, H = shape.T, shape.N, shape.H
+    parts = []
+    for b in range(shape.B):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed * 1000 + b)
+
+        def rn(*sz):
+            return torch.randn(*sz, generator=g, device=device, dtype=torch.float32)
+
+        def l2n(x):
+            return x / x.double().norm(dim=-1, keepdim=True).clamp_min(1e-30).float()
+
+        p = {
+            "q": l2n(rn(T, N, H, shape.d_k)).to(st),
+            "k": l2n(rn(T, N, H, shape.d_k)).to(st),
+            "v": rn(T, N, H, shape.d_v).to(st),
+            "beta": torch.sigmoid(rn(T, N, H)),
+            "alpha": torch.sigmoid(2.0 + 0.5 * rn(T, H)),
+            "gate_sm": rn(T, N, H, shape.d_v).to(st),
+            "gate_lin": rn(T, N, H, shape.d_v).to(st),
+        }
+        if shape.L > 0:
+            p["text_k"] = l2n(rn(shape.L, H, shape.d_k)).to(st)
+            p["text_v"] = rn(shape.L, H, shape.d_v).to(st)
+            p["text_beta"] = torch.sigmoid(rn(shape.L, H))
+        parts.append(p)
+    return {k: torch.stack([p[k] for p in parts]).contiguous() for k in parts[0]}
+
+
+def head_slice(t: dict, b: int, h: int) -> dict:
+    """One (batch, head) of device inputs as float32 NumPy arrays with unit
+    batch and head axes, for the oracle."""
+    out = {}
+    for k, x in t.items():
+        if k in ("init_state",):
+            y = x[b:b + 1, h:h + 1]
+        elif k == "rms_weight":
+            y = x[h:h + 1]
+        elif x.dim() >= 3:
+            y = x[b:b + 1, :, :, h:h + 1] if x.dim() >= 4 and k not in ("text_k", "text_v") else \
+                x[b:b + 1, :, h:h + 1]
+        else:
+            y = x[b:b + 1, :, h:h + 1]
+        out[k] = y.float().cpu().numpy()
+    return out
