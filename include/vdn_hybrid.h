@@ -142,6 +142,27 @@ vdn_status vdn_hybrid_attn_fwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args 
 vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
                                       unsigned stages, vdn_stream_t stream);
 
+/* The whole core without a caller workspace, for callers that cannot
+ * allocate device memory where they run it: runtimes that forbid allocation
+ * after start-up, and plug-ins of another framework that are handed only their
+ * input and output buffers.  The pages have no counterpart of this entry
+ * point; it is a deployment convenience of this library.
+ * Scratch: a library-owned device array of VDN_NOALLOC_SCRATCH_BYTES (static
+ * storage on every GPU that loads the library, held until the process exits).
+ * Arguments are those of vdn_hybrid_attn_fwd, except that args->workspace must
+ * be NULL and args->workspace_bytes 0 (else VDN_ERR_INVALID_ARG).  A cfg whose
+ * workspace (vdn_hybrid_attn_workspace_size) exceeds VDN_NOALLOC_SCRATCH_BYTES
+ * returns VDN_ERR_WORKSPACE and launches nothing.
+ * Set-up: the first call on each device looks up the array's device address
+ * with that device current; make that first call before any stream capture.
+ * Sharing: every call uses the same array, which keeps the last call's
+ * contents (each call clears what must start at zero); calls whose work
+ * overlaps on the GPU race on it and must be serialised by the caller.  The
+ * device status words of these calls are not readable by the caller. */
+#define VDN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+vdn_status vdn_hybrid_attn_fwd_noalloc(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
+                                       vdn_stream_t stream);
+
 /* Reads the device status words left by the most recent call on this
  * workspace (every fwd / fwd_stages call clears them first; synchronises `stream`).
  * Returns VDN_OK or VDN_ERR_TIMEOUT; *where (if not NULL) gets the kernel tag

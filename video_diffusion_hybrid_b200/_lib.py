@@ -22,7 +22,8 @@ STAGE_ALL = 31
 
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
-            "vdn_status_string")
+            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class VdnCfg(C.Structure):
@@ -101,6 +102,8 @@ def lib() -> C.CDLL:
                                                C.POINTER(C.c_uint)]
         L.vdn_hybrid_stage_impl.restype = C.c_int
         L.vdn_hybrid_stage_impl.argtypes = [C.POINTER(VdnCfg), C.c_uint]
+        L.vdn_hybrid_attn_fwd_noalloc.restype = C.c_int
+        L.vdn_hybrid_attn_fwd_noalloc.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
         L.vdn_status_string.restype = C.c_char_p
         L.vdn_status_string.argtypes = [C.c_int]
         _lib = L
@@ -177,3 +180,13 @@ def vdn_hybrid_device_status(cfg: HybridCfg, args: VdnArgs, stream=None) -> tupl
     c, where = cfg.c(), C.c_uint(0)
     st = lib().vdn_hybrid_device_status(C.byref(c), C.byref(args), _stream_handle(stream), C.byref(where))
     return st, int(where.value)
+
+
+def vdn_hybrid_attn_fwd_noalloc(cfg: HybridCfg, args: VdnArgs, stream=None, check: bool = True) -> int:
+    """The core with the library's own fixed scratch (args.workspace must be
+    None, workspace_bytes 0), for callers that cannot allocate."""
+    c = cfg.c()
+    st = lib().vdn_hybrid_attn_fwd_noalloc(C.byref(c), C.byref(args), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_hybrid_attn_fwd_noalloc")
+    return st

@@ -1,0 +1,66 @@
+// The hybrid attention core for callers that cannot allocate device memory.
+//
+// Some callers of this library cannot call cudaMalloc (or any allocator) at
+// the point where they run the core: code that runs inside another
+// framework's memory pool, hard real-time or certified runtimes that forbid
+// allocation after start-up, and plug-ins handed only the input and output
+// buffers.  For them this file keeps the core's scratch in a fixed device
+// array that the library owns, so the caller passes inputs and outputs only.
+//
+// The array has static storage on every GPU that loads the library and stays
+// allocated until the process exits.  All calls share it and it keeps the
+// previous call's contents: the status words are cleared by every call and
+// every other scratch region is fully written before it is read.  Calls whose
+// kernels overlap on the GPU (two streams, two host threads, two devices'
+// worth of work aimed at one device) race on the array; serialise them.
+#include <mutex>
+
+#include "vdn_internal.h"
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = VDN_NOALLOC_SCRATCH_BYTES;  // 16 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 128;
+void* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of the array on the current device, looked up once per
+// device.  In host code `g_noalloc_scratch` names a host-side stand-in, not
+// device memory, so only this address may be given to a kernel.
+vdn_status scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return VDN_ERR_CUDA;
+  if (dev >= kMaxDevices) return VDN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return VDN_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return VDN_OK;
+}
+
+}  // namespace
+
+extern "C" vdn_status vdn_hybrid_attn_fwd_noalloc(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args,
+                                                  vdn_stream_t stream) {
+  if (!cfg || !args) return VDN_ERR_INVALID_ARG;
+  if (args->workspace || args->workspace_bytes) return VDN_ERR_INVALID_ARG;
+  const size_t need = vdn_hybrid_attn_workspace_size(cfg);
+  if (need == 0) {
+    vdn_workspace_layout tmp;
+    return vdn_hybrid_workspace_layout(cfg, &tmp);  // the configuration's own error
+  }
+  if (need > kNoallocScratchBytes) return VDN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  vdn_status st = scratch_for_current_device(&scratch);
+  if (st != VDN_OK) return st;
+  vdn_hybrid_args a = *args;
+  a.workspace = scratch;
+  a.workspace_bytes = kNoallocScratchBytes;
+  return vdn_hybrid_attn_fwd(cfg, &a, stream);
+}
