@@ -109,8 +109,8 @@ enum {
   VDN_STAGE_ALL = 31u
 };
 
-/* Byte offsets of the intermediate values inside the workspace (all float32,
- * dense).  C = ceil(T / chunk).  Stable across calls with the same cfg, so that
+/* Byte offsets of the intermediate values inside the workspace (float32
+ * unless noted, dense).  C = ceil(T / chunk).  Stable across calls with the same cfg, so that
  * a caller can inspect the stages.
  *   status     : uint32 device status words (VDN_ERR_TIMEOUT flags)
  *   half_text  : [B,H,d_v,d_k]        S_x / 2, the start state of both scans
@@ -119,9 +119,12 @@ enum {
  *   fwd_snap   : [B,H,C+1,d_v,d_k]    forward state over frames < min(5j, T)
  *   bwd_snap   : [B,H,C+1,d_v,d_k]    backward state over frames >= min(5j, T)
  *   read_table : [B,H,C+1,d_v,d_k]    R[c] = fwd_snap[max(c-1,0)] + bwd_snap[min(c+2,C)],
- *                                     R[C] = half_text * 2 (anchor query frames)        */
+ *                                     R[C] = half_text * 2 (anchor query frames)
+ *   read_table_bf16 : [B,H,C+1,2,d_v,d_k] bfloat16 hi/lo split of read_table,
+ *                                     R_hi = bf16(R), R_lo = bf16(R - R_hi) (operand of
+ *                                     the tensor-core read; written only on that path) */
 typedef struct {
-  size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, total;
+  size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, read_table_bf16, total;
 } vdn_workspace_layout;
 
 /* Bytes of workspace the configuration needs; 0 if cfg is invalid. */

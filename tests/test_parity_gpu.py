@@ -120,6 +120,19 @@ def test_bf16_softmax_runs_on_tensor_cores():
         assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, d, d, 0), "bf16"), L.STAGE_SOFTMAX) == 1
     assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 32, 32, 0), "bf16"), L.STAGE_SOFTMAX) == 0
     assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 128, 128, 0), "f32"), L.STAGE_SOFTMAX) == 0
+    for d in (64, 128):
+        assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, d, d, 0), "bf16"), L.STAGE_READ) == 1
+    assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 64, 64, 0), "f32"), L.STAGE_READ) == 0
+
+
+def test_bf16_read_table_matches_oracle():
+    """The read table the tensor-core read consumes (fp32 copy), bf16 mode."""
+    w = WORKLOADS["small"]
+    inp, cfg, ha, _, _ = run(w.shape, w.dtype, w.seed)
+    R = ha.intermediates()["R"].double().cpu().numpy()
+    for h in (0, cfg.H - 1):
+        ref = O.vda_intermediates(inp, ocfg(cfg), 0, h)["R"]
+        np.testing.assert_allclose(R[0, h], ref, atol=1e-4 * np.sqrt(np.mean(ref ** 2)))
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

@@ -6,9 +6,6 @@
 
 namespace vdn {
 
-cudaError_t launch_softmax_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
-bool softmax_tc_supported(const Dims& d);
-
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -61,6 +58,7 @@ void layout_of(const vdn_hybrid_cfg* c, vdn_workspace_layout* L) {
   L->fwd_snap = off;   off += up(bh * (C + 1) * dd);
   L->bwd_snap = off;   off += up(bh * (C + 1) * dd);
   L->read_table = off; off += up(bh * (C + 1) * dd);
+  L->read_table_bf16 = off; off += up(bh * (C + 1) * dd);  // hi and lo bf16 terms
   L->total = off;
 }
 
@@ -97,6 +95,7 @@ Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
   w.fsnap = reinterpret_cast<float*>(base + L.fwd_snap);
   w.bsnap = reinterpret_cast<float*>(base + L.bwd_snap);
   w.R = reinterpret_cast<float*>(base + L.read_table);
+  w.R16 = base + L.read_table_bf16;
   return w;
 }
 
@@ -138,8 +137,9 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
     case VDN_STAGE_TEXT:
     case VDN_STAGE_SOLVE:
     case VDN_STAGE_SCAN:
-    case VDN_STAGE_READ:
       return 0;
+    case VDN_STAGE_READ:
+      return read_tc_supported(d) ? 1 : 0;
     case VDN_STAGE_SOFTMAX:
       return softmax_tc_supported(d) ? 1 : 0;
     default:
@@ -173,7 +173,8 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
   if (stages & VDN_STAGE_READ) {
-    if ((e = launch_read_simt(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+    e = read_tc_supported(d) ? launch_read_tc(d, in, w, w.R16, s) : launch_read_simt(d, in, w, s);
+    if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
   return VDN_OK;
 }

@@ -29,6 +29,7 @@ struct Work {
   float* fsnap;      // [B,H,C+1,dv,dk]
   float* bsnap;      // [B,H,C+1,dv,dk]
   float* R;          // [B,H,C+1,dv,dk]
+  void* R16;         // [B,H,C+1,dv,dk] bf16
 };
 
 struct Inputs {
@@ -50,5 +51,9 @@ cudaError_t launch_solve_simt(const Dims& d, const Inputs& in, const Work& w, cu
 cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_read_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_softmax_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+bool softmax_tc_supported(const Dims& d);
+cudaError_t launch_softmax_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+bool read_tc_supported(const Dims& d);
+cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void* r16, cudaStream_t s);
 
 }  // namespace vdn

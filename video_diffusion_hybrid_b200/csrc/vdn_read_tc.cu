@@ -1,0 +1,354 @@
+// State read of the linear branch on the tensor cores, with the RMSNorm and
+// sigmoid-gate epilogue fused (bf16 q / gates, fp32 accumulation).
+//
+// What it computes (PaperDaily digest section 三: the query reads the forward
+// state before its window and the backward state after it and adds the two;
+// the linear branch is RMS-normalised and then gated):
+//   R_c = S^f(frames < 5(c-1)) + S^b(frames >= 5(c+2))      per chunk c
+//   R_anchor = S_init_f + S_init_b                           anchor query frames
+//   o = R q,  y_lin = sigmoid(g_lin) * o / sqrt(mean(o^2) + eps) [* w]
+//
+// k_read_table builds every R once per (batch, head, chunk): fp32 for
+// inspection and, for the MMA, two bf16 terms R_hi = bf16(R) and
+// R_lo = bf16(R - R_hi).  q is exact in bf16 and products accumulate in fp32,
+// so o = Q R_hi^T + Q R_lo^T carries R to about 16 significant bits (a single
+// bf16 R loses too much: o can be small next to |R| |q|, and the RMSNorm then
+// scales the rounding up).  k_read_tc then runs, per CTA, a run of up to kTilesPerCta
+// tiles of 128 query tokens of one (batch, head, query group):
+//   warp 0      TMA producer: R once (resident), then Q and gate tiles into a
+//               two-stage ring.
+//   warp 1      TMEM allocator; lane 0 issues O_t = Q_t R_hi^T + Q_t R_lo^T
+//               (M=128 tokens, N=d_v, K=d_k, both operands K-major in SMEM)
+//               into one of two TMEM accumulators.
+//   warps 4..7  epilogue, one token per thread (= TMEM lane): sum of squares
+//               over d_v, rsqrt, gate from the SMEM tile, store y.
+#include "tc_common.cuh"
+
+namespace vdn {
+namespace {
+using namespace tc;
+
+constexpr int TQ = 128;          // tokens per tile
+constexpr int kTilesPerCta = 8;  // tiles of one query group handled by a CTA
+constexpr int kThreadsR = 256;
+
+// ------------------------------------------------------------ read table --
+__global__ void k_read_table(Dims dm, Work w, __nv_bfloat16* __restrict__ r16) {
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const long long DD = (long long)dm.dv * dm.dk;
+  const float* fs = w.fsnap + ((long long)bh * (dm.C + 1) + (c < dm.C ? max(c - 1, 0) : 0)) * DD;
+  const float* bs = w.bsnap + ((long long)bh * (dm.C + 1) + (c < dm.C ? min(c + 2, dm.C) : dm.C)) * DD;
+  float* R = w.R + ((long long)bh * (dm.C + 1) + c) * DD;
+  __nv_bfloat16* R16 = r16 + ((long long)bh * (dm.C + 1) + c) * 2 * DD;  // [hi | lo]
+  for (long long i = threadIdx.x; i < DD; i += blockDim.x) {
+    const float r = fs[i] + bs[i];
+    R[i] = r;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(r);
+    R16[i] = hi;
+    R16[DD + i] = __float2bfloat16_rn(r - __bfloat162float(hi));
+  }
+}
+
+// ------------------------------------------------------------ work items --
+struct Run {
+  int b, h, ridx;
+  long long tok0;  // absolute first token of the run
+  int ntiles;      // tiles in this run
+  int rows_left;   // valid rows from tok0 to the end of the group
+};
+
+__device__ __forceinline__ void group_of(const Dims& d, int g, int& f0, int& f1, int& ridx) {
+  if (g < d.C) {
+    f0 = g * d.chunk;
+    f1 = min(d.T, f0 + d.chunk);
+    if (d.anchors) {
+      if (f0 == 0) f0 = 1;
+      if (f1 == d.T) f1 = d.T - 1;
+    }
+    ridx = g;
+  } else {
+    f0 = (g == d.C) ? 0 : d.T - 1;
+    f1 = f0 + 1;
+    ridx = d.C;
+  }
+}
+
+__host__ __device__ inline int runs_of_rows(long long rows) {
+  const long long tiles = (rows + TQ - 1) / TQ;
+  return (int)((tiles + kTilesPerCta - 1) / kTilesPerCta);
+}
+
+__device__ bool decode_run(const Dims& d, long long item, Run& r) {
+  const int ngroups = d.C + (d.anchors ? 2 : 0);
+  long long per_bh = 0;
+  for (int g = 0; g < ngroups; ++g) {
+    int f0, f1, ri;
+    group_of(d, g, f0, f1, ri);
+    if (f1 > f0) per_bh += runs_of_rows((long long)(f1 - f0) * d.N);
+  }
+  if (per_bh == 0) return false;
+  const long long bh = item / per_bh;
+  if (bh >= (long long)d.B * d.H) return false;
+  long long rem = item % per_bh;
+  for (int g = 0; g < ngroups; ++g) {
+    int f0, f1, ri;
+    group_of(d, g, f0, f1, ri);
+    if (f1 <= f0) continue;
+    const long long rows = (long long)(f1 - f0) * d.N;
+    const int nr = runs_of_rows(rows);
+    if (rem < nr) {
+      r.b = (int)(bh / d.H);
+      r.h = (int)(bh % d.H);
+      r.ridx = ri;
+      const long long first_tile = rem * kTilesPerCta;
+      const long long tiles = (rows + TQ - 1) / TQ;
+      r.ntiles = (int)min((long long)kTilesPerCta, tiles - first_tile);
+      r.tok0 = (long long)r.b * d.T * d.N + (long long)f0 * d.N + first_tile * TQ;
+      r.rows_left = (int)(rows - first_tile * TQ);
+      return true;
+    }
+    rem -= nr;
+  }
+  return false;
+}
+
+template <typename To> __device__ __forceinline__ void put4(To* p, float a, float b, float c, float d, bool add);
+template <> __device__ __forceinline__ void put4<float>(float* p, float a, float b, float c, float d, bool add) {
+  float4 v = make_float4(a, b, c, d);
+  if (add) {
+    const float4 o = *reinterpret_cast<const float4*>(p);
+    v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+  }
+  *reinterpret_cast<float4*>(p) = v;
+}
+template <> __device__ __forceinline__ void put4<__nv_bfloat16>(__nv_bfloat16* p, float a, float b, float c, float d,
+                                                                 bool add) {
+  if (add) {
+    const uint2 o = *reinterpret_cast<const uint2*>(p);
+    a += __uint_as_float(o.x << 16); b += __uint_as_float(o.x & 0xFFFF0000u);
+    c += __uint_as_float(o.y << 16); d += __uint_as_float(o.y & 0xFFFF0000u);
+  }
+  uint2 u;
+  u.x = pack_bf16(a, b);
+  u.y = pack_bf16(c, d);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+// ------------------------------------------------------------------ kernel --
+template <int D, typename To>
+__global__ void __launch_bounds__(kThreadsR, 1)
+k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
+          const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmr) {
+  constexpr int NB = D / 64;
+  constexpr uint32_t RBYTES = 2 * D * D * 2;  // hi and lo terms
+  constexpr uint32_t TBYTES = TQ * D * 2;  // one Q or gate tile
+  constexpr int ST = 2;
+  constexpr uint32_t kCols = 2 * D <= 128 ? 128 : 256;
+  enum { B_R = 0, B_QFULL = 1, B_QEMPTY = 3, B_GFULL = 5, B_GEMPTY = 7, B_AFULL = 9, B_AEMPTY = 11, B_DRAIN = 13,
+         NBARS = 14 };
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sR = sm;
+  unsigned char* sQ = sR + RBYTES;
+  unsigned char* sG = sQ + ST * TBYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + ST * TBYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
+  Run run;
+  if (!decode_run(dm, blockIdx.x, run)) return;
+  const Ctl ctl{abort_flag, w.status, (unsigned)TAG_READ_TC};
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_GEMPTY || i == B_GEMPTY + 1 || i == B_AEMPTY ||
+                                                     i == B_AEMPTY + 1) ? 128 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int rrow = ((run.b * dm.H + run.h) * (dm.C + 1) + run.ridx) * 2 * D;
+      mbar_expect_tx(bar(B_R), RBYTES);
+      for (int part = 0; part < 2; ++part)
+        for (int c = 0; c < NB; ++c)
+          tma_load_2d(smem_u32(sR + part * D * D * 2 + c * D * 128), &tmr, bar(B_R), c * 64, rrow + part * D);
+      int last[ST] = {-1, -1};
+      for (int t = 0; t < run.ntiles; ++t) {
+        const int s = t % ST;
+        const int tok = (int)(run.tok0 + (long long)t * TQ);
+        if (t >= ST) {
+          if (!mbar_wait(bar(B_QEMPTY + s), (t / ST - 1) & 1, ctl)) break;
+          if (!mbar_wait(bar(B_GEMPTY + s), (t / ST - 1) & 1, ctl)) break;
+        }
+        mbar_expect_tx(bar(B_QFULL + s), TBYTES);
+        for (int c = 0; c < NB; ++c)
+          tma_load_3d(smem_u32(sQ + s * TBYTES + c * TQ * 128), &tmq, bar(B_QFULL + s), c * 64, run.h, tok);
+        mbar_expect_tx(bar(B_GFULL + s), TBYTES);
+        for (int c = 0; c < NB; ++c)
+          tma_load_3d(smem_u32(sG + s * TBYTES + c * TQ * 128), &tmg, bar(B_GFULL + s), c * 64, run.h, tok);
+        last[s] = t;
+      }
+      mbar_wait(bar(B_R), 0, ctl);
+      for (int s = 0; s < ST; ++s)
+        if (last[s] >= 0) {
+          mbar_wait(bar(B_QFULL + s), (last[s] / ST) & 1, ctl);
+          mbar_wait(bar(B_GFULL + s), (last[s] / ST) & 1, ctl);
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t ID = idesc_bf16(TQ, D, false);
+      const uint32_t ra = smem_u32(sR);
+      bool ok = mbar_wait(bar(B_R), 0, ctl);
+      for (int t = 0; ok && t < run.ntiles; ++t) {
+        const int s = t % ST;
+        if (!mbar_wait(bar(B_QFULL + s), (t / ST) & 1, ctl)) break;
+        if (t >= ST && !mbar_wait(bar(B_AEMPTY + s), (t / ST - 1) & 1, ctl)) break;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sQ + s * TBYTES);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t qoff = (k >> 2) * (TQ * 128) + (k & 3) * 32;
+            const uint32_t roff = part * D * D * 2 + (k >> 2) * (D * 128) + (k & 3) * 32;
+            mma_bf16(tmem + s * D, sdesc(qa + qoff, 16, 1024), sdesc(ra + roff, 16, 1024), ID,
+                     (part | k) ? 1u : 0u);
+          }
+        }
+        mma_commit(bar(B_AFULL + s));
+        mma_commit(bar(B_QEMPTY + s));
+      }
+      mma_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, ctl);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp - 4;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const float* wgt = in.rms_weight ? in.rms_weight + (long long)run.h * D : nullptr;
+    for (int t = 0; t < run.ntiles; ++t) {
+      const int s = t % ST;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + s), (t / ST) & 1, ctl))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_GFULL + s), (t / ST) & 1, ctl))) break;
+      tc_fence_after();
+      float o[D];
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        float v[32];
+        tmem_ld32(lane_addr + s * D + q * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[q * 32 + i] = v[i];
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_AEMPTY + s));  // accumulator free for tile t + ST
+      float ss[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ss[u] = 0.f;
+#pragma unroll
+      for (int i = 0; i < D; ++i) ss[i & 7] = fmaf(o[i], o[i], ss[i & 7]);
+      const float rs =
+          rsqrtf((((ss[0] + ss[1]) + (ss[2] + ss[3])) + ((ss[4] + ss[5]) + (ss[6] + ss[7]))) / D + dm.eps);
+      const int rows_valid = min(TQ, run.rows_left - t * TQ);
+      const bool valid = row < rows_valid;
+      const long long tok = run.tok0 + (long long)t * TQ + row;
+      const long long gi = (tok * dm.H + run.h) * D;
+      To* y = static_cast<To*>(in.y) + (dm.out_mode == 0 ? 2 * gi + D : gi);
+      const unsigned char* grow = sG + s * TBYTES + row * 128;
+#pragma unroll
+      for (int ch = 0; ch < D / 8; ++ch) {
+        // 8 gate values of this row from the 128B-swizzled tile
+        const uint4 raw = *reinterpret_cast<const uint4*>(grow + (ch >> 3) * (TQ * 128) + (((ch & 7) ^ (row & 7)) << 4));
+        const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+        float yv[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float g0 = __uint_as_float(u[e] << 16), g1 = __uint_as_float(u[e] & 0xFFFF0000u);
+          const int i0 = ch * 8 + 2 * e;
+          const float w0 = wgt ? __ldg(wgt + i0) : 1.f, w1 = wgt ? __ldg(wgt + i0 + 1) : 1.f;
+          yv[2 * e] = o[i0] * rs * w0 / (1.0f + __expf(-g0));
+          yv[2 * e + 1] = o[i0 + 1] * rs * w1 / (1.0f + __expf(-g1));
+        }
+        if (valid) {
+          put4<To>(y + ch * 8, yv[0], yv[1], yv[2], yv[3], dm.out_mode != 0);
+          put4<To>(y + ch * 8 + 4, yv[4], yv[5], yv[6], yv[7], dm.out_mode != 0);
+        }
+      }
+      mbar_arrive(bar(B_GEMPTY + s));  // gate tile free
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, kCols);
+}
+
+long long num_runs(const Dims& d) {
+  const int ngroups = d.C + (d.anchors ? 2 : 0);
+  long long per_bh = 0;
+  for (int g = 0; g < ngroups; ++g) {
+    int f0, f1;
+    if (g < d.C) {
+      f0 = g * d.chunk;
+      f1 = std::min(d.T, f0 + d.chunk);
+      if (d.anchors) {
+        if (f0 == 0) f0 = 1;
+        if (f1 == d.T) f1 = d.T - 1;
+      }
+    } else {
+      f0 = (g == d.C) ? 0 : d.T - 1;
+      f1 = f0 + 1;
+    }
+    if (f1 > f0) per_bh += runs_of_rows((long long)(f1 - f0) * d.N);
+  }
+  return per_bh * d.B * d.H;
+}
+
+template <int D, typename To>
+cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, __nv_bfloat16* r16, cudaStream_t s) {
+  k_read_table<<<dim3(d.C + 1, d.B * d.H), 256, 0, s>>>(d, w, r16);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mq, mg, mr;
+  const long long tokens = (long long)d.B * d.T * d.N;
+  if (!make_token_map(&mq, in.q, tokens, d.H, D, TQ) || !make_token_map(&mg, in.gate_lin, tokens, d.H, D, TQ) ||
+      !make_matrix_map(&mr, r16, (long long)d.B * d.H * (d.C + 1) * 2 * D, D, D))
+    return cudaErrorInvalidValue;
+  const size_t smem = 1024 + 2 * (size_t)D * D * 2 + 4 * (size_t)TQ * D * 2 + 14 * 8 + 16;
+  auto kern = k_read_tc<D, To>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long items = num_runs(d);
+  if (items <= 0 || items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  kern<<<(unsigned)items, kThreadsR, smem, s>>>(d, in, w, mq, mg, mr);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool read_tc_supported(const Dims& d) {
+  if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128)) return false;
+  if ((long long)d.B * d.T * d.N >= (1LL << 31)) return false;
+  if ((long long)d.B * d.H * (d.C + 1) * 2 * d.dk >= (1LL << 31)) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void* r16, cudaStream_t s) {
+  __nv_bfloat16* r = static_cast<__nv_bfloat16*>(r16);
+  if (d.dk == 128) return d.out_bf16 ? launch<128, __nv_bfloat16>(d, in, w, r, s) : launch<128, float>(d, in, w, r, s);
+  if (d.dk == 64) return d.out_bf16 ? launch<64, __nv_bfloat16>(d, in, w, r, s) : launch<64, float>(d, in, w, r, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

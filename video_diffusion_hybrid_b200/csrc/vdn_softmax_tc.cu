@@ -12,15 +12,17 @@
 // intervals (anchor frame 0, the window, anchor frame T-1).
 //
 // Roles (256 threads):
-//   warp 0      TMA producer: Q once, then K tiles (three-stage ring, freed
-//               as soon as S_j is computed) and V tiles (two-stage ring,
-//               freed after O += P_j V_j); 128B-swizzled boxes of 64 x 128.
+//   warp 0      TMA producer of Q (once) and of the K ring (three stages,
+//               freed as soon as S_j is computed).
+//   warp 2      TMA producer of the V ring (three stages, freed after
+//               O += P_j V_j).  Separate threads, so that neither ring waits
+//               behind the other.  128B-swizzled boxes of 64 dims x 128 rows.
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma:
-//                 S_j = Q K_j^T  (M=128, N=128, K=d)   into TMEM S[j % 2]
-//                 O  += P_j V_j  (M=128, N=d, K=128)   into TMEM O
+//                 S_j = Q K_j^T  (M=128, N=128, K=d; both from SMEM) -> TMEM S[j % 2]
+//                 O  += P_j V_j  (M=128, N=d, K=128; P from TMEM)    -> TMEM O
 //   warps 4..7  softmax: thread r owns query row r (= TMEM lane r).  It reads
-//               its row of S_j, keeps a running max / sum, writes P_j (bf16)
-//               to shared memory in the MMA's K-major 128B-swizzled layout and
+//               its row of S_j, keeps a running max / sum, computes P_j into
+//               registers, writes it (bf16, two per column) to TMEM and
 //               rescales its row of O only when the max grew by more than 2^8
 //               (exact: p <= 2^8 is then guaranteed, and O and the sum share
 //               the same stale max).  Epilogue: O / l, gate, store.
@@ -28,174 +30,19 @@
 // Every mbarrier wait is bounded (about one second of clock cycles); on
 // expiry the CTA records VDN_ERR_TIMEOUT in the workspace status words, stops
 // issuing, drains its own copies and MMAs and frees its TMEM.
-#include <cuda.h>
-
-#include "vdn_internal.h"
+#include "tc_common.cuh"
 
 namespace vdn {
 namespace {
+using namespace tc;
 
 constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 128;           // keys per tile
 constexpr int kThreadsTC = 256;
 constexpr int kSoftmaxWarp0 = 4;  // warps 4..7 (TMEM lane quadrants 0..3)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256;
+constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kColP = 384;
 constexpr float kRescaleLog2 = 8.0f;
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
-
-// ------------------------------------------------------------- PTX helpers --
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-struct Ctl {
-  volatile int* abort;  // shared flag: some wait of this CTA gave up
-  uint32_t* status;     // workspace status words
-};
-
-// Bounded wait: true when the phase completed; false after ~1 s or when
-// another role of the CTA already gave up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
-  if (mbar_try(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (*c.abort) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        *c.abort = 1;
-        atomicOr(c.status, 1u);
-        atomicExch(c.status + 1, (unsigned)TAG_SOFTMAX_TC);
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
-                                            int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
-      "[%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-// Shared-memory matrix descriptor (tcgen05), 128B swizzle, version 1.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
-  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-  return d;
-}
-
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 // ------------------------------------------------------ work decomposition --
 struct Tile {
@@ -320,17 +167,15 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   constexpr int NB = D / 64;                 // 64-wide column blocks of a row
   constexpr uint32_t QBYTES = BM * D * 2;
   constexpr uint32_t KVBYTES = BN * D * 2;
-  constexpr uint32_t PBYTES = BM * BN * 2;
-  constexpr int KST = 3, VST = 2;            // K and V ring depths
-  enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 9, B_SFULL = 11, B_PFULL = 13, B_ODONE = 14,
-         B_DRAIN = 15, NBARS = 16 };
+  constexpr int KST = 3, VST = 3;            // K and V ring depths
+  enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 15, B_ODONE = 16,
+         B_DRAIN = 17, NBARS = 18 };
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sQ = sm;
   unsigned char* sK = sQ + QBYTES;           // KST stages
   unsigned char* sV = sK + KST * KVBYTES;    // VST stages
-  unsigned char* sP = sV + VST * KVBYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + PBYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VST * KVBYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -340,7 +185,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   Tile tile;
   if (!decode_item(dm, blockIdx.x, tile)) return;  // uniform across the CTA
   const int ntiles = num_key_tiles(tile);
-  const Ctl ctl{abort_flag, w.status};
+  const Ctl ctl{abort_flag, w.status, (unsigned)TAG_SOFTMAX_TC};
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   if (threadIdx.x == 0) {
@@ -362,10 +207,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
     fence_barrier_init();
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
   }
   tc_fence_before();
   __syncthreads();
@@ -373,36 +215,46 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ Q and K producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmq)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
       mbar_expect_tx(bar(B_Q), QBYTES);
       for (int c = 0; c < NB; ++c)
         tma_load_3d(smem_u32(sQ + c * BM * 128), &tmq, bar(B_Q), c * 64, tile.h, tile.q0);
-      int lastk[KST], lastv[VST];
+      int lastk[KST];
       for (int s = 0; s < KST; ++s) lastk[s] = -1;
-      for (int s = 0; s < VST; ++s) lastv[s] = -1;
       for (int j = 0; j < ntiles; ++j) {
         int k0, kv;
         key_tile(tile, j, k0, kv);
-        const int sk = j % KST, sv = j % VST;
+        const int sk = j % KST;
         if (j >= KST && !mbar_wait(bar(B_KEMPTY + sk), (j / KST - 1) & 1, ctl)) break;
         mbar_expect_tx(bar(B_KFULL + sk), KVBYTES);
         for (int c = 0; c < NB; ++c)
           tma_load_3d(smem_u32(sK + sk * KVBYTES + c * BN * 128), &tmk, bar(B_KFULL + sk), c * 64, tile.h, k0);
         lastk[sk] = j;
+      }
+      // drain: every copy issued into this CTA's shared memory has landed
+      mbar_wait(bar(B_Q), 0, ctl);
+      for (int s = 0; s < KST; ++s)
+        if (lastk[s] >= 0) mbar_wait(bar(B_KFULL + s), (lastk[s] / KST) & 1, ctl);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
+      int lastv[VST];
+      for (int s = 0; s < VST; ++s) lastv[s] = -1;
+      for (int j = 0; j < ntiles; ++j) {
+        int k0, kv;
+        key_tile(tile, j, k0, kv);
+        const int sv = j % VST;
         if (j >= VST && !mbar_wait(bar(B_VEMPTY + sv), (j / VST - 1) & 1, ctl)) break;
         mbar_expect_tx(bar(B_VFULL + sv), KVBYTES);
         for (int c = 0; c < NB; ++c)
           tma_load_3d(smem_u32(sV + sv * KVBYTES + c * BN * 128), &tmv, bar(B_VFULL + sv), c * 64, tile.h, k0);
         lastv[sv] = j;
       }
-      // drain: every copy issued into this CTA's shared memory has landed
-      mbar_wait(bar(B_Q), 0, ctl);
-      for (int s = 0; s < KST; ++s)
-        if (lastk[s] >= 0) mbar_wait(bar(B_KFULL + s), (lastk[s] / KST) & 1, ctl);
       for (int s = 0; s < VST; ++s)
         if (lastv[s] >= 0) mbar_wait(bar(B_VFULL + s), (lastv[s] / VST) & 1, ctl);
     }
@@ -411,7 +263,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
     if (lane == 0) {
       constexpr uint32_t ID_S = idesc_bf16(BM, BN, false);
       constexpr uint32_t ID_O = idesc_bf16(BM, D, true);
-      const uint32_t qa = smem_u32(sQ), pa = smem_u32(sP);
+      const uint32_t qa = smem_u32(sQ);
       auto issue_s = [&](int j) -> bool {
         const int sk = j % KST, sb = j & 1;
         if (!mbar_wait(bar(B_KFULL + sk), (j / KST) & 1, ctl)) return false;
@@ -437,11 +289,9 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         tc_fence_after();
         const uint32_t va = smem_u32(sV + sv * KVBYTES);
 #pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          const uint32_t poff = (k >> 2) * (BM * 128) + (k & 3) * 32;
-          mma_bf16(tmem + kColO, sdesc(pa + poff, 16, 1024), sdesc(va + k * 16 * 128, BN * 128, 1024), ID_O,
-                   (j > 0 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < BN / 16; ++k)
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(va + k * 16 * 128, BN * 128, 1024), ID_O,
+                      (j > 0 || k > 0) ? 1u : 0u);
         mma_commit(bar(B_ODONE));
         mma_commit(bar(B_VEMPTY + sv));
         if (j + 2 < ntiles) ok = issue_s(j + 2);
@@ -458,8 +308,6 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
     const float c = dm.scale * 1.4426950408889634f;  // log2 units
     const float thresh = kRescaleLog2 / c;            // raw-score units
     float m_used = -INFINITY, l_sum = 0.f;
-    unsigned char* prow = sP + row * 128;
-    const int sw = row & 7;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j & 1;
@@ -468,13 +316,20 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       tc_fence_after();
       float x[BN];
       {
-        float v[32];
+        // four loads in flight, one wait
+        float v0[32], v1[32], v2[32], v3[32];
+        const uint32_t scol = lane_addr + (s ? kColS1 : kColS0);
+        tmem_ld32(scol + 0, v0);
+        tmem_ld32(scol + 32, v1);
+        tmem_ld32(scol + 64, v2);
+        tmem_ld32(scol + 96, v3);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < BN / 32; ++q) {
-          tmem_ld32(lane_addr + (s ? kColS1 : kColS0) + q * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[q * 32 + i] = v[i];
+        for (int i = 0; i < 32; ++i) {
+          x[i] = v0[i];
+          x[32 + i] = v1[i];
+          x[64 + i] = v2[i];
+          x[96 + i] = v3[i];
         }
       }
       int k0, kvalid;
@@ -484,20 +339,45 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         for (int i = 0; i < BN; ++i)
           if (i >= kvalid) x[i] = -INFINITY;
       }
-      float mx = x[0];
+      // row max with eight independent chains (one warp per SMSP: no other
+      // warp hides a long dependent chain)
+      float pm[8];
 #pragma unroll
-      for (int i = 1; i < BN; ++i) mx = fmaxf(mx, x[i]);
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ODONE), (j - 1) & 1, ctl))) { ok = false; break; }
-        tc_fence_after();
-      }
-      // lazy rescale: only rows whose max grew by more than 2^8 (in exp2 units)
+      for (int u = 0; u < 8; ++u) pm[u] = x[u];
+#pragma unroll
+      for (int i = 8; i < BN; ++i) pm[i & 7] = fmaxf(pm[i & 7], x[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      // lazy rescale decision: only rows whose max grew by more than 2^8
       const bool need = mx > m_used + thresh;
       float f = 1.0f;
       if (need) {
         f = (m_used == -INFINITY) ? 0.f : ex2((m_used - mx) * c);
         l_sum *= f;
         m_used = mx;
+      }
+      // exponentials into packed bf16 registers first: this overlaps with the
+      // tensor core still computing O += P_{j-1} V_{j-1} from shared memory
+      const float mc = m_used * c;
+      uint32_t pk[BN / 2];
+      float ps[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+#pragma unroll
+      for (int i = 0; i < BN / 2; ++i) {
+        const float p0 = ex2(fmaf(x[2 * i], c, -mc));
+        const float p1 = ex2(fmaf(x[2 * i + 1], c, -mc));
+        pk[i] = pack_bf16(p0, p1);
+        // the row sum uses the bf16-rounded weights the MMA multiplies by,
+        // so every output row is an exact convex combination of V rows
+        ps[(2 * i) & 7] += __uint_as_float(pk[i] << 16);
+        ps[(2 * i + 1) & 7] += __uint_as_float(pk[i] & 0xFFFF0000u);
+      }
+      const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      // O and the P buffer are free once O += P_{j-1} V_{j-1} has completed
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ODONE), (j - 1) & 1, ctl))) { ok = false; break; }
+        tc_fence_after();
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         float v[32];
@@ -511,27 +391,18 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         }
         tmem_wait_st();
       }
-      const float mc = m_used * c;
-      float sum = 0.f;
+      {
+        float h0[32], h1[32];
 #pragma unroll
-      for (int blk = 0; blk < BN / 64; ++blk) {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t u[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2(fmaf(x[blk * 64 + ch * 8 + 2 * e], c, -mc));
-            const float p1 = ex2(fmaf(x[blk * 64 + ch * 8 + 2 * e + 1], c, -mc));
-            u[e] = pack_bf16(p0, p1);
-            // the row sum uses the bf16-rounded weights the MMA multiplies by,
-            // so every output row is an exact convex combination of V rows
-            sum += __uint_as_float(u[e] << 16) + __uint_as_float(u[e] & 0xFFFF0000u);
-          }
-          *reinterpret_cast<uint4*>(prow + blk * (BM * 128) + ((ch ^ sw) << 4)) = make_uint4(u[0], u[1], u[2], u[3]);
+        for (int i = 0; i < 32; ++i) {
+          h0[i] = __uint_as_float(pk[i]);
+          h1[i] = __uint_as_float(pk[32 + i]);
         }
+        tmem_st32(lane_addr + kColP, h0);
+        tmem_st32(lane_addr + kColP + 32, h1);
+        tmem_wait_st();
       }
       l_sum += sum;
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(B_PFULL));
     }
@@ -584,41 +455,11 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    tmem_free(tmem, kTmemCols);
   }
 }
 
 // ------------------------------------------------------------------- host --
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
-// 3-D map over a [tokens][H][D] bf16 tensor; box = 64 dims x 1 head x 128 tokens.
-bool make_map(CUtensorMap* m, const void* base, const Dims& d, int D) {
-  EncodeTiled fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t tokens = (cuuint64_t)d.B * d.T * d.N;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)d.H, tokens};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)d.H * D * 2};
-  cuuint32_t box[3] = {64, 1, 128};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 long long num_items(const Dims& d) {
   const int n_anc = d.anchors ? 2 : 0;
   long long per_bh = 0;
@@ -636,9 +477,11 @@ long long num_items(const Dims& d) {
 template <int D, typename To>
 cudaError_t launch_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, in.q, d, D) || !make_map(&mk, in.k, d, D) || !make_map(&mv, in.v, d, D))
+  const long long tokens = (long long)d.B * d.T * d.N;
+  if (!make_token_map(&mq, in.q, tokens, d.H, D, BM) || !make_token_map(&mk, in.k, tokens, d.H, D, BN) ||
+      !make_token_map(&mv, in.v, tokens, d.H, D, BN))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + (size_t)BM * D * 2 + 5 * (size_t)BN * D * 2 + (size_t)BM * BN * 2 + 16 * 8 + 16;
+  const size_t smem = 1024 + (size_t)BM * D * 2 + 6 * (size_t)BN * D * 2 + 18 * 8 + 16;
   auto kern = k_softmax_tc<D, To>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -10,8 +10,10 @@
               90,720 video tokens per head.
 * long      : T=180, N=1008, H=24, d=128, L=512, B=2 (two seeds), bf16.
 * sweep_N{n}_d{d} : VDA-only shapes at T=90, H=24, bf16.
+* prof_d128 : the 768p shape cut to T=30 (about 1 GB of inputs, still larger
+              than L2) for detailed profiler captures of the same kernels.
 
-The seed of a workload is its index in the list above (1-based); batch
+Each workload has its own seed (listed below); batch
 element b draws from PCG64(seed * 1000 + b).
 """
 from __future__ import annotations
@@ -43,4 +45,5 @@ WORKLOADS = {w.name: w for w in [
     _w("small", 1, 20, 240, 8, 64, 64, "bf16", 2),
     _w("768p", 1, 90, 1008, 24, 128, 512, "bf16", 3),
     _w("long", 2, 180, 1008, 24, 128, 512, "bf16", 4),
+    _w("prof_d128", 1, 30, 1008, 24, 128, 512, "bf16", 6),
 ] + [_w(f"sweep_N{n}_d{d}", 1, 90, n, 24, d, 512, "bf16", 5) for n in (256, 1008, 4032) for d in (64, 128, 256)]}
