@@ -122,7 +122,22 @@ def test_bf16_softmax_runs_on_tensor_cores():
     assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 128, 128, 0), "f32"), L.STAGE_SOFTMAX) == 0
     for d in (64, 128):
         assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, d, d, 0), "bf16"), L.STAGE_READ) == 1
+        assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, d, d, 0), "bf16"), L.STAGE_SOLVE) == 1
     assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 64, 64, 0), "f32"), L.STAGE_READ) == 0
+
+
+@pytest.mark.parametrize("shape", [Shape(1, 20, 240, 2, 64, 64, 8), Shape(1, 12, 300, 2, 128, 128, 8),
+                                   Shape(2, 8, 40, 1, 128, 128, 0)])
+def test_bf16_frame_maps_match_oracle(shape):
+    """M_t and C_t after the tensor-core Gram + SPD solve (bf16 inputs)."""
+    inp, cfg, ha, _, _ = run(shape, "bf16", 13, drop_text=shape.L == 0)
+    it = {k: v.double().cpu().numpy() for k, v in ha.intermediates().items()}
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            ref = O.vda_intermediates(inp, ocfg(cfg), b, h)
+            for t in range(1, cfg.T - 1):
+                np.testing.assert_allclose(it["M"][b, t, h], ref["M"][t], atol=2e-5)
+                np.testing.assert_allclose(it["C"][b, t, h], ref["C"][t], atol=2e-5 * np.abs(ref["C"][t]).max())
 
 
 def test_bf16_read_table_matches_oracle():

@@ -135,9 +135,10 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
   Dims d = make_dims(cfg);
   switch (stage) {
     case VDN_STAGE_TEXT:
-    case VDN_STAGE_SOLVE:
     case VDN_STAGE_SCAN:
       return 0;
+    case VDN_STAGE_SOLVE:
+      return gram_tc_supported(d) ? 1 : 0;
     case VDN_STAGE_READ:
       return read_tc_supported(d) ? 1 : 0;
     case VDN_STAGE_SOFTMAX:
@@ -163,7 +164,12 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     if ((e = launch_text(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
   }
   if (stages & VDN_STAGE_SOLVE) {
-    if ((e = launch_solve_simt(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+    if (gram_tc_supported(d)) {
+      if ((e = launch_gram_tc(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+      if ((e = launch_solve_inplace(d, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+    } else if ((e = launch_solve_simt(d, in, w, s)) != cudaSuccess) {
+      return VDN_ERR_CUDA;
+    }
   }
   if (stages & VDN_STAGE_SCAN) {
     if ((e = launch_scan_simt(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;

@@ -1,0 +1,224 @@
+// Per-frame Gram and write matrices of Video Delta Attention on the tensor
+// cores (bf16 k / v, fp32 beta and accumulation).
+//
+// What it computes (PaperDaily digest section 四: all tokens of a frame are
+// written jointly; deepmagic post "用兩條分支取代一條": A is the weighted key
+// Gram matrix and B the value-key write matrix of the closed form):
+//   A_t = sum_i beta_i k_i k_i^T = K^T (beta K),   B_t = sum_i beta_i v_i k_i^T = V^T (beta K)
+// for every non-anchor frame t and head, over its N tokens.  The results go to
+// the M_t / C_t slots of the workspace, where the SPD solve replaces them by
+// M_t = (I + A_t)^-1 and C_t = B_t M_t.
+//
+// One CTA per (batch, frame, head); the frame's tokens in tiles of 128:
+//   warp 0      TMA producer: K and V tiles (two-stage ring, 128B-swizzled).
+//   warps 4..7  one token row per thread: beta K in two bf16 terms,
+//               hi = bf16(beta k), lo = bf16(beta k - hi), written in the same
+//               swizzled layout (tokens past the frame get beta = 0).  k and v
+//               are exact in bf16 and products accumulate in fp32, so the
+//               split carries beta k to about 16 significant bits.
+//               Afterwards: the epilogue, TMEM -> A_t, B_t rows in global.
+//   warp 1      TMEM allocator; lane 0 issues, per 16 tokens,
+//                 A += K^T (beta K)_hi + K^T (beta K)_lo
+//                 B += V^T (beta K)_hi + V^T (beta K)_lo
+//               with both operands MN-major (d contiguous), so no repacking.
+//               For d = 64, K and V stack into one M = 128 operand and one
+//               accumulator [A; B] (64 columns).
+#include "tc_common.cuh"
+
+namespace vdn {
+namespace {
+using namespace tc;
+
+constexpr int TT = 128;  // tokens per tile
+constexpr int kThreadsG = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kThreadsG, 1)
+k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
+          const __grid_constant__ CUtensorMap tmv) {
+  constexpr int NB = D / 64;
+  constexpr uint32_t TB = TT * D * 2;     // one K or V tile (bytes)
+  constexpr uint32_t STAGE = 2 * TB;      // K then V (adjacent: V = K + TB)
+  constexpr int ST = 2;
+  constexpr uint32_t kCols = D == 128 ? 256 : 64;
+  enum { B_KVFULL = 0, B_KVEMPTY = 2, B_KBFULL = 4, B_KBEMPTY = 5, B_ACC = 6, B_DRAIN = 7, NBARS = 8 };
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sKV = sm;                  // ST stages of [K | V]
+  unsigned char* sHi = sKV + ST * STAGE;    // beta K, high term
+  unsigned char* sLo = sHi + TB;            // beta K, low term
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sLo + TB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  if (is_anchor(dm, t)) return;
+  if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
+  const int ntiles = (dm.N + TT - 1) / TT;
+  const long long tok0 = ((long long)b * dm.T + t) * dm.N;  // first token of the frame
+  const long long fh = ((long long)b * dm.T + t) * dm.H + h;
+  const Ctl ctl{abort_flag, w.status, (unsigned)TAG_GRAM_TC};
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i == B_KBFULL ? 128 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int last[ST] = {-1, -1};
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % ST;
+        if (j >= ST && !mbar_wait(bar(B_KVEMPTY + s), (j / ST - 1) & 1, ctl)) break;
+        const int tok = (int)(tok0 + (long long)j * TT);
+        mbar_expect_tx(bar(B_KVFULL + s), STAGE);
+        for (int c = 0; c < NB; ++c) {
+          tma_load_3d(smem_u32(sKV + s * STAGE + c * TT * 128), &tmk, bar(B_KVFULL + s), c * 64, h, tok);
+          tma_load_3d(smem_u32(sKV + s * STAGE + TB + c * TT * 128), &tmv, bar(B_KVFULL + s), c * 64, h, tok);
+        }
+        last[s] = j;
+      }
+      for (int s = 0; s < ST; ++s)
+        if (last[s] >= 0) mbar_wait(bar(B_KVFULL + s), (last[s] / ST) & 1, ctl);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // MN-major operands: M (or N) = d in 64-wide chunks TT*128 bytes apart,
+      // 8-token groups 1024 bytes apart, 16 tokens (2048 bytes) per K-step.
+      constexpr uint32_t ID = D == 128 ? (idesc_bf16(128, 128, true) | (1u << 15)) : (idesc_bf16(128, 64, true) | (1u << 15));
+      const uint32_t hi = smem_u32(sHi), lo = smem_u32(sLo);
+      bool ok = true;
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const int s = j % ST;
+        if (!mbar_wait(bar(B_KBFULL), j & 1, ctl) || !mbar_wait(bar(B_KVFULL + s), (j / ST) & 1, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sKV + s * STAGE), va = ka + TB;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t kb = part ? lo : hi;
+#pragma unroll
+          for (int k = 0; k < TT / 16; ++k) {
+            const uint32_t acc = (j | part | k) ? 1u : 0u;
+            const uint64_t bdesc = sdesc(kb + k * 2048, TT * 128, 1024);
+            mma_bf16(tmem, sdesc(ka + k * 2048, TT * 128, 1024), bdesc, ID, acc);
+            if (D == 128) mma_bf16(tmem + 128, sdesc(va + k * 2048, TT * 128, 1024), bdesc, ID, acc);
+          }
+        }
+        mma_commit(bar(B_KVEMPTY + s));
+        mma_commit(bar(B_KBEMPTY));
+      }
+      if (ok) mma_commit(bar(B_ACC));
+      mma_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, ctl);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp - 4;
+    const int row = quad * 32 + lane;  // token row of the tile / TMEM lane
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j % ST;
+      if (!mbar_wait(bar(B_KVFULL + s), (j / ST) & 1, ctl)) { ok = false; break; }
+      if (j > 0 && !mbar_wait(bar(B_KBEMPTY), (j - 1) & 1, ctl)) { ok = false; break; }
+      const int tk = j * TT + row;
+      const float beta = tk < dm.N ? __ldg(in.beta + (tok0 + tk) * dm.H + h) : 0.f;
+#pragma unroll
+      for (int c = 0; c < NB; ++c) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t off = c * TT * 128 + row * 128 + ((q ^ (row & 7)) << 4);
+          const uint4 raw = *reinterpret_cast<const uint4*>(sKV + s * STAGE + off);
+          const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t hv[4], lv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(u[e] << 16) * beta;
+            const float x1 = __uint_as_float(u[e] & 0xFFFF0000u) * beta;
+            hv[e] = pack_bf16(x0, x1);
+            lv[e] = pack_bf16(x0 - __uint_as_float(hv[e] << 16), x1 - __uint_as_float(hv[e] & 0xFFFF0000u));
+          }
+          *reinterpret_cast<uint4*>(sHi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          *reinterpret_cast<uint4*>(sLo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_KBFULL));
+    }
+    // ---- epilogue: accumulators -> A_t, B_t (fp32, row-major) in the M_t / C_t slots
+    if (__all_sync(0xffffffffu, ok && mbar_wait(bar(B_ACC), 0, ctl))) {
+      tc_fence_after();
+      const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+      const long long DD = (long long)D * D;
+      if (D == 128) {
+        float* Ag = w.M + fh * DD + (long long)row * D;
+        float* Bg = w.Cm + fh * DD + (long long)row * D;
+#pragma unroll
+        for (int q = 0; q < 2 * D / 32; ++q) {
+          float v[32];
+          tmem_ld32(lane_addr + q * 32, v);
+          tmem_wait_ld();
+          float* dst = q < D / 32 ? Ag + q * 32 : Bg + (q - D / 32) * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      } else {
+        // lanes 0..63 hold A rows, lanes 64..127 hold B rows
+        float* dst0 = row < D ? w.M + fh * DD + (long long)row * D : w.Cm + fh * DD + (long long)(row - D) * D;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          float v[32];
+          tmem_ld32(lane_addr + q * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst0 + q * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, kCols);
+}
+
+template <int D>
+cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  CUtensorMap mk, mv;
+  const long long tokens = (long long)d.B * d.T * d.N;
+  if (!make_token_map(&mk, in.k, tokens, d.H, D, TT) || !make_token_map(&mv, in.v, tokens, d.H, D, TT))
+    return cudaErrorInvalidValue;
+  const size_t smem = 1024 + 2 * (2 * (size_t)TT * D * 2) + 2 * (size_t)TT * D * 2 + 8 * 8 + 16;
+  auto kern = k_gram_tc<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(d.T, d.H, d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gram_tc_supported(const Dims& d) {
+  if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128)) return false;
+  if ((long long)d.B * d.T * d.N >= (1LL << 31)) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  if (d.dk == 128) return launch<128>(d, in, w, s);
+  if (d.dk == 64) return launch<64>(d, in, w, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

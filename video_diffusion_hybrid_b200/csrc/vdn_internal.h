@@ -48,6 +48,9 @@ __host__ __device__ inline bool is_anchor(const Dims& d, int t) {
 // Launchers (return cudaGetLastError after the launch).
 cudaError_t launch_text(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_solve_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_solve_inplace(const Dims& d, const Work& w, cudaStream_t s);
+bool gram_tc_supported(const Dims& d);
+cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_read_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_softmax_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);

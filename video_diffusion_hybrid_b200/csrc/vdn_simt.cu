@@ -53,102 +53,16 @@ __device__ __forceinline__ bool query_group(const Dims& d, int g, int& f0, int& 
   return f0 < f1;
 }
 
-// ---------------------------------------------------------------------------
-// Gram/write + Cholesky solve.  text=true: the L text tokens of (b,h), output
-// C/2 into half_text, no M.  Otherwise frame t = blockIdx.x of (b,h).
-// ---------------------------------------------------------------------------
-template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-k_gram_solve(Dims dm, Inputs in, Work w, bool text) {
-  constexpr int TT = 32;            // tokens per smem stage
-  constexpr int RPT = 2 * D / 16;   // rows of [A;B] per thread
-  constexpr int CPT = D / 16;       // cols per thread
-  constexpr int P = D + 1;          // padded pitch of the solve matrices
-  extern __shared__ float sm[];
+// Cholesky-based SPD solve in shared memory, 256 threads.  On entry G = I + A
+// and Bs = B (pitch D+1); writes M = (I+A)^-1 (to outM when not null) and
+// cscale * B M (to outC).  Uses G, Bs and W = sm + 2*D*(D+1) as scratch.
+template <int D>
+__device__ __forceinline__ void spd_solve(float* sm, float* outM, float* outC, float cscale) {
+  constexpr int P = D + 1;
   const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
-  const int b = blockIdx.z, h = blockIdx.y, t = blockIdx.x;
-
-  const T *kp, *vp;
-  const float* bp;
-  long long ntok;
-  float* outM = nullptr;
-  float* outC;
-  float cscale = 1.0f;
-  if (text) {
-    kp = static_cast<const T*>(in.text_k) + ((long long)b * dm.L * dm.H + h) * D;
-    vp = static_cast<const T*>(in.text_v) + ((long long)b * dm.L * dm.H + h) * D;
-    bp = in.text_beta + (long long)b * dm.L * dm.H + h;
-    ntok = dm.L;
-    outC = w.half_text + ((long long)b * dm.H + h) * D * D;
-    cscale = 0.5f;
-  } else {
-    if (is_anchor(dm, t)) return;
-    long long tok0 = ((long long)b * dm.T + t) * dm.N;
-    kp = static_cast<const T*>(in.k) + (tok0 * dm.H + h) * D;
-    vp = static_cast<const T*>(in.v) + (tok0 * dm.H + h) * D;
-    bp = in.beta + tok0 * dm.H + h;
-    ntok = dm.N;
-    long long fh = ((long long)b * dm.T + t) * dm.H + h;
-    outM = w.M + fh * D * D;
-    outC = w.Cm + fh * D * D;
-  }
-  const long long ts = (long long)dm.H * D;  // element stride between tokens
-
-  // ---- phase 1: [A; B] = sum_i [beta_i k_i; beta_i v_i] k_i^T -------------
-  float* Lf = sm;              // [TT][2D]
-  float* Rf = sm + TT * 2 * D; // [TT][D]
-  float acc[RPT][CPT];
-#pragma unroll
-  for (int i = 0; i < RPT; ++i)
-#pragma unroll
-    for (int j = 0; j < CPT; ++j) acc[i][j] = 0.f;
-
-  for (long long base = 0; base < ntok; base += TT) {
-    for (int idx = tid; idx < TT * D; idx += kThreads) {
-      int i = idx / D, c = idx % D;
-      long long tok = base + i;
-      float kk = 0.f, vv = 0.f, bb = 0.f;
-      if (tok < ntok) {
-        kk = ldf(kp + tok * ts + c);
-        vv = ldf(vp + tok * ts + c);
-        bb = __ldg(bp + tok * dm.H);
-      }
-      Lf[i * 2 * D + c] = bb * kk;
-      Lf[i * 2 * D + D + c] = bb * vv;
-      Rf[i * D + c] = kk;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int i = 0; i < TT; ++i) {
-      float a[RPT], r[CPT];
-#pragma unroll
-      for (int x = 0; x < RPT; ++x) a[x] = Lf[i * 2 * D + ty + 16 * x];
-#pragma unroll
-      for (int y = 0; y < CPT; ++y) r[y] = Rf[i * D + tx + 16 * y];
-#pragma unroll
-      for (int x = 0; x < RPT; ++x)
-#pragma unroll
-        for (int y = 0; y < CPT; ++y) acc[x][y] = fmaf(a[x], r[y], acc[x][y]);
-    }
-    __syncthreads();
-  }
-
-  // ---- phase 2: G = I + A (lower Cholesky in place), Bs = B ---------------
-  float* G = sm;            // [D][P]
-  float* Bs = sm + D * P;   // [D][P]
-  float* W = sm + 2 * D * P;// [D][P]
-#pragma unroll
-  for (int x = 0; x < RPT; ++x) {
-    int r = ty + 16 * x;
-#pragma unroll
-    for (int y = 0; y < CPT; ++y) {
-      int c = tx + 16 * y;
-      if (r < D) G[r * P + c] = acc[x][y] + (r == c ? 1.0f : 0.0f);
-      else Bs[(r - D) * P + c] = acc[x][y];
-    }
-  }
-  __syncthreads();
-
+  float* G = sm;
+  float* Bs = sm + D * P;
+  float* W = sm + 2 * D * P;
   for (int j = 0; j < D; ++j) {
     const float piv = sqrtf(G[j * P + j]);
     const float inv = 1.0f / piv;
@@ -240,9 +154,131 @@ k_gram_solve(Dims dm, Inputs in, Work w, bool text) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Gram/write + Cholesky solve.  text=true: the L text tokens of (b,h), output
+// C/2 into half_text, no M.  Otherwise frame t = blockIdx.x of (b,h).
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+k_gram_solve(Dims dm, Inputs in, Work w, bool text) {
+  constexpr int TT = 32;            // tokens per smem stage
+  constexpr int RPT = 2 * D / 16;   // rows of [A;B] per thread
+  constexpr int CPT = D / 16;       // cols per thread
+  constexpr int P = D + 1;          // padded pitch of the solve matrices
+  extern __shared__ float sm[];
+  const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+  const int b = blockIdx.z, h = blockIdx.y, t = blockIdx.x;
+
+  const T *kp, *vp;
+  const float* bp;
+  long long ntok;
+  float* outM = nullptr;
+  float* outC;
+  float cscale = 1.0f;
+  if (text) {
+    kp = static_cast<const T*>(in.text_k) + ((long long)b * dm.L * dm.H + h) * D;
+    vp = static_cast<const T*>(in.text_v) + ((long long)b * dm.L * dm.H + h) * D;
+    bp = in.text_beta + (long long)b * dm.L * dm.H + h;
+    ntok = dm.L;
+    outC = w.half_text + ((long long)b * dm.H + h) * D * D;
+    cscale = 0.5f;
+  } else {
+    if (is_anchor(dm, t)) return;
+    long long tok0 = ((long long)b * dm.T + t) * dm.N;
+    kp = static_cast<const T*>(in.k) + (tok0 * dm.H + h) * D;
+    vp = static_cast<const T*>(in.v) + (tok0 * dm.H + h) * D;
+    bp = in.beta + tok0 * dm.H + h;
+    ntok = dm.N;
+    long long fh = ((long long)b * dm.T + t) * dm.H + h;
+    outM = w.M + fh * D * D;
+    outC = w.Cm + fh * D * D;
+  }
+  const long long ts = (long long)dm.H * D;  // element stride between tokens
+
+  // ---- phase 1: [A; B] = sum_i [beta_i k_i; beta_i v_i] k_i^T -------------
+  float* Lf = sm;              // [TT][2D]
+  float* Rf = sm + TT * 2 * D; // [TT][D]
+  float acc[RPT][CPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i)
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) acc[i][j] = 0.f;
+
+  for (long long base = 0; base < ntok; base += TT) {
+    for (int idx = tid; idx < TT * D; idx += kThreads) {
+      int i = idx / D, c = idx % D;
+      long long tok = base + i;
+      float kk = 0.f, vv = 0.f, bb = 0.f;
+      if (tok < ntok) {
+        kk = ldf(kp + tok * ts + c);
+        vv = ldf(vp + tok * ts + c);
+        bb = __ldg(bp + tok * dm.H);
+      }
+      Lf[i * 2 * D + c] = bb * kk;
+      Lf[i * 2 * D + D + c] = bb * vv;
+      Rf[i * D + c] = kk;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int i = 0; i < TT; ++i) {
+      float a[RPT], r[CPT];
+#pragma unroll
+      for (int x = 0; x < RPT; ++x) a[x] = Lf[i * 2 * D + ty + 16 * x];
+#pragma unroll
+      for (int y = 0; y < CPT; ++y) r[y] = Rf[i * D + tx + 16 * y];
+#pragma unroll
+      for (int x = 0; x < RPT; ++x)
+#pragma unroll
+        for (int y = 0; y < CPT; ++y) acc[x][y] = fmaf(a[x], r[y], acc[x][y]);
+    }
+    __syncthreads();
+  }
+
+  // ---- phase 2: G = I + A (lower Cholesky in place), Bs = B ---------------
+  float* G = sm;            // [D][P]
+  float* Bs = sm + D * P;   // [D][P]
+
+#pragma unroll
+  for (int x = 0; x < RPT; ++x) {
+    int r = ty + 16 * x;
+#pragma unroll
+    for (int y = 0; y < CPT; ++y) {
+      int c = tx + 16 * y;
+      if (r < D) G[r * P + c] = acc[x][y] + (r == c ? 1.0f : 0.0f);
+      else Bs[(r - D) * P + c] = acc[x][y];
+    }
+  }
+  __syncthreads();
+
+  spd_solve<D>(sm, outM, outC, cscale);
+}
+
 __global__ void k_half_init(Dims dm, const float* __restrict__ init, float* __restrict__ half, long long n) {
   long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) half[i] = 0.5f * init[i];
+}
+
+// SPD solve of frames whose A_t, B_t were left by the tensor-core Gram in the
+// M_t and C_t slots of the workspace; overwrites them with M_t and C_t.
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+k_solve_inplace(Dims dm, Work w) {
+  constexpr int P = D + 1;
+  extern __shared__ float sm[];
+  const int b = blockIdx.z, h = blockIdx.y, t = blockIdx.x;
+  if (is_anchor(dm, t)) return;
+  const long long fh = ((long long)b * dm.T + t) * dm.H + h;
+  float* gA = w.M + fh * D * D;
+  float* gB = w.Cm + fh * D * D;
+  float* G = sm;
+  float* Bs = sm + D * P;
+  for (int idx = threadIdx.x; idx < D * D; idx += kThreads) {
+    const int r = idx / D, c = idx % D;
+    G[r * P + c] = gA[idx] + (r == c ? 1.0f : 0.0f);
+    Bs[r * P + c] = gB[idx];
+  }
+  __syncthreads();
+  spd_solve<D>(sm, gA, gB, 1.0f);
 }
 
 // ---------------------------------------------------------------------------
@@ -582,6 +618,17 @@ cudaError_t solve_launch(const Dims& d, const Inputs& in, const Work& w, cudaStr
 }
 
 template <int D>
+cudaError_t solve_inplace_launch(const Dims& d, const Inputs&, const Work& w, cudaStream_t s) {
+  constexpr int P = D + 1;
+  const size_t smem = sizeof(float) * (size_t)(3 * D * P);
+  auto kern = k_solve_inplace<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(d.T, d.H, d.B), kThreads, smem, s>>>(d, w);
+  return cudaGetLastError();
+}
+
+template <int D>
 cudaError_t scan_launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   constexpr int RB = D >= 64 ? 16 : 32;
   const size_t smem = sizeof(float) * (size_t)(D * D + RB * D);
@@ -657,6 +704,11 @@ cudaError_t launch_text(const Dims& d, const Inputs& in, const Work& w, cudaStre
 
 cudaError_t launch_solve_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   VDN_DISPATCH_D(solve_f, d, in, w, s, false)
+}
+
+cudaError_t launch_solve_inplace(const Dims& d, const Work& w, cudaStream_t s) {
+  const Inputs in{};
+  VDN_DISPATCH_D(solve_inplace_launch, d, in, w, s)
 }
 
 cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
