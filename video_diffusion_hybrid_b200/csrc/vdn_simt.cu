@@ -258,28 +258,6 @@ __global__ void k_half_init(Dims dm, const float* __restrict__ init, float* __re
   if (i < n) half[i] = 0.5f * init[i];
 }
 
-// SPD solve of frames whose A_t, B_t were left by the tensor-core Gram in the
-// M_t and C_t slots of the workspace; overwrites them with M_t and C_t.
-template <int D>
-__global__ void __launch_bounds__(kThreads)
-k_solve_inplace(Dims dm, Work w) {
-  constexpr int P = D + 1;
-  extern __shared__ float sm[];
-  const int b = blockIdx.z, h = blockIdx.y, t = blockIdx.x;
-  if (is_anchor(dm, t)) return;
-  const long long fh = ((long long)b * dm.T + t) * dm.H + h;
-  float* gA = w.M + fh * D * D;
-  float* gB = w.Cm + fh * D * D;
-  float* G = sm;
-  float* Bs = sm + D * P;
-  for (int idx = threadIdx.x; idx < D * D; idx += kThreads) {
-    const int r = idx / D, c = idx % D;
-    G[r * P + c] = gA[idx] + (r == c ? 1.0f : 0.0f);
-    Bs[r * P + c] = gB[idx];
-  }
-  __syncthreads();
-  spd_solve<D>(sm, gA, gB, 1.0f);
-}
 
 // ---------------------------------------------------------------------------
 // State scan.  grid (D/RB row blocks, 2 directions, B*H).  Rows of the state
@@ -618,17 +596,6 @@ cudaError_t solve_launch(const Dims& d, const Inputs& in, const Work& w, cudaStr
 }
 
 template <int D>
-cudaError_t solve_inplace_launch(const Dims& d, const Inputs&, const Work& w, cudaStream_t s) {
-  constexpr int P = D + 1;
-  const size_t smem = sizeof(float) * (size_t)(3 * D * P);
-  auto kern = k_solve_inplace<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  kern<<<dim3(d.T, d.H, d.B), kThreads, smem, s>>>(d, w);
-  return cudaGetLastError();
-}
-
-template <int D>
 cudaError_t scan_launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   constexpr int RB = D >= 64 ? 16 : 32;
   const size_t smem = sizeof(float) * (size_t)(D * D + RB * D);
@@ -704,11 +671,6 @@ cudaError_t launch_text(const Dims& d, const Inputs& in, const Work& w, cudaStre
 
 cudaError_t launch_solve_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   VDN_DISPATCH_D(solve_f, d, in, w, s, false)
-}
-
-cudaError_t launch_solve_inplace(const Dims& d, const Work& w, cudaStream_t s) {
-  const Inputs in{};
-  VDN_DISPATCH_D(solve_inplace_launch, d, in, w, s)
 }
 
 cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
