@@ -96,6 +96,14 @@ static __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_by
   return d;
 }
 
+// A descriptor advanced by a byte offset: the start address lives in the low
+// bits as addr >> 4, and shared addresses stay below 256 KB, so adding
+// offset >> 4 never carries out of the field.  Keeps the MMA issue loop to
+// one add per instruction (a single issuing thread is otherwise the limit).
+static __device__ __forceinline__ uint64_t dadd(uint64_t desc, uint32_t byte_offset) {
+  return desc + (uint64_t)(byte_offset >> 4);
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |

@@ -94,7 +94,8 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       // MN-major operands: M (or N) = d in 64-wide chunks TT*128 bytes apart,
       // 8-token groups 1024 bytes apart, 16 tokens (2048 bytes) per K-step.
       constexpr uint32_t ID = D == 128 ? (idesc_bf16(128, 128, true) | (1u << 15)) : (idesc_bf16(128, 64, true) | (1u << 15));
-      const uint32_t hi = smem_u32(sHi), lo = smem_u32(sLo);
+      const uint64_t hidesc = sdesc(smem_u32(sHi), TT * 128, 1024), lodesc = sdesc(smem_u32(sLo), TT * 128, 1024);
+      const uint64_t kvdesc0 = sdesc(smem_u32(sKV), TT * 128, 1024);
       bool ok = true;
       for (int j = 0; ok && j < ntiles; ++j) {
         const int s = j % ST;
@@ -103,16 +104,15 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
           break;
         }
         tc_fence_after();
-        const uint32_t ka = smem_u32(sKV + s * STAGE), va = ka + TB;
+        const uint64_t kd = dadd(kvdesc0, s * STAGE), vd = dadd(kd, TB);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint32_t kb = part ? lo : hi;
+          const uint64_t bd = part ? lodesc : hidesc;
 #pragma unroll
           for (int k = 0; k < TT / 16; ++k) {
             const uint32_t acc = (j | part | k) ? 1u : 0u;
-            const uint64_t bdesc = sdesc(kb + k * 2048, TT * 128, 1024);
-            mma_bf16(tmem, sdesc(ka + k * 2048, TT * 128, 1024), bdesc, ID, acc);
-            if (D == 128) mma_bf16(tmem + 128, sdesc(va + k * 2048, TT * 128, 1024), bdesc, ID, acc);
+            mma_bf16(tmem, dadd(kd, k * 2048), dadd(bd, k * 2048), ID, acc);
+            if (D == 128) mma_bf16(tmem + 128, dadd(vd, k * 2048), dadd(bd, k * 2048), ID, acc);
           }
         }
         mma_commit(bar(B_KVEMPTY + s));

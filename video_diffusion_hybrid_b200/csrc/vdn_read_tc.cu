@@ -207,23 +207,20 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t ID = idesc_bf16(TQ, D, false);
-      const uint32_t ra = smem_u32(sR);
+      const uint64_t rdesc = sdesc(smem_u32(sR), 16, 1024), qdesc0 = sdesc(smem_u32(sQ), 16, 1024);
       bool ok = mbar_wait(bar(B_R), 0, ctl);
       for (int t = 0; ok && t < run.ntiles; ++t) {
         const int s = t % ST;
         if (!mbar_wait(bar(B_QFULL + s), (t / ST) & 1, ctl)) break;
         if (t >= ST && !mbar_wait(bar(B_AEMPTY + s), (t / ST - 1) & 1, ctl)) break;
         tc_fence_after();
-        const uint32_t qa = smem_u32(sQ + s * TBYTES);
+        const uint64_t qd = dadd(qdesc0, s * TBYTES);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t qoff = (k >> 2) * (TQ * 128) + (k & 3) * 32;
-            const uint32_t roff = part * D * D * 2 + (k >> 2) * (D * 128) + (k & 3) * 32;
-            mma_bf16(tmem + s * D, sdesc(qa + qoff, 16, 1024), sdesc(ra + roff, 16, 1024), ID,
-                     (part | k) ? 1u : 0u);
-          }
+          for (int k = 0; k < D / 16; ++k)
+            mma_bf16(tmem + s * D, dadd(qd, (k >> 2) * (TQ * 128) + (k & 3) * 32),
+                     dadd(rdesc, part * D * D * 2 + (k >> 2) * (D * 128) + (k & 3) * 32), ID, (part | k) ? 1u : 0u);
         }
         mma_commit(bar(B_AFULL + s));
         mma_commit(bar(B_QEMPTY + s));

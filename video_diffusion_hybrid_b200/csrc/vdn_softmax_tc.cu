@@ -6,26 +6,35 @@
 // c the keys of chunks c-1..c+1 (clipped) plus the two anchor frames; anchor
 // query frames attend to every frame; y_sm = sigmoid(g_sm) * softmax(s q K^T) V.
 //
-// One CTA = one tile of 128 query rows of one (batch, head, query group); a
-// query group is the non-anchor frames of one chunk, or one anchor frame, so
-// every row of a tile has the same key set: at most three contiguous token
-// intervals (anchor frame 0, the window, anchor frame T-1).
+// One CTA = two tiles of 128 query rows (256 rows) of one (batch, head, query
+// group); a query group is the non-anchor frames of one chunk, or one anchor
+// frame, so every row has the same key set: at most three contiguous token
+// intervals (anchor frame 0, the window, anchor frame T-1).  Both query tiles
+// share every K / V tile.
 //
-// Roles (256 threads):
-//   warp 0      TMA producer of Q (once) and of the K ring (three stages,
-//               freed as soon as S_j is computed).
-//   warp 2      TMA producer of the V ring (three stages, freed after
-//               O += P_j V_j).  Separate threads, so that neither ring waits
-//               behind the other.  128B-swizzled boxes of 64 dims x 128 rows.
-//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma:
-//                 S_j = Q K_j^T  (M=128, N=128, K=d; both from SMEM) -> TMEM S[j % 2]
-//                 O  += P_j V_j  (M=128, N=d, K=128; P from TMEM)    -> TMEM O
-//   warps 4..7  softmax: thread r owns query row r (= TMEM lane r).  It reads
-//               its row of S_j, keeps a running max / sum, computes P_j into
-//               registers, writes it (bf16, two per column) to TMEM and
-//               rescales its row of O only when the max grew by more than 2^8
-//               (exact: p <= 2^8 is then guaranteed, and O and the sum share
-//               the same stale max).  Epilogue: O / l, gate, store.
+// Roles (384 threads):
+//   warp 0      TMA producer of Q (both tiles, once) and of the K ring (three
+//               stages, freed after both S_0 and S_1 of that tile).
+//   warp 2      TMA producer of the V ring (two stages, freed after both PVs).
+//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma.  Per key tile
+//               j the tensor pipe runs, in this order,
+//                 O_0 += P_0(j) V_j,  S_0 = Q_0 K_{j+1}^T,  O_1 += P_1(j) V_j,  S_1 = Q_1 K_{j+1}^T
+//               so that while one softmax warpgroup works on its tile the pipe
+//               computes the other tile's product (ping-pong).  S: M=128, N=128,
+//               K=d, both operands from SMEM; PV: A = P from TMEM (TS form).
+//   warps 4..7  softmax of query tile 0, warps 8..11 of query tile 1: thread r
+//               owns row r (= TMEM lane r).  Pass 1 reads its row of S and takes
+//               the max; pass 2 re-reads it in halves, computes P (bf16) and
+//               writes it over the S columns already read.  O is rescaled only
+//               when a row max grew by more than 2^8 (exact: p <= 2^8 then, and
+//               O and the row sum share the same stale max).  The row sum uses
+//               the bf16-rounded P, so every output row is an exact convex
+//               combination of V rows.  Epilogue: O / l, gate, store.
+//
+// TMEM (512 columns): O_0 [0,128), O_1 [128,256), S_0 [256,384), S_1 [384,512);
+// P_t lives in the first 64 columns of S_t.  A tile's next S is issued after
+// its PV by the same thread, and tcgen05.mma operations of one thread run in
+// issue order, so P_t(j) is consumed before S_t(j+1) overwrites it.
 //
 // Every mbarrier wait is bounded (about one second of clock cycles); on
 // expiry the CTA records VDN_ERR_TIMEOUT in the workspace status words, stops
@@ -37,24 +46,26 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128;           // query rows per tile
+constexpr int NQ = 2;             // query tiles per CTA
 constexpr int BN = 128;           // keys per tile
-constexpr int kThreadsTC = 256;
-constexpr int kSoftmaxWarp0 = 4;  // warps 4..7 (TMEM lane quadrants 0..3)
+constexpr int kThreadsTC = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS0 = 128, kColS1 = 256, kColP = 384;
 constexpr float kRescaleLog2 = 8.0f;
+
+__host__ __device__ constexpr uint32_t col_o(int t) { return 128u * t; }
+__host__ __device__ constexpr uint32_t col_s(int t) { return 256u + 128u * t; }
 
 // ------------------------------------------------------ work decomposition --
 struct Tile {
-  int b, h, q0, qrows;      // absolute first query token and valid rows
+  int b, h, q0, qrows;      // absolute first query token, valid rows (of 256)
   int niv;                  // key intervals
   int kbeg[3], klen[3];     // absolute first key token, length
 };
 
-__device__ __forceinline__ void group_frames(const Dims& d, int g, int& f0, int& f1, int& ridx) {
+__host__ __device__ inline void group_frames(const Dims& d, int g, int& f0, int& f1, int& ridx) {
   if (g < d.C) {
     f0 = g * d.chunk;
-    f1 = min(d.T, f0 + d.chunk);
+    f1 = f0 + d.chunk < d.T ? f0 + d.chunk : d.T;
     if (d.anchors) {
       if (f0 == 0) f0 = 1;
       if (f1 == d.T) f1 = d.T - 1;
@@ -67,51 +78,54 @@ __device__ __forceinline__ void group_frames(const Dims& d, int g, int& f0, int&
   }
 }
 
-// Item order: all anchor-row tiles first (longest), then per (b, h) the
+__host__ __device__ inline long long pairs_of_rows(long long rows) { return (rows + NQ * BM - 1) / (NQ * BM); }
+
+// Item order: all anchor-row pairs first (longest), then per (b, h) the
 // regular groups in chunk order, so concurrent CTAs share K/V windows in L2.
 __device__ bool decode_item(const Dims& d, long long item, Tile& t) {
   const int n_anc = d.anchors ? 2 : 0;
-  const int tiles_a = (d.N + BM - 1) / BM;
-  const long long anc_items = (long long)d.B * d.H * n_anc * tiles_a;
-  int bh, g, qt;
+  const long long pairs_a = pairs_of_rows(d.N);
+  const long long anc_items = (long long)d.B * d.H * n_anc * pairs_a;
+  int g;
+  long long bh, qp;
   if (item < anc_items) {
-    bh = (int)(item / (n_anc * tiles_a));
-    const int r = (int)(item % (n_anc * tiles_a));
-    g = d.C + r / tiles_a;
-    qt = r % tiles_a;
+    bh = item / (n_anc * pairs_a);
+    const long long r = item % (n_anc * pairs_a);
+    g = d.C + (int)(r / pairs_a);
+    qp = r % pairs_a;
   } else {
-    long long it = item - anc_items;
+    const long long it = item - anc_items;
     long long per_bh = 0;
     for (int gg = 0; gg < d.C; ++gg) {
       int f0, f1, ri;
       group_frames(d, gg, f0, f1, ri);
-      if (f1 > f0) per_bh += ((long long)(f1 - f0) * d.N + BM - 1) / BM;
+      if (f1 > f0) per_bh += pairs_of_rows((long long)(f1 - f0) * d.N);
     }
     if (per_bh == 0) return false;
-    bh = (int)(it / per_bh);
+    bh = it / per_bh;
     long long rem = it % per_bh;
     g = -1;
-    qt = 0;
+    qp = 0;
     for (int gg = 0; gg < d.C; ++gg) {
       int f0, f1, ri;
       group_frames(d, gg, f0, f1, ri);
       if (f1 <= f0) continue;
-      const long long nt = ((long long)(f1 - f0) * d.N + BM - 1) / BM;
-      if (rem < nt) { g = gg; qt = (int)rem; break; }
-      rem -= nt;
+      const long long np = pairs_of_rows((long long)(f1 - f0) * d.N);
+      if (rem < np) { g = gg; qp = rem; break; }
+      rem -= np;
     }
     if (g < 0) return false;
   }
-  if (bh >= d.B * d.H) return false;
-  t.b = bh / d.H;
-  t.h = bh % d.H;
+  if (bh >= (long long)d.B * d.H) return false;
+  t.b = (int)(bh / d.H);
+  t.h = (int)(bh % d.H);
   int f0, f1, ridx;
   group_frames(d, g, f0, f1, ridx);
   if (f1 <= f0) return false;
   const int base = t.b * d.T * d.N;
   const int rows = (f1 - f0) * d.N;
-  t.q0 = base + f0 * d.N + qt * BM;
-  t.qrows = min(BM, rows - qt * BM);
+  t.q0 = base + f0 * d.N + (int)qp * NQ * BM;
+  t.qrows = min(NQ * BM, rows - (int)qp * NQ * BM);
   t.niv = 0;
   if (ridx == d.C) {
     t.kbeg[0] = base; t.klen[0] = d.T * d.N; t.niv = 1;
@@ -165,15 +179,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
              const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
   constexpr int NB = D / 64;                 // 64-wide column blocks of a row
-  constexpr uint32_t QBYTES = BM * D * 2;
+  constexpr uint32_t QTILE = BM * D * 2;
   constexpr uint32_t KVBYTES = BN * D * 2;
-  constexpr int KST = 3, VST = 3;            // K and V ring depths
-  enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 10, B_SFULL = 13, B_PFULL = 15, B_ODONE = 16,
+  constexpr int KST = 3, VST = 2;            // K and V ring depths
+  enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 9, B_SFULL = 11, B_PFULL = 13, B_ODONE = 15,
          B_DRAIN = 17, NBARS = 18 };
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sQ = sm;
-  unsigned char* sK = sQ + QBYTES;           // KST stages
+  unsigned char* sQ = sm;                    // NQ tiles
+  unsigned char* sK = sQ + NQ * QTILE;       // KST stages
   unsigned char* sV = sK + KST * KVBYTES;    // VST stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VST * KVBYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
@@ -189,26 +203,11 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_Q), 1);
-    for (int s = 0; s < KST; ++s) {
-      mbar_init(bar(B_KFULL + s), 1);
-      mbar_init(bar(B_KEMPTY + s), 1);
-    }
-    for (int s = 0; s < VST; ++s) {
-      mbar_init(bar(B_VFULL + s), 1);
-      mbar_init(bar(B_VEMPTY + s), 1);
-    }
-    mbar_init(bar(B_SFULL + 0), 1);
-    mbar_init(bar(B_SFULL + 1), 1);
-    mbar_init(bar(B_PFULL), 128);
-    mbar_init(bar(B_ODONE), 1);
-    mbar_init(bar(B_DRAIN), 1);
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_PFULL || i == B_PFULL + 1) ? 128 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -219,9 +218,10 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmq)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmk)) : "memory");
-      mbar_expect_tx(bar(B_Q), QBYTES);
-      for (int c = 0; c < NB; ++c)
-        tma_load_3d(smem_u32(sQ + c * BM * 128), &tmq, bar(B_Q), c * 64, tile.h, tile.q0);
+      mbar_expect_tx(bar(B_Q), NQ * QTILE);
+      for (int t = 0; t < NQ; ++t)
+        for (int c = 0; c < NB; ++c)
+          tma_load_3d(smem_u32(sQ + t * QTILE + c * BM * 128), &tmq, bar(B_Q), c * 64, tile.h, tile.q0 + t * BM);
       int lastk[KST];
       for (int s = 0; s < KST; ++s) lastk[s] = -1;
       for (int j = 0; j < ntiles; ++j) {
@@ -263,161 +263,207 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
     if (lane == 0) {
       constexpr uint32_t ID_S = idesc_bf16(BM, BN, false);
       constexpr uint32_t ID_O = idesc_bf16(BM, D, true);
-      const uint32_t qa = smem_u32(sQ);
-      auto issue_s = [&](int j) -> bool {
-        const int sk = j % KST, sb = j & 1;
-        if (!mbar_wait(bar(B_KFULL + sk), (j / KST) & 1, ctl)) return false;
+      // descriptors built once; each k-step adds a compile-time offset
+      const uint64_t qdesc[NQ] = {sdesc(smem_u32(sQ), 16, 1024), sdesc(smem_u32(sQ + QTILE), 16, 1024)};
+      const uint64_t kdesc0 = sdesc(smem_u32(sK), 16, 1024);
+      const uint64_t vdesc0 = sdesc(smem_u32(sV), BN * 128, 1024);
+      // S_t = Q_t K_j^T
+      auto issue_s = [&](int t, int j) -> bool {
+        const int sk = j % KST;
+        if (t == 0 && !mbar_wait(bar(B_KFULL + sk), (j / KST) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t ka = smem_u32(sK + sk * KVBYTES);
-        const uint32_t dcol = tmem + (sb ? kColS1 : kColS0);
+        const uint64_t qd = qdesc[t], kd = dadd(kdesc0, sk * KVBYTES);
+        const uint32_t dst = tmem + col_s(t);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * (BM * 128) + (k & 3) * 32;
-          const uint32_t koff = (k >> 2) * (BN * 128) + (k & 3) * 32;
-          mma_bf16(dcol, sdesc(qa + off, 16, 1024), sdesc(ka + koff, 16, 1024), ID_S, k > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(B_SFULL + sb));
-        mma_commit(bar(B_KEMPTY + sk));
+        for (int k = 0; k < D / 16; ++k)
+          mma_bf16(dst, dadd(qd, (k >> 2) * (BM * 128) + (k & 3) * 32), dadd(kd, (k >> 2) * (BN * 128) + (k & 3) * 32),
+                   ID_S, k > 0 ? 1u : 0u);
+        mma_commit(bar(B_SFULL + t));
+        if (t == NQ - 1) mma_commit(bar(B_KEMPTY + sk));  // K_j read by both tiles
+        return true;
+      };
+      // O_t += P_t(j) V_j
+      auto issue_pv = [&](int t, int j) -> bool {
+        const int sv = j % VST;
+        if (!mbar_wait(bar(B_PFULL + t), j & 1, ctl)) return false;
+        if (t == 0 && !mbar_wait(bar(B_VFULL + sv), (j / VST) & 1, ctl)) return false;
+        tc_fence_after();
+        const uint64_t vd = dadd(vdesc0, sv * KVBYTES);
+        const uint32_t dst = tmem + col_o(t), pa = tmem + col_s(t);
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)
+          mma_bf16_ts(dst, pa + 8 * k, dadd(vd, k * 16 * 128), ID_O, (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(bar(B_ODONE + t));
+        if (t == NQ - 1) mma_commit(bar(B_VEMPTY + sv));  // V_j read by both tiles
         return true;
       };
       bool ok = mbar_wait(bar(B_Q), 0, ctl);
-      if (ok) ok = issue_s(0);
-      if (ok && ntiles > 1) ok = issue_s(1);
+      if (ok) ok = issue_s(0, 0);
+      if (ok) ok = issue_s(1, 0);
       for (int j = 0; ok && j < ntiles; ++j) {
-        const int sv = j % VST;
-        if (!mbar_wait(bar(B_PFULL), j & 1, ctl) || !mbar_wait(bar(B_VFULL + sv), (j / VST) & 1, ctl)) break;
-        tc_fence_after();
-        const uint32_t va = smem_u32(sV + sv * KVBYTES);
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(va + k * 16 * 128, BN * 128, 1024), ID_O,
-                      (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(bar(B_ODONE));
-        mma_commit(bar(B_VEMPTY + sv));
-        if (j + 2 < ntiles) ok = issue_s(j + 2);
+        ok = issue_pv(0, j);
+        if (ok && j + 1 < ntiles) ok = issue_s(0, j + 1);
+        if (ok) ok = issue_pv(1, j);
+        if (ok && j + 1 < ntiles) ok = issue_s(1, j + 1);
       }
       // drain: completion of every MMA issued by this thread
       mma_commit(bar(B_DRAIN));
       mbar_wait(bar(B_DRAIN), 0, ctl);
     }
-  } else if (warp >= kSoftmaxWarp0) {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
-    const int quad = warp - kSoftmaxWarp0;  // TMEM lane quadrant
+    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
+    const int quad = warp & 3;              // TMEM lane quadrant
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t scol = lane_addr + col_s(t), ocol = lane_addr + col_o(t);
     const float c = dm.scale * 1.4426950408889634f;  // log2 units
     const float thresh = kRescaleLog2 / c;            // raw-score units
     float m_used = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int s = j & 1;
       // every TMEM access below is warp-collective: keep control flow warp-uniform
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + s), (j >> 1) & 1, ctl))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + t), j & 1, ctl))) { ok = false; break; }
       tc_fence_after();
-      float x[BN];
-      {
-        // four loads in flight, one wait
-        float v0[32], v1[32], v2[32], v3[32];
-        const uint32_t scol = lane_addr + (s ? kColS1 : kColS0);
-        tmem_ld32(scol + 0, v0);
-        tmem_ld32(scol + 32, v1);
-        tmem_ld32(scol + 64, v2);
-        tmem_ld32(scol + 96, v3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = v0[i];
-          x[32 + i] = v1[i];
-          x[64 + i] = v2[i];
-          x[96 + i] = v3[i];
-        }
-      }
       int k0, kvalid;
       key_tile(tile, j, k0, kvalid);
-      if (kvalid < BN) {
+      bool done = false;
+      // Fast path (full key tile after the first): one pass with the running
+      // max.  Nothing is stored until the whole row is known not to overflow
+      // (no score more than 2^8 above the running max), so a warp that sees
+      // an overflow redoes the tile on the exact two-pass path below.
+      if (j > 0 && kvalid == BN) {
+        const float mc = m_used * c, lim = m_used + thresh;
+        float pm[8], ps[8];
 #pragma unroll
-        for (int i = 0; i < BN; ++i)
-          if (i >= kvalid) x[i] = -INFINITY;
-      }
-      // row max with eight independent chains (one warp per SMSP: no other
-      // warp hides a long dependent chain)
-      float pm[8];
+        for (int u = 0; u < 8; ++u) { pm[u] = -INFINITY; ps[u] = 0.f; }
+        float pk0[32], pk1[32];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) pm[u] = x[u];
-#pragma unroll
-      for (int i = 8; i < BN; ++i) pm[i & 7] = fmaxf(pm[i & 7], x[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-      // lazy rescale decision: only rows whose max grew by more than 2^8
-      const bool need = mx > m_used + thresh;
-      float f = 1.0f;
-      if (need) {
-        f = (m_used == -INFINITY) ? 0.f : ex2((m_used - mx) * c);
-        l_sum *= f;
-        m_used = mx;
-      }
-      // exponentials into packed bf16 registers first: this overlaps with the
-      // tensor core still computing O += P_{j-1} V_{j-1} from shared memory
-      const float mc = m_used * c;
-      uint32_t pk[BN / 2];
-      float ps[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-#pragma unroll
-      for (int i = 0; i < BN / 2; ++i) {
-        const float p0 = ex2(fmaf(x[2 * i], c, -mc));
-        const float p1 = ex2(fmaf(x[2 * i + 1], c, -mc));
-        pk[i] = pack_bf16(p0, p1);
-        // the row sum uses the bf16-rounded weights the MMA multiplies by,
-        // so every output row is an exact convex combination of V rows
-        ps[(2 * i) & 7] += __uint_as_float(pk[i] << 16);
-        ps[(2 * i + 1) & 7] += __uint_as_float(pk[i] & 0xFFFF0000u);
-      }
-      const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      // O and the P buffer are free once O += P_{j-1} V_{j-1} has completed
-      if (j > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ODONE), (j - 1) & 1, ctl))) { ok = false; break; }
-        tc_fence_after();
-      }
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        float v[32];
-#pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          tmem_ld32(lane_addr + kColO + q * 32, v);
+        for (int hf = 0; hf < 2; ++hf) {
+          float v0[32], v1[32];
+          tmem_ld32(scol + 64 * hf, v0);
+          tmem_ld32(scol + 64 * hf + 32, v1);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= f;
-          tmem_st32(lane_addr + kColO + q * 32, v);
+          for (int i = 0; i < 32; ++i) {
+            const float a0 = i < 16 ? v0[2 * i] : v1[2 * i - 32];
+            const float a1 = i < 16 ? v0[2 * i + 1] : v1[2 * i - 31];
+            pm[(2 * i) & 7] = fmaxf(pm[(2 * i) & 7], a0);
+            pm[(2 * i + 1) & 7] = fmaxf(pm[(2 * i + 1) & 7], a1);
+            const uint32_t u = pack_bf16(ex2(fmaf(a0, c, -mc)), ex2(fmaf(a1, c, -mc)));
+            ps[(2 * i) & 7] += __uint_as_float(u << 16);
+            ps[(2 * i + 1) & 7] += __uint_as_float(u & 0xFFFF0000u);
+            if (hf == 0) pk0[i] = __uint_as_float(u); else pk1[i] = __uint_as_float(u);
+          }
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        if (!__any_sync(0xffffffffu, mx > lim)) {
+          tmem_st32(scol, pk0);        // P columns [0, 32)
+          tmem_st32(scol + 32, pk1);   // P columns [32, 64)
+          tmem_wait_st();
+          l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+          done = true;
+        }
+      }
+      if (!done) {
+        // Exact path: pass 1 takes the row max, O is rescaled if it grew by
+        // more than 2^8, pass 2 computes and stores P.
+        // pass 1: row max (eight independent chains)
+        float pm[8];
+  #pragma unroll
+        for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+  #pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v0[32], v1[32];
+          tmem_ld32(scol + 64 * hf, v0);
+          tmem_ld32(scol + 64 * hf + 32, v1);
+          tmem_wait_ld();
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int c0 = 64 * hf + i, c1 = 64 * hf + 32 + i;
+            pm[i & 7] = fmaxf(pm[i & 7], c0 < kvalid ? v0[i] : -INFINITY);
+            pm[i & 7] = fmaxf(pm[i & 7], c1 < kvalid ? v1[i] : -INFINITY);
+          }
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        // lazy rescale decision: only rows whose max grew by more than 2^8
+        const bool need = mx > m_used + thresh;
+        float f = 1.0f;
+        if (need) {
+          f = (m_used == -INFINITY) ? 0.f : ex2((m_used - mx) * c);
+          l_sum *= f;
+          m_used = mx;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O is stable once O += P(j-1) V(j-1) has completed
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ODONE + t), (j - 1) & 1, ctl))) { ok = false; break; }
+          tc_fence_after();
+          float v[32];
+  #pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            tmem_ld32(ocol + q * 32, v);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= f;
+            tmem_st32(ocol + q * 32, v);
+          }
+          tmem_wait_st();
+        }
+        // pass 2: P = exp2(s c - m c) in bf16, written over the S columns already read
+        const float mc = m_used * c;
+        float ps[8];
+  #pragma unroll
+        for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+  #pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v0[32], v1[32];
+          tmem_ld32(scol + 64 * hf, v0);
+          tmem_ld32(scol + 64 * hf + 32, v1);
+          tmem_wait_ld();
+          float pk[32];
+  #pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = 64 * hf + 2 * i;
+            const float p0 = c0 < kvalid ? ex2(fmaf(v0[2 * i], c, -mc)) : 0.f;
+            const float p1 = c0 + 1 < kvalid ? ex2(fmaf(v0[2 * i + 1], c, -mc)) : 0.f;
+            const uint32_t u = pack_bf16(p0, p1);
+            ps[(2 * i) & 7] += __uint_as_float(u << 16);
+            ps[(2 * i + 1) & 7] += __uint_as_float(u & 0xFFFF0000u);
+            pk[i] = __uint_as_float(u);
+          }
+  #pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = 64 * hf + 32 + 2 * i;
+            const float p0 = c0 < kvalid ? ex2(fmaf(v1[2 * i], c, -mc)) : 0.f;
+            const float p1 = c0 + 1 < kvalid ? ex2(fmaf(v1[2 * i + 1], c, -mc)) : 0.f;
+            const uint32_t u = pack_bf16(p0, p1);
+            ps[(2 * i) & 7] += __uint_as_float(u << 16);
+            ps[(2 * i + 1) & 7] += __uint_as_float(u & 0xFFFF0000u);
+            pk[16 + i] = __uint_as_float(u);
+          }
+          tmem_st32(scol + 32 * hf, pk);  // P columns [32 hf, 32 hf + 32) of this tile
         }
         tmem_wait_st();
+        l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       }
-      {
-        float h0[32], h1[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          h0[i] = __uint_as_float(pk[i]);
-          h1[i] = __uint_as_float(pk[32 + i]);
-        }
-        tmem_st32(lane_addr + kColP, h0);
-        tmem_st32(lane_addr + kColP + 32, h1);
-        tmem_wait_st();
-      }
-      l_sum += sum;
       tc_fence_before();
-      mbar_arrive(bar(B_PFULL));
+      mbar_arrive(bar(B_PFULL + t));
     }
     // ---- epilogue: O / l, gate, store
-    if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_ODONE), (ntiles - 1) & 1, ctl))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_ODONE + t), (ntiles - 1) & 1, ctl))) {
       tc_fence_after();
       const float inv = 1.0f / l_sum;
-      const bool valid = row < tile.qrows;
-      const long long tok = (long long)tile.q0 + row;
+      const int trow = t * BM + row;
+      const bool valid = trow < tile.qrows;
+      const long long tok = (long long)tile.q0 + trow;
       const long long gi = (tok * dm.H + tile.h) * D;
       To* y = static_cast<To*>(in.y) + (dm.out_mode == 0 ? 2 * gi : gi);
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         float v[32];
-        tmem_ld32(lane_addr + kColO + q * 32, v);
+        tmem_ld32(ocol + q * 32, v);
         tmem_wait_ld();
         if (valid) {
           float g[32];
@@ -454,9 +500,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) {
-    tmem_free(tmem, kTmemCols);
-  }
+  if (warp == 1) tmem_free(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------- host --
@@ -464,14 +508,11 @@ long long num_items(const Dims& d) {
   const int n_anc = d.anchors ? 2 : 0;
   long long per_bh = 0;
   for (int g = 0; g < d.C; ++g) {
-    int f0 = g * d.chunk, f1 = std::min(d.T, f0 + d.chunk);
-    if (d.anchors) {
-      if (f0 == 0) f0 = 1;
-      if (f1 == d.T) f1 = d.T - 1;
-    }
-    if (f1 > f0) per_bh += ((long long)(f1 - f0) * d.N + BM - 1) / BM;
+    int f0, f1, ri;
+    group_frames(d, g, f0, f1, ri);
+    if (f1 > f0) per_bh += pairs_of_rows((long long)(f1 - f0) * d.N);
   }
-  return (long long)d.B * d.H * (per_bh + n_anc * ((d.N + BM - 1) / BM));
+  return (long long)d.B * d.H * (per_bh + n_anc * pairs_of_rows(d.N));
 }
 
 template <int D, typename To>
@@ -481,7 +522,7 @@ cudaError_t launch_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream
   if (!make_token_map(&mq, in.q, tokens, d.H, D, BM) || !make_token_map(&mk, in.k, tokens, d.H, D, BN) ||
       !make_token_map(&mv, in.v, tokens, d.H, D, BN))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + (size_t)BM * D * 2 + 6 * (size_t)BN * D * 2 + 18 * 8 + 16;
+  const size_t smem = 1024 + (size_t)NQ * BM * D * 2 + 5 * (size_t)BN * D * 2 + 18 * 8 + 16;
   auto kern = k_softmax_tc<D, To>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -496,8 +537,8 @@ cudaError_t launch_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream
 bool softmax_tc_supported(const Dims& d) {
   if (!d.bf16 || d.dk != d.dv) return false;
   if (d.dk != 64 && d.dk != 128) return false;
-  // token indices of the TMA coordinates are int32
-  if ((long long)d.B * d.T * d.N >= (1LL << 31)) return false;
+  // token indices of the TMA coordinates are int32 (plus one tile of overhang)
+  if ((long long)d.B * d.T * d.N + NQ * BM >= (1LL << 31)) return false;
   return encode_fn() != nullptr;
 }
 
