@@ -333,10 +333,11 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       // (no score more than 2^8 above the running max), so a warp that sees
       // an overflow redoes the tile on the exact two-pass path below.
       if (j > 0 && kvalid == BN) {
-        const float mc = m_used * c, lim = m_used + thresh;
-        float pm[8], ps[8];
+        const float2 c2 = make_float2(c, c), nmc2 = make_float2(-m_used * c, -m_used * c);
+        float2 ps2[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) { pm[u] = -INFINITY; ps[u] = 0.f; }
+        for (int u = 0; u < 4; ++u) ps2[u] = make_float2(0.f, 0.f);
+        uint32_t pmax = 0u;  // running max of the packed P (bf16 pairs, all >= 0)
         float pk0[32], pk1[32];
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -346,23 +347,23 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float a0 = i < 16 ? v0[2 * i] : v1[2 * i - 32];
-            const float a1 = i < 16 ? v0[2 * i + 1] : v1[2 * i - 31];
-            pm[(2 * i) & 7] = fmaxf(pm[(2 * i) & 7], a0);
-            pm[(2 * i + 1) & 7] = fmaxf(pm[(2 * i + 1) & 7], a1);
-            const uint32_t u = pack_bf16(ex2(fmaf(a0, c, -mc)), ex2(fmaf(a1, c, -mc)));
-            ps[(2 * i) & 7] += __uint_as_float(u << 16);
-            ps[(2 * i + 1) & 7] += __uint_as_float(u & 0xFFFF0000u);
+            const float2 sv = i < 16 ? make_float2(v0[2 * i], v0[2 * i + 1]) : make_float2(v1[2 * i - 32], v1[2 * i - 31]);
+            const float2 x = fma2(sv, c2, nmc2);
+            const uint32_t u = pack_bf16(ex2(x.x), ex2(x.y));
+            pmax = max_bf16x2(pmax, u);
+            ps2[i & 3] = add2(ps2[i & 3], make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
             if (hf == 0) pk0[i] = __uint_as_float(u); else pk1[i] = __uint_as_float(u);
           }
         }
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        if (!__any_sync(0xffffffffu, mx > lim)) {
+        // overflow: some weight above 2^8, i.e. a score more than 2^8 (in exp2
+        // units) above the running max; the exact path then rescales
+        const float pmx = fmaxf(__uint_as_float(pmax << 16), __uint_as_float(pmax & 0xFFFF0000u));
+        if (!__any_sync(0xffffffffu, !(pmx <= 256.0f))) {
           tmem_st32(scol, pk0);        // P columns [0, 32)
           tmem_st32(scol + 32, pk1);   // P columns [32, 64)
           tmem_wait_st();
-          l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+          const float2 t2 = add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3]));
+          l_sum += t2.x + t2.y;
           done = true;
         }
       }
