@@ -47,9 +47,22 @@ struct Ctl {
   unsigned tag;         // kernel tag recorded on a timeout
 };
 
-// Bounded wait: true when the phase completed; false after ~1 s or when
-// another role of the CTA already gave up.
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
+// Non-suspending test of a phase.
+static __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait, slow path: true when the phase completed; false after ~1 s
+// or when another role of the CTA already gave up.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
@@ -64,6 +77,12 @@ static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, con
       }
     }
   }
+}
+
+// Bounded wait: an already completed phase costs one inline test, without the
+// call and the suspending try_wait of the slow path.
+static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
+  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, c);
 }
 
 static __device__ __forceinline__ void fence_barrier_init() {

@@ -267,44 +267,47 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       const uint64_t qdesc[NQ] = {sdesc(smem_u32(sQ), 16, 1024), sdesc(smem_u32(sQ + QTILE), 16, 1024)};
       const uint64_t kdesc0 = sdesc(smem_u32(sK), 16, 1024);
       const uint64_t vdesc0 = sdesc(smem_u32(sV), BN * 128, 1024);
-      // S_t = Q_t K_j^T
-      auto issue_s = [&](int t, int j) -> bool {
+      // S_t = Q_t K_j^T and O_t += P_t(j) V_j, issued once the barriers they
+      // need have been cleared (waits first, then the MMAs back to back).
+      auto mma_s = [&](int t, int j) {
         const int sk = j % KST;
-        if (t == 0 && !mbar_wait(bar(B_KFULL + sk), (j / KST) & 1, ctl)) return false;
-        tc_fence_after();
         const uint64_t qd = qdesc[t], kd = dadd(kdesc0, sk * KVBYTES);
         const uint32_t dst = tmem + col_s(t);
+        mma_bf16(dst, qd, kd, ID_S, 0u);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
+        for (int k = 1; k < D / 16; ++k)
           mma_bf16(dst, dadd(qd, (k >> 2) * (BM * 128) + (k & 3) * 32), dadd(kd, (k >> 2) * (BN * 128) + (k & 3) * 32),
-                   ID_S, k > 0 ? 1u : 0u);
+                   ID_S, 1u);
         mma_commit(bar(B_SFULL + t));
         if (t == NQ - 1) mma_commit(bar(B_KEMPTY + sk));  // K_j read by both tiles
-        return true;
       };
-      // O_t += P_t(j) V_j
-      auto issue_pv = [&](int t, int j) -> bool {
+      auto mma_pv = [&](int t, int j) {
         const int sv = j % VST;
-        if (!mbar_wait(bar(B_PFULL + t), j & 1, ctl)) return false;
-        if (t == 0 && !mbar_wait(bar(B_VFULL + sv), (j / VST) & 1, ctl)) return false;
-        tc_fence_after();
         const uint64_t vd = dadd(vdesc0, sv * KVBYTES);
         const uint32_t dst = tmem + col_o(t), pa = tmem + col_s(t);
+        mma_bf16_ts(dst, pa, vd, ID_O, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 0; k < BN / 16; ++k)
-          mma_bf16_ts(dst, pa + 8 * k, dadd(vd, k * 16 * 128), ID_O, (j > 0 || k > 0) ? 1u : 0u);
+        for (int k = 1; k < BN / 16; ++k) mma_bf16_ts(dst, pa + 8 * k, dadd(vd, k * 16 * 128), ID_O, 1u);
         mma_commit(bar(B_ODONE + t));
         if (t == NQ - 1) mma_commit(bar(B_VEMPTY + sv));  // V_j read by both tiles
-        return true;
       };
-      bool ok = mbar_wait(bar(B_Q), 0, ctl);
-      if (ok) ok = issue_s(0, 0);
-      if (ok) ok = issue_s(1, 0);
+      bool ok = mbar_wait(bar(B_Q), 0, ctl) && mbar_wait(bar(B_KFULL), 0, ctl);
+      if (ok) {
+        tc_fence_after();
+        mma_s(0, 0);
+        mma_s(1, 0);
+      }
       for (int j = 0; ok && j < ntiles; ++j) {
-        ok = issue_pv(0, j);
-        if (ok && j + 1 < ntiles) ok = issue_s(0, j + 1);
-        if (ok) ok = issue_pv(1, j);
-        if (ok && j + 1 < ntiles) ok = issue_s(1, j + 1);
+        const bool more = j + 1 < ntiles;
+        for (int t = 0; ok && t < NQ; ++t) {
+          ok = mbar_wait(bar(B_PFULL + t), j & 1, ctl) &&
+               (t > 0 || mbar_wait(bar(B_VFULL + j % VST), (j / VST) & 1, ctl)) &&
+               (t > 0 || !more || mbar_wait(bar(B_KFULL + (j + 1) % KST), ((j + 1) / KST) & 1, ctl));
+          if (!ok) break;
+          tc_fence_after();
+          mma_pv(t, j);
+          if (more) mma_s(t, j + 1);
+        }
       }
       // drain: completion of every MMA issued by this thread
       mma_commit(bar(B_DRAIN));
