@@ -122,9 +122,11 @@ enum {
  *                                     R[C] = half_text * 2 (anchor query frames)
  *   read_table_bf16 : [B,H,C+1,2,d_v,d_k] bfloat16 hi/lo split of read_table,
  *                                     R_hi = bf16(R), R_lo = bf16(R - R_hi) (operand of
- *                                     the tensor-core read; written only on that path) */
+ *                                     the tensor-core read; written only on that path)
+ *   text_gram  : [B,H,2,d,d]          A_x, B_x of the text tokens (tensor-core text
+ *                                     path only)                                         */
 typedef struct {
-  size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, read_table_bf16, total;
+  size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, read_table_bf16, text_gram, total;
 } vdn_workspace_layout;
 
 /* Bytes of workspace the configuration needs; 0 if cfg is invalid. */

@@ -52,7 +52,7 @@ def test_workspace_size_and_layout():
     assert lay["frame_C"] - lay["frame_M"] >= 90 * 24 * dd
     assert lay["read_table"] - lay["bwd_snap"] >= 24 * 19 * dd
     offs = [lay[k] for k in ("status", "half_text", "frame_M", "frame_C", "fwd_snap", "bwd_snap", "read_table",
-                             "read_table_bf16", "total")]
+                             "read_table_bf16", "text_gram", "total")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
 
 

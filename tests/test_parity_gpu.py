@@ -129,12 +129,15 @@ def test_bf16_softmax_runs_on_tensor_cores():
 @pytest.mark.parametrize("shape", [Shape(1, 20, 240, 2, 64, 64, 8), Shape(1, 12, 300, 2, 128, 128, 8),
                                    Shape(2, 8, 40, 1, 128, 128, 0)])
 def test_bf16_frame_maps_match_oracle(shape):
-    """M_t and C_t after the tensor-core Gram + SPD solve (bf16 inputs)."""
+    """M_t, C_t and the half-text state after the tensor-core Gram + SPD
+    solve (bf16 inputs)."""
     inp, cfg, ha, _, _ = run(shape, "bf16", 13, drop_text=shape.L == 0)
     it = {k: v.double().cpu().numpy() for k, v in ha.intermediates().items()}
     for b in range(cfg.B):
         for h in range(cfg.H):
             ref = O.vda_intermediates(inp, ocfg(cfg), b, h)
+            sx = np.abs(ref["S_init"]).max() + 1e-30
+            np.testing.assert_allclose(it["half_text"][b, h], ref["S_init"], atol=2e-5 * sx)
             for t in range(1, cfg.T - 1):
                 np.testing.assert_allclose(it["M"][b, t, h], ref["M"][t], atol=2e-5)
                 np.testing.assert_allclose(it["C"][b, t, h], ref["C"][t], atol=2e-5 * np.abs(ref["C"][t]).max())

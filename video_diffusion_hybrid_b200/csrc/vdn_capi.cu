@@ -59,6 +59,7 @@ void layout_of(const vdn_hybrid_cfg* c, vdn_workspace_layout* L) {
   L->bwd_snap = off;   off += up(bh * (C + 1) * dd);
   L->read_table = off; off += up(bh * (C + 1) * dd);
   L->read_table_bf16 = off; off += up(bh * (C + 1) * dd);  // hi and lo bf16 terms
+  L->text_gram = off;  off += up(bh * 2 * dd);
   L->total = off;
 }
 
@@ -96,6 +97,7 @@ Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
   w.bsnap = reinterpret_cast<float*>(base + L.bwd_snap);
   w.R = reinterpret_cast<float*>(base + L.read_table);
   w.R16 = base + L.read_table_bf16;
+  w.text_gram = reinterpret_cast<float*>(base + L.text_gram);
   return w;
 }
 
@@ -134,9 +136,9 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
   if (check_cfg(cfg) != VDN_OK) return -1;
   Dims d = make_dims(cfg);
   switch (stage) {
-    case VDN_STAGE_TEXT:
     case VDN_STAGE_SCAN:
       return 0;
+    case VDN_STAGE_TEXT:
     case VDN_STAGE_SOLVE:
       return gram_tc_supported(d) ? 1 : 0;
     case VDN_STAGE_READ:
@@ -161,7 +163,12 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
   cudaError_t e = cudaSuccess;
   if (cudaMemsetAsync(w.status, 0, 256, s) != cudaSuccess) return VDN_ERR_CUDA;
   if (stages & VDN_STAGE_TEXT) {
-    if ((e = launch_text(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+    if (d.L > 0 && gram_tc_supported(d)) {
+      if ((e = launch_text_gram_tc(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+      if ((e = launch_text_solve_sweep(d, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+    } else if ((e = launch_text(d, in, w, s)) != cudaSuccess) {
+      return VDN_ERR_CUDA;
+    }
   }
   if (stages & VDN_STAGE_SOLVE) {
     if (gram_tc_supported(d)) {

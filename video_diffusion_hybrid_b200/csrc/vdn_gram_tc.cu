@@ -32,7 +32,9 @@ using namespace tc;
 constexpr int TT = 128;  // tokens per tile
 constexpr int kThreadsG = 256;
 
-template <int D>
+// TEXT: the L text tokens of (b, h) instead of one frame; A_x, B_x go to the
+// text_gram region of the workspace.
+template <int D, bool TEXT>
 __global__ void __launch_bounds__(kThreadsG, 1)
 k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
           const __grid_constant__ CUtensorMap tmv) {
@@ -53,11 +55,17 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  if (is_anchor(dm, t)) return;
+  if (!TEXT && is_anchor(dm, t)) return;
   if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
-  const int ntiles = (dm.N + TT - 1) / TT;
-  const long long tok0 = ((long long)b * dm.T + t) * dm.N;  // first token of the frame
-  const long long fh = ((long long)b * dm.T + t) * dm.H + h;
+  const int ntok = TEXT ? dm.L : dm.N;
+  const int ntiles = (ntok + TT - 1) / TT;
+  // first token of the frame (or of batch b's text)
+  const long long tok0 = TEXT ? (long long)b * dm.L : ((long long)b * dm.T + t) * dm.N;
+  const float* betap = TEXT ? in.text_beta : in.beta;
+  const long long DDg = (long long)D * D;
+  float* outA = TEXT ? w.text_gram + ((long long)b * dm.H + h) * 2 * DDg
+                     : w.M + (((long long)b * dm.T + t) * dm.H + h) * DDg;
+  float* outB = TEXT ? outA + DDg : w.Cm + (((long long)b * dm.T + t) * dm.H + h) * DDg;
   const Ctl ctl{abort_flag, w.status, (unsigned)TAG_GRAM_TC};
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
@@ -131,7 +139,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       if (!mbar_wait(bar(B_KVFULL + s), (j / ST) & 1, ctl)) { ok = false; break; }
       if (j > 0 && !mbar_wait(bar(B_KBEMPTY), (j - 1) & 1, ctl)) { ok = false; break; }
       const int tk = j * TT + row;
-      const float beta = tk < dm.N ? __ldg(in.beta + (tok0 + tk) * dm.H + h) : 0.f;
+      const float beta = tk < ntok ? __ldg(betap + (tok0 + tk) * dm.H + h) : 0.f;
 #pragma unroll
       for (int c = 0; c < NB; ++c) {
 #pragma unroll
@@ -158,10 +166,9 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
     if (__all_sync(0xffffffffu, ok && mbar_wait(bar(B_ACC), 0, ctl))) {
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-      const long long DD = (long long)D * D;
       if (D == 128) {
-        float* Ag = w.M + fh * DD + (long long)row * D;
-        float* Bg = w.Cm + fh * DD + (long long)row * D;
+        float* Ag = outA + (long long)row * D;
+        float* Bg = outB + (long long)row * D;
 #pragma unroll
         for (int q = 0; q < 2 * D / 32; ++q) {
           float v[32];
@@ -173,7 +180,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
         }
       } else {
         // lanes 0..63 hold A rows, lanes 64..127 hold B rows
-        float* dst0 = row < D ? w.M + fh * DD + (long long)row * D : w.Cm + fh * DD + (long long)(row - D) * D;
+        float* dst0 = row < D ? outA + (long long)row * D : outB + (long long)(row - D) * D;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
           float v[32];
@@ -193,17 +200,18 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
   if (warp == 1) tmem_free(tmem, kCols);
 }
 
-template <int D>
+template <int D, bool TEXT>
 cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   CUtensorMap mk, mv;
-  const long long tokens = (long long)d.B * d.T * d.N;
-  if (!make_token_map(&mk, in.k, tokens, d.H, D, TT) || !make_token_map(&mv, in.v, tokens, d.H, D, TT))
+  const long long tokens = TEXT ? (long long)d.B * d.L : (long long)d.B * d.T * d.N;
+  if (!make_token_map(&mk, TEXT ? in.text_k : in.k, tokens, d.H, D, TT) ||
+      !make_token_map(&mv, TEXT ? in.text_v : in.v, tokens, d.H, D, TT))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 2 * (2 * (size_t)TT * D * 2) + 2 * (size_t)TT * D * 2 + 8 * 8 + 16;
-  auto kern = k_gram_tc<D>;
+  auto kern = k_gram_tc<D, TEXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(d.T, d.H, d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
+  kern<<<dim3(TEXT ? 1 : d.T, d.H, d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
   return cudaGetLastError();
 }
 
@@ -216,8 +224,15 @@ bool gram_tc_supported(const Dims& d) {
 }
 
 cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
-  if (d.dk == 128) return launch<128>(d, in, w, s);
-  if (d.dk == 64) return launch<64>(d, in, w, s);
+  if (d.dk == 128) return launch<128, false>(d, in, w, s);
+  if (d.dk == 64) return launch<64, false>(d, in, w, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_text_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  if (d.L <= 0 || (long long)d.B * d.L >= (1LL << 31)) return cudaErrorInvalidValue;
+  if (d.dk == 128) return launch<128, true>(d, in, w, s);
+  if (d.dk == 64) return launch<64, true>(d, in, w, s);
   return cudaErrorInvalidValue;
 }
 

@@ -29,7 +29,8 @@ struct Work {
   float* fsnap;      // [B,H,C+1,dv,dk]
   float* bsnap;      // [B,H,C+1,dv,dk]
   float* R;          // [B,H,C+1,dv,dk]
-  void* R16;         // [B,H,C+1,dv,dk] bf16
+  void* R16;         // [B,H,C+1,2,dv,dk] bf16 (hi, lo)
+  float* text_gram;  // [B,H,2,dk,dk] A_x, B_x
 };
 
 struct Inputs {
@@ -49,6 +50,8 @@ __host__ __device__ inline bool is_anchor(const Dims& d, int t) {
 cudaError_t launch_text(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_solve_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_solve_inplace(const Dims& d, const Work& w, cudaStream_t s);
+cudaError_t launch_text_solve_sweep(const Dims& d, const Work& w, cudaStream_t s);
+cudaError_t launch_text_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 bool gram_tc_supported(const Dims& d);
 cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);

@@ -262,57 +262,116 @@ __global__ void k_half_init(Dims dm, const float* __restrict__ init, float* __re
 // ---------------------------------------------------------------------------
 // State scan.  grid (D/RB row blocks, 2 directions, B*H).  Rows of the state
 // evolve independently (s_row <- alpha s_row M + c_row), so each CTA carries
-// RB rows of one chain and reads the whole M_t.
+// RB rows of one chain and reads the whole M_t.  Thread tile: 4 rows x CPT
+// columns of the new state, from S^T (rows contiguous, one 16-byte load per
+// k) and M (CPT contiguous columns per k).  The next frame's M, C rows and
+// alpha are loaded into registers while the current frame computes.
 // ---------------------------------------------------------------------------
 template <int D, int RB>
 __global__ void __launch_bounds__(kThreads)
 k_scan(Dims dm, Inputs in, Work w) {
-  constexpr int ROWS_PT = RB * D / kThreads;  // rows per thread
-  constexpr int GROUPS = kThreads / D;        // row groups
+  constexpr int RG = RB / 4;               // row groups of 4
+  constexpr int CG = kThreads / RG;        // column groups
+  constexpr int CPT = D / CG;              // columns per thread
+  constexpr int NV4 = D * D / 4 / kThreads;
+  static_assert(CPT >= 1 && CG * CPT == D, "scan tiling");
   extern __shared__ float sm[];
   float* Ms = sm;          // [D][D]
-  float* S = sm + D * D;   // [RB][D]
-  const int tid = threadIdx.x, j = tid % D, rg = tid / D;
+  float* St = sm + D * D;  // [D][RB]  (S transposed)
+  const int tid = threadIdx.x, cq = tid % CG, rq = tid / CG;
+  const int c0 = cq * CPT, r0 = rq * 4;
   const int row0 = blockIdx.x * RB, dir = blockIdx.y, bh = blockIdx.z;
   const int b = bh / dm.H, h = bh % dm.H;
   const long long DD = (long long)D * D;
   const float* half = w.half_text + (long long)bh * DD;
   float* snap = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD;
+  auto frame = [&](int st) { return dir == 0 ? st : dm.T - 1 - st; };
+  auto gidx = [&](int r, int c) { return (long long)(row0 + r0 + r) * D + c0 + c; };
 
-  float cur[ROWS_PT];
+  float cur[4][CPT];
 #pragma unroll
-  for (int x = 0; x < ROWS_PT; ++x) {
-    int r = rg + GROUPS * x;
-    cur[x] = half[(long long)(row0 + r) * D + j];
-    S[r * D + j] = cur[x];
-    snap[(dir == 0 ? 0 : (long long)dm.C * DD) + (long long)(row0 + r) * D + j] = cur[x];
-  }
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      cur[r][c] = half[gidx(r, c)];
+      snap[(dir == 0 ? 0 : (long long)dm.C * DD) + gidx(r, c)] = cur[r][c];
+    }
+#pragma unroll
+  for (int c = 0; c < CPT; ++c)
+    *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0) = make_float4(cur[0][c], cur[1][c], cur[2][c], cur[3][c]);
+
+  float4 mreg[NV4];
+  float creg[4][CPT];
+  float areg = 0.f;
+  auto prefetch = [&](int st) {
+    const int t = frame(st);
+    const long long fh = ((long long)b * dm.T + t) * dm.H + h;
+    const float4* Mg = reinterpret_cast<const float4*>(w.M + fh * DD);
+#pragma unroll
+    for (int v = 0; v < NV4; ++v) mreg[v] = __ldg(Mg + tid + v * kThreads);
+    const float* Cg = w.Cm + fh * DD;
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) creg[r][c] = __ldg(Cg + gidx(r, c));
+    areg = __ldg(in.alpha + fh);
+  };
+  auto next_write = [&](int st) {  // first step >= st whose frame is written
+    while (st < dm.T && is_anchor(dm, frame(st))) ++st;
+    return st;
+  };
+  int nxt = next_write(0);
+  if (nxt < dm.T) prefetch(nxt);
   __syncthreads();
 
-  for (int s = 0; s < dm.T; ++s) {
-    const int t = dir == 0 ? s : dm.T - 1 - s;
-    if (!is_anchor(dm, t)) {
-      const long long fh = ((long long)b * dm.T + t) * dm.H + h;
-      const float4* Mg = reinterpret_cast<const float4*>(w.M + fh * DD);
-      for (int idx = tid; idx < D * D / 4; idx += kThreads) reinterpret_cast<float4*>(Ms)[idx] = Mg[idx];
-      const float a = __ldg(in.alpha + fh);
-      const float* Cg = w.Cm + fh * DD;
-      __syncthreads();
-      float acc[ROWS_PT];
+  for (int st = 0; st < dm.T; ++st) {
+    const int t = frame(st);
+    if (st == nxt) {
 #pragma unroll
-      for (int x = 0; x < ROWS_PT; ++x) acc[x] = 0.f;
+      for (int v = 0; v < NV4; ++v) reinterpret_cast<float4*>(Ms)[tid + v * kThreads] = mreg[v];
+      const float a = areg;
+      float cc[4][CPT];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) cc[r][c] = creg[r][c];
+      __syncthreads();
+      nxt = next_write(st + 1);
+      if (nxt < dm.T) prefetch(nxt);  // in flight during this frame's arithmetic
+      float acc[4][CPT];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[r][c] = 0.f;
 #pragma unroll 8
       for (int i = 0; i < D; ++i) {
-        const float m = Ms[i * D + j];
+        const float4 sv = *reinterpret_cast<const float4*>(St + i * RB + r0);
+        float mv[CPT];
+        if (CPT == 2) {
+          const float2 m2 = *reinterpret_cast<const float2*>(Ms + i * D + c0);
+          mv[0] = m2.x;
+          mv[CPT - 1] = m2.y;
+        } else {
 #pragma unroll
-        for (int x = 0; x < ROWS_PT; ++x) acc[x] = fmaf(S[(rg + GROUPS * x) * D + i], m, acc[x]);
+          for (int c = 0; c < CPT; ++c) mv[c] = Ms[i * D + c0 + c];
+        }
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+          acc[0][c] = fmaf(sv.x, mv[c], acc[0][c]);
+          acc[1][c] = fmaf(sv.y, mv[c], acc[1][c]);
+          acc[2][c] = fmaf(sv.z, mv[c], acc[2][c]);
+          acc[3][c] = fmaf(sv.w, mv[c], acc[3][c]);
+        }
       }
 #pragma unroll
-      for (int x = 0; x < ROWS_PT; ++x) cur[x] = fmaf(a, acc[x], Cg[(long long)(row0 + rg + GROUPS * x) * D + j]);
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) cur[r][c] = fmaf(a, acc[r][c], cc[r][c]);
       __syncthreads();
 #pragma unroll
-      for (int x = 0; x < ROWS_PT; ++x) S[(rg + GROUPS * x) * D + j] = cur[x];
-      // the next step's M load is followed by a barrier before S is read
+      for (int c = 0; c < CPT; ++c)
+        *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0) = make_float4(cur[0][c], cur[1][c], cur[2][c], cur[3][c]);
+      // the next written frame's M store is followed by a barrier before S is read
     }
     int snap_idx = -1;
     if (dir == 0) {
@@ -323,8 +382,9 @@ k_scan(Dims dm, Inputs in, Work w) {
     }
     if (snap_idx >= 0) {
 #pragma unroll
-      for (int x = 0; x < ROWS_PT; ++x)
-        snap[(long long)snap_idx * DD + (long long)(row0 + rg + GROUPS * x) * D + j] = cur[x];
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) snap[(long long)snap_idx * DD + gidx(r, c)] = cur[r][c];
     }
   }
 }

@@ -20,7 +20,9 @@ namespace {
 
 constexpr int kThreadsS = 256;
 
-template <int D>
+// TEXT: A_x, B_x from the text_gram region; writes S_x / 2 = B_x M_x / 2 to
+// the half-text state and no M.
+template <int D, bool TEXT>
 __global__ void __launch_bounds__(kThreadsS)
 k_solve_sweep(Dims dm, Work w) {
   constexpr int R = D / 16;   // register tile edge
@@ -30,10 +32,13 @@ k_solve_sweep(Dims dm, Work w) {
   float* Ms = sm + 2 * D;     // [D][P]
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  if (is_anchor(dm, t)) return;
+  if (!TEXT && is_anchor(dm, t)) return;
   const long long fh = ((long long)b * dm.T + t) * dm.H + h;
-  float* gA = w.M + fh * D * D;
-  float* gB = w.Cm + fh * D * D;
+  const long long bh = (long long)b * dm.H + h;
+  float* gA = TEXT ? w.text_gram + bh * 2 * D * D : w.M + fh * D * D;
+  float* gB = TEXT ? gA + D * D : w.Cm + fh * D * D;
+  float* outC = TEXT ? w.half_text + bh * D * D : gB;
+  const float cscale = TEXT ? 0.5f : 1.0f;
 
   float g[R][R];
 #pragma unroll
@@ -67,18 +72,25 @@ k_solve_sweep(Dims dm, Work w) {
     for (int a = 0; a < R; ++a) colv[a] = buf[ty + 16 * a];
 #pragma unroll
     for (int c = 0; c < R; ++c) rowv[c] = buf[tx + 16 * c] * inv;
+    // every element takes the rank-one update ...
 #pragma unroll
-    for (int a = 0; a < R; ++a) {
-      const int i = ty + 16 * a;
+    for (int a = 0; a < R; ++a)
 #pragma unroll
-      for (int c = 0; c < R; ++c) {
-        const int j = tx + 16 * c;
-        float v = fmaf(-colv[a], rowv[c], g[a][c]);
-        if (i == p) v = rowv[c];
-        if (j == p) v = colv[a] * inv;
-        if (i == p && j == p) v = -inv;
-        g[a][c] = v;
-      }
+      for (int c = 0; c < R; ++c) g[a][c] = fmaf(-colv[a], rowv[c], g[a][c]);
+    // ... then the owners of row p and of column p overwrite those (one tile
+    // row / column each, selected by register moves, not dynamic indexing)
+    const int pa = p >> 4;
+    if (ty == (p & 15)) {
+#pragma unroll
+      for (int a = 0; a < R; ++a)
+#pragma unroll
+        for (int c = 0; c < R; ++c) g[a][c] = (a == pa) ? rowv[c] : g[a][c];
+    }
+    if (tx == (p & 15)) {
+#pragma unroll
+      for (int a = 0; a < R; ++a)
+#pragma unroll
+        for (int c = 0; c < R; ++c) g[a][c] = (c == pa) ? ((ty + 16 * a == p) ? -inv : colv[a] * inv) : g[a][c];
     }
   }
 
@@ -89,7 +101,7 @@ k_solve_sweep(Dims dm, Work w) {
     for (int c = 0; c < R; ++c) {
       const int i = ty + 16 * a, j = tx + 16 * c;
       Ms[i * P + j] = -g[a][c];
-      gA[i * D + j] = -g[a][c];
+      if (!TEXT) gA[i * D + j] = -g[a][c];
     }
   __syncthreads();
   float acc[R][R];
@@ -113,16 +125,16 @@ k_solve_sweep(Dims dm, Work w) {
 #pragma unroll
   for (int a = 0; a < R; ++a)
 #pragma unroll
-    for (int c = 0; c < R; ++c) gB[(ty + 16 * a) * D + tx + 16 * c] = acc[a][c];
+    for (int c = 0; c < R; ++c) outC[(ty + 16 * a) * D + tx + 16 * c] = cscale * acc[a][c];
 }
 
-template <int D>
+template <int D, bool TEXT>
 cudaError_t launch(const Dims& d, const Work& w, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)(2 * D + D * (D + 1));
-  auto kern = k_solve_sweep<D>;
+  auto kern = k_solve_sweep<D, TEXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(d.T, d.H, d.B), kThreadsS, smem, s>>>(d, w);
+  kern<<<dim3(TEXT ? 1 : d.T, d.H, d.B), kThreadsS, smem, s>>>(d, w);
   return cudaGetLastError();
 }
 
@@ -130,9 +142,18 @@ cudaError_t launch(const Dims& d, const Work& w, cudaStream_t s) {
 
 cudaError_t launch_solve_inplace(const Dims& d, const Work& w, cudaStream_t s) {
   switch (d.dk) {
-    case 32: return launch<32>(d, w, s);
-    case 64: return launch<64>(d, w, s);
-    case 128: return launch<128>(d, w, s);
+    case 32: return launch<32, false>(d, w, s);
+    case 64: return launch<64, false>(d, w, s);
+    case 128: return launch<128, false>(d, w, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_text_solve_sweep(const Dims& d, const Work& w, cudaStream_t s) {
+  switch (d.dk) {
+    case 32: return launch<32, true>(d, w, s);
+    case 64: return launch<64, true>(d, w, s);
+    case 128: return launch<128, true>(d, w, s);
     default: return cudaErrorInvalidValue;
   }
 }
