@@ -10,9 +10,20 @@
 // needs no pivoting: each pivot is a Schur complement of I + A_t and is >= 1.
 // Sweeping all d pivots turns G = I + A into -G^-1 in d^3 multiply-adds, the
 // same work as Cholesky + triangular inverse + W^T W, in one pass with one
-// barrier per pivot and every thread busy: thread (ty, tx) of a 16 x 16 grid
-// keeps the (d/16) x (d/16) elements G[ty + 16a][tx + 16b] in registers, and
-// the only exchange per pivot is row p (column p equals it by symmetry).
+// barrier per pivot and every thread busy.
+//
+// Thread (ty, tx) of a 16 x 16 grid keeps the R x R block G[ty R + a][tx R + c]
+// (R = d / 16) in registers.  The only exchange per pivot is row p (column p
+// equals it by symmetry), and the pivot loop is unrolled by R so the owner
+// reads its row from a fixed register.  The sweep's special rules for row p,
+// column p and the pivot itself are folded into the one rank-one update by
+// broadcasting g_pp - 1 in place of g_pp:
+//   g_ij - g_ip (g_pj / g_pp)              (i, j != p)  the ordinary update
+//   g_ip - g_ip (g_pp - 1) / g_pp = g_ip / g_pp          column p
+//   g_pj - (g_pp - 1) g_pj / g_pp = g_pj / g_pp          row p
+//   g_pp - (g_pp - 1)^2 / g_pp    = 2 - 1 / g_pp         pivot: the sweep wants
+// -1 / g_pp, and since later pivots only add to this entry the surplus 2 is
+// removed from the whole diagonal once, at the end.
 #include "vdn_internal.h"
 
 namespace vdn {
@@ -20,16 +31,47 @@ namespace {
 
 constexpr int kThreadsS = 256;
 
+template <int R>
+__device__ __forceinline__ void ld_row(float (&dst)[R], const float* src) {
+  if constexpr (R % 4 == 0) {
+#pragma unroll
+    for (int c = 0; c < R; c += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(src + c);
+      dst[c] = v.x; dst[c + 1] = v.y; dst[c + 2] = v.z; dst[c + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < R; c += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(src + c);
+      dst[c] = v.x; dst[c + 1] = v.y;
+    }
+  }
+}
+
+template <int R>
+__device__ __forceinline__ void st_row(float* dst, const float (&src)[R], float sgn) {
+  if constexpr (R % 4 == 0) {
+#pragma unroll
+    for (int c = 0; c < R; c += 4)
+      *reinterpret_cast<float4*>(dst + c) = make_float4(sgn * src[c], sgn * src[c + 1], sgn * src[c + 2], sgn * src[c + 3]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < R; c += 2) *reinterpret_cast<float2*>(dst + c) = make_float2(sgn * src[c], sgn * src[c + 1]);
+  }
+}
+
 // TEXT: A_x, B_x from the text_gram region; writes S_x / 2 = B_x M_x / 2 to
 // the half-text state and no M.
 template <int D, bool TEXT>
-__global__ void __launch_bounds__(kThreadsS)
+__global__ void __launch_bounds__(kThreadsS, 2)
 k_solve_sweep(Dims dm, Work w) {
   constexpr int R = D / 16;   // register tile edge
-  constexpr int P = D + 1;    // shared pitch
+  constexpr int P = D + 4;    // shared pitch (16-byte rows)
+  constexpr int BP = D + 4;   // pivot buffer: row p, then 1 / g_pp at [D]
+  static_assert(R % 2 == 0, "pivot buffers alternate with the parity of p");
   extern __shared__ float sm[];
-  float* rowbuf = sm;         // [2][D]  pivot row, double-buffered
-  float* Ms = sm + 2 * D;     // [D][P]
+  float* rowbuf = sm;         // [2][BP]
+  float* Ms = sm + 2 * BP;    // [D][P]
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (!TEXT && is_anchor(dm, t)) return;
@@ -39,98 +81,84 @@ k_solve_sweep(Dims dm, Work w) {
   float* gB = TEXT ? gA + D * D : w.Cm + fh * D * D;
   float* outC = TEXT ? w.half_text + bh * D * D : gB;
   const float cscale = TEXT ? 0.5f : 1.0f;
+  const int r0 = ty * R, c0 = tx * R;
 
   float g[R][R];
 #pragma unroll
-  for (int a = 0; a < R; ++a)
-#pragma unroll
-    for (int c = 0; c < R; ++c) {
-      const int i = ty + 16 * a, j = tx + 16 * c;
-      g[a][c] = gA[i * D + j] + (i == j ? 1.0f : 0.0f);
-    }
+  for (int a = 0; a < R; ++a) {
+    ld_row<R>(g[a], gA + (r0 + a) * D + c0);
+    if (ty == tx) g[a][a] += 1.0f;
+  }
 
-  for (int p = 0; p < D; ++p) {
-    float* buf = rowbuf + (p & 1) * D;
-    if (ty == (p & 15)) {
-      // row p lives in tile row p / 16 of these threads; select it with
-      // register moves (no dynamic indexing of g, which would spill it)
-      const int pa = p >> 4;
-      float rsel[R];
+  for (int pb = 0; pb < 16; ++pb) {
 #pragma unroll
-      for (int cc = 0; cc < R; ++cc) rsel[cc] = g[0][cc];
+    for (int a = 0; a < R; ++a) {
+      float* buf = rowbuf + (a & 1) * BP;
+      if (ty == pb) {
+        float v[R];
 #pragma unroll
-      for (int a = 1; a < R; ++a)
+        for (int c = 0; c < R; ++c) v[c] = g[a][c];
+        if (tx == pb) {
+          buf[D] = 1.0f / v[a];
+          v[a] -= 1.0f;
+        }
+        st_row<R>(buf + c0, v, 1.0f);
+      }
+      __syncthreads();  // also orders the reads of this buffer two pivots ago
+      const float inv = buf[D];
+      float colv[R], rowv[R];
+      ld_row<R>(colv, buf + r0);
+      ld_row<R>(rowv, buf + c0);
 #pragma unroll
-        for (int cc = 0; cc < R; ++cc) rsel[cc] = (a == pa) ? g[a][cc] : rsel[cc];
+      for (int c = 0; c < R; ++c) rowv[c] *= inv;
 #pragma unroll
-      for (int cc = 0; cc < R; ++cc) buf[tx + 16 * cc] = rsel[cc];
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int c = 0; c < R; ++c) g[i][c] = fmaf(-colv[i], rowv[c], g[i][c]);
     }
-    __syncthreads();  // also orders the previous reads of this buffer (two pivots ago)
-    const float inv = 1.0f / buf[p];
-    float colv[R], rowv[R];
+  }
+  if (ty == tx) {
 #pragma unroll
-    for (int a = 0; a < R; ++a) colv[a] = buf[ty + 16 * a];
-#pragma unroll
-    for (int c = 0; c < R; ++c) rowv[c] = buf[tx + 16 * c] * inv;
-    // every element takes the rank-one update ...
-#pragma unroll
-    for (int a = 0; a < R; ++a)
-#pragma unroll
-      for (int c = 0; c < R; ++c) g[a][c] = fmaf(-colv[a], rowv[c], g[a][c]);
-    // ... then the owners of row p and of column p overwrite those (one tile
-    // row / column each, selected by register moves, not dynamic indexing)
-    const int pa = p >> 4;
-    if (ty == (p & 15)) {
-#pragma unroll
-      for (int a = 0; a < R; ++a)
-#pragma unroll
-        for (int c = 0; c < R; ++c) g[a][c] = (a == pa) ? rowv[c] : g[a][c];
-    }
-    if (tx == (p & 15)) {
-#pragma unroll
-      for (int a = 0; a < R; ++a)
-#pragma unroll
-        for (int c = 0; c < R; ++c) g[a][c] = (c == pa) ? ((ty + 16 * a == p) ? -inv : colv[a] * inv) : g[a][c];
-    }
+    for (int a = 0; a < R; ++a) g[a][a] -= 2.0f;
   }
 
   // M = -G_swept: to global and to shared for C = B M
 #pragma unroll
-  for (int a = 0; a < R; ++a)
-#pragma unroll
-    for (int c = 0; c < R; ++c) {
-      const int i = ty + 16 * a, j = tx + 16 * c;
-      Ms[i * P + j] = -g[a][c];
-      if (!TEXT) gA[i * D + j] = -g[a][c];
-    }
+  for (int a = 0; a < R; ++a) {
+    st_row<R>(Ms + (r0 + a) * P + c0, g[a], -1.0f);
+    if (!TEXT) st_row<R>(gA + (r0 + a) * D + c0, g[a], -1.0f);
+  }
   __syncthreads();
   float acc[R][R];
 #pragma unroll
   for (int a = 0; a < R; ++a)
 #pragma unroll
     for (int c = 0; c < R; ++c) acc[a][c] = 0.f;
-#pragma unroll 4
-  for (int k = 0; k < D; ++k) {
-    float bv[R], mv[R];
+#pragma unroll 1
+  for (int k = 0; k < D; k += 4) {
+    float4 bv[R];
 #pragma unroll
-    for (int a = 0; a < R; ++a) bv[a] = gB[(ty + 16 * a) * D + k];  // B read from global (L1)
+    for (int a = 0; a < R; ++a) bv[a] = *reinterpret_cast<const float4*>(gB + (r0 + a) * D + k);
 #pragma unroll
-    for (int c = 0; c < R; ++c) mv[c] = Ms[k * P + tx + 16 * c];
+    for (int kk = 0; kk < 4; ++kk) {
+      float mv[R];
+      ld_row<R>(mv, Ms + (k + kk) * P + c0);
 #pragma unroll
-    for (int a = 0; a < R; ++a)
+      for (int a = 0; a < R; ++a) {
+        const float bb = kk == 0 ? bv[a].x : kk == 1 ? bv[a].y : kk == 2 ? bv[a].z : bv[a].w;
 #pragma unroll
-      for (int c = 0; c < R; ++c) acc[a][c] = fmaf(bv[a], mv[c], acc[a][c]);
+        for (int c = 0; c < R; ++c) acc[a][c] = fmaf(bb, mv[c], acc[a][c]);
+      }
+    }
   }
   __syncthreads();  // every read of B done before C overwrites it in place
 #pragma unroll
-  for (int a = 0; a < R; ++a)
-#pragma unroll
-    for (int c = 0; c < R; ++c) outC[(ty + 16 * a) * D + tx + 16 * c] = cscale * acc[a][c];
+  for (int a = 0; a < R; ++a) st_row<R>(outC + (r0 + a) * D + c0, acc[a], cscale);
 }
 
 template <int D, bool TEXT>
 cudaError_t launch(const Dims& d, const Work& w, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (size_t)(2 * D + D * (D + 1));
+  const size_t smem = sizeof(float) * (size_t)(2 * (D + 4) + D * (D + 4));
   auto kern = k_solve_sweep<D, TEXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
