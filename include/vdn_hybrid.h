@@ -94,7 +94,10 @@ typedef struct {
                                       text solve (each direction starts from S_x / 2);
                                       only allowed with L == 0; NULL = zero state          */
   const float *rms_weight;         /* [H,d_v] RMSNorm weight, NULL = ones                 */
-  void *y;                         /* output, cfg.y_dtype, shape per cfg.out_mode         */
+  void *y;                         /* output, cfg.y_dtype, shape per cfg.out_mode; every
+                                      array pointer is 16-byte aligned, and a 32-byte
+                                      aligned y lets the state read use its tensor-core
+                                      kernel (same results either way)                    */
   void *workspace;                 /* device scratch, 256-byte aligned                   */
   size_t workspace_bytes;
 } vdn_hybrid_args;

@@ -186,7 +186,9 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
   if (stages & VDN_STAGE_READ) {
-    e = read_tc_supported(d) ? launch_read_tc(d, in, w, w.R16, s) : launch_read_simt(d, in, w, s);
+    // the tensor-core read writes y rows with 32-byte stores
+    e = (read_tc_supported(d) && aligned(in.y, 32)) ? launch_read_tc(d, in, w, w.R16, s)
+                                                    : launch_read_simt(d, in, w, s);
     if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
   return VDN_OK;

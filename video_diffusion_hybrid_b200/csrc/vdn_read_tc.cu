@@ -20,8 +20,10 @@
 //   warp 1      TMEM allocator; lane 0 issues O_t = Q_t R_hi^T + Q_t R_lo^T
 //               (M=128 tokens, N=d_v, K=d_k, both operands K-major in SMEM)
 //               into one of two TMEM accumulators.
-//   warps 4..7  epilogue, one token per thread (= TMEM lane): sum of squares
-//               over d_v, rsqrt, gate from the SMEM tile, store y.
+//   warps 4..11 epilogue, one token per thread (= TMEM lane) and half of d_v
+//               per warp (warps w and w + 4 share the TMEM lanes of one
+//               32-token quarter): sum of squares over all of d_v, rsqrt,
+//               gate from the SMEM tile, one 32-byte store per 8 outputs.
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -30,7 +32,7 @@ using namespace tc;
 
 constexpr int TQ = 128;          // tokens per tile
 constexpr int kTilesPerCta = 8;  // tiles of one query group handled by a CTA
-constexpr int kThreadsR = 256;
+constexpr int kThreadsR = 384;
 
 // ------------------------------------------------------------ read table --
 __global__ void k_read_table(Dims dm, Work w, __nv_bfloat16* __restrict__ r16) {
@@ -112,26 +114,42 @@ __device__ bool decode_run(const Dims& d, long long item, Run& r) {
   return false;
 }
 
-template <typename To> __device__ __forceinline__ void put4(To* p, float a, float b, float c, float d, bool add);
-template <> __device__ __forceinline__ void put4<float>(float* p, float a, float b, float c, float d, bool add) {
-  float4 v = make_float4(a, b, c, d);
+// y[0..8) (+)= v: fp32 rows go out as one 256-bit store (32-byte aligned),
+// bf16 rows as one 128-bit store.
+template <typename To> __device__ __forceinline__ void put8(To* p, float (&v)[8], bool add);
+template <> __device__ __forceinline__ void put8<float>(float* p, float (&v)[8], bool add) {
   if (add) {
-    const float4 o = *reinterpret_cast<const float4*>(p);
-    v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+    float o[8];
+    asm volatile("ld.global.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(o[0]), "=f"(o[1]), "=f"(o[2]), "=f"(o[3]), "=f"(o[4]), "=f"(o[5]), "=f"(o[6]), "=f"(o[7])
+                 : "l"(p));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] += o[i];
   }
-  *reinterpret_cast<float4*>(p) = v;
+  asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+               "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
 }
-template <> __device__ __forceinline__ void put4<__nv_bfloat16>(__nv_bfloat16* p, float a, float b, float c, float d,
-                                                                 bool add) {
+template <> __device__ __forceinline__ void put8<__nv_bfloat16>(__nv_bfloat16* p, float (&v)[8], bool add) {
   if (add) {
-    const uint2 o = *reinterpret_cast<const uint2*>(p);
-    a += __uint_as_float(o.x << 16); b += __uint_as_float(o.x & 0xFFFF0000u);
-    c += __uint_as_float(o.y << 16); d += __uint_as_float(o.y & 0xFFFF0000u);
+    const uint4 o = *reinterpret_cast<const uint4*>(p);
+    const uint32_t u[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] += __uint_as_float(u[e] << 16);
+      v[2 * e + 1] += __uint_as_float(u[e] & 0xFFFF0000u);
+    }
   }
-  uint2 u;
-  u.x = pack_bf16(a, b);
-  u.y = pack_bf16(c, d);
-  *reinterpret_cast<uint2*>(p) = u;
+  *reinterpret_cast<uint4*>(p) =
+      make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+}
+
+// sigmoid from the exponential and an approximate reciprocal (both a few ulp;
+// exp(-g) overflowing to inf gives 0, the limit)
+__device__ __forceinline__ float sigmoid_fast(float g) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + __expf(-g)));
+  return r;
 }
 
 // ------------------------------------------------------------------ kernel --
@@ -144,6 +162,7 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
   constexpr uint32_t TBYTES = TQ * D * 2;  // one Q or gate tile
   constexpr int ST = 2;
   constexpr uint32_t kCols = 2 * D <= 128 ? 128 : 256;
+  constexpr int HD = D / 2;  // columns per epilogue warp
   enum { B_R = 0, B_QFULL = 1, B_QEMPTY = 3, B_GFULL = 5, B_GEMPTY = 7, B_AFULL = 9, B_AEMPTY = 11, B_DRAIN = 13,
          NBARS = 14 };
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -154,6 +173,7 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
   uint64_t* bars = reinterpret_cast<uint64_t*>(sG + ST * TBYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sW = reinterpret_cast<float*>(tmem_slot + 4);  // [D] RMSNorm weight (ones if none)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
@@ -164,11 +184,13 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_GEMPTY || i == B_GEMPTY + 1 || i == B_AEMPTY ||
-                                                     i == B_AEMPTY + 1) ? 128 : 1);
+                                                     i == B_AEMPTY + 1) ? 256 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kCols);
+  for (int i = threadIdx.x; i < D; i += blockDim.x)
+    sW[i] = in.rms_weight ? in.rms_weight[(long long)run.h * D + i] : 1.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -229,57 +251,60 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
       mbar_wait(bar(B_DRAIN), 0, ctl);
     }
   } else if (warp >= 4) {
-    const int quad = warp - 4;
+    const int quad = warp & 3, half = (warp - 4) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const float* wgt = in.rms_weight ? in.rms_weight + (long long)run.h * D : nullptr;
+    const bool add = dm.out_mode != 0;
     for (int t = 0; t < run.ntiles; ++t) {
       const int s = t % ST;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + s), (t / ST) & 1, ctl))) break;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_GFULL + s), (t / ST) & 1, ctl))) break;
       tc_fence_after();
-      float o[D];
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        float v[32];
-        tmem_ld32(lane_addr + s * D + q * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[q * 32 + i] = v[i];
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_AEMPTY + s));  // accumulator free for tile t + ST
+      // own half of the row into o, the other half only for the sum of squares
+      float o[HD];
       float ss[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) ss[u] = 0.f;
 #pragma unroll
-      for (int i = 0; i < D; ++i) ss[i & 7] = fmaf(o[i], o[i], ss[i & 7]);
+      for (int q = 0; q < HD / 32; ++q) tmem_ld32(lane_addr + s * D + half * HD + q * 32, *reinterpret_cast<float(*)[32]>(o + q * 32));
+#pragma unroll
+      for (int q = 0; q < HD / 32; ++q) {
+        float v[32];
+        tmem_ld32(lane_addr + s * D + (1 - half) * HD + q * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss[i & 7] = fmaf(v[i], v[i], ss[i & 7]);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_AEMPTY + s));  // accumulator free for tile t + ST
+#pragma unroll
+      for (int i = 0; i < HD; ++i) ss[i & 7] = fmaf(o[i], o[i], ss[i & 7]);
       const float rs =
           rsqrtf((((ss[0] + ss[1]) + (ss[2] + ss[3])) + ((ss[4] + ss[5]) + (ss[6] + ss[7]))) / D + dm.eps);
       const int rows_valid = min(TQ, run.rows_left - t * TQ);
       const bool valid = row < rows_valid;
       const long long tok = run.tok0 + (long long)t * TQ + row;
       const long long gi = (tok * dm.H + run.h) * D;
-      To* y = static_cast<To*>(in.y) + (dm.out_mode == 0 ? 2 * gi + D : gi);
+      To* y = static_cast<To*>(in.y) + (dm.out_mode == 0 ? 2 * gi + D : gi) + half * HD;
       const unsigned char* grow = sG + s * TBYTES + row * 128;
 #pragma unroll
-      for (int ch = 0; ch < D / 8; ++ch) {
-        // 8 gate values of this row from the 128B-swizzled tile
-        const uint4 raw = *reinterpret_cast<const uint4*>(grow + (ch >> 3) * (TQ * 128) + (((ch & 7) ^ (row & 7)) << 4));
+      for (int ch = 0; ch < HD / 8; ++ch) {
+        const int col0 = half * HD + ch * 8;
+        // 8 gate values of this row from the 128B-swizzled tile (64 columns per slab)
+        const uint4 raw =
+            *reinterpret_cast<const uint4*>(grow + (col0 >> 6) * (TQ * 128) + ((((col0 & 63) >> 3) ^ (row & 7)) << 4));
+        const float4 w0 = *reinterpret_cast<const float4*>(sW + col0);
+        const float4 w1 = *reinterpret_cast<const float4*>(sW + col0 + 4);
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
         float yv[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float g0 = __uint_as_float(u[e] << 16), g1 = __uint_as_float(u[e] & 0xFFFF0000u);
-          const int i0 = ch * 8 + 2 * e;
-          const float w0 = wgt ? __ldg(wgt + i0) : 1.f, w1 = wgt ? __ldg(wgt + i0 + 1) : 1.f;
-          yv[2 * e] = o[i0] * rs * w0 / (1.0f + __expf(-g0));
-          yv[2 * e + 1] = o[i0 + 1] * rs * w1 / (1.0f + __expf(-g1));
+          yv[2 * e] = o[ch * 8 + 2 * e] * rs * wv[2 * e] * sigmoid_fast(g0);
+          yv[2 * e + 1] = o[ch * 8 + 2 * e + 1] * rs * wv[2 * e + 1] * sigmoid_fast(g1);
         }
-        if (valid) {
-          put4<To>(y + ch * 8, yv[0], yv[1], yv[2], yv[3], dm.out_mode != 0);
-          put4<To>(y + ch * 8 + 4, yv[4], yv[5], yv[6], yv[7], dm.out_mode != 0);
-        }
+        if (valid) put8<To>(y + ch * 8, yv, add);
       }
       mbar_arrive(bar(B_GEMPTY + s));  // gate tile free
     }
@@ -322,7 +347,7 @@ cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, __nv_bfloat16
   if (!make_token_map(&mq, in.q, tokens, d.H, D, TQ) || !make_token_map(&mg, in.gate_lin, tokens, d.H, D, TQ) ||
       !make_matrix_map(&mr, r16, (long long)d.B * d.H * (d.C + 1) * 2 * D, D, D))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + 2 * (size_t)D * D * 2 + 4 * (size_t)TQ * D * 2 + 14 * 8 + 16;
+  const size_t smem = 1024 + 2 * (size_t)D * D * 2 + 4 * (size_t)TQ * D * 2 + 14 * 8 + 16 + D * 4;
   auto kern = k_read_tc<D, To>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
