@@ -127,9 +127,13 @@ enum {
  *                                     R_hi = bf16(R), R_lo = bf16(R - R_hi) (operand of
  *                                     the tensor-core read; written only on that path)
  *   text_gram  : [B,H,2,d,d]          A_x, B_x of the text tokens (tensor-core text
- *                                     path only)                                         */
+ *                                     path only)
+ *   frame_M16  : [B,T,H,2,d,d]        bfloat16 hi/lo split of frame_M, the operand of the
+ *                                     tensor-core scan (bf16 inputs with d = 128 only;
+ *                                     an empty region otherwise)                         */
 typedef struct {
-  size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, read_table_bf16, text_gram, total;
+  size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, read_table_bf16, text_gram, frame_M16,
+      total;
 } vdn_workspace_layout;
 
 /* Bytes of workspace the configuration needs; 0 if cfg is invalid. */

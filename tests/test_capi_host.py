@@ -51,8 +51,10 @@ def test_workspace_size_and_layout():
     dd = 128 * 128 * 4
     assert lay["frame_C"] - lay["frame_M"] >= 90 * 24 * dd
     assert lay["read_table"] - lay["bwd_snap"] >= 24 * 19 * dd
+    if cfg.dtype == L.VDN_BF16 and cfg.d_k == 128:  # bf16 hi/lo of every frame's M
+        assert lay["total"] - lay["frame_M16"] >= 90 * 24 * dd
     offs = [lay[k] for k in ("status", "half_text", "frame_M", "frame_C", "fwd_snap", "bwd_snap", "read_table",
-                             "read_table_bf16", "text_gram", "total")]
+                             "read_table_bf16", "text_gram", "frame_M16", "total")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
 
 

@@ -124,6 +124,9 @@ def test_bf16_softmax_runs_on_tensor_cores():
         assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, d, d, 0), "bf16"), L.STAGE_READ) == 1
         assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, d, d, 0), "bf16"), L.STAGE_SOLVE) == 1
     assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 64, 64, 0), "f32"), L.STAGE_READ) == 0
+    assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 128, 128, 0), "bf16"), L.STAGE_SCAN) == 1
+    assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 64, 64, 0), "bf16"), L.STAGE_SCAN) == 0
+    assert L.vdn_hybrid_stage_impl(cfg_for(Shape(1, 10, 16, 2, 128, 128, 0), "f32"), L.STAGE_SCAN) == 0
 
 
 @pytest.mark.parametrize("shape", [Shape(1, 20, 240, 2, 64, 64, 8), Shape(1, 12, 300, 2, 128, 128, 8),

@@ -43,7 +43,8 @@ class VdnArgs(C.Structure):
 
 class VdnLayout(C.Structure):
     _fields_ = [(n, C.c_size_t) for n in ("status", "half_text", "frame_M", "frame_C", "fwd_snap",
-                                          "bwd_snap", "read_table", "read_table_bf16", "text_gram", "total")]
+                                          "bwd_snap", "read_table", "read_table_bf16", "text_gram", "frame_M16",
+                                          "total")]
 
 
 @dataclass

@@ -60,6 +60,9 @@ void layout_of(const vdn_hybrid_cfg* c, vdn_workspace_layout* L) {
   L->read_table = off; off += up(bh * (C + 1) * dd);
   L->read_table_bf16 = off; off += up(bh * (C + 1) * dd);  // hi and lo bf16 terms
   L->text_gram = off;  off += up(bh * 2 * dd);
+  L->frame_M16 = off;
+  if (scan_tc_layout(c->dtype == VDN_BF16, c->d_k, c->d_v))
+    off += up(bh * (size_t)c->T * 2 * (size_t)c->d_k * c->d_k * sizeof(__nv_bfloat16));
   L->total = off;
 }
 
@@ -98,6 +101,7 @@ Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
   w.R = reinterpret_cast<float*>(base + L.read_table);
   w.R16 = base + L.read_table_bf16;
   w.text_gram = reinterpret_cast<float*>(base + L.text_gram);
+  w.M16 = L.total > L.frame_M16 ? base + L.frame_M16 : nullptr;
   return w;
 }
 
@@ -137,7 +141,7 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
   Dims d = make_dims(cfg);
   switch (stage) {
     case VDN_STAGE_SCAN:
-      return 0;
+      return scan_tc_supported(d) ? 1 : 0;
     case VDN_STAGE_TEXT:
     case VDN_STAGE_SOLVE:
       return gram_tc_supported(d) ? 1 : 0;
@@ -179,7 +183,9 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     }
   }
   if (stages & VDN_STAGE_SCAN) {
-    if ((e = launch_scan_simt(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+    // the tensor-core scan reads the bf16 split of M that the sweep solve writes
+    e = (scan_tc_supported(d) && w.M16 != nullptr) ? launch_scan_tc(d, in, w, s) : launch_scan_simt(d, in, w, s);
+    if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
   if (stages & VDN_STAGE_SOFTMAX) {
     e = softmax_tc_supported(d) ? launch_softmax_tc(d, in, w, s) : launch_softmax_simt(d, in, w, s);

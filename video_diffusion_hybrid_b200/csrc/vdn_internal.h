@@ -19,7 +19,7 @@ struct Dims {
 };
 
 // Device-side status words at the head of the workspace.
-enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3 };
+enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4 };
 
 struct Work {
   uint32_t* status;
@@ -31,6 +31,7 @@ struct Work {
   float* R;          // [B,H,C+1,dv,dk]
   void* R16;         // [B,H,C+1,2,dv,dk] bf16 (hi, lo)
   float* text_gram;  // [B,H,2,dk,dk] A_x, B_x
+  void* M16;         // [B,T,H,2,dk,dk] bf16 (hi, lo) of M; nullptr off the tensor-core scan
 };
 
 struct Inputs {
@@ -60,6 +61,10 @@ cudaError_t launch_softmax_simt(const Dims& d, const Inputs& in, const Work& w, 
 bool softmax_tc_supported(const Dims& d);
 cudaError_t launch_softmax_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 bool read_tc_supported(const Dims& d);
+// the workspace holds the bf16 split of M (and the solve writes it) exactly when this holds
+__host__ __device__ inline bool scan_tc_layout(bool bf16, int dk, int dv) { return bf16 && dk == 128 && dv == 128; }
+bool scan_tc_supported(const Dims& d);
+cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void* r16, cudaStream_t s);
 
 }  // namespace vdn

@@ -1,0 +1,274 @@
+// Forward and backward state scan on the tensor cores (bf16 inputs, d = 128).
+//
+// What it computes (deepmagic post "用兩條分支取代一條", the frame-wise closed
+// form; PaperDaily digest section 三, the two directions and the half-text
+// start states): per (batch, head) and direction, from S = S_x / 2,
+//   S <- alpha_t S M_t + C_t        for every written (non-anchor) frame t,
+// frames in increasing order forward and decreasing order backward, anchor
+// frames leaving S unchanged, with the state saved at every chunk boundary:
+//   forward  slot j : frames < min(5j, T)      (slot 0 = start state)
+//   backward slot j : frames >= min(5j, T)     (slot C = start state)
+//
+// Rows of S evolve independently, but a whole 128-row state is exactly one
+// M = 128 tcgen05 tile, so one CTA carries one chain and each step is one
+// 128 x 128 x 128 product S M_t.  fp32 accuracy comes from the bf16 hi/lo
+// split of both factors (x = hi + lo with hi = bf16(x), lo = bf16(x - hi)):
+//   S M ~ S_hi M_hi + S_hi M_lo + S_lo M_hi
+// which keeps about 16 significant bits per step; M_t's split is written by
+// the solve, S's by this kernel's epilogue.  M_t is symmetric (the inverse
+// of an SPD matrix), so its rows serve as the K-major B operand.
+//
+// Roles (256 threads, one CTA per chain; the two directions of a head read
+// the same M_t, C_t, in opposite orders):
+//   warp 0      TMA producer: M_t split (64 KB) once the previous product is
+//               done, C_t (fp32, 64 KB) once the previous epilogue has read it.
+//   warp 1      TMEM allocator; lane 0 issues the 24 MMAs of S M_t.
+//   warps 4..7  epilogue, one state row per thread (= TMEM lane):
+//               S = alpha_t (S M_t) + C_t in fp32, chunk-boundary snapshots to
+//               global memory, and the new S split back into the A operand.
+// Everything is single-buffered: each step depends on the one before.
+#include "tc_common.cuh"
+
+namespace vdn {
+namespace {
+using namespace tc;
+
+constexpr int D = 128;
+constexpr int kThreadsScan = 256;
+constexpr uint32_t CHUNK = D * 128;      // 64 K-columns of a 128-row bf16 operand (SW128): 16 KB
+constexpr uint32_t OPBYTES = 2 * CHUNK;  // one 128 x 128 bf16 operand
+constexpr uint32_t SPLIT = 2 * OPBYTES;  // hi then lo: 64 KB
+constexpr uint32_t CBOX = D * 128;       // 32 fp32 columns x 128 rows (SW128): 16 KB
+constexpr uint32_t CBYTES = 4 * CBOX;    // C_t: 64 KB
+enum { B_BFULL = 0, B_CFULL = 1, B_SREADY = 2, B_MDONE = 3, B_DRAIN = 4, NBARS = 5 };
+
+__device__ __forceinline__ int frame_at(const Dims& d, int dir, int st) { return dir == 0 ? st : d.T - 1 - st; }
+
+// first scan position >= st whose frame is written (T if none)
+__device__ __forceinline__ int next_written(const Dims& d, int dir, int st) {
+  while (st < d.T && is_anchor(d, frame_at(d, dir, st))) ++st;
+  return st;
+}
+
+// snapshot slot taken after the frame at scan position st, or -1
+__device__ __forceinline__ int snap_slot(const Dims& d, int dir, int st) {
+  const int t = frame_at(d, dir, st);
+  if (dir == 0) {
+    if ((t + 1) % d.chunk == 0) return (t + 1) / d.chunk;
+    return (t + 1 == d.T) ? d.C : -1;
+  }
+  return (t % d.chunk == 0) ? t / d.chunk : -1;
+}
+
+// Bounded wait for this CTA's own copies or MMAs in flight, which end by
+// themselves: ignores the abort flag of the other roles.
+__device__ __noinline__ bool wait_own(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+
+__device__ __forceinline__ void st_global_v8(float* p, const float* v) {
+  asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+               "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
+}
+
+// 32 consecutive state values of `row` (columns 32q..32q+31): into the snapshot
+// slots of scan positions [p0, p1), and split into the A operand.
+__device__ __forceinline__ void emit_chunk(const Dims& dm, int dir, int p0, int p1, float* snap_row, int q, int row,
+                                           unsigned char* sA, const float (&s)[32]) {
+  const long long DD = (long long)D * D;
+  for (int p = p0; p < p1; ++p) {
+    const int sl = snap_slot(dm, dir, p);
+    if (sl >= 0) {
+      float* dst = snap_row + sl * DD + q * 32;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) st_global_v8(dst + 8 * u, s + 8 * u);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int k0 = q * 32 + 8 * e;
+    const uint32_t off = (k0 >> 6) * CHUNK + row * 128 + (((((k0 & 63) >> 3) ^ (row & 7))) << 4);
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float x0 = s[8 * e + 2 * j], x1 = s[8 * e + 2 * j + 1];
+      const __nv_bfloat16 a = __float2bfloat16_rn(x0), b = __float2bfloat16_rn(x1);
+      h[j] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+      l[j] = pack_bf16(x0 - __bfloat162float(a), x1 - __bfloat162float(b));
+    }
+    *reinterpret_cast<uint4*>(sA + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(sA + OPBYTES + off) = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreadsScan, 1)
+k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, const __grid_constant__ CUtensorMap tmc) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = sm;            // S  hi | lo, K-major SW128
+  unsigned char* sB = sA + SPLIT;    // M_t hi | lo, K-major SW128
+  unsigned char* sC = sB + SPLIT;    // C_t fp32, 4 boxes of 32 columns, SW128
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + CBYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
+  const int dir = blockIdx.x & 1, bh = blockIdx.x >> 1;
+  const int b = bh / dm.H, h = bh % dm.H;
+  const Ctl ctl{abort_flag, w.status, (unsigned)TAG_SCAN_TC};
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  auto fh_of = [&](int t) { return ((long long)b * dm.T + t) * dm.H + h; };
+  int nw = 0;  // written frames
+  for (int t = 0; t < dm.T; ++t) nw += is_anchor(dm, t) ? 0 : 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(B_BFULL), 1);
+    mbar_init(bar(B_CFULL), 1);
+    mbar_init(bar(B_SREADY), 128);
+    mbar_init(bar(B_MDONE), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Phases: BFULL, CFULL and MDONE complete once per written step i; SREADY
+  // once for the start state and once per step, so step i's MMA waits for
+  // SREADY phase i.  No role can run two phases ahead of a waiter.
+  if (warp == 0) {
+    if (lane == 0) {
+      int nb = 0, nc = 0;
+      int st = next_written(dm, dir, 0);
+      for (int i = 0; i < nw; ++i, st = next_written(dm, dir, st + 1)) {
+        const long long fh = fh_of(frame_at(dm, dir, st));
+        if (i > 0 && !mbar_wait(bar(B_MDONE), (i - 1) & 1, ctl)) break;  // B free
+        mbar_expect_tx(bar(B_BFULL), SPLIT);
+        for (int part = 0; part < 2; ++part)
+          for (int c = 0; c < 2; ++c)
+            tma_load_2d(smem_u32(sB + part * OPBYTES + c * CHUNK), &tmm, bar(B_BFULL), c * 64,
+                        (int)((fh * 2 + part) * D));
+        ++nb;
+        if (i > 0 && !mbar_wait(bar(B_SREADY), i & 1, ctl)) break;  // C read by the previous epilogue
+        mbar_expect_tx(bar(B_CFULL), CBYTES);
+        for (int c = 0; c < 4; ++c) tma_load_2d(smem_u32(sC + c * CBOX), &tmc, bar(B_CFULL), c * 32, (int)(fh * D));
+        ++nc;
+      }
+      // the last copies land before the CTA can exit
+      if (nb > 0) wait_own(bar(B_BFULL), (nb - 1) & 1);
+      if (nc > 0) wait_own(bar(B_CFULL), (nc - 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t ID = idesc_bf16(128, D, false);
+      const uint64_t a0 = sdesc(smem_u32(sA), 16, 1024), b0 = sdesc(smem_u32(sB), 16, 1024);
+      for (int i = 0; i < nw; ++i) {
+        if (!mbar_wait(bar(B_SREADY), i & 1, ctl)) break;
+        if (!mbar_wait(bar(B_BFULL), i & 1, ctl)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int pass = 0; pass < 3; ++pass) {  // hi hi, hi lo, lo hi
+          const uint32_t ao = pass == 2 ? OPBYTES : 0u, bo = pass == 1 ? OPBYTES : 0u;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k)
+            mma_bf16(tmem, dadd(a0, ao + (k >> 2) * CHUNK + (k & 3) * 32),
+                     dadd(b0, bo + (k >> 2) * CHUNK + (k & 3) * 32), ID, (pass | k) ? 1u : 0u);
+        }
+        mma_commit(bar(B_MDONE));
+      }
+      mma_commit(bar(B_DRAIN));
+      wait_own(bar(B_DRAIN), 0);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp - 4, row = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const long long DD = (long long)D * D;
+    float* snap_row = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD + (long long)row * D;
+    // start state: its own slot, then the slots of leading unwritten frames
+    int st = next_written(dm, dir, 0);
+    {
+      const float* src = w.half_text + (long long)bh * DD + (long long)row * D;
+      const int start_slot = dir == 0 ? 0 : dm.C;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        float s[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(src + q * 32) + u);
+          s[4 * u] = v.x; s[4 * u + 1] = v.y; s[4 * u + 2] = v.z; s[4 * u + 3] = v.w;
+        }
+        float* dst = snap_row + start_slot * DD + q * 32;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) st_global_v8(dst + 8 * u, s + 8 * u);
+        emit_chunk(dm, dir, 0, st, snap_row, q, row, sA, s);
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(bar(B_SREADY));
+    for (int i = 0; i < nw; ++i) {
+      const int st_next = next_written(dm, dir, st + 1);
+      const float alpha = __ldg(in.alpha + fh_of(frame_at(dm, dir, st)));
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MDONE), i & 1, ctl))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_CFULL), i & 1, ctl))) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        float v[32];
+        tmem_ld32(lane_addr + q * 32, v);
+        tmem_wait_ld();
+        const unsigned char* crow = sC + q * CBOX + row * 128;
+        float s[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 c4 = *reinterpret_cast<const float4*>(crow + ((u ^ (row & 7)) << 4));
+          s[4 * u] = fmaf(alpha, v[4 * u], c4.x);
+          s[4 * u + 1] = fmaf(alpha, v[4 * u + 1], c4.y);
+          s[4 * u + 2] = fmaf(alpha, v[4 * u + 2], c4.z);
+          s[4 * u + 3] = fmaf(alpha, v[4 * u + 3], c4.w);
+        }
+        emit_chunk(dm, dir, st, st_next, snap_row, q, row, sA, s);
+      }
+      tc_fence_before();        // TMEM reads done before the next product
+      fence_proxy_async_smem();  // new A operand visible to the tensor cores
+      mbar_arrive(bar(B_SREADY));
+      st = st_next;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, 128);
+}
+
+}  // namespace
+
+bool scan_tc_supported(const Dims& d) {
+  if (!scan_tc_layout(d.bf16 != 0, d.dk, d.dv) || !gram_tc_supported(d)) return false;
+  if ((long long)d.B * d.T * d.H * 2 * d.dk >= (1LL << 31)) return false;  // TMA row coordinates
+  if ((long long)d.B * d.H * 2 > 0x7FFFFFFFLL) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  if (d.dk != D || w.M16 == nullptr) return cudaErrorInvalidValue;
+  CUtensorMap mm, mc;
+  const long long fh = (long long)d.B * d.T * d.H;
+  if (!make_matrix_map(&mm, w.M16, fh * 2 * D, D, 128) || !make_matrix_map_f32(&mc, w.Cm, fh * D, D, 128))
+    return cudaErrorInvalidValue;
+  const size_t smem = 1024 + 2 * (size_t)SPLIT + CBYTES + NBARS * 8 + 16;
+  cudaError_t e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_scan_tc<<<(unsigned)(d.B * d.H * 2), kThreadsScan, smem, s>>>(d, in, w, mm, mc);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

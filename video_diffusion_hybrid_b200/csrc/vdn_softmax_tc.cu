@@ -159,7 +159,13 @@ __device__ __forceinline__ void key_tile(const Tile& t, int j, int& k0, int& kva
   kvalid = 0;
 }
 
-__device__ __forceinline__ float sigm(float x) { return 1.0f / (1.0f + __expf(-x)); }
+// sigmoid from the exponential and an approximate reciprocal (a few ulp;
+// exp(-x) overflowing to inf gives 0, the limit)
+__device__ __forceinline__ float sigm(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + __expf(-x)));
+  return r;
+}
 
 template <typename To> __device__ __forceinline__ void store4(To* p, float a, float b, float c, float d);
 template <> __device__ __forceinline__ void store4<float>(float* p, float a, float b, float c, float d) {

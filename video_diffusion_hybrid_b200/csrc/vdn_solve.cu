@@ -60,6 +60,21 @@ __device__ __forceinline__ void st_row(float* dst, const float (&src)[R], float 
   }
 }
 
+// bf16 hi/lo split of 8 consecutive values: hi = bf16(x), lo = bf16(x - hi)
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat16 a = __float2bfloat16_rn(x[2 * j]), b = __float2bfloat16_rn(x[2 * j + 1]);
+    const __nv_bfloat16 ra = __float2bfloat16_rn(x[2 * j] - __bfloat162float(a));
+    const __nv_bfloat16 rb = __float2bfloat16_rn(x[2 * j + 1] - __bfloat162float(b));
+    h[j] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+    l[j] = (uint32_t)__bfloat16_as_ushort(ra) | ((uint32_t)__bfloat16_as_ushort(rb) << 16);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 // TEXT: A_x, B_x from the text_gram region; writes S_x / 2 = B_x M_x / 2 to
 // the half-text state and no M.
 template <int D, bool TEXT>
@@ -127,6 +142,22 @@ k_solve_sweep(Dims dm, Work w) {
   for (int a = 0; a < R; ++a) {
     st_row<R>(Ms + (r0 + a) * P + c0, g[a], -1.0f);
     if (!TEXT) st_row<R>(gA + (r0 + a) * D + c0, g[a], -1.0f);
+  }
+  if constexpr (!TEXT && R == 8) {
+    // operand of the tensor-core scan: [hi | lo] bf16 rows of M
+    if (w.M16 != nullptr) {
+      __nv_bfloat16* mh = static_cast<__nv_bfloat16*>(w.M16) + fh * 2 * D * D;
+#pragma unroll
+      for (int a = 0; a < R; ++a) {
+        float m[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) m[c] = -g[a][c];
+        uint4 hi, lo;
+        split8(m, hi, lo);
+        *reinterpret_cast<uint4*>(mh + (r0 + a) * D + c0) = hi;
+        *reinterpret_cast<uint4*>(mh + D * D + (r0 + a) * D + c0) = lo;
+      }
+    }
   }
   __syncthreads();
   float acc[R][R];
