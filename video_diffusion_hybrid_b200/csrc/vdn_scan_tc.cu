@@ -18,14 +18,16 @@
 // the solve, S's by this kernel's epilogue.  M_t is symmetric (the inverse
 // of an SPD matrix), so its rows serve as the K-major B operand.
 //
-// Roles (256 threads, one CTA per chain; the two directions of a head read
+// Roles (384 threads, one CTA per chain; the two directions of a head read
 // the same M_t, C_t, in opposite orders):
 //   warp 0      TMA producer: M_t split (64 KB) once the previous product is
 //               done, C_t (fp32, 64 KB) once the previous epilogue has read it.
 //   warp 1      TMEM allocator; lane 0 issues the 24 MMAs of S M_t.
-//   warps 4..7  epilogue, one state row per thread (= TMEM lane):
-//               S = alpha_t (S M_t) + C_t in fp32, chunk-boundary snapshots to
-//               global memory, and the new S split back into the A operand.
+//   warps 4..11 epilogue, one state row per thread (= TMEM lane) and half
+//               of the columns per warp (warps w and w + 4 share the lanes of
+//               one 32-row quarter): S = alpha_t (S M_t) + C_t in fp32,
+//               chunk-boundary snapshots to global memory, and the new S
+//               split back into the A operand.
 // Everything is single-buffered: each step depends on the one before.
 #include "tc_common.cuh"
 
@@ -34,7 +36,7 @@ namespace {
 using namespace tc;
 
 constexpr int D = 128;
-constexpr int kThreadsScan = 256;
+constexpr int kThreadsScan = 384;
 constexpr uint32_t CHUNK = D * 128;      // 64 K-columns of a 128-row bf16 operand (SW128): 16 KB
 constexpr uint32_t OPBYTES = 2 * CHUNK;  // one 128 x 128 bf16 operand
 constexpr uint32_t SPLIT = 2 * OPBYTES;  // hi then lo: 64 KB
@@ -69,25 +71,42 @@ __device__ __noinline__ bool wait_own(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void st_global_v8(float* p, const float* v) {
   asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
                "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
                : "memory");
 }
 
-// 32 consecutive state values of `row` (columns 32q..32q+31): into the snapshot
-// slots of scan positions [p0, p1), and split into the A operand.
-__device__ __forceinline__ void emit_chunk(const Dims& dm, int dir, int p0, int p1, float* snap_row, int q, int row,
+// Snapshot slots taken after the frames at scan positions [p0, p1) (the
+// state is the same across them): at most two with anchors at both ends; a
+// longer run (never produced by the anchor rule) falls back to the loop.
+struct Slots {
+  int a, b, p0, p1;
+};
+__device__ __forceinline__ Slots slots_of(const Dims& dm, int dir, int p0, int p1) {
+  Slots r{-1, -1, p0, p1};
+  if (p1 - p0 <= 2) {
+    if (p0 < p1) r.a = snap_slot(dm, dir, p0);
+    if (p0 + 1 < p1) r.b = snap_slot(dm, dir, p0 + 1);
+    r.p0 = r.p1 = 0;
+  }
+  return r;
+}
+
+__device__ __forceinline__ void store_row32(float* dst, const float* s) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) st_global_v8(dst + 8 * u, s + 8 * u);
+}
+
+// 32 consecutive state values of `row` (columns 32q..32q+31): into the
+// snapshot slots, and split into the A operand.
+__device__ __forceinline__ void emit_chunk(const Dims& dm, int dir, const Slots& sl, float* snap_row, int q, int row,
                                            unsigned char* sA, const float (&s)[32]) {
   const long long DD = (long long)D * D;
-  for (int p = p0; p < p1; ++p) {
-    const int sl = snap_slot(dm, dir, p);
-    if (sl >= 0) {
-      float* dst = snap_row + sl * DD + q * 32;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) st_global_v8(dst + 8 * u, s + 8 * u);
-    }
-  }
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int k0 = q * 32 + 8 * e;
@@ -96,12 +115,17 @@ __device__ __forceinline__ void emit_chunk(const Dims& dm, int dir, int p0, int 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float x0 = s[8 * e + 2 * j], x1 = s[8 * e + 2 * j + 1];
-      const __nv_bfloat16 a = __float2bfloat16_rn(x0), b = __float2bfloat16_rn(x1);
-      h[j] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
-      l[j] = pack_bf16(x0 - __bfloat162float(a), x1 - __bfloat162float(b));
+      h[j] = pack_bf16(x0, x1);
+      l[j] = pack_bf16(x0 - __uint_as_float(h[j] << 16), x1 - __uint_as_float(h[j] & 0xFFFF0000u));
     }
     *reinterpret_cast<uint4*>(sA + off) = make_uint4(h[0], h[1], h[2], h[3]);
     *reinterpret_cast<uint4*>(sA + OPBYTES + off) = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+  if (sl.a >= 0) store_row32(snap_row + sl.a * DD + q * 32, s);
+  if (sl.b >= 0) store_row32(snap_row + sl.b * DD + q * 32, s);
+  for (int p = sl.p0; p < sl.p1; ++p) {
+    const int k = snap_slot(dm, dir, p);
+    if (k >= 0) store_row32(snap_row + k * DD + q * 32, s);
   }
 }
 
@@ -129,7 +153,7 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
   if (threadIdx.x == 0) {
     mbar_init(bar(B_BFULL), 1);
     mbar_init(bar(B_CFULL), 1);
-    mbar_init(bar(B_SREADY), 128);
+    mbar_init(bar(B_SREADY), 256);
     mbar_init(bar(B_MDONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -147,9 +171,24 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
   if (warp == 0) {
     if (lane == 0) {
       int nb = 0, nc = 0;
+      // M_t, C_t of the step two ahead are pulled into L2 early, so that the
+      // single-buffered loads below (issued only when their buffer frees) run
+      // at L2 rather than HBM latency
+      auto prefetch_step = [&](int pst) {
+        if (pst >= dm.T) return;
+        const long long pfh = fh_of(frame_at(dm, dir, pst));
+        prefetch_l2(static_cast<const __nv_bfloat16*>(w.M16) + pfh * 2 * D * D, SPLIT);
+        prefetch_l2(w.Cm + pfh * D * D, CBYTES);
+      };
       int st = next_written(dm, dir, 0);
+      int pst = st;
+      prefetch_step(pst);
+      pst = next_written(dm, dir, pst + 1);
+      prefetch_step(pst);
       for (int i = 0; i < nw; ++i, st = next_written(dm, dir, st + 1)) {
         const long long fh = fh_of(frame_at(dm, dir, st));
+        pst = next_written(dm, dir, pst + 1);
+        prefetch_step(pst);
         if (i > 0 && !mbar_wait(bar(B_MDONE), (i - 1) & 1, ctl)) break;  // B free
         mbar_expect_tx(bar(B_BFULL), SPLIT);
         for (int part = 0; part < 2; ++part)
@@ -188,8 +227,8 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
       wait_own(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
-    const int quad = warp - 4, row = quad * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const int quad = warp & 3, half = (warp - 4) >> 2, row = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + half * 64;
     const long long DD = (long long)D * D;
     float* snap_row = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD + (long long)row * D;
     // start state: its own slot, then the slots of leading unwritten frames
@@ -198,17 +237,15 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
       const float* src = w.half_text + (long long)bh * DD + (long long)row * D;
       const int start_slot = dir == 0 ? 0 : dm.C;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = 2 * half; q < 2 * half + 2; ++q) {
         float s[32];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const float4 v = __ldg(reinterpret_cast<const float4*>(src + q * 32) + u);
           s[4 * u] = v.x; s[4 * u + 1] = v.y; s[4 * u + 2] = v.z; s[4 * u + 3] = v.w;
         }
-        float* dst = snap_row + start_slot * DD + q * 32;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) st_global_v8(dst + 8 * u, s + 8 * u);
-        emit_chunk(dm, dir, 0, st, snap_row, q, row, sA, s);
+        store_row32(snap_row + start_slot * DD + q * 32, s);
+        emit_chunk(dm, dir, slots_of(dm, dir, 0, st), snap_row, q, row, sA, s);
       }
     }
     fence_proxy_async_smem();
@@ -216,27 +253,29 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
     for (int i = 0; i < nw; ++i) {
       const int st_next = next_written(dm, dir, st + 1);
       const float alpha = __ldg(in.alpha + fh_of(frame_at(dm, dir, st)));
+      const Slots sl = slots_of(dm, dir, st, st_next);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MDONE), i & 1, ctl))) break;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_CFULL), i & 1, ctl))) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
-        float v[32];
-        tmem_ld32(lane_addr + q * 32, v);
-        tmem_wait_ld();
-        const unsigned char* crow = sC + q * CBOX + row * 128;
-        float s[32];
+      float v[2][32];
+      tmem_ld32(lane_addr, v[0]);
+      tmem_ld32(lane_addr + 32, v[1]);
+      tmem_wait_ld();
+      tc_fence_before();  // TMEM reads done before the next product
+      const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {  // S = alpha (S M) + C in place, both chunks first
+        const unsigned char* crow = sC + (2 * half + qq) * CBOX + row * 128;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const float4 c4 = *reinterpret_cast<const float4*>(crow + ((u ^ (row & 7)) << 4));
-          s[4 * u] = fmaf(alpha, v[4 * u], c4.x);
-          s[4 * u + 1] = fmaf(alpha, v[4 * u + 1], c4.y);
-          s[4 * u + 2] = fmaf(alpha, v[4 * u + 2], c4.z);
-          s[4 * u + 3] = fmaf(alpha, v[4 * u + 3], c4.w);
+          const float2 lo = fma2(a2, make_float2(v[qq][4 * u], v[qq][4 * u + 1]), make_float2(c4.x, c4.y));
+          const float2 hi = fma2(a2, make_float2(v[qq][4 * u + 2], v[qq][4 * u + 3]), make_float2(c4.z, c4.w));
+          v[qq][4 * u] = lo.x; v[qq][4 * u + 1] = lo.y; v[qq][4 * u + 2] = hi.x; v[qq][4 * u + 3] = hi.y;
         }
-        emit_chunk(dm, dir, st, st_next, snap_row, q, row, sA, s);
       }
-      tc_fence_before();        // TMEM reads done before the next product
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) emit_chunk(dm, dir, sl, snap_row, 2 * half + qq, row, sA, v[qq]);
       fence_proxy_async_smem();  // new A operand visible to the tensor cores
       mbar_arrive(bar(B_SREADY));
       st = st_next;
