@@ -47,18 +47,32 @@ def parse():
 
 
 # ----------------------------------------------------------------- oracle --
-def oracle_sample(workload, n_na_tokens=128, n_a_tokens=64, head=0, seed_offset=0):
-    """Time the fp64 oracle on a bounded sample of one head of the workload:
-    the full bidirectional VDA chain of that head, both branches for
-    `n_na_tokens` queries of a non-anchor frame and `n_a_tokens` queries of an
-    anchor frame.  Extrapolates per-token costs to the whole layer (all heads,
-    all frames).  Returns (tokens/s, seconds of CPU work, description)."""
+def oracle_prepare(workload, seed_offset=0):
+    """Inputs of head 0 of the workload for the oracle (generated once, untimed)."""
     from oracle import vdn_oracle as O
     from video_diffusion_hybrid_b200.synth import Shape, make_inputs
     s = workload.shape
     one = Shape(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
     inp = make_inputs(one, workload.seed + seed_offset, workload.dtype)
     cfg = O.Cfg(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
+    return inp, cfg
+
+
+def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
+    """Time the fp64 oracle on a bounded sample of head 0 of the workload: the
+    full bidirectional VDA chain of the head (text solve, every frame's solve,
+    both scans), both branches for every query of the non-anchor frames in
+    `frames`, and both branches for `n_anchor_q` queries of anchor frame 0.
+    With `target_s`, further whole non-anchor frames (spread over the
+    sequence) are added until the sample holds about that much CPU work.
+    The per-frame costs are extrapolated to all frames of the head and the
+    head's cost to all B x H heads.  Returns (tokens/s, seconds of CPU work,
+    description)."""
+    from oracle import vdn_oracle as O
+    inp, cfg = prep
+    s = workload.shape
+    frames = frames if frames is not None else (s.T // 2, s.T // 4)
+    n_anchor_q = min(n_anchor_q if n_anchor_q is not None else s.N, s.N)
     t0 = time.perf_counter()
     F, G = O.head_states(inp, cfg, 0, 0)
     t_chain = time.perf_counter() - t0
@@ -71,17 +85,25 @@ def oracle_sample(workload, n_na_tokens=128, n_a_tokens=64, head=0, seed_offset=
         O.rms_gate(q[t, :n] @ R.T, inp["gate_lin"][0, t, :n, 0], cfg.rms_eps)
         o = O.softmax_frame(q[t, :n], k, v, t, s.T, cfg.chunk, cfg.anchors, cfg.scale)
         O.sigmoid(inp["gate_sm"][0, t, :n, 0]) * o
-        return (time.perf_counter() - t1) / n
+        return time.perf_counter() - t1
 
-    c_na = frame_cost(s.T // 2, min(n_na_tokens, s.N))
-    c_a = frame_cost(0, min(n_a_tokens, s.N))
-    n_anchor = 2
-    per_head = t_chain + (s.T - n_anchor) * s.N * c_na + n_anchor * s.N * c_a
+    frames = list(frames)
+    c_frames = [frame_cost(t, s.N) for t in frames]
+    c_anchor = frame_cost(0, n_anchor_q)
+    if target_s:
+        order = list(dict.fromkeys(t for t in (s.T * (2 * i + 1) // 64 for i in range(32))
+                                  if 0 < t < s.T - 1 and t not in frames))
+        while order and t_chain + sum(c_frames) + c_anchor < target_s:
+            frames.append(order.pop(0))
+            c_frames.append(frame_cost(frames[-1], s.N))
+    n_anchor = 2 if cfg.anchors else 0
+    per_head = (t_chain + (s.T - n_anchor) * statistics.mean(c_frames)
+                + n_anchor * c_anchor * s.N / n_anchor_q)
     layer = per_head * s.H * s.B
-    work = t_chain + min(n_na_tokens, s.N) * c_na + min(n_a_tokens, s.N) * c_a
-    desc = (f"head {head} of {workload.name}: full VDA chain over {s.T} frames + both branches for "
-            f"{min(n_na_tokens, s.N)} queries of a non-anchor frame and {min(n_a_tokens, s.N)} of an anchor "
-            f"frame; per-token costs extrapolated to {s.B}x{s.H} heads x {s.T * s.N} tokens")
+    work = t_chain + sum(c_frames) + c_anchor
+    desc = (f"head 0 of {workload.name}: the full VDA chain over {s.T} frames, both branches for all {s.N} "
+            f"queries of frames {list(frames)} and {n_anchor_q} queries of anchor frame 0; costs extrapolated "
+            f"to {s.T} frames x {s.B * s.H} heads")
     return s.B * s.T * s.N / layer, work, desc
 
 
@@ -100,11 +122,12 @@ def run_reference(args):
     if int(os.environ.get("RANK", "0")) != 0:
         return
     w = WORKLOADS[args.workload]
+    prep = oracle_prepare(w)
     vals, times = [], []
     desc = ""
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        val, _work, desc = oracle_sample(w, n_na_tokens=32, n_a_tokens=8)
+        val, _work, desc = oracle_sample(w, prep, frames=(w.shape.T // 2,), n_anchor_q=128)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             vals.append(val)
@@ -198,6 +221,33 @@ def kernel_traffic(kernel_file: str, key: str):
     return d.get("dram_bytes_per_launch")
 
 
+def stage_rooflines(s, cfg, ms, y_elem, peaks, sm_mhz):
+    """Each stage's time (CUDA events, the stage launched alone on resident
+    inputs) against the roofline of what it must compute or move."""
+    from video_diffusion_hybrid_b200 import roofline as R
+    elem = 2 if cfg.dtype == 1 else 4
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops_sustained"]
+    simt = R.fp32_simt_tflops(sm_mhz)
+    out = {"text": {"ms": ms["text"]}}
+    f = R.softmax_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.chunk, cfg.anchors)
+    a = f / (ms["softmax"] / 1e3) / 1e12
+    out["softmax"] = {"ms": ms["softmax"], "bound": "tensor", "achieved": a, "peak": tc, "unit": "TFLOP/s",
+                      "frac": a / tc, "work": f}
+    for name, by in (("read", R.read_bytes(s.B, s.T, s.N, s.H, s.d_k, elem, y_elem)),
+                     ("scan", R.scan_bytes(s.B, s.T, s.H, s.d_k, cfg.chunk, cfg.anchors))):
+        a = by / (ms[name] / 1e3) / 1e9
+        out[name] = {"ms": ms[name], "bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
+                     "work": by}
+    # per-frame Gram (HBM-bound) followed by the SPD sweep (fp32 SIMT-bound):
+    # the floor is the sum of the two
+    gb = R.gram_bytes(s.B, s.T, s.N, s.H, s.d_k, cfg.anchors, elem)
+    sf = R.sweep_flops(s.B, s.T, s.H, s.d_k, cfg.anchors)
+    floor_ms = 1e3 * (gb / (hbm * 1e9) + sf / (simt * 1e12))
+    out["solve"] = {"ms": ms["solve"], "bound": "hbm+alu", "floor_ms": floor_ms, "frac": floor_ms / ms["solve"],
+                    "gram_bytes": gb, "sweep_flops": sf, "alu_peak_tflops": simt}
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -223,7 +273,7 @@ def run_ours(args):
     s = w.shape
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, work, desc = oracle_sample(w)
+        val, work, desc = oracle_sample(w, oracle_prepare(w), target_s=12.0)
         cpu = {"value": val, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc,
                "sample_cpu_seconds": round(work, 2)}
 
@@ -232,7 +282,12 @@ def run_ours(args):
     ha = HybridAttention(cfg, dev)
     stream = torch.cuda.current_stream(dev)
     pre = L.STAGE_TEXT | L.STAGE_SOLVE | L.STAGE_SCAN
-    launches_per_step = 5 if (s.L > 0) else 4
+    # kernels a step launches: text (Gram + sweep on tensor cores, else one
+    # SIMT kernel), frame Gram + sweep (else one SIMT solve), scan, softmax,
+    # read table + read (else one SIMT read)
+    tc = lambda st: L.vdn_hybrid_stage_impl(cfg, st) == 1
+    text_k = (2 if tc(L.STAGE_TEXT) else 1) if s.L > 0 else 0  # no text: a memset, no kernel
+    launches_per_step = text_k + (2 if tc(L.STAGE_SOLVE) else 1) + 1 + 1 + (2 if tc(L.STAGE_READ) else 1)
     K, W = args.steps, args.warmup
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
 
@@ -309,6 +364,19 @@ def run_ours(args):
         e2e = {"value": world * w.tokens / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems}
 
+    # stage by stage, each launched alone (inputs and earlier stages' results resident)
+    stage_ms = {}
+    for name, st in (("text", L.STAGE_TEXT), ("solve", L.STAGE_SOLVE), ("scan", L.STAGE_SCAN),
+                     ("softmax", L.STAGE_SOFTMAX), ("read", L.STAGE_READ)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ha(t, stages=st)
+        a.record(stream)
+        for _ in range(3):
+            ha(t, stages=st)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        stage_ms[name] = a.elapsed_time(b) / 3
+
     if rank == 0:
         peaks, src = load_peaks()
         flops = softmax_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.chunk, cfg.anchors)
@@ -329,6 +397,8 @@ def run_ours(args):
                          "flops_per_launch": flops,
                          "traffic": kernel_traffic("vdn_softmax_tc.cu" if impl == 1 else "vdn_simt.cu",
                                                    "window_softmax")},
+            "stages": stage_rooflines(s, cfg, stage_ms, ha.y.element_size(), peaks,
+                                      (clocks or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * K,

@@ -29,6 +29,17 @@ static __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One arrival per warp: the warp barrier orders every lane's earlier
+// operations (after that lane's own fences) before lane 0's release-arrive,
+// and 32x fewer arrivals contend for the barrier word.  The barrier's count
+// is then the number of arriving warps.  Call with the whole warp.
+static __device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+  }
+}
+
 static __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -184,7 +184,7 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_GEMPTY || i == B_GEMPTY + 1 || i == B_AEMPTY ||
-                                                     i == B_AEMPTY + 1) ? 256 : 1);
+                                                     i == B_AEMPTY + 1) ? 8 : 1);  // one arrival per epilogue warp
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -276,7 +276,7 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
         for (int i = 0; i < 32; ++i) ss[i & 7] = fmaf(v[i], v[i], ss[i & 7]);
       }
       tc_fence_before();
-      mbar_arrive(bar(B_AEMPTY + s));  // accumulator free for tile t + ST
+      mbar_arrive_warp(bar(B_AEMPTY + s));  // accumulator free for tile t + ST
 #pragma unroll
       for (int i = 0; i < HD; ++i) ss[i & 7] = fmaf(o[i], o[i], ss[i & 7]);
       const float rs =
@@ -306,7 +306,7 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
         }
         if (valid) put8<To>(y + ch * 8, yv, add);
       }
-      mbar_arrive(bar(B_GEMPTY + s));  // gate tile free
+      mbar_arrive_warp(bar(B_GEMPTY + s));  // gate tile free
     }
   }
 

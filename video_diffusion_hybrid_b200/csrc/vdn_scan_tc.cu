@@ -153,7 +153,7 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
   if (threadIdx.x == 0) {
     mbar_init(bar(B_BFULL), 1);
     mbar_init(bar(B_CFULL), 1);
-    mbar_init(bar(B_SREADY), 256);
+    mbar_init(bar(B_SREADY), 8);  // one arrival per epilogue warp
     mbar_init(bar(B_MDONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -249,7 +249,7 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
       }
     }
     fence_proxy_async_smem();
-    mbar_arrive(bar(B_SREADY));
+    mbar_arrive_warp(bar(B_SREADY));
     for (int i = 0; i < nw; ++i) {
       const int st_next = next_written(dm, dir, st + 1);
       const float alpha = __ldg(in.alpha + fh_of(frame_at(dm, dir, st)));
@@ -277,7 +277,7 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) emit_chunk(dm, dir, sl, snap_row, 2 * half + qq, row, sA, v[qq]);
       fence_proxy_async_smem();  // new A operand visible to the tensor cores
-      mbar_arrive(bar(B_SREADY));
+      mbar_arrive_warp(bar(B_SREADY));
       st = st_next;
     }
   }

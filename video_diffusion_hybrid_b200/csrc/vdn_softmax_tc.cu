@@ -58,7 +58,7 @@ __host__ __device__ constexpr uint32_t col_s(int t) { return 256u + 128u * t; }
 // ------------------------------------------------------ work decomposition --
 struct Tile {
   int b, h, q0, qrows;      // absolute first query token, valid rows (of 256)
-  int niv;                  // key intervals
+  int niv;                  // key interval slots (always 3; unused ones empty)
   int kbeg[3], klen[3];     // absolute first key token, length
 };
 
@@ -126,37 +126,48 @@ __device__ bool decode_item(const Dims& d, long long item, Tile& t) {
   const int rows = (f1 - f0) * d.N;
   t.q0 = base + f0 * d.N + (int)qp * NQ * BM;
   t.qrows = min(NQ * BM, rows - (int)qp * NQ * BM);
-  t.niv = 0;
+  // three fixed interval slots (static indices keep the tile in registers);
+  // an unused slot has length 0 and holds no key tile
+  t.niv = 3;
   if (ridx == d.C) {
-    t.kbeg[0] = base; t.klen[0] = d.T * d.N; t.niv = 1;
+    t.kbeg[0] = base; t.klen[0] = d.T * d.N;
+    t.kbeg[1] = base; t.klen[1] = 0;
+    t.kbeg[2] = base; t.klen[2] = 0;
   } else {
     const int lo = max(0, (ridx - 1) * d.chunk), hi = min(d.T, (ridx + 2) * d.chunk);
-    if (d.anchors && lo > 0) { t.kbeg[t.niv] = base; t.klen[t.niv] = d.N; ++t.niv; }
-    t.kbeg[t.niv] = base + lo * d.N; t.klen[t.niv] = (hi - lo) * d.N; ++t.niv;
-    if (d.anchors && hi < d.T) { t.kbeg[t.niv] = base + (d.T - 1) * d.N; t.klen[t.niv] = d.N; ++t.niv; }
+    t.kbeg[0] = base; t.klen[0] = (d.anchors && lo > 0) ? d.N : 0;
+    t.kbeg[1] = base + lo * d.N; t.klen[1] = (hi - lo) * d.N;
+    t.kbeg[2] = base + (d.T - 1) * d.N; t.klen[2] = (d.anchors && hi < d.T) ? d.N : 0;
   }
   return true;
 }
 
 __device__ __forceinline__ int num_key_tiles(const Tile& t) {
   int n = 0;
-  for (int i = 0; i < t.niv; ++i) n += (t.klen[i] + BN - 1) / BN;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) n += (t.klen[i] + BN - 1) / BN;
   return n;
 }
 
 // Key tile j -> (first key token, valid keys).
 __device__ __forceinline__ void key_tile(const Tile& t, int j, int& k0, int& kvalid) {
-  for (int i = 0; i < t.niv; ++i) {
-    const int nt = (t.klen[i] + BN - 1) / BN;
-    if (j < nt) {
-      k0 = t.kbeg[i] + j * BN;
-      kvalid = min(BN, t.klen[i] - j * BN);
-      return;
-    }
-    j -= nt;
-  }
+  // fixed trip count and static indices: the tile stays in registers
   k0 = 0;
   kvalid = 0;
+  bool found = false;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const int nt = (t.klen[i] + BN - 1) / BN;
+    if (!found) {
+      if (j < nt) {
+        k0 = t.kbeg[i] + j * BN;
+        kvalid = min(BN, t.klen[i] - j * BN);
+        found = true;
+      } else {
+        j -= nt;
+      }
+    }
+  }
 }
 
 // sigmoid from the exponential and an approximate reciprocal (a few ulp;
@@ -209,7 +220,8 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_PFULL || i == B_PFULL + 1) ? 128 : 1);
+    // P_FULL: one arrival per softmax warp
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_PFULL || i == B_PFULL + 1) ? 4 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -228,8 +240,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       for (int t = 0; t < NQ; ++t)
         for (int c = 0; c < NB; ++c)
           tma_load_3d(smem_u32(sQ + t * QTILE + c * BM * 128), &tmq, bar(B_Q), c * 64, tile.h, tile.q0 + t * BM);
-      int lastk[KST];
-      for (int s = 0; s < KST; ++s) lastk[s] = -1;
+      int nk = 0;  // K tiles issued
       for (int j = 0; j < ntiles; ++j) {
         int k0, kv;
         key_tile(tile, j, k0, kv);
@@ -238,19 +249,19 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         mbar_expect_tx(bar(B_KFULL + sk), KVBYTES);
         for (int c = 0; c < NB; ++c)
           tma_load_3d(smem_u32(sK + sk * KVBYTES + c * BN * 128), &tmk, bar(B_KFULL + sk), c * 64, tile.h, k0);
-        lastk[sk] = j;
+        nk = j + 1;
       }
       // drain: every copy issued into this CTA's shared memory has landed
+      // (the last tile issued into each stage is one of the last KST)
       mbar_wait(bar(B_Q), 0, ctl);
-      for (int s = 0; s < KST; ++s)
-        if (lastk[s] >= 0) mbar_wait(bar(B_KFULL + s), (lastk[s] / KST) & 1, ctl);
+      for (int jj = nk - KST < 0 ? 0 : nk - KST; jj < nk; ++jj)
+        mbar_wait(bar(B_KFULL + jj % KST), (jj / KST) & 1, ctl);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ V producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmv)) : "memory");
-      int lastv[VST];
-      for (int s = 0; s < VST; ++s) lastv[s] = -1;
+      int nv = 0;  // V tiles issued
       for (int j = 0; j < ntiles; ++j) {
         int k0, kv;
         key_tile(tile, j, k0, kv);
@@ -259,10 +270,10 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         mbar_expect_tx(bar(B_VFULL + sv), KVBYTES);
         for (int c = 0; c < NB; ++c)
           tma_load_3d(smem_u32(sV + sv * KVBYTES + c * BN * 128), &tmv, bar(B_VFULL + sv), c * 64, tile.h, k0);
-        lastv[sv] = j;
+        nv = j + 1;
       }
-      for (int s = 0; s < VST; ++s)
-        if (lastv[s] >= 0) mbar_wait(bar(B_VFULL + s), (lastv[s] / VST) & 1, ctl);
+      for (int jj = nv - VST < 0 ? 0 : nv - VST; jj < nv; ++jj)
+        mbar_wait(bar(B_VFULL + jj % VST), (jj / VST) & 1, ctl);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -277,7 +288,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       // need have been cleared (waits first, then the MMAs back to back).
       auto mma_s = [&](int t, int j) {
         const int sk = j % KST;
-        const uint64_t qd = qdesc[t], kd = dadd(kdesc0, sk * KVBYTES);
+        const uint64_t qd = t == 0 ? qdesc[0] : qdesc[1], kd = dadd(kdesc0, sk * KVBYTES);
         const uint32_t dst = tmem + col_s(t);
         mma_bf16(dst, qd, kd, ID_S, 0u);
 #pragma unroll
@@ -459,7 +470,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       }
       tc_fence_before();
-      mbar_arrive(bar(B_PFULL + t));
+      mbar_arrive_warp(bar(B_PFULL + t));
     }
     // ---- epilogue: O / l, gate, store
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_ODONE + t), (ntiles - 1) & 1, ctl))) {

@@ -45,3 +45,40 @@ def softmax_bytes(B, T, N, H, d, elem=2, out_slot_bytes=None) -> float:
     """q, k, v, gate_sm read once; y softmax slot written once."""
     tok = B * T * N * H * d
     return tok * elem * 4 + tok * (out_slot_bytes or elem)
+
+
+def written_frames(T: int, anchors: int = 4) -> int:
+    return T - (2 if anchors and T >= 2 else 0)
+
+
+def gram_bytes(B, T, N, H, d, anchors=4, elem=2) -> float:
+    """Per-frame write: k, v (elem bytes) and beta (fp32) of the written frames
+    read once; A_t, B_t (fp32 d x d) written once."""
+    nw = written_frames(T, anchors)
+    return nw * B * H * (N * (2 * d * elem + 4) + 2 * d * d * 4)
+
+
+def sweep_flops(B, T, H, d, anchors=4) -> float:
+    """SPD solve per written frame-head: d pivots of a d x d rank-one update
+    (d^3 multiply-adds) plus C = B M (d^3 multiply-adds)."""
+    return 4.0 * d ** 3 * written_frames(T, anchors) * B * H
+
+
+def scan_bytes(B, T, H, d, chunk=5, anchors=4) -> float:
+    """Both directions read every written frame's M_t (as its bf16 hi/lo
+    split, 4 bytes an entry) and C_t (fp32); the chunk-boundary states (fp32,
+    C + 1 per direction) are written once and the start state read once."""
+    C = (T + chunk - 1) // chunk
+    nw = written_frames(T, anchors)
+    return B * H * (2 * nw * 2 * d * d * 4 + 2 * (C + 1) * d * d * 4 + 2 * d * d * 4)
+
+
+def read_bytes(B, T, N, H, d, elem=2, y_elem=4) -> float:
+    """q and gate_lin read once, the linear slot of y written once (the read
+    table itself is a few MB and stays in L2)."""
+    return B * T * N * H * d * (2 * elem + y_elem)
+
+
+def fp32_simt_tflops(sm_mhz: float, sms: int = 148) -> float:
+    """SIMT fp32 peak: 128 FMA lanes per SM per clock, 2 flops each."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
