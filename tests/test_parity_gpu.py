@@ -225,11 +225,12 @@ def _sample_rows(cfg, heads, per_head, rng):
     return rows
 
 
-@pytest.mark.parametrize("name", ["768p"])
+@pytest.mark.parametrize("name", ["768p", "long"])
 def test_full_size_sampled_parity(name):
     """At the benchmark's size and launch configuration (inputs drawn on the
-    device): sampled outputs against the oracle evaluated position by
-    position on two heads."""
+    device), and at the long-video size (T=180, two batch elements with their
+    own seeds): sampled outputs against the oracle evaluated position by
+    position on a head of the first and of the last batch element."""
     from video_diffusion_hybrid_b200.synth import head_slice, make_inputs_torch
     w = WORKLOADS[name]
     t = make_inputs_torch(w.shape, w.seed, w.dtype, "cuda")
@@ -241,14 +242,46 @@ def test_full_size_sampled_parity(name):
     assert bool(torch.isfinite(y).all())
     rng = np.random.default_rng(0)
     s = w.shape
-    for h in (0, s.H - 1):
-        inp = head_slice(t, 0, h)
+    for b, h in ((0, 0), (s.B - 1, s.H - 1)):
+        inp = head_slice(t, b, h)
         oc = O.Cfg(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
         rows = _sample_rows(oc, heads=(0,), per_head=24, rng=rng)
         ref = O.hybrid_attn_rows(inp, oc, rows)
         idx = torch.tensor([(t_, n) for (_, t_, n, _) in rows], device=y.device)
-        got = y[0, idx[:, 0], idx[:, 1], h].float().cpu().numpy()
+        got = y[b, idx[:, 0], idx[:, 1], h].float().cpu().numpy()
         for sl in (0, 1):
             rms = np.sqrt(np.mean(ref[:, sl] ** 2))
             err = np.max(np.abs(got[:, sl] - ref[:, sl])) / rms
-            assert err <= TOL[w.dtype], (h, sl, err)
+            assert err <= TOL[w.dtype], (b, h, sl, err)
+    del t, y, ha
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["sweep_N256_d64", "sweep_N1008_d64", "sweep_N4032_d64", "sweep_N256_d128",
+                                  "sweep_N4032_d128"])
+def test_vda_sweep_sampled_parity(name):
+    """The VDA-only sweep shapes (T=90, H=24): the four VDA stages alone
+    (text, frame write + solve, scans, read), the linear slot of sampled
+    outputs against the oracle on two heads."""
+    from video_diffusion_hybrid_b200.synth import head_slice, make_inputs_torch
+    w = WORKLOADS[name]
+    t = make_inputs_torch(w.shape, w.seed, w.dtype, "cuda")
+    cfg = cfg_for(w.shape, w.dtype)
+    ha = HybridAttention(cfg)
+    vda = L.STAGE_TEXT | L.STAGE_SOLVE | L.STAGE_SCAN | L.STAGE_READ
+    y = ha(t, stages=vda)
+    torch.cuda.synchronize()
+    assert L.vdn_hybrid_device_status(cfg, ha.args(t))[0] == L.VDN_OK
+    rng = np.random.default_rng(1)
+    s = w.shape
+    for h in (0, s.H - 1):
+        inp = head_slice(t, 0, h)
+        oc = O.Cfg(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
+        rows = _sample_rows(oc, heads=(0,), per_head=24, rng=rng)
+        ref = O.hybrid_attn_rows(inp, oc, rows)[:, 1]
+        idx = torch.tensor([(t_, n) for (_, t_, n, _) in rows], device=y.device)
+        got = y[0, idx[:, 0], idx[:, 1], h, 1].float().cpu().numpy()
+        err = np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref ** 2))
+        assert err <= TOL[w.dtype], (h, err)
+    del t, y, ha
+    torch.cuda.empty_cache()
