@@ -69,7 +69,10 @@ typedef struct {
   int T;        /* latent frames                                                  >= 2 */
   int N;        /* spatial tokens per frame                                       >= 1 */
   int H;        /* heads                                                          >= 1 */
-  int d_k;      /* key/query head dim: 32, 64 or 128                                   */
+  int d_k;      /* key/query head dim: 32, 64, 128 or 256.  256 needs dtype VDN_BF16
+                   and runs the Video Delta Attention stages only (TEXT, SOLVE, SCAN,
+                   READ); a call that includes VDN_STAGE_SOFTMAX returns
+                   VDN_ERR_UNSUPPORTED without launching                            */
   int d_v;      /* value head dim; must equal d_k in this build                        */
   int L;        /* text tokens; 0 = no text (states start from init_state or zero)     */
   int chunk;    /* latent frames per chunk; must be 5                                  */

@@ -96,6 +96,16 @@ def test_bad_args_rejected_before_launch(over, status):
     assert L.vdn_hybrid_attn_fwd_stages(cfg, args, L.STAGE_SOFTMAX, stream=0, check=False) == status
 
 
+def test_d256_softmax_refused_before_launch():
+    """d = 256 runs the Video Delta Attention stages only: a call that asks for
+    the softmax is refused during validation, before any launch."""
+    cfg = _cfg(d_k=256, d_v=256)
+    args = _fake_args(cfg)
+    assert L.vdn_hybrid_attn_fwd(cfg, args, stream=0, check=False) == L.VDN_ERR_UNSUPPORTED
+    assert L.vdn_hybrid_attn_fwd_stages(cfg, args, L.STAGE_SOFTMAX | L.STAGE_READ, stream=0, check=False) == \
+        L.VDN_ERR_UNSUPPORTED
+
+
 def test_text_pointers_forbidden_without_text():
     cfg = _cfg(L=0)
     assert L.vdn_hybrid_attn_fwd(cfg, _fake_args(cfg), stream=0, check=False) == L.VDN_ERR_INVALID_ARG
@@ -124,4 +134,11 @@ def test_status_strings_and_stage_impl():
     for st in (L.STAGE_TEXT, L.STAGE_SOLVE, L.STAGE_SCAN, L.STAGE_READ, L.STAGE_SOFTMAX):
         assert L.vdn_hybrid_stage_impl(cfg, st) in (0, 1)
     assert L.vdn_hybrid_stage_impl(cfg, 3) == -1
-    assert L.vdn_hybrid_stage_impl(_cfg(d_k=256, d_v=256), L.STAGE_SOLVE) == -1
+    # d = 256: the Video Delta Attention stages only, bf16 inputs only
+    big = _cfg(d_k=256, d_v=256)
+    assert L.vdn_hybrid_stage_impl(big, L.STAGE_SOFTMAX) == -1
+    for st in (L.STAGE_TEXT, L.STAGE_SOLVE, L.STAGE_SCAN, L.STAGE_READ):
+        assert L.vdn_hybrid_stage_impl(big, st) in (0, 1)
+    assert L.vdn_hybrid_attn_workspace_size(big) > 0
+    assert L.vdn_hybrid_stage_impl(_cfg(d_k=256, d_v=256, dtype=L.VDN_F32), L.STAGE_SOLVE) == -1
+    assert L.vdn_hybrid_attn_workspace_size(_cfg(d_k=256, d_v=256, dtype=L.VDN_F32)) == 0

@@ -31,7 +31,7 @@ def ocfg(cfg: L.HybridCfg) -> O.Cfg:
                  out_mode=cfg.out_mode)
 
 
-def run(shape: Shape, dtype: str, seed: int, extra=None, drop_text=False, **kw):
+def run(shape: Shape, dtype: str, seed: int, extra=None, drop_text=False, stages=L.STAGE_ALL, **kw):
     inp = make_inputs(shape, seed, dtype)
     if drop_text:
         for k in ("text_k", "text_v", "text_beta", "text_k_bits", "text_v_bits"):
@@ -43,11 +43,14 @@ def run(shape: Shape, dtype: str, seed: int, extra=None, drop_text=False, **kw):
         cfg.L = 0
     t = to_torch(inp, dtype, "cuda")
     ha = HybridAttention(cfg)
-    y = ha(t)
+    y = ha(t, stages=stages)
     torch.cuda.synchronize()
     st, where = L.vdn_hybrid_device_status(cfg, ha.args(t))
     assert st == L.VDN_OK, where
     return inp, cfg, ha, t, y.float().cpu().numpy().astype(np.float64)
+
+
+VDA = L.STAGE_TEXT | L.STAGE_SOLVE | L.STAGE_SCAN | L.STAGE_READ
 
 
 def rel_err(got, ref, allowance=None):
@@ -144,6 +147,29 @@ def test_bf16_frame_maps_match_oracle(shape):
             for t in range(1, cfg.T - 1):
                 np.testing.assert_allclose(it["M"][b, t, h], ref["M"][t], atol=2e-5)
                 np.testing.assert_allclose(it["C"][b, t, h], ref["C"][t], atol=2e-5 * np.abs(ref["C"][t]).max())
+
+
+@pytest.mark.parametrize("shape", [Shape(1, 12, 96, 2, 256, 256, 16), Shape(1, 10, 40, 1, 256, 256, 0)])
+def test_d256_vda_matches_oracle(shape):
+    """d = 256, the Video Delta Attention stages (the only ones at this size):
+    M_t, C_t and S_x / 2 after the block-mode Gram and the block solve, the
+    read table after the chunked scans, and the linear slot of every output
+    after the chunked read, against the oracle."""
+    inp, cfg, ha, t, y = run(shape, "bf16", 21, drop_text=shape.L == 0, stages=VDA)
+    it = {k: v.double().cpu().numpy() for k, v in ha.intermediates().items()}
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            ref = O.vda_intermediates(inp, ocfg(cfg), b, h)
+            sx = np.abs(ref["S_init"]).max() + 1e-30
+            np.testing.assert_allclose(it["half_text"][b, h], ref["S_init"], atol=2e-5 * sx)
+            for f in range(1, cfg.T - 1):
+                np.testing.assert_allclose(it["M"][b, f, h], ref["M"][f], atol=2e-5)
+                np.testing.assert_allclose(it["C"][b, f, h], ref["C"][f], atol=2e-5 * np.abs(ref["C"][f]).max())
+            np.testing.assert_allclose(it["R"][b, h], ref["R"], atol=1e-4 * np.sqrt(np.mean(ref["R"] ** 2)) + 1e-30)
+    ref_y = O.hybrid_attn(inp, ocfg(cfg))
+    assert rel_err(y[..., 1, :], ref_y[..., 1, :]) <= TOL["bf16"]
+    # the softmax stage has no kernel at this size: refused before any launch
+    assert L.vdn_hybrid_attn_fwd(cfg, ha.args(t), check=False) == L.VDN_ERR_UNSUPPORTED
 
 
 def test_bf16_read_table_matches_oracle():
@@ -258,7 +284,7 @@ def test_full_size_sampled_parity(name):
 
 
 @pytest.mark.parametrize("name", ["sweep_N256_d64", "sweep_N1008_d64", "sweep_N4032_d64", "sweep_N256_d128",
-                                  "sweep_N4032_d128"])
+                                  "sweep_N4032_d128", "sweep_N256_d256", "sweep_N1008_d256", "sweep_N4032_d256"])
 def test_vda_sweep_sampled_parity(name):
     """The VDA-only sweep shapes (T=90, H=24): the four VDA stages alone
     (text, frame write + solve, scans, read), the linear slot of sampled

@@ -22,8 +22,11 @@ vdn_status check_cfg(const vdn_hybrid_cfg* c) {
   if (c->out_mode != 0 && c->out_mode != 1) return VDN_ERR_INVALID_ARG;
   if (c->y_dtype != VDN_F32 && c->y_dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
   if (!(c->softmax_scale == c->softmax_scale) || !(c->rms_eps == c->rms_eps)) return VDN_ERR_INVALID_ARG;
-  if (c->d_k != 32 && c->d_k != 64 && c->d_k != 128) return VDN_ERR_UNSUPPORTED;
+  if (c->d_k != 32 && c->d_k != 64 && c->d_k != 128 && c->d_k != 256) return VDN_ERR_UNSUPPORTED;
   if (c->d_v != c->d_k) return VDN_ERR_UNSUPPORTED;
+  // d = 256: the per-frame Gram runs on the tensor cores only (bf16 inputs)
+  if (c->d_k == 256 && c->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
+  if (c->d_k == 256 && (long long)c->H * 6 > 65535) return VDN_ERR_UNSUPPORTED;
   if (c->chunk != 5) return VDN_ERR_UNSUPPORTED;
   // grid limits of the launches (gridDim.y / gridDim.z <= 65535)
   if ((long long)c->B * c->H > 65535) return VDN_ERR_UNSUPPORTED;
@@ -148,6 +151,7 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
     case VDN_STAGE_READ:
       return read_tc_supported(d) ? 1 : 0;
     case VDN_STAGE_SOFTMAX:
+      if (big_d(d)) return -1;
       return softmax_tc_supported(d) ? 1 : 0;
     default:
       return -1;
@@ -164,12 +168,16 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
   const Dims d = make_dims(cfg);
   const Work w = work_of(cfg, args);
   const Inputs in = inputs_of(args);
+  const bool big = big_d(d);
+  // d = 256: the VDA stages only (the softmax stage has no kernel at this size)
+  if (big && ((stages & VDN_STAGE_SOFTMAX) || !gram_tc_supported(d))) return VDN_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
   if (cudaMemsetAsync(w.status, 0, 256, s) != cudaSuccess) return VDN_ERR_CUDA;
   if (stages & VDN_STAGE_TEXT) {
     if (d.L > 0 && gram_tc_supported(d)) {
       if ((e = launch_text_gram_tc(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
-      if ((e = launch_text_solve_sweep(d, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+      e = big ? launch_solve_big(d, w, s, true) : launch_text_solve_sweep(d, w, s);
+      if (e != cudaSuccess) return VDN_ERR_CUDA;
     } else if ((e = launch_text(d, in, w, s)) != cudaSuccess) {
       return VDN_ERR_CUDA;
     }
@@ -177,12 +185,15 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
   if (stages & VDN_STAGE_SOLVE) {
     if (gram_tc_supported(d)) {
       if ((e = launch_gram_tc(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
-      if ((e = launch_solve_inplace(d, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
+      e = big ? launch_solve_big(d, w, s, false) : launch_solve_inplace(d, w, s);
+      if (e != cudaSuccess) return VDN_ERR_CUDA;
     } else if ((e = launch_solve_simt(d, in, w, s)) != cudaSuccess) {
       return VDN_ERR_CUDA;
     }
   }
-  if (stages & VDN_STAGE_SCAN) {
+  if (big && (stages & VDN_STAGE_SCAN)) {
+    if (launch_scan_big(d, in, w, s) != cudaSuccess) return VDN_ERR_CUDA;
+  } else if (stages & VDN_STAGE_SCAN) {
     // the tensor-core scan reads the bf16 split of M that the sweep solve writes
     e = (scan_tc_supported(d) && w.M16 != nullptr) ? launch_scan_tc(d, in, w, s) : launch_scan_simt(d, in, w, s);
     if (e != cudaSuccess) return VDN_ERR_CUDA;
@@ -191,7 +202,9 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     e = softmax_tc_supported(d) ? launch_softmax_tc(d, in, w, s) : launch_softmax_simt(d, in, w, s);
     if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
-  if (stages & VDN_STAGE_READ) {
+  if (big && (stages & VDN_STAGE_READ)) {
+    if (launch_read_big(d, in, w, s) != cudaSuccess) return VDN_ERR_CUDA;
+  } else if (stages & VDN_STAGE_READ) {
     // the tensor-core read writes y rows with 32-byte stores
     e = (read_tc_supported(d) && aligned(in.y, 32)) ? launch_read_tc(d, in, w, w.R16, s)
                                                     : launch_read_simt(d, in, w, s);

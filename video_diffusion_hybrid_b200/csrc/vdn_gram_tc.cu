@@ -23,6 +23,13 @@
 //               with both operands MN-major (d contiguous), so no repacking.
 //               For d = 64, K and V stack into one M = 128 operand and one
 //               accumulator [A; B] (64 columns).
+// d = 256 (block mode): A_t and B_t are 2 x 2 blocks of 128 x 128, and every
+// block is the second product of a CTA of the d = 128 form run on 128-column
+// views: with X = K[:, 128x : 128x + 128] for beta K and Y a 128-column view
+// of K or V, the CTA forms X^T (beta X) = A(x, x) and Y^T (beta X), which is
+// the block (y, x) of A (Y from K) or of B (Y from V).  Six CTAs per frame-head
+// cover the eight blocks: (x, Y) = (0, V0): A00 B00; (0, V1): B10; (1, V0):
+// A11 B01; (1, V1): B11; (0, K1): A10; (1, K0): A01.
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -33,8 +40,9 @@ constexpr int TT = 128;  // tokens per tile
 constexpr int kThreadsG = 256;
 
 // TEXT: the L text tokens of (b, h) instead of one frame; A_x, B_x go to the
-// text_gram region of the workspace.
-template <int D, bool TEXT>
+// text_gram region of the workspace.  BLK: the d = 256 block mode above (D is
+// then the 128-column view width).
+template <int D, bool TEXT, bool BLK>
 __global__ void __launch_bounds__(kThreadsG, 1)
 k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
           const __grid_constant__ CUtensorMap tmv) {
@@ -53,8 +61,14 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  constexpr int DF = BLK ? 2 * D : D;  // row length of k, v and of A_t, B_t
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int t = blockIdx.x, b = blockIdx.z;
+  const int h = BLK ? blockIdx.y / 6 : blockIdx.y, call = BLK ? blockIdx.y % 6 : 0;
+  // block mode: view columns of X (beta K) and of Y, and where Y^T (beta X) goes
+  const int bx = (call == 2 || call == 3 || call == 5) ? 1 : 0;
+  const int by = (call == 1 || call == 3 || call == 4) ? 1 : 0;
+  const bool y_from_v = call < 4, write_a = call == 0 || call == 2;
   if (!TEXT && is_anchor(dm, t)) return;
   if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
   const int ntok = TEXT ? dm.L : dm.N;
@@ -62,7 +76,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
   // first token of the frame (or of batch b's text)
   const long long tok0 = TEXT ? (long long)b * dm.L : ((long long)b * dm.T + t) * dm.N;
   const float* betap = TEXT ? in.text_beta : in.beta;
-  const long long DDg = (long long)D * D;
+  const long long DDg = (long long)DF * DF;
   float* outA = TEXT ? w.text_gram + ((long long)b * dm.H + h) * 2 * DDg
                      : w.M + (((long long)b * dm.T + t) * dm.H + h) * DDg;
   float* outB = TEXT ? outA + DDg : w.Cm + (((long long)b * dm.T + t) * dm.H + h) * DDg;
@@ -89,8 +103,9 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
         const int tok = (int)(tok0 + (long long)j * TT);
         mbar_expect_tx(bar(B_KVFULL + s), STAGE);
         for (int c = 0; c < NB; ++c) {
-          tma_load_3d(smem_u32(sKV + s * STAGE + c * TT * 128), &tmk, bar(B_KVFULL + s), c * 64, h, tok);
-          tma_load_3d(smem_u32(sKV + s * STAGE + TB + c * TT * 128), &tmv, bar(B_KVFULL + s), c * 64, h, tok);
+          tma_load_3d(smem_u32(sKV + s * STAGE + c * TT * 128), &tmk, bar(B_KVFULL + s), c * 64 + bx * D, h, tok);
+          tma_load_3d(smem_u32(sKV + s * STAGE + TB + c * TT * 128), (!BLK || y_from_v) ? &tmv : &tmk,
+                      bar(B_KVFULL + s), c * 64 + by * D, h, tok);
         }
         last[s] = j;
       }
@@ -167,13 +182,17 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
       if (D == 128) {
-        float* Ag = outA + (long long)row * D;
-        float* Bg = outB + (long long)row * D;
+        // rows of X^T (beta X) and Y^T (beta X); in block mode placed as the
+        // blocks (bx, bx) and (by, bx) of the d = 256 matrices
+        float* Ag = outA + (long long)(bx * D + row) * DF + bx * D;
+        float* Bg = (!BLK || y_from_v ? outB : outA) + (long long)(by * D + row) * DF + bx * D;
+        const bool wa = !BLK || write_a;
 #pragma unroll
         for (int q = 0; q < 2 * D / 32; ++q) {
           float v[32];
           tmem_ld32(lane_addr + q * 32, v);
           tmem_wait_ld();
+          if (q < D / 32 && !wa) continue;
           float* dst = q < D / 32 ? Ag + q * 32 : Bg + (q - D / 32) * 32;
 #pragma unroll
           for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
@@ -200,30 +219,33 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
   if (warp == 1) tmem_free(tmem, kCols);
 }
 
-template <int D, bool TEXT>
+template <int D, bool TEXT, bool BLK = false>
 cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  constexpr int DF = BLK ? 2 * D : D;
   CUtensorMap mk, mv;
   const long long tokens = TEXT ? (long long)d.B * d.L : (long long)d.B * d.T * d.N;
-  if (!make_token_map(&mk, TEXT ? in.text_k : in.k, tokens, d.H, D, TT) ||
-      !make_token_map(&mv, TEXT ? in.text_v : in.v, tokens, d.H, D, TT))
+  if (!make_token_map(&mk, TEXT ? in.text_k : in.k, tokens, d.H, DF, TT) ||
+      !make_token_map(&mv, TEXT ? in.text_v : in.v, tokens, d.H, DF, TT))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 2 * (2 * (size_t)TT * D * 2) + 2 * (size_t)TT * D * 2 + 8 * 8 + 16;
-  auto kern = k_gram_tc<D, TEXT>;
+  auto kern = k_gram_tc<D, TEXT, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(TEXT ? 1 : d.T, d.H, d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
+  kern<<<dim3(TEXT ? 1 : d.T, d.H * (BLK ? 6 : 1), d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool gram_tc_supported(const Dims& d) {
-  if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128)) return false;
+  if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128 && d.dk != 256)) return false;
   if ((long long)d.B * d.T * d.N >= (1LL << 31)) return false;
+  if ((long long)d.H * 6 > 65535) return false;
   return encode_fn() != nullptr;
 }
 
 cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  if (d.dk == 256) return launch<128, false, true>(d, in, w, s);
   if (d.dk == 128) return launch<128, false>(d, in, w, s);
   if (d.dk == 64) return launch<64, false>(d, in, w, s);
   return cudaErrorInvalidValue;
@@ -231,6 +253,7 @@ cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaS
 
 cudaError_t launch_text_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   if (d.L <= 0 || (long long)d.B * d.L >= (1LL << 31)) return cudaErrorInvalidValue;
+  if (d.dk == 256) return launch<128, true, true>(d, in, w, s);
   if (d.dk == 128) return launch<128, true>(d, in, w, s);
   if (d.dk == 64) return launch<64, true>(d, in, w, s);
   return cudaErrorInvalidValue;

@@ -64,6 +64,11 @@ bool read_tc_supported(const Dims& d);
 // the workspace holds the bf16 split of M (and the solve writes it) exactly when this holds
 __host__ __device__ inline bool scan_tc_layout(bool bf16, int dk, int dv) { return bf16 && dk == 128 && dv == 128; }
 bool scan_tc_supported(const Dims& d);
+// d = 256: block solve, chunked scan and chunked read (SIMT), Gram in block mode
+bool big_d(const Dims& d);
+cudaError_t launch_solve_big(const Dims& d, const Work& w, cudaStream_t s, bool text);
+cudaError_t launch_scan_big(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_read_big(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void* r16, cudaStream_t s);
 

@@ -25,40 +25,12 @@
 // -1 / g_pp, and since later pivots only add to this entry the surplus 2 is
 // removed from the whole diagonal once, at the end.
 #include "vdn_internal.h"
+#include "sweep.cuh"
 
 namespace vdn {
 namespace {
 
 constexpr int kThreadsS = 256;
-
-template <int R>
-__device__ __forceinline__ void ld_row(float (&dst)[R], const float* src) {
-  if constexpr (R % 4 == 0) {
-#pragma unroll
-    for (int c = 0; c < R; c += 4) {
-      const float4 v = *reinterpret_cast<const float4*>(src + c);
-      dst[c] = v.x; dst[c + 1] = v.y; dst[c + 2] = v.z; dst[c + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < R; c += 2) {
-      const float2 v = *reinterpret_cast<const float2*>(src + c);
-      dst[c] = v.x; dst[c + 1] = v.y;
-    }
-  }
-}
-
-template <int R>
-__device__ __forceinline__ void st_row(float* dst, const float (&src)[R], float sgn) {
-  if constexpr (R % 4 == 0) {
-#pragma unroll
-    for (int c = 0; c < R; c += 4)
-      *reinterpret_cast<float4*>(dst + c) = make_float4(sgn * src[c], sgn * src[c + 1], sgn * src[c + 2], sgn * src[c + 3]);
-  } else {
-#pragma unroll
-    for (int c = 0; c < R; c += 2) *reinterpret_cast<float2*>(dst + c) = make_float2(sgn * src[c], sgn * src[c + 1]);
-  }
-}
 
 // bf16 hi/lo split of 8 consecutive values: hi = bf16(x), lo = bf16(x - hi)
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
@@ -105,37 +77,7 @@ k_solve_sweep(Dims dm, Work w) {
     if (ty == tx) g[a][a] += 1.0f;
   }
 
-  for (int pb = 0; pb < 16; ++pb) {
-#pragma unroll
-    for (int a = 0; a < R; ++a) {
-      float* buf = rowbuf + (a & 1) * BP;
-      if (ty == pb) {
-        float v[R];
-#pragma unroll
-        for (int c = 0; c < R; ++c) v[c] = g[a][c];
-        if (tx == pb) {
-          buf[D] = 1.0f / v[a];
-          v[a] -= 1.0f;
-        }
-        st_row<R>(buf + c0, v, 1.0f);
-      }
-      __syncthreads();  // also orders the reads of this buffer two pivots ago
-      const float inv = buf[D];
-      float colv[R], rowv[R];
-      ld_row<R>(colv, buf + r0);
-      ld_row<R>(rowv, buf + c0);
-#pragma unroll
-      for (int c = 0; c < R; ++c) rowv[c] *= inv;
-#pragma unroll
-      for (int i = 0; i < R; ++i)
-#pragma unroll
-        for (int c = 0; c < R; ++c) g[i][c] = fmaf(-colv[i], rowv[c], g[i][c]);
-    }
-  }
-  if (ty == tx) {
-#pragma unroll
-    for (int a = 0; a < R; ++a) g[a][a] -= 2.0f;
-  }
+  sweep_regs<D>(g, rowbuf);  // g = -G^-1
 
   // M = -G_swept: to global and to shared for C = B M
 #pragma unroll
