@@ -359,22 +359,32 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         for (int u = 0; u < 4; ++u) ps2[u] = make_float2(0.f, 0.f);
         uint32_t pmax = 0u;  // running max of the packed P (bf16 pairs, all >= 0)
         float pk0[32], pk1[32];
+        // 32 scores at a time; the next chunk's TMEM load is in flight while
+        // this chunk computes (a load is complete only after the wait that
+        // follows the computation)
+        auto chunk = [&](const float (&v)[32], float (&pk)[32], int o) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float v0[32], v1[32];
-          tmem_ld32(scol + 64 * hf, v0);
-          tmem_ld32(scol + 64 * hf + 32, v1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float2 sv = i < 16 ? make_float2(v0[2 * i], v0[2 * i + 1]) : make_float2(v1[2 * i - 32], v1[2 * i - 31]);
-            const float2 x = fma2(sv, c2, nmc2);
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = fma2(make_float2(v[2 * i], v[2 * i + 1]), c2, nmc2);
             const uint32_t u = pack_bf16(ex2(x.x), ex2(x.y));
             pmax = max_bf16x2(pmax, u);
             ps2[i & 3] = add2(ps2[i & 3], make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
-            if (hf == 0) pk0[i] = __uint_as_float(u); else pk1[i] = __uint_as_float(u);
+            pk[o + i] = __uint_as_float(u);
           }
-        }
+        };
+        float va[32], vb[32];
+        tmem_ld32(scol, va);
+        tmem_wait_ld();
+        tmem_ld32(scol + 32, vb);
+        chunk(va, pk0, 0);
+        tmem_wait_ld();
+        tmem_ld32(scol + 64, va);
+        chunk(vb, pk0, 16);
+        tmem_wait_ld();
+        tmem_ld32(scol + 96, vb);
+        chunk(va, pk1, 0);
+        tmem_wait_ld();
+        chunk(vb, pk1, 16);
         // overflow: some weight above 2^8, i.e. a score more than 2^8 (in exp2
         // units) above the running max; the exact path then rescales
         const float pmx = fmaxf(__uint_as_float(pmax << 16), __uint_as_float(pmax & 0xFFFF0000u));
