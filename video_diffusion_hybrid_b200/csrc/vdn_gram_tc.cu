@@ -39,6 +39,13 @@ using namespace tc;
 constexpr int TT = 128;  // tokens per tile
 constexpr int kThreadsG = 256;
 
+// 8 consecutive fp32 values as one 32-byte store (full sectors; dst 32-byte aligned)
+__device__ __forceinline__ void st_v8(float* p, const float* v) {
+  asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+               "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+               : "memory");
+}
+
 // TEXT: the L text tokens of (b, h) instead of one frame; A_x, B_x go to the
 // text_gram region of the workspace.  BLK: the d = 256 block mode above (D is
 // then the 128-column view width).
@@ -149,12 +156,18 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
     const int quad = warp - 4;
     const int row = quad * 32 + lane;  // token row of the tile / TMEM lane
     bool ok = true;
+    // beta of this thread's token, one tile ahead (its load overlaps the waits)
+    auto beta_of = [&](int j) {
+      const int tk = j * TT + row;
+      return tk < ntok ? __ldg(betap + (tok0 + tk) * dm.H + h) : 0.f;
+    };
+    float beta_next = beta_of(0);
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % ST;
+      const float beta = beta_next;
+      if (j + 1 < ntiles) beta_next = beta_of(j + 1);
       if (!mbar_wait(bar(B_KVFULL + s), (j / ST) & 1, ctl)) { ok = false; break; }
       if (j > 0 && !mbar_wait(bar(B_KBEMPTY), (j - 1) & 1, ctl)) { ok = false; break; }
-      const int tk = j * TT + row;
-      const float beta = tk < ntok ? __ldg(betap + (tok0 + tk) * dm.H + h) : 0.f;
 #pragma unroll
       for (int c = 0; c < NB; ++c) {
 #pragma unroll
@@ -195,7 +208,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
           if (q < D / 32 && !wa) continue;
           float* dst = q < D / 32 ? Ag + q * 32 : Bg + (q - D / 32) * 32;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          for (int i = 0; i < 32; i += 8) st_v8(dst + i, v + i);
         }
       } else {
         // lanes 0..63 hold A rows, lanes 64..127 hold B rows
