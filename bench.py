@@ -91,8 +91,10 @@ def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
     c_frames = [frame_cost(t, s.N) for t in frames]
     c_anchor = frame_cost(0, n_anchor_q)
     if target_s:
-        order = list(dict.fromkeys(t for t in (s.T * (2 * i + 1) // 64 for i in range(32))
-                                  if 0 < t < s.T - 1 and t not in frames))
+        # positions spread over the sequence first, then the remaining frames:
+        # at most the whole head is timed
+        spread = [s.T * (2 * i + 1) // 64 for i in range(32)] + list(range(1, s.T - 1))
+        order = list(dict.fromkeys(t for t in spread if 0 < t < s.T - 1 and t not in frames))
         while order and t_chain + sum(c_frames) + c_anchor < target_s:
             frames.append(order.pop(0))
             c_frames.append(frame_cost(frames[-1], s.N))
@@ -102,8 +104,8 @@ def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
     layer = per_head * s.H * s.B
     work = t_chain + sum(c_frames) + c_anchor
     desc = (f"head 0 of {workload.name}: the full VDA chain over {s.T} frames, both branches for all {s.N} "
-            f"queries of frames {list(frames)} and {n_anchor_q} queries of anchor frame 0; costs extrapolated "
-            f"to {s.T} frames x {s.B * s.H} heads")
+            f"queries of {len(frames)} non-anchor frames spread over the sequence and {n_anchor_q} queries of "
+            f"anchor frame 0; costs extrapolated to {s.T} frames x {s.B * s.H} heads")
     return s.B * s.T * s.N / layer, work, desc
 
 
