@@ -9,9 +9,9 @@
 // the M_t / C_t slots of the workspace, where the SPD solve replaces them by
 // M_t = (I + A_t)^-1 and C_t = B_t M_t.
 //
-// One CTA per (batch, frame, head); the frame's tokens in tiles of 128:
+// One CTA per (batch, frame, head); the frame's tokens in tiles of 64:
 //   warp 0      TMA producer: K and V tiles (two-stage ring, 128B-swizzled).
-//   warps 4..7  one token row per thread: beta K in two bf16 terms,
+//   warps 4..7  two threads per token row: beta K in two bf16 terms,
 //               hi = bf16(beta k), lo = bf16(beta k - hi), written in the same
 //               swizzled layout (tokens past the frame get beta = 0).  k and v
 //               are exact in bf16 and products accumulate in fp32, so the
@@ -36,7 +36,7 @@ namespace vdn {
 namespace {
 using namespace tc;
 
-constexpr int TT = 128;  // tokens per tile
+constexpr int TT = 64;   // tokens per tile (two CTAs per SM: 96 KB of shared memory, 256 TMEM columns)
 constexpr int kThreadsG = 256;
 
 // 8 consecutive fp32 values as one 32-byte store (full sectors; dst 32-byte aligned)
@@ -50,7 +50,7 @@ __device__ __forceinline__ void st_v8(float* p, const float* v) {
 // text_gram region of the workspace.  BLK: the d = 256 block mode above (D is
 // then the 128-column view width).
 template <int D, bool TEXT, bool BLK>
-__global__ void __launch_bounds__(kThreadsG, 1)
+__global__ void __launch_bounds__(kThreadsG, 2)
 k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
           const __grid_constant__ CUtensorMap tmv) {
   constexpr int NB = D / 64;
@@ -156,9 +156,12 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
     const int quad = warp - 4;
     const int row = quad * 32 + lane;  // token row of the tile / TMEM lane
     bool ok = true;
+    // token row of the tile for the beta K split: two threads per row, each
+    // taking half of the row's 16-byte units
+    const int srow = (quad * 32 + lane) % TT, shalf = (quad * 32 + lane) / TT;
     // beta of this thread's token, one tile ahead (its load overlaps the waits)
     auto beta_of = [&](int j) {
-      const int tk = j * TT + row;
+      const int tk = j * TT + srow;
       return tk < ntok ? __ldg(betap + (tok0 + tk) * dm.H + h) : 0.f;
     };
     float beta_next = beta_of(0);
@@ -169,10 +172,10 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       if (!mbar_wait(bar(B_KVFULL + s), (j / ST) & 1, ctl)) { ok = false; break; }
       if (j > 0 && !mbar_wait(bar(B_KBEMPTY), (j - 1) & 1, ctl)) { ok = false; break; }
 #pragma unroll
-      for (int c = 0; c < NB; ++c) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t off = c * TT * 128 + row * 128 + ((q ^ (row & 7)) << 4);
+      for (int uu = 0; uu < NB * 4; ++uu) {
+        {
+          const int unit = shalf * NB * 4 + uu, c = unit >> 3, q = unit & 7;
+          const uint32_t off = c * TT * 128 + srow * 128 + ((q ^ (srow & 7)) << 4);
           const uint4 raw = *reinterpret_cast<const uint4*>(sKV + s * STAGE + off);
           const uint32_t u[4] = {raw.x, raw.y, raw.z, raw.w};
           uint32_t hv[4], lv[4];
