@@ -203,7 +203,9 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
   if (big && (stages & VDN_STAGE_READ)) {
-    if (launch_read_big(d, in, w, s) != cudaSuccess) return VDN_ERR_CUDA;
+    // the tensor-core read writes y rows with 32-byte stores; else the chunked SIMT read
+    e = (read_tc_supported(d) && aligned(in.y, 32)) ? launch_read_tc(d, in, w, w.R16, s) : launch_read_big(d, in, w, s);
+    if (e != cudaSuccess) return VDN_ERR_CUDA;
   } else if (stages & VDN_STAGE_READ) {
     // the tensor-core read writes y rows with 32-byte stores
     e = (read_tc_supported(d) && aligned(in.y, 32)) ? launch_read_tc(d, in, w, w.R16, s)

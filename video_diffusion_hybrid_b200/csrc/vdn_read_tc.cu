@@ -144,6 +144,15 @@ template <> __device__ __forceinline__ void put8<__nv_bfloat16>(__nv_bfloat16* p
       make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
 }
 
+// Bounded wait for this CTA's own copies or MMAs in flight, which end by
+// themselves: ignores the abort flag of the other roles.
+__device__ __noinline__ bool wait_landed(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+
 // sigmoid from the exponential and an approximate reciprocal (both a few ulp;
 // exp(-g) overflowing to inf gives 0, the limit)
 __device__ __forceinline__ float sigmoid_fast(float g) {
@@ -316,6 +325,169 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
   if (warp == 1) tmem_free(tmem, kCols);
 }
 
+// ------------------------------------------------------------ d = 256 --
+// The same read at d = 256.  R's split (256 KB) does not fit beside a query
+// tile, so it streams through shared memory in K-chunks of 64 (hi and lo of
+// all 256 rows, 64 KB per chunk, two-stage ring) once per 128-token tile; the
+// chunks stay in L2 across the CTAs of a query group.  Per tile, 32 MMAs of
+// M = 128, N = 256, K = 16 accumulate O = Q R_hi^T + Q R_lo^T into one of two
+// 256-column TMEM accumulators.  Epilogue: eight warps, each owning 128 of the
+// 256 columns of its 32 rows; a first pass over all 256 TMEM columns forms the
+// sum of squares, a second pass its own outputs (gates read from global).
+constexpr int D2 = 256;
+
+template <typename To>
+__global__ void __launch_bounds__(kThreadsR, 1)
+k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
+             const __grid_constant__ CUtensorMap tmr) {
+  constexpr uint32_t QCH = TQ * 128;        // one 64-column chunk of the Q tile: 16 KB
+  constexpr uint32_t QBYTES = 4 * QCH;      // the Q tile
+  constexpr uint32_t RHALF = D2 * 128;      // 64 columns of all 256 rows of R_hi (or R_lo): 32 KB
+  constexpr uint32_t RST = 2 * RHALF;       // one ring stage: hi then lo
+  enum { B_QFULL = 0, B_QEMPTY = 1, B_RFULL = 2, B_REMPTY = 4, B_AFULL = 6, B_AEMPTY = 8, B_DRAIN = 10, NBARS = 11 };
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = sm;
+  unsigned char* sR = sQ + QBYTES;          // 2 stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + 2 * RST);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sW = reinterpret_cast<float*>(tmem_slot + 4);  // [256] RMSNorm weight (ones if none)
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
+  Run run;
+  if (!decode_run(dm, blockIdx.x, run)) return;
+  const Ctl ctl{abort_flag, w.status, (unsigned)TAG_READ_TC};
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_AEMPTY || i == B_AEMPTY + 1) ? 8 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+  for (int i = threadIdx.x; i < D2; i += blockDim.x)
+    sW[i] = in.rms_weight ? in.rms_weight[(long long)run.h * D2 + i] : 1.0f;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int rrow = ((run.b * dm.H + run.h) * (dm.C + 1) + run.ridx) * 2 * D2;
+      int nq = 0, nr = 0;
+      for (int j = 0; j < run.ntiles; ++j) {
+        const int tok = (int)(run.tok0 + (long long)j * TQ);
+        if (j > 0 && !mbar_wait(bar(B_QEMPTY), (j - 1) & 1, ctl)) break;
+        mbar_expect_tx(bar(B_QFULL), QBYTES);
+        for (int c = 0; c < 4; ++c) tma_load_3d(smem_u32(sQ + c * QCH), &tmq, bar(B_QFULL), c * 64, run.h, tok);
+        ++nq;
+        bool ok = true;
+        for (int kc = 0; kc < 4; ++kc) {
+          const int u = j * 4 + kc, s = u & 1;
+          if (u >= 2 && !mbar_wait(bar(B_REMPTY + s), ((u >> 1) - 1) & 1, ctl)) { ok = false; break; }
+          mbar_expect_tx(bar(B_RFULL + s), RST);
+          tma_load_2d(smem_u32(sR + s * RST), &tmr, bar(B_RFULL + s), kc * 64, rrow);
+          tma_load_2d(smem_u32(sR + s * RST + RHALF), &tmr, bar(B_RFULL + s), kc * 64, rrow + D2);
+          ++nr;
+        }
+        if (!ok) break;
+      }
+      // the last copies land before the CTA can exit (bounded, whatever the other roles do)
+      if (nq > 0) wait_landed(bar(B_QFULL), (nq - 1) & 1);
+      for (int u = nr - 2 < 0 ? 0 : nr - 2; u < nr; ++u) wait_landed(bar(B_RFULL + (u & 1)), (u >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t ID = idesc_bf16(TQ, D2, false);
+      const uint64_t qdesc = sdesc(smem_u32(sQ), 16, 1024), rdesc = sdesc(smem_u32(sR), 16, 1024);
+      bool ok = true;
+      for (int j = 0; ok && j < run.ntiles; ++j) {
+        const int acc = j & 1;
+        if (j >= 2 && !mbar_wait(bar(B_AEMPTY + acc), ((j >> 1) - 1) & 1, ctl)) break;
+        if (!mbar_wait(bar(B_QFULL), j & 1, ctl)) break;
+        for (int kc = 0; kc < 4; ++kc) {
+          const int u = j * 4 + kc, s = u & 1;
+          if (!mbar_wait(bar(B_RFULL + s), (u >> 1) & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16(tmem + acc * D2, dadd(qdesc, kc * QCH + ks * 32), dadd(rdesc, s * RST + part * RHALF + ks * 32),
+                       ID, (kc | part | ks) ? 1u : 0u);
+          mma_commit(bar(B_REMPTY + s));
+        }
+        if (!ok) break;
+        mma_commit(bar(B_AFULL + acc));
+        mma_commit(bar(B_QEMPTY));
+      }
+      mma_commit(bar(B_DRAIN));
+      wait_landed(bar(B_DRAIN), 0);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3, half = (warp - 4) >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const bool add = dm.out_mode != 0;
+    for (int j = 0; j < run.ntiles; ++j) {
+      const int acc = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + acc), (j >> 1) & 1, ctl))) break;
+      tc_fence_after();
+      float ss[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ss[u] = 0.f;
+#pragma unroll 1
+      for (int q = 0; q < D2 / 32; ++q) {
+        float v[32];
+        tmem_ld32(lane_addr + acc * D2 + q * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ss[i & 7] = fmaf(v[i], v[i], ss[i & 7]);
+      }
+      const float rs =
+          rsqrtf((((ss[0] + ss[1]) + (ss[2] + ss[3])) + ((ss[4] + ss[5]) + (ss[6] + ss[7]))) / D2 + dm.eps);
+      const int rows_valid = min(TQ, run.rows_left - j * TQ);
+      const bool valid = row < rows_valid;
+      const long long tok = run.tok0 + (long long)j * TQ + row;
+      const long long gi = (tok * dm.H + run.h) * D2;
+      To* y = static_cast<To*>(in.y) + (dm.out_mode == 0 ? 2 * gi + D2 : gi);
+      const __nv_bfloat16* grow = static_cast<const __nv_bfloat16*>(in.gate_lin) + gi;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        const int col0 = half * 128 + q * 32;
+        float v[32];
+        tmem_ld32(lane_addr + acc * D2 + col0, v);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(grow + col0 + ch * 8));
+            const uint32_t gu[4] = {raw.x, raw.y, raw.z, raw.w};
+            float yv[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i0 = ch * 8 + 2 * e;
+              yv[2 * e] = v[i0] * rs * sW[col0 + i0] * sigmoid_fast(__uint_as_float(gu[e] << 16));
+              yv[2 * e + 1] = v[i0 + 1] * rs * sW[col0 + i0 + 1] * sigmoid_fast(__uint_as_float(gu[e] & 0xFFFF0000u));
+            }
+            put8<To>(y + col0 + ch * 8, yv, add);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_warp(bar(B_AEMPTY + acc));  // accumulator free for tile j + 2
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, 512);
+}
+
 long long num_runs(const Dims& d) {
   const int ngroups = d.C + (d.anchors ? 2 : 0);
   long long per_bh = 0;
@@ -357,10 +529,30 @@ cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, __nv_bfloat16
   return cudaGetLastError();
 }
 
+template <typename To>
+cudaError_t launch256(const Dims& d, const Inputs& in, const Work& w, __nv_bfloat16* r16, cudaStream_t s) {
+  k_read_table<<<dim3(d.C + 1, d.B * d.H), 256, 0, s>>>(d, w, r16);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mq, mr;
+  const long long tokens = (long long)d.B * d.T * d.N;
+  if (!make_token_map(&mq, in.q, tokens, d.H, D2, TQ) ||
+      !make_matrix_map(&mr, r16, (long long)d.B * d.H * (d.C + 1) * 2 * D2, D2, D2))
+    return cudaErrorInvalidValue;
+  const size_t smem = 1024 + 4 * (size_t)TQ * 128 + 2 * 2 * (size_t)D2 * 128 + 11 * 8 + 16 + D2 * 4;
+  auto kern = k_read256_tc<To>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long items = num_runs(d);
+  if (items <= 0 || items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  kern<<<(unsigned)items, kThreadsR, smem, s>>>(d, in, w, mq, mr);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool read_tc_supported(const Dims& d) {
-  if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128)) return false;
+  if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128 && d.dk != 256)) return false;
   if ((long long)d.B * d.T * d.N >= (1LL << 31)) return false;
   if ((long long)d.B * d.H * (d.C + 1) * 2 * d.dk >= (1LL << 31)) return false;
   return encode_fn() != nullptr;
@@ -368,6 +560,7 @@ bool read_tc_supported(const Dims& d) {
 
 cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void* r16, cudaStream_t s) {
   __nv_bfloat16* r = static_cast<__nv_bfloat16*>(r16);
+  if (d.dk == 256) return d.out_bf16 ? launch256<__nv_bfloat16>(d, in, w, r, s) : launch256<float>(d, in, w, r, s);
   if (d.dk == 128) return d.out_bf16 ? launch<128, __nv_bfloat16>(d, in, w, r, s) : launch<128, float>(d, in, w, r, s);
   if (d.dk == 64) return d.out_bf16 ? launch<64, __nv_bfloat16>(d, in, w, r, s) : launch<64, float>(d, in, w, r, s);
   return cudaErrorInvalidValue;
