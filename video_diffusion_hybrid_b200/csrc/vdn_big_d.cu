@@ -217,8 +217,20 @@ k_solve_block(Dims dm, Work w) {
 // independently (s_row <- alpha s_row M + c_row), so a CTA carries RB rows of
 // one chain: thread (rq, cq) holds rows 8 rq .. 8 rq + 7 and columns 4 cq ..
 // 4 cq + 3 of its block, and the block's transpose sits in shared memory for
-// the products.  M_t streams through shared memory KC rows at a time.
-constexpr int RB = 32, KC = 32;
+// the products.  M_t streams through a double buffer in shared memory, KC
+// rows at a time, the next chunk's asynchronous copy in flight while the
+// current one computes.  Three CTAs per SM keep every chain of a launch
+// resident at once (each CTA runs all the frames, so a second wave would
+// double the time).
+constexpr int RB = 32, KC = 16;
+
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ int snap_slot_big(const Dims& d, int dir, int t) {
   if (dir == 0) {
@@ -228,11 +240,11 @@ __device__ __forceinline__ int snap_slot_big(const Dims& d, int dir, int t) {
   return (t % d.chunk == 0) ? t / d.chunk : -1;
 }
 
-__global__ void __launch_bounds__(kThreadsB)
+__global__ void __launch_bounds__(kThreadsB, 3)
 k_scan_big(Dims dm, Inputs in, Work w) {
   extern __shared__ __align__(16) float smb[];
-  float* St = smb;            // [DB][RB]  this CTA's rows of S, transposed
-  float* Mc = St + DB * RB;   // [KC][DB]  a chunk of M_t's rows
+  float* St = smb;            // [DB][RB]     this CTA's rows of S, transposed
+  float* Mc = St + DB * RB;   // [2][KC][DB]  chunks of M_t's rows
   const int tid = threadIdx.x, cq = tid & 63, rq = tid >> 6;
   const int r0 = rq * 8, c0 = cq * 4;
   const int row0 = blockIdx.x * RB, dir = blockIdx.y, bh = blockIdx.z;
@@ -242,25 +254,34 @@ k_scan_big(Dims dm, Inputs in, Work w) {
   float* snap = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD;
   auto gidx = [&](int r, int c) { return (long long)(row0 + r0 + r) * DB + c0 + c; };
 
-  float cur[8][4];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const float4 v = *reinterpret_cast<const float4*>(half + gidx(r, 0));
-    cur[r][0] = v.x; cur[r][1] = v.y; cur[r][2] = v.z; cur[r][3] = v.w;
-    *reinterpret_cast<float4*>(snap + (dir == 0 ? 0 : (long long)dm.C * DD) + gidx(r, 0)) = v;
-  }
-  auto put_state = [&]() {
+  // the state lives in St (transposed); a thread's 8 x 4 block is in registers
+  // only while it is formed
+  auto put_state = [&](const float (&v)[8][4]) {
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0) = make_float4(cur[0][c], cur[1][c], cur[2][c], cur[3][c]);
-      *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0 + 4) =
-          make_float4(cur[4][c], cur[5][c], cur[6][c], cur[7][c]);
+      *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0) = make_float4(v[0][c], v[1][c], v[2][c], v[3][c]);
+      *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0 + 4) = make_float4(v[4][c], v[5][c], v[6][c], v[7][c]);
     }
   };
-  put_state();
+  auto snapshot = [&](int slot, const float (&v)[8][4]) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      *reinterpret_cast<float4*>(snap + (long long)slot * DD + gidx(r, 0)) = make_float4(v[r][0], v[r][1], v[r][2], v[r][3]);
+  };
+  {
+    float v[8][4];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float4 x = *reinterpret_cast<const float4*>(half + gidx(r, 0));
+      v[r][0] = x.x; v[r][1] = x.y; v[r][2] = x.z; v[r][3] = x.w;
+    }
+    snapshot(dir == 0 ? 0 : dm.C, v);
+    put_state(v);
+  }
 
   for (int st = 0; st < dm.T; ++st) {
     const int t = dir == 0 ? st : dm.T - 1 - st;
+    const int slot = snap_slot_big(dm, dir, t);
     if (!is_anchor(dm, t)) {
       const long long fh = ((long long)b * dm.T + t) * dm.H + h;
       const float* Mg = w.M + fh * DD;
@@ -271,19 +292,31 @@ k_scan_big(Dims dm, Inputs in, Work w) {
       for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-      for (int k0 = 0; k0 < DB; k0 += KC) {
-        __syncthreads();  // the previous chunk (and the state) fully read / written
+      auto fetch = [&](int kc) {  // rows [KC kc, KC kc + KC) of M_t into buffer kc & 1
+        float* dst = Mc + (kc & 1) * KC * DB;
 #pragma unroll
         for (int v = 0; v < KC * DB / 4 / kThreadsB; ++v) {
           const int e = (tid + v * kThreadsB) * 4;
-          *reinterpret_cast<float4*>(Mc + e) = *reinterpret_cast<const float4*>(Mg + (long long)k0 * DB + e);
+          cp_async16(dst + e, Mg + (long long)kc * KC * DB + e);
         }
-        __syncthreads();
+        cp_async_commit();
+      };
+      fetch(0);
+      for (int kc = 0; kc < DB / KC; ++kc) {
+        if (kc + 1 < DB / KC) {
+          fetch(kc + 1);
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
+        }
+        __syncthreads();  // chunk kc (and the state) visible to every thread
+        const float* mc = Mc + (kc & 1) * KC * DB;
+        const int k0 = kc * KC;
 #pragma unroll 4
         for (int k = 0; k < KC; ++k) {
           const float4 s0 = *reinterpret_cast<const float4*>(St + (k0 + k) * RB + r0);
           const float4 s1 = *reinterpret_cast<const float4*>(St + (k0 + k) * RB + r0 + 4);
-          const float4 m = *reinterpret_cast<const float4*>(Mc + k * DB + c0);
+          const float4 m = *reinterpret_cast<const float4*>(mc + k * DB + c0);
           const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
           const float mv[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
@@ -291,24 +324,28 @@ k_scan_big(Dims dm, Inputs in, Work w) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(sv[r], mv[c], acc[r][c]);
         }
+        __syncthreads();  // chunk kc read by every thread before its buffer is refilled
       }
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const float4 cv = *reinterpret_cast<const float4*>(Cg + gidx(r, 0));
-        cur[r][0] = fmaf(alpha, acc[r][0], cv.x);
-        cur[r][1] = fmaf(alpha, acc[r][1], cv.y);
-        cur[r][2] = fmaf(alpha, acc[r][2], cv.z);
-        cur[r][3] = fmaf(alpha, acc[r][3], cv.w);
+        acc[r][0] = fmaf(alpha, acc[r][0], cv.x);
+        acc[r][1] = fmaf(alpha, acc[r][1], cv.y);
+        acc[r][2] = fmaf(alpha, acc[r][2], cv.z);
+        acc[r][3] = fmaf(alpha, acc[r][3], cv.w);
       }
-      __syncthreads();  // every read of the old state done
-      put_state();
-    }
-    const int slot = snap_slot_big(dm, dir, t);
-    if (slot >= 0) {
+      put_state(acc);  // every read of the old state finished at the last barrier
+      if (slot >= 0) snapshot(slot, acc);
+    } else if (slot >= 0) {
+      float v[8][4];
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        *reinterpret_cast<float4*>(snap + (long long)slot * DD + gidx(r, 0)) =
-            make_float4(cur[r][0], cur[r][1], cur[r][2], cur[r][3]);
+      for (int c = 0; c < 4; ++c) {
+        const float4 x = *reinterpret_cast<const float4*>(St + (c0 + c) * RB + r0);
+        const float4 y = *reinterpret_cast<const float4*>(St + (c0 + c) * RB + r0 + 4);
+        v[0][c] = x.x; v[1][c] = x.y; v[2][c] = x.z; v[3][c] = x.w;
+        v[4][c] = y.x; v[5][c] = y.y; v[6][c] = y.z; v[7][c] = y.w;
+      }
+      snapshot(slot, v);
     }
   }
 }
@@ -445,7 +482,7 @@ cudaError_t launch_solve_big(const Dims& d, const Work& w, cudaStream_t s, bool 
 
 cudaError_t launch_scan_big(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   if (!big_d(d)) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(float) * (size_t)(DB * RB + KC * DB);
+  const size_t smem = sizeof(float) * (size_t)(DB * RB + 2 * KC * DB);
   cudaError_t e = cudaFuncSetAttribute(k_scan_big, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k_scan_big<<<dim3(DB / RB, 2, d.B * d.H), kThreadsB, smem, s>>>(d, in, w);
