@@ -172,6 +172,32 @@ def test_d256_vda_matches_oracle(shape):
     assert L.vdn_hybrid_attn_fwd(cfg, ha.args(t), check=False) == L.VDN_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("y_bf16,out_mode", [(False, 1), (True, 0), (True, 1)])
+def test_d256_output_options(y_bf16, out_mode):
+    """d = 256 with a caller-given text state, an RMSNorm weight, bf16 y and
+    the summed output: the linear branch (the only one at this size, added
+    into a zeroed y when summed) against the oracle."""
+    shape = Shape(1, 12, 48, 2, 256, 256, 0)
+    r = np.random.default_rng(7)
+    inp = make_inputs(shape, 11, "bf16")
+    for k in ("text_k", "text_v", "text_beta", "text_k_bits", "text_v_bits"):
+        inp.pop(k, None)
+    inp["init_state"] = r.standard_normal((1, 2, 256, 256)).astype(np.float32) * 0.1
+    inp["rms_weight"] = (1 + 0.5 * r.standard_normal((2, 256))).astype(np.float32)
+    cfg = cfg_for(shape, "bf16", out_mode=out_mode, y_dtype=L.VDN_BF16 if y_bf16 else L.VDN_F32)
+    cfg.L = 0
+    t = to_torch(inp, "bf16", "cuda")
+    ha = HybridAttention(cfg)
+    ha.y.zero_()
+    ha(t, stages=VDA)
+    torch.cuda.synchronize()
+    assert L.vdn_hybrid_device_status(cfg, ha.args(t))[0] == L.VDN_OK
+    y = ha.y.float().cpu().numpy().astype(np.float64)
+    ref = oracle(inp, cfg)[..., 1, :]
+    got = y[..., 1, :] if out_mode == 0 else y
+    assert rel_err(got, ref, U_BF16 * np.abs(ref) if y_bf16 else None) <= TOL["bf16"]
+
+
 def test_bf16_read_table_matches_oracle():
     """The read table the tensor-core read consumes (fp32 copy), bf16 mode."""
     w = WORKLOADS["small"]
