@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--workload", default="768p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--vda-only", action="store_true",
+                    help="the Video Delta Attention stages only (the d = 256 sweep shapes have no softmax)")
     return ap.parse_args()
 
 
@@ -231,10 +233,11 @@ def stage_rooflines(s, cfg, ms, y_elem, peaks, sm_mhz):
     hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops_sustained"]
     simt = R.fp32_simt_tflops(sm_mhz)
     out = {"text": {"ms": ms["text"]}}
-    f = R.softmax_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.chunk, cfg.anchors)
-    a = f / (ms["softmax"] / 1e3) / 1e12
-    out["softmax"] = {"ms": ms["softmax"], "bound": "tensor", "achieved": a, "peak": tc, "unit": "TFLOP/s",
-                      "frac": a / tc, "work": f}
+    if "softmax" in ms:
+        f = R.softmax_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.chunk, cfg.anchors)
+        a = f / (ms["softmax"] / 1e3) / 1e12
+        out["softmax"] = {"ms": ms["softmax"], "bound": "tensor", "achieved": a, "peak": tc, "unit": "TFLOP/s",
+                          "frac": a / tc, "work": f}
     for name, by in (("read", R.read_bytes(s.B, s.T, s.N, s.H, s.d_k, elem, y_elem)),
                      ("scan", R.scan_bytes(s.B, s.T, s.H, s.d_k, cfg.chunk, cfg.anchors))):
         a = by / (ms[name] / 1e3) / 1e9
@@ -274,7 +277,7 @@ def run_ours(args):
     w = WORKLOADS[args.workload]
     s = w.shape
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.vda_only:
         val, work, desc = oracle_sample(w, oracle_prepare(w), target_s=12.0)
         cpu = {"value": val, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc,
                "sample_cpu_seconds": round(work, 2)}
@@ -284,23 +287,29 @@ def run_ours(args):
     ha = HybridAttention(cfg, dev)
     stream = torch.cuda.current_stream(dev)
     pre = L.STAGE_TEXT | L.STAGE_SOLVE | L.STAGE_SCAN
+    vda_only = args.vda_only
     # kernels a step launches: text (Gram + sweep on tensor cores, else one
     # SIMT kernel), frame Gram + sweep (else one SIMT solve), scan, softmax,
     # read table + read (else one SIMT read)
     tc = lambda st: L.vdn_hybrid_stage_impl(cfg, st) == 1
     text_k = (2 if tc(L.STAGE_TEXT) else 1) if s.L > 0 else 0  # no text: a memset, no kernel
-    launches_per_step = text_k + (2 if tc(L.STAGE_SOLVE) else 1) + 1 + 1 + (2 if tc(L.STAGE_READ) else 1)
+    launches_per_step = (text_k + (2 if tc(L.STAGE_SOLVE) else 1) + 1 + (0 if vda_only else 1)
+                         + (2 if tc(L.STAGE_READ) else 1))
     K, W = args.steps, args.warmup
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    # the dominant kernel's events: the softmax, or the read in the VDA-only mode
+    dom = L.STAGE_READ if vda_only else L.STAGE_SOFTMAX
 
     def step(i=None):
         ha(t, stages=pre)
         if i is not None:
             ev[i][0].record(stream)
-        ha(t, stages=L.STAGE_SOFTMAX)
+        ha(t, stages=dom)
         if i is not None:
             ev[i][1].record(stream)
-        ha(t, stages=L.STAGE_READ)
+        if not vda_only:
+            ha(t, stages=L.STAGE_READ)
 
     for _ in range(W):
         step()
@@ -344,7 +353,7 @@ def run_ours(args):
         def e2e_step():
             for k, v in host.items():
                 t[k].copy_(v, non_blocking=True)
-            ha(t)
+            ha(t, stages=(pre | L.STAGE_READ) if vda_only else L.STAGE_ALL)
             yh.copy_(ha.y, non_blocking=True)
 
         for _ in range(max(1, W)):
@@ -370,6 +379,8 @@ def run_ours(args):
     stage_ms = {}
     for name, st in (("text", L.STAGE_TEXT), ("solve", L.STAGE_SOLVE), ("scan", L.STAGE_SCAN),
                      ("softmax", L.STAGE_SOFTMAX), ("read", L.STAGE_READ)):
+        if vda_only and st == L.STAGE_SOFTMAX:
+            continue
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ha(t, stages=st)
         a.record(stream)
@@ -381,24 +392,35 @@ def run_ours(args):
 
     if rank == 0:
         peaks, src = load_peaks()
-        flops = softmax_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.chunk, cfg.anchors)
-        achieved = flops / (sm_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        impl = L.vdn_hybrid_stage_impl(cfg, L.STAGE_SOFTMAX)
+        in_gb = 5 * s.B * s.T * s.N * s.H * s.d_k * (2 if w.dtype == "bf16" else 4) / 1e9
+        if vda_only:
+            from video_diffusion_hybrid_b200.roofline import read_bytes
+            by = read_bytes(s.B, s.T, s.N, s.H, s.d_k, 2 if w.dtype == "bf16" else 4, ha.y.element_size())
+            achieved = by / (sm_ms / 1e3) / 1e9
+            roof = {"kernel": "state_read" + ("_tcgen05" if tc(L.STAGE_READ) else "_simt"), "bound": "hbm",
+                    "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "peak_source": f"hbm_gbs ({src})", "ms_per_launch": sm_ms,
+                    "bytes_per_launch": by, "traffic": None}
+        else:
+            flops = softmax_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.chunk, cfg.anchors)
+            achieved = flops / (sm_ms / 1e3) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            impl = L.vdn_hybrid_stage_impl(cfg, L.STAGE_SOFTMAX)
+            roof = {"kernel": "window_softmax" + ("_tcgen05" if impl == 1 else "_simt"), "bound": "tensor",
+                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "peak_source": f"bf16_tflops_sustained ({src})", "ms_per_launch": sm_ms,
+                    "flops_per_launch": flops,
+                    "traffic": kernel_traffic("vdn_softmax_tc.cu" if impl == 1 else "vdn_simt.cu", "window_softmax")}
         line = {
             "metric": METRIC, "value": world * w.tokens / (ms / 1e3), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.name, "B": s.B, "T": s.T, "N": s.N, "H": s.H, "d": s.d_k, "L": s.L,
                        "chunk": 5, "anchors": 4, "state": "fp32", "accumulate": "fp32",
+                       "stages": "vda" if vda_only else "all",
                        "parallelism": f"replicas{world}" if world > 1 else "single",
-                       "l2": "inputs exceed L2 (2.8 GB of q/k/v/gates per step at 768p)"},
-            "roofline": {"kernel": "window_softmax" + ("_tcgen05" if impl == 1 else "_simt"), "bound": "tensor",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"bf16_tflops_sustained ({src})", "ms_per_launch": sm_ms,
-                         "flops_per_launch": flops,
-                         "traffic": kernel_traffic("vdn_softmax_tc.cu" if impl == 1 else "vdn_simt.cu",
-                                                   "window_softmax")},
+                       "l2": f"inputs exceed L2 ({in_gb:.1f} GB of q/k/v/gates per step)"},
+            "roofline": roof,
             "stages": stage_rooflines(s, cfg, stage_ms, ha.y.element_size(), peaks,
                                       (clocks or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)),
             "cpu_baseline": cpu,
