@@ -111,6 +111,18 @@ def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
     return s.B * s.T * s.N / layer, work, desc
 
 
+def max_over_ranks(vals, device=None):
+    """Each value's maximum over the ranks of the process group (the slowest
+    rank defines a step); the values themselves on a single process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    x = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(x, op=dist.ReduceOp.MAX)
+    return x.tolist()
+
+
 def host_cores():
     try:
         import threadpoolctl
@@ -337,10 +349,7 @@ def run_ours(args):
         dist.barrier()
     ms = start.elapsed_time(end) / K
     sm_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    if world > 1:
-        x = torch.tensor([ms, sm_ms], device=dev)
-        dist.all_reduce(x, op=dist.ReduceOp.MAX)
-        ms, sm_ms = x.tolist()
+    ms, sm_ms = max_over_ranks([ms, sm_ms], dev)
 
     # end to end: pinned host inputs -> device, the call, the whole output back,
     # every step.  Two device buffer sets let the upload of step i + 1 (copy
@@ -390,11 +399,7 @@ def run_ours(args):
         pipeline(max(2, W))
         if world > 1:
             dist.barrier()
-        ems = pipeline(K) / K
-        if world > 1:
-            x = torch.tensor([ems], device=dev)
-            dist.all_reduce(x, op=dist.ReduceOp.MAX)
-            ems = x.item()
+        ems = max_over_ranks([pipeline(K) / K], dev)[0]
         e2e = {"value": world * w.tokens / (ems / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": ems,
                "overlap": "upload of step i+1 and download of step i-1 run during step i (3 streams)"}
