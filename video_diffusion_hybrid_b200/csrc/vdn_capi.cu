@@ -26,7 +26,6 @@ vdn_status check_cfg(const vdn_hybrid_cfg* c) {
   if (c->d_v != c->d_k) return VDN_ERR_UNSUPPORTED;
   // d = 256: the per-frame Gram runs on the tensor cores only (bf16 inputs)
   if (c->d_k == 256 && c->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
-  if (c->d_k == 256 && (long long)c->H * 6 > 65535) return VDN_ERR_UNSUPPORTED;
   if (c->chunk != 5) return VDN_ERR_UNSUPPORTED;
   // grid limits of the launches (gridDim.y / gridDim.z <= 65535)
   if ((long long)c->B * c->H > 65535) return VDN_ERR_UNSUPPORTED;

@@ -29,7 +29,9 @@
 // of K or V, the CTA forms X^T (beta X) = A(x, x) and Y^T (beta X), which is
 // the block (y, x) of A (Y from K) or of B (Y from V).  Six CTAs per frame-head
 // cover the eight blocks: (x, Y) = (0, V0): A00 B00; (0, V1): B10; (1, V0):
-// A11 B01; (1, V1): B11; (0, K1): A10; (1, K0): A01.
+// A11 B01; (1, V1): B11; (0, K1): A10; (1, K0): A01.  The four CTAs that do
+// not write X^T (beta X) skip that product (16 MMAs per 16 tokens and
+// frame-head instead of 24), and the six are adjacent in the grid.
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -70,8 +72,10 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
 
   constexpr int DF = BLK ? 2 * D : D;  // row length of k, v and of A_t, B_t
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x, b = blockIdx.z;
-  const int h = BLK ? blockIdx.y / 6 : blockIdx.y, call = BLK ? blockIdx.y % 6 : 0;
+  // block mode: the six CTAs of a frame-head are adjacent in launch order, so
+  // five of them find the frame's k and v in L2
+  const int t = BLK ? blockIdx.x / 6 : blockIdx.x, b = blockIdx.z;
+  const int h = blockIdx.y, call = BLK ? blockIdx.x % 6 : 0;
   // block mode: view columns of X (beta K) and of Y, and where Y^T (beta X) goes
   const int bx = (call == 2 || call == 3 || call == 5) ? 1 : 0;
   const int by = (call == 1 || call == 3 || call == 4) ? 1 : 0;
@@ -126,6 +130,8 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       constexpr uint32_t ID = D == 128 ? (idesc_bf16(128, 128, true) | (1u << 15)) : (idesc_bf16(128, 64, true) | (1u << 15));
       const uint64_t hidesc = sdesc(smem_u32(sHi), TT * 128, 1024), lodesc = sdesc(smem_u32(sLo), TT * 128, 1024);
       const uint64_t kvdesc0 = sdesc(smem_u32(sKV), TT * 128, 1024);
+      // block mode: X^T (beta X) only where the CTA writes it
+      const bool first = !BLK || write_a;
       bool ok = true;
       for (int j = 0; ok && j < ntiles; ++j) {
         const int s = j % ST;
@@ -141,7 +147,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
 #pragma unroll
           for (int k = 0; k < TT / 16; ++k) {
             const uint32_t acc = (j | part | k) ? 1u : 0u;
-            mma_bf16(tmem, dadd(kd, k * 2048), dadd(bd, k * 2048), ID, acc);
+            if (first) mma_bf16(tmem, dadd(kd, k * 2048), dadd(bd, k * 2048), ID, acc);
             if (D == 128) mma_bf16(tmem + 128, dadd(vd, k * 2048), dadd(bd, k * 2048), ID, acc);
           }
         }
@@ -205,10 +211,10 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
         const bool wa = !BLK || write_a;
 #pragma unroll
         for (int q = 0; q < 2 * D / 32; ++q) {
+          if (q < D / 32 && !wa) continue;
           float v[32];
           tmem_ld32(lane_addr + q * 32, v);
           tmem_wait_ld();
-          if (q < D / 32 && !wa) continue;
           float* dst = q < D / 32 ? Ag + q * 32 : Bg + (q - D / 32) * 32;
 #pragma unroll
           for (int i = 0; i < 32; i += 8) st_v8(dst + i, v + i);
@@ -247,7 +253,7 @@ cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t 
   auto kern = k_gram_tc<D, TEXT, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(TEXT ? 1 : d.T, d.H * (BLK ? 6 : 1), d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
+  kern<<<dim3((TEXT ? 1 : d.T) * (BLK ? 6 : 1), d.H, d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
   return cudaGetLastError();
 }
 
@@ -256,7 +262,7 @@ cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t 
 bool gram_tc_supported(const Dims& d) {
   if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128 && d.dk != 256)) return false;
   if ((long long)d.B * d.T * d.N >= (1LL << 31)) return false;
-  if ((long long)d.H * 6 > 65535) return false;
+  if ((long long)d.T * 6 > 0x7FFFFFFFLL) return false;
   return encode_fn() != nullptr;
 }
 

@@ -23,13 +23,16 @@
 //               computes the other tile's product (ping-pong).  S: M=128, N=128,
 //               K=d, both operands from SMEM; PV: A = P from TMEM (TS form).
 //   warps 4..7  softmax of query tile 0, warps 8..11 of query tile 1: thread r
-//               owns row r (= TMEM lane r).  Pass 1 reads its row of S and takes
-//               the max; pass 2 re-reads it in halves, computes P (bf16) and
-//               writes it over the S columns already read.  O is rescaled only
-//               when a row max grew by more than 2^8 (exact: p <= 2^8 then, and
-//               O and the row sum share the same stale max).  The row sum uses
-//               the bf16-rounded P, so every output row is an exact convex
-//               combination of V rows.  Epilogue: O / l, gate, store.
+//               owns row r (= TMEM lane r).  A full key tile after the first
+//               takes one pass: P = 2^(s c - m c) with the running max m, kept
+//               when the row's sum of P is at most 2^8 (then no weight exceeds
+//               2^8).  Otherwise, and for the first and partial tiles, two
+//               passes: the row max, then P.  O is rescaled only when a row max
+//               grew by more than 8 in exp2 units (exact: p <= 2^8 then, and O
+//               and the row sum share the same stale max).  The row sum adds
+//               the bf16-rounded P (mixed bf16 + fp32 adds), so every output
+//               row is an exact convex combination of V rows.  Epilogue:
+//               O / l, gate, store.
 //
 // TMEM (512 columns): O_0 [0,128), O_1 [128,256), S_0 [256,384), S_1 [384,512);
 // P_t lives in the first 64 columns of S_t.  A tile's next S is issued after
@@ -188,6 +191,14 @@ template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16*
   u.x = pack_bf16(a, b);
   u.y = pack_bf16(c, d);
   *reinterpret_cast<uint2*>(p) = u;
+}
+
+// lo and hi halves of a packed bf16 pair added exactly into two fp32 sums
+__device__ __forceinline__ void add_bf16x2_f32(float& s_lo, float& s_hi, uint32_t u) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tadd.rn.f32.bf16 %0, lo, %0;\n\t"
+      "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(s_lo), "+f"(s_hi)
+      : "r"(u));
 }
 
 // ------------------------------------------------------------------ kernel --
@@ -350,14 +361,13 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       bool done = false;
       // Fast path (full key tile after the first): one pass with the running
       // max.  Nothing is stored until the whole row is known not to overflow
-      // (no score more than 2^8 above the running max), so a warp that sees
-      // an overflow redoes the tile on the exact two-pass path below.
+      // (no weight above 2^8), so a warp that sees a possible overflow redoes
+      // the tile on the exact two-pass path below.
       if (j > 0 && kvalid == BN) {
         const float2 c2 = make_float2(c, c), nmc2 = make_float2(-m_used * c, -m_used * c);
-        float2 ps2[4];
+        float ps[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) ps2[u] = make_float2(0.f, 0.f);
-        uint32_t pmax = 0u;  // running max of the packed P (bf16 pairs, all >= 0)
+        for (int u = 0; u < 8; ++u) ps[u] = 0.f;
         float pk0[32], pk1[32];
         // 32 scores at a time; the next chunk's TMEM load is in flight while
         // this chunk computes (a load is complete only after the wait that
@@ -367,8 +377,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
           for (int i = 0; i < 16; ++i) {
             const float2 x = fma2(make_float2(v[2 * i], v[2 * i + 1]), c2, nmc2);
             const uint32_t u = pack_bf16(ex2(x.x), ex2(x.y));
-            pmax = max_bf16x2(pmax, u);
-            ps2[i & 3] = add2(ps2[i & 3], make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u)));
+            add_bf16x2_f32(ps[2 * (i & 3)], ps[2 * (i & 3) + 1], u);
             pk[o + i] = __uint_as_float(u);
           }
         };
@@ -385,15 +394,16 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         chunk(va, pk1, 0);
         tmem_wait_ld();
         chunk(vb, pk1, 16);
-        // overflow: some weight above 2^8, i.e. a score more than 2^8 (in exp2
-        // units) above the running max; the exact path then rescales
-        const float pmx = fmaxf(__uint_as_float(pmax << 16), __uint_as_float(pmax & 0xFFFF0000u));
-        if (!__any_sync(0xffffffffu, !(pmx <= 256.0f))) {
+        // overflow test on the row's sum of P: every P is >= 0 and a rounded
+        // sum of non-negative terms is >= each term, so a sum <= 2^8 proves
+        // that no weight exceeds 2^8; otherwise (some score possibly more
+        // than 8 above the running max, in exp2 units) the exact path decides
+        const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        if (!__any_sync(0xffffffffu, !(psum <= 256.0f))) {
           tmem_st32(scol, pk0);        // P columns [0, 32)
           tmem_st32(scol + 32, pk1);   // P columns [32, 64)
           tmem_wait_st();
-          const float2 t2 = add2(add2(ps2[0], ps2[1]), add2(ps2[2], ps2[3]));
-          l_sum += t2.x + t2.y;
+          l_sum += psum;
           done = true;
         }
       }
