@@ -19,15 +19,19 @@
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma.  Per key tile
 //               j the tensor pipe runs, in this order,
 //                 O_0 += P_0(j) V_j,  S_0 = Q_0 K_{j+1}^T,  O_1 += P_1(j) V_j,  S_1 = Q_1 K_{j+1}^T
+//               where each P V is issued as two 64-key halves, the first as
+//               soon as the softmax has stored that half of P (it then runs
+//               while the softmax computes the second half)
 //               so that while one softmax warpgroup works on its tile the pipe
 //               computes the other tile's product (ping-pong).  S: M=128, N=128,
 //               K=d, both operands from SMEM; PV: A = P from TMEM (TS form).
 //   warps 4..7  softmax of query tile 0, warps 8..11 of query tile 1: thread r
-//               owns row r (= TMEM lane r).  A full key tile after the first
-//               takes one pass: P = 2^(s c - m c) with the running max m, kept
-//               when the row's sum of P is at most 2^8 (then no weight exceeds
-//               2^8).  Otherwise, and for the first and partial tiles, two
-//               passes: the row max, then P.  O is rescaled only when a row max
+//               owns row r (= TMEM lane r), a key tile in two halves of 64
+//               keys.  A full half after the first key tile takes one pass:
+//               P = 2^(s c - m c) with the running max m, kept when the half's
+//               sum of P is at most 2^8 (then no weight exceeds 2^8).
+//               Otherwise, and in the first and partial tiles, two passes over
+//               the half: its max, then P.  O is rescaled only when a row max
 //               grew by more than 8 in exp2 units (exact: p <= 2^8 then, and O
 //               and the row sum share the same stale max).  The row sum adds
 //               the bf16-rounded P (mixed bf16 + fp32 adds), so every output
@@ -35,8 +39,8 @@
 //               O / l, gate, store.
 //
 // TMEM (512 columns): O_0 [0,128), O_1 [128,256), S_0 [256,384), S_1 [384,512);
-// P_t lives in the first 64 columns of S_t.  A tile's next S is issued after
-// its PV by the same thread, and tcgen05.mma operations of one thread run in
+// P_t lives in the first 64 columns of S_t (keys 0..63 in the first 32).  A
+// tile's next S is issued after its PV by the same thread, and tcgen05.mma operations of one thread run in
 // issue order, so P_t(j) is consumed before S_t(j+1) overwrites it.
 //
 // Every mbarrier wait is bounded (about one second of clock cycles); on
@@ -210,8 +214,10 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   constexpr uint32_t QTILE = BM * D * 2;
   constexpr uint32_t KVBYTES = BN * D * 2;
   constexpr int KST = 3, VST = 2;            // K and V ring depths
+  // P_t of a key tile is handed over in two 64-key halves: B_PFULL (keys
+  // 0..63) and B_PFULL2 (64..127); B_OHALF marks O += P_t(j)[:, :64] V_j done
   enum { B_Q = 0, B_KFULL = 1, B_KEMPTY = 4, B_VFULL = 7, B_VEMPTY = 9, B_SFULL = 11, B_PFULL = 13, B_ODONE = 15,
-         B_DRAIN = 17, NBARS = 18 };
+         B_DRAIN = 17, B_PFULL2 = 18, B_OHALF = 20, NBARS = 22 };
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sQ = sm;                    // NQ tiles
@@ -232,7 +238,8 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
 
   if (threadIdx.x == 0) {
     // P_FULL: one arrival per softmax warp
-    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_PFULL || i == B_PFULL + 1) ? 4 : 1);
+    for (int i = 0; i < NBARS; ++i)
+      mbar_init(bar(i), (i == B_PFULL || i == B_PFULL + 1 || i == B_PFULL2 || i == B_PFULL2 + 1) ? 4 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -309,15 +316,20 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         mma_commit(bar(B_SFULL + t));
         if (t == NQ - 1) mma_commit(bar(B_KEMPTY + sk));  // K_j read by both tiles
       };
-      auto mma_pv = [&](int t, int j) {
+      // O_t += P_t(j)[:, 64 h : 64 h + 64] V_j[64 h : 64 h + 64, :]
+      auto mma_pv = [&](int t, int j, int h) {
         const int sv = j % VST;
         const uint64_t vd = dadd(vdesc0, sv * KVBYTES);
         const uint32_t dst = tmem + col_o(t), pa = tmem + col_s(t);
-        mma_bf16_ts(dst, pa, vd, ID_O, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int k = 1; k < BN / 16; ++k) mma_bf16_ts(dst, pa + 8 * k, dadd(vd, k * 16 * 128), ID_O, 1u);
-        mma_commit(bar(B_ODONE + t));
-        if (t == NQ - 1) mma_commit(bar(B_VEMPTY + sv));  // V_j read by both tiles
+        for (int k = 4 * h; k < 4 * h + 4; ++k)
+          mma_bf16_ts(dst, pa + 8 * k, dadd(vd, k * 16 * 128), ID_O, (j > 0 || k > 0) ? 1u : 0u);
+        if (h == 0) {
+          mma_commit(bar(B_OHALF + t));
+        } else {
+          mma_commit(bar(B_ODONE + t));
+          if (t == NQ - 1) mma_commit(bar(B_VEMPTY + sv));  // V_j read by both tiles
+        }
       };
       bool ok = mbar_wait(bar(B_Q), 0, ctl) && mbar_wait(bar(B_KFULL), 0, ctl);
       if (ok) {
@@ -329,11 +341,15 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         const bool more = j + 1 < ntiles;
         for (int t = 0; ok && t < NQ; ++t) {
           ok = mbar_wait(bar(B_PFULL + t), j & 1, ctl) &&
-               (t > 0 || mbar_wait(bar(B_VFULL + j % VST), (j / VST) & 1, ctl)) &&
+               (t > 0 || mbar_wait(bar(B_VFULL + j % VST), (j / VST) & 1, ctl));
+          if (!ok) break;
+          tc_fence_after();
+          mma_pv(t, j, 0);
+          ok = mbar_wait(bar(B_PFULL2 + t), j & 1, ctl) &&
                (t > 0 || !more || mbar_wait(bar(B_KFULL + (j + 1) % KST), ((j + 1) / KST) & 1, ctl));
           if (!ok) break;
           tc_fence_after();
-          mma_pv(t, j);
+          mma_pv(t, j, 1);
           if (more) mma_s(t, j + 1);
         }
       }
@@ -352,145 +368,119 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
     const float thresh = kRescaleLog2 / c;            // raw-score units
     float m_used = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; ok && j < ntiles; ++j) {
       // every TMEM access below is warp-collective: keep control flow warp-uniform
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + t), j & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       int k0, kvalid;
       key_tile(tile, j, k0, kvalid);
-      bool done = false;
-      // Fast path (full key tile after the first): one pass with the running
-      // max.  Nothing is stored until the whole row is known not to overflow
-      // (no weight above 2^8), so a warp that sees a possible overflow redoes
-      // the tile on the exact two-pass path below.
-      if (j > 0 && kvalid == BN) {
-        const float2 c2 = make_float2(c, c), nmc2 = make_float2(-m_used * c, -m_used * c);
-        float ps[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-        float pk0[32], pk1[32];
-        // 32 scores at a time; the next chunk's TMEM load is in flight while
-        // this chunk computes (a load is complete only after the wait that
-        // follows the computation)
-        auto chunk = [&](const float (&v)[32], float (&pk)[32], int o) {
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t sh = scol + 64 * h;  // scores of keys [64 h, 64 h + 64)
+        const int kvh = kvalid - 64 * h;    // valid keys of this half (may be <= 0)
+        bool done = false;
+        // Fast path (a full half after the first key tile): one pass with the
+        // running max, kept when the half's sum of P is at most 2^8 (a rounded
+        // sum of non-negative terms bounds each term, so no weight exceeds 2^8).
+        if (j > 0 && kvh >= 64) {
+          const float2 c2 = make_float2(c, c), nmc2 = make_float2(-m_used * c, -m_used * c);
+          float ps[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 x = fma2(make_float2(v[2 * i], v[2 * i + 1]), c2, nmc2);
-            const uint32_t u = pack_bf16(ex2(x.x), ex2(x.y));
-            add_bf16x2_f32(ps[2 * (i & 3)], ps[2 * (i & 3) + 1], u);
-            pk[o + i] = __uint_as_float(u);
-          }
-        };
-        float va[32], vb[32];
-        tmem_ld32(scol, va);
-        tmem_wait_ld();
-        tmem_ld32(scol + 32, vb);
-        chunk(va, pk0, 0);
-        tmem_wait_ld();
-        tmem_ld32(scol + 64, va);
-        chunk(vb, pk0, 16);
-        tmem_wait_ld();
-        tmem_ld32(scol + 96, vb);
-        chunk(va, pk1, 0);
-        tmem_wait_ld();
-        chunk(vb, pk1, 16);
-        // overflow test on the row's sum of P: every P is >= 0 and a rounded
-        // sum of non-negative terms is >= each term, so a sum <= 2^8 proves
-        // that no weight exceeds 2^8; otherwise (some score possibly more
-        // than 8 above the running max, in exp2 units) the exact path decides
-        const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        if (!__any_sync(0xffffffffu, !(psum <= 256.0f))) {
-          tmem_st32(scol, pk0);        // P columns [0, 32)
-          tmem_st32(scol + 32, pk1);   // P columns [32, 64)
-          tmem_wait_st();
-          l_sum += psum;
-          done = true;
-        }
-      }
-      if (!done) {
-        // Exact path: pass 1 takes the row max, O is rescaled if it grew by
-        // more than 2^8, pass 2 computes and stores P.
-        // pass 1: row max (eight independent chains)
-        float pm[8];
-  #pragma unroll
-        for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
-  #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float v0[32], v1[32];
-          tmem_ld32(scol + 64 * hf, v0);
-          tmem_ld32(scol + 64 * hf + 32, v1);
-          tmem_wait_ld();
-  #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c0 = 64 * hf + i, c1 = 64 * hf + 32 + i;
-            pm[i & 7] = fmaxf(pm[i & 7], c0 < kvalid ? v0[i] : -INFINITY);
-            pm[i & 7] = fmaxf(pm[i & 7], c1 < kvalid ? v1[i] : -INFINITY);
-          }
-        }
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        // lazy rescale decision: only rows whose max grew by more than 2^8
-        const bool need = mx > m_used + thresh;
-        float f = 1.0f;
-        if (need) {
-          f = (m_used == -INFINITY) ? 0.f : ex2((m_used - mx) * c);
-          l_sum *= f;
-          m_used = mx;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O is stable once O += P(j-1) V(j-1) has completed
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(B_ODONE + t), (j - 1) & 1, ctl))) { ok = false; break; }
-          tc_fence_after();
-          float v[32];
-  #pragma unroll
-          for (int q = 0; q < D / 32; ++q) {
-            tmem_ld32(ocol + q * 32, v);
-            tmem_wait_ld();
-  #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= f;
-            tmem_st32(ocol + q * 32, v);
-          }
-          tmem_wait_st();
-        }
-        // pass 2: P = exp2(s c - m c) in bf16, written over the S columns already read
-        const float mc = m_used * c;
-        float ps[8];
-  #pragma unroll
-        for (int u = 0; u < 8; ++u) ps[u] = 0.f;
-  #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float v0[32], v1[32];
-          tmem_ld32(scol + 64 * hf, v0);
-          tmem_ld32(scol + 64 * hf + 32, v1);
-          tmem_wait_ld();
+          for (int u = 0; u < 8; ++u) ps[u] = 0.f;
           float pk[32];
-  #pragma unroll
+          auto chunk = [&](const float (&v)[32], int o) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 x = fma2(make_float2(v[2 * i], v[2 * i + 1]), c2, nmc2);
+              const uint32_t u = pack_bf16(ex2(x.x), ex2(x.y));
+              add_bf16x2_f32(ps[2 * (i & 3)], ps[2 * (i & 3) + 1], u);
+              pk[o + i] = __uint_as_float(u);
+            }
+          };
+          float va[32], vb[32];
+          tmem_ld32(sh, va);
+          tmem_wait_ld();
+          tmem_ld32(sh + 32, vb);
+          chunk(va, 0);
+          tmem_wait_ld();
+          chunk(vb, 16);
+          const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+          if (!__any_sync(0xffffffffu, !(psum <= 256.0f))) {
+            tmem_st32(scol + 32 * h, pk);  // P columns [32 h, 32 h + 32): keys of this half
+            l_sum += psum;
+            done = true;
+          }
+        }
+        if (!done) {
+          // Exact path on the half: its max, O rescaled if the row max grew by
+          // more than 8 (exp2 units), then P.
+          float v0[32], v1[32];
+          tmem_ld32(sh, v0);
+          tmem_ld32(sh + 32, v1);
+          tmem_wait_ld();
+          float pm[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            pm[i & 7] = fmaxf(pm[i & 7], i < kvh ? v0[i] : -INFINITY);
+            pm[i & 7] = fmaxf(pm[i & 7], 32 + i < kvh ? v1[i] : -INFINITY);
+          }
+          const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+          const bool need = mx > m_used + thresh;
+          float f = 1.0f;
+          if (need) {
+            f = (m_used == -INFINITY) ? 0.f : ex2((m_used - mx) * c);
+            l_sum *= f;
+            m_used = mx;
+          }
+          // O holds products already issued: those of key tile j - 1 (h = 0) or
+          // the first half of tile j (h = 1); rescale once they are complete
+          if ((j > 0 || h == 1) && __any_sync(0xffffffffu, need)) {
+            const bool st = h == 0 ? mbar_wait(bar(B_ODONE + t), (j - 1) & 1, ctl)
+                                   : mbar_wait(bar(B_OHALF + t), j & 1, ctl);
+            if (!__all_sync(0xffffffffu, st)) { ok = false; break; }
+            tc_fence_after();
+            float v[32];
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+              tmem_ld32(ocol + q * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] *= f;
+              tmem_st32(ocol + q * 32, v);
+            }
+            tmem_wait_st();
+          }
+          const float mc = m_used * c;
+          float ps[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ps[u] = 0.f;
+          float pk[32];
+#pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int c0 = 64 * hf + 2 * i;
-            const float p0 = c0 < kvalid ? ex2(fmaf(v0[2 * i], c, -mc)) : 0.f;
-            const float p1 = c0 + 1 < kvalid ? ex2(fmaf(v0[2 * i + 1], c, -mc)) : 0.f;
+            const float p0 = 2 * i < kvh ? ex2(fmaf(v0[2 * i], c, -mc)) : 0.f;
+            const float p1 = 2 * i + 1 < kvh ? ex2(fmaf(v0[2 * i + 1], c, -mc)) : 0.f;
             const uint32_t u = pack_bf16(p0, p1);
-            ps[(2 * i) & 7] += __uint_as_float(u << 16);
-            ps[(2 * i + 1) & 7] += __uint_as_float(u & 0xFFFF0000u);
+            add_bf16x2_f32(ps[2 * (i & 3)], ps[2 * (i & 3) + 1], u);
             pk[i] = __uint_as_float(u);
           }
-  #pragma unroll
+#pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int c0 = 64 * hf + 32 + 2 * i;
-            const float p0 = c0 < kvalid ? ex2(fmaf(v1[2 * i], c, -mc)) : 0.f;
-            const float p1 = c0 + 1 < kvalid ? ex2(fmaf(v1[2 * i + 1], c, -mc)) : 0.f;
+            const float p0 = 32 + 2 * i < kvh ? ex2(fmaf(v1[2 * i], c, -mc)) : 0.f;
+            const float p1 = 32 + 2 * i + 1 < kvh ? ex2(fmaf(v1[2 * i + 1], c, -mc)) : 0.f;
             const uint32_t u = pack_bf16(p0, p1);
-            ps[(2 * i) & 7] += __uint_as_float(u << 16);
-            ps[(2 * i + 1) & 7] += __uint_as_float(u & 0xFFFF0000u);
+            add_bf16x2_f32(ps[2 * (i & 3)], ps[2 * (i & 3) + 1], u);
             pk[16 + i] = __uint_as_float(u);
           }
-          tmem_st32(scol + 32 * hf, pk);  // P columns [32 hf, 32 hf + 32) of this tile
+          tmem_st32(scol + 32 * h, pk);
+          l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         }
         tmem_wait_st();
-        l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        tc_fence_before();
+        mbar_arrive_warp(bar(h == 0 ? B_PFULL + t : B_PFULL2 + t));
       }
-      tc_fence_before();
-      mbar_arrive_warp(bar(B_PFULL + t));
     }
     // ---- epilogue: O / l, gate, store
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_ODONE + t), (ntiles - 1) & 1, ctl))) {
@@ -563,7 +553,7 @@ cudaError_t launch_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream
   if (!make_token_map(&mq, in.q, tokens, d.H, D, BM) || !make_token_map(&mk, in.k, tokens, d.H, D, BN) ||
       !make_token_map(&mv, in.v, tokens, d.H, D, BN))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + (size_t)NQ * BM * D * 2 + 5 * (size_t)BN * D * 2 + 18 * 8 + 16;
+  const size_t smem = 1024 + (size_t)NQ * BM * D * 2 + 5 * (size_t)BN * D * 2 + 22 * 8 + 16;
   auto kern = k_softmax_tc<D, To>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
