@@ -259,6 +259,113 @@ static __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------------- CTA pairs (2-SM) --
+// A cluster of two CTAs on neighbouring SMs can run one product as
+// tcgen05.mma.cta_group::2: the A rows and the B columns (N) are split
+// between the two CTAs' shared memory, and each CTA's TMEM holds its rows of
+// the accumulator.  Every tcgen05 instruction of such a kernel (alloc,
+// dealloc, mma, commit) uses cta_group::2.
+static __device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared::cta offset in CTA `rank`
+static __device__ __forceinline__ uint32_t map_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// One arrival per warp on a barrier of either CTA, with the default
+// (CTA-scope release) semantics: what the waiter's MMA reads in this CTA's
+// shared memory is read by this SM's own tensor core, ordered by the
+// fence.proxy.async that precedes the arrival.  (A cluster-scope release
+// measured about 1,700 cycles per arrival.)
+static __device__ __forceinline__ void arrive_cluster_warp(uint32_t caddr) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+static __device__ __forceinline__ bool mbar_try_cl(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+static __device__ __forceinline__ bool mbar_test_cl(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (arrivals may come from the peer
+// CTA).  Gives up after ~1 s, when another role of this CTA gave up, or once
+// any CTA of the launch has recorded a timeout, so that a failing pair ends
+// quickly and both CTAs still reach their final cluster barrier.
+static __device__ __noinline__ bool mbar_wait_cl_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
+  const long long t0 = clock64();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_cl(bar, parity)) return true;
+    if ((it & 255u) == 255u) {
+      if (*c.abort || *reinterpret_cast<volatile uint32_t*>(c.status) != 0u) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *c.abort = 1;
+        atomicOr(c.status, 1u);
+        atomicExch(c.status + 1, c.tag);
+        return false;
+      }
+    }
+  }
+}
+static __device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity, const Ctl& c) {
+  return mbar_test_cl(bar, parity) || mbar_wait_cl_slow(bar, parity, c);
+}
+// all threads of both CTAs; nothing may return early before it
+static __device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA into this CTA's shared memory, bytes counted on a barrier of either
+// CTA of the pair (no multicast)
+static __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cl, int x,
+                                                        int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cl), "r"(x), "r"(y)
+      : "memory");
+}
+static __device__ __forceinline__ void mma2_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// one arrival on a barrier of either CTA once this thread's earlier MMAs are done
+static __device__ __forceinline__ void commit2(uint32_t bar_cl) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cl)
+               : "memory");
+}
+static __device__ __forceinline__ void tmem_alloc2(uint32_t slot_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+static __device__ __forceinline__ void tmem_free2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
 // ------------------------------------------------------------------ host --
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
 // against libcuda); nullptr when no driver is present.

@@ -9,26 +9,34 @@
 //   forward  slot j : frames < min(5j, T)      (slot 0 = start state)
 //   backward slot j : frames >= min(5j, T)     (slot C = start state)
 //
-// Rows of S evolve independently, but a whole 128-row state is exactly one
-// M = 128 tcgen05 tile, so one CTA carries one chain and each step is one
-// 128 x 128 x 128 product S M_t.  fp32 accuracy comes from the bf16 hi/lo
-// split of both factors (x = hi + lo with hi = bf16(x), lo = bf16(x - hi)):
+// Rows of S evolve independently (each row is its own affine recurrence), so
+// a chain is carried by a pair of CTAs on neighbouring SMs (a cluster of
+// two), each holding 64 of the 128 state rows.  Each step is one
+// tcgen05.mma.cta_group::2 product S M_t with M = 128 (64 rows per CTA) and
+// N = 128 (each CTA holds 64 of M_t's rows as its half of B, so M_t crosses
+// from memory once per pair).  fp32 accuracy comes from the bf16 hi/lo split
+// of both factors (x = hi + lo with hi = bf16(x), lo = bf16(x - hi)):
 //   S M ~ S_hi M_hi + S_hi M_lo + S_lo M_hi
 // which keeps about 16 significant bits per step; M_t's split is written by
 // the solve, S's by this kernel's epilogue.  M_t is symmetric (the inverse
-// of an SPD matrix), so its rows serve as the K-major B operand.
+// of an SPD matrix), so its rows serve as the K-major B operand.  Two SMs per
+// chain double the SMs a batch of chains occupies and halve each SM's
+// product and epilogue per step.
 //
-// Roles (384 threads, one CTA per chain; the two directions of a head read
-// the same M_t, C_t, in opposite orders):
-//   warp 0      TMA producer: M_t split (64 KB) once the previous product is
-//               done, C_t (fp32, 64 KB) once the previous epilogue has read it.
-//   warp 1      TMEM allocator; lane 0 issues the 24 MMAs of S M_t.
-//   warps 4..11 epilogue, one state row per thread (= TMEM lane) and half
-//               of the columns per warp (warps w and w + 4 share the lanes of
-//               one 32-row quarter): S = alpha_t (S M_t) + C_t in fp32,
-//               chunk-boundary snapshots to global memory, and the new S
-//               split back into the A operand.
-// Everything is single-buffered: each step depends on the one before.
+// Roles (384 threads per CTA; the two directions of a head read the same
+// M_t, C_t, in opposite orders):
+//   warp 0      TMA producer (both CTAs): this CTA's half of M_t's split once
+//               the previous product is done (bytes counted on the leader's
+//               barrier), its 64 rows of C_t once its epilogue has read them.
+//   warp 1      TMEM allocator (both CTAs); lane 0 of the leader (rank 0)
+//               issues the 24 MMAs of S M_t for the pair.
+//   warps 4..11 epilogue (both CTAs): accumulator layout of a 64-row CTA
+//               share, TMEM lane l = row (l mod 64), column half (l / 64);
+//               warps w and w + 4 take 32 columns each.  S = alpha_t (S M_t)
+//               + C_t in fp32, chunk-boundary snapshots to global memory, and
+//               the new S split back into the A operand.
+// M_t and C_t are double-buffered, so the copies for step i + 1 overlap step
+// i; S is single-buffered (each step depends on the one before).
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -36,13 +44,18 @@ namespace {
 using namespace tc;
 
 constexpr int D = 128;
+constexpr int R = 64;                    // state rows per CTA
 constexpr int kThreadsScan = 384;
-constexpr uint32_t CHUNK = D * 128;      // 64 K-columns of a 128-row bf16 operand (SW128): 16 KB
-constexpr uint32_t OPBYTES = 2 * CHUNK;  // one 128 x 128 bf16 operand
-constexpr uint32_t SPLIT = 2 * OPBYTES;  // hi then lo: 64 KB
-constexpr uint32_t CBOX = D * 128;       // 32 fp32 columns x 128 rows (SW128): 16 KB
-constexpr uint32_t CBYTES = 4 * CBOX;    // C_t: 64 KB
-enum { B_BFULL = 0, B_CFULL = 1, B_SREADY = 2, B_MDONE = 3, B_DRAIN = 4, NBARS = 5 };
+constexpr uint32_t CHUNK = R * 128;      // 64 K-columns of a 64-row bf16 operand (SW128): 8 KB
+constexpr uint32_t OPBYTES = 2 * CHUNK;  // one 64 x 128 bf16 operand
+constexpr uint32_t SPLIT = 2 * OPBYTES;  // hi then lo: 32 KB
+constexpr uint32_t CBOX = R * 128;       // 32 fp32 columns x 64 rows (SW128): 8 KB
+constexpr uint32_t CBYTES = 4 * CBOX;    // this CTA's rows of C_t: 32 KB
+constexpr uint32_t kTmemScan = 64;       // accumulator columns (64 rows x 128 as 128 lanes x 64)
+// M_t and C_t are double-buffered (slot = step & 1).  SREADY lives on the
+// leader (one arrival per epilogue warp of both CTAs); BEMPTY is committed by
+// the leader's MMAs to both CTAs; CEMPTY takes this CTA's eight warps.
+enum { B_BFULL = 0, B_CFULL = 2, B_BEMPTY = 4, B_CEMPTY = 6, B_SREADY = 8, B_MDONE = 9, B_DRAIN = 10, NBARS = 11 };
 
 __device__ __forceinline__ int frame_at(const Dims& d, int dir, int st) { return dir == 0 ? st : d.T - 1 - st; }
 
@@ -102,11 +115,9 @@ __device__ __forceinline__ void store_row32(float* dst, const float* s) {
   for (int u = 0; u < 4; ++u) st_global_v8(dst + 8 * u, s + 8 * u);
 }
 
-// 32 consecutive state values of `row` (columns 32q..32q+31): into the
-// snapshot slots, and split into the A operand.
-__device__ __forceinline__ void emit_chunk(const Dims& dm, int dir, const Slots& sl, float* snap_row, int q, int row,
-                                           unsigned char* sA, const float (&s)[32]) {
-  const long long DD = (long long)D * D;
+// 32 consecutive state values (columns 32q..32q+31) of the row at `row` of
+// this CTA's 64-row share, split into the A operand.
+__device__ __forceinline__ void split_chunk(int q, int row, unsigned char* sA, const float (&s)[32]) {
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int k0 = q * 32 + 8 * e;
@@ -121,6 +132,12 @@ __device__ __forceinline__ void emit_chunk(const Dims& dm, int dir, const Slots&
     *reinterpret_cast<uint4*>(sA + off) = make_uint4(h[0], h[1], h[2], h[3]);
     *reinterpret_cast<uint4*>(sA + OPBYTES + off) = make_uint4(l[0], l[1], l[2], l[3]);
   }
+}
+
+// ... and into the snapshot slots the scan positions it stands for take.
+__device__ __forceinline__ void snap_chunk(const Dims& dm, int dir, const Slots& sl, float* snap_row, int q,
+                                           const float (&s)[32]) {
+  const long long DD = (long long)D * D;
   if (sl.a >= 0) store_row32(snap_row + sl.a * DD + q * 32, s);
   if (sl.b >= 0) store_row32(snap_row + sl.b * DD + q * 32, s);
   for (int p = sl.p0; p < sl.p1; ++p) {
@@ -129,56 +146,68 @@ __device__ __forceinline__ void emit_chunk(const Dims& dm, int dir, const Slots&
   }
 }
 
-__global__ void __launch_bounds__(kThreadsScan, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsScan, 1)
 k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, const __grid_constant__ CUtensorMap tmc) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sA = sm;            // S  hi | lo, K-major SW128
-  unsigned char* sB = sA + SPLIT;    // M_t hi | lo, K-major SW128
-  unsigned char* sC = sB + SPLIT;    // C_t fp32, 4 boxes of 32 columns, SW128
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + CBYTES);
+  unsigned char* sA = sm;            // this CTA's rows of S, hi | lo, K-major SW128
+  unsigned char* sB = sA + SPLIT;    // 2 slots: this CTA's half of M_t (64 rows), hi | lo, K-major SW128
+  unsigned char* sC = sB + 2 * SPLIT;  // 2 slots: this CTA's rows of C_t, fp32, 4 boxes of 32 columns, SW128
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + 2 * CBYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
-  const int dir = blockIdx.x & 1, bh = blockIdx.x >> 1;
+  // no early exit: both CTAs of the pair must reach the cluster barriers
+  const uint32_t rank = cta_rank();
+  const bool lead = rank == 0;
+  const int chain = blockIdx.x >> 1;
+  const int dir = chain & 1, bh = chain >> 1;
   const int b = bh / dm.H, h = bh % dm.H;
+  const int row0 = R * (int)rank;  // first state row of this CTA
   const Ctl ctl{abort_flag, w.status, (unsigned)TAG_SCAN_TC};
   auto bar = [&](int i) { return smem_u32(bars + i); };
+  auto lbar = [&](int i) { return map_rank(smem_u32(bars + i), 0); };
   auto fh_of = [&](int t) { return ((long long)b * dm.T + t) * dm.H + h; };
   int nw = 0;  // written frames
   for (int t = 0; t < dm.T; ++t) nw += is_anchor(dm, t) ? 0 : 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(B_BFULL), 1);
-    mbar_init(bar(B_CFULL), 1);
-    mbar_init(bar(B_SREADY), 8);  // one arrival per epilogue warp
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(bar(B_BFULL + k), 1);
+      mbar_init(bar(B_CFULL + k), 1);
+      mbar_init(bar(B_BEMPTY + k), 1);
+      mbar_init(bar(B_CEMPTY + k), 8);  // one arrival per epilogue warp of this CTA
+    }
+    mbar_init(bar(B_SREADY), 16);  // one arrival per epilogue warp of the pair
     mbar_init(bar(B_MDONE), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 128);
+  if (warp == 1) tmem_alloc2(smem_u32(tmem_slot), kTmemScan);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Phases: BFULL, CFULL and MDONE complete once per written step i; SREADY
-  // once for the start state and once per step, so step i's MMA waits for
-  // SREADY phase i.  No role can run two phases ahead of a waiter.
+  // Phases: MDONE completes once per written step i, SREADY once for the
+  // start state and once per step (step i's MMA waits for phase i); a slot's
+  // FULL and EMPTY barriers once per use of the slot (step i uses slot i & 1,
+  // its (i >> 1)-th use).  No role can run two phases ahead of a waiter.
   if (warp == 0) {
     if (lane == 0) {
       int nb = 0, nc = 0;
-      // M_t, C_t of the step two ahead are pulled into L2 early, so that the
-      // single-buffered loads below (issued only when their buffer frees) run
-      // at L2 rather than HBM latency
+      // this CTA's halves of M_t, C_t of the step two ahead are pulled into
+      // L2 early, so that the single-buffered loads below (issued only when
+      // their buffer frees) run at L2 rather than HBM latency
       auto prefetch_step = [&](int pst) {
         if (pst >= dm.T) return;
         const long long pfh = fh_of(frame_at(dm, dir, pst));
-        prefetch_l2(static_cast<const __nv_bfloat16*>(w.M16) + pfh * 2 * D * D, SPLIT);
-        prefetch_l2(w.Cm + pfh * D * D, CBYTES);
+        const __nv_bfloat16* m16 = static_cast<const __nv_bfloat16*>(w.M16);
+        prefetch_l2(m16 + ((pfh * 2) * D + row0) * D, OPBYTES);
+        prefetch_l2(m16 + ((pfh * 2 + 1) * D + row0) * D, OPBYTES);
+        prefetch_l2(w.Cm + (pfh * D + row0) * D, CBYTES);
       };
       int st = next_written(dm, dir, 0);
       int pst = st;
@@ -189,103 +218,123 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
         const long long fh = fh_of(frame_at(dm, dir, st));
         pst = next_written(dm, dir, pst + 1);
         prefetch_step(pst);
-        if (i > 0 && !mbar_wait(bar(B_MDONE), (i - 1) & 1, ctl)) break;  // B free
-        mbar_expect_tx(bar(B_BFULL), SPLIT);
+        const int slot = i & 1;
+        // slot free: the product (B) and this CTA's epilogue (C) of step i - 2 are done
+        if (i >= 2 && !mbar_wait_cl(bar(B_BEMPTY + slot), ((i - 2) >> 1) & 1, ctl)) break;
+        if (lead) mbar_expect_tx(bar(B_BFULL + slot), 2 * SPLIT);
         for (int part = 0; part < 2; ++part)
           for (int c = 0; c < 2; ++c)
-            tma_load_2d(smem_u32(sB + part * OPBYTES + c * CHUNK), &tmm, bar(B_BFULL), c * 64,
-                        (int)((fh * 2 + part) * D));
+            tma_load_2d_pair(smem_u32(sB + slot * SPLIT + part * OPBYTES + c * CHUNK), &tmm, lbar(B_BFULL + slot),
+                             c * 64, (int)((fh * 2 + part) * D + row0));
         ++nb;
-        if (i > 0 && !mbar_wait(bar(B_SREADY), i & 1, ctl)) break;  // C read by the previous epilogue
-        mbar_expect_tx(bar(B_CFULL), CBYTES);
-        for (int c = 0; c < 4; ++c) tma_load_2d(smem_u32(sC + c * CBOX), &tmc, bar(B_CFULL), c * 32, (int)(fh * D));
+        if (i >= 2 && !mbar_wait_cl(bar(B_CEMPTY + slot), ((i - 2) >> 1) & 1, ctl)) break;
+        mbar_expect_tx(bar(B_CFULL + slot), CBYTES);
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(smem_u32(sC + slot * CBYTES + c * CBOX), &tmc, bar(B_CFULL + slot), c * 32,
+                      (int)(fh * D + row0));
         ++nc;
       }
-      // the last copies land before the CTA can exit
-      if (nb > 0) wait_own(bar(B_BFULL), (nb - 1) & 1);
-      if (nc > 0) wait_own(bar(B_CFULL), (nc - 1) & 1);
+      // the last copies land before the pair can exit (the leader's B
+      // barriers count both CTAs' bytes)
+      for (int n = nb - 2 < 0 ? 0 : nb - 2; lead && n < nb; ++n) wait_own(bar(B_BFULL + (n & 1)), (n >> 1) & 1);
+      for (int n = nc - 2 < 0 ? 0 : nc - 2; n < nc; ++n) wait_own(bar(B_CFULL + (n & 1)), (n >> 1) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t ID = idesc_bf16(128, D, false);
+    if (lane == 0 && lead) {
+      constexpr uint32_t ID = idesc_bf16(2 * R, D, false);  // M = 128 over the pair, N = 128
       const uint64_t a0 = sdesc(smem_u32(sA), 16, 1024), b0 = sdesc(smem_u32(sB), 16, 1024);
       for (int i = 0; i < nw; ++i) {
-        if (!mbar_wait(bar(B_SREADY), i & 1, ctl)) break;
-        if (!mbar_wait(bar(B_BFULL), i & 1, ctl)) break;
+        const int slot = i & 1;
+        if (!mbar_wait_cl(bar(B_SREADY), i & 1, ctl)) break;
+        if (!mbar_wait_cl(bar(B_BFULL + slot), (i >> 1) & 1, ctl)) break;
         tc_fence_after();
+        const uint64_t bs = dadd(b0, slot * SPLIT);
 #pragma unroll
         for (int pass = 0; pass < 3; ++pass) {  // hi hi, hi lo, lo hi
           const uint32_t ao = pass == 2 ? OPBYTES : 0u, bo = pass == 1 ? OPBYTES : 0u;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_bf16(tmem, dadd(a0, ao + (k >> 2) * CHUNK + (k & 3) * 32),
-                     dadd(b0, bo + (k >> 2) * CHUNK + (k & 3) * 32), ID, (pass | k) ? 1u : 0u);
+            mma2_bf16(tmem, dadd(a0, ao + (k >> 2) * CHUNK + (k & 3) * 32),
+                      dadd(bs, bo + (k >> 2) * CHUNK + (k & 3) * 32), ID, (pass | k) ? 1u : 0u);
         }
-        mma_commit(bar(B_MDONE));
+        commit2(bar(B_MDONE));
+        commit2(map_rank(bar(B_MDONE), 1));
+        commit2(bar(B_BEMPTY + slot));
+        commit2(map_rank(bar(B_BEMPTY + slot), 1));
       }
-      mma_commit(bar(B_DRAIN));
+      commit2(bar(B_DRAIN));
       wait_own(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
-    const int quad = warp & 3, half = (warp - 4) >> 2, row = quad * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + half * 64;
+    const int quad = warp & 3, half = (warp - 4) >> 2;
+    const int tl = quad * 32 + lane;             // TMEM lane
+    const int srow = tl & (R - 1), ch = tl >> 6;  // row of this CTA's share, column half
+    const int q = 2 * ch + half;                  // this thread's 32 columns: 32q .. 32q + 31
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16) + half * 32;
     const long long DD = (long long)D * D;
+    const int row = row0 + srow;  // state row
     float* snap_row = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD + (long long)row * D;
     // start state: its own slot, then the slots of leading unwritten frames
     int st = next_written(dm, dir, 0);
     {
       const float* src = w.half_text + (long long)bh * DD + (long long)row * D;
       const int start_slot = dir == 0 ? 0 : dm.C;
-#pragma unroll 1
-      for (int q = 2 * half; q < 2 * half + 2; ++q) {
-        float s[32];
+      float s[32];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(src + q * 32) + u);
-          s[4 * u] = v.x; s[4 * u + 1] = v.y; s[4 * u + 2] = v.z; s[4 * u + 3] = v.w;
-        }
-        store_row32(snap_row + start_slot * DD + q * 32, s);
-        emit_chunk(dm, dir, slots_of(dm, dir, 0, st), snap_row, q, row, sA, s);
+      for (int u = 0; u < 8; ++u) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(src + q * 32) + u);
+        s[4 * u] = v.x; s[4 * u + 1] = v.y; s[4 * u + 2] = v.z; s[4 * u + 3] = v.w;
       }
+      split_chunk(q, srow, sA, s);
+      fence_proxy_async_smem();
+      arrive_cluster_warp(lbar(B_SREADY));
+      store_row32(snap_row + start_slot * DD + q * 32, s);
+      snap_chunk(dm, dir, slots_of(dm, dir, 0, st), snap_row, q, s);
     }
-    fence_proxy_async_smem();
-    mbar_arrive_warp(bar(B_SREADY));
     for (int i = 0; i < nw; ++i) {
+      const int slot = i & 1;
       const int st_next = next_written(dm, dir, st + 1);
       const float alpha = __ldg(in.alpha + fh_of(frame_at(dm, dir, st)));
       const Slots sl = slots_of(dm, dir, st, st_next);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MDONE), i & 1, ctl))) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_CFULL), i & 1, ctl))) break;
+      // this step's C row chunk into registers first (it does not depend on
+      // the product), then the slot goes back to the producer
+      if (!__all_sync(0xffffffffu, mbar_wait_cl(bar(B_CFULL + slot), (i >> 1) & 1, ctl))) break;
+      float cv[32];
+      {
+        const unsigned char* crow = sC + slot * CBYTES + q * CBOX + srow * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 c4 = *reinterpret_cast<const float4*>(crow + ((u ^ (srow & 7)) << 4));
+          cv[4 * u] = c4.x; cv[4 * u + 1] = c4.y; cv[4 * u + 2] = c4.z; cv[4 * u + 3] = c4.w;
+        }
+      }
+      mbar_arrive_warp(bar(B_CEMPTY + slot));
+      if (!__all_sync(0xffffffffu, mbar_wait_cl(bar(B_MDONE), i & 1, ctl))) break;
       tc_fence_after();
-      float v[2][32];
-      tmem_ld32(lane_addr, v[0]);
-      tmem_ld32(lane_addr + 32, v[1]);
+      float v[32];
+      tmem_ld32(lane_addr, v);
       tmem_wait_ld();
       tc_fence_before();  // TMEM reads done before the next product
       const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {  // S = alpha (S M) + C in place, both chunks first
-        const unsigned char* crow = sC + (2 * half + qq) * CBOX + row * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 c4 = *reinterpret_cast<const float4*>(crow + ((u ^ (row & 7)) << 4));
-          const float2 lo = fma2(a2, make_float2(v[qq][4 * u], v[qq][4 * u + 1]), make_float2(c4.x, c4.y));
-          const float2 hi = fma2(a2, make_float2(v[qq][4 * u + 2], v[qq][4 * u + 3]), make_float2(c4.z, c4.w));
-          v[qq][4 * u] = lo.x; v[qq][4 * u + 1] = lo.y; v[qq][4 * u + 2] = hi.x; v[qq][4 * u + 3] = hi.y;
-        }
+      for (int u = 0; u < 16; ++u) {  // S = alpha (S M) + C
+        const float2 r = fma2(a2, make_float2(v[2 * u], v[2 * u + 1]), make_float2(cv[2 * u], cv[2 * u + 1]));
+        v[2 * u] = r.x;
+        v[2 * u + 1] = r.y;
       }
-#pragma unroll
-      for (int qq = 0; qq < 2; ++qq) emit_chunk(dm, dir, sl, snap_row, 2 * half + qq, row, sA, v[qq]);
+      split_chunk(q, srow, sA, v);
       fence_proxy_async_smem();  // new A operand visible to the tensor cores
-      mbar_arrive_warp(bar(B_SREADY));
+      arrive_cluster_warp(lbar(B_SREADY));
+      // snapshots after the hand-off: the next product does not wait for them
+      snap_chunk(dm, dir, sl, snap_row, q, v);
       st = st_next;
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its memory or barriers
   tc_fence_after();
-  if (warp == 1) tmem_free(tmem, 128);
+  if (warp == 1) tmem_free2(tmem, kTmemScan);
 }
 
 }  // namespace
@@ -293,7 +342,7 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
 bool scan_tc_supported(const Dims& d) {
   if (!scan_tc_layout(d.bf16 != 0, d.dk, d.dv) || !gram_tc_supported(d)) return false;
   if ((long long)d.B * d.T * d.H * 2 * d.dk >= (1LL << 31)) return false;  // TMA row coordinates
-  if ((long long)d.B * d.H * 2 > 0x7FFFFFFFLL) return false;
+  if ((long long)d.B * d.H * 4 > 0x7FFFFFFFLL) return false;
   return encode_fn() != nullptr;
 }
 
@@ -301,12 +350,14 @@ cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaS
   if (d.dk != D || w.M16 == nullptr) return cudaErrorInvalidValue;
   CUtensorMap mm, mc;
   const long long fh = (long long)d.B * d.T * d.H;
-  if (!make_matrix_map(&mm, w.M16, fh * 2 * D, D, 128) || !make_matrix_map_f32(&mc, w.Cm, fh * D, D, 128))
+  if (!make_matrix_map(&mm, w.M16, fh * 2 * D, D, R) || !make_matrix_map_f32(&mc, w.Cm, fh * D, D, R))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + 2 * (size_t)SPLIT + CBYTES + NBARS * 8 + 16;
+  // one CTA per SM (the two CTAs of a pair sit on two SMs): at least 120 KB
+  const size_t need = 1024 + 3 * (size_t)SPLIT + 2 * (size_t)CBYTES + NBARS * 8 + 16;
+  const size_t smem = need < 120 * 1024 ? 120 * 1024 : need;
   cudaError_t e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_scan_tc<<<(unsigned)(d.B * d.H * 2), kThreadsScan, smem, s>>>(d, in, w, mm, mc);
+  k_scan_tc<<<(unsigned)(2 * d.B * d.H * 2), kThreadsScan, smem, s>>>(d, in, w, mm, mc);  // a CTA pair per chain
   return cudaGetLastError();
 }
 
