@@ -200,6 +200,65 @@ def backward_states(S0, k, v, beta, alpha, anchors: int = 4) -> np.ndarray:
     return G
 
 
+def chunk_maps(k, v, beta, alpha, chunk: int = 5, anchors: int = 4):
+    """Chunk composition of the frame maps for one (batch, head).
+
+    Each written frame acts on the state as the affine map S -> alpha_t S M_t
+    + C_t (frame_map; [P4] closed form), so the frames of one chunk compose
+    into one map of the same form (the north star's "prefix composition of
+    the affine frame maps where it helps").  For chunk c, with its written
+    frames f_1 < ... < f_n (anchor frames are identity maps and drop out):
+
+    * forward (frames in increasing order): S -> Lam_c S P_c + Cf_c with
+      P_c = M_{f_1} ... M_{f_n}, Lam_c = alpha_{f_1} ... alpha_{f_n}, and
+      Cf_c by Horner's rule, Cf <- alpha_f Cf M_f + C_f from Cf = 0;
+    * backward (decreasing order): S -> Lam_c S P_c^T + Cb_c, since each
+      M_f = (I + A_f)^{-1} is symmetric and the reversed product is the
+      transpose; Cb <- alpha_f Cb M_f + C_f for f from f_n down to f_1.
+
+    Returns P [C, d_k, d_k], Cf, Cb [C, d_v, d_k], Lam [C]; a chunk with no
+    written frame gives the identity map (P = I, Cf = Cb = 0, Lam = 1)."""
+    T, d_k, d_v = k.shape[0], k.shape[-1], v.shape[-1]
+    anc = set(anchor_frames(T, anchors))
+    nc = num_chunks(T, chunk)
+    P = np.empty((nc, d_k, d_k))
+    Cf = np.empty((nc, d_v, d_k))
+    Cb = np.empty((nc, d_v, d_k))
+    Lam = np.empty(nc)
+    for c in range(nc):
+        frames = [f for f in range(c * chunk, min((c + 1) * chunk, T)) if f not in anc]
+        maps = {f: frame_map(k[f], v[f], beta[f]) for f in frames}
+        Pc, cf, cb, lam = np.eye(d_k), np.zeros((d_v, d_k)), np.zeros((d_v, d_k)), 1.0
+        for f in frames:
+            M, Cm = maps[f]
+            Pc = Pc @ M
+            cf = alpha[f] * cf @ M + Cm
+            lam *= alpha[f]
+        for f in reversed(frames):
+            M, Cm = maps[f]
+            cb = alpha[f] * cb @ M + Cm
+        P[c], Cf[c], Cb[c], Lam[c] = Pc, cf, cb, lam
+    return P, Cf, Cb, Lam
+
+
+def chunk_scan(S0, P, Cf, Cb, Lam):
+    """The two scans stepped by whole chunks with the maps of chunk_maps.
+    Returns Fc [C+1, ...] with Fc[j] the forward state over the first j
+    chunks (Fc[0] = S0) and Gc [C+1, ...] with Gc[j] the backward state over
+    chunks >= j (Gc[C] = S0): the forward / backward states at every chunk
+    boundary, which is all the read needs."""
+    nc = len(Lam)
+    Fc = np.empty((nc + 1,) + np.shape(S0))
+    Gc = np.empty((nc + 1,) + np.shape(S0))
+    Fc[0] = S0
+    for c in range(nc):
+        Fc[c + 1] = Lam[c] * Fc[c] @ P[c] + Cf[c]
+    Gc[nc] = S0
+    for c in range(nc - 1, -1, -1):
+        Gc[c] = Lam[c] * Gc[c + 1] @ P[c].T + Cb[c]
+    return Fc, Gc
+
+
 def read_state(F, G, t: int, T: int, chunk: int = 5, anchors: int = 4, anchor_read: str = "text"):
     """The state a query in frame t reads: the forward state over the frames
     before its window plus the backward state over the frames after it

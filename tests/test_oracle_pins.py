@@ -371,3 +371,58 @@ def test_pins_catch_transposed_write(monkeypatch):
     monkeypatch.setattr(O, "gram_write", lambda K, V, b: (orig(K, V, b)[0], orig(K, V, b)[1].T))
     with pytest.raises(AssertionError):
         test_update_matches_token_space_woodbury(5, 16)
+
+
+# ---------------------------------------------------------------- chunk maps
+@pytest.mark.parametrize("T,anchors", [(17, 4), (23, 4), (10, 0), (12, 4)])
+def test_chunk_composed_scan_equals_frame_scan(T, anchors):
+    """Stepping the two scans by composed chunk maps reproduces the
+    frame-by-frame scans (each step a joint least-squares solve) at every
+    chunk boundary, which is where the read takes its states."""
+    S0, k, v, beta, alpha = _scan_inputs(T, 5, 6, 11 + T)
+    F = O.forward_states(S0, k, v, beta, alpha, anchors=anchors)
+    G = O.backward_states(S0, k, v, beta, alpha, anchors=anchors)
+    Fc, Gc = O.chunk_scan(S0, *O.chunk_maps(k, v, beta, alpha, chunk=5, anchors=anchors))
+    nc = O.num_chunks(T, 5)
+    scale = np.abs(F).max()
+    for j in range(nc + 1):
+        b = min(5 * j, T)
+        np.testing.assert_allclose(Fc[j], F[b], rtol=0, atol=1e-12 * scale)
+        np.testing.assert_allclose(Gc[j], G[b], rtol=0, atol=1e-12 * scale)
+
+
+def test_chunk_map_backward_uses_the_transpose():
+    """Applying a chunk's frames in decreasing order, each as the joint solve
+    from the decayed state, equals Lam S P^T + Cb: the reversed product of
+    the symmetric M_t is the transpose of the forward product."""
+    T = 15
+    S0, k, v, beta, alpha = _scan_inputs(T, 7, 5, 5)
+    P, Cf, Cb, Lam = O.chunk_maps(k, v, beta, alpha, chunk=5, anchors=4)
+    S = rng.standard_normal((5, 5))
+    for c in range(3):
+        X = S.copy()
+        for f in range(min(5 * c + 4, T - 1), 5 * c - 1, -1):
+            if f not in (0, T - 1):
+                X = O.vda_update(alpha[f] * X, k[f], v[f], beta[f])
+        np.testing.assert_allclose(X, Lam[c] * S @ P[c].T + Cb[c], rtol=0, atol=1e-12 * np.abs(X).max())
+        Y = S.copy()
+        for f in range(5 * c, min(5 * c + 5, T)):
+            if f not in (0, T - 1):
+                Y = O.vda_update(alpha[f] * Y, k[f], v[f], beta[f])
+        np.testing.assert_allclose(Y, Lam[c] * S @ P[c] + Cf[c], rtol=0, atol=1e-12 * np.abs(Y).max())
+
+
+def test_chunk_map_special_cases():
+    """A chunk of anchor frames only is the identity map; a chunk with one
+    written frame is that frame's own map (M_t, C_t, alpha_t)."""
+    S0, k, v, beta, alpha = _scan_inputs(2, 4, 6, 9)
+    P, Cf, Cb, Lam = O.chunk_maps(k, v, beta, alpha, chunk=5, anchors=4)
+    np.testing.assert_array_equal(P[0], np.eye(6))
+    assert not Cf.any() and not Cb.any() and Lam[0] == 1.0
+    S0, k, v, beta, alpha = _scan_inputs(3, 4, 6, 10)
+    P, Cf, Cb, Lam = O.chunk_maps(k, v, beta, alpha, chunk=5, anchors=4)
+    M, C = O.frame_map(k[1], v[1], beta[1])
+    np.testing.assert_allclose(P[0], M, atol=1e-14)
+    np.testing.assert_allclose(Cf[0], C, atol=1e-14)
+    np.testing.assert_allclose(Cb[0], C, atol=1e-14)
+    assert Lam[0] == alpha[1]

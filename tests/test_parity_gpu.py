@@ -114,6 +114,9 @@ CASES = {
     "d128_ragged_keys": (Shape(1, 30, 130, 1, 128, 128, 4), {}),
     "d128_scale40_rescale": (Shape(1, 25, 70, 2, 128, 128, 4), dict(softmax_scale=40.0)),
     "d64_scale40_no_anchor": (Shape(1, 25, 70, 2, 64, 64, 4), dict(softmax_scale=40.0, anchors=0)),
+    # d = 128 scans with no written frame and with one (both ends anchors)
+    "d128_T2_all_anchor": (Shape(1, 2, 40, 2, 128, 128, 4), {}),
+    "d128_T3_one_written": (Shape(1, 3, 40, 3, 128, 128, 4), {}),
 }
 
 
