@@ -84,6 +84,13 @@ typedef struct {
                           1: y[B,T,N,H,d_v] = sum of the two gated branches           */
   int y_dtype;         /* vdn_dtype of y: VDN_F32 (default, also in bf16 mode) or
                           VDN_BF16 (rounded to nearest even on store)                  */
+  int scan_mode;       /* how the tensor-core scan (VDN_BF16, d = 128) steps: 0 = auto,
+                          1 = by frames, 2 = by chunks with composed chunk maps (the
+                          frames of a chunk composed first, then one step per chunk).
+                          Auto takes chunks when there are at least 4 and the 2*B*C*H
+                          compositions fit one wave of the GPU's SMs (few chains, long
+                          sequences), frames otherwise.  Other configurations step by
+                          frames whatever the mode.                                    */
 } vdn_hybrid_cfg;
 
 typedef struct {
@@ -133,10 +140,18 @@ enum {
  *                                     path only)
  *   frame_M16  : [B,T,H,2,d,d]        bfloat16 hi/lo split of frame_M, the operand of the
  *                                     tensor-core scan (bf16 inputs with d = 128 only;
- *                                     an empty region otherwise)                         */
+ *                                     an empty region otherwise)
+ *   chunk_P16  : [B,C,H,2,d,d]        chunk maps (same condition): bfloat16 hi/lo split of
+ *                                     P_c = M_f1 ... M_fn over the chunk's written frames
+ *   chunk_C    : [2,B,C,H,d_v,d_k]    the forward and backward constants Cf_c, Cb_c: the
+ *                                     frames of chunk c map a state S to Lam_c S P_c + Cf_c
+ *                                     (increasing order), Lam_c S P_c^T + Cb_c (decreasing)
+ *   chunk_lam  : [B,C,H]              Lam_c, the product of the chunk's alpha_t
+ *   The chunk maps are written when the scan steps by chunks (C >= 4), and left
+ *   unset otherwise.                                                                     */
 typedef struct {
   size_t status, half_text, frame_M, frame_C, fwd_snap, bwd_snap, read_table, read_table_bf16, text_gram, frame_M16,
-      total;
+      chunk_P16, chunk_C, chunk_lam, total;
 } vdn_workspace_layout;
 
 /* Bytes of workspace the configuration needs; 0 if cfg is invalid. */

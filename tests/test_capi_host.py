@@ -51,10 +51,14 @@ def test_workspace_size_and_layout():
     dd = 128 * 128 * 4
     assert lay["frame_C"] - lay["frame_M"] >= 90 * 24 * dd
     assert lay["read_table"] - lay["bwd_snap"] >= 24 * 19 * dd
-    if cfg.dtype == L.VDN_BF16 and cfg.d_k == 128:  # bf16 hi/lo of every frame's M
-        assert lay["total"] - lay["frame_M16"] >= 90 * 24 * dd
+    if cfg.dtype == L.VDN_BF16 and cfg.d_k == 128:  # bf16 hi/lo of every frame's M; the chunk maps
+        assert lay["chunk_P16"] - lay["frame_M16"] >= 90 * 24 * dd
+        assert lay["chunk_C"] - lay["chunk_P16"] >= 18 * 24 * dd
+        assert lay["chunk_lam"] - lay["chunk_C"] >= 2 * 18 * 24 * dd
+        assert lay["total"] - lay["chunk_lam"] >= 18 * 24 * 4
     offs = [lay[k] for k in ("status", "half_text", "frame_M", "frame_C", "fwd_snap", "bwd_snap", "read_table",
-                             "read_table_bf16", "text_gram", "frame_M16", "total")]
+                             "read_table_bf16", "text_gram", "frame_M16", "chunk_P16", "chunk_C", "chunk_lam",
+                             "total")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
 
 
@@ -64,6 +68,7 @@ def test_workspace_size_and_layout():
     (dict(L=-1), L.VDN_ERR_INVALID_ARG), (dict(chunk=0), L.VDN_ERR_INVALID_ARG),
     (dict(d_k=48, d_v=48), L.VDN_ERR_UNSUPPORTED), (dict(d_v=64), L.VDN_ERR_UNSUPPORTED),
     (dict(chunk=4), L.VDN_ERR_UNSUPPORTED), (dict(B=3000, H=24), L.VDN_ERR_UNSUPPORTED),
+    (dict(scan_mode=3), L.VDN_ERR_INVALID_ARG), (dict(scan_mode=-1), L.VDN_ERR_INVALID_ARG),
 ])
 def test_bad_config_rejected(kw, status):
     cfg = _cfg(**kw)

@@ -254,6 +254,48 @@ def test_intermediates_match_oracle():
         np.testing.assert_allclose(it["R"][0, h], ref["R"], atol=1e-5 * scale)
 
 
+@pytest.mark.parametrize("shape", [Shape(1, 22, 48, 2, 128, 128, 4), Shape(2, 40, 24, 1, 128, 128, 0)])
+def test_chunk_maps_match_oracle(shape):
+    """The composed chunk maps of the chunk-stepped scan (P_c from its bf16
+    split, the two Horner constants, Lam_c) against the oracle's chunk_maps
+    on the same frames; chunk 0 and the last chunk hold an anchor frame."""
+    inp, cfg, ha, _, _ = run(shape, "bf16", 5)
+    assert cfg.C >= 4  # the chunk-stepped scan runs
+    cm = {k: v.double().cpu().numpy() for k, v in ha.chunk_maps().items()}
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            f64 = lambda a: np.asarray(a, np.float64)
+            P, Cf, Cb, Lam = O.chunk_maps(f64(inp["k"][b, :, :, h]), f64(inp["v"][b, :, :, h]),
+                                          f64(inp["beta"][b, :, :, h]), f64(inp["alpha"][b, :, h]),
+                                          chunk=cfg.chunk, anchors=cfg.anchors)
+            for c in range(cfg.C):
+                np.testing.assert_allclose(cm["P"][b, c, h], P[c], rtol=0, atol=2e-4 * np.abs(P[c]).max())
+                sc = np.abs(Cf[c]).max()
+                np.testing.assert_allclose(cm["Cf"][b, c, h], Cf[c], rtol=0, atol=2e-4 * sc)
+                np.testing.assert_allclose(cm["Cb"][b, c, h], Cb[c], rtol=0, atol=2e-4 * np.abs(Cb[c]).max())
+                np.testing.assert_allclose(cm["Lam"][b, c, h], Lam[c], rtol=1e-6)
+
+
+@pytest.mark.parametrize("scan_mode", [1, 2])
+def test_scan_modes_match_oracle(scan_mode):
+    """The tensor-core scan stepped by frames (1) and by composed chunk maps
+    (2) on the same inputs: both reach the oracle's output, and their
+    chunk-boundary states agree with the oracle's frame scan."""
+    shape = Shape(1, 30, 40, 3, 128, 128, 4)
+    inp, cfg, ha, _, y = run(shape, "bf16", 13, scan_mode=scan_mode)
+    check(y, oracle(inp, cfg), cfg, "bf16")
+    it = {k: v.double().cpu().numpy() for k, v in ha.intermediates().items()}
+    for h in range(cfg.H):
+        ref = O.vda_intermediates(inp, ocfg(cfg), 0, h)
+        scale = np.sqrt(np.mean(ref["R"] ** 2))
+        for j in range(cfg.C + 1):
+            fj = min(5 * j, cfg.T)
+            # M_t, C_t carry ~2e-5 relative error (bf16-mode Gram, fp32 solve) and each
+            # step's split keeps ~16 bits; over <= 28 non-expansive steps: < 1e-3
+            np.testing.assert_allclose(it["fwd_snap"][0, h, j], ref["F"][fj], atol=1e-3 * scale)
+            np.testing.assert_allclose(it["bwd_snap"][0, h, j], ref["G"][fj], atol=1e-3 * scale)
+
+
 def test_stages_compose_to_full_call_and_are_deterministic():
     w = WORKLOADS["small"]
     inp, cfg, ha, t, y = run(w.shape, w.dtype, w.seed)

@@ -30,7 +30,7 @@ class VdnCfg(C.Structure):
     _fields_ = [("B", C.c_int), ("T", C.c_int), ("N", C.c_int), ("H", C.c_int), ("d_k", C.c_int),
                 ("d_v", C.c_int), ("L", C.c_int), ("chunk", C.c_int), ("anchors", C.c_int),
                 ("dtype", C.c_int), ("softmax_scale", C.c_float), ("rms_eps", C.c_float),
-                ("out_mode", C.c_int), ("y_dtype", C.c_int)]
+                ("out_mode", C.c_int), ("y_dtype", C.c_int), ("scan_mode", C.c_int)]
 
 
 class VdnArgs(C.Structure):
@@ -44,7 +44,7 @@ class VdnArgs(C.Structure):
 class VdnLayout(C.Structure):
     _fields_ = [(n, C.c_size_t) for n in ("status", "half_text", "frame_M", "frame_C", "fwd_snap",
                                           "bwd_snap", "read_table", "read_table_bf16", "text_gram", "frame_M16",
-                                          "total")]
+                                          "chunk_P16", "chunk_C", "chunk_lam", "total")]
 
 
 @dataclass
@@ -64,6 +64,7 @@ class HybridCfg:
     rms_eps: float = 0.0
     out_mode: int = 0
     y_dtype: int = VDN_F32
+    scan_mode: int = 0
 
     def c(self) -> VdnCfg:
         return VdnCfg(**{f.name: getattr(self, f.name) for f in fields(self)})

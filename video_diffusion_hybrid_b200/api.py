@@ -86,3 +86,19 @@ class HybridAttention:
             "bwd_snap": f(lay["bwd_snap"], (c.B, c.H, C + 1, c.d_v, c.d_k)),
             "R": f(lay["read_table"], (c.B, c.H, C + 1, c.d_v, c.d_k)),
         }
+
+    def chunk_maps(self) -> dict:
+        """The chunk maps of the chunk-stepped tensor-core scan (bf16 mode,
+        d = 128, C >= 4): P_c as hi + lo (float32), Cf_c, Cb_c, Lam_c."""
+        lay = L.vdn_hybrid_workspace_layout(self.cfg)
+        c = self.cfg
+        C, d = c.C, c.d_k
+        n = c.B * C * c.H
+        if lay["chunk_C"] == lay["chunk_P16"]:
+            raise ValueError("no chunk maps for this configuration")
+        p16 = self.workspace[lay["chunk_P16"]:lay["chunk_P16"] + 2 * n * 2 * d * d].view(torch.bfloat16)
+        p16 = p16.view(c.B, C, c.H, 2, d, d).float()
+        cc = self.workspace[lay["chunk_C"]:lay["chunk_C"] + 4 * 2 * n * d * d].view(torch.float32)
+        cc = cc.view(2, c.B, C, c.H, d, d)
+        lam = self.workspace[lay["chunk_lam"]:lay["chunk_lam"] + 4 * n].view(torch.float32).view(c.B, C, c.H)
+        return {"P": p16[:, :, :, 0] + p16[:, :, :, 1], "Cf": cc[0], "Cb": cc[1], "Lam": lam}

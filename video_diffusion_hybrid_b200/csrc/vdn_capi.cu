@@ -21,6 +21,7 @@ vdn_status check_cfg(const vdn_hybrid_cfg* c) {
   if (c->dtype != VDN_F32 && c->dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
   if (c->out_mode != 0 && c->out_mode != 1) return VDN_ERR_INVALID_ARG;
   if (c->y_dtype != VDN_F32 && c->y_dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
+  if (c->scan_mode < 0 || c->scan_mode > 2) return VDN_ERR_INVALID_ARG;
   if (!(c->softmax_scale == c->softmax_scale) || !(c->rms_eps == c->rms_eps)) return VDN_ERR_INVALID_ARG;
   if (c->d_k != 32 && c->d_k != 64 && c->d_k != 128 && c->d_k != 256) return VDN_ERR_UNSUPPORTED;
   if (c->d_v != c->d_k) return VDN_ERR_UNSUPPORTED;
@@ -45,6 +46,7 @@ Dims make_dims(const vdn_hybrid_cfg* c) {
   d.out_mode = c->out_mode;
   d.bf16 = c->dtype == VDN_BF16;
   d.out_bf16 = c->y_dtype == VDN_BF16;
+  d.scan_mode = c->scan_mode;
   return d;
 }
 
@@ -62,9 +64,16 @@ void layout_of(const vdn_hybrid_cfg* c, vdn_workspace_layout* L) {
   L->read_table = off; off += up(bh * (C + 1) * dd);
   L->read_table_bf16 = off; off += up(bh * (C + 1) * dd);  // hi and lo bf16 terms
   L->text_gram = off;  off += up(bh * 2 * dd);
+  const bool tc_scan = scan_tc_layout(c->dtype == VDN_BF16, c->d_k, c->d_v);
+  const size_t kk2 = 2 * (size_t)c->d_k * c->d_k * sizeof(__nv_bfloat16);  // one hi/lo split
   L->frame_M16 = off;
-  if (scan_tc_layout(c->dtype == VDN_BF16, c->d_k, c->d_v))
-    off += up(bh * (size_t)c->T * 2 * (size_t)c->d_k * c->d_k * sizeof(__nv_bfloat16));
+  if (tc_scan) off += up(bh * (size_t)c->T * kk2);
+  L->chunk_P16 = off;
+  if (tc_scan) off += up(bh * C * kk2);
+  L->chunk_C = off;
+  if (tc_scan) off += up(2 * bh * C * dd);
+  L->chunk_lam = off;
+  if (tc_scan) off += up(bh * C * sizeof(float));
   L->total = off;
 }
 
@@ -103,7 +112,13 @@ Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
   w.R = reinterpret_cast<float*>(base + L.read_table);
   w.R16 = base + L.read_table_bf16;
   w.text_gram = reinterpret_cast<float*>(base + L.text_gram);
-  w.M16 = L.total > L.frame_M16 ? base + L.frame_M16 : nullptr;
+  const bool tc_scan = L.chunk_P16 > L.frame_M16;
+  w.M16 = tc_scan ? base + L.frame_M16 : nullptr;
+  w.P16 = tc_scan ? base + L.chunk_P16 : nullptr;
+  w.Cf = tc_scan ? reinterpret_cast<float*>(base + L.chunk_C) : nullptr;
+  w.Cb = tc_scan ? w.Cf + (size_t)c->B * c->H * ((c->T + c->chunk - 1) / c->chunk) * c->d_v * c->d_k
+                 : nullptr;
+  w.lam = tc_scan ? reinterpret_cast<float*>(base + L.chunk_lam) : nullptr;
   return w;
 }
 
@@ -193,8 +208,20 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
   if (big && (stages & VDN_STAGE_SCAN)) {
     if (launch_scan_big(d, in, w, s) != cudaSuccess) return VDN_ERR_CUDA;
   } else if (stages & VDN_STAGE_SCAN) {
-    // the tensor-core scan reads the bf16 split of M that the sweep solve writes
-    e = (scan_tc_supported(d) && w.M16 != nullptr) ? launch_scan_tc(d, in, w, s) : launch_scan_simt(d, in, w, s);
+    // the tensor-core scan reads the bf16 split of M that the sweep solve
+    // writes; with enough chunks it first composes each chunk's frame maps
+    // and steps by whole chunks
+    if (scan_tc_supported(d) && w.M16 != nullptr) {
+      int dev = 0, sms = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VDN_ERR_CUDA;
+      const bool chunks = use_chunk_scan(d, sms);
+      if (chunks && launch_compose_tc(d, in, w, s) != cudaSuccess) return VDN_ERR_CUDA;
+      e = launch_scan_tc(d, in, w, s, chunks);
+    } else {
+      e = launch_scan_simt(d, in, w, s);
+    }
     if (e != cudaSuccess) return VDN_ERR_CUDA;
   }
   if (stages & VDN_STAGE_SOFTMAX) {

@@ -16,10 +16,11 @@ struct Dims {
   int out_mode;
   int bf16;      // inputs stored as bf16
   int out_bf16;  // y stored as bf16
+  int scan_mode;  // 0 auto, 1 frame steps, 2 chunk steps (tensor-core scan)
 };
 
 // Device-side status words at the head of the workspace.
-enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4 };
+enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4, TAG_COMPOSE_TC = 5 };
 
 struct Work {
   uint32_t* status;
@@ -32,6 +33,11 @@ struct Work {
   void* R16;         // [B,H,C+1,2,dv,dk] bf16 (hi, lo)
   float* text_gram;  // [B,H,2,dk,dk] A_x, B_x
   void* M16;         // [B,T,H,2,dk,dk] bf16 (hi, lo) of M; nullptr off the tensor-core scan
+  // chunk maps (tensor-core scan only): P_c split, [Cf; Cb], Lam
+  void* P16;         // [B,C,H,2,dk,dk] bf16 (hi, lo) of P_c
+  float* Cf;         // [B,C,H,dv,dk]; Cb follows at Cf + B*C*H*dv*dk
+  float* Cb;         // [B,C,H,dv,dk]
+  float* lam;        // [B,C,H]
 };
 
 struct Inputs {
@@ -69,7 +75,17 @@ bool big_d(const Dims& d);
 cudaError_t launch_solve_big(const Dims& d, const Work& w, cudaStream_t s, bool text);
 cudaError_t launch_scan_big(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_read_big(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
-cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+// chunks = false: the frame-stepped scan; true: stepped by the chunk maps of launch_compose_tc
+cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s, bool chunks);
+cudaError_t launch_compose_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+// The chunk-composed scan where it helps: the compositions (one CTA per
+// chunk, batch-head and direction) take about one wave of the SMs, and then
+// the sequential chain is 5x shorter; with more chains than that the frame
+// scan already fills the GPU and the composition is extra work.
+inline bool use_chunk_scan(const Dims& d, int sms) {
+  if (d.scan_mode != 0) return d.scan_mode == 2;
+  return d.C >= 4 && 2LL * d.B * d.C * d.H <= sms;
+}
 cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void* r16, cudaStream_t s);
 
 }  // namespace vdn

@@ -146,6 +146,12 @@ __device__ __forceinline__ void snap_chunk(const Dims& dm, int dir, const Slots&
   }
 }
 
+// CH = false: one step per written frame, S <- alpha_t S M_t + C_t (tmm over
+// M's split, tmc over C_t).  CH = true: one step per chunk with the composed
+// maps, S <- Lam_c S P_c + Cf_c forward and S <- Lam_c S P_c^T + Cb_c
+// backward (tmm over P_c's split, tmc over [Cf; Cb]); every step ends on a
+// chunk boundary, so every step is a snapshot.
+template <bool CH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsScan, 1)
 k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, const __grid_constant__ CUtensorMap tmc) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -169,8 +175,19 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
   auto bar = [&](int i) { return smem_u32(bars + i); };
   auto lbar = [&](int i) { return map_rank(smem_u32(bars + i), 0); };
   auto fh_of = [&](int t) { return ((long long)b * dm.T + t) * dm.H + h; };
-  int nw = 0;  // written frames
-  for (int t = 0; t < dm.T; ++t) nw += is_anchor(dm, t) ? 0 : 1;
+  int nw = 0;  // steps: written frames, or chunks
+  if (CH) nw = dm.C;
+  else
+    for (int t = 0; t < dm.T; ++t) nw += is_anchor(dm, t) ? 0 : 1;
+  // chunk mode: the chunk of step i, its chunk-map index, and the rows of its
+  // C constant (Cb after all Cf) in the [Cf; Cb] array
+  const long long nbch = (long long)dm.B * dm.C * dm.H;
+  auto chunk_of = [&](int i) { return dir == 0 ? i : dm.C - 1 - i; };
+  auto bch_of = [&](int c) { return ((long long)b * dm.C + c) * dm.H + h; };
+  // forward chunk steps multiply by P_c (not symmetric): B is P_c read
+  // N-contiguous (MN-major); every other step reads rows of a symmetric M_t
+  // or of P_c for P_c^T (K-major)
+  const bool mn = CH && dir == 0;
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < 2; ++k) {
@@ -202,6 +219,13 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
       // L2 early, so that the single-buffered loads below (issued only when
       // their buffer frees) run at L2 rather than HBM latency
       auto prefetch_step = [&](int pst) {
+        if (CH) {
+          if (pst >= nw) return;
+          const long long pb = bch_of(chunk_of(pst));
+          prefetch_l2(static_cast<const __nv_bfloat16*>(w.P16) + pb * 2 * D * D, SPLIT * 2);
+          prefetch_l2(w.Cf + ((dir == 0 ? 0 : nbch) + pb) * D * D + (long long)row0 * D, CBYTES);
+          return;
+        }
         if (pst >= dm.T) return;
         const long long pfh = fh_of(frame_at(dm, dir, pst));
         const __nv_bfloat16* m16 = static_cast<const __nv_bfloat16*>(w.M16);
@@ -209,29 +233,37 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
         prefetch_l2(m16 + ((pfh * 2 + 1) * D + row0) * D, OPBYTES);
         prefetch_l2(w.Cm + (pfh * D + row0) * D, CBYTES);
       };
-      int st = next_written(dm, dir, 0);
+      auto next_pos = [&](int p) { return CH ? p + 1 : next_written(dm, dir, p + 1); };
+      int st = CH ? 0 : next_written(dm, dir, 0);
       int pst = st;
       prefetch_step(pst);
-      pst = next_written(dm, dir, pst + 1);
+      pst = next_pos(pst);
       prefetch_step(pst);
-      for (int i = 0; i < nw; ++i, st = next_written(dm, dir, st + 1)) {
-        const long long fh = fh_of(frame_at(dm, dir, st));
-        pst = next_written(dm, dir, pst + 1);
+      for (int i = 0; i < nw; ++i, st = next_pos(st)) {
+        // B rows (of M's or P_c's split) and C rows of this step
+        const long long mrow = CH ? bch_of(chunk_of(i)) : fh_of(frame_at(dm, dir, st));
+        const long long crow = CH ? (dir == 0 ? 0 : nbch) + mrow : mrow;
+        pst = next_pos(pst);
         prefetch_step(pst);
         const int slot = i & 1;
         // slot free: the product (B) and this CTA's epilogue (C) of step i - 2 are done
         if (i >= 2 && !mbar_wait_cl(bar(B_BEMPTY + slot), ((i - 2) >> 1) & 1, ctl)) break;
         if (lead) mbar_expect_tx(bar(B_BFULL + slot), 2 * SPLIT);
         for (int part = 0; part < 2; ++part)
-          for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 2; ++c) {
+            // K-major: rows row0.. of the matrix, K chunk c; MN-major: its
+            // columns row0.. (this CTA's half of N), K rows 64c..
+            const int x = mn ? row0 : c * 64;
+            const int y = (int)((mrow * 2 + part) * D + (mn ? 64 * c : row0));
             tma_load_2d_pair(smem_u32(sB + slot * SPLIT + part * OPBYTES + c * CHUNK), &tmm, lbar(B_BFULL + slot),
-                             c * 64, (int)((fh * 2 + part) * D + row0));
+                             x, y);
+          }
         ++nb;
         if (i >= 2 && !mbar_wait_cl(bar(B_CEMPTY + slot), ((i - 2) >> 1) & 1, ctl)) break;
         mbar_expect_tx(bar(B_CFULL + slot), CBYTES);
         for (int c = 0; c < 4; ++c)
           tma_load_2d(smem_u32(sC + slot * CBYTES + c * CBOX), &tmc, bar(B_CFULL + slot), c * 32,
-                      (int)(fh * D + row0));
+                      (int)(crow * D + row0));
         ++nc;
       }
       // the last copies land before the pair can exit (the leader's B
@@ -241,7 +273,8 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
     }
   } else if (warp == 1) {
     if (lane == 0 && lead) {
-      constexpr uint32_t ID = idesc_bf16(2 * R, D, false);  // M = 128 over the pair, N = 128
+      // M = 128 over the pair, N = 128; B K-major, or MN-major (forward chunk steps)
+      const uint32_t ID = mn ? idesc_bf16(2 * R, D, true) : idesc_bf16(2 * R, D, false);
       const uint64_t a0 = sdesc(smem_u32(sA), 16, 1024), b0 = sdesc(smem_u32(sB), 16, 1024);
       for (int i = 0; i < nw; ++i) {
         const int slot = i & 1;
@@ -255,7 +288,7 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             mma2_bf16(tmem, dadd(a0, ao + (k >> 2) * CHUNK + (k & 3) * 32),
-                      dadd(bs, bo + (k >> 2) * CHUNK + (k & 3) * 32), ID, (pass | k) ? 1u : 0u);
+                      dadd(bs, bo + (mn ? k * 16 * 128 : (k >> 2) * CHUNK + (k & 3) * 32)), ID, (pass | k) ? 1u : 0u);
         }
         commit2(bar(B_MDONE));
         commit2(map_rank(bar(B_MDONE), 1));
@@ -274,8 +307,9 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
     const long long DD = (long long)D * D;
     const int row = row0 + srow;  // state row
     float* snap_row = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD + (long long)row * D;
-    // start state: its own slot, then the slots of leading unwritten frames
-    int st = next_written(dm, dir, 0);
+    // start state: its own slot, then (frame steps) the slots of leading
+    // unwritten frames
+    int st = CH ? 0 : next_written(dm, dir, 0);
     {
       const float* src = w.half_text + (long long)bh * DD + (long long)row * D;
       const int start_slot = dir == 0 ? 0 : dm.C;
@@ -289,13 +323,15 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
       fence_proxy_async_smem();
       arrive_cluster_warp(lbar(B_SREADY));
       store_row32(snap_row + start_slot * DD + q * 32, s);
-      snap_chunk(dm, dir, slots_of(dm, dir, 0, st), snap_row, q, s);
+      if (!CH) snap_chunk(dm, dir, slots_of(dm, dir, 0, st), snap_row, q, s);
     }
     for (int i = 0; i < nw; ++i) {
       const int slot = i & 1;
-      const int st_next = next_written(dm, dir, st + 1);
-      const float alpha = __ldg(in.alpha + fh_of(frame_at(dm, dir, st)));
-      const Slots sl = slots_of(dm, dir, st, st_next);
+      const int st_next = CH ? st + 1 : next_written(dm, dir, st + 1);
+      // chunk step: the map's Lam, and the slot of the chunk boundary it ends on
+      const int cst = chunk_of(i);
+      const float alpha = CH ? w.lam[bch_of(cst)] : __ldg(in.alpha + fh_of(frame_at(dm, dir, st)));
+      const Slots sl = CH ? Slots{dir == 0 ? cst + 1 : cst, -1, 0, 0} : slots_of(dm, dir, st, st_next);
       // this step's C row chunk into registers first (it does not depend on
       // the product), then the slot goes back to the producer
       if (!__all_sync(0xffffffffu, mbar_wait_cl(bar(B_CFULL + slot), (i >> 1) & 1, ctl))) break;
@@ -346,18 +382,25 @@ bool scan_tc_supported(const Dims& d) {
   return encode_fn() != nullptr;
 }
 
-cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
-  if (d.dk != D || w.M16 == nullptr) return cudaErrorInvalidValue;
+cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s, bool chunks) {
+  if (d.dk != D || w.M16 == nullptr || (chunks && w.P16 == nullptr)) return cudaErrorInvalidValue;
   CUtensorMap mm, mc;
-  const long long fh = (long long)d.B * d.T * d.H;
-  if (!make_matrix_map(&mm, w.M16, fh * 2 * D, D, R) || !make_matrix_map_f32(&mc, w.Cm, fh * D, D, R))
-    return cudaErrorInvalidValue;
+  if (chunks) {
+    const long long nbch = (long long)d.B * d.C * d.H;
+    if (!make_matrix_map(&mm, w.P16, nbch * 2 * D, D, R) || !make_matrix_map_f32(&mc, w.Cf, 2 * nbch * D, D, R))
+      return cudaErrorInvalidValue;
+  } else {
+    const long long fh = (long long)d.B * d.T * d.H;
+    if (!make_matrix_map(&mm, w.M16, fh * 2 * D, D, R) || !make_matrix_map_f32(&mc, w.Cm, fh * D, D, R))
+      return cudaErrorInvalidValue;
+  }
   // one CTA per SM (the two CTAs of a pair sit on two SMs): at least 120 KB
   const size_t need = 1024 + 3 * (size_t)SPLIT + 2 * (size_t)CBYTES + NBARS * 8 + 16;
   const size_t smem = need < 120 * 1024 ? 120 * 1024 : need;
-  cudaError_t e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = chunks ? k_scan_tc<true> : k_scan_tc<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k_scan_tc<<<(unsigned)(2 * d.B * d.H * 2), kThreadsScan, smem, s>>>(d, in, w, mm, mc);  // a CTA pair per chain
+  kern<<<(unsigned)(2 * d.B * d.H * 2), kThreadsScan, smem, s>>>(d, in, w, mm, mc);  // a CTA pair per chain
   return cudaGetLastError();
 }
 
