@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--vda-only", action="store_true",
                     help="the Video Delta Attention stages only (the d = 256 sweep shapes have no softmax)")
+    ap.add_argument("--proj", action="store_true",
+                    help="time the layer's output projection (one GEMM over the core's concat axis) at the "
+                         "workload's shape instead of the core")
     return ap.parse_args()
 
 
@@ -465,8 +468,50 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_proj(args):
+    """The layer's output projection out = y W at the workload's layer shape:
+    M = B*T*N tokens, K = H*2*d_v (the core's concat axis), N = H*d_v (the
+    model width), bf16 operands and output, fp32 accumulation.  One GPU."""
+    import torch
+    from video_diffusion_hybrid_b200 import _lib as L
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    s = w.shape
+    M, K, N = s.B * s.T * s.N, s.H * 2 * s.d_v, s.H * s.d_v
+    gen = torch.Generator(device="cuda").manual_seed(w.seed)
+    y = torch.randn((M, K), device="cuda", generator=gen).to(torch.bfloat16)
+    wt = (torch.randn((K, N), device="cuda", generator=gen) / K ** 0.5).to(torch.bfloat16)
+    out = torch.empty((M, N), device="cuda", dtype=torch.bfloat16)
+    for _ in range(max(args.warmup, 3)):
+        L.vdn_out_proj(M, K, N, L.VDN_BF16, y, wt, out)
+    torch.cuda.synchronize()
+    clk = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0])
+    clk.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        L.vdn_out_proj(M, K, N, L.VDN_BF16, y, wt, out)
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, src = load_peaks()
+    tflops = 2.0 * M * K * N / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", 1590.0)
+    print(json.dumps({
+        "metric": "layer output projection (one GEMM over the concat axis)", "value": tflops, "unit": "TFLOP/s",
+        "ms_per_step": ms, "steps": args.steps, "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": args.workload, "M": M, "K": K, "N": N, "library": "cuBLASLt"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                     "peak_source": f"bf16_tflops ({src})"},
+        "clocks": clocks}), flush=True)
+
+
 def main():
     args = parse()
+    if args.proj:
+        run_proj(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -207,6 +207,29 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg *cfg, unsigned stage);
 /* Static description of a status code. */
 const char *vdn_status_string(vdn_status s);
 
+/* ------------------------------------------------ the layer's output projection
+ * PaperDaily digest section 三: each branch is gated, then projected back to
+ * the model width.  With the core's output in out_mode 0 (y[B,T,N,H,2,d_v],
+ * slot 0 softmax, slot 1 linear), one GEMM with the stacked weight equals the
+ * sum of the two separate projections:
+ *   out[m, n] = sum_k y[m, k] w[k, n],   y viewed as [M = B*T*N, K = H*2*d_v]
+ * with row k = (h * 2 + slot) * d_v + i of w the weight of that output element. */
+typedef struct {
+  int M;          /* rows (tokens)                                                    >= 1 */
+  int K;          /* the per-token output block, H*2*d_v; a multiple of 8           >= 8 */
+  int N;          /* output width; a multiple of 8                                     >= 8 */
+  int out_dtype;  /* vdn_dtype of out: VDN_F32 or VDN_BF16 (rounded to nearest even)       */
+} vdn_proj_cfg;
+
+/* out = y w on `stream`: y bfloat16 [M, K] row-major (the core's output with
+ * y_dtype VDN_BF16), w bfloat16 [K, N] row-major, out [M, N] row-major in
+ * out_dtype; fp32 accumulation.  Device pointers, 16-byte aligned, no overlap
+ * of out with y or w.  A plain dense GEMM run by cuBLASLt without workspace
+ * (a cuBLASLt handle is created on the first call of the process).  Errors:
+ * VDN_ERR_INVALID_ARG (a NULL or misaligned pointer, sizes), VDN_ERR_UNSUPPORTED
+ * (no GEMM algorithm for the sizes), VDN_ERR_CUDA. */
+vdn_status vdn_out_proj(const vdn_proj_cfg *cfg, const void *y, const void *w, void *out, vdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

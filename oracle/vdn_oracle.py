@@ -283,6 +283,17 @@ def read_table(F, G, T: int, chunk: int = 5, anchors: int = 4):
     return R
 
 
+def out_proj(y, W):
+    """The layer's output projection over the core's concat axis ([P1] 三:
+    each gated branch is projected back to the model width; with the two
+    branches on a size-2 axis, one product with the stacked weight is the
+    sum of the two projections).  y [..., H, 2, d_v] is flattened per token
+    to H*2*d_v values, row (h*2 + slot)*d_v + i, times W [H*2*d_v, n]."""
+    y = np.asarray(y, F64)
+    H, two, dv = y.shape[-3:]
+    return y.reshape(y.shape[:-3] + (H * two * dv,)) @ np.asarray(W, F64)
+
+
 def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-np.asarray(x, F64)))
 

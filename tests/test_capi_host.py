@@ -147,3 +147,12 @@ def test_status_strings_and_stage_impl():
     assert L.vdn_hybrid_attn_workspace_size(big) > 0
     assert L.vdn_hybrid_stage_impl(_cfg(d_k=256, d_v=256, dtype=L.VDN_F32), L.STAGE_SOLVE) == -1
     assert L.vdn_hybrid_attn_workspace_size(_cfg(d_k=256, d_v=256, dtype=L.VDN_F32)) == 0
+
+
+def test_out_proj_bad_args_rejected():
+    """vdn_out_proj validates before any launch (no device needed)."""
+    p = 1 << 20
+    for M, K, N, od, y, w, o in [(0, 64, 64, 0, p, p, p), (8, 60, 64, 0, p, p, p), (8, 64, 12, 0, p, p, p),
+                                 (8, 64, 64, 7, p, p, p), (8, 64, 64, 0, None, p, p), (8, 64, 64, 0, p + 8, p, p)]:
+        assert L.vdn_out_proj(M, K, N, od, y, w, o, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.lib().vdn_out_proj(None, None, None, None, None) == L.VDN_ERR_INVALID_ARG

@@ -426,3 +426,20 @@ def test_chunk_map_special_cases():
     np.testing.assert_allclose(Cf[0], C, atol=1e-14)
     np.testing.assert_allclose(Cb[0], C, atol=1e-14)
     assert Lam[0] == alpha[1]
+
+
+def test_out_proj_is_the_sum_of_the_branch_projections():
+    """One product over the concat axis with the stacked weight equals the
+    softmax branch projected by its weight plus the linear branch projected
+    by its own, head by head (the reason the core puts the two branches on a
+    size-2 axis)."""
+    r = np.random.default_rng(21)
+    H, dv, n = 3, 4, 5
+    y = r.standard_normal((2, 7, H, 2, dv))
+    W_sm = r.standard_normal((H, dv, n))
+    W_lin = r.standard_normal((H, dv, n))
+    W = np.stack([W_sm, W_lin], axis=1).reshape(H * 2 * dv, n)
+    ref = np.zeros((2, 7, n))
+    for h in range(H):
+        ref += y[..., h, 0, :] @ W_sm[h] + y[..., h, 1, :] @ W_lin[h]
+    np.testing.assert_allclose(O.out_proj(y, W), ref, rtol=0, atol=1e-12)

@@ -382,3 +382,42 @@ def test_vda_sweep_sampled_parity(name):
         assert err <= TOL[w.dtype], (h, err)
     del t, y, ha
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------ output projection
+def _bf16_tensor(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).cuda()
+
+
+@pytest.mark.parametrize("out_dtype", [L.VDN_F32, L.VDN_BF16])
+@pytest.mark.parametrize("M,H,dv,n", [(1000, 2, 64, 192), (77, 3, 128, 256)])
+def test_out_proj_matches_oracle(out_dtype, M, H, dv, n):
+    """y [M, H, 2, d_v] (bf16) times the stacked weight [H*2*d_v, n] (bf16),
+    fp32 accumulation, against the oracle's product of the same bf16 values."""
+    r = np.random.default_rng(M + n)
+    yt = _bf16_tensor(r.standard_normal((M, H, 2, dv)))
+    wt = _bf16_tensor(r.standard_normal((H * 2 * dv, n)) / np.sqrt(H * 2 * dv))
+    out = torch.empty((M, n), dtype=torch.float32 if out_dtype == L.VDN_F32 else torch.bfloat16, device="cuda")
+    L.vdn_out_proj(M, H * 2 * dv, n, out_dtype, yt, wt, out)
+    torch.cuda.synchronize()
+    ref = O.out_proj(yt.float().cpu().numpy(), wt.float().cpu().numpy())
+    got = out.float().cpu().numpy().astype(np.float64)
+    # fp32 accumulation of K = H*2*d_v products: ~sqrt(K) * 2^-24 relative; a bf16 store adds 2^-9
+    tol = 2e-5 * np.abs(ref).max() + (2.0 ** -8 * np.abs(ref) if out_dtype == L.VDN_BF16 else 0.0)
+    assert np.all(np.abs(got - ref) <= tol)
+
+
+def test_out_proj_on_core_output():
+    """The projection of the core's own bf16 output (out_mode 0) matches the
+    oracle's projection of the oracle's output within the bf16-mode tolerance."""
+    w = WORKLOADS["small"]
+    inp, cfg, ha, _, y = run(w.shape, w.dtype, w.seed, y_dtype=L.VDN_BF16)
+    M, K, n = cfg.B * cfg.T * cfg.N, cfg.H * 2 * cfg.d_v, 96
+    r = np.random.default_rng(4)
+    wt = _bf16_tensor(r.standard_normal((K, n)) / np.sqrt(K))
+    out = torch.empty((M, n), dtype=torch.float32, device="cuda")
+    L.vdn_out_proj(M, K, n, L.VDN_F32, ha.y, wt, out)
+    torch.cuda.synchronize()
+    ref = O.out_proj(oracle(inp, cfg), wt.float().cpu().numpy()).reshape(M, n)
+    e = rel_err(out.cpu().numpy().astype(np.float64), ref)
+    assert e <= TOL["bf16"], e

@@ -22,7 +22,7 @@ STAGE_ALL = 31
 
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
-            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc")
+            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -39,6 +39,11 @@ class VdnArgs(C.Structure):
                 ("text_k", C.c_void_p), ("text_v", C.c_void_p), ("text_beta", C.c_void_p),
                 ("init_state", C.c_void_p), ("rms_weight", C.c_void_p), ("y", C.c_void_p),
                 ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t)]
+
+
+class ProjCfg(C.Structure):
+    """Mirror of ``vdn_proj_cfg``."""
+    _fields_ = [("M", C.c_int), ("K", C.c_int), ("N", C.c_int), ("out_dtype", C.c_int)]
 
 
 class VdnLayout(C.Structure):
@@ -106,6 +111,8 @@ def lib() -> C.CDLL:
         L.vdn_hybrid_stage_impl.argtypes = [C.POINTER(VdnCfg), C.c_uint]
         L.vdn_hybrid_attn_fwd_noalloc.restype = C.c_int
         L.vdn_hybrid_attn_fwd_noalloc.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
+        L.vdn_out_proj.restype = C.c_int
+        L.vdn_out_proj.argtypes = [C.POINTER(ProjCfg), C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
         L.vdn_status_string.restype = C.c_char_p
         L.vdn_status_string.argtypes = [C.c_int]
         _lib = L
@@ -127,6 +134,15 @@ def vdn_hybrid_workspace_layout(cfg: HybridCfg) -> dict:
     if st != VDN_OK:
         raise VdnError(st, "vdn_hybrid_workspace_layout")
     return {n: int(getattr(out, n)) for n, _ in VdnLayout._fields_}
+
+
+def vdn_out_proj(M: int, K: int, N: int, out_dtype: int, y, w, out, stream=None, check: bool = True) -> int:
+    """out[M, N] = y[M, K] w[K, N] (device pointers or tensors)."""
+    c = ProjCfg(M=M, K=K, N=N, out_dtype=out_dtype)
+    st = lib().vdn_out_proj(C.byref(c), _ptr(y), _ptr(w), _ptr(out), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_out_proj")
+    return st
 
 
 def vdn_hybrid_stage_impl(cfg: HybridCfg, stage: int) -> int:

@@ -263,6 +263,14 @@ vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg* cfg, const vdn_hybrid_
   return host[0] ? VDN_ERR_TIMEOUT : VDN_OK;
 }
 
+vdn_status vdn_out_proj(const vdn_proj_cfg* cfg, const void* y, const void* w, void* out, vdn_stream_t stream) {
+  if (!cfg || !y || !w || !out) return VDN_ERR_INVALID_ARG;
+  if (cfg->M < 1 || cfg->K < 8 || cfg->N < 8 || cfg->K % 8 || cfg->N % 8) return VDN_ERR_INVALID_ARG;
+  if (cfg->out_dtype != VDN_F32 && cfg->out_dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
+  if (!aligned(y, 16) || !aligned(w, 16) || !aligned(out, 16)) return VDN_ERR_INVALID_ARG;
+  return out_proj(cfg->M, cfg->K, cfg->N, cfg->out_dtype, y, w, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
 const char* vdn_status_string(vdn_status s) {
   switch (s) {
     case VDN_OK: return "ok";
