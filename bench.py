@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--vda-only", action="store_true",
                     help="the Video Delta Attention stages only (the d = 256 sweep shapes have no softmax)")
+    ap.add_argument("--xattn", action="store_true",
+                    help="time the text cross-attention (every video query over the L text tokens) at the "
+                         "workload's shape instead of the core")
     ap.add_argument("--proj", action="store_true",
                     help="time the layer's output projection (one GEMM over the core's concat axis) at the "
                          "workload's shape instead of the core")
@@ -507,8 +510,57 @@ def run_proj(args):
         "clocks": clocks}), flush=True)
 
 
+def run_xattn(args):
+    """The block's text cross-attention at the workload's shape: B*T*N video
+    queries per head over the L text tokens, bf16 q / k / v, fp32 output."""
+    import torch
+    from video_diffusion_hybrid_b200 import _lib as L
+    from video_diffusion_hybrid_b200.api import cfg_for
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    s = w.shape
+    cfg = cfg_for(s, "bf16")
+    gen = torch.Generator(device="cuda").manual_seed(w.seed)
+    q = torch.randn((s.B, s.T, s.N, s.H, s.d_k), device="cuda", generator=gen).to(torch.bfloat16)
+    tk = torch.randn((s.B, s.L, s.H, s.d_k), device="cuda", generator=gen).to(torch.bfloat16)
+    tv = torch.randn((s.B, s.L, s.H, s.d_v), device="cuda", generator=gen).to(torch.bfloat16)
+    y = torch.empty((s.B, s.T, s.N, s.H, s.d_v), device="cuda", dtype=torch.float32)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    a = L.make_args(q, None, None, None, None, None, None, y, ws, text_k=tk, text_v=tv)
+    for _ in range(max(args.warmup, 3)):
+        L.vdn_text_cross_attn(cfg, a)
+    torch.cuda.synchronize()
+    clk = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0])
+    clk.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        L.vdn_text_cross_attn(cfg, a)
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    assert L.vdn_hybrid_device_status(cfg, a)[0] == L.VDN_OK
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, src = load_peaks()
+    flops = 4.0 * s.d_k * s.L * s.B * s.T * s.N * s.H
+    tflops = flops / (ms * 1e-3) / 1e12
+    hbm = (2 * s.B * s.T * s.N * s.H * s.d_k + 4 * s.B * s.T * s.N * s.H * s.d_v) / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": "text cross-attention", "value": s.B * s.T * s.N / (ms * 1e-3), "unit": "video tokens/s",
+        "ms_per_step": ms, "steps": args.steps, "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": args.workload, "B": s.B, "T": s.T, "N": s.N, "H": s.H,
+                                        "d": s.d_k, "L": s.L},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks.get("bf16_tflops", 1590.0),
+                     "unit": "TFLOP/s", "frac": tflops / peaks.get("bf16_tflops", 1590.0),
+                     "peak_source": f"bf16_tflops ({src})", "hbm_gbs": hbm},
+        "clocks": clocks}), flush=True)
+
+
 def main():
     args = parse()
+    if args.xattn:
+        run_xattn(args)
+        return
     if args.proj:
         run_proj(args)
         return

@@ -207,6 +207,22 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg *cfg, unsigned stage);
 /* Static description of a status code. */
 const char *vdn_status_string(vdn_status s);
 
+/* ------------------------------------------------------- text cross-attention
+ * The DiT block's softmax cross-attention from the video tokens to the text
+ * tokens (PaperDaily digest section 三: text enters the block both through the
+ * states' initialisation and through cross-attention): for every video query
+ * of batch b and head h, o = softmax(s q K_b^T) V_b over that batch's L text
+ * tokens (no mask, no gate), s = cfg.softmax_scale (<= 0: 1/sqrt(d_k)).
+ * Reads cfg B, T, N, H, d_k = d_v (64 or 128), L >= 1, dtype (VDN_BF16 only),
+ * softmax_scale, y_dtype; args q [B,T,N,H,d_k], text_k [B,L,H,d_k],
+ * text_v [B,L,H,d_v], y = the output o [B,T,N,H,d_v] in y_dtype, and the first
+ * 256 bytes of workspace (status words, read by vdn_hybrid_device_status);
+ * the other pointers are ignored.  On the tensor cores (the windowed softmax's
+ * kernel with one key interval).  Errors: VDN_ERR_INVALID_ARG (L = 0, a NULL or
+ * misaligned pointer), VDN_ERR_WORKSPACE (workspace NULL, misaligned or under
+ * 256 bytes), VDN_ERR_UNSUPPORTED (fp32 inputs, d not 64 or 128). */
+vdn_status vdn_text_cross_attn(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args, vdn_stream_t stream);
+
 /* ------------------------------------------------ the layer's output projection
  * PaperDaily digest section 三: each branch is gated, then projected back to
  * the model width.  With the core's output in out_mode 0 (y[B,T,N,H,2,d_v],

@@ -320,6 +320,17 @@ def softmax_attend(q, keys, vals, scale: float):
     return p @ np.asarray(vals, F64)
 
 
+def text_cross_attn(q_bh, text_k_bh, text_v_bh, scale: float):
+    """The block's softmax cross-attention from the video tokens to the text
+    tokens ([P1] 三: the prompt reaches the block through cross-attention as
+    well as through the half-text states): every query of one (batch, head),
+    q_bh [T, N, d_k], over all L text tokens of that batch, no mask, no gate.
+    Returns [T, N, d_v]."""
+    T, N, dk = np.shape(q_bh)
+    o = softmax_attend(np.reshape(q_bh, (T * N, dk)), text_k_bh, text_v_bh, scale)
+    return o.reshape(T, N, -1)
+
+
 def softmax_frame(q_t, k_bh, v_bh, t: int, T: int, chunk: int, anchors: int, scale: float):
     """Softmax output for the queries of frame t of one (batch, head):
     keys are the tokens of every frame the frame mask allows."""

@@ -156,3 +156,18 @@ def test_out_proj_bad_args_rejected():
                                  (8, 64, 64, 7, p, p, p), (8, 64, 64, 0, None, p, p), (8, 64, 64, 0, p + 8, p, p)]:
         assert L.vdn_out_proj(M, K, N, od, y, w, o, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
     assert L.lib().vdn_out_proj(None, None, None, None, None) == L.VDN_ERR_INVALID_ARG
+
+
+def test_text_cross_attn_rejected_before_launch():
+    p = 1 << 20
+    def call(cfg, **over):
+        a = dict(q=p, k=None, v=None, beta=None, alpha=None, gate_sm=None, gate_lin=None, y=p, workspace=p,
+                 workspace_bytes=256, text_k=p, text_v=p)
+        a.update(over)
+        return L.vdn_text_cross_attn(cfg, L.make_args(**a), stream=0, check=False)
+    assert call(_cfg(L=0)) == L.VDN_ERR_INVALID_ARG
+    assert call(_cfg(), text_k=None) == L.VDN_ERR_INVALID_ARG
+    assert call(_cfg(), y=p + 4) == L.VDN_ERR_INVALID_ARG
+    assert call(_cfg(), workspace_bytes=128) == L.VDN_ERR_WORKSPACE
+    assert call(_cfg(dtype=L.VDN_F32)) == L.VDN_ERR_UNSUPPORTED
+    assert call(_cfg(d_k=32, d_v=32)) == L.VDN_ERR_UNSUPPORTED

@@ -443,3 +443,15 @@ def test_out_proj_is_the_sum_of_the_branch_projections():
     for h in range(H):
         ref += y[..., h, 0, :] @ W_sm[h] + y[..., h, 1, :] @ W_lin[h]
     np.testing.assert_allclose(O.out_proj(y, W), ref, rtol=0, atol=1e-12)
+
+
+def test_text_cross_attn_equals_torch_sdpa():
+    """The text cross-attention against torch's scaled-dot-product attention
+    (no mask), a library routine, on random fp64 inputs."""
+    r = np.random.default_rng(31)
+    T, N, L, d = 3, 5, 7, 8
+    q, k, v = r.standard_normal((T, N, d)), r.standard_normal((L, d)), r.standard_normal((L, d))
+    got = O.text_cross_attn(q, k, v, 0.4)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q.reshape(1, T * N, d)), torch.from_numpy(k[None]), torch.from_numpy(v[None]), scale=0.4)
+    np.testing.assert_allclose(got, ref.numpy().reshape(T, N, d), rtol=0, atol=1e-12)

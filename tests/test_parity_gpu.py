@@ -421,3 +421,28 @@ def test_out_proj_on_core_output():
     ref = O.out_proj(oracle(inp, cfg), wt.float().cpu().numpy()).reshape(M, n)
     e = rel_err(out.cpu().numpy().astype(np.float64), ref)
     assert e <= TOL["bf16"], e
+
+
+# ------------------------------------------------------------ text cross-attention
+@pytest.mark.parametrize("y_bf16", [False, True])
+@pytest.mark.parametrize("shape", [Shape(1, 6, 50, 2, 64, 64, 40), Shape(2, 4, 70, 3, 128, 128, 300)])
+def test_text_cross_attn_matches_oracle(shape, y_bf16):
+    """Every video query over its batch's L text tokens (one partial key tile
+    at L = 40; three tiles, the last partial, at L = 300), against the oracle."""
+    inp = make_inputs(shape, 17, "bf16")
+    cfg = cfg_for(shape, "bf16", y_dtype=L.VDN_BF16 if y_bf16 else L.VDN_F32)
+    t = to_torch(inp, "bf16", "cuda")
+    y = torch.empty((shape.B, shape.T, shape.N, shape.H, shape.d_v),
+                    dtype=torch.bfloat16 if y_bf16 else torch.float32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    args = L.make_args(t["q"], None, None, None, None, None, None, y, ws, text_k=t["text_k"], text_v=t["text_v"])
+    L.vdn_text_cross_attn(cfg, args)
+    torch.cuda.synchronize()
+    assert L.vdn_hybrid_device_status(cfg, args)[0] == L.VDN_OK
+    got = y.float().cpu().numpy().astype(np.float64)
+    scale = 1.0 / np.sqrt(shape.d_k)
+    for b in range(shape.B):
+        for h in range(shape.H):
+            ref = O.text_cross_attn(inp["q"][b, :, :, h], inp["text_k"][b, :, h], inp["text_v"][b, :, h], scale)
+            e = rel_err(got[b, :, :, h], ref, U_BF16 * np.abs(ref) if y_bf16 else None)
+            assert e <= TOL["bf16"], (b, h, e)

@@ -22,7 +22,7 @@ STAGE_ALL = 31
 
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
-            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj")
+            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -111,6 +111,8 @@ def lib() -> C.CDLL:
         L.vdn_hybrid_stage_impl.argtypes = [C.POINTER(VdnCfg), C.c_uint]
         L.vdn_hybrid_attn_fwd_noalloc.restype = C.c_int
         L.vdn_hybrid_attn_fwd_noalloc.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
+        L.vdn_text_cross_attn.restype = C.c_int
+        L.vdn_text_cross_attn.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
         L.vdn_out_proj.restype = C.c_int
         L.vdn_out_proj.argtypes = [C.POINTER(ProjCfg), C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
         L.vdn_status_string.restype = C.c_char_p
@@ -142,6 +144,15 @@ def vdn_out_proj(M: int, K: int, N: int, out_dtype: int, y, w, out, stream=None,
     st = lib().vdn_out_proj(C.byref(c), _ptr(y), _ptr(w), _ptr(out), _stream_handle(stream))
     if check and st != VDN_OK:
         raise VdnError(st, "vdn_out_proj")
+    return st
+
+
+def vdn_text_cross_attn(cfg: HybridCfg, args: VdnArgs, stream=None, check: bool = True) -> int:
+    """Text cross-attention: args.q, text_k, text_v in, args.y out, args.workspace (status words)."""
+    c = cfg.c()
+    st = lib().vdn_text_cross_attn(C.byref(c), C.byref(args), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_text_cross_attn")
     return st
 
 

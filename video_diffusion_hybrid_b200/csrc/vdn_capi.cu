@@ -263,6 +263,25 @@ vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg* cfg, const vdn_hybrid_
   return host[0] ? VDN_ERR_TIMEOUT : VDN_OK;
 }
 
+vdn_status vdn_text_cross_attn(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, vdn_stream_t stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!args) return VDN_ERR_INVALID_ARG;
+  if (cfg->L <= 0) return VDN_ERR_INVALID_ARG;
+  const void* req[] = {args->q, args->text_k, args->text_v, args->y};
+  for (const void* p : req)
+    if (!p || !aligned(p, 16)) return VDN_ERR_INVALID_ARG;
+  if (!args->workspace || !aligned(args->workspace, kAlign) || args->workspace_bytes < kAlign) return VDN_ERR_WORKSPACE;
+  const Dims d = make_dims(cfg);
+  if (!softmax_tc_supported(d)) return VDN_ERR_UNSUPPORTED;  // bf16, d = 64 or 128
+  if ((long long)d.B * d.L + 256 >= (1LL << 31)) return VDN_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Work w{};
+  w.status = static_cast<uint32_t*>(args->workspace);  // the status words (as in the core's layout)
+  if (cudaMemsetAsync(w.status, 0, kAlign, s) != cudaSuccess) return VDN_ERR_CUDA;
+  return launch_text_xattn_tc(d, inputs_of(args), w, s) == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
 vdn_status vdn_out_proj(const vdn_proj_cfg* cfg, const void* y, const void* w, void* out, vdn_stream_t stream) {
   if (!cfg || !y || !w || !out) return VDN_ERR_INVALID_ARG;
   if (cfg->M < 1 || cfg->K < 8 || cfg->N < 8 || cfg->K % 8 || cfg->N % 8) return VDN_ERR_INVALID_ARG;

@@ -66,6 +66,8 @@ cudaError_t launch_read_simt(const Dims& d, const Inputs& in, const Work& w, cud
 cudaError_t launch_softmax_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 bool softmax_tc_supported(const Dims& d);
 cudaError_t launch_softmax_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+// text cross-attention: every query over the L text tokens of its batch, y[B,T,N,H,d_v]
+cudaError_t launch_text_xattn_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 bool read_tc_supported(const Dims& d);
 // the workspace holds the bf16 split of M (and the solve writes it) exactly when this holds
 __host__ __device__ inline bool scan_tc_layout(bool bf16, int dk, int dv) { return bf16 && dk == 128 && dv == 128; }

@@ -87,6 +87,24 @@ __host__ __device__ inline void group_frames(const Dims& d, int g, int& f0, int&
 
 __host__ __device__ inline long long pairs_of_rows(long long rows) { return (rows + NQ * BM - 1) / (NQ * BM); }
 
+// Text cross-attention: item -> 256 query rows of one (b, h) over all T*N
+// video tokens; one key interval, the L text tokens of batch b.
+__device__ bool decode_item_cross(const Dims& d, long long item, Tile& t) {
+  const long long rows = (long long)d.T * d.N;
+  const long long per_bh = pairs_of_rows(rows);
+  const long long bh = item / per_bh, qp = item % per_bh;
+  if (bh >= (long long)d.B * d.H) return false;
+  t.b = (int)(bh / d.H);
+  t.h = (int)(bh % d.H);
+  t.q0 = (int)((long long)t.b * rows + qp * NQ * BM);
+  t.qrows = (int)min((long long)NQ * BM, rows - qp * NQ * BM);
+  t.niv = 3;
+  t.kbeg[0] = t.b * d.L; t.klen[0] = d.L;
+  t.kbeg[1] = 0; t.klen[1] = 0;
+  t.kbeg[2] = 0; t.klen[2] = 0;
+  return true;
+}
+
 // Item order: all anchor-row pairs first (longest), then per (b, h) the
 // regular groups in chunk order, so concurrent CTAs share K/V windows in L2.
 __device__ bool decode_item(const Dims& d, long long item, Tile& t) {
@@ -206,7 +224,9 @@ __device__ __forceinline__ void add_bf16x2_f32(float& s_lo, float& s_hi, uint32_
 }
 
 // ------------------------------------------------------------------ kernel --
-template <int D, typename To>
+// X: the text cross-attention (keys and values from the text tokens, every
+// query sees all of its batch's L text tokens, no gate, y[B,T,N,H,d_v]).
+template <int D, typename To, bool X>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
              const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
@@ -231,7 +251,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   // a CTA of this launch already gave up on a wait: fail fast, touch nothing
   if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
   Tile tile;
-  if (!decode_item(dm, blockIdx.x, tile)) return;  // uniform across the CTA
+  if (!(X ? decode_item_cross(dm, blockIdx.x, tile) : decode_item(dm, blockIdx.x, tile))) return;  // uniform
   const int ntiles = num_key_tiles(tile);
   const Ctl ctl{abort_flag, w.status, (unsigned)TAG_SOFTMAX_TC};
   auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -490,13 +510,17 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       const bool valid = trow < tile.qrows;
       const long long tok = (long long)tile.q0 + trow;
       const long long gi = (tok * dm.H + tile.h) * D;
-      To* y = static_cast<To*>(in.y) + (dm.out_mode == 0 ? 2 * gi : gi);
+      To* y = static_cast<To*>(in.y) + ((!X && dm.out_mode == 0) ? 2 * gi : gi);
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         float v[32];
         tmem_ld32(ocol + q * 32, v);
         tmem_wait_ld();
-        if (valid) {
+        if (valid && X) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            store4<To>(y + q * 32 + i, v[i] * inv, v[i + 1] * inv, v[i + 2] * inv, v[i + 3] * inv);
+        } else if (valid) {
           float g[32];
           if (dm.bf16) {
             const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(in.gate_sm) + gi + q * 32);
@@ -546,18 +570,20 @@ long long num_items(const Dims& d) {
   return (long long)d.B * d.H * (per_bh + n_anc * pairs_of_rows(d.N));
 }
 
-template <int D, typename To>
+template <int D, typename To, bool X>
 cudaError_t launch_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   const long long tokens = (long long)d.B * d.T * d.N;
-  if (!make_token_map(&mq, in.q, tokens, d.H, D, BM) || !make_token_map(&mk, in.k, tokens, d.H, D, BN) ||
-      !make_token_map(&mv, in.v, tokens, d.H, D, BN))
+  const long long ktok = X ? (long long)d.B * d.L : tokens;  // key / value tokens
+  if (!make_token_map(&mq, in.q, tokens, d.H, D, BM) ||
+      !make_token_map(&mk, X ? in.text_k : in.k, ktok, d.H, D, BN) ||
+      !make_token_map(&mv, X ? in.text_v : in.v, ktok, d.H, D, BN))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + (size_t)NQ * BM * D * 2 + 5 * (size_t)BN * D * 2 + 22 * 8 + 16;
-  auto kern = k_softmax_tc<D, To>;
+  auto kern = k_softmax_tc<D, To, X>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long long items = num_items(d);
+  const long long items = X ? (long long)d.B * d.H * pairs_of_rows((long long)d.T * d.N) : num_items(d);
   if (items <= 0 || items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
   kern<<<(unsigned)items, kThreadsTC, smem, s>>>(d, in, w, mq, mk, mv);
   return cudaGetLastError();
@@ -574,8 +600,19 @@ bool softmax_tc_supported(const Dims& d) {
 }
 
 cudaError_t launch_softmax_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
-  if (d.dk == 128) return d.out_bf16 ? launch_tc<128, __nv_bfloat16>(d, in, w, s) : launch_tc<128, float>(d, in, w, s);
-  if (d.dk == 64) return d.out_bf16 ? launch_tc<64, __nv_bfloat16>(d, in, w, s) : launch_tc<64, float>(d, in, w, s);
+  if (d.dk == 128)
+    return d.out_bf16 ? launch_tc<128, __nv_bfloat16, false>(d, in, w, s) : launch_tc<128, float, false>(d, in, w, s);
+  if (d.dk == 64)
+    return d.out_bf16 ? launch_tc<64, __nv_bfloat16, false>(d, in, w, s) : launch_tc<64, float, false>(d, in, w, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_text_xattn_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  if (d.L <= 0 || (long long)d.B * d.L + NQ * BM >= (1LL << 31)) return cudaErrorInvalidValue;
+  if (d.dk == 128)
+    return d.out_bf16 ? launch_tc<128, __nv_bfloat16, true>(d, in, w, s) : launch_tc<128, float, true>(d, in, w, s);
+  if (d.dk == 64)
+    return d.out_bf16 ? launch_tc<64, __nv_bfloat16, true>(d, in, w, s) : launch_tc<64, float, true>(d, in, w, s);
   return cudaErrorInvalidValue;
 }
 
