@@ -247,6 +247,7 @@ def stage_rooflines(s, cfg, ms, y_elem, peaks, sm_mhz):
     """Each stage's time (CUDA events, the stage launched alone on resident
     inputs) against the roofline of what it must compute or move."""
     from video_diffusion_hybrid_b200 import roofline as R
+    from video_diffusion_hybrid_b200 import _lib as L
     elem = 2 if cfg.dtype == 1 else 4
     hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops_sustained"]
     simt = R.fp32_simt_tflops(sm_mhz)
@@ -264,7 +265,8 @@ def stage_rooflines(s, cfg, ms, y_elem, peaks, sm_mhz):
     # per-frame Gram (HBM-bound) followed by the SPD sweep (fp32 SIMT-bound):
     # the floor is the sum of the two
     gb = R.gram_bytes(s.B, s.T, s.N, s.H, s.d_k, cfg.anchors, elem)
-    sf = R.sweep_flops(s.B, s.T, s.H, s.d_k, cfg.anchors)
+    # the tensor-core scan takes B_t itself, so its solve forms no C = B M
+    sf = R.sweep_flops(s.B, s.T, s.H, s.d_k, cfg.anchors, with_c=L.vdn_hybrid_stage_impl(cfg, L.STAGE_SCAN) != 1)
     floor_ms = 1e3 * (gb / (hbm * 1e9) + sf / (simt * 1e12))
     out["solve"] = {"ms": ms["solve"], "bound": "hbm+alu", "floor_ms": floor_ms, "frac": floor_ms / ms["solve"],
                     "gram_bytes": gb, "sweep_flops": sf, "alu_peak_tflops": simt}

@@ -102,7 +102,7 @@ Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
   vdn_workspace_layout L;
   layout_of(c, &L);
   char* base = static_cast<char*>(a->workspace);
-  Work w;
+  Work w{};
   w.status = reinterpret_cast<uint32_t*>(base + L.status);
   w.half_text = reinterpret_cast<float*>(base + L.half_text);
   w.M = reinterpret_cast<float*>(base + L.frame_M);
@@ -180,9 +180,13 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
   if (st != VDN_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const Dims d = make_dims(cfg);
-  const Work w = work_of(cfg, args);
   const Inputs in = inputs_of(args);
   const bool big = big_d(d);
+  Work w = work_of(cfg, args);
+  // the tensor-core scan (and its solve) take the B form: every call with this
+  // configuration decides the same way, so stages run in separate calls agree
+  const bool tc_scan = !big && scan_tc_supported(d) && w.M16 != nullptr;
+  w.bform = tc_scan ? 1 : 0;
   // d = 256: the VDA stages only (the softmax stage has no kernel at this size)
   if (big && ((stages & VDN_STAGE_SOFTMAX) || !gram_tc_supported(d))) return VDN_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
@@ -211,7 +215,7 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     // the tensor-core scan reads the bf16 split of M that the sweep solve
     // writes; with enough chunks it first composes each chunk's frame maps
     // and steps by whole chunks
-    if (scan_tc_supported(d) && w.M16 != nullptr) {
+    if (tc_scan) {
       int dev = 0, sms = 0;
       if (cudaGetDevice(&dev) != cudaSuccess ||
           cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

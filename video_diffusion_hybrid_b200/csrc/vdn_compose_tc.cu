@@ -11,7 +11,8 @@
 //   backward S -> Lam S P^T + Cb,  Cb <- alpha_f Cb M_f + C_f  (f decreasing, from 0)
 // (the reversed product of the symmetric M_f is P^T).  Both chains are the
 // scan's own step X <- alpha X M + C over the chunk's frames: the P chain
-// from X = I with alpha = 1 and no C, the two Horner chains from X = 0.
+// from X = I with alpha = 1 and no C, the two Horner chains from X = 0, run
+// as X <- (alpha X + B_f) M_f since C_f = B_f M_f (the solve leaves B_f).
 // The chunk-stepped scan then takes 1 / chunk of the frame scan's steps.
 //
 // One CTA per (chunk, batch-head) and direction (384 threads): the forward
@@ -198,7 +199,11 @@ k_compose_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm
     __nv_bfloat16* p_lo = p_hi + DD;
     float* cf_row = w.Cf + bch * DD + (long long)row * D;
     float* cb_row = w.Cb + bch * DD + (long long)row * D;
-    // start operands: P = I (forward), Cf = Cb = 0
+    // The Horner chains in the B form (the solve left B_f in the C_f slot):
+    // X <- alpha_f X M_f + B_f M_f = (alpha_f X + B_f) M_f, so step i multiplies
+    // alpha_{f_i} X_{i-1} + B_{f_i} (formed here) by M_{f_i}.  Start operands:
+    // P = I (forward) and the first frame's B (X_0 = 0).
+    auto brow = [&](int i) { return w.Cm + fh_of(fr.f[i]) * DD + (long long)row * D; };
 #pragma unroll 1
     for (int q = 2 * half; q < 2 * half + 2; ++q) {
       float s0[32], z[32];
@@ -215,8 +220,17 @@ k_compose_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm
           store_f32(cb_row + q * 32, z);
         }
       } else {
-        split_to_smem(q, row, sA0, s0);
-        if (fwd) split_to_smem(q, row, sA1, z);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 b4 = __ldg(reinterpret_cast<const float4*>(brow(0) + q * 32) + u);
+          z[4 * u] = b4.x; z[4 * u + 1] = b4.y; z[4 * u + 2] = b4.z; z[4 * u + 3] = b4.w;
+        }
+        if (fwd) {
+          split_to_smem(q, row, sA0, s0);
+          split_to_smem(q, row, sA1, z);
+        } else {
+          split_to_smem(q, row, sA0, z);
+        }
       }
     }
     if (n > 0) {
@@ -225,11 +239,11 @@ k_compose_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm
     }
     float lam = 1.f;
     for (int i = 0; i < n; ++i) {
-      const long long fh = fh_of(fr.f[i]);
-      const float alpha = __ldg(in.alpha + fh);
-      lam *= alpha;
-      const float* crow = w.Cm + fh * DD + (long long)row * D;
+      lam *= __ldg(in.alpha + fh_of(fr.f[i]));
       const bool last = i == n - 1;
+      // the next frame's alpha and B rows (the next step's operand)
+      const float anext = last ? 0.f : __ldg(in.alpha + fh_of(fr.f[i + 1]));
+      const float* bnext = last ? nullptr : brow(i + 1);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MDONE), i & 1, ctl))) break;
       tc_fence_after();
 #pragma unroll 1
@@ -239,27 +253,25 @@ k_compose_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm
         tmem_ld32(lane_addr + qq * 32, x);
         if (fwd) tmem_ld32(lane_addr + 128 + qq * 32, y);
         tmem_wait_ld();
-        // the Horner chain: alpha (X M) + C_f
-        float* acc = fwd ? y : x;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 c4 = __ldg(reinterpret_cast<const float4*>(crow + q * 32) + u);
-          acc[4 * u] = fmaf(alpha, acc[4 * u], c4.x);
-          acc[4 * u + 1] = fmaf(alpha, acc[4 * u + 1], c4.y);
-          acc[4 * u + 2] = fmaf(alpha, acc[4 * u + 2], c4.z);
-          acc[4 * u + 3] = fmaf(alpha, acc[4 * u + 3], c4.w);
-        }
-        if (fwd) {
-          if (last) {
+        float* acc = fwd ? y : x;  // the Horner chain's new value
+        if (last) {
+          if (fwd) {
             split_to_global(p_hi, p_lo, q, x);
             store_f32(cf_row + q * 32, y);
           } else {
-            split_to_smem(q, row, sA0, x);
-            split_to_smem(q, row, sA1, y);
+            store_f32(cb_row + q * 32, x);
           }
         } else {
-          if (last) store_f32(cb_row + q * 32, x);
-          else split_to_smem(q, row, sA0, x);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {  // the next operand: alpha_next X + B_next
+            const float4 b4 = __ldg(reinterpret_cast<const float4*>(bnext + q * 32) + u);
+            acc[4 * u] = fmaf(anext, acc[4 * u], b4.x);
+            acc[4 * u + 1] = fmaf(anext, acc[4 * u + 1], b4.y);
+            acc[4 * u + 2] = fmaf(anext, acc[4 * u + 2], b4.z);
+            acc[4 * u + 3] = fmaf(anext, acc[4 * u + 3], b4.w);
+          }
+          split_to_smem(q, row, sA0, x);
+          if (fwd) split_to_smem(q, row, sA1, y);
         }
       }
       tc_fence_before();  // TMEM reads done before the next products

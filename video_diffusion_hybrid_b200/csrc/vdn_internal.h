@@ -38,6 +38,9 @@ struct Work {
   float* Cf;         // [B,C,H,dv,dk]; Cb follows at Cf + B*C*H*dv*dk
   float* Cb;         // [B,C,H,dv,dk]
   float* lam;        // [B,C,H]
+  // 1 when the tensor-core scan runs: it forms (alpha S + B_t) M_t itself, so
+  // the solve leaves B_t in the C_t slot and skips the product C_t = B_t M_t
+  int bform;
 };
 
 struct Inputs {

@@ -307,10 +307,40 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
     const long long DD = (long long)D * D;
     const int row = row0 + srow;  // state row
     float* snap_row = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD + (long long)row * D;
-    // start state: its own slot, then (frame steps) the slots of leading
-    // unwritten frames
+    // C-slot item k (one per step, slot k & 1): this CTA's 32 columns of its
+    // row, into registers; the slot goes back to the producer at once
+    auto read_c = [&](int k, float (&cv)[32]) -> bool {
+      const int slot = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait_cl(bar(B_CFULL + slot), (k >> 1) & 1, ctl))) return false;
+      const unsigned char* crow = sC + slot * CBYTES + q * CBOX + srow * 128;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4 c4 = *reinterpret_cast<const float4*>(crow + ((u ^ (srow & 7)) << 4));
+        cv[4 * u] = c4.x; cv[4 * u + 1] = c4.y; cv[4 * u + 2] = c4.z; cv[4 * u + 3] = c4.w;
+      }
+      mbar_arrive_warp(bar(B_CEMPTY + slot));
+      return true;
+    };
+    // x <- a x + c (both 32 values, paired fp32 FMAs)
+    auto axpy = [&](float a, float (&x)[32], const float (&c)[32], float (&out)[32]) {
+      const float2 a2 = make_float2(a, a);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float2 r = fma2(a2, make_float2(x[2 * u], x[2 * u + 1]), make_float2(c[2 * u], c[2 * u + 1]));
+        out[2 * u] = r.x;
+        out[2 * u + 1] = r.y;
+      }
+    };
+    // Frame steps (B form): step i's product is X_i M_t with X_i = alpha_t S + B_t
+    // (the solve left B_t in the C_t slot), so the product is the new state and
+    // the epilogue of step i forms X_{i+1} from the next frame's alpha and B.
+    // Chunk steps (C form): the product is S P (or S P^T), the epilogue adds
+    // Lam and the chunk constant.
     int st = CH ? 0 : next_written(dm, dir, 0);
+    bool ok = true;
     {
+      // start state: its own slot, then (frame steps) the slots of leading
+      // unwritten frames
       const float* src = w.half_text + (long long)bh * DD + (long long)row * D;
       const int start_slot = dir == 0 ? 0 : dm.C;
       float s[32];
@@ -319,48 +349,53 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
         const float4 v = __ldg(reinterpret_cast<const float4*>(src + q * 32) + u);
         s[4 * u] = v.x; s[4 * u + 1] = v.y; s[4 * u + 2] = v.z; s[4 * u + 3] = v.w;
       }
-      split_chunk(q, srow, sA, s);
-      fence_proxy_async_smem();
-      arrive_cluster_warp(lbar(B_SREADY));
+      if (CH) {
+        split_chunk(q, srow, sA, s);
+      } else if (nw > 0) {
+        float x[32];
+        ok = read_c(0, x);
+        if (ok) {
+          axpy(__ldg(in.alpha + fh_of(frame_at(dm, dir, st))), s, x, x);
+          split_chunk(q, srow, sA, x);
+        }
+      }
+      if (ok) {
+        fence_proxy_async_smem();
+        arrive_cluster_warp(lbar(B_SREADY));
+      }
       store_row32(snap_row + start_slot * DD + q * 32, s);
       if (!CH) snap_chunk(dm, dir, slots_of(dm, dir, 0, st), snap_row, q, s);
     }
-    for (int i = 0; i < nw; ++i) {
-      const int slot = i & 1;
+    for (int i = 0; ok && i < nw; ++i) {
       const int st_next = CH ? st + 1 : next_written(dm, dir, st + 1);
-      // chunk step: the map's Lam, and the slot of the chunk boundary it ends on
-      const int cst = chunk_of(i);
-      const float alpha = CH ? w.lam[bch_of(cst)] : __ldg(in.alpha + fh_of(frame_at(dm, dir, st)));
+      const int cst = chunk_of(i);  // chunk steps: the chunk, and the boundary slot it ends on
       const Slots sl = CH ? Slots{dir == 0 ? cst + 1 : cst, -1, 0, 0} : slots_of(dm, dir, st, st_next);
-      // this step's C row chunk into registers first (it does not depend on
-      // the product), then the slot goes back to the producer
-      if (!__all_sync(0xffffffffu, mbar_wait_cl(bar(B_CFULL + slot), (i >> 1) & 1, ctl))) break;
+      const bool more = i + 1 < nw;
+      // the C-slot values this epilogue adds (they do not depend on the
+      // product): chunk steps this step's constant, frame steps the next B
       float cv[32];
-      {
-        const unsigned char* crow = sC + slot * CBYTES + q * CBOX + srow * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 c4 = *reinterpret_cast<const float4*>(crow + ((u ^ (srow & 7)) << 4));
-          cv[4 * u] = c4.x; cv[4 * u + 1] = c4.y; cv[4 * u + 2] = c4.z; cv[4 * u + 3] = c4.w;
-        }
+      if (CH || more) {
+        if (!read_c(CH ? i : i + 1, cv)) break;
       }
-      mbar_arrive_warp(bar(B_CEMPTY + slot));
+      const float alpha = CH ? w.lam[bch_of(cst)]
+                             : (more ? __ldg(in.alpha + fh_of(frame_at(dm, dir, st_next))) : 0.f);
       if (!__all_sync(0xffffffffu, mbar_wait_cl(bar(B_MDONE), i & 1, ctl))) break;
       tc_fence_after();
       float v[32];
       tmem_ld32(lane_addr, v);
       tmem_wait_ld();
       tc_fence_before();  // TMEM reads done before the next product
-      const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {  // S = alpha (S M) + C
-        const float2 r = fma2(a2, make_float2(v[2 * u], v[2 * u + 1]), make_float2(cv[2 * u], cv[2 * u + 1]));
-        v[2 * u] = r.x;
-        v[2 * u + 1] = r.y;
+      if (CH) {
+        axpy(alpha, v, cv, v);  // S = Lam (S P) + Cf
+        split_chunk(q, srow, sA, v);
+      } else if (more) {
+        axpy(alpha, v, cv, cv);  // X = alpha_next S + B_next; v is the new state
+        split_chunk(q, srow, sA, cv);
       }
-      split_chunk(q, srow, sA, v);
-      fence_proxy_async_smem();  // new A operand visible to the tensor cores
-      arrive_cluster_warp(lbar(B_SREADY));
+      if (CH || more) {
+        fence_proxy_async_smem();  // new A operand visible to the tensor cores
+        arrive_cluster_warp(lbar(B_SREADY));
+      }
       // snapshots after the hand-off: the next product does not wait for them
       snap_chunk(dm, dir, sl, snap_row, q, v);
       st = st_next;

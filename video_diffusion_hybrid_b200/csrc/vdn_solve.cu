@@ -79,10 +79,12 @@ k_solve_sweep(Dims dm, Work w) {
 
   sweep_regs<D>(g, rowbuf);  // g = -G^-1
 
+  // the tensor-core scan forms (alpha S + B_t) M_t itself: no C_t
+  const bool skip_c = !TEXT && w.bform;
   // M = -G_swept: to global and to shared for C = B M
 #pragma unroll
   for (int a = 0; a < R; ++a) {
-    st_row<R>(Ms + (r0 + a) * P + c0, g[a], -1.0f);
+    if (!skip_c) st_row<R>(Ms + (r0 + a) * P + c0, g[a], -1.0f);
     if (!TEXT) st_row<R>(gA + (r0 + a) * D + c0, g[a], -1.0f);
   }
   if constexpr (!TEXT && R == 8) {
@@ -101,6 +103,7 @@ k_solve_sweep(Dims dm, Work w) {
       }
     }
   }
+  if (skip_c) return;  // uniform: B_t stays in the C_t slot
   __syncthreads();
   float acc[R][R];
 #pragma unroll

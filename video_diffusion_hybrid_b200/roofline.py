@@ -58,10 +58,11 @@ def gram_bytes(B, T, N, H, d, anchors=4, elem=2) -> float:
     return nw * B * H * (N * (2 * d * elem + 4) + 2 * d * d * 4)
 
 
-def sweep_flops(B, T, H, d, anchors=4) -> float:
+def sweep_flops(B, T, H, d, anchors=4, with_c=True) -> float:
     """SPD solve per written frame-head: d pivots of a d x d rank-one update
-    (d^3 multiply-adds) plus C = B M (d^3 multiply-adds)."""
-    return 4.0 * d ** 3 * written_frames(T, anchors) * B * H
+    (d^3 multiply-adds), plus C = B M (d^3 multiply-adds) where the scan
+    needs C (the tensor-core scan forms (alpha S + B) M itself: with_c=False)."""
+    return (4.0 if with_c else 2.0) * d ** 3 * written_frames(T, anchors) * B * H
 
 
 def scan_bytes(B, T, H, d, chunk=5, anchors=4) -> float:
