@@ -129,8 +129,9 @@ enum {
  *   half_text  : [B,H,d_v,d_k]        S_x / 2, the start state of both scans
  *   frame_M    : [B,T,H,d_k,d_k]      (I + A_t)^{-1}        (anchor frames unset)
  *   frame_C    : [B,T,H,d_v,d_k]      C_t = B_t (I + A_t)^{-1}  (anchor frames unset); with the
- *                                     tensor-core scan (bf16, d = 128) the write matrix B_t
- *                                     itself, since that scan steps S <- (alpha_t S + B_t) M_t
+ *                                     tensor-core scan (bf16, d = 128) and at d = 256 the write
+ *                                     matrix B_t itself, since those scans step
+ *                                     S <- (alpha_t S + B_t) M_t
  *   fwd_snap   : [B,H,C+1,d_v,d_k]    forward state over frames < min(5j, T)
  *   bwd_snap   : [B,H,C+1,d_v,d_k]    backward state over frames >= min(5j, T)
  *   read_table : [B,H,C+1,d_v,d_k]    R[c] = fwd_snap[max(c-1,0)] + bwd_snap[min(c+2,C)],

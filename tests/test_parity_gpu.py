@@ -159,7 +159,8 @@ def test_bf16_frame_maps_match_oracle(shape):
 @pytest.mark.parametrize("shape", [Shape(1, 12, 96, 2, 256, 256, 16), Shape(1, 10, 40, 1, 256, 256, 0)])
 def test_d256_vda_matches_oracle(shape):
     """d = 256, the Video Delta Attention stages (the only ones at this size):
-    M_t, C_t and S_x / 2 after the block-mode Gram and the block solve, the
+    M_t, B_t (the scan steps S <- (alpha S + B_t) M_t, so the C_t slot keeps
+    B_t) and S_x / 2 after the block-mode Gram and the block solve, the
     read table after the chunked scans, and the linear slot of every output
     after the chunked read, against the oracle."""
     inp, cfg, ha, t, y = run(shape, "bf16", 21, drop_text=shape.L == 0, stages=VDA)
@@ -171,7 +172,10 @@ def test_d256_vda_matches_oracle(shape):
             np.testing.assert_allclose(it["half_text"][b, h], ref["S_init"], atol=2e-5 * sx)
             for f in range(1, cfg.T - 1):
                 np.testing.assert_allclose(it["M"][b, f, h], ref["M"][f], atol=2e-5)
-                np.testing.assert_allclose(it["C"][b, f, h], ref["C"][f], atol=2e-5 * np.abs(ref["C"][f]).max())
+                Bf = O.gram_write(np.asarray(inp["k"][b, f, :, h], np.float64),
+                                  np.asarray(inp["v"][b, f, :, h], np.float64),
+                                  np.asarray(inp["beta"][b, f, :, h], np.float64))[1]
+                np.testing.assert_allclose(it["C"][b, f, h], Bf, atol=2e-5 * np.abs(Bf).max())
             np.testing.assert_allclose(it["R"][b, h], ref["R"], atol=1e-4 * np.sqrt(np.mean(ref["R"] ** 2)) + 1e-30)
     ref_y = O.hybrid_attn(inp, ocfg(cfg))
     assert rel_err(y[..., 1, :], ref_y[..., 1, :]) <= TOL["bf16"]

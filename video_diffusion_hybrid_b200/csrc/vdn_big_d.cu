@@ -9,8 +9,8 @@
 // "用兩條分支取代一條", the closed form S_t = (alpha_t S_{t-1} + B_t)(I + A_t)^-1;
 // PaperDaily digest sections 三 and 四, the two scans, the half-text start
 // states and the read):
-//   M_t = (I + A_t)^-1,  C_t = B_t M_t,
-//   S <- alpha_t S M_t + C_t forward and backward (anchors: identity),
+//   M_t = (I + A_t)^-1,
+//   S <- (alpha_t S + B_t) M_t forward and backward (anchors: identity),
 //   o = R q with R = forward + backward chunk-boundary states, RMSNorm, gate.
 #include "vdn_internal.h"
 #include "simt_common.cuh"
@@ -187,6 +187,8 @@ k_solve_block(Dims dm, Work w) {
   mm128<false, true, true>(g, T0, T2);
   tile_st(blk(gM, 0, 0), DB, g, 1.f);
   __syncthreads();  // M complete in global memory
+  // frames: the scan steps S <- (alpha S + B_t) M_t itself, B_t stays in the C_t slot
+  if (!TEXT && w.bform) return;
 
   // C = B M by blocks: C(rb, cb) = B(rb, 0) M(0, cb) + B(rb, 1) M(1, cb).  B's row
   // block is in shared memory before C overwrites it (in place for frames).
@@ -214,7 +216,7 @@ k_solve_block(Dims dm, Work w) {
 
 // ------------------------------------------------------------------ scan --
 // grid (DB / RB row blocks, 2 directions, B * H).  Rows of the state evolve
-// independently (s_row <- alpha s_row M + c_row), so a CTA carries RB rows of
+// independently (s_row <- (alpha s_row + b_row) M), so a CTA carries RB rows of
 // one chain: thread (rq, cq) holds rows 8 rq .. 8 rq + 7 and columns 4 cq ..
 // 4 cq + 3 of its block, and the block's transpose sits in shared memory for
 // the products.  M_t streams through a double buffer in shared memory, KC
@@ -279,14 +281,41 @@ k_scan_big(Dims dm, Inputs in, Work w) {
     put_state(v);
   }
 
+  bool x_ready = false;  // St holds X = alpha S + B of the next written frame
   for (int st = 0; st < dm.T; ++st) {
     const int t = dir == 0 ? st : dm.T - 1 - st;
     const int slot = snap_slot_big(dm, dir, t);
     if (!is_anchor(dm, t)) {
       const long long fh = ((long long)b * dm.T + t) * dm.H + h;
       const float* Mg = w.M + fh * DD;
-      const float* Cg = w.Cm + fh * DD;
+      const float* Bg = w.Cm + fh * DD;  // B_t (the solve leaves it in the C_t slot)
       const float alpha = __ldg(in.alpha + fh);
+      // X = alpha S + B_t in place of this CTA's rows (the closed form
+      // S_t = (alpha S + B_t) M_t).  After a written frame the previous
+      // step already left X in St; here only before the first one.
+      if (!x_ready) {
+        float bv[8][4];  // this thread's 8 x 4 block of B_t, one 16-byte load per row
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(Bg + gidx(r, 0)));
+          bv[r][0] = v.x; bv[r][1] = v.y; bv[r][2] = v.z; bv[r][3] = v.w;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float4 x = *reinterpret_cast<const float4*>(St + (c0 + c) * RB + r0);
+          float4 y = *reinterpret_cast<const float4*>(St + (c0 + c) * RB + r0 + 4);
+          x.x = fmaf(alpha, x.x, bv[0][c]);
+          x.y = fmaf(alpha, x.y, bv[1][c]);
+          x.z = fmaf(alpha, x.z, bv[2][c]);
+          x.w = fmaf(alpha, x.w, bv[3][c]);
+          y.x = fmaf(alpha, y.x, bv[4][c]);
+          y.y = fmaf(alpha, y.y, bv[5][c]);
+          y.z = fmaf(alpha, y.z, bv[6][c]);
+          y.w = fmaf(alpha, y.w, bv[7][c]);
+          *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0) = x;
+          *reinterpret_cast<float4*>(St + (c0 + c) * RB + r0 + 4) = y;
+        }
+      }
       float acc[8][4];
 #pragma unroll
       for (int r = 0; r < 8; ++r)
@@ -326,16 +355,33 @@ k_scan_big(Dims dm, Inputs in, Work w) {
         }
         __syncthreads();  // chunk kc read by every thread before its buffer is refilled
       }
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const float4 cv = *reinterpret_cast<const float4*>(Cg + gidx(r, 0));
-        acc[r][0] = fmaf(alpha, acc[r][0], cv.x);
-        acc[r][1] = fmaf(alpha, acc[r][1], cv.y);
-        acc[r][2] = fmaf(alpha, acc[r][2], cv.z);
-        acc[r][3] = fmaf(alpha, acc[r][3], cv.w);
-      }
-      put_state(acc);  // every read of the old state finished at the last barrier
       if (slot >= 0) snapshot(slot, acc);
+      // the next written frame's X = alpha' S + B' straight from the new state
+      // in registers (anchors lie only before the first and after the last
+      // written frame, so nothing reads S from St in between); every read of
+      // this step's X finished at its last barrier
+      int tn = -1;
+      for (int sn = st + 1; sn < dm.T && tn < 0; ++sn) {
+        const int tt = dir == 0 ? sn : dm.T - 1 - sn;
+        if (!is_anchor(dm, tt)) tn = tt;
+      }
+      if (tn >= 0) {
+        const long long fn = ((long long)b * dm.T + tn) * dm.H + h;
+        const float* Bn = w.Cm + fn * DD;
+        const float an = __ldg(in.alpha + fn);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(Bn + gidx(r, 0)));
+          acc[r][0] = fmaf(an, acc[r][0], v.x);
+          acc[r][1] = fmaf(an, acc[r][1], v.y);
+          acc[r][2] = fmaf(an, acc[r][2], v.z);
+          acc[r][3] = fmaf(an, acc[r][3], v.w);
+        }
+        x_ready = true;
+      } else {
+        x_ready = false;
+      }
+      put_state(acc);  // X for the next written frame, or the final state
     } else if (slot >= 0) {
       float v[8][4];
 #pragma unroll

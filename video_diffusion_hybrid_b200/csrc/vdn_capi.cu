@@ -186,7 +186,7 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
   // the tensor-core scan (and its solve) take the B form: every call with this
   // configuration decides the same way, so stages run in separate calls agree
   const bool tc_scan = !big && scan_tc_supported(d) && w.M16 != nullptr;
-  w.bform = tc_scan ? 1 : 0;
+  w.bform = (tc_scan || big) ? 1 : 0;  // the d = 256 scan takes the B form too
   // d = 256: the VDA stages only (the softmax stage has no kernel at this size)
   if (big && ((stages & VDN_STAGE_SOFTMAX) || !gram_tc_supported(d))) return VDN_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
