@@ -140,7 +140,7 @@ k_solve_block(Dims dm, Work w) {
   float* T0 = smb;              // [128][PB] each
   float* T1 = T0 + TB * PB;
   float* T2 = T1 + TB * PB;
-  float* rowbuf = T2 + TB * PB;  // 2 (128 + 4) floats for the sweep
+  float* rowbuf = T2 + TB * PB;  // 4 (128 + 4) floats for the sweep
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (!TEXT && is_anchor(dm, t)) return;
   const long long DD = (long long)DB * DB;
@@ -518,7 +518,7 @@ bool big_d(const Dims& d) { return d.dk == DB && d.dv == DB; }
 
 cudaError_t launch_solve_big(const Dims& d, const Work& w, cudaStream_t s, bool text) {
   if (!big_d(d)) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(float) * (size_t)(3 * TB * PB + 2 * (TB + 4));
+  const size_t smem = sizeof(float) * (size_t)(3 * TB * PB + 4 * (TB + 4));
   auto kern = text ? k_solve_block<true> : k_solve_block<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -10,7 +10,7 @@
 // needs no pivoting: each pivot is a Schur complement of I + A_t and is >= 1.
 // Sweeping all d pivots turns G = I + A into -G^-1 in d^3 multiply-adds, the
 // same work as Cholesky + triangular inverse + W^T W, in one pass with one
-// barrier per pivot and every thread busy.
+// barrier per two pivots (sweep.cuh) and every thread busy.
 //
 // Thread (ty, tx) of a 16 x 16 grid keeps the R x R block G[ty R + a][tx R + c]
 // (R = d / 16) in registers.  The only exchange per pivot is row p (column p
@@ -54,11 +54,11 @@ __global__ void __launch_bounds__(kThreadsS, 2)
 k_solve_sweep(Dims dm, Work w) {
   constexpr int R = D / 16;   // register tile edge
   constexpr int P = D + 4;    // shared pitch (16-byte rows)
-  constexpr int BP = D + 4;   // pivot buffer: row p, then 1 / g_pp at [D]
+  constexpr int BP = D + 4;   // pivot buffers: rows p and p + 1, then Z at [D], [D + 1]
   static_assert(R % 2 == 0, "pivot buffers alternate with the parity of p");
   extern __shared__ float sm[];
-  float* rowbuf = sm;         // [2][BP]
-  float* Ms = sm + 2 * BP;    // [D][P]
+  float* rowbuf = sm;         // [4][BP]
+  float* Ms = sm + 4 * BP;    // [D][P]
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (!TEXT && is_anchor(dm, t)) return;
@@ -134,7 +134,7 @@ k_solve_sweep(Dims dm, Work w) {
 
 template <int D, bool TEXT>
 cudaError_t launch(const Dims& d, const Work& w, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (size_t)(2 * (D + 4) + D * (D + 4));
+  const size_t smem = sizeof(float) * (size_t)(4 * (D + 4) + D * (D + 4));
   auto kern = k_solve_sweep<D, TEXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
