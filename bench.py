@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--xattn", action="store_true",
                     help="time the text cross-attention (every video query over the L text tokens) at the "
                          "workload's shape instead of the core")
+    ap.add_argument("--fp8", action="store_true",
+                    help="with --proj: e4m3 operands (the activation quantised in the timed region)")
     ap.add_argument("--proj", action="store_true",
                     help="time the layer's output projection (one GEMM over the core's concat axis) at the "
                          "workload's shape instead of the core")
@@ -487,28 +489,52 @@ def run_proj(args):
     y = torch.randn((M, K), device="cuda", generator=gen).to(torch.bfloat16)
     wt = (torch.randn((K, N), device="cuda", generator=gen) / K ** 0.5).to(torch.bfloat16)
     out = torch.empty((M, N), device="cuda", dtype=torch.bfloat16)
+    if args.fp8:
+        # the weight once (transposed, [N, K]); the activation every step
+        qy = torch.empty((M, K), device="cuda", dtype=torch.uint8)
+        qw = torch.empty((N, K), device="cuda", dtype=torch.uint8)
+        scales = torch.zeros(2, device="cuda", dtype=torch.float32)
+        L.vdn_quantize_fp8(wt.t().contiguous(), L.VDN_BF16, N * K, qw, scales[1:2])
+
+        def step():
+            L.vdn_quantize_fp8(y, L.VDN_BF16, M * K, qy, scales[0:1])
+            L.vdn_out_proj_fp8(M, K, N, L.VDN_BF16, qy, qw, scales, out)
+    else:
+        def step():
+            L.vdn_out_proj(M, K, N, L.VDN_BF16, y, wt, out)
     for _ in range(max(args.warmup, 3)):
-        L.vdn_out_proj(M, K, N, L.VDN_BF16, y, wt, out)
+        step()
     torch.cuda.synchronize()
     clk = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0])
     clk.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
-        L.vdn_out_proj(M, K, N, L.VDN_BF16, y, wt, out)
+        step()
     e1.record()
     torch.cuda.synchronize()
     clocks = clk.stop()
     ms = e0.elapsed_time(e1) / args.steps
+    gemm_ms = None
+    if args.fp8:  # the GEMM alone, for its roofline
+        e0.record()
+        for _ in range(args.steps):
+            L.vdn_out_proj_fp8(M, K, N, L.VDN_BF16, qy, qw, scales, out)
+        e1.record()
+        torch.cuda.synchronize()
+        gemm_ms = e0.elapsed_time(e1) / args.steps
     peaks, src = load_peaks()
-    tflops = 2.0 * M * K * N / (ms * 1e-3) / 1e12
-    peak = peaks.get("bf16_tflops", 1590.0)
+    tflops = 2.0 * M * K * N / ((gemm_ms or ms) * 1e-3) / 1e12
+    # fp8 dense peak: the measured bf16 figure times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    peak = peaks.get("bf16_tflops", 1590.0) * (2.0 if args.fp8 else 1.0)
     print(json.dumps({
         "metric": "layer output projection (one GEMM over the concat axis)", "value": tflops, "unit": "TFLOP/s",
-        "ms_per_step": ms, "steps": args.steps, "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
-        "data": "synthetic", "config": {"workload": args.workload, "M": M, "K": K, "N": N, "library": "cuBLASLt"},
+        "ms_per_step": ms, "gemm_ms": gemm_ms, "steps": args.steps, "n_gpus": 1, "higher_is_better": True,
+        "dtype": "fp8_e4m3" if args.fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "library": "cuBLASLt",
+                   "step": "quantise y + FP8 GEMM" if args.fp8 else "bf16 GEMM"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
-                     "peak_source": f"bf16_tflops ({src})"},
+                     "peak_source": f"bf16_tflops ({src})" + (" x 2 (nominal fp8 / bf16)" if args.fp8 else "")},
         "clocks": clocks}), flush=True)
 
 

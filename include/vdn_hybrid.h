@@ -249,6 +249,28 @@ typedef struct {
  * (no GEMM algorithm for the sizes), VDN_ERR_CUDA. */
 vdn_status vdn_out_proj(const vdn_proj_cfg *cfg, const void *y, const void *w, void *out, vdn_stream_t stream);
 
+/* ------------------------------------------------------------ FP8 linear layers
+ * deepmagic post "生成比播放還快", section 實測數據: the per-block latency reaches
+ * its lowest figure once optimized kernels and FP8 linear layers are added.  Tensors go to
+ * FP8 E4M3 with one scale per tensor, s = amax|x| / 448 (the largest finite
+ * e4m3; 1 for an all-zero tensor), q = e4m3(x * (1 / s)) rounded to nearest
+ * even and saturated, so that x ~ q * s. */
+
+/* q[i] = e4m3(x[i] / s) for the n elements of x (x_dtype VDN_F32 or VDN_BF16),
+ * and s into *scale, all on `stream` (device pointers; x and q 16-byte aligned).
+ * Errors: VDN_ERR_INVALID_ARG (NULL or misaligned pointers, n = 0, a dtype),
+ * VDN_ERR_CUDA. */
+vdn_status vdn_quantize_fp8(const void *x, int x_dtype, size_t n, void *q, float *scale, vdn_stream_t stream);
+
+/* The output projection with e4m3 operands: out[M, N] = (s_y y)(s_w w) with y
+ * e4m3 [M, K] row-major, the weight given TRANSPOSED as w_t e4m3 [N, K]
+ * row-major (FP8 tensor-core GEMMs take both operands K-contiguous), scales =
+ * {s_y, s_w} (two floats in device memory, e.g. as written by
+ * vdn_quantize_fp8), out in cfg->out_dtype; fp32 accumulation, cuBLASLt, no
+ * workspace.  K and N multiples of 16.  Errors as vdn_out_proj. */
+vdn_status vdn_out_proj_fp8(const vdn_proj_cfg *cfg, const void *y, const void *w_t, const float *scales, void *out,
+                            vdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

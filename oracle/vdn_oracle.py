@@ -294,6 +294,29 @@ def out_proj(y, W):
     return y.reshape(y.shape[:-3] + (H * two * dv,)) @ np.asarray(W, F64)
 
 
+def quantize_e4m3(x):
+    """FP8 E4M3 with one scale per tensor (deepmagic post, section 實測數據:
+    FP8 linear layers): s = amax|x| / 448 in float32 (448 is the largest
+    finite e4m3; s = 1 for an all-zero tensor), q = e4m3(x * (1 / s)) with the
+    product in float32 and the rounding to nearest even of torch's
+    float8_e4m3fn conversion (a library routine).  Returns the codes as a
+    torch float8 tensor and s (float32), so that x ~ q * s."""
+    import torch
+    x32 = np.asarray(x, np.float32)
+    amax = np.float32(np.abs(x32).max()) if x32.size else np.float32(0.0)
+    s = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+    inv = np.float32(np.float32(1.0) / s)
+    return torch.from_numpy(np.ascontiguousarray(x32 * inv)).to(torch.float8_e4m3fn), s
+
+
+def out_proj_fp8(qy, sy, qw_t, sw):
+    """The output projection with e4m3 operands: (s_y q_y)(s_w q_w_t)^T in
+    float64, q_y [M, K], q_w_t [N, K] (the weight transposed)."""
+    y = qy.to(dtype=__import__("torch").float64).numpy() * float(sy)
+    w = qw_t.to(dtype=__import__("torch").float64).numpy() * float(sw)
+    return y @ w.T
+
+
 def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-np.asarray(x, F64)))
 

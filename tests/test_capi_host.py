@@ -171,3 +171,12 @@ def test_text_cross_attn_rejected_before_launch():
     assert call(_cfg(), workspace_bytes=128) == L.VDN_ERR_WORKSPACE
     assert call(_cfg(dtype=L.VDN_F32)) == L.VDN_ERR_UNSUPPORTED
     assert call(_cfg(d_k=32, d_v=32)) == L.VDN_ERR_UNSUPPORTED
+
+
+def test_fp8_entries_reject_bad_args():
+    p = 1 << 20
+    assert L.vdn_quantize_fp8(p, L.VDN_BF16, 0, p, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.vdn_quantize_fp8(p, 7, 16, p, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.vdn_quantize_fp8(None, L.VDN_F32, 16, p, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.vdn_out_proj_fp8(8, 24, 32, 0, p, p, p, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.vdn_out_proj_fp8(8, 32, 32, 0, p, p, None, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG

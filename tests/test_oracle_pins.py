@@ -455,3 +455,22 @@ def test_text_cross_attn_equals_torch_sdpa():
     ref = torch.nn.functional.scaled_dot_product_attention(
         torch.from_numpy(q.reshape(1, T * N, d)), torch.from_numpy(k[None]), torch.from_numpy(v[None]), scale=0.4)
     np.testing.assert_allclose(got, ref.numpy().reshape(T, N, d), rtol=0, atol=1e-12)
+
+
+def test_quantize_e4m3_round_trip():
+    """The per-tensor e4m3 quantisation: values on the scaled e4m3 grid come
+    back exactly, every other normal-range value within half an e4m3 step
+    (3 mantissa bits: 2^-4 relative), and nothing exceeds amax."""
+    s0 = np.float32(0.5)
+    grid = np.array([1.0, 1.125, 1.25, 2.0, 3.5, 448.0, 0.015625], np.float32) * s0
+    q, s = O.quantize_e4m3(grid)
+    assert s == np.float32(448.0) * s0 / np.float32(448.0)
+    np.testing.assert_array_equal(q.float().numpy() * s, grid)
+    r = np.random.default_rng(41)
+    x = r.standard_normal(5000).astype(np.float32)
+    q, s = O.quantize_e4m3(x)
+    back = q.float().numpy().astype(np.float64) * s
+    normal = np.abs(x) >= s * 2.0 ** -6
+    assert np.all(np.abs(back - x)[normal] <= 2.0 ** -4 * np.abs(x)[normal] * (1 + 1e-6))
+    assert np.abs(back).max() <= np.abs(x).max() * (1 + 2.0 ** -4)
+    assert O.quantize_e4m3(np.zeros(4))[1] == np.float32(1.0)

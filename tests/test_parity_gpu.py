@@ -454,3 +454,46 @@ def test_text_cross_attn_matches_oracle(shape, y_bf16):
             ref = O.text_cross_attn(inp["q"][b, :, :, h], inp["text_k"][b, :, h], inp["text_v"][b, :, h], scale)
             e = rel_err(got[b, :, :, h], ref, U_BF16 * np.abs(ref) if y_bf16 else None)
             assert e <= TOL["bf16"], (b, h, e)
+
+
+# ------------------------------------------------------------ FP8 projection
+@pytest.mark.parametrize("src", ["bf16", "f32"])
+def test_quantize_fp8_matches_oracle(src):
+    """e4m3 codes and the per-tensor scale, bit for bit against the oracle's
+    quantisation of the same values."""
+    r = np.random.default_rng(7)
+    x = (r.standard_normal((1000, 256)) * 3).astype(np.float32)
+    xt = torch.from_numpy(x).cuda()
+    if src == "bf16":
+        xt = xt.to(torch.bfloat16)
+        x = xt.float().cpu().numpy()
+    q = torch.empty(x.shape, dtype=torch.uint8, device="cuda")
+    sc = torch.zeros(1, dtype=torch.float32, device="cuda")
+    L.vdn_quantize_fp8(xt, L.VDN_BF16 if src == "bf16" else L.VDN_F32, x.size, q, sc)
+    torch.cuda.synchronize()
+    qo, so = O.quantize_e4m3(x)
+    assert sc.item() == so
+    np.testing.assert_array_equal(q.cpu().numpy(), qo.view(torch.uint8).numpy())
+
+
+@pytest.mark.parametrize("out_dtype", [L.VDN_F32, L.VDN_BF16])
+def test_out_proj_fp8_matches_oracle(out_dtype):
+    """The FP8 projection of quantised operands against the oracle's float64
+    product of the same dequantised values."""
+    r = np.random.default_rng(9)
+    M, K, N = 777, 512, 256
+    y = torch.from_numpy(r.standard_normal((M, K)).astype(np.float32)).cuda().to(torch.bfloat16)
+    w_t = torch.from_numpy((r.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32)).cuda().to(torch.bfloat16)
+    qy = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    qw = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros(2, dtype=torch.float32, device="cuda")
+    L.vdn_quantize_fp8(y, L.VDN_BF16, M * K, qy, scales[0:1])
+    L.vdn_quantize_fp8(w_t, L.VDN_BF16, N * K, qw, scales[1:2])
+    out = torch.empty((M, N), dtype=torch.float32 if out_dtype == L.VDN_F32 else torch.bfloat16, device="cuda")
+    L.vdn_out_proj_fp8(M, K, N, out_dtype, qy, qw, scales, out)
+    torch.cuda.synchronize()
+    sy, sw = scales.cpu().numpy()
+    ref = O.out_proj_fp8(qy.cpu().view(torch.float8_e4m3fn), sy, qw.cpu().view(torch.float8_e4m3fn), sw)
+    got = out.float().cpu().numpy().astype(np.float64)
+    tol = 1e-5 * np.abs(ref).max() + (2.0 ** -8 * np.abs(ref) if out_dtype == L.VDN_BF16 else 0.0)
+    assert np.all(np.abs(got - ref) <= tol)

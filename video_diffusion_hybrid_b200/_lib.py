@@ -22,7 +22,8 @@ STAGE_ALL = 31
 
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
-            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn")
+            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn",
+            "vdn_quantize_fp8", "vdn_out_proj_fp8")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -113,6 +114,11 @@ def lib() -> C.CDLL:
         L.vdn_hybrid_attn_fwd_noalloc.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
         L.vdn_text_cross_attn.restype = C.c_int
         L.vdn_text_cross_attn.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
+        L.vdn_quantize_fp8.restype = C.c_int
+        L.vdn_quantize_fp8.argtypes = [C.c_void_p, C.c_int, C.c_size_t, C.c_void_p, C.c_void_p, C.c_void_p]
+        L.vdn_out_proj_fp8.restype = C.c_int
+        L.vdn_out_proj_fp8.argtypes = [C.POINTER(ProjCfg), C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                                       C.c_void_p]
         L.vdn_out_proj.restype = C.c_int
         L.vdn_out_proj.argtypes = [C.POINTER(ProjCfg), C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
         L.vdn_status_string.restype = C.c_char_p
@@ -144,6 +150,24 @@ def vdn_out_proj(M: int, K: int, N: int, out_dtype: int, y, w, out, stream=None,
     st = lib().vdn_out_proj(C.byref(c), _ptr(y), _ptr(w), _ptr(out), _stream_handle(stream))
     if check and st != VDN_OK:
         raise VdnError(st, "vdn_out_proj")
+    return st
+
+
+def vdn_quantize_fp8(x, x_dtype: int, n: int, q, scale, stream=None, check: bool = True) -> int:
+    """q = e4m3(x / s), s = amax|x| / 448 into scale (device pointers or tensors)."""
+    st = lib().vdn_quantize_fp8(_ptr(x), x_dtype, n, _ptr(q), _ptr(scale), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_quantize_fp8")
+    return st
+
+
+def vdn_out_proj_fp8(M: int, K: int, N: int, out_dtype: int, y, w_t, scales, out, stream=None,
+                     check: bool = True) -> int:
+    """out[M, N] = (s_y y)(s_w w) with e4m3 y [M, K], w_t [N, K] and scales {s_y, s_w}."""
+    c = ProjCfg(M=M, K=K, N=N, out_dtype=out_dtype)
+    st = lib().vdn_out_proj_fp8(C.byref(c), _ptr(y), _ptr(w_t), _ptr(scales), _ptr(out), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_out_proj_fp8")
     return st
 
 

@@ -294,6 +294,22 @@ vdn_status vdn_out_proj(const vdn_proj_cfg* cfg, const void* y, const void* w, v
   return out_proj(cfg->M, cfg->K, cfg->N, cfg->out_dtype, y, w, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+vdn_status vdn_quantize_fp8(const void* x, int x_dtype, size_t n, void* q, float* scale, vdn_stream_t stream) {
+  if (!x || !q || !scale || n == 0 || n > (size_t)1 << 62) return VDN_ERR_INVALID_ARG;
+  if (x_dtype != VDN_F32 && x_dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(scale, 4)) return VDN_ERR_INVALID_ARG;
+  return quantize_fp8(x, x_dtype, (long long)n, q, scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+vdn_status vdn_out_proj_fp8(const vdn_proj_cfg* cfg, const void* y, const void* w_t, const float* scales, void* out,
+                            vdn_stream_t stream) {
+  if (!cfg || !y || !w_t || !scales || !out) return VDN_ERR_INVALID_ARG;
+  if (cfg->M < 1 || cfg->K < 16 || cfg->N < 16 || cfg->K % 16 || cfg->N % 16) return VDN_ERR_INVALID_ARG;
+  if (cfg->out_dtype != VDN_F32 && cfg->out_dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
+  if (!aligned(y, 16) || !aligned(w_t, 16) || !aligned(out, 16) || !aligned(scales, 8)) return VDN_ERR_INVALID_ARG;
+  return out_proj(cfg->M, cfg->K, cfg->N, cfg->out_dtype, y, w_t, out, reinterpret_cast<cudaStream_t>(stream), scales);
+}
+
 const char* vdn_status_string(vdn_status s) {
   switch (s) {
     case VDN_OK: return "ok";

@@ -84,7 +84,10 @@ cudaError_t launch_read_big(const Dims& d, const Inputs& in, const Work& w, cuda
 cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s, bool chunks);
 cudaError_t launch_compose_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 // out[M, N] = y[M, K] w[K, N] (bf16 operands, fp32 accumulation), cuBLASLt
-vdn_status out_proj(int M, int K, int N, int out_dtype, const void* y, const void* w, void* out, cudaStream_t s);
+// scales != nullptr: e4m3 y [M, K] and w [N, K], dequantisation scales {s_y, s_w} in device memory
+vdn_status out_proj(int M, int K, int N, int out_dtype, const void* y, const void* w, void* out, cudaStream_t s,
+                    const float* scales = nullptr);
+vdn_status quantize_fp8(const void* x, int dtype, long long n, void* q, float* scale, cudaStream_t s);
 // The chunk-composed scan where it helps: the compositions (one CTA per
 // chunk, batch-head and direction) take about one wave of the SMs, and then
 // the sequential chain is 5x shorter; with more chains than that the frame
