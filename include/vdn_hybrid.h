@@ -110,6 +110,15 @@ typedef struct {
                                       kernel (same results either way)                    */
   void *workspace;                 /* device scratch, 256-byte aligned                   */
   size_t workspace_bytes;
+  const float *fwd_init;           /* [B,H,d_v,d_k] streaming: the forward scan's start
+                                      state (the forward state the previous segment ended
+                                      with, slot C of its fwd_snap), carried across
+                                      appended chunks of a live stream (Video DeltaNet,
+                                      the livestream setting of the abstract).  NULL =
+                                      half the text state, as the backward scan always
+                                      starts.  Anchor query frames then read
+                                      fwd_init + S_x / 2.  16-byte aligned, outside the
+                                      workspace.                                           */
 } vdn_hybrid_args;
 
 /* Pipeline stages; vdn_hybrid_attn_fwd runs VDN_STAGE_ALL in this order. */

@@ -382,7 +382,10 @@ def softmax_dense_masked(q_bh, k_bh, v_bh, T, N, chunk, anchors, scale):
 # ---------------------------------------------------------------------------
 def head_states(inp: dict, cfg: Cfg, b: int, h: int):
     """F, G (forward / backward states for every frame boundary) of one
-    (batch, head), both started from half the text state."""
+    (batch, head), both started from half the text state; with
+    inp["fwd_init"] [B, H, d_v, d_k] the forward scan starts from that state
+    instead (streaming: the state the previous segment's forward scan ended
+    with, carried across appended chunks, [P2] livestream setting)."""
     if cfg.L > 0 and inp.get("text_k") is not None:
         Sx = text_state(inp["text_k"][b, :, h], inp["text_v"][b, :, h], inp["text_beta"][b, :, h],
                         cfg.d_v, cfg.d_k)
@@ -395,7 +398,8 @@ def head_states(inp: dict, cfg: Cfg, b: int, h: int):
     v = inp["v"][b, :, :, h]
     beta = inp["beta"][b, :, :, h]
     alpha = inp["alpha"][b, :, h]
-    F = forward_states(S0, k, v, beta, alpha, cfg.anchors)
+    F0 = np.asarray(inp["fwd_init"][b, h], F64) if inp.get("fwd_init") is not None else S0
+    F = forward_states(F0, k, v, beta, alpha, cfg.anchors)
     G = backward_states(S0, k, v, beta, alpha, cfg.anchors)
     return F, G
 
@@ -463,5 +467,7 @@ def vda_intermediates(inp: dict, cfg: Cfg, b: int, h: int):
             continue
         Ms[t], Cs[t] = frame_map(inp["k"][b, t, :, h], inp["v"][b, t, :, h], inp["beta"][b, t, :, h])
     F, G = head_states(inp, cfg, b, h)
-    return {"M": Ms, "C": Cs, "S_init": F[0], "F": F, "G": G,
+    # the backward scan always starts from half the text state (the forward
+    # one from fwd_init when that is given)
+    return {"M": Ms, "C": Cs, "S_init": G[T], "F": F, "G": G,
             "R": read_table(F, G, T, cfg.chunk, cfg.anchors)}

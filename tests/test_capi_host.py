@@ -93,6 +93,8 @@ def _fake_args(cfg, **over):
     (dict(k=(1 << 20) + 2), L.VDN_ERR_INVALID_ARG), (dict(text_k=None), L.VDN_ERR_INVALID_ARG),
     (dict(init_state=1 << 20), L.VDN_ERR_INVALID_ARG), (dict(workspace=None), L.VDN_ERR_WORKSPACE),
     (dict(workspace=(1 << 20) + 16), L.VDN_ERR_WORKSPACE), (dict(workspace_bytes=1024), L.VDN_ERR_WORKSPACE),
+    # the carried forward state: 16-byte aligned and outside the workspace
+    (dict(fwd_init=(1 << 24) + 4), L.VDN_ERR_INVALID_ARG), (dict(fwd_init=(1 << 20) + 4096), L.VDN_ERR_INVALID_ARG),
 ])
 def test_bad_args_rejected_before_launch(over, status):
     cfg = _cfg()

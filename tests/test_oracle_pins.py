@@ -474,3 +474,71 @@ def test_quantize_e4m3_round_trip():
     assert np.all(np.abs(back - x)[normal] <= 2.0 ** -4 * np.abs(x)[normal] * (1 + 1e-6))
     assert np.abs(back).max() <= np.abs(x).max() * (1 + 2.0 ** -4)
     assert O.quantize_e4m3(np.zeros(4))[1] == np.float32(1.0)
+
+
+# ----------------------------------------------------------- streaming ----
+def _tag_segment(frames, d, T):
+    """One head, one token per frame: frame f (global index) carries the key
+    and value e_f, beta = 1, alpha = 1, so a state's diagonal lists the
+    frames written into it (each at beta / (1 + beta) = 1/2)."""
+    k = np.zeros((1, T, 1, 1, d))
+    for i, f in enumerate(frames):
+        k[0, i, 0, 0, f] = 1.0
+    return {"k": k, "v": k.copy(), "beta": np.ones((1, T, 1, 1)), "alpha": np.ones((1, T, 1))}
+
+
+@pytest.mark.parametrize("T1,T2,anchors", [(12, 13, 4), (10, 7, 4), (9, 11, 0)])
+def test_stream_carried_state_holds_the_past(T1, T2, anchors):
+    """Streaming ([P2] livestream setting): the second segment's forward
+    scan starts from the state the first segment's forward scan ended with.
+    With one tagged frame per key, every query of the second segment then
+    reads each written frame of the first segment once, plus its own
+    segment's written frames outside its window, and never a frame in its
+    window or an anchor; an anchor query reads the carried past alone."""
+    d = T1 + T2
+    seg1 = _tag_segment(range(T1), d, T1)
+    c1 = O.Cfg(B=1, T=T1, N=1, H=1, d_k=d, d_v=d, L=0, anchors=anchors)
+    F1, _ = O.head_states(seg1, c1, 0, 0)
+    seg2 = _tag_segment(range(T1, d), d, T2)
+    seg2["fwd_init"] = F1[T1][None, None]
+    c2 = O.Cfg(B=1, T=T2, N=1, H=1, d_k=d, d_v=d, L=0, anchors=anchors)
+    F2, G2 = O.head_states(seg2, c2, 0, 0)
+    past = {f for f in range(T1) if f not in O.anchor_frames(T1, anchors)}
+    anc2 = set(O.anchor_frames(T2, anchors))
+    for t in range(T2):
+        held_d = np.diag(O.read_state(F2, G2, t, T2, 5, anchors))
+        np.testing.assert_allclose(held_d[held_d > 1e-9], 0.5, atol=1e-12)
+        held = set(np.nonzero(held_d > 1e-9)[0])
+        if t in anc2:
+            assert held == past
+            continue
+        lo, hi = O.window_frames(t, T2, 5)
+        own = {T1 + f for f in range(T2) if f not in anc2 and not lo <= f < hi}
+        assert held == past | own
+
+
+def test_stream_forward_continues_one_long_scan():
+    """Cutting a sequence in two and carrying the forward state gives the
+    forward states of the uncut sequence (no anchors, so the cut writes
+    every frame either way)."""
+    shp = Shape(B=1, T=14, N=6, H=1, d_k=8, d_v=8, L=0)
+    inp = make_inputs(shp, seed=3)
+    long_cfg = O.Cfg(B=1, T=14, N=6, H=1, d_k=8, d_v=8, L=0, anchors=0)
+    F, _ = O.head_states(inp, long_cfg, 0, 0)
+    T1 = 6
+    seg = {n: inp[n][:, T1:] for n in ("q", "k", "v", "beta", "alpha", "gate_sm", "gate_lin")}
+    seg["fwd_init"] = F[T1][None, None]
+    F2, _ = O.head_states(seg, O.Cfg(B=1, T=14 - T1, N=6, H=1, d_k=8, d_v=8, L=0, anchors=0), 0, 0)
+    np.testing.assert_allclose(F2, F[T1:], rtol=0, atol=1e-13)
+
+
+def test_stream_default_start_is_half_the_text_state():
+    """fwd_init = S_x / 2 reproduces the call without it, bit for bit."""
+    shp = Shape(B=1, T=12, N=8, H=2, d_k=16, d_v=16, L=6)
+    inp = make_inputs(shp, seed=4)
+    cfg = O.Cfg(B=1, T=12, N=8, H=2, d_k=16, d_v=16, L=6)
+    half = np.stack([0.5 * O.text_state(inp["text_k"][0, :, h], inp["text_v"][0, :, h], inp["text_beta"][0, :, h],
+                                        16, 16) for h in range(2)])[None]
+    want = O.hybrid_attn(inp, cfg)
+    got = O.hybrid_attn({**inp, "fwd_init": half}, cfg)
+    np.testing.assert_array_equal(got, want)

@@ -497,3 +497,62 @@ def test_out_proj_fp8_matches_oracle(out_dtype):
     got = out.float().cpu().numpy().astype(np.float64)
     tol = 1e-5 * np.abs(ref).max() + (2.0 ** -8 * np.abs(ref) if out_dtype == L.VDN_BF16 else 0.0)
     assert np.all(np.abs(got - ref) <= tol)
+
+
+STREAM_CASES = {
+    "d64_simt_f32": (Shape(1, 20, 24, 2, 64, 64, 6), "f32", {}),
+    "d64_bf16": (Shape(1, 20, 24, 2, 64, 64, 6), "bf16", {}),
+    "d128_frames": (Shape(1, 22, 40, 2, 128, 128, 4), "bf16", dict(scan_mode=1)),
+    "d128_chunks": (Shape(1, 22, 40, 2, 128, 128, 4), "bf16", dict(scan_mode=2)),
+    "d128_f32": (Shape(1, 12, 30, 1, 128, 128, 4), "f32", {}),
+}
+
+
+@pytest.mark.parametrize("case", sorted(STREAM_CASES))
+def test_stream_fwd_init_matches_oracle(case):
+    """Streaming: a given forward start state (the state carried from the
+    previous segment) on every scan kernel (SIMT, tensor-core frame steps,
+    composed chunk steps), against the oracle with the same start."""
+    shape, dtype, kw = STREAM_CASES[case]
+    r = np.random.default_rng(17)
+    extra = {"fwd_init": (0.3 * r.standard_normal((shape.B, shape.H, shape.d_v, shape.d_k))).astype(np.float32)}
+    inp, cfg, ha, _, y = run(shape, dtype, 23, extra=extra, **kw)
+    check(y, oracle(inp, cfg), cfg, dtype)
+    it = ha.intermediates()["fwd_snap"].double().cpu().numpy()
+    np.testing.assert_array_equal(it[:, :, 0], extra["fwd_init"].astype(np.float64))
+
+
+def test_stream_d256_fwd_init_matches_oracle():
+    shape = Shape(1, 12, 40, 1, 256, 256, 8)
+    r = np.random.default_rng(18)
+    extra = {"fwd_init": (0.3 * r.standard_normal((1, 1, 256, 256))).astype(np.float32)}
+    inp, cfg, ha, t, y = run(shape, "bf16", 29, extra=extra, stages=VDA)
+    ref_y = O.hybrid_attn(inp, ocfg(cfg))
+    assert rel_err(y[..., 1, :], ref_y[..., 1, :]) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_stream_two_segments_match_oracle(dtype, d):
+    """Two appended segments: the second call starts its forward scan from
+    the first call's forward end state (read back from the workspace); the
+    oracle chains its own end state the same way."""
+    s1, s2 = Shape(1, 17, 32, 2, d, d, 6), Shape(1, 13, 32, 2, d, d, 0)
+    inp1, cfg1, ha1, _, y1 = run(s1, dtype, 31)
+    oc1 = ocfg(cfg1)
+    ends = [O.head_states(inp1, oc1, 0, h)[0][cfg1.T] for h in range(cfg1.H)]
+    carried = np.stack(ends)[None]
+    got_end = ha1.forward_end_state().double().cpu().numpy()
+    assert rel_err(got_end, carried) <= TOL[dtype]
+    # the second segment's text state is zero: it reads only the carried past
+    # and its own frames
+    inp2 = make_inputs(s2, 32, dtype)
+    for k in ("text_k", "text_v", "text_beta", "text_k_bits", "text_v_bits"):
+        inp2.pop(k, None)
+    cfg2 = cfg_for(s2, dtype)
+    t2 = to_torch(inp2, dtype, "cuda")
+    t2["fwd_init"] = ha1.forward_end_state()
+    ha2 = HybridAttention(cfg2)
+    y2 = ha2(t2).float().cpu().numpy().astype(np.float64)
+    torch.cuda.synchronize()
+    ref2 = O.hybrid_attn({**inp2, "fwd_init": carried}, O.Cfg(**{**ocfg(cfg2).__dict__, "out_mode": 0}))
+    check(y2, ref2, cfg2, dtype)

@@ -39,7 +39,7 @@ class VdnArgs(C.Structure):
                 ("alpha", C.c_void_p), ("gate_sm", C.c_void_p), ("gate_lin", C.c_void_p),
                 ("text_k", C.c_void_p), ("text_v", C.c_void_p), ("text_beta", C.c_void_p),
                 ("init_state", C.c_void_p), ("rms_weight", C.c_void_p), ("y", C.c_void_p),
-                ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t)]
+                ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t), ("fwd_init", C.c_void_p)]
 
 
 class ProjCfg(C.Structure):
@@ -194,14 +194,15 @@ def _ptr(t) -> int | None:
 
 
 def make_args(q, k, v, beta, alpha, gate_sm, gate_lin, y, workspace, workspace_bytes=None,
-              text_k=None, text_v=None, text_beta=None, init_state=None, rms_weight=None) -> VdnArgs:
+              text_k=None, text_v=None, text_beta=None, init_state=None, rms_weight=None,
+              fwd_init=None) -> VdnArgs:
     """Build a ``vdn_hybrid_args`` from torch tensors (or raw integer device
     pointers).  The caller keeps the tensors alive for the call."""
     if workspace_bytes is None:
         workspace_bytes = workspace.numel() * workspace.element_size()
     return VdnArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate_sm), _ptr(gate_lin),
                    _ptr(text_k), _ptr(text_v), _ptr(text_beta), _ptr(init_state), _ptr(rms_weight),
-                   _ptr(y), _ptr(workspace), int(workspace_bytes))
+                   _ptr(y), _ptr(workspace), int(workspace_bytes), _ptr(fwd_init))
 
 
 def _stream_handle(stream) -> int | None:

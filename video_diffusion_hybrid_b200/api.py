@@ -13,7 +13,7 @@ from . import _lib as L
 from .synth import Shape
 
 TENSOR_NAMES = ("q", "k", "v", "beta", "alpha", "gate_sm", "gate_lin", "text_k", "text_v", "text_beta",
-                "init_state", "rms_weight")
+                "init_state", "rms_weight", "fwd_init")
 
 
 def cfg_for(shape: Shape, dtype: str, **kw) -> L.HybridCfg:
@@ -62,7 +62,7 @@ class HybridAttention:
         return L.make_args(t["q"], t["k"], t["v"], t["beta"], t["alpha"], t["gate_sm"], t["gate_lin"], self.y,
                            self.workspace, self.ws_bytes, text_k=t.get("text_k"), text_v=t.get("text_v"),
                            text_beta=t.get("text_beta"), init_state=t.get("init_state"),
-                           rms_weight=t.get("rms_weight"))
+                           rms_weight=t.get("rms_weight"), fwd_init=t.get("fwd_init"))
 
     def __call__(self, t: dict, stages: int = L.STAGE_ALL, stream=None) -> torch.Tensor:
         a = self.args(t)
@@ -86,6 +86,11 @@ class HybridAttention:
             "bwd_snap": f(lay["bwd_snap"], (c.B, c.H, C + 1, c.d_v, c.d_k)),
             "R": f(lay["read_table"], (c.B, c.H, C + 1, c.d_v, c.d_k)),
         }
+
+    def forward_end_state(self) -> torch.Tensor:
+        """A copy of the forward state after the last frame (fwd_snap slot C),
+        [B, H, d_v, d_k] float32: the next appended segment's ``fwd_init``."""
+        return self.intermediates()["fwd_snap"][:, :, self.cfg.C].clone()
 
     def chunk_maps(self) -> dict:
         """The chunk maps of the chunk-stepped tensor-core scan (bf16 mode,

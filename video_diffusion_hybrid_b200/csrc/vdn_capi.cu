@@ -95,6 +95,13 @@ vdn_status check_args(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a, unsigne
   vdn_workspace_layout L;
   layout_of(c, &L);
   if (!a->workspace || !aligned(a->workspace, kAlign) || a->workspace_bytes < L.total) return VDN_ERR_WORKSPACE;
+  if (a->fwd_init) {
+    // the scans overwrite the snapshot slots while they read the start state
+    const char* f = static_cast<const char*>(static_cast<const void*>(a->fwd_init));
+    const char* ws = static_cast<const char*>(a->workspace);
+    const size_t fb = sizeof(float) * (size_t)c->B * c->H * c->d_v * c->d_k;
+    if (!aligned(a->fwd_init, 16) || (f < ws + a->workspace_bytes && ws < f + fb)) return VDN_ERR_INVALID_ARG;
+  }
   return VDN_OK;
 }
 
@@ -128,6 +135,7 @@ Inputs inputs_of(const vdn_hybrid_args* a) {
   in.gate_sm = a->gate_sm; in.gate_lin = a->gate_lin;
   in.text_k = a->text_k; in.text_v = a->text_v; in.text_beta = a->text_beta;
   in.init_state = a->init_state; in.rms_weight = a->rms_weight; in.y = a->y;
+  in.fwd_init = a->fwd_init;
   return in;
 }
 

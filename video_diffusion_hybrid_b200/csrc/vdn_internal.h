@@ -50,6 +50,7 @@ struct Inputs {
   const void *text_k, *text_v;
   const float *text_beta, *init_state, *rms_weight;
   void* y;
+  const float* fwd_init;  // forward start state, or null (half the text state)
 };
 
 __host__ __device__ inline bool is_anchor(const Dims& d, int t) {

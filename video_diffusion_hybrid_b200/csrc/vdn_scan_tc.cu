@@ -341,7 +341,8 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
     {
       // start state: its own slot, then (frame steps) the slots of leading
       // unwritten frames
-      const float* src = w.half_text + (long long)bh * DD + (long long)row * D;
+      const float* start = (dir == 0 && in.fwd_init) ? in.fwd_init : w.half_text;
+      const float* src = start + (long long)bh * DD + (long long)row * D;
       const int start_slot = dir == 0 ? 0 : dm.C;
       float s[32];
 #pragma unroll

@@ -250,7 +250,8 @@ k_scan(Dims dm, Inputs in, Work w) {
   const int row0 = blockIdx.x * RB, dir = blockIdx.y, bh = blockIdx.z;
   const int b = bh / dm.H, h = bh % dm.H;
   const long long DD = (long long)D * D;
-  const float* half = w.half_text + (long long)bh * DD;
+  // start state: half the text state, or the carried forward state
+  const float* half = ((dir == 0 && in.fwd_init) ? in.fwd_init : w.half_text) + (long long)bh * DD;
   float* snap = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD;
   auto frame = [&](int st) { return dir == 0 ? st : dm.T - 1 - st; };
   auto gidx = [&](int r, int c) { return (long long)(row0 + r0 + r) * D + c0 + c; };
