@@ -50,6 +50,9 @@ def parse():
                          "workload's shape instead of the core")
     ap.add_argument("--fp8", action="store_true",
                     help="with --proj: e4m3 operands (the activation quantised in the timed region)")
+    ap.add_argument("--update", type=int, choices=(0, 1, 2), default=0,
+                    help="the linear branch's frame write: 0 the joint solve; ablation baselines 1 frame-level "
+                         "independent writes (1/N rescaled), 2 the token-wise delta rule")
     ap.add_argument("--proj", action="store_true",
                     help="time the layer's output projection (one GEMM over the core's concat axis) at the "
                          "workload's shape instead of the core")
@@ -264,9 +267,25 @@ def stage_rooflines(s, cfg, ms, y_elem, peaks, sm_mhz):
         a = by / (ms[name] / 1e3) / 1e9
         out[name] = {"ms": ms[name], "bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
                      "work": by}
+    gb = R.gram_bytes(s.B, s.T, s.N, s.H, s.d_k, cfg.anchors, elem)
+    if cfg.update == 1 and L.vdn_hybrid_stage_impl(cfg, L.STAGE_TEXT) == 1 and s.d_k <= 128:
+        # frame-level writes from the tensor-core Gram, then the in-place
+        # rescale (reads and writes the M and C slots once)
+        by = gb + 4 * R.written_frames(s.T, cfg.anchors) * s.B * s.H * s.d_k * s.d_k * 4
+        a = by / (ms["solve"] / 1e3) / 1e9
+        out["solve"] = {"ms": ms["solve"], "kernel": "gram_tc+rescale", "bound": "hbm", "achieved": a, "peak": hbm,
+                        "unit": "GB/s", "frac": a / hbm, "work": by}
+        return out
+    if cfg.update != 0:
+        # the ablation writes' map kernel: fp32 FMA per token on the 2d x d
+        # stacked map (the update; the token rule adds the dot product)
+        f = R.variant_map_flops(s.B, s.T, s.N, s.H, s.d_k, cfg.anchors, cfg.update)
+        a = f / (ms["solve"] / 1e3) / 1e12
+        out["solve"] = {"ms": ms["solve"], "kernel": "variant_map", "bound": "alu", "achieved": a, "peak": simt,
+                        "unit": "TFLOP/s", "frac": a / simt, "work": f, "hbm_floor_ms": 1e3 * gb / (hbm * 1e9)}
+        return out
     # per-frame Gram (HBM-bound) followed by the SPD sweep (fp32 SIMT-bound):
     # the floor is the sum of the two
-    gb = R.gram_bytes(s.B, s.T, s.N, s.H, s.d_k, cfg.anchors, elem)
     # the tensor-core scan takes B_t itself, so its solve forms no C = B M
     sf = R.sweep_flops(s.B, s.T, s.H, s.d_k, cfg.anchors, with_c=L.vdn_hybrid_stage_impl(cfg, L.STAGE_SCAN) != 1)
     floor_ms = 1e3 * (gb / (hbm * 1e9) + sf / (simt * 1e12))
@@ -299,13 +318,13 @@ def run_ours(args):
     w = WORKLOADS[args.workload]
     s = w.shape
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.vda_only:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.vda_only and args.update == 0:
         val, work, desc = oracle_sample(w, oracle_prepare(w), target_s=12.0)
         cpu = {"value": val, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc,
                "sample_cpu_seconds": round(work, 2)}
 
     t = make_inputs_torch(s, w.seed + 17 * rank, w.dtype, dev)
-    cfg = cfg_for(s, w.dtype)
+    cfg = cfg_for(s, w.dtype, update=args.update)
     ha = HybridAttention(cfg, dev)
     stream = torch.cuda.current_stream(dev)
     pre = L.STAGE_TEXT | L.STAGE_SOLVE | L.STAGE_SCAN
@@ -315,7 +334,9 @@ def run_ours(args):
     # read table + read (else one SIMT read)
     tc = lambda st: L.vdn_hybrid_stage_impl(cfg, st) == 1
     text_k = (2 if tc(L.STAGE_TEXT) else 1) if s.L > 0 else 0  # no text: a memset, no kernel
-    launches_per_step = (text_k + (2 if tc(L.STAGE_SOLVE) else 1) + 1 + (0 if vda_only else 1)
+    # the frame-level ablation write on bf16 inputs: tensor-core Gram + rescale
+    variant_gram = args.update == 1 and tc(L.STAGE_TEXT) and s.d_k <= 128
+    launches_per_step = (text_k + (2 if tc(L.STAGE_SOLVE) or variant_gram else 1) + 1 + (0 if vda_only else 1)
                          + (2 if tc(L.STAGE_READ) else 1))
     K, W = args.steps, args.warmup
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -459,6 +480,7 @@ def run_ours(args):
             "config": {"workload": w.name, "B": s.B, "T": s.T, "N": s.N, "H": s.H, "d": s.d_k, "L": s.L,
                        "chunk": 5, "anchors": 4, "state": "fp32", "accumulate": "fp32",
                        "stages": "vda" if vda_only else "all",
+                       "frame_write": ("joint solve", "frame-level independent (1/N)", "token-wise delta rule")[args.update],
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": f"inputs exceed L2 ({in_gb:.1f} GB of q/k/v/gates per step)"},
             "roofline": roof,

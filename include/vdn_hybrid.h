@@ -91,6 +91,17 @@ typedef struct {
                           compositions fit one wave of the GPU's SMs (few chains, long
                           sequences), frames otherwise.  Other configurations step by
                           frames whatever the mode.                                    */
+  int update;          /* the per-frame write of the linear branch: 0 = the joint
+                          solve S_t = (alpha S + B_t)(I + A_t)^-1 (Video DeltaNet);
+                          ablation baselines the pages compare it with (deepmagic
+                          post, its Video Delta Attention paragraph; aimodeling
+                          news, "The VDN split"): 1 = frame-level independent writes
+                          against the frozen inherited state, rescaled by the frame
+                          size (SANA-WM): S_t = S_bar (I - A_t/N) + B_t/N; 2 = the
+                          token-wise delta rule, tokens written one after another
+                          in token order.  The text state is the joint solve's in
+                          every mode.  Modes 1 and 2 run the SIMT scan and need
+                          d_k <= 128 (VDN_ERR_UNSUPPORTED otherwise)                 */
 } vdn_hybrid_cfg;
 
 typedef struct {
@@ -213,7 +224,8 @@ vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg *cfg, const vdn_hybrid_
                                     vdn_stream_t stream, unsigned *where);
 
 /* Which implementation a stage uses for cfg: 0 = SIMT fp32, 1 = tcgen05 tensor
- * cores (TMA + TMEM), -1 = stage not supported for cfg. */
+ * cores (TMA + TMEM), 2 = the ablation variants' per-frame map kernel (SOLVE
+ * with cfg.update != 0), -1 = stage not supported for cfg. */
 int vdn_hybrid_stage_impl(const vdn_hybrid_cfg *cfg, unsigned stage);
 
 /* Static description of a status code. */

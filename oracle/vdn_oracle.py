@@ -75,6 +75,7 @@ class Cfg:
     softmax_scale: float = 0.0  # <= 0 -> 1/sqrt(d_k)
     rms_eps: float = 1e-6
     out_mode: int = 0         # 0 = [.., 2, d_v] slots, 1 = summed [.., d_v]
+    update: int = 0           # frame write: 0 joint solve, 1 frame-level independent, 2 token-wise
 
     @property
     def scale(self) -> float:
@@ -159,6 +160,51 @@ def frame_map(K: np.ndarray, V: np.ndarray, beta: np.ndarray):
     return M, Bw @ M
 
 
+# ---------------------------------------------------------------------------
+# ablation baselines of the frame write  ([P4] VDA paragraph: earlier
+# frame-level updates such as SANA-WM let every token update a frozen state on
+# its own; [P5] The VDN split: unlike SANA-WM, no frame-size rescaling is
+# needed; [P1] 四: the classic token-by-token delta rule is the one-token case)
+# ---------------------------------------------------------------------------
+def frame_independent_update(S_bar: np.ndarray, K: np.ndarray, V: np.ndarray, beta: np.ndarray) -> np.ndarray:
+    """Frame-level independent writes (the SANA-WM style baseline): each token
+    i proposes the delta-rule step beta_i (v_i - S_bar k_i) k_i^T against the
+    same frozen inherited state, and the N proposals are summed and divided
+    by the frame size N (the rescaling that keeps the map non-expansive)."""
+    S_bar = np.asarray(S_bar, F64)
+    K, V, beta = np.asarray(K, F64), np.asarray(V, F64), np.asarray(beta, F64)
+    resid = V - K @ S_bar.T                     # row i: v_i - S_bar k_i
+    return S_bar + (beta[:, None] * resid).T @ K / K.shape[0]
+
+
+def token_delta_update(S_bar: np.ndarray, K: np.ndarray, V: np.ndarray, beta: np.ndarray) -> np.ndarray:
+    """The token-wise delta rule: tokens write one after another in token
+    order, S <- S + beta_i (v_i - S k_i) k_i^T, each against the state the
+    previous token left."""
+    S = np.array(S_bar, F64)
+    for i in range(K.shape[0]):
+        k = np.asarray(K[i], F64)
+        S = S + beta[i] * np.outer(np.asarray(V[i], F64) - S @ k, k)
+    return S
+
+
+def frame_update(update: int):
+    """The frame write of mode `update` (0 joint solve, 1 frame-level
+    independent, 2 token-wise delta rule)."""
+    return {0: vda_update, 1: frame_independent_update, 2: token_delta_update}[update]
+
+
+def variant_frame_map(K: np.ndarray, V: np.ndarray, beta: np.ndarray, update: int):
+    """Every mode's write is affine in the inherited state, S = S_bar M + C:
+    M is the write of the identity with zero values, C the write of the zero
+    state.  Returned for intermediate-value checks of the per-frame maps."""
+    f = frame_update(update)
+    dk, dv = K.shape[1], V.shape[1]
+    M = f(np.eye(dk), K, np.zeros((K.shape[0], dk)), beta)
+    C = f(np.zeros((dv, dk)), K, V, beta)
+    return M, C
+
+
 def text_state(text_k: np.ndarray, text_v: np.ndarray, text_beta: np.ndarray, d_v: int, d_k: int) -> np.ndarray:
     """Text is pre-written by one joint solve from the zero state over the L
     text tokens ([P1] 三: the prompt is written into both states, half each).
@@ -168,11 +214,12 @@ def text_state(text_k: np.ndarray, text_v: np.ndarray, text_beta: np.ndarray, d_
     return vda_update(np.zeros((d_v, d_k)), text_k, text_v, text_beta)
 
 
-def forward_states(S0, k, v, beta, alpha, anchors: int = 4) -> np.ndarray:
+def forward_states(S0, k, v, beta, alpha, anchors: int = 4, update=vda_update) -> np.ndarray:
     """Forward scan for one (batch, head).  k [T, N, d_k], v [T, N, d_v],
     beta [T, N], alpha [T].  F[t] is the state that covers frames < t
     (F[0] = S0); at a non-anchor frame the inherited state is alpha_t F[t]
-    and the frame is written jointly; anchor frames are not written."""
+    and the frame is written jointly (or by the ablation write `update`);
+    anchor frames are not written."""
     T = k.shape[0]
     anc = set(anchor_frames(T, anchors))
     F = np.empty((T + 1,) + np.shape(S0))
@@ -181,13 +228,14 @@ def forward_states(S0, k, v, beta, alpha, anchors: int = 4) -> np.ndarray:
         if t in anc:
             F[t + 1] = F[t]
         else:
-            F[t + 1] = vda_update(alpha[t] * F[t], k[t], v[t], beta[t])
+            F[t + 1] = update(alpha[t] * F[t], k[t], v[t], beta[t])
     return F
 
 
-def backward_states(S0, k, v, beta, alpha, anchors: int = 4) -> np.ndarray:
+def backward_states(S0, k, v, beta, alpha, anchors: int = 4, update=vda_update) -> np.ndarray:
     """Backward scan: G[t] covers frames >= t (G[T] = S0), built from the
-    last frame down with the same per-frame update."""
+    last frame down with the same per-frame update (the tokens of a frame
+    keep their order under the token-wise rule)."""
     T = k.shape[0]
     anc = set(anchor_frames(T, anchors))
     G = np.empty((T + 1,) + np.shape(S0))
@@ -196,7 +244,7 @@ def backward_states(S0, k, v, beta, alpha, anchors: int = 4) -> np.ndarray:
         if t in anc:
             G[t] = G[t + 1]
         else:
-            G[t] = vda_update(alpha[t] * G[t + 1], k[t], v[t], beta[t])
+            G[t] = update(alpha[t] * G[t + 1], k[t], v[t], beta[t])
     return G
 
 
@@ -399,8 +447,9 @@ def head_states(inp: dict, cfg: Cfg, b: int, h: int):
     beta = inp["beta"][b, :, :, h]
     alpha = inp["alpha"][b, :, h]
     F0 = np.asarray(inp["fwd_init"][b, h], F64) if inp.get("fwd_init") is not None else S0
-    F = forward_states(F0, k, v, beta, alpha, cfg.anchors)
-    G = backward_states(S0, k, v, beta, alpha, cfg.anchors)
+    f = frame_update(cfg.update)
+    F = forward_states(F0, k, v, beta, alpha, cfg.anchors, f)
+    G = backward_states(S0, k, v, beta, alpha, cfg.anchors, f)
     return F, G
 
 
@@ -465,7 +514,8 @@ def vda_intermediates(inp: dict, cfg: Cfg, b: int, h: int):
     for t in range(T):
         if t in anc:
             continue
-        Ms[t], Cs[t] = frame_map(inp["k"][b, t, :, h], inp["v"][b, t, :, h], inp["beta"][b, t, :, h])
+        kk, vv, bb = inp["k"][b, t, :, h], inp["v"][b, t, :, h], inp["beta"][b, t, :, h]
+        Ms[t], Cs[t] = frame_map(kk, vv, bb) if cfg.update == 0 else variant_frame_map(kk, vv, bb, cfg.update)
     F, G = head_states(inp, cfg, b, h)
     # the backward scan always starts from half the text state (the forward
     # one from fwd_init when that is given)

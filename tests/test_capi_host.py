@@ -69,6 +69,8 @@ def test_workspace_size_and_layout():
     (dict(d_k=48, d_v=48), L.VDN_ERR_UNSUPPORTED), (dict(d_v=64), L.VDN_ERR_UNSUPPORTED),
     (dict(chunk=4), L.VDN_ERR_UNSUPPORTED), (dict(B=3000, H=24), L.VDN_ERR_UNSUPPORTED),
     (dict(scan_mode=3), L.VDN_ERR_INVALID_ARG), (dict(scan_mode=-1), L.VDN_ERR_INVALID_ARG),
+    (dict(update=3), L.VDN_ERR_INVALID_ARG), (dict(update=-1), L.VDN_ERR_INVALID_ARG),
+    (dict(update=2, d_k=256, d_v=256), L.VDN_ERR_UNSUPPORTED),
 ])
 def test_bad_config_rejected(kw, status):
     cfg = _cfg(**kw)
@@ -148,6 +150,11 @@ def test_status_strings_and_stage_impl():
         assert L.vdn_hybrid_stage_impl(big, st) in (0, 1)
     assert L.vdn_hybrid_attn_workspace_size(big) > 0
     assert L.vdn_hybrid_stage_impl(_cfg(d_k=256, d_v=256, dtype=L.VDN_F32), L.STAGE_SOLVE) == -1
+    # the ablation writes: their own per-frame map kernel, then the SIMT scan
+    for u in (1, 2):
+        v = _cfg(update=u, d_k=128, d_v=128)
+        assert L.vdn_hybrid_stage_impl(v, L.STAGE_SOLVE) == 2
+        assert L.vdn_hybrid_stage_impl(v, L.STAGE_SCAN) == 0
     assert L.vdn_hybrid_attn_workspace_size(_cfg(d_k=256, d_v=256, dtype=L.VDN_F32)) == 0
 
 

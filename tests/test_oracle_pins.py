@@ -542,3 +542,91 @@ def test_stream_default_start_is_half_the_text_state():
     want = O.hybrid_attn(inp, cfg)
     got = O.hybrid_attn({**inp, "fwd_init": half}, cfg)
     np.testing.assert_array_equal(got, want)
+
+
+# ------------------------------------------------------ ablation writes ----
+def _explicit_token_chain(Sbar, K, V, beta):
+    """The token-wise rule as explicit matrices: S_bar P_1 ... P_N + sum_i
+    beta_i v_i k_i^T P_{i+1} ... P_N with P_i = I - beta_i k_i k_i^T."""
+    d = K.shape[1]
+    P = [np.eye(d) - b * np.outer(k, k) for k, b in zip(K, beta)]
+    tail = [np.linalg.multi_dot(P[i + 1:] + [np.eye(d), np.eye(d)]) for i in range(len(P))]
+    S = Sbar @ np.linalg.multi_dot(P + [np.eye(d)])
+    for i in range(len(P)):
+        S = S + beta[i] * np.outer(V[i], K[i]) @ tail[i]
+    return S
+
+
+def test_token_rule_equals_explicit_matrix_chain():
+    Sbar, K, V, beta = _frame(7, 6, 5, seed=11)
+    np.testing.assert_allclose(O.token_delta_update(Sbar, K, V, beta), _explicit_token_chain(Sbar, K, V, beta),
+                               rtol=0, atol=1e-13)
+
+
+def test_token_rule_recalls_the_last_write_exactly():
+    """beta = 1 with a unit key is the classic delta rule's exact overwrite:
+    afterwards S k_N = v_N whatever came before."""
+    Sbar, K, V, _ = _frame(9, 8, 8, seed=12)
+    S = O.token_delta_update(Sbar, K, V, np.ones(9))
+    np.testing.assert_allclose(S @ K[-1], V[-1], atol=1e-13)
+
+
+def test_token_rule_depends_on_order_the_others_do_not():
+    """Only the token-wise rule sees the token order (the joint solve and the
+    frame-level writes treat the frame as a set)."""
+    Sbar, K, V, beta = _frame(6, 4, 4, seed=13)
+    perm = np.arange(6)[::-1]
+    for u in (0, 1):
+        f = O.frame_update(u)
+        np.testing.assert_allclose(f(Sbar, K, V, beta), f(Sbar, K[perm], V[perm], beta[perm]), atol=1e-13)
+    a = O.token_delta_update(Sbar, K, V, beta)
+    b = O.token_delta_update(Sbar, K[perm], V[perm], beta[perm])
+    assert np.max(np.abs(a - b)) > 1e-3
+
+
+def test_frame_rule_is_size_invariant_and_averages_orthogonal_writes():
+    """Frame-level writes with the 1/N rescaling: N copies of one token write
+    what the single token writes; with orthonormal keys (where the token rule's
+    steps do not interact) the frame rule moves S_bar 1/N of the way the token
+    rule does."""
+    Sbar, K, V, beta = _frame(1, 6, 5, seed=14)
+    one = O.frame_independent_update(Sbar, K, V, beta)
+    many = O.frame_independent_update(Sbar, np.repeat(K, 9, 0), np.repeat(V, 9, 0), np.repeat(beta, 9))
+    np.testing.assert_allclose(many, one, atol=1e-13)
+    Q = np.linalg.qr(np.random.default_rng(15).standard_normal((6, 6)))[0][:4]
+    V4 = np.random.default_rng(16).standard_normal((4, 5))
+    b4 = np.array([0.3, 0.9, 0.5, 0.7])
+    tok = O.token_delta_update(Sbar, Q, V4, b4)
+    frm = O.frame_independent_update(Sbar, Q, V4, b4)
+    np.testing.assert_allclose(frm - Sbar, (tok - Sbar) / 4, atol=1e-13)
+
+
+@pytest.mark.parametrize("update", [0, 1, 2])
+def test_every_write_is_the_affine_map_of_its_frame(update):
+    """S = S_bar M + C for any S_bar, with (M, C) from variant_frame_map; for
+    the joint solve (M, C) equal frame_map's closed form."""
+    _, K, V, beta = _frame(11, 8, 6, seed=17)
+    M, C = O.variant_frame_map(K, V, beta, update)
+    f = O.frame_update(update)
+    for s in range(3):
+        Sbar = np.random.default_rng(20 + s).standard_normal((6, 8))
+        np.testing.assert_allclose(f(Sbar, K, V, beta), Sbar @ M + C, atol=1e-12)
+    if update == 0:
+        M0, C0 = O.frame_map(K, V, beta)
+        np.testing.assert_allclose(M, M0, atol=1e-13)
+        np.testing.assert_allclose(C, C0, atol=1e-13)
+
+
+def test_frame_rule_needs_its_rescaling_to_stay_non_expansive():
+    """With unit keys and beta <= 1, I - A/N has spectral norm <= 1; the
+    unrescaled I - A of a frame of many aligned tokens does not ([P5]: the
+    joint solve needs no frame-size rescaling, unlike SANA-WM)."""
+    r = np.random.default_rng(18)
+    k0 = r.standard_normal(8)
+    K = k0 + 0.1 * r.standard_normal((50, 8))
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    beta = 1 / (1 + np.exp(-r.standard_normal(50)))
+    M, _ = O.variant_frame_map(K, np.zeros((50, 8)), beta, 1)
+    assert np.linalg.norm(M, 2) <= 1 + 1e-12
+    A = (beta[:, None] * K).T @ K
+    assert np.linalg.norm(np.eye(8) - A, 2) > 1

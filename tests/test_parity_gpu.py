@@ -28,7 +28,7 @@ def _built(cuda_ok):
 def ocfg(cfg: L.HybridCfg) -> O.Cfg:
     return O.Cfg(B=cfg.B, T=cfg.T, N=cfg.N, H=cfg.H, d_k=cfg.d_k, d_v=cfg.d_v, L=cfg.L, chunk=cfg.chunk,
                  anchors=cfg.anchors, softmax_scale=cfg.softmax_scale, rms_eps=cfg.rms_eps or 1e-6,
-                 out_mode=cfg.out_mode)
+                 out_mode=cfg.out_mode, update=cfg.update)
 
 
 def run(shape: Shape, dtype: str, seed: int, extra=None, drop_text=False, stages=L.STAGE_ALL, **kw):
@@ -556,3 +556,39 @@ def test_stream_two_segments_match_oracle(dtype, d):
     torch.cuda.synchronize()
     ref2 = O.hybrid_attn({**inp2, "fwd_init": carried}, O.Cfg(**{**ocfg(cfg2).__dict__, "out_mode": 0}))
     check(y2, ref2, cfg2, dtype)
+
+
+VARIANT_SHAPES = [Shape(1, 12, 40, 2, 32, 32, 4), Shape(1, 15, 70, 2, 64, 64, 8), Shape(1, 12, 50, 1, 128, 128, 8)]
+
+
+@pytest.mark.parametrize("update", [1, 2])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", VARIANT_SHAPES, ids=lambda s: f"d{s.d_k}")
+def test_ablation_write_matches_oracle(shape, dtype, update):
+    """The ablation writes (1: frame-level independent writes with the 1/N
+    rescaling; 2: the token-wise delta rule): their per-frame maps M'_t, C'_t
+    in the M_t, C_t slots, the chunk-boundary states of both scans and the
+    whole output, against the oracle with the same write."""
+    inp, cfg, ha, _, y = run(shape, dtype, 41, update=update)
+    oc = ocfg(cfg)
+    check(y, O.hybrid_attn(inp, O.Cfg(**{**oc.__dict__, "out_mode": 0})), cfg, dtype)
+    it = {k: v.double().cpu().numpy() for k, v in ha.intermediates().items()}
+    for h in range(cfg.H):
+        ref = O.vda_intermediates(inp, oc, 0, h)
+        scale = np.sqrt(np.mean(ref["R"] ** 2))
+        for t in range(1, cfg.T - 1):
+            np.testing.assert_allclose(it["M"][0, t, h], ref["M"][t], rtol=0, atol=2e-5)
+            np.testing.assert_allclose(it["C"][0, t, h], ref["C"][t], rtol=0, atol=2e-5 * np.abs(ref["C"][t]).max())
+        for j in range(cfg.C + 1):
+            fj = min(5 * j, cfg.T)
+            np.testing.assert_allclose(it["fwd_snap"][0, h, j], ref["F"][fj], rtol=0, atol=1e-4 * scale)
+            np.testing.assert_allclose(it["bwd_snap"][0, h, j], ref["G"][fj], rtol=0, atol=1e-4 * scale)
+
+
+def test_ablation_write_ragged_frame():
+    """A frame of 37 tokens: two full staged blocks and a partial third."""
+    shape = Shape(1, 7, 37, 3, 64, 64, 0)
+    for update in (1, 2):
+        inp, cfg, _, _, y = run(shape, "bf16", 43, drop_text=True, update=update)
+        oc = ocfg(cfg)
+        check(y, O.hybrid_attn(inp, O.Cfg(**{**oc.__dict__, "out_mode": 0})), cfg, "bf16")

@@ -31,7 +31,8 @@ class VdnCfg(C.Structure):
     _fields_ = [("B", C.c_int), ("T", C.c_int), ("N", C.c_int), ("H", C.c_int), ("d_k", C.c_int),
                 ("d_v", C.c_int), ("L", C.c_int), ("chunk", C.c_int), ("anchors", C.c_int),
                 ("dtype", C.c_int), ("softmax_scale", C.c_float), ("rms_eps", C.c_float),
-                ("out_mode", C.c_int), ("y_dtype", C.c_int), ("scan_mode", C.c_int)]
+                ("out_mode", C.c_int), ("y_dtype", C.c_int), ("scan_mode", C.c_int),
+                ("update", C.c_int)]
 
 
 class VdnArgs(C.Structure):
@@ -71,6 +72,7 @@ class HybridCfg:
     out_mode: int = 0
     y_dtype: int = VDN_F32
     scan_mode: int = 0
+    update: int = 0  # 0 joint solve, 1 frame-level independent writes (1/N), 2 token-wise delta rule
 
     def c(self) -> VdnCfg:
         return VdnCfg(**{f.name: getattr(self, f.name) for f in fields(self)})

@@ -22,11 +22,14 @@ vdn_status check_cfg(const vdn_hybrid_cfg* c) {
   if (c->out_mode != 0 && c->out_mode != 1) return VDN_ERR_INVALID_ARG;
   if (c->y_dtype != VDN_F32 && c->y_dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
   if (c->scan_mode < 0 || c->scan_mode > 2) return VDN_ERR_INVALID_ARG;
+  if (c->update < 0 || c->update > 2) return VDN_ERR_INVALID_ARG;
   if (!(c->softmax_scale == c->softmax_scale) || !(c->rms_eps == c->rms_eps)) return VDN_ERR_INVALID_ARG;
   if (c->d_k != 32 && c->d_k != 64 && c->d_k != 128 && c->d_k != 256) return VDN_ERR_UNSUPPORTED;
   if (c->d_v != c->d_k) return VDN_ERR_UNSUPPORTED;
   // d = 256: the per-frame Gram runs on the tensor cores only (bf16 inputs)
   if (c->d_k == 256 && c->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
+  // the ablation variants run the SIMT (C-form) scan, built for d <= 128
+  if (c->update != 0 && c->d_k > 128) return VDN_ERR_UNSUPPORTED;
   if (c->chunk != 5) return VDN_ERR_UNSUPPORTED;
   // grid limits of the launches (gridDim.y / gridDim.z <= 65535)
   if ((long long)c->B * c->H > 65535) return VDN_ERR_UNSUPPORTED;
@@ -47,6 +50,7 @@ Dims make_dims(const vdn_hybrid_cfg* c) {
   d.bf16 = c->dtype == VDN_BF16;
   d.out_bf16 = c->y_dtype == VDN_BF16;
   d.scan_mode = c->scan_mode;
+  d.update = c->update;
   return d;
 }
 
@@ -167,8 +171,10 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
   switch (stage) {
     case VDN_STAGE_SCAN:
       return scan_tc_supported(d) ? 1 : 0;
-    case VDN_STAGE_TEXT:
     case VDN_STAGE_SOLVE:
+      if (d.update != 0) return 2;  // the variant-map kernel
+      return gram_tc_supported(d) ? 1 : 0;
+    case VDN_STAGE_TEXT:
       return gram_tc_supported(d) ? 1 : 0;
     case VDN_STAGE_READ:
       return read_tc_supported(d) ? 1 : 0;
@@ -209,7 +215,9 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     }
   }
   if (stages & VDN_STAGE_SOLVE) {
-    if (gram_tc_supported(d)) {
+    if (d.update != 0) {
+      if (launch_variant_maps(d, in, w, s) != cudaSuccess) return VDN_ERR_CUDA;
+    } else if (gram_tc_supported(d)) {
       if ((e = launch_gram_tc(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
       e = big ? launch_solve_big(d, w, s, false) : launch_solve_inplace(d, w, s);
       if (e != cudaSuccess) return VDN_ERR_CUDA;

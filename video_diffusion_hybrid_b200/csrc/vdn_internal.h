@@ -17,6 +17,7 @@ struct Dims {
   int bf16;      // inputs stored as bf16
   int out_bf16;  // y stored as bf16
   int scan_mode;  // 0 auto, 1 frame steps, 2 chunk steps (tensor-core scan)
+  int update;     // 0 joint solve, 1 frame-level independent writes (1/N), 2 token-wise delta rule
 };
 
 // Device-side status words at the head of the workspace.
@@ -66,6 +67,8 @@ cudaError_t launch_text_gram_tc(const Dims& d, const Inputs& in, const Work& w, 
 bool gram_tc_supported(const Dims& d);
 cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+// the ablation variants' per-frame maps (M'_t, C'_t) into the M_t, C_t slots
+cudaError_t launch_variant_maps(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_read_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_softmax_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 bool softmax_tc_supported(const Dims& d);

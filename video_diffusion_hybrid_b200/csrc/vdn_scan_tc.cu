@@ -412,6 +412,8 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
 }  // namespace
 
 bool scan_tc_supported(const Dims& d) {
+  // the tensor-core scan steps the joint solve's B form only
+  if (d.update != 0) return false;
   if (!scan_tc_layout(d.bf16 != 0, d.dk, d.dv) || !gram_tc_supported(d)) return false;
   if ((long long)d.B * d.T * d.H * 2 * d.dk >= (1LL << 31)) return false;  // TMA row coordinates
   if ((long long)d.B * d.H * 4 > 0x7FFFFFFFLL) return false;

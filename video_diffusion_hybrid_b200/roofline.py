@@ -65,6 +65,14 @@ def sweep_flops(B, T, H, d, anchors=4, with_c=True) -> float:
     return (4.0 if with_c else 2.0) * d ** 3 * written_frames(T, anchors) * B * H
 
 
+def variant_map_flops(B, T, N, H, d, anchors=4, update=2) -> float:
+    """The ablation writes' per-frame maps: every token updates each of the
+    2d rows of the stacked [M'; C'] (d multiply-adds a row), and the
+    token-wise rule first takes each row's dot product with the key (d more)."""
+    per_token = (4.0 if update == 2 else 2.0) * 2 * d * d
+    return per_token * N * written_frames(T, anchors) * B * H
+
+
 def scan_bytes(B, T, H, d, chunk=5, anchors=4) -> float:
     """Both directions read every written frame's M_t (as its bf16 hi/lo
     split, 4 bytes an entry) and C_t (fp32); the chunk-boundary states (fp32,
