@@ -27,9 +27,9 @@
 //   token rule: coef = beta_i (target_r - row_r . k_i),
 //   frame rule: coef = beta_i (target_r - e_r . k_i) / N   (the frozen state),
 // target_r = 0 for rows of M' and v_i[r - D] for rows of C'.  Rows never
-// interact; tokens are staged in shared memory 16 at a time (k and v as
-// fp32), double-buffered with the next block prefetched into registers while
-// the current one is applied.  With bf16 inputs (d = 64, 128) the frame rule
+// interact; tokens are staged in shared memory 16 at a time in their stored
+// type by asynchronous copies, double-buffered, the next block in flight
+// while the current one is applied.  With bf16 inputs (d = 64, 128) the frame rule
 // instead takes A_t and B_t from the tensor-core Gram kernel and rescales
 // them in place: M'_t = I - A_t / N, C'_t = B_t / N.
 #include <cuda_bf16.h>
@@ -41,91 +41,120 @@ namespace {
 
 constexpr int kTB = 16;  // tokens per staged block
 
-__device__ __forceinline__ float ld_f(const float* p) { return __ldg(p); }
-__device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-
 // Thread tile: RT = 4 rows x CT = 16 columns of the stacked map.  The CG =
 // D / 16 threads of a row group are adjacent lanes, so a row's dot product
-// with the key is their partial sums reduced by log2(CG) xor shuffles.  Per
-// token a thread loads 16 key columns (four 16-byte shared loads) and the 4
-// targets, and does 64 (+ 64 for the dot) multiply-adds.
+// with the key is their partial sums reduced by log2(CG) xor shuffles.  Keys
+// stay in shared memory in their stored type (VW = 16 / sizeof(T) to a
+// 16-byte load); lane cg of a group holds the columns VW cg + VW CG m +
+// (0 .. VW - 1), so the group's 16-byte loads fall on distinct banks.  Per
+// token a thread loads its 16 key columns and the 4 targets, and does 64
+// (+ 64 for the dot) multiply-adds.
 constexpr int RT = 4, CT = 16;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+// asynchronous copies into shared memory; an invalid source fills zeros
+// (no bytes are read, src stays a valid address)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// 16 bytes of shared memory as floats
+__device__ __forceinline__ void ld_vec(const float* p, float* out) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+}
+__device__ __forceinline__ void ld_vec(const __nv_bfloat16* p, float* out) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    out[2 * i] = __uint_as_float(u[i] << 16);
+    out[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+  }
+}
+// 4 consecutive entries as floats
+__device__ __forceinline__ void ld4(const float* p, float* out) { ld_vec(p, out); }
+__device__ __forceinline__ void ld4(const __nv_bfloat16* p, float* out) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  out[0] = __uint_as_float(v.x << 16);
+  out[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  out[2] = __uint_as_float(v.y << 16);
+  out[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
 
 template <typename T, int D, int VAR>
 __global__ void __launch_bounds__(2 * D / RT * (D / CT)) k_variant_map(Dims dm, Inputs in, Work w) {
-  constexpr int R = 2 * D;          // rows of [M'; C']
-  constexpr int CG = D / CT;        // threads per row group
-  constexpr int NT = R / RT * CG;   // threads
-  constexpr int PRE = kTB * R / NT; // staged elements per thread and block
-  static_assert(kTB * R % NT == 0 && 32 % CG == 0, "variant tiling");
-  __shared__ __align__(16) float sk[2][kTB][R];  // token j: k at [0, D), v at [D, 2D)
-  __shared__ float sb[2][kTB];
+  constexpr int R = 2 * D;            // rows of [M'; C']
+  constexpr int CG = D / CT;          // threads per row group
+  constexpr int NT = R / RT * CG;     // threads
+  constexpr int VW = 16 / (int)sizeof(T);  // entries in 16 bytes
+  constexpr int CPR = R / VW;         // 16-byte chunks of a token's [k; v] row
+  static_assert(CT % VW == 0 && 32 % CG == 0, "variant tiling");
+  __shared__ __align__(16) T sk[2][kTB][R];  // token j: k at [0, D), v at [D, 2D)
+  __shared__ __align__(16) float sb[2][kTB];
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (is_anchor(dm, t)) return;  // anchor frames are not written
-  const int tid = threadIdx.x, r0 = (tid / CG) * RT, c0 = (tid % CG) * CT;
+  const int tid = threadIdx.x, r0 = (tid / CG) * RT, cg = tid % CG;
+  // column of this thread's entry c (0 .. CT - 1)
+  auto col = [&](int c) { return VW * cg + (c / VW) * (VW * CG) + (c % VW); };
   const long long fh = ((long long)b * dm.T + t) * dm.H + h;
   const T* kp = static_cast<const T*>(in.k);
   const T* vp = static_cast<const T*>(in.v);
   const long long tok0 = ((long long)b * dm.T + t) * dm.N;  // first token of the frame
-  // staged element e = i NT + tid of a block: token e / R, entry e % R of its
-  // [k; v] row, 0 past the frame's last token
-  auto fetch = [&](int n0, int i) -> float {
-    const int e = i * NT + tid, n = n0 + e / R, u = e % R;
-    if (n >= dm.N) return 0.f;
-    const long long row = (tok0 + n) * dm.H + h;
-    return u < D ? ld_f(kp + row * D + u) : ld_f(vp + row * D + (u - D));
-  };
-  auto fetch_beta = [&](int n) -> float {
-    return n < dm.N ? __ldg(in.beta + (tok0 + n) * dm.H + h) : 0.f;
-  };
-  auto stage = [&](int buf, const float (&v)[PRE]) {
-#pragma unroll
-    for (int i = 0; i < PRE; ++i) {
-      const int e = i * NT + tid;
-      sk[buf][e / R][e % R] = v[i];
+  // stage tokens n0 .. n0 + kTB - 1 into buffer buf (zeros past the frame)
+  auto stage = [&](int buf, int n0) {
+    for (int q = tid; q < kTB * CPR; q += NT) {
+      const int j = q / CPR, u = (q % CPR) * VW, n = n0 + j;
+      const bool ok = n < dm.N;
+      const long long row = (tok0 + (ok ? n : 0)) * dm.H + h;
+      const T* src = u < D ? kp + row * D + u : vp + row * D + (u - D);
+      cp_async16(&sk[buf][j][u], src, ok);
     }
+    if (tid < kTB) {
+      const int n = n0 + tid;
+      const bool ok = n < dm.N;
+      cp_async4(&sb[buf][tid], in.beta + (tok0 + (ok ? n : 0)) * dm.H + h, ok);
+    }
+    cp_async_commit();
   };
 
   float z[RT][CT];
 #pragma unroll
   for (int i = 0; i < RT; ++i)
 #pragma unroll
-    for (int c = 0; c < CT; ++c) z[i][c] = (r0 + i == c0 + c) ? 1.f : 0.f;  // e_r on rows of M'
+    for (int c = 0; c < CT; ++c) z[i][c] = (r0 + i == col(c)) ? 1.f : 0.f;  // e_r on rows of M'
   const float inv_n = 1.0f / (float)dm.N;
   const int nblk = (dm.N + kTB - 1) / kTB;
 
-  float pre[PRE];
-  float preb = 0.f;
-#pragma unroll
-  for (int i = 0; i < PRE; ++i) pre[i] = fetch(0, i);
-  if (tid < kTB) preb = fetch_beta(tid);
-  stage(0, pre);
-  if (tid < kTB) sb[0][tid] = preb;
+  stage(0, 0);
+  cp_async_wait_all();
   __syncthreads();
 
   for (int blk = 0; blk < nblk; ++blk) {
     const int cur = blk & 1;
     const bool more = blk + 1 < nblk;
-    if (more) {
-      const int n0 = (blk + 1) * kTB;
-#pragma unroll
-      for (int i = 0; i < PRE; ++i) pre[i] = fetch(n0, i);
-      if (tid < kTB) preb = fetch_beta(n0 + tid);
-    }
+    // the other buffer was last read before the previous barrier
+    if (more) stage(cur ^ 1, (blk + 1) * kTB);
 #pragma unroll 1
     for (int j = 0; j < kTB; ++j) {
-      const float* kv = sk[cur][j];
+      const T* kv = sk[cur][j];
       const float beta = sb[cur][j];
       float k[CT];
 #pragma unroll
-      for (int c = 0; c < CT; c += 4) {
-        const float4 k4 = *reinterpret_cast<const float4*>(kv + c0 + c);
-        k[c] = k4.x; k[c + 1] = k4.y; k[c + 2] = k4.z; k[c + 3] = k4.w;
-      }
+      for (int c = 0; c < CT; c += VW) ld_vec(kv + col(c), k + c);
       // entries r0 .. r0 + 3 of [k; v]: the rows' k entries (rows of M') or
       // their value targets (rows of C')
-      const float4 e4 = *reinterpret_cast<const float4*>(kv + r0);
-      const float ent[RT] = {e4.x, e4.y, e4.z, e4.w};
+      float ent[RT];
+      ld4(kv + r0, ent);
       const bool mrow = r0 < D;
       float coef[RT];
       if (VAR == 2) {
@@ -156,11 +185,7 @@ __global__ void __launch_bounds__(2 * D / RT * (D / CT)) k_variant_map(Dims dm, 
 #pragma unroll
         for (int c = 0; c < CT; ++c) z[i][c] = fmaf(coef[i], k[c], z[i][c]);
     }
-    if (more) {
-      // the other buffer was last read before the previous barrier
-      stage(cur ^ 1, pre);
-      if (tid < kTB) sb[cur ^ 1][tid] = preb;
-    }
+    cp_async_wait_all();
     __syncthreads();
   }
 
@@ -168,10 +193,10 @@ __global__ void __launch_bounds__(2 * D / RT * (D / CT)) k_variant_map(Dims dm, 
 #pragma unroll
   for (int i = 0; i < RT; ++i) {
     const int r = r0 + i;
-    float* dst = (r < D ? w.M + fh * DD + (long long)r * D : w.Cm + fh * DD + (long long)(r - D) * D) + c0;
+    float* dst = r < D ? w.M + fh * DD + (long long)r * D : w.Cm + fh * DD + (long long)(r - D) * D;
 #pragma unroll
     for (int c = 0; c < CT; c += 4)
-      *reinterpret_cast<float4*>(dst + c) = make_float4(z[i][c], z[i][c + 1], z[i][c + 2], z[i][c + 3]);
+      *reinterpret_cast<float4*>(dst + col(c)) = make_float4(z[i][c], z[i][c + 1], z[i][c + 2], z[i][c + 3]);
   }
 }
 
