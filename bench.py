@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--update", type=int, choices=(0, 1, 2), default=0,
                     help="the linear branch's frame write: 0 the joint solve; ablation baselines 1 frame-level "
                          "independent writes (1/N rescaled), 2 the token-wise delta rule")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="one problem of the workload's shape over the launched ranks, heads split across them "
+                         "(sequence-sharded in and out, two all-to-alls around the core): strong scaling")
     ap.add_argument("--proj", action="store_true",
                     help="time the layer's output projection (one GEMM over the core's concat axis) at the "
                          "workload's shape instead of the core")
@@ -606,8 +609,77 @@ def run_xattn(args):
         "clocks": clocks}), flush=True)
 
 
+def run_ulysses(args):
+    """The workload's one problem over the launched ranks with the heads split
+    (Ulysses): every rank holds 1/P of the token sequence of every head, two
+    all-to-alls (NCCL) move it to and from head shards around the core.  The
+    whole job is one problem, so value = its tokens / the slowest rank's time."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from video_diffusion_hybrid_b200 import _lib as L
+    from video_diffusion_hybrid_b200.api import cfg_for
+    from video_diffusion_hybrid_b200.synth import make_inputs_torch
+    from video_diffusion_hybrid_b200.ulysses import PER_TOKEN, UlyssesHybridAttention
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    L.lib()
+    w = WORKLOADS[args.workload]
+    s = w.shape
+    # the same problem on every rank; each keeps its shard of the token sequence
+    full = make_inputs_torch(s, w.seed, w.dtype, dev)
+    sl = s.T * s.N // world
+    t = {k: (v.flatten(1, 2).narrow(1, rank * sl, sl).contiguous() if k in PER_TOKEN else v)
+         for k, v in full.items()}
+    del full
+    u = UlyssesHybridAttention(cfg_for(s, w.dtype), None, dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(args.warmup, 3)):
+        y = u(t)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        y = u(t)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
+    # the core's device status words (bounded waits that gave up, if any)
+    st, where = u.device_status()
+    if st != L.VDN_OK:
+        raise SystemExit(f"rank {rank}: device status {st} (kernel tag {where})")
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": w.tokens / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "B": s.B, "T": s.T, "N": s.N, "H": s.H, "d": s.d_k, "L": s.L,
+                       "parallelism": f"ulysses{world}", "heads_per_rank": s.H // world,
+                       "exchange": "NCCL all_to_all_single, sequence <-> heads, before and after the core"},
+            "output_shape": list(y.shape)}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
+    if args.ulysses:
+        run_ulysses(args)
+        return
     if args.xattn:
         run_xattn(args)
         return

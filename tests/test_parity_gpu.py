@@ -592,3 +592,19 @@ def test_ablation_write_ragged_frame():
         inp, cfg, _, _, y = run(shape, "bf16", 43, drop_text=True, update=update)
         oc = ocfg(cfg)
         check(y, O.hybrid_attn(inp, O.Cfg(**{**oc.__dict__, "out_mode": 0})), cfg, "bf16")
+
+
+def test_ulysses_wrapper_single_rank_matches_oracle():
+    """The Ulysses wrapper in one process (no exchange): sequence-flattened
+    inputs in, [B, T N, H, 2, d_v] out, against the oracle."""
+    from video_diffusion_hybrid_b200.ulysses import PER_TOKEN, UlyssesHybridAttention
+    shape = Shape(1, 12, 40, 2, 64, 64, 6)
+    inp = make_inputs(shape, 51, "bf16")
+    cfg = cfg_for(shape, "bf16")
+    t = to_torch(inp, "bf16", "cuda")
+    t = {k: (v.flatten(1, 2) if k in PER_TOKEN else v) for k, v in t.items()}
+    u = UlyssesHybridAttention(cfg)
+    y = u(t)
+    assert u.device_status()[0] == L.VDN_OK
+    got = y.float().cpu().numpy().astype(np.float64).reshape(1, 12, 40, 2, 2, 64)
+    check(got, oracle(inp, cfg), cfg, "bf16")
