@@ -1,0 +1,57 @@
+"""Pins of the gradient oracle of the linear branch: its forward is the
+numpy oracle's linear slot, and its gradients match central finite
+differences of the numpy oracle along random directions."""
+import numpy as np
+import pytest
+
+from oracle import vdn_oracle as O
+from oracle import vdn_oracle_grad as OG
+from video_diffusion_hybrid_b200.synth import Shape, make_inputs
+
+
+def _case(anchors=4, L=3, weight=True, T=12):
+    shp = Shape(B=1, T=T, N=5, H=2, d_k=6, d_v=6, L=L)
+    inp = {k: np.asarray(v, np.float64) for k, v in make_inputs(shp, seed=21).items() if not k.endswith("_bits")}
+    r = np.random.default_rng(22)
+    if weight:
+        inp["rms_weight"] = 1 + 0.3 * r.standard_normal((2, 6))
+    cfg = O.Cfg(B=1, T=T, N=5, H=2, d_k=6, d_v=6, L=L, anchors=anchors)
+    return inp, cfg
+
+
+@pytest.mark.parametrize("anchors", [4, 0])
+def test_torch_forward_is_the_oracle(anchors):
+    inp, cfg = _case(anchors)
+    np.testing.assert_allclose(OG.linear_branch_forward(inp, cfg), O.hybrid_attn(inp, cfg)[..., 1, :],
+                               rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("anchors,weight", [(4, True), (0, False)])
+def test_gradients_match_finite_differences(anchors, weight):
+    inp, cfg = _case(anchors, weight=weight)
+    r = np.random.default_rng(23)
+    dy = r.standard_normal((1, cfg.T, 5, 2, 6))
+    grads = OG.linear_branch_grads(inp, cfg, dy)
+    f = lambda d: float(np.sum(O.hybrid_attn(d, cfg)[..., 1, :] * dy))
+    for name, g in grads.items():
+        u = r.standard_normal(g.shape)
+        if name == "beta":
+            u *= 0.1
+        eps = 1e-6
+        plus, minus = dict(inp), dict(inp)
+        plus[name] = inp[name] + eps * u
+        minus[name] = inp[name] - eps * u
+        fd = (f(plus) - f(minus)) / (2 * eps)
+        an = float(np.sum(g * u))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_anchor_tokens_get_no_write_gradient():
+    """Anchor frames are never written, so their k, v and beta do not reach
+    the linear branch; their q still reads."""
+    inp, cfg = _case(4)
+    g = OG.linear_branch_grads(inp, cfg, np.ones((1, cfg.T, 5, 2, 6)))
+    for name in ("k", "v", "beta"):
+        assert np.all(g[name][:, 0] == 0) and np.all(g[name][:, -1] == 0)
+        assert np.any(g[name][:, 1] != 0)
+    assert np.any(g["q"][:, 0] != 0)
