@@ -7,9 +7,10 @@ torch ops, step for step as ``vdn_oracle`` defines it (joint frame write
 S_t = (alpha_t S + B_t)(I + A_t)^-1, both scans from their start states, the
 read of the summed states, RMSNorm and the sigmoid gate: [P1] 三, 四; [P4]
 closed form), and torch's reverse-mode autograd is the library step that
-differentiates it.  The text state (and fwd_init / init_state) is held
-constant: gradients reach the video tokens' q, k, v, beta, the decay alpha,
-the gate logits and the RMSNorm weight.
+differentiates it.  The text state (and init_state) is held constant:
+gradients reach the video tokens' q, k, v, beta, the decay alpha, the gate
+logits, the RMSNorm weight and, when it is given, the streaming forward start
+state fwd_init (the state carried in from the previous segment).
 
 Pinned in the tests by (a) its forward equal to ``vdn_oracle``'s linear slot
 and (b) central finite differences of ``vdn_oracle``'s numpy forward along
@@ -22,7 +23,7 @@ import torch
 
 from . import vdn_oracle as O
 
-GRAD_INPUTS = ("q", "k", "v", "beta", "alpha", "gate_lin", "rms_weight")
+GRAD_INPUTS = ("q", "k", "v", "beta", "alpha", "gate_lin", "rms_weight", "fwd_init")
 
 
 def start_states(inp: dict, cfg: O.Cfg, b: int, h: int):
@@ -42,7 +43,8 @@ def start_states(inp: dict, cfg: O.Cfg, b: int, h: int):
 
 def linear_branch(x: dict, cfg: O.Cfg, starts) -> torch.Tensor:
     """y_lin [B, T, N, H, d_v] from the float64 tensors x (q, k, v, beta,
-    alpha, gate_lin, rms_weight or None); starts[(b, h)] = (F0, S0)."""
+    alpha, gate_lin, rms_weight or None, fwd_init or None); starts[(b, h)] =
+    (F0, S0), F0 replaced by x["fwd_init"][b, h] when that is given."""
     B, T, H = cfg.B, cfg.T, cfg.H
     anc = set(O.anchor_frames(T, cfg.anchors))
     eye = torch.eye(cfg.d_k, dtype=torch.float64)
@@ -51,6 +53,8 @@ def linear_branch(x: dict, cfg: O.Cfg, starts) -> torch.Tensor:
         heads = []
         for h in range(H):
             F0, S0 = (torch.from_numpy(s) for s in starts[(b, h)])
+            if x.get("fwd_init") is not None:
+                F0 = x["fwd_init"][b, h]
 
             def write(S, t):
                 kt, vt, bt = x["k"][b, t, :, h], x["v"][b, t, :, h], x["beta"][b, t, :, h]

@@ -9,26 +9,28 @@ from oracle import vdn_oracle_grad as OG
 from video_diffusion_hybrid_b200.synth import Shape, make_inputs
 
 
-def _case(anchors=4, L=3, weight=True, T=12):
+def _case(anchors=4, L=3, weight=True, T=12, fwd_init=False):
     shp = Shape(B=1, T=T, N=5, H=2, d_k=6, d_v=6, L=L)
     inp = {k: np.asarray(v, np.float64) for k, v in make_inputs(shp, seed=21).items() if not k.endswith("_bits")}
     r = np.random.default_rng(22)
     if weight:
         inp["rms_weight"] = 1 + 0.3 * r.standard_normal((2, 6))
+    if fwd_init:
+        inp["fwd_init"] = 0.5 * r.standard_normal((1, 2, 6, 6))
     cfg = O.Cfg(B=1, T=T, N=5, H=2, d_k=6, d_v=6, L=L, anchors=anchors)
     return inp, cfg
 
 
-@pytest.mark.parametrize("anchors", [4, 0])
-def test_torch_forward_is_the_oracle(anchors):
-    inp, cfg = _case(anchors)
+@pytest.mark.parametrize("anchors,fwd_init", [(4, False), (0, False), (4, True)])
+def test_torch_forward_is_the_oracle(anchors, fwd_init):
+    inp, cfg = _case(anchors, fwd_init=fwd_init)
     np.testing.assert_allclose(OG.linear_branch_forward(inp, cfg), O.hybrid_attn(inp, cfg)[..., 1, :],
                                rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("anchors,weight", [(4, True), (0, False)])
-def test_gradients_match_finite_differences(anchors, weight):
-    inp, cfg = _case(anchors, weight=weight)
+@pytest.mark.parametrize("anchors,weight,fwd_init", [(4, True, False), (0, False, False), (4, False, True)])
+def test_gradients_match_finite_differences(anchors, weight, fwd_init):
+    inp, cfg = _case(anchors, weight=weight, fwd_init=fwd_init)
     r = np.random.default_rng(23)
     dy = r.standard_normal((1, cfg.T, 5, 2, 6))
     grads = OG.linear_branch_grads(inp, cfg, dy)
