@@ -96,7 +96,9 @@ def linear_branch_grads(inp: dict, cfg: O.Cfg, dy: np.ndarray) -> dict:
             x[name] = torch.tensor(np.asarray(inp[name], np.float64), requires_grad=True)
     y = linear_branch(x, cfg, starts)
     (y * torch.from_numpy(np.asarray(dy, np.float64))).sum().backward()
-    return {name: t.grad.numpy() for name, t in x.items()}
+    # an input the output does not reach (at T <= 10 every query reads the
+    # start states only) has gradient zero
+    return {name: (t.grad.numpy() if t.grad is not None else np.zeros(t.shape)) for name, t in x.items()}
 
 
 def linear_branch_forward(inp: dict, cfg: O.Cfg) -> np.ndarray:

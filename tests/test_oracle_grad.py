@@ -57,3 +57,18 @@ def test_anchor_tokens_get_no_write_gradient():
         assert np.all(g[name][:, 0] == 0) and np.all(g[name][:, -1] == 0)
         assert np.any(g[name][:, 1] != 0)
     assert np.any(g["q"][:, 0] != 0)
+
+
+def test_unreached_inputs_get_zero_gradient():
+    """At T = 10 (two chunks) every query reads only the start states, so the
+    frame writes (k, v, beta, alpha) do not reach the output: zero gradients,
+    as finite differences of the numpy oracle also give."""
+    inp, cfg = _case(4, T=10)
+    g = OG.linear_branch_grads(inp, cfg, np.ones((1, 10, 5, 2, 6)))
+    for name in ("k", "v", "beta", "alpha"):
+        assert g[name].shape == inp[name].shape and np.all(g[name] == 0)
+    f = lambda d: float(np.sum(O.hybrid_attn(d, cfg)[..., 1, :]))
+    plus = dict(inp)
+    plus["k"] = inp["k"] + 1e-3
+    assert f(plus) == f(inp)
+    assert np.any(g["q"] != 0)
