@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--ulysses", action="store_true",
                     help="one problem of the workload's shape over the launched ranks, heads split across them "
                          "(sequence-sharded in and out, two all-to-alls around the core): strong scaling")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward of the linear branch (vdn_hybrid_lin_bwd) after one forward")
     ap.add_argument("--proj", action="store_true",
                     help="time the layer's output projection (one GEMM over the core's concat axis) at the "
                          "workload's shape instead of the core")
@@ -609,6 +611,74 @@ def run_xattn(args):
         "clocks": clocks}), flush=True)
 
 
+def bwd_work(s, bf16: bool):
+    """Algorithmic work of one backward of the linear branch: fp32 flops and
+    the bytes it must move.  Per token-head 12 d^2 multiply-adds pairs (o = R q
+    again, dq = R^T do, dR += do q^T; K dA, V dB, K dB^T); per written
+    frame-head four d^3 products for the two state and the two adjoint chains
+    and two for dA.  Bytes: q, k, v, gate_lin in their storage type, beta,
+    dy's linear slot (fp32), and the fp32 dq, dk, dv, dgate_lin, dbeta out."""
+    tok = s.B * s.T * s.N * s.H
+    fh = s.B * (s.T - 2) * s.H
+    d = s.d_k
+    flops = 2.0 * (6 * d * d) * tok + 2.0 * 6 * d ** 3 * fh
+    el = 2 if bf16 else 4
+    byts = tok * (4 * d * el + 4 + 4 * d + 4 * 4 * d + 4)
+    return flops, byts
+
+
+def run_bwd(args):
+    """The linear branch's backward at the workload's size: one forward
+    (which leaves M_t and the write matrices in the workspace), then the timed
+    backward calls, each giving every gradient of q, k, v, beta, alpha,
+    gate_lin and the RMS weight for a fixed upstream gradient dy."""
+    import torch
+    from video_diffusion_hybrid_b200 import _lib as L
+    from video_diffusion_hybrid_b200.api import HybridAttention, cfg_for, output_shape
+    from video_diffusion_hybrid_b200.synth import make_inputs_torch
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    s = w.shape
+    t = make_inputs_torch(s, w.seed, w.dtype, "cuda")
+    cfg = cfg_for(s, w.dtype)
+    ha = HybridAttention(cfg)
+    ha(t)
+    gen = torch.Generator(device="cuda").manual_seed(w.seed + 1)
+    dy = torch.randn(output_shape(cfg), generator=gen, device="cuda")
+    g = ha.linear_backward(t, dy, want_rms=True)
+    lg = L.make_lin_grads(dy, g["dq"], g["dk"], g["dv"], g["dbeta"], g["dalpha"], g["dgate_lin"],
+                          ha.bwd_workspace, drms_weight=g["drms_weight"])
+    a = ha.args(t)
+    for _ in range(max(args.warmup, 3)):
+        L.vdn_hybrid_lin_bwd(cfg, a, lg)
+    torch.cuda.synchronize()
+    clk = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0])
+    clk.start()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        L.vdn_hybrid_lin_bwd(cfg, a, lg)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops, byts = bwd_work(s, w.dtype == "bf16")
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FMA lanes x 2 flops x max SM clock
+    tf = flops / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "linear-branch backward", "value": w.tokens / (ms * 1e-3), "unit": "video tokens/s",
+        "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "n_gpus": 1, "higher_is_better": True,
+        "dtype": "f32" if w.dtype == "f32" else "bf16 in, f32 compute", "data": "synthetic",
+        "config": {"workload": w.name, "B": s.B, "T": s.T, "N": s.N, "H": s.H, "d": s.d_k, "L": s.L,
+                   "l2": "inputs larger than L2"},
+        "gpu_launches": 6 * args.steps,
+        "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                     "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1.965 GHz", "flops": flops,
+                     "hbm_gbs": byts / (ms * 1e-3) / 1e9},
+        "clocks": clocks}), flush=True)
+
+
 def run_ulysses(args):
     """The workload's one problem over the launched ranks with the heads split
     (Ulysses): every rank holds 1/P of the token sequence of every head, two
@@ -682,6 +752,9 @@ def main():
         return
     if args.xattn:
         run_xattn(args)
+        return
+    if args.bwd:
+        run_bwd(args)
         return
     if args.proj:
         run_proj(args)

@@ -231,6 +231,53 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg *cfg, unsigned stage);
 /* Static description of a status code. */
 const char *vdn_status_string(vdn_status s);
 
+/* ------------------------------------------------ backward of the linear branch
+ * Gradients of a loss through the Video Delta Attention branch (its forward as
+ * defined at the top of this header: PaperDaily digest sections 三 and 四,
+ * deepmagic post closed form S_t = (alpha_t S + B_t)(I + A_t)^-1, RMSNorm and
+ * gate of section 三).  The pages describe the forward only; the gradient is
+ * that forward's exact derivative.  Given dy = dL/dy for the core's output,
+ * the call writes dL/dq, dL/dk, dL/dv, dL/dbeta, dL/dalpha and dL/dgate_lin as
+ * far as they flow through y's LINEAR slot (out_mode 0: slot 1 of dy is read;
+ * out_mode 1: dy itself), plus dL/drms_weight and dL/dfwd_init if asked.  The
+ * text state (text_k / text_v / text_beta, init_state) is a constant here.
+ * The softmax branch's share of dq, dk, dv is not included.
+ *
+ * Precondition: args->workspace holds what vdn_hybrid_attn_fwd (or at least its
+ * TEXT and SOLVE stages) wrote for the same cfg and the same inputs: M_t, the
+ * write matrices and S_x / 2 are taken from there, not recomputed.
+ * Reads cfg (update must be 0 and d_k 32, 64 or 128, else VDN_ERR_UNSUPPORTED)
+ * and args q, k, v, beta, alpha, gate_lin, rms_weight, fwd_init, workspace
+ * (y, gate_sm and the text pointers are ignored).  Computes in fp32 (SIMT) for
+ * both input dtypes. */
+typedef struct {
+  const void *dy;      /* dL/dy in y's shape (per cfg.out_mode) and cfg.y_dtype; 16-byte aligned */
+  float *dq, *dk, *dv; /* [B,T,N,H,d] float32, overwritten; anchor frames' dk, dv are zero    */
+  float *dbeta;        /* [B,T,N,H]   float32, overwritten                                   */
+  float *dalpha;       /* [B,T,H]     float32, overwritten (zero at anchor frames)            */
+  float *dgate_lin;    /* [B,T,N,H,d_v] float32, overwritten                                 */
+  float *drms_weight;  /* [H,d_v] float32 or NULL; also when args->rms_weight is NULL (the
+                          gradient at weight = ones)                                         */
+  float *dfwd_init;    /* [B,H,d_v,d_k] float32 or NULL: dL/d(forward start state), i.e.
+                          of args->fwd_init, or of S_x / 2 when that is NULL                  */
+  void *workspace;     /* backward scratch, 256-byte aligned, no overlap with anything else  */
+  size_t workspace_bytes; /* >= vdn_hybrid_lin_bwd_workspace_size(cfg)                       */
+} vdn_lin_grads;
+
+/* Bytes of backward scratch for cfg: every state of both scans and four
+ * d x d matrices per frame-head (0.7 GB at B=1, T=90, H=24, d=128); 0 if cfg
+ * is invalid or not supported by the backward. */
+size_t vdn_hybrid_lin_bwd_workspace_size(const vdn_hybrid_cfg *cfg);
+
+/* Enqueue the backward on `stream` (no synchronisation, no allocation).
+ * Errors (nothing enqueued): VDN_ERR_INVALID_ARG (a NULL or misaligned pointer:
+ * 16 bytes for q, k, v, gate_lin, dy, dq, dk, dv, dgate_lin, fwd_init,
+ * dfwd_init; 4 for the others), VDN_ERR_UNSUPPORTED, VDN_ERR_WORKSPACE (either
+ * workspace missing, misaligned or too small); VDN_ERR_CUDA for a launch
+ * failure. */
+vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args, const vdn_lin_grads *grads,
+                              vdn_stream_t stream);
+
 /* ------------------------------------------------------- text cross-attention
  * The DiT block's softmax cross-attention from the video tokens to the text
  * tokens (PaperDaily digest section 三: text enters the block both through the

@@ -1,0 +1,178 @@
+"""GPU parity of the linear branch's backward (``vdn_hybrid_lin_bwd``, through
+the C ABI) against the float64 autograd oracle of that branch, on the same
+seeded inputs.
+
+Bar, per gradient: max |g_gpu - g_oracle| <= tol * RMS(g_oracle).  tol is
+1e-3 in fp32 mode: the backward runs two adjoint scans whose every step is a
+d x d fp32 product (rounding about d * 2^-24 per step) compounded over up to T
+frames, ten times the forward's fp32 bar.  In bf16-input mode both sides see
+the same bf16-rounded inputs and the backward computes in fp32, so the
+forward's bf16 bar (2e-2) is kept.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vdn_oracle as O
+from oracle import vdn_oracle_grad as OG
+from video_diffusion_hybrid_b200 import _lib as L
+from video_diffusion_hybrid_b200.api import HybridAttention, cfg_for, output_shape, to_torch
+from video_diffusion_hybrid_b200.build import build
+from video_diffusion_hybrid_b200.synth import Shape, bf16_round, bf16_to_f32, make_inputs
+
+pytestmark = pytest.mark.gpu
+TOL = {"f32": 1e-3, "bf16": 2e-2}
+NAMES = ("q", "k", "v", "beta", "alpha", "gate_lin", "rms_weight", "fwd_init")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built(cuda_ok):
+    build()
+
+
+def _ocfg(cfg: L.HybridCfg) -> O.Cfg:
+    return O.Cfg(B=cfg.B, T=cfg.T, N=cfg.N, H=cfg.H, d_k=cfg.d_k, d_v=cfg.d_v, L=cfg.L, chunk=cfg.chunk,
+                 anchors=cfg.anchors, rms_eps=cfg.rms_eps or 1e-6, out_mode=cfg.out_mode)
+
+
+def _dy(cfg: L.HybridCfg, seed: int) -> np.ndarray:
+    """A seeded upstream gradient in y's shape, rounded to y's dtype."""
+    dy = np.random.default_rng(seed).standard_normal(output_shape(cfg))
+    return bf16_to_f32(bf16_round(dy)).astype(np.float64) if cfg.y_dtype == L.VDN_BF16 else \
+        dy.astype(np.float32).astype(np.float64)
+
+
+def _lin_slot(cfg: L.HybridCfg, dy: np.ndarray) -> np.ndarray:
+    return dy[..., 1, :] if cfg.out_mode == 0 else dy
+
+
+def _rel(got, ref):
+    rms = np.sqrt(np.mean(ref ** 2))
+    err = np.max(np.abs(got - ref))
+    return float(err / rms) if rms > 0 else (0.0 if err == 0 else float("inf"))
+
+
+def _run(shape: Shape, dtype: str, seed: int, rms=True, fwd_init=False, **kw):
+    inp = make_inputs(shape, seed, dtype)
+    r = np.random.default_rng(seed + 7)
+    if rms:
+        inp["rms_weight"] = (1 + 0.3 * r.standard_normal((shape.H, shape.d_v))).astype(np.float32).astype(np.float64)
+    if fwd_init:
+        inp["fwd_init"] = (0.3 * r.standard_normal((shape.B, shape.H, shape.d_v, shape.d_k))).astype(
+            np.float32).astype(np.float64)
+    cfg = cfg_for(shape, dtype, **kw)
+    t = to_torch(inp, dtype, "cuda")
+    ha = HybridAttention(cfg)
+    ha(t)
+    dy = _dy(cfg, seed + 11)
+    tdt = torch.bfloat16 if cfg.y_dtype == L.VDN_BF16 else torch.float32
+    dyt = torch.from_numpy(dy.astype(np.float32)).to(tdt).cuda()
+    g = ha.linear_backward(t, dyt, want_rms=True, want_fwd_init=True)
+    torch.cuda.synchronize()
+    ref = OG.linear_branch_grads(inp, _ocfg(cfg), _lin_slot(cfg, dy))
+    return cfg, g, ref
+
+
+CASES = [
+    # (shape, dtype, options): fp32 SIMT forward at d = 32 with text and anchors;
+    # d = 64 with a short last chunk, three token tiles (ragged), no anchors,
+    # summed output and no RMS weight; bf16 d = 128 (tensor-core forward, the
+    # B-form write slot) with a bf16 y and a carried forward state; bf16 d = 64
+    # (tensor-core Gram, C-form write slot); fp32 d = 128 with a forward state.
+    (Shape(B=1, T=12, N=37, H=2, d_k=32, d_v=32, L=3), "f32", dict()),
+    (Shape(B=1, T=23, N=70, H=2, d_k=64, d_v=64, L=5), "f32", dict(anchors=0, out_mode=1, rms=False)),
+    (Shape(B=1, T=12, N=40, H=2, d_k=128, d_v=128, L=8), "bf16", dict(y_dtype=L.VDN_BF16, fwd_init=True)),
+    (Shape(B=2, T=15, N=33, H=3, d_k=64, d_v=64, L=4), "bf16", dict()),
+    (Shape(B=1, T=10, N=20, H=1, d_k=128, d_v=128, L=0), "f32", dict(fwd_init=True)),
+]
+
+
+@pytest.mark.parametrize("shape,dtype,opts", CASES)
+def test_lin_bwd_matches_oracle(shape, dtype, opts):
+    opts = dict(opts)
+    rms, fwd = opts.pop("rms", True), opts.pop("fwd_init", False)
+    cfg, g, ref = _run(shape, dtype, seed=31, rms=rms, fwd_init=fwd, **opts)
+    errs = {}
+    for name in NAMES:
+        key = "d" + name if name != "gate_lin" else "dgate_lin"
+        if name not in ref:
+            continue
+        got = g[key].cpu().numpy().astype(np.float64)
+        errs[name] = _rel(got, ref[name])
+    print("relative errors:", {k: f"{v:.2e}" for k, v in errs.items()})
+    for name, e in errs.items():
+        assert e <= TOL[dtype], (name, e)
+    # anchor frames are not written: exact zeros
+    if cfg.anchors:
+        for key in ("dk", "dv", "dbeta"):
+            assert torch.all(g[key][:, 0] == 0) and torch.all(g[key][:, -1] == 0)
+        assert torch.all(g["dalpha"][:, 0] == 0) and torch.all(g["dalpha"][:, -1] == 0)
+
+
+def test_lin_bwd_rms_weight_gradient_at_ones():
+    """Without an RMS weight the call still returns the gradient at weight = 1,
+    which the oracle gives when it is handed explicit ones."""
+    shape = Shape(B=1, T=12, N=25, H=2, d_k=32, d_v=32, L=3)
+    inp = make_inputs(shape, 41, "f32")
+    cfg = cfg_for(shape, "f32")
+    t = to_torch(inp, "f32", "cuda")
+    ha = HybridAttention(cfg)
+    ha(t)
+    dy = _dy(cfg, 42)
+    g = ha.linear_backward(t, torch.from_numpy(dy.astype(np.float32)).cuda(), want_rms=True)
+    torch.cuda.synchronize()
+    inp1 = dict(inp)
+    inp1["rms_weight"] = np.ones((2, 32))
+    ref = OG.linear_branch_grads(inp1, _ocfg(cfg), dy[..., 1, :])
+    assert _rel(g["drms_weight"].cpu().numpy(), ref["rms_weight"]) <= TOL["f32"]
+    assert _rel(g["dq"].cpu().numpy(), ref["q"]) <= TOL["f32"]
+
+
+def test_lin_bwd_repeatable():
+    """Two backward calls on the same forward workspace give the same bits
+    (no state carried between calls, no atomics)."""
+    shape = Shape(B=1, T=12, N=40, H=2, d_k=128, d_v=128, L=8)
+    inp = make_inputs(shape, 51, "bf16")
+    cfg = cfg_for(shape, "bf16")
+    t = to_torch(inp, "bf16", "cuda")
+    ha = HybridAttention(cfg)
+    ha(t)
+    dyt = torch.from_numpy(_dy(cfg, 52).astype(np.float32)).cuda()
+    g1 = {k: v.clone() for k, v in ha.linear_backward(t, dyt, want_rms=True, want_fwd_init=True).items()}
+    g2 = ha.linear_backward(t, dyt, want_rms=True, want_fwd_init=True)
+    torch.cuda.synchronize()
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_lin_bwd_full_size_one_head():
+    """At the 768p size (B=1, T=90, N=1008, H=24, d=128, L=512, bf16, inputs
+    drawn on the device as the benchmark does): every gradient of one head
+    against the oracle run on that head alone (the heads of the linear branch
+    are independent)."""
+    from video_diffusion_hybrid_b200.synth import head_slice, make_inputs_torch
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    w = WORKLOADS["768p"]
+    s = w.shape
+    t = make_inputs_torch(s, w.seed, w.dtype, "cuda")
+    cfg = cfg_for(s, w.dtype)
+    ha = HybridAttention(cfg)
+    ha(t)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    dy = torch.randn(output_shape(cfg), generator=gen, device="cuda")
+    g = ha.linear_backward(t, dy)
+    torch.cuda.synchronize()
+    h = s.H - 1
+    inp = {k: v.astype(np.float64) for k, v in head_slice(t, 0, h).items()}
+    oc = O.Cfg(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=s.L)
+    ref = OG.linear_branch_grads(inp, oc, dy[0:1, :, :, h:h + 1, 1].double().cpu().numpy())
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("beta", "dbeta"), ("gate_lin", "dgate_lin")):
+        got = g[key][0:1, :, :, h:h + 1].double().cpu().numpy()
+        e = _rel(got, ref[name])
+        print(name, f"{e:.2e}")
+        assert e <= TOL["bf16"], (name, e)
+    e = _rel(g["dalpha"][0:1, :, h:h + 1].double().cpu().numpy(), ref["alpha"])
+    assert e <= TOL["bf16"], ("alpha", e)
+    del t, g, ha, dy
+    torch.cuda.empty_cache()

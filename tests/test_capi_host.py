@@ -189,3 +189,48 @@ def test_fp8_entries_reject_bad_args():
     assert L.vdn_quantize_fp8(None, L.VDN_F32, 16, p, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
     assert L.vdn_out_proj_fp8(8, 24, 32, 0, p, p, p, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
     assert L.vdn_out_proj_fp8(8, 32, 32, 0, p, p, None, p, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+
+
+def test_lin_bwd_workspace_size():
+    """Every state of both scans ([B,H,T+1,d,d] twice), three d x d matrices
+    per frame-head and the RMS partials, each region 256-byte aligned."""
+    cfg = _cfg()
+    dd = 128 * 128 * 4
+    want = 2 * 24 * 91 * dd + 3 * 90 * 24 * dd + 90 * 24 * 128 * 4
+    assert L.vdn_hybrid_lin_bwd_workspace_size(cfg) == want
+    for kw in (dict(update=1), dict(update=2), dict(d_k=256, d_v=256), dict(T=1)):
+        assert L.vdn_hybrid_lin_bwd_workspace_size(_cfg(**kw)) == 0
+
+
+def _fake_grads(cfg, **over):
+    p = 1 << 26
+    g = dict(dy=p, dq=p, dk=p, dv=p, dbeta=p, dalpha=p, dgate_lin=p, workspace=p,
+             workspace_bytes=L.vdn_hybrid_lin_bwd_workspace_size(cfg))
+    g.update(over)
+    return L.make_lin_grads(**g)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(dy=None), L.VDN_ERR_INVALID_ARG), (dict(dq=(1 << 26) + 4), L.VDN_ERR_INVALID_ARG),
+    (dict(dbeta=None), L.VDN_ERR_INVALID_ARG), (dict(dalpha=(1 << 26) + 2), L.VDN_ERR_INVALID_ARG),
+    (dict(dfwd_init=(1 << 26) + 4), L.VDN_ERR_INVALID_ARG), (dict(workspace=None), L.VDN_ERR_WORKSPACE),
+    (dict(workspace=(1 << 26) + 64), L.VDN_ERR_WORKSPACE), (dict(workspace_bytes=4096), L.VDN_ERR_WORKSPACE),
+])
+def test_lin_bwd_bad_grads_rejected_before_launch(over, status):
+    cfg = _cfg()
+    assert L.vdn_hybrid_lin_bwd(cfg, _fake_args(cfg), _fake_grads(cfg, **over), stream=0, check=False) == status
+
+
+def test_lin_bwd_bad_config_and_forward_workspace_rejected():
+    cfg = _cfg()
+    assert L.vdn_hybrid_lin_bwd(cfg, _fake_args(cfg, workspace_bytes=1024), _fake_grads(cfg), stream=0,
+                                check=False) == L.VDN_ERR_WORKSPACE
+    assert L.vdn_hybrid_lin_bwd(cfg, _fake_args(cfg, gate_lin=None), _fake_grads(cfg), stream=0,
+                                check=False) == L.VDN_ERR_INVALID_ARG
+    for kw in (dict(update=1), dict(d_k=256, d_v=256)):
+        c = _cfg(**kw)
+        assert L.vdn_hybrid_lin_bwd(c, _fake_args(c), _fake_grads(cfg), stream=0, check=False) == \
+            L.VDN_ERR_UNSUPPORTED
+    lib = L.lib()
+    c = cfg.c()
+    assert lib.vdn_hybrid_lin_bwd(C.byref(c), None, None, None) == L.VDN_ERR_INVALID_ARG

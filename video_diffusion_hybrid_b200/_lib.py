@@ -23,7 +23,7 @@ STAGE_ALL = 31
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
             "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn",
-            "vdn_quantize_fp8", "vdn_out_proj_fp8")
+            "vdn_quantize_fp8", "vdn_out_proj_fp8", "vdn_hybrid_lin_bwd_workspace_size", "vdn_hybrid_lin_bwd")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -41,6 +41,14 @@ class VdnArgs(C.Structure):
                 ("text_k", C.c_void_p), ("text_v", C.c_void_p), ("text_beta", C.c_void_p),
                 ("init_state", C.c_void_p), ("rms_weight", C.c_void_p), ("y", C.c_void_p),
                 ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t), ("fwd_init", C.c_void_p)]
+
+
+class VdnLinGrads(C.Structure):
+    """Mirror of ``vdn_lin_grads``."""
+    _fields_ = [("dy", C.c_void_p), ("dq", C.c_void_p), ("dk", C.c_void_p), ("dv", C.c_void_p),
+                ("dbeta", C.c_void_p), ("dalpha", C.c_void_p), ("dgate_lin", C.c_void_p),
+                ("drms_weight", C.c_void_p), ("dfwd_init", C.c_void_p), ("workspace", C.c_void_p),
+                ("workspace_bytes", C.c_size_t)]
 
 
 class ProjCfg(C.Structure):
@@ -123,6 +131,10 @@ def lib() -> C.CDLL:
                                        C.c_void_p]
         L.vdn_out_proj.restype = C.c_int
         L.vdn_out_proj.argtypes = [C.POINTER(ProjCfg), C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]
+        L.vdn_hybrid_lin_bwd_workspace_size.restype = C.c_size_t
+        L.vdn_hybrid_lin_bwd_workspace_size.argtypes = [C.POINTER(VdnCfg)]
+        L.vdn_hybrid_lin_bwd.restype = C.c_int
+        L.vdn_hybrid_lin_bwd.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.POINTER(VdnLinGrads), C.c_void_p]
         L.vdn_status_string.restype = C.c_char_p
         L.vdn_status_string.argtypes = [C.c_int]
         _lib = L
@@ -245,4 +257,27 @@ def vdn_hybrid_attn_fwd_noalloc(cfg: HybridCfg, args: VdnArgs, stream=None, chec
     st = lib().vdn_hybrid_attn_fwd_noalloc(C.byref(c), C.byref(args), _stream_handle(stream))
     if check and st != VDN_OK:
         raise VdnError(st, "vdn_hybrid_attn_fwd_noalloc")
+    return st
+
+
+def vdn_hybrid_lin_bwd_workspace_size(cfg: HybridCfg) -> int:
+    c = cfg.c()
+    return int(lib().vdn_hybrid_lin_bwd_workspace_size(C.byref(c)))
+
+
+def make_lin_grads(dy, dq, dk, dv, dbeta, dalpha, dgate_lin, workspace, workspace_bytes=None, drms_weight=None,
+                   dfwd_init=None) -> VdnLinGrads:
+    """Build a ``vdn_lin_grads`` from torch tensors (or raw device pointers)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return VdnLinGrads(_ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dalpha), _ptr(dgate_lin),
+                       _ptr(drms_weight), _ptr(dfwd_init), _ptr(workspace), int(workspace_bytes))
+
+
+def vdn_hybrid_lin_bwd(cfg: HybridCfg, args: VdnArgs, grads: VdnLinGrads, stream=None, check: bool = True) -> int:
+    """Backward of the linear branch; args.workspace holds the forward's."""
+    c = cfg.c()
+    st = lib().vdn_hybrid_lin_bwd(C.byref(c), C.byref(args), C.byref(grads), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_hybrid_lin_bwd")
     return st

@@ -72,6 +72,31 @@ class HybridAttention:
             L.vdn_hybrid_attn_fwd_stages(self.cfg, a, stages, stream)
         return self.y
 
+    def linear_backward(self, t: dict, dy: torch.Tensor, want_rms: bool = False, want_fwd_init: bool = False,
+                        stream=None) -> dict:
+        """Gradients through the linear branch after a forward call on the same
+        inputs `t` (the forward's workspace is read): dy has y's shape and
+        dtype.  Returns float32 tensors dq, dk, dv, dbeta, dalpha, dgate_lin
+        (and drms_weight, dfwd_init when asked)."""
+        c = self.cfg
+        if getattr(self, "bwd_workspace", None) is None:
+            nb = L.vdn_hybrid_lin_bwd_workspace_size(c)
+            if nb == 0:
+                raise L.VdnError(L.VDN_ERR_UNSUPPORTED, "vdn_hybrid_lin_bwd_workspace_size")
+            self.bwd_workspace = torch.empty(nb, dtype=torch.uint8, device=self.device)
+        f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=self.device)
+        tok = (c.B, c.T, c.N, c.H)
+        g = {"dq": f(*tok, c.d_k), "dk": f(*tok, c.d_k), "dv": f(*tok, c.d_v), "dbeta": f(*tok),
+             "dalpha": f(c.B, c.T, c.H), "dgate_lin": f(*tok, c.d_v)}
+        if want_rms:
+            g["drms_weight"] = f(c.H, c.d_v)
+        if want_fwd_init:
+            g["dfwd_init"] = f(c.B, c.H, c.d_v, c.d_k)
+        lg = L.make_lin_grads(dy, g["dq"], g["dk"], g["dv"], g["dbeta"], g["dalpha"], g["dgate_lin"],
+                              self.bwd_workspace, drms_weight=g.get("drms_weight"), dfwd_init=g.get("dfwd_init"))
+        L.vdn_hybrid_lin_bwd(c, self.args(t), lg, stream)
+        return g
+
     def intermediates(self) -> dict:
         """Views of the workspace's intermediate values (float32)."""
         lay = L.vdn_hybrid_workspace_layout(self.cfg)

@@ -143,6 +143,14 @@ Inputs inputs_of(const vdn_hybrid_args* a) {
   return in;
 }
 
+// the backward covers the joint solve's write at d <= 128
+vdn_status check_bwd_cfg(const vdn_hybrid_cfg* c) {
+  vdn_status st = check_cfg(c);
+  if (st != VDN_OK) return st;
+  if (c->update != 0 || c->d_k > 128) return VDN_ERR_UNSUPPORTED;
+  return VDN_OK;
+}
+
 }  // namespace
 }  // namespace vdn
 
@@ -281,6 +289,43 @@ vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg* cfg, const vdn_hybrid_
   if (cudaStreamSynchronize(s) != cudaSuccess) return VDN_ERR_CUDA;
   if (where) *where = host[1];
   return host[0] ? VDN_ERR_TIMEOUT : VDN_OK;
+}
+
+size_t vdn_hybrid_lin_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {
+  if (check_bwd_cfg(cfg) != VDN_OK) return 0;
+  return lin_bwd_workspace(make_dims(cfg), nullptr);
+}
+
+vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_lin_grads* g,
+                              vdn_stream_t stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!args || !g) return VDN_ERR_INVALID_ARG;
+  const void* req[] = {args->q, args->k, args->v, args->gate_lin, g->dy, g->dq, g->dk, g->dv, g->dgate_lin};
+  for (const void* p : req)
+    if (!p || !aligned(p, 16)) return VDN_ERR_INVALID_ARG;
+  if (!args->beta || !args->alpha || !g->dbeta || !g->dalpha) return VDN_ERR_INVALID_ARG;
+  if (!aligned(args->beta, 4) || !aligned(args->alpha, 4) || !aligned(g->dbeta, 4) || !aligned(g->dalpha, 4))
+    return VDN_ERR_INVALID_ARG;
+  if (args->rms_weight && !aligned(args->rms_weight, 4)) return VDN_ERR_INVALID_ARG;
+  if (args->fwd_init && !aligned(args->fwd_init, 16)) return VDN_ERR_INVALID_ARG;
+  if ((g->drms_weight && !aligned(g->drms_weight, 4)) || (g->dfwd_init && !aligned(g->dfwd_init, 16)))
+    return VDN_ERR_INVALID_ARG;
+  vdn_workspace_layout L;
+  layout_of(cfg, &L);
+  if (!args->workspace || !aligned(args->workspace, kAlign) || args->workspace_bytes < L.total)
+    return VDN_ERR_WORKSPACE;
+  const Dims d = make_dims(cfg);
+  if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < lin_bwd_workspace(d, nullptr))
+    return VDN_ERR_WORKSPACE;
+  Work w = work_of(cfg, args);
+  // the forward's choice of write form (B_t or C_t in the C_t slot)
+  w.bform = (scan_tc_supported(d) && w.M16 != nullptr) ? 1 : 0;
+  LinBwdArgs a{g->dy, g->dq, g->dk, g->dv, g->dbeta, g->dalpha, g->dgate_lin, g->drms_weight, g->dfwd_init,
+               g->workspace};
+  return launch_lin_bwd(d, inputs_of(args), w, a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? VDN_OK
+             : VDN_ERR_CUDA;
 }
 
 vdn_status vdn_text_cross_attn(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, vdn_stream_t stream) {

@@ -102,4 +102,15 @@ inline bool use_chunk_scan(const Dims& d, int sms) {
 }
 cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void* r16, cudaStream_t s);
 
+// Backward of the linear branch (vdn_lin_bwd.cu): outputs and scratch
+struct LinBwdArgs {
+  const void* dy;  // gradient of y, y's layout and dtype (the linear slot is read)
+  float *dq, *dk, *dv, *dbeta, *dalpha, *dgate, *drms, *dfwd;  // drms, dfwd may be null
+  void* workspace;
+};
+// bytes of the backward's scratch; off[0..5] (if not null) get the offsets of
+// the all-frame states F, G, the per-frame dR, dXf, dXb and the RMS partials
+size_t lin_bwd_workspace(const Dims& d, size_t* off);
+cudaError_t launch_lin_bwd(const Dims& d, const Inputs& in, const Work& w, const LinBwdArgs& a, cudaStream_t s);
+
 }  // namespace vdn
