@@ -1,4 +1,5 @@
-"""Gradients of the linear (Video Delta Attention) branch of the hybrid core.
+"""Gradients of the two branches of the hybrid core: the linear (Video Delta
+Attention) branch and, at the end of this file, the windowed softmax branch.
 
 TEST INFRASTRUCTURE ONLY, like ``vdn_oracle``: only the test suite may import
 it.  The pages describe the forward pass only; the gradient of that forward is
@@ -107,3 +108,61 @@ def linear_branch_forward(inp: dict, cfg: O.Cfg) -> np.ndarray:
     x = {n: torch.from_numpy(np.asarray(inp[n], np.float64)) for n in GRAD_INPUTS if inp.get(n) is not None}
     with torch.no_grad():
         return linear_branch(x, cfg, starts).numpy()
+
+
+# ---------------------------------------------------------------------------
+# The softmax branch: y_sm = sigmoid(g_sm) * softmax(s q K^T over the allowed
+# keys) V, the allowed keys being the query chunk and its two neighbours plus
+# the anchor frames, and every key for an anchor query frame ([P1] 二; [P4]
+# and [P5], the windowed softmax with first/last-frame anchors).
+# ---------------------------------------------------------------------------
+SM_INPUTS = ("q", "k", "v", "gate_sm")
+
+
+def _sm_frame(x: dict, cfg: O.Cfg, b: int, h: int, t: int, keys: np.ndarray) -> torch.Tensor:
+    """y_sm of query frame t of (b, h) over the key frames `keys` (in order)."""
+    N = cfg.N
+    K = x["k"][b, keys, :, h].reshape(len(keys) * N, -1)
+    V = x["v"][b, keys, :, h].reshape(len(keys) * N, -1)
+    P = torch.softmax(cfg.scale * (x["q"][b, t, :, h] @ K.T), dim=-1)
+    return torch.sigmoid(x["gate_sm"][b, t, :, h]) * (P @ V)
+
+
+def softmax_branch(x: dict, cfg: O.Cfg) -> torch.Tensor:
+    """y_sm [B, T, N, H, d_v]: every query frame over the key frames the
+    frame mask allows it."""
+    allowed = O.frame_mask(cfg.T, cfg.chunk, cfg.anchors)
+    out = []
+    for b in range(cfg.B):
+        heads = []
+        for h in range(cfg.H):
+            heads.append(torch.stack([_sm_frame(x, cfg, b, h, t, np.flatnonzero(allowed[t]))
+                                      for t in range(cfg.T)]))
+        out.append(torch.stack(heads, dim=2))
+    return torch.stack(out)
+
+
+def _sm_leaves(inp: dict) -> dict:
+    return {n: torch.tensor(np.asarray(inp[n], np.float64), requires_grad=True) for n in SM_INPUTS}
+
+
+def softmax_branch_grads(inp: dict, cfg: O.Cfg, dy: np.ndarray) -> dict:
+    """d<y_sm, dy> / d input for q, k, v, gate_sm (numpy float64)."""
+    x = _sm_leaves(inp)
+    y = softmax_branch(x, cfg)
+    (y * torch.from_numpy(np.asarray(dy, np.float64))).sum().backward()
+    return {n: t.grad.numpy() for n, t in x.items()}
+
+
+def softmax_branch_grads_frames(inp: dict, cfg: O.Cfg, dy: np.ndarray, b: int, h: int, frames) -> dict:
+    """The gradients of sum over the query frames `frames` of <y_sm(b, h, t),
+    dy[b, t, :, h]> for one (b, h), one query frame at a time (so that at full
+    size only one frame's score matrix is held).  With `frames` = every query
+    frame that sees key frame f, the rows of k and v of frame f are complete;
+    the rows of q and gate_sm of those query frames always are."""
+    allowed = O.frame_mask(cfg.T, cfg.chunk, cfg.anchors)
+    x = _sm_leaves(inp)
+    for t in frames:
+        y = _sm_frame(x, cfg, b, h, t, np.flatnonzero(allowed[t]))
+        (y * torch.from_numpy(np.asarray(dy[b, t, :, h], np.float64))).sum().backward()
+    return {n: (t.grad.numpy() if t.grad is not None else np.zeros(t.shape)) for n, t in x.items()}
