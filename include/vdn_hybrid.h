@@ -278,6 +278,36 @@ size_t vdn_hybrid_lin_bwd_workspace_size(const vdn_hybrid_cfg *cfg);
 vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args, const vdn_lin_grads *grads,
                               vdn_stream_t stream);
 
+/* ----------------------------------------------- backward of the softmax branch
+ * Gradients through the windowed softmax branch (defined at the top of this
+ * header: PaperDaily digest section 二, the anchors of the deepmagic post and
+ * the aimodeling news): given dy = dL/dy, the call writes dL/dq, dL/dk, dL/dv
+ * and dL/dgate_sm as far as they flow through y's SOFTMAX slot (out_mode 0:
+ * slot 0 of dy; out_mode 1: dy itself).  With vdn_hybrid_lin_bwd the two
+ * branches' shares of dq, dk and dv add up to the whole core's gradient.
+ * The exact derivative of the forward (the pages describe the forward only):
+ * the softmax statistics are recomputed, no forward workspace is read.
+ * Reads cfg (update 0 and d_k 32, 64 or 128, else VDN_ERR_UNSUPPORTED) and
+ * args q, k, v, gate_sm (the other pointers are ignored).  fp32 arithmetic
+ * (SIMT) for both input dtypes. */
+typedef struct {
+  const void *dy;      /* dL/dy in y's shape (per cfg.out_mode) and cfg.y_dtype; 16-byte aligned */
+  float *dq, *dk, *dv; /* [B,T,N,H,d] float32, overwritten                                     */
+  float *dgate_sm;     /* [B,T,N,H,d_v] float32, overwritten                                   */
+  void *workspace;     /* scratch: dO, log-sum-exp and <dO, o> per query row; 256-byte aligned  */
+  size_t workspace_bytes; /* >= vdn_hybrid_sm_bwd_workspace_size(cfg)                           */
+} vdn_sm_grads;
+
+/* Bytes of scratch for cfg ((d_v + 2) floats per query row and head, each
+ * region 256-byte aligned); 0 if cfg is invalid or not supported. */
+size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg *cfg);
+
+/* Enqueue the softmax branch's backward on `stream`.  Errors (nothing
+ * enqueued): VDN_ERR_INVALID_ARG (a NULL or a not 16-byte aligned pointer),
+ * VDN_ERR_UNSUPPORTED, VDN_ERR_WORKSPACE; VDN_ERR_CUDA for a launch failure. */
+vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args, const vdn_sm_grads *grads,
+                             vdn_stream_t stream);
+
 /* ------------------------------------------------------- text cross-attention
  * The DiT block's softmax cross-attention from the video tokens to the text
  * tokens (PaperDaily digest section 三: text enters the block both through the

@@ -1,6 +1,7 @@
-"""GPU parity of the linear branch's backward (``vdn_hybrid_lin_bwd``, through
-the C ABI) against the float64 autograd oracle of that branch, on the same
-seeded inputs.
+"""GPU parity of the core's backward through the C ABI: the linear branch
+(``vdn_hybrid_lin_bwd``) and the windowed softmax branch (``vdn_hybrid_sm_bwd``)
+against the float64 autograd oracles of those branches, on the same seeded
+inputs.
 
 Bar, per gradient: max |g_gpu - g_oracle| <= tol * RMS(g_oracle).  tol is
 1e-3 in fp32 mode: the backward runs two adjoint scans whose every step is a
@@ -32,7 +33,8 @@ def _built(cuda_ok):
 
 def _ocfg(cfg: L.HybridCfg) -> O.Cfg:
     return O.Cfg(B=cfg.B, T=cfg.T, N=cfg.N, H=cfg.H, d_k=cfg.d_k, d_v=cfg.d_v, L=cfg.L, chunk=cfg.chunk,
-                 anchors=cfg.anchors, rms_eps=cfg.rms_eps or 1e-6, out_mode=cfg.out_mode)
+                 anchors=cfg.anchors, rms_eps=cfg.rms_eps or 1e-6, out_mode=cfg.out_mode,
+                 softmax_scale=cfg.softmax_scale)
 
 
 def _dy(cfg: L.HybridCfg, seed: int) -> np.ndarray:
@@ -174,5 +176,97 @@ def test_lin_bwd_full_size_one_head():
         assert e <= TOL["bf16"], (name, e)
     e = _rel(g["dalpha"][0:1, :, h:h + 1].double().cpu().numpy(), ref["alpha"])
     assert e <= TOL["bf16"], ("alpha", e)
+    del t, g, ha, dy
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------ softmax branch
+SM_CASES = [
+    # fp32 d = 32 with anchors; fp32 d = 64 without anchors, a short last chunk,
+    # ragged 64-row tiles, summed output and a large scale (the max subtraction
+    # matters); bf16 d = 128 with a bf16 y; bf16 d = 64, two batch elements.
+    (Shape(B=1, T=12, N=37, H=2, d_k=32, d_v=32, L=0), "f32", dict()),
+    (Shape(B=1, T=23, N=70, H=2, d_k=64, d_v=64, L=0), "f32", dict(anchors=0, out_mode=1, softmax_scale=10.0)),
+    (Shape(B=1, T=12, N=40, H=2, d_k=128, d_v=128, L=0), "bf16", dict(y_dtype=L.VDN_BF16)),
+    (Shape(B=2, T=15, N=33, H=3, d_k=64, d_v=64, L=0), "bf16", dict()),
+]
+
+
+def _sm_slot(cfg, dy):
+    return dy[..., 0, :] if cfg.out_mode == 0 else dy
+
+
+@pytest.mark.parametrize("shape,dtype,opts", SM_CASES)
+def test_sm_bwd_matches_oracle(shape, dtype, opts):
+    inp = make_inputs(shape, 61, dtype)
+    cfg = cfg_for(shape, dtype, **opts)
+    t = to_torch(inp, dtype, "cuda")
+    ha = HybridAttention(cfg)
+    dy = _dy(cfg, 62)
+    tdt = torch.bfloat16 if cfg.y_dtype == L.VDN_BF16 else torch.float32
+    g = ha.softmax_backward(t, torch.from_numpy(dy.astype(np.float32)).to(tdt).cuda())
+    torch.cuda.synchronize()
+    ref = OG.softmax_branch_grads(inp, _ocfg(cfg), _sm_slot(cfg, dy))
+    errs = {n: _rel(g["d" + n].cpu().numpy().astype(np.float64), ref[n]) for n in ("q", "k", "v", "gate_sm")}
+    print("relative errors:", {k: f"{v:.2e}" for k, v in errs.items()})
+    for n, e in errs.items():
+        assert e <= TOL[dtype], (n, e)
+
+
+def test_whole_core_backward_is_the_sum_of_the_branches():
+    """HybridAttention.backward: dq, dk, dv of the core equal the two oracles'
+    branch gradients added; the gate gradients are each branch's own."""
+    shape = Shape(B=1, T=12, N=30, H=2, d_k=64, d_v=64, L=4)
+    inp = make_inputs(shape, 71, "f32")
+    cfg = cfg_for(shape, "f32")
+    t = to_torch(inp, "f32", "cuda")
+    ha = HybridAttention(cfg)
+    ha(t)
+    dy = _dy(cfg, 72)
+    g = ha.backward(t, torch.from_numpy(dy.astype(np.float32)).cuda())
+    torch.cuda.synchronize()
+    oc = _ocfg(cfg)
+    rl = OG.linear_branch_grads(inp, oc, dy[..., 1, :])
+    rs = OG.softmax_branch_grads(inp, oc, dy[..., 0, :])
+    for n in ("q", "k", "v"):
+        assert _rel(g["d" + n].cpu().numpy(), rl[n] + rs[n]) <= TOL["f32"], n
+    assert _rel(g["dgate_sm"].cpu().numpy(), rs["gate_sm"]) <= TOL["f32"]
+    assert _rel(g["dgate_lin"].cpu().numpy(), rl["gate_lin"]) <= TOL["f32"]
+    assert _rel(g["dbeta"].cpu().numpy(), rl["beta"]) <= TOL["f32"]
+
+
+def test_sm_bwd_full_size_one_key_frame():
+    """At the 768p size (inputs drawn on the device): for one head and key
+    frame f = 47, the oracle, one query frame at a time, over every query frame
+    that sees f (its chunk and the two neighbours, and the two anchor frames,
+    which see every key): dk, dv of frame f's tokens and dq, dgate_sm of those
+    query frames."""
+    from video_diffusion_hybrid_b200.synth import head_slice, make_inputs_torch
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    w = WORKLOADS["768p"]
+    s = w.shape
+    t = make_inputs_torch(s, w.seed, w.dtype, "cuda")
+    cfg = cfg_for(s, w.dtype)
+    ha = HybridAttention(cfg)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(6)
+    dy = torch.randn(output_shape(cfg), generator=gen, device="cuda")
+    g = ha.softmax_backward(t, dy)
+    torch.cuda.synchronize()
+    h, f = 3, 47
+    frames = np.flatnonzero(O.frame_mask(s.T, 5, 4)[f])
+    inp = {k: v.astype(np.float64) for k, v in head_slice(t, 0, h).items()}
+    oc = O.Cfg(B=1, T=s.T, N=s.N, H=1, d_k=s.d_k, d_v=s.d_v, L=0)
+    dyh = dy[0:1, :, :, h:h + 1, 0].double().cpu().numpy()
+    ref = OG.softmax_branch_grads_frames(inp, oc, dyh, 0, 0, frames)
+    pick = lambda key, fr: g[key][0:1, fr, :, h:h + 1].double().cpu().numpy()
+    for n in ("k", "v"):
+        e = _rel(pick("d" + n, [f]), ref[n][:, [f]])
+        print(n, f"{e:.2e}")
+        assert e <= TOL["bf16"], (n, e)
+    for n in ("q", "gate_sm"):
+        e = _rel(pick("d" + n, frames), ref[n][:, frames])
+        print(n, f"{e:.2e}")
+        assert e <= TOL["bf16"], (n, e)
     del t, g, ha, dy
     torch.cuda.empty_cache()

@@ -234,3 +234,22 @@ def test_lin_bwd_bad_config_and_forward_workspace_rejected():
     lib = L.lib()
     c = cfg.c()
     assert lib.vdn_hybrid_lin_bwd(C.byref(c), None, None, None) == L.VDN_ERR_INVALID_ARG
+
+
+def test_sm_bwd_workspace_and_rejections():
+    cfg = _cfg()
+    rows = 90 * 1008 * 24
+    assert L.vdn_hybrid_sm_bwd_workspace_size(cfg) == rows * 128 * 4 + 2 * ((rows * 4 + 255) // 256 * 256)
+    for kw in (dict(update=1), dict(d_k=256, d_v=256)):
+        assert L.vdn_hybrid_sm_bwd_workspace_size(_cfg(**kw)) == 0
+    p = 1 << 26
+    good = dict(dy=p, dq=p, dk=p, dv=p, dgate_sm=p, workspace=p, workspace_bytes=L.vdn_hybrid_sm_bwd_workspace_size(cfg))
+    for over, status in ((dict(dy=None), L.VDN_ERR_INVALID_ARG), (dict(dgate_sm=p + 8), L.VDN_ERR_INVALID_ARG),
+                         (dict(workspace=None), L.VDN_ERR_WORKSPACE), (dict(workspace_bytes=64), L.VDN_ERR_WORKSPACE)):
+        g = L.make_sm_grads(**{**good, **over})
+        assert L.vdn_hybrid_sm_bwd(cfg, _fake_args(cfg), g, stream=0, check=False) == status
+    assert L.vdn_hybrid_sm_bwd(cfg, _fake_args(cfg, gate_sm=None), L.make_sm_grads(**good), stream=0,
+                               check=False) == L.VDN_ERR_INVALID_ARG
+    c = _cfg(update=2)
+    assert L.vdn_hybrid_sm_bwd(c, _fake_args(c), L.make_sm_grads(**good), stream=0, check=False) == \
+        L.VDN_ERR_UNSUPPORTED

@@ -23,7 +23,8 @@ STAGE_ALL = 31
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
             "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn",
-            "vdn_quantize_fp8", "vdn_out_proj_fp8", "vdn_hybrid_lin_bwd_workspace_size", "vdn_hybrid_lin_bwd")
+            "vdn_quantize_fp8", "vdn_out_proj_fp8", "vdn_hybrid_lin_bwd_workspace_size", "vdn_hybrid_lin_bwd",
+            "vdn_hybrid_sm_bwd_workspace_size", "vdn_hybrid_sm_bwd")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -49,6 +50,12 @@ class VdnLinGrads(C.Structure):
                 ("dbeta", C.c_void_p), ("dalpha", C.c_void_p), ("dgate_lin", C.c_void_p),
                 ("drms_weight", C.c_void_p), ("dfwd_init", C.c_void_p), ("workspace", C.c_void_p),
                 ("workspace_bytes", C.c_size_t)]
+
+
+class VdnSmGrads(C.Structure):
+    """Mirror of ``vdn_sm_grads``."""
+    _fields_ = [("dy", C.c_void_p), ("dq", C.c_void_p), ("dk", C.c_void_p), ("dv", C.c_void_p),
+                ("dgate_sm", C.c_void_p), ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t)]
 
 
 class ProjCfg(C.Structure):
@@ -135,6 +142,10 @@ def lib() -> C.CDLL:
         L.vdn_hybrid_lin_bwd_workspace_size.argtypes = [C.POINTER(VdnCfg)]
         L.vdn_hybrid_lin_bwd.restype = C.c_int
         L.vdn_hybrid_lin_bwd.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.POINTER(VdnLinGrads), C.c_void_p]
+        L.vdn_hybrid_sm_bwd_workspace_size.restype = C.c_size_t
+        L.vdn_hybrid_sm_bwd_workspace_size.argtypes = [C.POINTER(VdnCfg)]
+        L.vdn_hybrid_sm_bwd.restype = C.c_int
+        L.vdn_hybrid_sm_bwd.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.POINTER(VdnSmGrads), C.c_void_p]
         L.vdn_status_string.restype = C.c_char_p
         L.vdn_status_string.argtypes = [C.c_int]
         _lib = L
@@ -280,4 +291,25 @@ def vdn_hybrid_lin_bwd(cfg: HybridCfg, args: VdnArgs, grads: VdnLinGrads, stream
     st = lib().vdn_hybrid_lin_bwd(C.byref(c), C.byref(args), C.byref(grads), _stream_handle(stream))
     if check and st != VDN_OK:
         raise VdnError(st, "vdn_hybrid_lin_bwd")
+    return st
+
+
+def vdn_hybrid_sm_bwd_workspace_size(cfg: HybridCfg) -> int:
+    c = cfg.c()
+    return int(lib().vdn_hybrid_sm_bwd_workspace_size(C.byref(c)))
+
+
+def make_sm_grads(dy, dq, dk, dv, dgate_sm, workspace, workspace_bytes=None) -> VdnSmGrads:
+    """Build a ``vdn_sm_grads`` from torch tensors (or raw device pointers)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return VdnSmGrads(_ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate_sm), _ptr(workspace), int(workspace_bytes))
+
+
+def vdn_hybrid_sm_bwd(cfg: HybridCfg, args: VdnArgs, grads: VdnSmGrads, stream=None, check: bool = True) -> int:
+    """Backward of the windowed softmax branch (recomputes its statistics)."""
+    c = cfg.c()
+    st = lib().vdn_hybrid_sm_bwd(C.byref(c), C.byref(args), C.byref(grads), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_hybrid_sm_bwd")
     return st

@@ -97,6 +97,35 @@ class HybridAttention:
         L.vdn_hybrid_lin_bwd(c, self.args(t), lg, stream)
         return g
 
+    def softmax_backward(self, t: dict, dy: torch.Tensor, stream=None) -> dict:
+        """Gradients through the windowed softmax branch (no forward state is
+        needed): float32 tensors dq, dk, dv, dgate_sm."""
+        c = self.cfg
+        if getattr(self, "sm_workspace", None) is None:
+            nb = L.vdn_hybrid_sm_bwd_workspace_size(c)
+            if nb == 0:
+                raise L.VdnError(L.VDN_ERR_UNSUPPORTED, "vdn_hybrid_sm_bwd_workspace_size")
+            self.sm_workspace = torch.empty(nb, dtype=torch.uint8, device=self.device)
+        f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=self.device)
+        tok = (c.B, c.T, c.N, c.H)
+        g = {"dq": f(*tok, c.d_k), "dk": f(*tok, c.d_k), "dv": f(*tok, c.d_v), "dgate_sm": f(*tok, c.d_v)}
+        sg = L.make_sm_grads(dy, g["dq"], g["dk"], g["dv"], g["dgate_sm"], self.sm_workspace)
+        L.vdn_hybrid_sm_bwd(c, self.args(t), sg, stream)
+        return g
+
+    def backward(self, t: dict, dy: torch.Tensor, stream=None) -> dict:
+        """The whole core's gradients after a forward call on the same inputs:
+        both branches' shares of dq, dk, dv summed (one elementwise torch add
+        each, on the same stream), and the branch-specific gradients."""
+        lin = self.linear_backward(t, dy, want_rms=t.get("rms_weight") is not None,
+                                   want_fwd_init=t.get("fwd_init") is not None, stream=stream)
+        sm = self.softmax_backward(t, dy, stream=stream)
+        out = dict(lin)
+        for k in ("dq", "dk", "dv"):
+            out[k] = lin[k] + sm[k]
+        out["dgate_sm"] = sm["dgate_sm"]
+        return out
+
     def intermediates(self) -> dict:
         """Views of the workspace's intermediate values (float32)."""
         lay = L.vdn_hybrid_workspace_layout(self.cfg)

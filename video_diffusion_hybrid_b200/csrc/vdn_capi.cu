@@ -328,6 +328,29 @@ vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* 
              : VDN_ERR_CUDA;
 }
 
+size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {
+  if (check_bwd_cfg(cfg) != VDN_OK) return 0;
+  return sm_bwd_workspace(make_dims(cfg), nullptr);
+}
+
+vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_sm_grads* g,
+                             vdn_stream_t stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!args || !g) return VDN_ERR_INVALID_ARG;
+  const void* req[] = {args->q, args->k, args->v, args->gate_sm, g->dy, g->dq, g->dk, g->dv, g->dgate_sm};
+  for (const void* p : req)
+    if (!p || !aligned(p, 16)) return VDN_ERR_INVALID_ARG;
+  const Dims d = make_dims(cfg);
+  if ((long long)d.T * d.N > (1LL << 40)) return VDN_ERR_UNSUPPORTED;
+  if ((d.N + 63) / 64 > 0x7FFFFFFF) return VDN_ERR_UNSUPPORTED;
+  if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < sm_bwd_workspace(d, nullptr))
+    return VDN_ERR_WORKSPACE;
+  SmBwdArgs a{g->dy, g->dq, g->dk, g->dv, g->dgate_sm, g->workspace};
+  return launch_sm_bwd(d, inputs_of(args), a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? VDN_OK
+                                                                                                  : VDN_ERR_CUDA;
+}
+
 vdn_status vdn_text_cross_attn(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, vdn_stream_t stream) {
   vdn_status st = check_cfg(cfg);
   if (st != VDN_OK) return st;

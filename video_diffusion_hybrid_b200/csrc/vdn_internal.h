@@ -113,4 +113,14 @@ struct LinBwdArgs {
 size_t lin_bwd_workspace(const Dims& d, size_t* off);
 cudaError_t launch_lin_bwd(const Dims& d, const Inputs& in, const Work& w, const LinBwdArgs& a, cudaStream_t s);
 
+// Backward of the windowed softmax branch (vdn_sm_bwd.cu)
+struct SmBwdArgs {
+  const void* dy;  // gradient of y, y's layout and dtype (the softmax slot is read)
+  float *dq, *dk, *dv, *dgate;
+  void* workspace;
+};
+// bytes of its scratch (dO, LSE, Delta per query row); off[0..2] the offsets
+size_t sm_bwd_workspace(const Dims& d, size_t* off);
+cudaError_t launch_sm_bwd(const Dims& d, const Inputs& in, const SmBwdArgs& a, cudaStream_t s);
+
 }  // namespace vdn
