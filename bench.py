@@ -628,10 +628,12 @@ def bwd_work(s, bf16: bool):
 
 
 def run_bwd(args):
-    """The linear branch's backward at the workload's size: one forward
-    (which leaves M_t and the write matrices in the workspace), then the timed
-    backward calls, each giving every gradient of q, k, v, beta, alpha,
-    gate_lin and the RMS weight for a fixed upstream gradient dy."""
+    """The core's backward at the workload's size: one forward (which leaves
+    M_t and the write matrices in the workspace), then the timed steps, each
+    one call of each branch's backward for a fixed upstream gradient dy: the
+    linear branch (gradients of q, k, v, beta, alpha, gate_lin, the RMS weight)
+    and the windowed softmax branch (q, k, v, gate_sm).  Each branch is timed
+    with CUDA events of its own on the launching stream."""
     import torch
     from video_diffusion_hybrid_b200 import _lib as L
     from video_diffusion_hybrid_b200.api import HybridAttention, cfg_for, output_shape
@@ -648,35 +650,57 @@ def run_bwd(args):
     g = ha.linear_backward(t, dy, want_rms=True)
     lg = L.make_lin_grads(dy, g["dq"], g["dk"], g["dv"], g["dbeta"], g["dalpha"], g["dgate_lin"],
                           ha.bwd_workspace, drms_weight=g["drms_weight"])
+    gs = ha.softmax_backward(t, dy)
+    sg = L.make_sm_grads(dy, gs["dq"], gs["dk"], gs["dv"], gs["dgate_sm"], ha.sm_workspace)
     a = ha.args(t)
     for _ in range(max(args.warmup, 3)):
         L.vdn_hybrid_lin_bwd(cfg, a, lg)
+        L.vdn_hybrid_sm_bwd(cfg, a, sg)
     torch.cuda.synchronize()
     clk = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0])
     clk.start()
     stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
         L.vdn_hybrid_lin_bwd(cfg, a, lg)
-    e1.record(stream)
+        ev[2 * i + 1].record(stream)
+        L.vdn_hybrid_sm_bwd(cfg, a, sg)
+        ev[2 * i + 2].record(stream)
     torch.cuda.synchronize()
     clocks = clk.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    lin_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps)) / args.steps
+    sm_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(args.steps)) / args.steps
+    ms = lin_ms + sm_ms
     flops, byts = bwd_work(s, w.dtype == "bf16")
+    pairs = O_density(s) * (s.T * s.N) ** 2 * s.H * s.B
+    sm_flops = 10.0 * s.d_k * pairs  # s, dP, dq, dk, dv: 2 d flops each per allowed pair
     peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FMA lanes x 2 flops x max SM clock
-    tf = flops / (ms * 1e-3) / 1e12
+    tf = (flops + sm_flops) / (ms * 1e-3) / 1e12
     print(json.dumps({
-        "metric": "linear-branch backward", "value": w.tokens / (ms * 1e-3), "unit": "video tokens/s",
+        "metric": "hybrid-attn core backward", "value": w.tokens / (ms * 1e-3), "unit": "video tokens/s",
         "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "n_gpus": 1, "higher_is_better": True,
         "dtype": "f32" if w.dtype == "f32" else "bf16 in, f32 compute", "data": "synthetic",
         "config": {"workload": w.name, "B": s.B, "T": s.T, "N": s.N, "H": s.H, "d": s.d_k, "L": s.L,
                    "l2": "inputs larger than L2"},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": 8 * args.steps,
+        "branches": {
+            "linear": {"ms": lin_ms, "kernels": 6, "flops": flops, "hbm_bytes": byts,
+                       "tflops": flops / (lin_ms * 1e-3) / 1e12, "frac": flops / (lin_ms * 1e-3) / 1e12 / peak},
+            "softmax": {"ms": sm_ms, "kernels": 2, "flops": sm_flops, "pairs": pairs,
+                        "tflops": sm_flops / (sm_ms * 1e-3) / 1e12, "frac": sm_flops / (sm_ms * 1e-3) / 1e12 / peak}},
         "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                     "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1.965 GHz", "flops": flops,
-                     "hbm_gbs": byts / (ms * 1e-3) / 1e9},
+                     "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1.965 GHz (SIMT fp32)",
+                     "flops": flops + sm_flops},
         "clocks": clocks}), flush=True)
+
+
+def O_density(s) -> float:
+    """Fraction of (query, key) frame pairs the mask allows (chunk 5, anchors)."""
+    c = [t // 5 for t in range(s.T)]
+    anc = {0, s.T - 1}
+    n = sum(1 for a in range(s.T) for b in range(s.T) if abs(c[a] - c[b]) <= 1 or a in anc or b in anc)
+    return n / s.T ** 2
 
 
 def run_ulysses(args):
