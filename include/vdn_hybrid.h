@@ -139,7 +139,9 @@ enum {
   VDN_STAGE_SCAN = 4u,   /* forward/backward state scans -> chunk-boundary states     */
   VDN_STAGE_SOFTMAX = 8u,/* windowed softmax + gate -> y slot 0 (or y)                */
   VDN_STAGE_READ = 16u,  /* state read + RMSNorm + gate -> y slot 1 (or y += )        */
-  VDN_STAGE_ALL = 31u
+  VDN_STAGE_ALL = 31u,
+  VDN_STAGE_SOFTMAX_BWD = 32u /* not a forward stage: vdn_hybrid_stage_impl's key for the
+                                 softmax branch's backward (vdn_hybrid_sm_bwd)            */
 };
 
 /* Byte offsets of the intermediate values inside the workspace (float32
@@ -225,7 +227,8 @@ vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg *cfg, const vdn_hybrid_
 
 /* Which implementation a stage uses for cfg: 0 = SIMT fp32, 1 = tcgen05 tensor
  * cores (TMA + TMEM), 2 = the ablation variants' per-frame map kernel (SOLVE
- * with cfg.update != 0), -1 = stage not supported for cfg. */
+ * with cfg.update != 0), -1 = stage not supported for cfg.  Also answers for
+ * VDN_STAGE_SOFTMAX_BWD, the softmax branch's backward. */
 int vdn_hybrid_stage_impl(const vdn_hybrid_cfg *cfg, unsigned stage);
 
 /* Static description of a status code. */
@@ -285,26 +288,40 @@ vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *
  * and dL/dgate_sm as far as they flow through y's SOFTMAX slot (out_mode 0:
  * slot 0 of dy; out_mode 1: dy itself).  With vdn_hybrid_lin_bwd the two
  * branches' shares of dq, dk and dv add up to the whole core's gradient.
- * The exact derivative of the forward (the pages describe the forward only):
- * the softmax statistics are recomputed, no forward workspace is read.
+ * The exact derivative of the forward (the pages describe the forward only).
  * Reads cfg (update 0 and d_k 32, 64 or 128, else VDN_ERR_UNSUPPORTED) and
- * args q, k, v, gate_sm (the other pointers are ignored).  fp32 arithmetic
- * (SIMT) for both input dtypes. */
+ * args q, k, v, gate_sm (the other pointers, the forward's workspace and its
+ * output are not read: the softmax statistics and o are recomputed).  Two
+ * implementations, chosen by cfg (vdn_hybrid_stage_impl(cfg,
+ * VDN_STAGE_SOFTMAX_BWD) says which):
+ *   - tensor cores (tcgen05) when dtype is VDN_BF16 and d_k is 64 or 128: the
+ *     products take fp16 operands with fp32 accumulation.  q, k, v are copied
+ *     to fp16 exactly (their magnitudes must stay below 65504); P, dS and dO
+ *     are rounded to fp16, dO after scaling by one power of two per call (so
+ *     that small upstream gradients keep their precision).  The status words of
+ *     its bounded waits sit in the first 256 bytes of grads->workspace: read
+ *     them with vdn_hybrid_device_status called with args->workspace set to
+ *     grads->workspace;
+ *   - otherwise SIMT fp32. */
 typedef struct {
   const void *dy;      /* dL/dy in y's shape (per cfg.out_mode) and cfg.y_dtype; 16-byte aligned */
   float *dq, *dk, *dv; /* [B,T,N,H,d] float32, overwritten                                     */
   float *dgate_sm;     /* [B,T,N,H,d_v] float32, overwritten                                   */
-  void *workspace;     /* scratch: dO, log-sum-exp and <dO, o> per query row; 256-byte aligned  */
+  void *workspace;     /* scratch (status words, operand copies, dO, log-sum-exp and <dO, o> per
+                          query row); 256-byte aligned                                        */
   size_t workspace_bytes; /* >= vdn_hybrid_sm_bwd_workspace_size(cfg)                           */
 } vdn_sm_grads;
 
-/* Bytes of scratch for cfg ((d_v + 2) floats per query row and head, each
- * region 256-byte aligned); 0 if cfg is invalid or not supported. */
+/* Bytes of scratch for cfg (the larger of its two layouts: four fp16 rows of d and two
+ * floats per query row and head, plus 512 bytes, for the tensor cores; each
+ * region 256-byte aligned); 0 if cfg is invalid or
+ * not supported. */
 size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg *cfg);
 
 /* Enqueue the softmax branch's backward on `stream`.  Errors (nothing
  * enqueued): VDN_ERR_INVALID_ARG (a NULL or a not 16-byte aligned pointer),
- * VDN_ERR_UNSUPPORTED, VDN_ERR_WORKSPACE; VDN_ERR_CUDA for a launch failure. */
+ * VDN_ERR_UNSUPPORTED, VDN_ERR_WORKSPACE (grads->workspace missing,
+ * misaligned or too small); VDN_ERR_CUDA for a launch failure. */
 vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args, const vdn_sm_grads *grads,
                              vdn_stream_t stream);
 

@@ -182,13 +182,19 @@ def test_lin_bwd_full_size_one_head():
 
 # ------------------------------------------------------------ softmax branch
 SM_CASES = [
-    # fp32 d = 32 with anchors; fp32 d = 64 without anchors, a short last chunk,
-    # ragged 64-row tiles, summed output and a large scale (the max subtraction
-    # matters); bf16 d = 128 with a bf16 y; bf16 d = 64, two batch elements.
+    # SIMT fp32 path: fp32 d = 32 with anchors; fp32 d = 64 without anchors, a
+    # short last chunk, ragged 64-row tiles, summed output and a large scale
+    # (the max subtraction matters); bf16 d = 32 with a summed output.
+    # Tensor-core path (bf16, d = 64 or 128): d = 128 with a bf16 y; d = 64 with
+    # two batch elements; d = 128 with ragged 128-row tiles over several frames,
+    # no anchors and scale 10; d = 128 with N < 128 and a summed output.
     (Shape(B=1, T=12, N=37, H=2, d_k=32, d_v=32, L=0), "f32", dict()),
     (Shape(B=1, T=23, N=70, H=2, d_k=64, d_v=64, L=0), "f32", dict(anchors=0, out_mode=1, softmax_scale=10.0)),
+    (Shape(B=1, T=12, N=40, H=2, d_k=32, d_v=32, L=0), "bf16", dict(out_mode=1)),
     (Shape(B=1, T=12, N=40, H=2, d_k=128, d_v=128, L=0), "bf16", dict(y_dtype=L.VDN_BF16)),
     (Shape(B=2, T=15, N=33, H=3, d_k=64, d_v=64, L=0), "bf16", dict()),
+    (Shape(B=1, T=23, N=300, H=2, d_k=128, d_v=128, L=0), "bf16", dict(anchors=0, softmax_scale=10.0)),
+    (Shape(B=1, T=20, N=100, H=3, d_k=128, d_v=128, L=0), "bf16", dict(out_mode=1)),
 ]
 
 
@@ -202,10 +208,13 @@ def test_sm_bwd_matches_oracle(shape, dtype, opts):
     cfg = cfg_for(shape, dtype, **opts)
     t = to_torch(inp, dtype, "cuda")
     ha = HybridAttention(cfg)
+    tc = dtype == "bf16" and shape.d_k in (64, 128)
+    assert L.vdn_hybrid_stage_impl(cfg, L.STAGE_SOFTMAX_BWD) == (1 if tc else 0)
     dy = _dy(cfg, 62)
     tdt = torch.bfloat16 if cfg.y_dtype == L.VDN_BF16 else torch.float32
     g = ha.softmax_backward(t, torch.from_numpy(dy.astype(np.float32)).to(tdt).cuda())
     torch.cuda.synchronize()
+    assert ha.softmax_backward_status()[0] == L.VDN_OK
     ref = OG.softmax_branch_grads(inp, _ocfg(cfg), _sm_slot(cfg, dy))
     errs = {n: _rel(g["d" + n].cpu().numpy().astype(np.float64), ref[n]) for n in ("q", "k", "v", "gate_sm")}
     print("relative errors:", {k: f"{v:.2e}" for k, v in errs.items()})
@@ -251,8 +260,10 @@ def test_sm_bwd_full_size_one_key_frame():
     gen = torch.Generator(device="cuda")
     gen.manual_seed(6)
     dy = torch.randn(output_shape(cfg), generator=gen, device="cuda")
+    assert L.vdn_hybrid_stage_impl(cfg, L.STAGE_SOFTMAX_BWD) == 1
     g = ha.softmax_backward(t, dy)
     torch.cuda.synchronize()
+    assert ha.softmax_backward_status()[0] == L.VDN_OK
     h, f = 3, 47
     frames = np.flatnonzero(O.frame_mask(s.T, 5, 4)[f])
     inp = {k: v.astype(np.float64) for k, v in head_slice(t, 0, h).items()}

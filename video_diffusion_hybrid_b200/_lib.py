@@ -19,6 +19,7 @@ VDN_OK, VDN_ERR_INVALID_ARG, VDN_ERR_UNSUPPORTED, VDN_ERR_WORKSPACE, VDN_ERR_CUD
 VDN_F32, VDN_BF16 = 0, 1
 STAGE_TEXT, STAGE_SOLVE, STAGE_SCAN, STAGE_SOFTMAX, STAGE_READ = 1, 2, 4, 8, 16
 STAGE_ALL = 31
+STAGE_SOFTMAX_BWD = 32  # vdn_hybrid_stage_impl key of the softmax branch's backward
 
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",

@@ -99,7 +99,8 @@ class HybridAttention:
 
     def softmax_backward(self, t: dict, dy: torch.Tensor, stream=None) -> dict:
         """Gradients through the windowed softmax branch (no forward state is
-        needed): float32 tensors dq, dk, dv, dgate_sm."""
+        read; the statistics are recomputed): float32 tensors dq, dk, dv,
+        dgate_sm."""
         c = self.cfg
         if getattr(self, "sm_workspace", None) is None:
             nb = L.vdn_hybrid_sm_bwd_workspace_size(c)
@@ -112,6 +113,14 @@ class HybridAttention:
         sg = L.make_sm_grads(dy, g["dq"], g["dk"], g["dv"], g["dgate_sm"], self.sm_workspace)
         L.vdn_hybrid_sm_bwd(c, self.args(t), sg, stream)
         return g
+
+    def softmax_backward_status(self, stream=None) -> tuple:
+        """(status, kernel tag) of the last softmax backward's bounded waits,
+        from the status words at the head of its scratch."""
+        a = L.VdnArgs()
+        a.workspace = self.sm_workspace.data_ptr()
+        a.workspace_bytes = self.sm_workspace.numel()
+        return L.vdn_hybrid_device_status(self.cfg, a, stream)
 
     def backward(self, t: dict, dy: torch.Tensor, stream=None) -> dict:
         """The whole core's gradients after a forward call on the same inputs:

@@ -189,6 +189,9 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
     case VDN_STAGE_SOFTMAX:
       if (big_d(d)) return -1;
       return softmax_tc_supported(d) ? 1 : 0;
+    case VDN_STAGE_SOFTMAX_BWD:
+      if (check_bwd_cfg(cfg) != VDN_OK) return -1;
+      return sm_bwd_tc_supported(d) ? 1 : 0;
     default:
       return -1;
   }
@@ -330,7 +333,9 @@ vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* 
 
 size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {
   if (check_bwd_cfg(cfg) != VDN_OK) return 0;
-  return sm_bwd_workspace(make_dims(cfg), nullptr);
+  const Dims d = make_dims(cfg);
+  const size_t a = sm_bwd_workspace(d, nullptr), b = sm_bwd_tc_workspace(d, nullptr);
+  return a > b ? a : b;
 }
 
 vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_sm_grads* g,
@@ -343,12 +348,24 @@ vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* a
     if (!p || !aligned(p, 16)) return VDN_ERR_INVALID_ARG;
   const Dims d = make_dims(cfg);
   if ((long long)d.T * d.N > (1LL << 40)) return VDN_ERR_UNSUPPORTED;
-  if ((d.N + 63) / 64 > 0x7FFFFFFF) return VDN_ERR_UNSUPPORTED;
-  if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < sm_bwd_workspace(d, nullptr))
+  if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < vdn_hybrid_sm_bwd_workspace_size(cfg))
     return VDN_ERR_WORKSPACE;
-  SmBwdArgs a{g->dy, g->dq, g->dk, g->dv, g->dgate_sm, g->workspace};
-  return launch_sm_bwd(d, inputs_of(args), a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? VDN_OK
-                                                                                                  : VDN_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(g->workspace);
+  if (sm_bwd_tc_supported(d)) {
+    size_t off[8];
+    sm_bwd_tc_workspace(d, off);
+    SmTcArgs a{g->dy, g->dq, g->dk, g->dv, g->dgate_sm, base + off[1], base + off[2], base + off[3], base + off[4],
+               reinterpret_cast<float*>(base + off[5]), reinterpret_cast<float*>(base + off[6]),
+               reinterpret_cast<unsigned*>(base + off[7]), reinterpret_cast<uint32_t*>(base + off[0])};
+    if (cudaMemsetAsync(base + off[0], 0, kAlign, s) != cudaSuccess ||
+        cudaMemsetAsync(base + off[7], 0, kAlign, s) != cudaSuccess)
+      return VDN_ERR_CUDA;
+    return launch_sm_bwd_tc(d, inputs_of(args), a, s) == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+  }
+  if (cudaMemsetAsync(base, 0, kAlign, s) != cudaSuccess) return VDN_ERR_CUDA;  // no status on this path
+  SmBwdArgs a{g->dy, g->dq, g->dk, g->dv, g->dgate_sm, base + kAlign};
+  return launch_sm_bwd(d, inputs_of(args), a, s) == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
 }
 
 vdn_status vdn_text_cross_attn(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, vdn_stream_t stream) {

@@ -21,7 +21,7 @@ struct Dims {
 };
 
 // Device-side status words at the head of the workspace.
-enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4, TAG_COMPOSE_TC = 5 };
+enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4, TAG_COMPOSE_TC = 5, TAG_SMBWD_TC = 6 };
 
 struct Work {
   uint32_t* status;
@@ -122,5 +122,19 @@ struct SmBwdArgs {
 // bytes of its scratch (dO, LSE, Delta per query row); off[0..2] the offsets
 size_t sm_bwd_workspace(const Dims& d, size_t* off);
 cudaError_t launch_sm_bwd(const Dims& d, const Inputs& in, const SmBwdArgs& a, cudaStream_t s);
+// its tensor-core form (vdn_sm_bwd_tc.cu): bf16 inputs, d = 64 or 128; fp16
+// operands (exact copies of q, k, v; P, dS and a power-of-two scaled dO rounded)
+struct SmTcArgs {
+  const void* dy;
+  float *dq, *dk, *dv, *dgate;
+  void *q16, *k16, *v16, *dO16;  // [B*T*N, H, D] fp16 scratch
+  float *lse2, *delta;           // [B*T*N, H] scratch
+  unsigned* amax;                // max |dO| (cleared by the caller)
+  uint32_t* status;              // bounded-wait status words (cleared by the caller)
+};
+bool sm_bwd_tc_supported(const Dims& d);
+// bytes of its scratch; off[0..7] (if not null): status, q16, k16, v16, dO16, lse2, delta, amax
+size_t sm_bwd_tc_workspace(const Dims& d, size_t* off);
+cudaError_t launch_sm_bwd_tc(const Dims& d, const Inputs& in, const SmTcArgs& a, cudaStream_t s);
 
 }  // namespace vdn

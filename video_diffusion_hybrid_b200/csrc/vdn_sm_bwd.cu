@@ -373,6 +373,8 @@ cudaError_t launch_sm_d(const Dims& d, const Inputs& in, const SmBwdWork& ws, co
 
 }  // namespace
 
+// offsets relative to the scratch handed to launch_sm_bwd; the C ABI places
+// it after the 256-byte status region that heads the caller's workspace
 size_t sm_bwd_workspace(const Dims& d, size_t* off) {
   const size_t rows = (size_t)d.B * d.T * d.N * d.H;
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -382,7 +384,7 @@ size_t sm_bwd_workspace(const Dims& d, size_t* off) {
     if (off) off[i] = o;
     o += up(sizes[i]);
   }
-  return o;
+  return o + 256;
 }
 
 cudaError_t launch_sm_bwd(const Dims& d, const Inputs& in, const SmBwdArgs& a, cudaStream_t s) {

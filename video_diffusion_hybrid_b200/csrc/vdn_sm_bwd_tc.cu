@@ -1,0 +1,735 @@
+// Backward of the windowed softmax branch on the tensor cores (tcgen05):
+// fp16 operands, fp32 scores, statistics and accumulation.
+//
+// The forward (PaperDaily digest section 二; deepmagic post and aimodeling
+// news, the windowed softmax with first/last-frame anchors) gives, per query
+// row, y_sm = sigmoid(g) o with o = softmax(s q K^T) V over the keys its mask
+// allows.  With dy the gradient of y's softmax slot:
+//   dO = dy sigmoid(g),  Delta = <dO, o>,  dg = dy o sigmoid'(g)
+//   P = exp(s q k^T - LSE),  dS = P (dO v^T - Delta)
+//   dq = s dS K,  dk = s dS^T Q,  dv = P^T dO
+// the plain derivative of the forward (the pages describe the forward only).
+//
+// Operand precision.  The products take fp16 operands (11 significant bits):
+// q, k, v are converted exactly from bf16 (any |x| < 65504), and P, dS and dO
+// are rounded to fp16, which keeps the gradients within about 2e-3 of their
+// RMS where bf16 operands gave about 1.5e-2.  dO is scaled by one power of two
+// per call (its largest magnitude to [0.5, 1)) so that small upstream
+// gradients do not underflow; the scale is taken out in the epilogues.
+//
+//   k_sbwd_cvt   : fp16 copies of q, k, v
+//   k_sbwd_amax  : max |dO| over the call, k_sbwd_do: the scaled fp16 dO
+//   k_sbwd_q_tc  : 128 query rows of one frame-head, three passes over the
+//                  key tiles: (A) S = Q K^T, row max and sum -> LSE; (B) P as
+//                  fp16 over S in TMEM, O += P V -> o, then dg and Delta in
+//                  fp32 from o, dy and g; (C) S and dP = dO V^T, dS = P (dP -
+//                  Delta) over S, dQ += dS K.
+//   k_sbwd_kv_tc : 128 key rows of one frame-head, over every query tile that
+//                  sees the key frame (the mask is symmetric): S^T = K Q^T,
+//                  dP^T = V dO^T, P^T and dS^T over them, dV += P^T dO,
+//                  dK += dS^T Q.
+//
+// Roles (256 threads): warp 0 producer (TMA; in the key kernel its lanes also
+// stage LSE and Delta of each query tile), warp 1 TMEM allocator and MMA
+// issuer (lane 0), warps 4..7 softmax and epilogues (thread = TMEM lane = row).
+// Every mbarrier wait is bounded; on expiry the CTA records VDN_ERR_TIMEOUT in
+// the status words, stops issuing, drains and frees its TMEM.
+#include <cuda_fp16.h>
+
+#include "tc_common.cuh"
+
+namespace vdn {
+namespace {
+using namespace tc;
+
+constexpr int BR = 128;  // rows of a tile (queries or keys)
+constexpr int kThr = 256;
+constexpr int ST = 2;    // ring stages
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct SmTcWork {
+  __half *q16, *k16, *v16;  // [B*T*N, H, D]  fp16 copies of q, k, v
+  __half* dO;               // [B*T*N, H, D]  dy sigmoid(g_sm) times the call's scale
+  float* lse2;              // [B*T*N, H]     log2-sum-exp2 of the scores in log2 units
+  float* delta;             // [B*T*N, H]     <dO, o> (unscaled)
+  unsigned* amax;           // max |dO| as float bits (non-negative)
+  uint32_t* status;         // bounded-wait status words
+};
+
+// Instruction descriptor, kind::f16 with fp16 A and B, fp32 D, dense (the
+// same tcgen05.mma kind as bf16: mma_bf16 / mma_bf16_ts issue it, the types
+// come from this descriptor).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The power of two that brings max |dO| into [0.5, 1) (1 for an all-zero dO).
+__device__ __forceinline__ float do_scale(const unsigned* amax) {
+  const float a = __uint_as_float(*amax);
+  if (!(a > 0.f) || !(a < 3.0e38f)) return 1.0f;
+  return exp2f(-ceilf(log2f(a)));
+}
+
+static __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ float sigmf(float x) { return 1.0f / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float tof(float x) { return x; }
+__device__ __forceinline__ float tof(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Work item -> (frame, b, h, first row of the tile within the frame).  The
+// anchor frames' items (whose row or key sets span every frame) come first.
+__device__ __forceinline__ void decode(const Dims& d, long long item, int& f, int& b, int& h, int& n0) {
+  const int per = (d.N + BR - 1) / BR;
+  const long long BH = (long long)d.B * d.H;
+  long long bh, rem;
+  if (d.anchors) {
+    const long long na = 2 * BH * per;
+    if (item < na) {
+      const long long a = item / (BH * per);
+      rem = item % (BH * per);
+      bh = rem / per;
+      n0 = (int)(rem % per) * BR;
+      f = a == 0 ? 0 : d.T - 1;
+    } else {
+      const long long it = item - na, per_bh = (long long)(d.T - 2) * per;
+      bh = it / per_bh;
+      rem = it % per_bh;
+      f = 1 + (int)(rem / per);
+      n0 = (int)(rem % per) * BR;
+    }
+  } else {
+    const long long per_bh = (long long)d.T * per;
+    bh = item / per_bh;
+    rem = item % per_bh;
+    f = (int)(rem / per);
+    n0 = (int)(rem % per) * BR;
+  }
+  b = (int)(bh / d.H);
+  h = (int)(bh % d.H);
+}
+
+// The token intervals (absolute token rows) of the frames a query of frame f
+// attends to; by the symmetry of the mask also the query rows that see key
+// frame f.  Three fixed slots, unused ones empty.
+struct Iv {
+  int beg[3], len[3];
+};
+__device__ __forceinline__ Iv intervals(const Dims& d, int f, int base) {
+  Iv v;
+  if (is_anchor(d, f)) {
+    v.beg[0] = base; v.len[0] = d.T * d.N;
+    v.beg[1] = base; v.len[1] = 0;
+    v.beg[2] = base; v.len[2] = 0;
+    return v;
+  }
+  const int c = f / d.chunk;
+  const int lo = max(0, d.chunk * (c - 1)), hi = min(d.T, d.chunk * (c + 2));
+  v.beg[0] = base; v.len[0] = (d.anchors && lo > 0) ? d.N : 0;
+  v.beg[1] = base + lo * d.N; v.len[1] = (hi - lo) * d.N;
+  v.beg[2] = base + (d.T - 1) * d.N; v.len[2] = (d.anchors && hi < d.T) ? d.N : 0;
+  return v;
+}
+__device__ __forceinline__ int n_tiles(const Iv& v) {
+  int n = 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) n += (v.len[i] + BR - 1) / BR;
+  return n;
+}
+__device__ __forceinline__ void tile_of(const Iv& v, int j, int& r0, int& valid) {
+  r0 = 0;
+  valid = 0;
+  bool found = false;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const int nt = (v.len[i] + BR - 1) / BR;
+    if (!found) {
+      if (j < nt) {
+        r0 = v.beg[i] + j * BR;
+        valid = min(BR, v.len[i] - j * BR);
+        found = true;
+      } else {
+        j -= nt;
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------- elementwise (SIMT) --
+__global__ void __launch_bounds__(256) k_sbwd_cvt(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                                                  const __nv_bfloat16* __restrict__ c, __half* __restrict__ a16,
+                                                  __half* __restrict__ b16, __half* __restrict__ c16, long long n8) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const __nv_bfloat16* src[3] = {a, b, c};
+    __half* dst[3] = {a16, b16, c16};
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src[t]) + i);
+      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      uint4 out;
+      uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(x[e]);
+        o[e] = pack_h2(f.x, f.y);
+      }
+      reinterpret_cast<uint4*>(dst[t])[i] = out;
+    }
+  }
+}
+
+// dO = dy sigmoid(g) over every (row, column); dy in y's layout (slot 0 of
+// [.., 2, D], or the summed y).  MODE 0: max |dO| into ws.amax; MODE 1: the
+// scaled fp16 dO.
+template <typename Ty, int D, int MODE>
+__global__ void __launch_bounds__(256) k_sbwd_do(Dims dm, Inputs in, const void* dyp, SmTcWork ws, long long rows) {
+  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(in.gate_sm);
+  const Ty* dy = static_cast<const Ty*>(dyp);
+  const int ys = dm.out_mode == 0 ? 2 : 1;
+  const float sc = MODE == 1 ? do_scale(ws.amax) : 1.0f;
+  float mx = 0.f;
+  const long long n = rows * D;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long row = e / D;
+    const int c = (int)(e % D);
+    const float v = tof(dy[row * ys * D + c]) * sigmf(__bfloat162float(g[e]));
+    if (MODE == 0) mx = fmaxf(mx, fabsf(v));
+    else ws.dO[e] = __float2half_rn(v * sc);
+  }
+  if (MODE == 0) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(ws.amax, __float_as_uint(mx));
+  }
+}
+
+// ------------------------------------------------------------- dQ kernel --
+template <int D, typename Ty>
+__global__ void __launch_bounds__(kThr, 1)
+k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* dgate,
+            const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
+            const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+  constexpr int NB = D / 64;
+  constexpr uint32_t TILE = BR * D * 2;
+  constexpr uint32_t COL_S = 0, COL_P = 128, COL_Q = 256, COL_O = 384;
+  enum { B_QD = 0, B_FULL = 1, B_EMPTY = B_FULL + ST, B_SFULL = B_EMPTY + ST, B_SDONE, B_ODONE, B_DQ, B_DRAIN, NBARS };
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = sm;
+  unsigned char* sDO = sQ + TILE;
+  unsigned char* sK = sDO + TILE;       // ST stages
+  unsigned char* sV = sK + ST * TILE;   // ST stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + ST * TILE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*reinterpret_cast<volatile uint32_t*>(ws.status) != 0u) return;
+  int f, b, h, n0;
+  decode(dm, blockIdx.x, f, b, h, n0);
+  const int base = b * dm.T * dm.N;
+  const int q0 = base + f * dm.N + n0, qvalid = min(BR, dm.N - n0);
+  const Iv iv = intervals(dm, f, base);
+  const int nt = n_tiles(iv), nsteps = 3 * nt;
+  const Ctl ctl{abort_flag, ws.status, (unsigned)TAG_SMBWD_TC};
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i == B_SDONE ? 4 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---- producer: Q and dO once; K for pass A, K and V for passes B and C
+    if (lane == 0) {
+      mbar_expect_tx(bar(B_QD), 2 * TILE);
+      for (int c = 0; c < NB; ++c) {
+        tma_load_3d(smem_u32(sQ + c * BR * 128), &tmq, bar(B_QD), c * 64, h, q0);
+        tma_load_3d(smem_u32(sDO + c * BR * 128), &tmdo, bar(B_QD), c * 64, h, q0);
+      }
+      int issued = 0;
+      for (int s = 0; s < nsteps; ++s) {
+        const bool withv = s >= nt;
+        int k0, kv;
+        tile_of(iv, s % nt, k0, kv);
+        const int st = s % ST;
+        if (s >= ST && !mbar_wait(bar(B_EMPTY + st), (s / ST - 1) & 1, ctl)) break;
+        mbar_expect_tx(bar(B_FULL + st), withv ? 2 * TILE : TILE);
+        for (int c = 0; c < NB; ++c) {
+          tma_load_3d(smem_u32(sK + st * TILE + c * BR * 128), &tmk, bar(B_FULL + st), c * 64, h, k0);
+          if (withv) tma_load_3d(smem_u32(sV + st * TILE + c * BR * 128), &tmv, bar(B_FULL + st), c * 64, h, k0);
+        }
+        issued = s + 1;
+      }
+      mbar_wait(bar(B_QD), 0, ctl);
+      for (int s = issued - ST < 0 ? 0 : issued - ST; s < issued; ++s)
+        mbar_wait(bar(B_FULL + s % ST), (s / ST) & 1, ctl);
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_S = idesc_f16(BR, BR, false);
+      constexpr uint32_t ID_G = idesc_f16(BR, D, true);
+      const uint64_t qd = sdesc(smem_u32(sQ), 16, 1024), dod = sdesc(smem_u32(sDO), 16, 1024);
+      const uint64_t kd0 = sdesc(smem_u32(sK), 16, 1024), vd0 = sdesc(smem_u32(sV), 16, 1024);
+      const uint64_t kmn0 = sdesc(smem_u32(sK), BR * 128, 1024);  // K as the MN-major B of dQ += dS K
+      const uint64_t vmn0 = sdesc(smem_u32(sV), BR * 128, 1024);  // V as the MN-major B of O += P V
+      // D(128 x 128) = A(128 x D) B(128 x D)^T, both K-major in 64-column blocks
+      auto gemm_t = [&](uint32_t dst, uint64_t a, uint64_t bdsc) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * (BR * 128) + (k & 3) * 32;
+          mma_bf16(dst, dadd(a, off), dadd(bdsc, off), ID_S, k > 0 ? 1u : 0u);
+        }
+      };
+      // D(128 x D) += A(TMEM, 128 x 128 fp16 pairs) B(128 x D, MN-major)
+      auto gemm_ts = [&](uint32_t dst, uint32_t a, uint64_t bmn, bool first) {
+#pragma unroll
+        for (int k = 0; k < BR / 16; ++k)
+          mma_bf16_ts(dst, a + 8 * k, dadd(bmn, k * 16 * 128), ID_G, (first && k == 0) ? 0u : 1u);
+      };
+      bool ok = mbar_wait(bar(B_QD), 0, ctl);
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int pass = s / nt, j = s % nt, st = s % ST;
+        ok = mbar_wait(bar(B_FULL + st), (s / ST) & 1, ctl) &&
+             (!((pass == 0 && s > 0) || s == nt) || mbar_wait(bar(B_SDONE), (s - 1) & 1, ctl));
+        if (!ok) break;
+        tc_fence_after();
+        gemm_t(tmem + COL_S, qd, dadd(kd0, st * TILE));
+        if (pass == 2) gemm_t(tmem + COL_P, dod, dadd(vd0, st * TILE));
+        mma_commit(bar(B_SFULL));
+        if (pass > 0) {
+          ok = mbar_wait(bar(B_SDONE), s & 1, ctl);
+          if (!ok) break;
+          tc_fence_after();
+          if (pass == 1) gemm_ts(tmem + COL_O, tmem + COL_S, dadd(vmn0, st * TILE), j == 0);
+          else gemm_ts(tmem + COL_Q, tmem + COL_S, dadd(kmn0, st * TILE), j == 0);
+        }
+        mma_commit(bar(B_EMPTY + st));
+        if (s == 2 * nt - 1) mma_commit(bar(B_ODONE));
+      }
+      mma_commit(bar(B_DQ));
+      mma_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, ctl);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3, row = quad * 32 + lane;
+    const uint32_t la = tmem + ((uint32_t)(quad * 32) << 16);
+    const float c = dm.scale * kLog2e;
+    const bool valid = row < qvalid;
+    const long long grow = (long long)(q0 + row) * dm.H + h;
+    const float sc = do_scale(ws.amax);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    // ---- pass A: row max and sum of 2^(s c)
+    for (int s = 0; ok && s < nt; ++s) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+      int k0, kv;
+      tile_of(iv, s, k0, kv);
+#pragma unroll
+      for (int q = 0; q < BR / 32; ++q) {
+        float v[32];
+        tmem_ld32(la + COL_S + 32 * q, v);
+        tmem_wait_ld();
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, 32 * q + i < kv ? v[i] : -INFINITY);
+        const float mn = fmaxf(m, mx);
+        if (mn != -INFINITY) {
+          float sum = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sum += 32 * q + i < kv ? ex2((v[i] - mn) * c) : 0.f;
+          l = (m == -INFINITY ? 0.f : l * ex2((m - mn) * c)) + sum;
+          m = mn;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_warp(bar(B_SDONE));
+    }
+    const float lse2 = m * c + __log2f(l);
+    if (ok && valid) ws.lse2[grow] = lse2;
+    // ---- pass B: P (fp16) over S for O += P V
+    for (int s = nt; ok && s < 2 * nt; ++s) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+      int k0, kv;
+      tile_of(iv, s - nt, k0, kv);
+#pragma unroll
+      for (int q = 0; q < BR / 32; ++q) {
+        float v[32];
+        tmem_ld32(la + COL_S + 32 * q, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k = 32 * q + 2 * i;
+          pk[i] = pack_h2(k < kv ? ex2(fmaf(v[2 * i], c, -lse2)) : 0.f,
+                          k + 1 < kv ? ex2(fmaf(v[2 * i + 1], c, -lse2)) : 0.f);
+        }
+        tmem_st16(la + COL_S + 16 * q, pk);  // columns [16 q, 16 q + 16): never ahead of the reads
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(bar(B_SDONE));
+    }
+    // ---- o: dg = dy o sigmoid'(g), Delta = <dy sigmoid(g), o>
+    float del = 0.f;
+    if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_ODONE), 0, ctl))) {
+      tc_fence_after();
+      const int ys = dm.out_mode == 0 ? 2 : 1;
+      const Ty* dy = static_cast<const Ty*>(dyp) + grow * ys * D;
+      const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(in.gate_sm) + grow * D;
+      float* dgr = dgate + grow * D;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        float o[32];
+        tmem_ld32(la + COL_O + 32 * q, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            float4 dg4;
+            float* dgp = reinterpret_cast<float*>(&dg4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int col = 32 * q + i + e;
+              const float sg = sigmf(__bfloat162float(g[col]));
+              const float dyv = tof(dy[col]);
+              del = fmaf(dyv * sg, o[i + e], del);
+              dgp[e] = dyv * o[i + e] * sg * (1.0f - sg);
+            }
+            *reinterpret_cast<float4*>(dgr + 32 * q + i) = dg4;
+          }
+        }
+      }
+      if (valid) ws.delta[grow] = del;
+    } else {
+      ok = false;
+    }
+    const float dels = del * sc;  // in the units of the scaled dO
+    // ---- pass C: dS = P (dP - Delta) (fp16) over S for dQ += dS K
+    for (int s = 2 * nt; ok && s < nsteps; ++s) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+      int k0, kv;
+      tile_of(iv, s - 2 * nt, k0, kv);
+#pragma unroll
+      for (int q = 0; q < BR / 32; ++q) {
+        float vs[32], vp[32];
+        tmem_ld32(la + COL_S + 32 * q, vs);
+        tmem_ld32(la + COL_P + 32 * q, vp);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k = 32 * q + 2 * i;
+          const float p0 = k < kv ? ex2(fmaf(vs[2 * i], c, -lse2)) : 0.f;
+          const float p1 = k + 1 < kv ? ex2(fmaf(vs[2 * i + 1], c, -lse2)) : 0.f;
+          pk[i] = pack_h2(p0 * (vp[2 * i] - dels), p1 * (vp[2 * i + 1] - dels));
+        }
+        tmem_st16(la + COL_S + 16 * q, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(bar(B_SDONE));
+    }
+    // ---- epilogue: dq = s dQ / scale of dO
+    if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, ctl))) {
+      tc_fence_after();
+      const float f = dm.scale / sc;
+      float* dst = dq + grow * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        float v[32];
+        tmem_ld32(la + COL_Q + 32 * q, v);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + 32 * q + i) = make_float4(v[i] * f, v[i + 1] * f, v[i + 2] * f, v[i + 3] * f);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, 512);
+}
+
+// ---------------------------------------------------------- dK, dV kernel --
+template <int D>
+__global__ void __launch_bounds__(kThr, 1)
+k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__ CUtensorMap tmq,
+             const __grid_constant__ CUtensorMap tmdo, const __grid_constant__ CUtensorMap tmk,
+             const __grid_constant__ CUtensorMap tmv) {
+  constexpr int NB = D / 64;
+  constexpr uint32_t TILE = BR * D * 2;
+  constexpr uint32_t COL_S = 0, COL_P = 128, COL_V = 256, COL_K = 256 + D;
+  enum { B_KV = 0, B_FULL = 1, B_EMPTY = B_FULL + ST, B_SFULL = B_EMPTY + ST, B_SDONE, B_DONE, B_DRAIN, NBARS };
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sK = sm;
+  unsigned char* sV = sK + TILE;
+  unsigned char* sQ = sV + TILE;        // ST stages
+  unsigned char* sDO = sQ + ST * TILE;  // ST stages
+  float* sL = reinterpret_cast<float*>(sDO + ST * TILE);  // [ST][BR] LSE (log2 units) of the tile's queries
+  float* sD = sL + ST * BR;                               // [ST][BR] Delta
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + ST * BR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (*reinterpret_cast<volatile uint32_t*>(ws.status) != 0u) return;
+  int f, b, h, n0;
+  decode(dm, blockIdx.x, f, b, h, n0);
+  const int base = b * dm.T * dm.N;
+  const int k0 = base + f * dm.N + n0, kvalid = min(BR, dm.N - n0);
+  const Iv iv = intervals(dm, f, base);
+  const int nt = n_tiles(iv);
+  const Ctl ctl{abort_flag, ws.status, (unsigned)TAG_SMBWD_TC};
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  const float sc = do_scale(ws.amax);
+
+  if (threadIdx.x == 0) {
+    // FULL: the TMA transaction arrival plus the producer warp's arrival after
+    // it staged LSE and Delta; SDONE: one arrival per softmax warp
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i == B_SDONE ? 4 : (i == B_FULL || i == B_FULL + 1) ? 2 : 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---- producer: K, V once; per query tile Q and dO by TMA, LSE and Delta by the lanes
+    if (lane == 0) {
+      mbar_expect_tx(bar(B_KV), 2 * TILE);
+      for (int c = 0; c < NB; ++c) {
+        tma_load_3d(smem_u32(sK + c * BR * 128), &tmk, bar(B_KV), c * 64, h, k0);
+        tma_load_3d(smem_u32(sV + c * BR * 128), &tmv, bar(B_KV), c * 64, h, k0);
+      }
+    }
+    int issued = 0;
+    for (int j = 0; j < nt; ++j) {
+      int r0, rv;
+      tile_of(iv, j, r0, rv);
+      const int st = j % ST;
+      if (j >= ST && !__all_sync(0xffffffffu, mbar_wait(bar(B_EMPTY + st), (j / ST - 1) & 1, ctl))) break;
+      if (lane == 0) {
+        mbar_expect_tx(bar(B_FULL + st), 2 * TILE);
+        for (int c = 0; c < NB; ++c) {
+          tma_load_3d(smem_u32(sQ + st * TILE + c * BR * 128), &tmq, bar(B_FULL + st), c * 64, h, r0);
+          tma_load_3d(smem_u32(sDO + st * TILE + c * BR * 128), &tmdo, bar(B_FULL + st), c * 64, h, r0);
+        }
+      }
+      for (int r = lane; r < BR; r += 32) {
+        const bool v = r < rv;
+        const long long gi = (long long)(r0 + r) * dm.H + h;
+        sL[st * BR + r] = v ? ws.lse2[gi] : INFINITY;  // 2^(s c - inf) = 0: no weight
+        sD[st * BR + r] = v ? ws.delta[gi] * sc : 0.f;  // in the units of the scaled dO
+      }
+      mbar_arrive_warp(bar(B_FULL + st));
+      issued = j + 1;
+    }
+    if (lane == 0) {
+      mbar_wait(bar(B_KV), 0, ctl);
+      for (int j = issued - ST < 0 ? 0 : issued - ST; j < issued; ++j)
+        mbar_wait(bar(B_FULL + j % ST), (j / ST) & 1, ctl);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t ID_S = idesc_f16(BR, BR, false);
+      constexpr uint32_t ID_G = idesc_f16(BR, D, true);
+      const uint64_t kd = sdesc(smem_u32(sK), 16, 1024), vd = sdesc(smem_u32(sV), 16, 1024);
+      const uint64_t qd0 = sdesc(smem_u32(sQ), 16, 1024), dod0 = sdesc(smem_u32(sDO), 16, 1024);
+      const uint64_t qmn0 = sdesc(smem_u32(sQ), BR * 128, 1024), domn0 = sdesc(smem_u32(sDO), BR * 128, 1024);
+      auto gemm_t = [&](uint32_t dst, uint64_t a, uint64_t bdsc) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * (BR * 128) + (k & 3) * 32;
+          mma_bf16(dst, dadd(a, off), dadd(bdsc, off), ID_S, k > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(B_KV), 0, ctl);
+      for (int j = 0; ok && j < nt; ++j) {
+        const int st = j % ST;
+        ok = mbar_wait(bar(B_FULL + st), (j / ST) & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        gemm_t(tmem + COL_S, kd, dadd(qd0, st * TILE));   // S^T = K Q^T
+        gemm_t(tmem + COL_P, vd, dadd(dod0, st * TILE));  // dP^T = V dO^T
+        mma_commit(bar(B_SFULL));
+        ok = mbar_wait(bar(B_SDONE), j & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t qmn = dadd(qmn0, st * TILE), domn = dadd(domn0, st * TILE);
+#pragma unroll
+        for (int k = 0; k < BR / 16; ++k) {
+          const uint32_t acc = (j > 0 || k > 0) ? 1u : 0u;
+          mma_bf16_ts(tmem + COL_V, tmem + COL_S + 8 * k, dadd(domn, k * 16 * 128), ID_G, acc);  // dV += P^T dO
+          mma_bf16_ts(tmem + COL_K, tmem + COL_P + 8 * k, dadd(qmn, k * 16 * 128), ID_G, acc);   // dK += dS^T Q
+        }
+        mma_commit(bar(B_EMPTY + st));
+      }
+      mma_commit(bar(B_DONE));
+      mma_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, ctl);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3, row = quad * 32 + lane;
+    const uint32_t la = tmem + ((uint32_t)(quad * 32) << 16);
+    const float c = dm.scale * kLog2e;
+    bool ok = true;
+    for (int j = 0; ok && j < nt; ++j) {
+      const int st = j % ST;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), j & 1, ctl) &&
+                                       mbar_wait(bar(B_FULL + st), (j / ST) & 1, ctl))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* L = sL + st * BR;
+      const float* Dl = sD + st * BR;
+#pragma unroll
+      for (int q = 0; q < BR / 32; ++q) {
+        float vs[32], vp[32];
+        tmem_ld32(la + COL_S + 32 * q, vs);
+        tmem_ld32(la + COL_P + 32 * q, vp);
+        tmem_wait_ld();
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int qc = 32 * q + 2 * i;
+          const float p0 = ex2(fmaf(vs[2 * i], c, -L[qc]));
+          const float p1 = ex2(fmaf(vs[2 * i + 1], c, -L[qc + 1]));
+          pp[i] = pack_h2(p0, p1);
+          pd[i] = pack_h2(p0 * (vp[2 * i] - Dl[qc]), p1 * (vp[2 * i + 1] - Dl[qc + 1]));
+        }
+        tmem_st16(la + COL_S + 16 * q, pp);
+        tmem_st16(la + COL_P + 16 * q, pd);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(bar(B_SDONE));
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_DONE), 0, ctl))) {
+      tc_fence_after();
+      const bool valid = row < kvalid;
+      const long long gi = ((long long)(k0 + row) * dm.H + h) * D;
+      const float fv = 1.0f / sc, fk = dm.scale / sc;  // the scale of dO taken out
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        float a[32], g[32];
+        tmem_ld32(la + COL_V + 32 * q, a);
+        tmem_ld32(la + COL_K + 32 * q, g);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            *reinterpret_cast<float4*>(dv + gi + 32 * q + i) =
+                make_float4(a[i] * fv, a[i + 1] * fv, a[i + 2] * fv, a[i + 3] * fv);
+            *reinterpret_cast<float4*>(dk + gi + 32 * q + i) =
+                make_float4(g[i] * fk, g[i + 1] * fk, g[i + 2] * fk, g[i + 3] * fk);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, 512);
+}
+
+template <int D> constexpr size_t q_smem() { return 1024 + (2 + 2 * ST) * (size_t)BR * D * 2 + 16 * 8 + 16; }
+template <int D> constexpr size_t kv_smem() {
+  return 1024 + (2 + 2 * ST) * (size_t)BR * D * 2 + 2 * ST * BR * 4 + 16 * 8 + 16;
+}
+
+unsigned grid_for(long long n) {
+  const long long b = (n + 255) / 256;
+  return (unsigned)(b < 148LL * 16 ? (b > 0 ? b : 1) : 148LL * 16);
+}
+
+template <int D, typename Ty>
+cudaError_t launch_d(const Dims& d, const Inputs& in, const SmTcArgs& a, cudaStream_t s) {
+  const long long tokens = (long long)d.B * d.T * d.N, rows = tokens * d.H;
+  SmTcWork ws{static_cast<__half*>(a.q16), static_cast<__half*>(a.k16), static_cast<__half*>(a.v16),
+              static_cast<__half*>(a.dO16), a.lse2, a.delta, a.amax, a.status};
+  cudaError_t e;
+  const long long n8 = rows * D / 8;
+  k_sbwd_cvt<<<grid_for(n8), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(in.q), static_cast<const __nv_bfloat16*>(in.k),
+                                          static_cast<const __nv_bfloat16*>(in.v), ws.q16, ws.k16, ws.v16, n8);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_sbwd_do<Ty, D, 0><<<grid_for(rows * D), 256, 0, s>>>(d, in, a.dy, ws, rows);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_sbwd_do<Ty, D, 1><<<grid_for(rows * D), 256, 0, s>>>(d, in, a.dy, ws, rows);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  CUtensorMap mq, mdo, mk, mv;
+  if (!make_token_map(&mq, ws.q16, tokens, d.H, D, BR) || !make_token_map(&mdo, ws.dO, tokens, d.H, D, BR) ||
+      !make_token_map(&mk, ws.k16, tokens, d.H, D, BR) || !make_token_map(&mv, ws.v16, tokens, d.H, D, BR))
+    return cudaErrorInvalidValue;
+  const long long items = (long long)d.B * d.H * d.T * ((d.N + BR - 1) / BR);
+  auto kq = k_sbwd_q_tc<D, Ty>;
+  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem<D>())) != cudaSuccess)
+    return e;
+  kq<<<(unsigned)items, kThr, q_smem<D>(), s>>>(d, in, a.dy, ws, a.dq, a.dgate, mq, mdo, mk, mv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(k_sbwd_kv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem<D>())) !=
+      cudaSuccess)
+    return e;
+  k_sbwd_kv_tc<D><<<(unsigned)items, kThr, kv_smem<D>(), s>>>(d, ws, a.dk, a.dv, mq, mdo, mk, mv);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sm_bwd_tc_supported(const Dims& d) {
+  if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128)) return false;
+  if ((long long)d.B * d.T * d.N + BR >= (1LL << 31)) return false;  // int32 TMA row coordinates
+  if ((long long)d.B * d.H * d.T * ((d.N + BR - 1) / BR) > 0x7FFFFFFFLL) return false;
+  return encode_fn() != nullptr;
+}
+
+// [status 256 B][q16][k16][v16][dO16][lse2][delta][amax 256 B], 256-byte aligned regions
+size_t sm_bwd_tc_workspace(const Dims& d, size_t* off) {
+  const size_t rows = (size_t)d.B * d.T * d.N * d.H;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t sizes[8] = {256, rows * d.dk * 2, rows * d.dk * 2, rows * d.dv * 2, rows * d.dv * 2, rows * 4, rows * 4, 256};
+  size_t o = 0;
+  for (int i = 0; i < 8; ++i) {
+    if (off) off[i] = o;
+    o += up(sizes[i]);
+  }
+  return o;
+}
+
+cudaError_t launch_sm_bwd_tc(const Dims& d, const Inputs& in, const SmTcArgs& a, cudaStream_t s) {
+  if (d.dk == 128) return d.out_bf16 ? launch_d<128, __nv_bfloat16>(d, in, a, s) : launch_d<128, float>(d, in, a, s);
+  if (d.dk == 64) return d.out_bf16 ? launch_d<64, __nv_bfloat16>(d, in, a, s) : launch_d<64, float>(d, in, a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn
