@@ -675,23 +675,35 @@ def run_bwd(args):
     flops, byts = bwd_work(s, w.dtype == "bf16")
     pairs = O_density(s) * (s.T * s.N) ** 2 * s.H * s.B
     sm_flops = 10.0 * s.d_k * pairs  # s, dP, dq, dk, dv: 2 d flops each per allowed pair
-    peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FMA lanes x 2 flops x max SM clock
-    tf = (flops + sm_flops) / (ms * 1e-3) / 1e12
+    simt_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # fp32 FMA lanes x 2 flops x max SM clock
+    peaks, src = load_peaks()
+    # the softmax backward runs on the tensor cores for bf16 inputs (fp16 operands:
+    # the dense fp16 rate equals the bf16 one); a step of both branches is long,
+    # so the sustained GEMM rate is the denominator
+    sm_tc = L.vdn_hybrid_stage_impl(cfg, L.STAGE_SOFTMAX_BWD) == 1
+    tc_peak = peaks.get("bf16_tflops_sustained", 1400.0)
+    sm_peak = tc_peak if sm_tc else simt_peak
+    sm_tf = sm_flops / (sm_ms * 1e-3) / 1e12
+    lin_tf = flops / (lin_ms * 1e-3) / 1e12
     print(json.dumps({
         "metric": "hybrid-attn core backward", "value": w.tokens / (ms * 1e-3), "unit": "video tokens/s",
         "ms_per_step": ms, "steps": args.steps, "warmup": args.warmup, "n_gpus": 1, "higher_is_better": True,
-        "dtype": "f32" if w.dtype == "f32" else "bf16 in, f32 compute", "data": "synthetic",
+        "dtype": "f32" if w.dtype == "f32" else "bf16 in; fp16 tensor-core operands (softmax), f32 SIMT (linear)",
+        "data": "synthetic",
         "config": {"workload": w.name, "B": s.B, "T": s.T, "N": s.N, "H": s.H, "d": s.d_k, "L": s.L,
                    "l2": "inputs larger than L2"},
-        "gpu_launches": 8 * args.steps,
+        "gpu_launches": (6 + (5 if sm_tc else 2)) * args.steps,
         "branches": {
-            "linear": {"ms": lin_ms, "kernels": 6, "flops": flops, "hbm_bytes": byts,
-                       "tflops": flops / (lin_ms * 1e-3) / 1e12, "frac": flops / (lin_ms * 1e-3) / 1e12 / peak},
-            "softmax": {"ms": sm_ms, "kernels": 2, "flops": sm_flops, "pairs": pairs,
-                        "tflops": sm_flops / (sm_ms * 1e-3) / 1e12, "frac": sm_flops / (sm_ms * 1e-3) / 1e12 / peak}},
-        "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                     "peak_source": "148 SMs x 128 fp32 lanes x 2 x 1.965 GHz (SIMT fp32)",
-                     "flops": flops + sm_flops},
+            "linear": {"ms": lin_ms, "kernels": 6, "bound": "alu", "flops": flops, "hbm_bytes": byts,
+                       "tflops": lin_tf, "peak": simt_peak, "frac": lin_tf / simt_peak},
+            "softmax": {"ms": sm_ms, "kernels": 5 if sm_tc else 2, "bound": "tensor" if sm_tc else "alu",
+                        "flops": sm_flops, "pairs": pairs, "tflops": sm_tf, "peak": sm_peak,
+                        "frac": sm_tf / sm_peak}},
+        "roofline": {"bound": "tensor" if sm_tc else "alu", "kernel": "softmax-branch backward (dq + dk/dv kernels)",
+                     "achieved": sm_tf, "peak": sm_peak, "unit": "TFLOP/s", "frac": sm_tf / sm_peak,
+                     "peak_source": (f"bf16_tflops_sustained ({src})" if sm_tc else
+                                     "148 SMs x 128 fp32 lanes x 2 x 1.965 GHz (SIMT fp32)"),
+                     "flops": sm_flops, "traffic": None},
         "clocks": clocks}), flush=True)
 
 
