@@ -29,9 +29,10 @@
 //                  dP^T = V dO^T, P^T and dS^T over them, dV += P^T dO,
 //                  dK += dS^T Q.
 //
-// Roles (256 threads): warp 0 producer (TMA; in the key kernel its lanes also
+// Roles (384 threads): warp 0 producer (TMA; in the key kernel its lanes also
 // stage LSE and Delta of each query tile), warp 1 TMEM allocator and MMA
-// issuer (lane 0), warps 4..7 softmax and epilogues (thread = TMEM lane = row).
+// issuer (lane 0), warps 4..11 softmax and epilogues: two warps per TMEM lane
+// quadrant (thread = TMEM lane = row), each with half of the columns.
 // Every mbarrier wait is bounded; on expiry the CTA records VDN_ERR_TIMEOUT in
 // the status words, stops issuing, drains and frees its TMEM.
 #include <cuda_fp16.h>
@@ -43,7 +44,8 @@ namespace {
 using namespace tc;
 
 constexpr int BR = 128;  // rows of a tile (queries or keys)
-constexpr int kThr = 256;
+constexpr int kThr = 384;       // warps 0..3 roles, 4..11 softmax
+constexpr int kSoftWarps = 8;   // two per TMEM lane quadrant, each with half the columns
 constexpr int ST = 2;    // ring stages
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -83,6 +85,17 @@ static __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t 
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
+
+// Packed fp16 pairs of a 128-column score tile written back by two warps per
+// row: the warp of half h reads columns [64 h, 64 h + 64) and writes its 32
+// packed columns inside that range, chunk q (32 scores) at pk_col(q), so no
+// write lands on columns the other warp has still to read.  The 16 keys of
+// k-step k then sit at pk_k(k).
+__host__ __device__ constexpr uint32_t pk_col(int q) { return 64u * (q >> 1) + 16u * (q & 1); }
+__host__ __device__ constexpr uint32_t pk_k(int k) { return 8u * k + 32u * (k >> 2); }
+
+// Named barrier of the eight softmax warps (barrier 0 is __syncthreads).
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ float sigmf(float x) { return 1.0f / (1.0f + __expf(-x)); }
 __device__ __forceinline__ float tof(float x) { return x; }
@@ -215,6 +228,11 @@ __global__ void __launch_bounds__(256) k_sbwd_do(Dims dm, Inputs in, const void*
 }
 
 // ------------------------------------------------------------- dQ kernel --
+// TMEM: S buffers 0 and 1 at columns 0 and 384, dP at 128, and at 256 the
+// accumulator of the pass: O in pass B, dQ in pass C (O is read out before
+// the first dQ product, which waits for the softmax of pass C's first tile).
+// Passes A and B alternate the S buffers, so the product of tile s + 1 runs
+// while the softmax works on tile s; pass C uses buffer 0 and dP.
 template <int D, typename Ty>
 __global__ void __launch_bounds__(kThr, 1)
 k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* dgate,
@@ -222,15 +240,17 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
             const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
   constexpr int NB = D / 64;
   constexpr uint32_t TILE = BR * D * 2;
-  constexpr uint32_t COL_S = 0, COL_P = 128, COL_Q = 256, COL_O = 384;
-  enum { B_QD = 0, B_FULL = 1, B_EMPTY = B_FULL + ST, B_SFULL = B_EMPTY + ST, B_SDONE, B_ODONE, B_DQ, B_DRAIN, NBARS };
+  constexpr uint32_t COL_P = 128, COL_ACC = 256;
+  enum { B_QD = 0, B_FULL = 1, B_EMPTY = B_FULL + ST, B_SFULL = B_EMPTY + ST, B_SFULLC = B_SFULL + 2, B_SDONE,
+         B_ODONE, B_DQ, B_DRAIN, NBARS };
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sQ = sm;
   unsigned char* sDO = sQ + TILE;
   unsigned char* sK = sDO + TILE;       // ST stages
   unsigned char* sV = sK + ST * TILE;   // ST stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + ST * TILE);
+  float* red = reinterpret_cast<float*>(sV + ST * TILE);  // [3][2][BR]: row max, sum, Delta of each half
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 6 * BR);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -241,12 +261,13 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
   const int base = b * dm.T * dm.N;
   const int q0 = base + f * dm.N + n0, qvalid = min(BR, dm.N - n0);
   const Iv iv = intervals(dm, f, base);
-  const int nt = n_tiles(iv), nsteps = 3 * nt;
+  const int nt = n_tiles(iv), nab = 2 * nt, nsteps = 3 * nt;
   const Ctl ctl{abort_flag, ws.status, (unsigned)TAG_SMBWD_TC};
   auto bar = [&](int i) { return smem_u32(bars + i); };
+  auto sbuf = [](int s) { return (s & 1) ? 384u : 0u; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i == B_SDONE ? 4 : 1);
+    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i == B_SDONE ? kSoftWarps : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -303,34 +324,53 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
       auto gemm_ts = [&](uint32_t dst, uint32_t a, uint64_t bmn, bool first) {
 #pragma unroll
         for (int k = 0; k < BR / 16; ++k)
-          mma_bf16_ts(dst, a + 8 * k, dadd(bmn, k * 16 * 128), ID_G, (first && k == 0) ? 0u : 1u);
+          mma_bf16_ts(dst, a + pk_k(k), dadd(bmn, k * 16 * 128), ID_G, (first && k == 0) ? 0u : 1u);
       };
-      bool ok = mbar_wait(bar(B_QD), 0, ctl);
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int pass = s / nt, j = s % nt, st = s % ST;
-        ok = mbar_wait(bar(B_FULL + st), (s / ST) & 1, ctl) &&
-             (!((pass == 0 && s > 0) || s == nt) || mbar_wait(bar(B_SDONE), (s - 1) & 1, ctl));
+      // S(s) of passes A and B into buffer s & 1; in pass A the stage is free
+      // once S has read K
+      auto issue_s = [&](int s) -> bool {
+        const int st = s % ST;
+        if (!mbar_wait(bar(B_FULL + st), (s / ST) & 1, ctl)) return false;
+        tc_fence_after();
+        gemm_t(tmem + sbuf(s), qd, dadd(kd0, st * TILE));
+        mma_commit(bar(B_SFULL + (s & 1)));
+        if (s < nt) mma_commit(bar(B_EMPTY + st));
+        return true;
+      };
+      bool ok = mbar_wait(bar(B_QD), 0, ctl) && issue_s(0) && (nab < 2 || issue_s(1));
+      for (int s = 0; ok && s < nab; ++s) {
+        ok = mbar_wait(bar(B_SDONE), s & 1, ctl);
         if (!ok) break;
         tc_fence_after();
-        gemm_t(tmem + COL_S, qd, dadd(kd0, st * TILE));
-        if (pass == 2) gemm_t(tmem + COL_P, dod, dadd(vd0, st * TILE));
-        mma_commit(bar(B_SFULL));
-        if (pass > 0) {
-          ok = mbar_wait(bar(B_SDONE), s & 1, ctl);
-          if (!ok) break;
-          tc_fence_after();
-          if (pass == 1) gemm_ts(tmem + COL_O, tmem + COL_S, dadd(vmn0, st * TILE), j == 0);
-          else gemm_ts(tmem + COL_Q, tmem + COL_S, dadd(kmn0, st * TILE), j == 0);
+        if (s >= nt) {
+          gemm_ts(tmem + COL_ACC, tmem + sbuf(s), dadd(vmn0, (s % ST) * TILE), s == nt);  // O += P V
+          mma_commit(bar(B_EMPTY + s % ST));
         }
+        // buffer s & 1 again: P(s) is read by the P V above, issued first
+        if (s + 2 < nab) ok = issue_s(s + 2);
+      }
+      if (ok) mma_commit(bar(B_ODONE));
+      for (int s = nab; ok && s < nsteps; ++s) {
+        const int st = s % ST;
+        ok = mbar_wait(bar(B_FULL + st), (s / ST) & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        gemm_t(tmem, qd, dadd(kd0, st * TILE));
+        gemm_t(tmem + COL_P, dod, dadd(vd0, st * TILE));
+        mma_commit(bar(B_SFULLC));
+        ok = mbar_wait(bar(B_SDONE), s & 1, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        gemm_ts(tmem + COL_ACC, tmem, dadd(kmn0, st * TILE), s == nab);  // dQ += dS K
         mma_commit(bar(B_EMPTY + st));
-        if (s == 2 * nt - 1) mma_commit(bar(B_ODONE));
       }
       mma_commit(bar(B_DQ));
       mma_commit(bar(B_DRAIN));
       mbar_wait(bar(B_DRAIN), 0, ctl);
     }
   } else if (warp >= 4) {
-    const int quad = warp & 3, row = quad * 32 + lane;
+    // ---- softmax: two warps per TMEM lane quadrant, each with half the columns
+    const int quad = warp & 3, half = (warp - 4) >> 2, row = quad * 32 + lane;
     const uint32_t la = tmem + ((uint32_t)(quad * 32) << 16);
     const float c = dm.scale * kLog2e;
     const bool valid = row < qvalid;
@@ -338,16 +378,17 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
     const float sc = do_scale(ws.amax);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    // ---- pass A: row max and sum of 2^(s c)
+    // ---- pass A: this half's row max and sum of 2^(s c)
     for (int s = 0; ok && s < nt; ++s) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, ctl))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + (s & 1)), (s >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       int k0, kv;
       tile_of(iv, s, k0, kv);
 #pragma unroll
-      for (int q = 0; q < BR / 32; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * half + qq;
         float v[32];
-        tmem_ld32(la + COL_S + 32 * q, v);
+        tmem_ld32(la + sbuf(s) + 32 * q, v);
         tmem_wait_ld();
         float mx = -INFINITY;
 #pragma unroll
@@ -364,18 +405,26 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
       tc_fence_before();
       mbar_arrive_warp(bar(B_SDONE));
     }
-    const float lse2 = m * c + __log2f(l);
-    if (ok && valid) ws.lse2[grow] = lse2;
+    // the two halves of each row combined (every softmax warp reaches this barrier)
+    red[half * BR + row] = m;
+    red[2 * BR + half * BR + row] = l;
+    softmax_bar();
+    const float mo = red[(1 - half) * BR + row], lo = red[2 * BR + (1 - half) * BR + row];
+    const float mm = fmaxf(m, mo);
+    const float lt = (m == -INFINITY ? 0.f : l * ex2((m - mm) * c)) + (mo == -INFINITY ? 0.f : lo * ex2((mo - mm) * c));
+    const float lse2 = mm * c + __log2f(lt);
+    if (ok && valid && half == 0) ws.lse2[grow] = lse2;
     // ---- pass B: P (fp16) over S for O += P V
-    for (int s = nt; ok && s < 2 * nt; ++s) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, ctl))) { ok = false; break; }
+    for (int s = nt; ok && s < nab; ++s) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + (s & 1)), (s >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       int k0, kv;
       tile_of(iv, s - nt, k0, kv);
 #pragma unroll
-      for (int q = 0; q < BR / 32; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * half + qq;
         float v[32];
-        tmem_ld32(la + COL_S + 32 * q, v);
+        tmem_ld32(la + sbuf(s) + 32 * q, v);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -384,13 +433,13 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
           pk[i] = pack_h2(k < kv ? ex2(fmaf(v[2 * i], c, -lse2)) : 0.f,
                           k + 1 < kv ? ex2(fmaf(v[2 * i + 1], c, -lse2)) : 0.f);
         }
-        tmem_st16(la + COL_S + 16 * q, pk);  // columns [16 q, 16 q + 16): never ahead of the reads
+        tmem_st16(la + sbuf(s) + pk_col(q), pk);  // inside this half's columns, behind its reads
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(bar(B_SDONE));
     }
-    // ---- o: dg = dy o sigmoid'(g), Delta = <dy sigmoid(g), o>
+    // ---- o: dg = dy o sigmoid'(g), Delta = <dy sigmoid(g), o>, this half's columns
     float del = 0.f;
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_ODONE), 0, ctl))) {
       tc_fence_after();
@@ -399,9 +448,9 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
       const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(in.gate_sm) + grow * D;
       float* dgr = dgate + grow * D;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = half * (D / 64); q < (half + 1) * (D / 64); ++q) {
         float o[32];
-        tmem_ld32(la + COL_O + 32 * q, o);
+        tmem_ld32(la + COL_ACC + 32 * q, o);
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
@@ -420,21 +469,25 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
           }
         }
       }
-      if (valid) ws.delta[grow] = del;
     } else {
       ok = false;
     }
+    red[4 * BR + half * BR + row] = del;
+    softmax_bar();
+    del += red[4 * BR + (1 - half) * BR + row];
+    if (ok && valid && half == 0) ws.delta[grow] = del;
     const float dels = del * sc;  // in the units of the scaled dO
     // ---- pass C: dS = P (dP - Delta) (fp16) over S for dQ += dS K
-    for (int s = 2 * nt; ok && s < nsteps; ++s) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, ctl))) { ok = false; break; }
+    for (int s = nab; ok && s < nsteps; ++s) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULLC), (s - nab) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       int k0, kv;
-      tile_of(iv, s - 2 * nt, k0, kv);
+      tile_of(iv, s - nab, k0, kv);
 #pragma unroll
-      for (int q = 0; q < BR / 32; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * half + qq;
         float vs[32], vp[32];
-        tmem_ld32(la + COL_S + 32 * q, vs);
+        tmem_ld32(la + 32 * q, vs);
         tmem_ld32(la + COL_P + 32 * q, vp);
         tmem_wait_ld();
         uint32_t pk[16];
@@ -445,26 +498,27 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
           const float p1 = k + 1 < kv ? ex2(fmaf(vs[2 * i + 1], c, -lse2)) : 0.f;
           pk[i] = pack_h2(p0 * (vp[2 * i] - dels), p1 * (vp[2 * i + 1] - dels));
         }
-        tmem_st16(la + COL_S + 16 * q, pk);
+        tmem_st16(la + pk_col(q), pk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(bar(B_SDONE));
     }
-    // ---- epilogue: dq = s dQ / scale of dO
+    // ---- epilogue: dq = s dQ / scale of dO, this half's columns
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_DQ), 0, ctl))) {
       tc_fence_after();
-      const float f = dm.scale / sc;
+      const float fq = dm.scale / sc;
       float* dst = dq + grow * D;
 #pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = half * (D / 64); q < (half + 1) * (D / 64); ++q) {
         float v[32];
-        tmem_ld32(la + COL_Q + 32 * q, v);
+        tmem_ld32(la + COL_ACC + 32 * q, v);
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + 32 * q + i) = make_float4(v[i] * f, v[i + 1] * f, v[i + 2] * f, v[i + 3] * f);
+            *reinterpret_cast<float4*>(dst + 32 * q + i) =
+                make_float4(v[i] * fq, v[i + 1] * fq, v[i + 2] * fq, v[i + 3] * fq);
         }
       }
     }
@@ -512,7 +566,8 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
   if (threadIdx.x == 0) {
     // FULL: the TMA transaction arrival plus the producer warp's arrival after
     // it staged LSE and Delta; SDONE: one arrival per softmax warp
-    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i == B_SDONE ? 4 : (i == B_FULL || i == B_FULL + 1) ? 2 : 1);
+    for (int i = 0; i < NBARS; ++i)
+      mbar_init(bar(i), i == B_SDONE ? kSoftWarps : (i == B_FULL || i == B_FULL + 1) ? 2 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -588,8 +643,8 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
 #pragma unroll
         for (int k = 0; k < BR / 16; ++k) {
           const uint32_t acc = (j > 0 || k > 0) ? 1u : 0u;
-          mma_bf16_ts(tmem + COL_V, tmem + COL_S + 8 * k, dadd(domn, k * 16 * 128), ID_G, acc);  // dV += P^T dO
-          mma_bf16_ts(tmem + COL_K, tmem + COL_P + 8 * k, dadd(qmn, k * 16 * 128), ID_G, acc);   // dK += dS^T Q
+          mma_bf16_ts(tmem + COL_V, tmem + COL_S + pk_k(k), dadd(domn, k * 16 * 128), ID_G, acc);  // dV += P^T dO
+          mma_bf16_ts(tmem + COL_K, tmem + COL_P + pk_k(k), dadd(qmn, k * 16 * 128), ID_G, acc);   // dK += dS^T Q
         }
         mma_commit(bar(B_EMPTY + st));
       }
@@ -598,7 +653,8 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
       mbar_wait(bar(B_DRAIN), 0, ctl);
     }
   } else if (warp >= 4) {
-    const int quad = warp & 3, row = quad * 32 + lane;
+    // ---- softmax: two warps per TMEM lane quadrant, each with half the query columns
+    const int quad = warp & 3, half = (warp - 4) >> 2, row = quad * 32 + lane;
     const uint32_t la = tmem + ((uint32_t)(quad * 32) << 16);
     const float c = dm.scale * kLog2e;
     bool ok = true;
@@ -613,7 +669,8 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
       const float* L = sL + st * BR;
       const float* Dl = sD + st * BR;
 #pragma unroll
-      for (int q = 0; q < BR / 32; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * half + qq;
         float vs[32], vp[32];
         tmem_ld32(la + COL_S + 32 * q, vs);
         tmem_ld32(la + COL_P + 32 * q, vp);
@@ -627,8 +684,8 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
           pp[i] = pack_h2(p0, p1);
           pd[i] = pack_h2(p0 * (vp[2 * i] - Dl[qc]), p1 * (vp[2 * i + 1] - Dl[qc + 1]));
         }
-        tmem_st16(la + COL_S + 16 * q, pp);
-        tmem_st16(la + COL_P + 16 * q, pd);
+        tmem_st16(la + COL_S + pk_col(q), pp);
+        tmem_st16(la + COL_P + pk_col(q), pd);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -640,7 +697,7 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
       const long long gi = ((long long)(k0 + row) * dm.H + h) * D;
       const float fv = 1.0f / sc, fk = dm.scale / sc;  // the scale of dO taken out
 #pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
+      for (int q = half * (D / 64); q < (half + 1) * (D / 64); ++q) {
         float a[32], g[32];
         tmem_ld32(la + COL_V + 32 * q, a);
         tmem_ld32(la + COL_K + 32 * q, g);
@@ -663,7 +720,9 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
   if (warp == 1) tmem_free(tmem, 512);
 }
 
-template <int D> constexpr size_t q_smem() { return 1024 + (2 + 2 * ST) * (size_t)BR * D * 2 + 16 * 8 + 16; }
+template <int D> constexpr size_t q_smem() {
+  return 1024 + (2 + 2 * ST) * (size_t)BR * D * 2 + 6 * BR * 4 + 16 * 8 + 16;
+}
 template <int D> constexpr size_t kv_smem() {
   return 1024 + (2 + 2 * ST) * (size_t)BR * D * 2 + 2 * ST * BR * 4 + 16 * 8 + 16;
 }
