@@ -20,10 +20,10 @@
 //   k_sbwd_cvt   : fp16 copies of q, k, v
 //   k_sbwd_amax  : max |dO| over the call, k_sbwd_do: the scaled fp16 dO
 //   k_sbwd_q_tc  : 128 query rows of one frame-head, three passes over the
-//                  key tiles: (A) S = Q K^T, row max and sum -> LSE; (B) P as
-//                  fp16 over S in TMEM, O += P V -> o, then dg and Delta in
-//                  fp32 from o, dy and g; (C) S and dP = dO V^T, dS = P (dP -
-//                  Delta) over S, dQ += dS K.
+//                  key tiles: (A) S = Q K^T, the row max m; (B) P = 2^(s c - m c)
+//                  as fp16 over S in TMEM, O += P V and the row sum l -> LSE and
+//                  o = O / l, then dg and Delta in fp32 from o, dy and g; (C) S
+//                  and dP = dO V^T, dS = P (dP - Delta) over S, dQ += dS K.
 //   k_sbwd_kv_tc : 128 key rows of one frame-head, over every query tile that
 //                  sees the key frame (the mask is symmetric): S^T = K Q^T,
 //                  dP^T = V dO^T, P^T and dS^T over them, dV += P^T dO,
@@ -376,9 +376,9 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
     const bool valid = row < qvalid;
     const long long grow = (long long)(q0 + row) * dm.H + h;
     const float sc = do_scale(ws.amax);
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY;
     bool ok = true;
-    // ---- pass A: this half's row max and sum of 2^(s c)
+    // ---- pass A: this half's row max of the scores (no exponentials)
     for (int s = 0; ok && s < nt; ++s) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + (s & 1)), (s >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
@@ -390,31 +390,19 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
         float v[32];
         tmem_ld32(la + sbuf(s) + 32 * q, v);
         tmem_wait_ld();
-        float mx = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, 32 * q + i < kv ? v[i] : -INFINITY);
-        const float mn = fmaxf(m, mx);
-        if (mn != -INFINITY) {
-          float sum = 0.f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sum += 32 * q + i < kv ? ex2((v[i] - mn) * c) : 0.f;
-          l = (m == -INFINITY ? 0.f : l * ex2((m - mn) * c)) + sum;
-          m = mn;
-        }
+        for (int i = 0; i < 32; ++i) m = fmaxf(m, 32 * q + i < kv ? v[i] : -INFINITY);
       }
       tc_fence_before();
       mbar_arrive_warp(bar(B_SDONE));
     }
-    // the two halves of each row combined (every softmax warp reaches this barrier)
+    // the row max over both halves (every softmax warp reaches this barrier);
+    // finite: the first key of every tile is valid
     red[half * BR + row] = m;
-    red[2 * BR + half * BR + row] = l;
     softmax_bar();
-    const float mo = red[(1 - half) * BR + row], lo = red[2 * BR + (1 - half) * BR + row];
-    const float mm = fmaxf(m, mo);
-    const float lt = (m == -INFINITY ? 0.f : l * ex2((m - mm) * c)) + (mo == -INFINITY ? 0.f : lo * ex2((mo - mm) * c));
-    const float lse2 = mm * c + __log2f(lt);
-    if (ok && valid && half == 0) ws.lse2[grow] = lse2;
-    // ---- pass B: P (fp16) over S for O += P V
+    const float mc = fmaxf(m, red[(1 - half) * BR + row]) * c;
+    // ---- pass B: P = 2^(s c - m c) <= 1 (fp16) over S for O += P V; the row sum l
+    float l = 0.f;
     for (int s = nt; ok && s < nab; ++s) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + (s & 1)), (s >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
@@ -427,18 +415,28 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
         tmem_ld32(la + sbuf(s) + 32 * q, v);
         tmem_wait_ld();
         uint32_t pk[16];
+        float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int k = 32 * q + 2 * i;
-          pk[i] = pack_h2(k < kv ? ex2(fmaf(v[2 * i], c, -lse2)) : 0.f,
-                          k + 1 < kv ? ex2(fmaf(v[2 * i + 1], c, -lse2)) : 0.f);
+          const float p0 = k < kv ? ex2(fmaf(v[2 * i], c, -mc)) : 0.f;
+          const float p1 = k + 1 < kv ? ex2(fmaf(v[2 * i + 1], c, -mc)) : 0.f;
+          ps0 += p0;
+          ps1 += p1;
+          pk[i] = pack_h2(p0, p1);
         }
+        l += ps0 + ps1;
         tmem_st16(la + sbuf(s) + pk_col(q), pk);  // inside this half's columns, behind its reads
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(bar(B_SDONE));
     }
+    red[2 * BR + half * BR + row] = l;
+    softmax_bar();
+    l += red[2 * BR + (1 - half) * BR + row];
+    const float lse2 = mc + __log2f(l), inv_l = 1.0f / l;
+    if (ok && valid && half == 0) ws.lse2[grow] = lse2;
     // ---- o: dg = dy o sigmoid'(g), Delta = <dy sigmoid(g), o>, this half's columns
     float del = 0.f;
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar(B_ODONE), 0, ctl))) {
@@ -452,6 +450,8 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
         float o[32];
         tmem_ld32(la + COL_ACC + 32 * q, o);
         tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] *= inv_l;
         if (valid) {
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
