@@ -231,8 +231,9 @@ __global__ void __launch_bounds__(256) k_sbwd_do(Dims dm, Inputs in, const void*
 // TMEM: S buffers 0 and 1 at columns 0 and 384, dP at 128, and at 256 the
 // accumulator of the pass: O in pass B, dQ in pass C (O is read out before
 // the first dQ product, which waits for the softmax of pass C's first tile).
-// Passes A and B alternate the S buffers, so the product of tile s + 1 runs
-// while the softmax works on tile s; pass C uses buffer 0 and dP.
+// Every pass alternates the S buffers, so the product of tile s + 1 runs
+// while the softmax works on tile s (in pass C, dP of tile s + 1 waits for
+// the softmax of s, then the softmax of s + 1 overlaps dQ(s) and S(s + 2)).
 template <int D, typename Ty>
 __global__ void __launch_bounds__(kThr, 1)
 k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* dgate,
@@ -350,19 +351,36 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
         if (s + 2 < nab) ok = issue_s(s + 2);
       }
       if (ok) mma_commit(bar(B_ODONE));
-      for (int s = nab; ok && s < nsteps; ++s) {
-        const int st = s % ST;
-        ok = mbar_wait(bar(B_FULL + st), (s / ST) & 1, ctl);
-        if (!ok) break;
+      // pass C: S(s) into buffer s & 1 as soon as the buffer's dS was read by
+      // dQ, dP(s + 1) right after the softmax of s, then dQ(s): the softmax of
+      // s + 1 starts while dQ(s) and S(s + 2) run
+      auto wait_full = [&](int s) {
+        if (!mbar_wait(bar(B_FULL + s % ST), (s / ST) & 1, ctl)) return false;
         tc_fence_after();
-        gemm_t(tmem, qd, dadd(kd0, st * TILE));
-        gemm_t(tmem + COL_P, dod, dadd(vd0, st * TILE));
-        mma_commit(bar(B_SFULLC));
+        return true;
+      };
+      if (ok && nsteps > nab) {
+        ok = wait_full(nab);
+        if (ok) {
+          gemm_t(tmem + sbuf(nab), qd, dadd(kd0, (nab % ST) * TILE));
+          gemm_t(tmem + COL_P, dod, dadd(vd0, (nab % ST) * TILE));
+          mma_commit(bar(B_SFULLC));
+          if (nab + 1 < nsteps && (ok = wait_full(nab + 1)))
+            gemm_t(tmem + sbuf(nab + 1), qd, dadd(kd0, ((nab + 1) % ST) * TILE));
+        }
+      }
+      for (int s = nab; ok && s < nsteps; ++s) {
         ok = mbar_wait(bar(B_SDONE), s & 1, ctl);
         if (!ok) break;
         tc_fence_after();
-        gemm_ts(tmem + COL_ACC, tmem, dadd(kmn0, st * TILE), s == nab);  // dQ += dS K
-        mma_commit(bar(B_EMPTY + st));
+        if (s + 1 < nsteps) {  // its stage was waited for with S(s + 1)
+          gemm_t(tmem + COL_P, dod, dadd(vd0, ((s + 1) % ST) * TILE));
+          mma_commit(bar(B_SFULLC));
+        }
+        gemm_ts(tmem + COL_ACC, tmem + sbuf(s), dadd(kmn0, (s % ST) * TILE), s == nab);  // dQ += dS K
+        mma_commit(bar(B_EMPTY + s % ST));
+        if (s + 2 < nsteps && (ok = wait_full(s + 2)))
+          gemm_t(tmem + sbuf(s + 2), qd, dadd(kd0, ((s + 2) % ST) * TILE));
       }
       mma_commit(bar(B_DQ));
       mma_commit(bar(B_DRAIN));
@@ -487,7 +505,7 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
       for (int qq = 0; qq < 2; ++qq) {
         const int q = 2 * half + qq;
         float vs[32], vp[32];
-        tmem_ld32(la + 32 * q, vs);
+        tmem_ld32(la + sbuf(s) + 32 * q, vs);
         tmem_ld32(la + COL_P + 32 * q, vp);
         tmem_wait_ld();
         uint32_t pk[16];
@@ -498,7 +516,7 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
           const float p1 = k + 1 < kv ? ex2(fmaf(vs[2 * i + 1], c, -lse2)) : 0.f;
           pk[i] = pack_h2(p0 * (vp[2 * i] - dels), p1 * (vp[2 * i + 1] - dels));
         }
-        tmem_st16(la + pk_col(q), pk);
+        tmem_st16(la + sbuf(s) + pk_col(q), pk);
       }
       tmem_wait_st();
       tc_fence_before();
