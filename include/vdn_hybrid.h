@@ -251,8 +251,12 @@ const char *vdn_status_string(vdn_status s);
  * write matrices and S_x / 2 are taken from there, not recomputed.
  * Reads cfg (update must be 0 and d_k 32, 64 or 128, else VDN_ERR_UNSUPPORTED)
  * and args q, k, v, beta, alpha, gate_lin, rms_weight, fwd_init, workspace
- * (y, gate_sm and the text pointers are ignored).  Computes in fp32 (SIMT) for
- * both input dtypes. */
+ * (y, gate_sm and the text pointers are ignored).  Computes in fp32: SIMT
+ * kernels, except the per-token products of the frame write's gradient
+ * (dk, dv, dbeta), which run on the tensor cores for VDN_BF16 inputs with d_k
+ * 64 or 128 (the fp32 d x d factors as bf16 hi + lo pairs).  The call clears
+ * and uses the status words at the head of args->workspace
+ * (vdn_hybrid_device_status reads them). */
 typedef struct {
   const void *dy;      /* dL/dy in y's shape (per cfg.out_mode) and cfg.y_dtype; 16-byte aligned */
   float *dq, *dk, *dv; /* [B,T,N,H,d] float32, overwritten; anchor frames' dk, dv are zero    */

@@ -325,10 +325,10 @@ vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* 
   // the forward's choice of write form (B_t or C_t in the C_t slot)
   w.bform = (scan_tc_supported(d) && w.M16 != nullptr) ? 1 : 0;
   LinBwdArgs a{g->dy, g->dq, g->dk, g->dv, g->dbeta, g->dalpha, g->dgate_lin, g->drms_weight, g->dfwd_init,
-               g->workspace};
-  return launch_lin_bwd(d, inputs_of(args), w, a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? VDN_OK
-             : VDN_ERR_CUDA;
+               g->workspace, w.status};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(w.status, 0, 256, s) != cudaSuccess) return VDN_ERR_CUDA;
+  return launch_lin_bwd(d, inputs_of(args), w, a, s) == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
 }
 
 size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {

@@ -21,7 +21,7 @@ struct Dims {
 };
 
 // Device-side status words at the head of the workspace.
-enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4, TAG_COMPOSE_TC = 5, TAG_SMBWD_TC = 6 };
+enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4, TAG_COMPOSE_TC = 5, TAG_SMBWD_TC = 6, TAG_LINBWD_TC = 7 };
 
 struct Work {
   uint32_t* status;
@@ -107,11 +107,17 @@ struct LinBwdArgs {
   const void* dy;  // gradient of y, y's layout and dtype (the linear slot is read)
   float *dq, *dk, *dv, *dbeta, *dalpha, *dgate, *drms, *dfwd;  // drms, dfwd may be null
   void* workspace;
+  uint32_t* status;  // bounded-wait status words of the tensor-core kernels (cleared by the caller)
 };
 // bytes of the backward's scratch; off[0..5] (if not null) get the offsets of
 // the all-frame states F, G, the per-frame dR, dXf, dXb and the RMS partials
 size_t lin_bwd_workspace(const Dims& d, size_t* off);
 cudaError_t launch_lin_bwd(const Dims& d, const Inputs& in, const Work& w, const LinBwdArgs& a, cudaStream_t s);
+// its per-token step on the tensor cores (vdn_lin_bwd_tc.cu): bf16 k, v, d = 64 or 128;
+// dAs = dA + dA^T and dB per frame-head [B,T,H,d,d]; clears and fills dbeta
+bool bwd_tokens_tc_supported(const Dims& d);
+cudaError_t launch_bwd_tokens_tc(const Dims& d, const Inputs& in, const float* dAs, const float* dB, float* dk,
+                                 float* dv, float* dbeta, uint32_t* status, cudaStream_t s);
 
 // Backward of the windowed softmax branch (vdn_sm_bwd.cu)
 struct SmBwdArgs {

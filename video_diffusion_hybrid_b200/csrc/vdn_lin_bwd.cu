@@ -19,7 +19,8 @@
 //   k_bwd_frame   : dA_t = -(F_{t+1}^T dXf_t + G_t^T dXb_t) symmetrised,
 //                   dB_t = dXf_t + dXb_t, dalpha_t
 //   k_bwd_tokens  : dk = beta ((dA + dA^T) k + dB^T v), dv = beta dB k,
-//                   dbeta = k^T dA k + v^T dB k
+//                   dbeta = k^T dA k + v^T dB k (SIMT; for bf16 k, v with d = 64
+//                   or 128 the tensor-core form in vdn_lin_bwd_tc.cu runs instead)
 //   k_bwd_rms     : the RMS weight's gradient, summed over frames and batch
 #include "vdn_internal.h"
 #include "simt_common.cuh"
@@ -42,6 +43,7 @@ struct BwdWork {
 struct Grads {
   const void* dy;
   float *dq, *dk, *dv, *dbeta, *dalpha, *dgate, *drms, *dfwd;
+  uint32_t* status;
 };
 
 // The states a query of frame t reads: F[read_lo] + G[read_hi].
@@ -648,9 +650,14 @@ cudaError_t launch_all(const Dims& d, const Inputs& in, const Work& w, const Bwd
   if ((e = set_smem(k_bwd_frame<D>, frame_smem<D>())) != cudaSuccess) return e;
   k_bwd_frame<D><<<frames, kBT, frame_smem<D>(), s>>>(d, bw, g.dalpha);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = set_smem(k_bwd_tokens<Ti, D>, tokens_smem<D>())) != cudaSuccess) return e;
-  k_bwd_tokens<Ti, D><<<frames, kBT, tokens_smem<D>(), s>>>(d, in, bw, g);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (bwd_tokens_tc_supported(d)) {
+    e = launch_bwd_tokens_tc(d, in, bw.dXf, bw.dXb, g.dk, g.dv, g.dbeta, g.status, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    if ((e = set_smem(k_bwd_tokens<Ti, D>, tokens_smem<D>())) != cudaSuccess) return e;
+    k_bwd_tokens<Ti, D><<<frames, kBT, tokens_smem<D>(), s>>>(d, in, bw, g);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   if (g.drms != nullptr) {
     k_bwd_rms<D><<<d.H, 128, 0, s>>>(d, bw.dwp, g.drms);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -695,7 +702,7 @@ cudaError_t launch_lin_bwd(const Dims& d, const Inputs& in, const Work& w, const
   bw.dXf = reinterpret_cast<float*>(base + off[3]);
   bw.dXb = reinterpret_cast<float*>(base + off[4]);
   bw.dwp = a.drms ? reinterpret_cast<float*>(base + off[5]) : nullptr;
-  Grads g{a.dy, a.dq, a.dk, a.dv, a.dbeta, a.dalpha, a.dgate, a.drms, a.dfwd};
+  Grads g{a.dy, a.dq, a.dk, a.dv, a.dbeta, a.dalpha, a.dgate, a.drms, a.dfwd, a.status};
   switch (d.dk) {
     case 32: return launch_d<32>(d, in, w, bw, g, s);
     case 64: return launch_d<64>(d, in, w, bw, g, s);
