@@ -252,9 +252,10 @@ const char *vdn_status_string(vdn_status s);
  * Reads cfg (update must be 0 and d_k 32, 64 or 128, else VDN_ERR_UNSUPPORTED)
  * and args q, k, v, beta, alpha, gate_lin, rms_weight, fwd_init, workspace
  * (y, gate_sm and the text pointers are ignored).  Computes in fp32: SIMT
- * kernels, except the per-token products of the frame write's gradient
- * (dk, dv, dbeta), which run on the tensor cores for VDN_BF16 inputs with d_k
- * 64 or 128 (the fp32 d x d factors as bf16 hi + lo pairs).  The call clears
+ * kernels, except the per-token products, which run on the tensor cores for
+ * VDN_BF16 inputs (the fp32 d x d factors and dO as bf16 hi + lo pairs): the
+ * frame write's gradient (dk, dv, dbeta) at d_k 64 or 128, and the read's
+ * (o again, dq, the per-frame dR) at d_k 128.  The call clears
  * and uses the status words at the head of args->workspace
  * (vdn_hybrid_device_status reads them). */
 typedef struct {

@@ -116,6 +116,12 @@ cudaError_t launch_lin_bwd(const Dims& d, const Inputs& in, const Work& w, const
 // its per-token step on the tensor cores (vdn_lin_bwd_tc.cu): bf16 k, v, d = 64 or 128;
 // dAs = dA + dA^T and dB per frame-head [B,T,H,d,d]; clears and fills dbeta
 bool bwd_tokens_tc_supported(const Dims& d);
+// its read step on the tensor cores (vdn_lin_bwd_read_tc.cu): bf16, d = 128;
+// Fst/Gst every state [B,H,T+1,d,d]; writes dq, dgate, dRp [B,T,H,d,d] and
+// (if dwp) the RMS weight partials [B,T,H,d]
+bool bwd_read_tc_supported(const Dims& d);
+cudaError_t launch_bwd_read_tc(const Dims& d, const Inputs& in, const float* Fst, const float* Gst, const void* dy,
+                               float* dq, float* dgate, float* dRp, float* dwp, uint32_t* status, cudaStream_t s);
 cudaError_t launch_bwd_tokens_tc(const Dims& d, const Inputs& in, const float* dAs, const float* dB, float* dk,
                                  float* dv, float* dbeta, uint32_t* status, cudaStream_t s);
 

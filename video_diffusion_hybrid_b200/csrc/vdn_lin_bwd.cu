@@ -13,6 +13,8 @@
 //   k_bwd_states  : every F_j and G_j (the forward keeps chunk snapshots only)
 //   k_bwd_read    : RMSNorm / gate backward, dq = R^T do, dR_t = sum do q^T,
 //                   per query frame t; the RMS weight's per-frame partials
+//                   (SIMT; for bf16 with d = 128 the tensor-core form in
+//                   vdn_lin_bwd_read_tc.cu runs instead)
 //   k_bwd_adjoint : lambda_j = dL/dF_j from j = T down, mu_j = dL/dG_j from
 //                   j = 0 up; per written frame the products lambda_{t+1} M_t
 //                   and mu_t M_t (dX of the frame's two writes)
@@ -641,9 +643,14 @@ cudaError_t launch_all(const Dims& d, const Inputs& in, const Work& w, const Bwd
   if ((e = set_smem(k_bwd_states<D>, Chain<D>::smem)) != cudaSuccess) return e;
   k_bwd_states<D><<<chain, kBT, Chain<D>::smem, s>>>(d, in, w, bw);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = set_smem(k_bwd_read<Ti, Ty, D>, read_smem<D>())) != cudaSuccess) return e;
-  k_bwd_read<Ti, Ty, D><<<frames, kBT, read_smem<D>(), s>>>(d, in, w, bw, g);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (bwd_read_tc_supported(d)) {
+    e = launch_bwd_read_tc(d, in, bw.Fst, bw.Gst, g.dy, g.dq, g.dgate, bw.dRp, bw.dwp, g.status, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    if ((e = set_smem(k_bwd_read<Ti, Ty, D>, read_smem<D>())) != cudaSuccess) return e;
+    k_bwd_read<Ti, Ty, D><<<frames, kBT, read_smem<D>(), s>>>(d, in, w, bw, g);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   if ((e = set_smem(k_bwd_adjoint<D>, Chain<D>::smem)) != cudaSuccess) return e;
   k_bwd_adjoint<D><<<chain, kBT, Chain<D>::smem, s>>>(d, in, w, bw, g.dfwd);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
