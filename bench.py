@@ -629,7 +629,8 @@ def bwd_work(s, bf16: bool):
 
 def run_bwd(args):
     """The core's backward at the workload's size: one forward (which leaves
-    M_t and the write matrices in the workspace), then the timed steps, each
+    M_t and the write matrices in the workspace and the softmax log-sum-exp
+    in its own buffer), then the timed steps, each
     one call of each branch's backward for a fixed upstream gradient dy: the
     linear branch (gradients of q, k, v, beta, alpha, gate_lin, the RMS weight)
     and the windowed softmax branch (q, k, v, gate_sm).  Each branch is timed
@@ -643,7 +644,7 @@ def run_bwd(args):
     s = w.shape
     t = make_inputs_torch(s, w.seed, w.dtype, "cuda")
     cfg = cfg_for(s, w.dtype)
-    ha = HybridAttention(cfg)
+    ha = HybridAttention(cfg, keep_lse=True)  # the forward keeps the softmax log-sum-exp for the backward
     ha(t)
     gen = torch.Generator(device="cuda").manual_seed(w.seed + 1)
     dy = torch.randn(output_shape(cfg), generator=gen, device="cuda")
@@ -651,7 +652,7 @@ def run_bwd(args):
     lg = L.make_lin_grads(dy, g["dq"], g["dk"], g["dv"], g["dbeta"], g["dalpha"], g["dgate_lin"],
                           ha.bwd_workspace, drms_weight=g["drms_weight"])
     gs = ha.softmax_backward(t, dy)
-    sg = L.make_sm_grads(dy, gs["dq"], gs["dk"], gs["dv"], gs["dgate_sm"], ha.sm_workspace)
+    sg = L.make_sm_grads(dy, gs["dq"], gs["dk"], gs["dv"], gs["dgate_sm"], ha.sm_workspace, sm_lse=ha.sm_lse)
     a = ha.args(t)
     for _ in range(max(args.warmup, 3)):
         L.vdn_hybrid_lin_bwd(cfg, a, lg)

@@ -130,6 +130,11 @@ typedef struct {
                                       starts.  Anchor query frames then read
                                       fwd_init + S_x / 2.  16-byte aligned, outside the
                                       workspace.                                           */
+  float *sm_lse;                   /* [B,T,N,H] optional output of the forward's softmax
+                                      stage: ln sum_j exp(s q k_j) over each query row's
+                                      allowed keys, float32, 4-byte aligned; NULL = not
+                                      written.  vdn_hybrid_sm_bwd takes it (grads->sm_lse)
+                                      to skip recomputing the row statistics.              */
 } vdn_hybrid_args;
 
 /* Pipeline stages; vdn_hybrid_attn_fwd runs VDN_STAGE_ALL in this order. */
@@ -315,6 +320,11 @@ typedef struct {
   void *workspace;     /* scratch (status words, operand copies, dO, log-sum-exp and <dO, o> per
                           query row); 256-byte aligned                                        */
   size_t workspace_bytes; /* >= vdn_hybrid_sm_bwd_workspace_size(cfg)                           */
+  const float *sm_lse; /* [B,T,N,H] or NULL: the forward's args->sm_lse for these inputs.  On the
+                          tensor-core path it replaces the pass that recomputes each row's
+                          maximum score (the log-sum-exp bounds every score, so it serves as the
+                          exponent reference; the row sums are still formed here); the SIMT
+                          path does not read it.  4-byte aligned                               */
 } vdn_sm_grads;
 
 /* Bytes of scratch for cfg (the larger of its two layouts: four fp16 rows of d and two

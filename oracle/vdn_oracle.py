@@ -428,6 +428,23 @@ def softmax_dense_masked(q_bh, k_bh, v_bh, T, N, chunk, anchors, scale):
 # ---------------------------------------------------------------------------
 # the whole core
 # ---------------------------------------------------------------------------
+def softmax_lse(inp: dict, cfg: Cfg) -> np.ndarray:
+    """[B, T, N, H]: the log-sum-exp ln sum_j exp(s q . k_j) of every query row
+    over the keys its mask allows ([P1] 二; the normaliser of the softmax
+    branch, which a backward pass reuses)."""
+    allowed = frame_mask(cfg.T, cfg.chunk, cfg.anchors)
+    out = np.empty((cfg.B, cfg.T, cfg.N, cfg.H))
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            for t in range(cfg.T):
+                keys = np.flatnonzero(allowed[t])
+                K = np.asarray(inp["k"][b, keys, :, h], F64).reshape(len(keys) * cfg.N, -1)
+                S = cfg.scale * (np.asarray(inp["q"][b, t, :, h], F64) @ K.T)
+                m = S.max(axis=1)
+                out[b, t, :, h] = m + np.log(np.exp(S - m[:, None]).sum(axis=1))
+    return out
+
+
 def head_states(inp: dict, cfg: Cfg, b: int, h: int):
     """F, G (forward / backward states for every frame boundary) of one
     (batch, head), both started from half the text state; with

@@ -281,3 +281,51 @@ def test_sm_bwd_full_size_one_key_frame():
         assert e <= TOL["bf16"], (n, e)
     del t, g, ha, dy
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dtype,d", [("f32", 32), ("bf16", 64), ("bf16", 128)])
+def test_forward_softmax_lse_matches_oracle(dtype, d):
+    """The forward's optional log-sum-exp output (args.sm_lse) against the
+    oracle's. fp32 (SIMT): 1e-5 absolute. bf16 (tensor cores): the row sum adds
+    bf16-rounded weights (each within 2^-9 relative), so the log is within
+    about 2^-9; the bar is 2^-7."""
+    shape = Shape(B=1, T=12, N=40, H=2, d_k=d, d_v=d, L=0)
+    inp = make_inputs(shape, 81, dtype)
+    cfg = cfg_for(shape, dtype, softmax_scale=3.0)
+    t = to_torch(inp, dtype, "cuda")
+    ha = HybridAttention(cfg, keep_lse=True)
+    ha(t)
+    torch.cuda.synchronize()
+    err = np.max(np.abs(ha.sm_lse.cpu().numpy() - O.softmax_lse(inp, _ocfg(cfg))))
+    print("lse max abs error", err)
+    assert err <= (1e-5 if dtype == "f32" else 2.0 ** -7)
+
+
+@pytest.mark.parametrize("shape,opts", [
+    (Shape(B=1, T=12, N=40, H=2, d_k=128, d_v=128, L=0), dict(y_dtype=L.VDN_BF16)),
+    (Shape(B=2, T=15, N=33, H=3, d_k=64, d_v=64, L=0), dict()),
+    (Shape(B=1, T=23, N=300, H=2, d_k=128, d_v=128, L=0), dict(anchors=0, softmax_scale=10.0)),
+])
+def test_sm_bwd_with_forward_lse_matches_oracle(shape, opts):
+    """The tensor-core softmax backward given the forward's log-sum-exp (no
+    row-max pass): the same bar as without, and close to the result without."""
+    inp = make_inputs(shape, 61, "bf16")
+    cfg = cfg_for(shape, "bf16", **opts)
+    t = to_torch(inp, "bf16", "cuda")
+    dy = _dy(cfg, 62)
+    tdt = torch.bfloat16 if cfg.y_dtype == L.VDN_BF16 else torch.float32
+    dyt = torch.from_numpy(dy.astype(np.float32)).to(tdt).cuda()
+    ha = HybridAttention(cfg, keep_lse=True)
+    ha(t)
+    g = {k: v.clone() for k, v in ha.softmax_backward(t, dyt).items()}
+    torch.cuda.synchronize()
+    assert ha.softmax_backward_status()[0] == L.VDN_OK
+    plain = HybridAttention(cfg).softmax_backward(t, dyt)
+    torch.cuda.synchronize()
+    ref = OG.softmax_branch_grads(inp, _ocfg(cfg), _sm_slot(cfg, dy))
+    for n in ("q", "k", "v", "gate_sm"):
+        got = g["d" + n].cpu().numpy().astype(np.float64)
+        e = _rel(got, ref[n])
+        e2 = _rel(got, plain["d" + n].cpu().numpy().astype(np.float64))
+        print(n, f"{e:.2e} (vs without: {e2:.2e})")
+        assert e <= TOL["bf16"], (n, e)

@@ -630,3 +630,36 @@ def test_frame_rule_needs_its_rescaling_to_stay_non_expansive():
     assert np.linalg.norm(M, 2) <= 1 + 1e-12
     A = (beta[:, None] * K).T @ K
     assert np.linalg.norm(np.eye(8) - A, 2) > 1
+
+
+def test_softmax_lse_normalises_the_softmax_output():
+    """exp(s q.k - LSE) over the allowed keys are the softmax weights: they
+    sum to one and, times v and the gate, give the softmax slot of the output."""
+    shp = Shape(B=1, T=12, N=4, H=2, d_k=8, d_v=8, L=0)
+    inp = {k: np.asarray(v, np.float64) for k, v in make_inputs(shp, seed=31).items() if not k.endswith("_bits")}
+    cfg = O.Cfg(B=1, T=12, N=4, H=2, d_k=8, d_v=8, L=0, softmax_scale=2.0)
+    lse = O.softmax_lse(inp, cfg)
+    allowed = O.frame_mask(12, 5, 4)
+    y = O.hybrid_attn(inp, cfg)[..., 0, :]
+    for h in range(2):
+        for t in (0, 3, 7, 11):
+            keys = np.flatnonzero(allowed[t])
+            K = inp["k"][0, keys, :, h].reshape(-1, 8)
+            V = inp["v"][0, keys, :, h].reshape(-1, 8)
+            W = np.exp(2.0 * inp["q"][0, t, :, h] @ K.T - lse[0, t, :, h][:, None])
+            np.testing.assert_allclose(W.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(O.sigmoid(inp["gate_sm"][0, t, :, h]) * (W @ V), y[0, t, :, h], rtol=0,
+                                       atol=1e-12)
+
+
+def test_softmax_lse_two_keys_closed_form():
+    """T = 2 (both frames anchors) with one token per frame: each query sees
+    the two keys, LSE = ln(exp(s q.k0) + exp(s q.k1))."""
+    shp = Shape(B=1, T=2, N=1, H=1, d_k=4, d_v=4, L=0)
+    inp = {k: np.asarray(v, np.float64) for k, v in make_inputs(shp, seed=32).items() if not k.endswith("_bits")}
+    cfg = O.Cfg(B=1, T=2, N=1, H=1, d_k=4, d_v=4, L=0, softmax_scale=3.0)
+    lse = O.softmax_lse(inp, cfg)
+    for t in range(2):
+        q = inp["q"][0, t, 0, 0]
+        a, b = 3.0 * q @ inp["k"][0, 0, 0, 0], 3.0 * q @ inp["k"][0, 1, 0, 0]
+        assert abs(lse[0, t, 0, 0] - np.log(np.exp(a) + np.exp(b))) < 1e-13

@@ -42,7 +42,8 @@ class VdnArgs(C.Structure):
                 ("alpha", C.c_void_p), ("gate_sm", C.c_void_p), ("gate_lin", C.c_void_p),
                 ("text_k", C.c_void_p), ("text_v", C.c_void_p), ("text_beta", C.c_void_p),
                 ("init_state", C.c_void_p), ("rms_weight", C.c_void_p), ("y", C.c_void_p),
-                ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t), ("fwd_init", C.c_void_p)]
+                ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t), ("fwd_init", C.c_void_p),
+                ("sm_lse", C.c_void_p)]
 
 
 class VdnLinGrads(C.Structure):
@@ -56,7 +57,8 @@ class VdnLinGrads(C.Structure):
 class VdnSmGrads(C.Structure):
     """Mirror of ``vdn_sm_grads``."""
     _fields_ = [("dy", C.c_void_p), ("dq", C.c_void_p), ("dk", C.c_void_p), ("dv", C.c_void_p),
-                ("dgate_sm", C.c_void_p), ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t)]
+                ("dgate_sm", C.c_void_p), ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t),
+                ("sm_lse", C.c_void_p)]
 
 
 class ProjCfg(C.Structure):
@@ -221,14 +223,14 @@ def _ptr(t) -> int | None:
 
 def make_args(q, k, v, beta, alpha, gate_sm, gate_lin, y, workspace, workspace_bytes=None,
               text_k=None, text_v=None, text_beta=None, init_state=None, rms_weight=None,
-              fwd_init=None) -> VdnArgs:
+              fwd_init=None, sm_lse=None) -> VdnArgs:
     """Build a ``vdn_hybrid_args`` from torch tensors (or raw integer device
     pointers).  The caller keeps the tensors alive for the call."""
     if workspace_bytes is None:
         workspace_bytes = workspace.numel() * workspace.element_size()
     return VdnArgs(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(alpha), _ptr(gate_sm), _ptr(gate_lin),
                    _ptr(text_k), _ptr(text_v), _ptr(text_beta), _ptr(init_state), _ptr(rms_weight),
-                   _ptr(y), _ptr(workspace), int(workspace_bytes), _ptr(fwd_init))
+                   _ptr(y), _ptr(workspace), int(workspace_bytes), _ptr(fwd_init), _ptr(sm_lse))
 
 
 def _stream_handle(stream) -> int | None:
@@ -300,11 +302,12 @@ def vdn_hybrid_sm_bwd_workspace_size(cfg: HybridCfg) -> int:
     return int(lib().vdn_hybrid_sm_bwd_workspace_size(C.byref(c)))
 
 
-def make_sm_grads(dy, dq, dk, dv, dgate_sm, workspace, workspace_bytes=None) -> VdnSmGrads:
+def make_sm_grads(dy, dq, dk, dv, dgate_sm, workspace, workspace_bytes=None, sm_lse=None) -> VdnSmGrads:
     """Build a ``vdn_sm_grads`` from torch tensors (or raw device pointers)."""
     if workspace_bytes is None:
         workspace_bytes = workspace.numel() * workspace.element_size()
-    return VdnSmGrads(_ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate_sm), _ptr(workspace), int(workspace_bytes))
+    return VdnSmGrads(_ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgate_sm), _ptr(workspace), int(workspace_bytes),
+                      _ptr(sm_lse))
 
 
 def vdn_hybrid_sm_bwd(cfg: HybridCfg, args: VdnArgs, grads: VdnSmGrads, stream=None, check: bool = True) -> int:

@@ -48,7 +48,7 @@ class HybridAttention:
     """Calls ``vdn_hybrid_attn_fwd`` on torch tensors.  Workspace and output
     are allocated once (by torch) and reused."""
 
-    def __init__(self, cfg: L.HybridCfg, device="cuda"):
+    def __init__(self, cfg: L.HybridCfg, device="cuda", keep_lse: bool = False):
         self.cfg = cfg
         self.ws_bytes = L.vdn_hybrid_attn_workspace_size(cfg)
         if self.ws_bytes == 0:
@@ -57,12 +57,16 @@ class HybridAttention:
         self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
         tdt = torch.bfloat16 if cfg.y_dtype == L.VDN_BF16 else torch.float32
         self.y = torch.empty(output_shape(cfg), dtype=tdt, device=self.device)
+        # the forward's softmax log-sum-exp per query row, which the softmax
+        # backward then takes in place of recomputing the row statistics
+        self.sm_lse = (torch.empty((cfg.B, cfg.T, cfg.N, cfg.H), dtype=torch.float32, device=self.device)
+                       if keep_lse else None)
 
     def args(self, t: dict) -> L.VdnArgs:
         return L.make_args(t["q"], t["k"], t["v"], t["beta"], t["alpha"], t["gate_sm"], t["gate_lin"], self.y,
                            self.workspace, self.ws_bytes, text_k=t.get("text_k"), text_v=t.get("text_v"),
                            text_beta=t.get("text_beta"), init_state=t.get("init_state"),
-                           rms_weight=t.get("rms_weight"), fwd_init=t.get("fwd_init"))
+                           rms_weight=t.get("rms_weight"), fwd_init=t.get("fwd_init"), sm_lse=self.sm_lse)
 
     def __call__(self, t: dict, stages: int = L.STAGE_ALL, stream=None) -> torch.Tensor:
         a = self.args(t)
@@ -98,9 +102,10 @@ class HybridAttention:
         return g
 
     def softmax_backward(self, t: dict, dy: torch.Tensor, stream=None) -> dict:
-        """Gradients through the windowed softmax branch (no forward state is
-        read; the statistics are recomputed): float32 tensors dq, dk, dv,
-        dgate_sm."""
+        """Gradients through the windowed softmax branch: float32 tensors dq,
+        dk, dv, dgate_sm.  With keep_lse, the forward's log-sum-exp (kept by
+        the last forward call on the same inputs) replaces the recomputed row
+        statistics."""
         c = self.cfg
         if getattr(self, "sm_workspace", None) is None:
             nb = L.vdn_hybrid_sm_bwd_workspace_size(c)
@@ -110,7 +115,7 @@ class HybridAttention:
         f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=self.device)
         tok = (c.B, c.T, c.N, c.H)
         g = {"dq": f(*tok, c.d_k), "dk": f(*tok, c.d_k), "dv": f(*tok, c.d_v), "dgate_sm": f(*tok, c.d_v)}
-        sg = L.make_sm_grads(dy, g["dq"], g["dk"], g["dv"], g["dgate_sm"], self.sm_workspace)
+        sg = L.make_sm_grads(dy, g["dq"], g["dk"], g["dv"], g["dgate_sm"], self.sm_workspace, sm_lse=self.sm_lse)
         L.vdn_hybrid_sm_bwd(c, self.args(t), sg, stream)
         return g
 

@@ -96,6 +96,7 @@ vdn_status check_args(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a, unsigne
   }
   if (a->init_state && !aligned(a->init_state, 16)) return VDN_ERR_INVALID_ARG;
   if (a->rms_weight && !aligned(a->rms_weight, 4)) return VDN_ERR_INVALID_ARG;
+  if (a->sm_lse && !aligned(a->sm_lse, 4)) return VDN_ERR_INVALID_ARG;
   vdn_workspace_layout L;
   layout_of(c, &L);
   if (!a->workspace || !aligned(a->workspace, kAlign) || a->workspace_bytes < L.total) return VDN_ERR_WORKSPACE;
@@ -140,6 +141,7 @@ Inputs inputs_of(const vdn_hybrid_args* a) {
   in.text_k = a->text_k; in.text_v = a->text_v; in.text_beta = a->text_beta;
   in.init_state = a->init_state; in.rms_weight = a->rms_weight; in.y = a->y;
   in.fwd_init = a->fwd_init;
+  in.sm_lse = a->sm_lse;
   return in;
 }
 
@@ -347,6 +349,7 @@ vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* a
   for (const void* p : req)
     if (!p || !aligned(p, 16)) return VDN_ERR_INVALID_ARG;
   const Dims d = make_dims(cfg);
+  if (g->sm_lse && !aligned(g->sm_lse, 4)) return VDN_ERR_INVALID_ARG;
   if ((long long)d.T * d.N > (1LL << 40)) return VDN_ERR_UNSUPPORTED;
   if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < vdn_hybrid_sm_bwd_workspace_size(cfg))
     return VDN_ERR_WORKSPACE;
@@ -357,7 +360,7 @@ vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* a
     sm_bwd_tc_workspace(d, off);
     SmTcArgs a{g->dy, g->dq, g->dk, g->dv, g->dgate_sm, base + off[1], base + off[2], base + off[3], base + off[4],
                reinterpret_cast<float*>(base + off[5]), reinterpret_cast<float*>(base + off[6]),
-               reinterpret_cast<unsigned*>(base + off[7]), reinterpret_cast<uint32_t*>(base + off[0])};
+               reinterpret_cast<unsigned*>(base + off[7]), reinterpret_cast<uint32_t*>(base + off[0]), g->sm_lse};
     if (cudaMemsetAsync(base + off[0], 0, kAlign, s) != cudaSuccess ||
         cudaMemsetAsync(base + off[7], 0, kAlign, s) != cudaSuccess)
       return VDN_ERR_CUDA;

@@ -52,6 +52,7 @@ struct Inputs {
   const float *text_beta, *init_state, *rms_weight;
   void* y;
   const float* fwd_init;  // forward start state, or null (half the text state)
+  float* sm_lse;          // softmax log-sum-exp per query row [B*T*N, H] (natural log), or null
 };
 
 __host__ __device__ inline bool is_anchor(const Dims& d, int t) {
@@ -143,6 +144,7 @@ struct SmTcArgs {
   float *lse2, *delta;           // [B*T*N, H] scratch
   unsigned* amax;                // max |dO| (cleared by the caller)
   uint32_t* status;              // bounded-wait status words (cleared by the caller)
+  const float* lse_in;           // the forward's softmax log-sum-exp [B*T*N, H], or null
 };
 bool sm_bwd_tc_supported(const Dims& d);
 // bytes of its scratch; off[0..7] (if not null): status, q16, k16, v16, dO16, lse2, delta, amax

@@ -599,6 +599,8 @@ k_softmax(Dims dm, Inputs in, Work w) {
     if (tok >= ntok) continue;
     const float invl = 1.0f / lrow[rr];
     const long long row = bq + (long long)f0 * dm.N + tok;
+    if (in.sm_lse != nullptr && lane == 0)  // natural log of the row's sum of exp(s q k)
+      in.sm_lse[row * dm.H + h] = (mrow[rr] + log2f(lrow[rr])) * 0.6931471805599453f;
 #pragma unroll
     for (int u = 0; u < DPL; ++u) {
       const int i = lane + 32 * u;

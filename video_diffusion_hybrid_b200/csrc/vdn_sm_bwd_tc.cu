@@ -24,6 +24,9 @@
 //                  as fp16 over S in TMEM, O += P V and the row sum l -> LSE and
 //                  o = O / l, then dg and Delta in fp32 from o, dy and g; (C) S
 //                  and dP = dO V^T, dS = P (dP - Delta) over S, dQ += dS K.
+//                  Given the forward's log-sum-exp, pass A is skipped and pass
+//                  B takes it as the reference in place of m (P stays <= 1; l
+//                  and with it o and LSE are still formed here).
 //   k_sbwd_kv_tc : 128 key rows of one frame-head, over every query tile that
 //                  sees the key frame (the mask is symmetric): S^T = K Q^T,
 //                  dP^T = V dO^T, P^T and dS^T over them, dV += P^T dO,
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(256) k_sbwd_do(Dims dm, Inputs in, const void*
 // the softmax of s, then the softmax of s + 1 overlaps dQ(s) and S(s + 2)).
 template <int D, typename Ty>
 __global__ void __launch_bounds__(kThr, 1)
-k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* dgate,
+k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* dgate, const float* lse_in,
             const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
             const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
   constexpr int NB = D / 64;
@@ -262,7 +265,8 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
   const int base = b * dm.T * dm.N;
   const int q0 = base + f * dm.N + n0, qvalid = min(BR, dm.N - n0);
   const Iv iv = intervals(dm, f, base);
-  const int nt = n_tiles(iv), nab = 2 * nt, nsteps = 3 * nt;
+  // with the forward's log-sum-exp (lse_in) there is no pass A
+  const int nt = n_tiles(iv), pa = lse_in != nullptr ? 0 : nt, nab = pa + nt, nsteps = pa + 2 * nt;
   const Ctl ctl{abort_flag, ws.status, (unsigned)TAG_SMBWD_TC};
   auto bar = [&](int i) { return smem_u32(bars + i); };
   auto sbuf = [](int s) { return (s & 1) ? 384u : 0u; };
@@ -288,9 +292,9 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
       }
       int issued = 0;
       for (int s = 0; s < nsteps; ++s) {
-        const bool withv = s >= nt;
+        const bool withv = s >= pa;
         int k0, kv;
-        tile_of(iv, s % nt, k0, kv);
+        tile_of(iv, s < pa ? s : (s < nab ? s - pa : s - nab), k0, kv);
         const int st = s % ST;
         if (s >= ST && !mbar_wait(bar(B_EMPTY + st), (s / ST - 1) & 1, ctl)) break;
         mbar_expect_tx(bar(B_FULL + st), withv ? 2 * TILE : TILE);
@@ -335,7 +339,7 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
         tc_fence_after();
         gemm_t(tmem + sbuf(s), qd, dadd(kd0, st * TILE));
         mma_commit(bar(B_SFULL + (s & 1)));
-        if (s < nt) mma_commit(bar(B_EMPTY + st));
+        if (s < pa) mma_commit(bar(B_EMPTY + st));
         return true;
       };
       bool ok = mbar_wait(bar(B_QD), 0, ctl) && issue_s(0) && (nab < 2 || issue_s(1));
@@ -343,8 +347,8 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
         ok = mbar_wait(bar(B_SDONE), s & 1, ctl);
         if (!ok) break;
         tc_fence_after();
-        if (s >= nt) {
-          gemm_ts(tmem + COL_ACC, tmem + sbuf(s), dadd(vmn0, (s % ST) * TILE), s == nt);  // O += P V
+        if (s >= pa) {
+          gemm_ts(tmem + COL_ACC, tmem + sbuf(s), dadd(vmn0, (s % ST) * TILE), s == pa);  // O += P V
           mma_commit(bar(B_EMPTY + s % ST));
         }
         // buffer s & 1 again: P(s) is read by the P V above, issued first
@@ -397,7 +401,7 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
     float m = -INFINITY;
     bool ok = true;
     // ---- pass A: this half's row max of the scores (no exponentials)
-    for (int s = 0; ok && s < nt; ++s) {
+    for (int s = 0; ok && s < pa; ++s) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + (s & 1)), (s >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       int k0, kv;
@@ -414,18 +418,25 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
       tc_fence_before();
       mbar_arrive_warp(bar(B_SDONE));
     }
-    // the row max over both halves (every softmax warp reaches this barrier);
-    // finite: the first key of every tile is valid
-    red[half * BR + row] = m;
-    softmax_bar();
-    const float mc = fmaxf(m, red[(1 - half) * BR + row]) * c;
-    // ---- pass B: P = 2^(s c - m c) <= 1 (fp16) over S for O += P V; the row sum l
+    // the exponent reference mc: the forward's log-sum-exp (in log2 units;
+    // it bounds every scaled score, rows past the frame take the tile's first
+    // row's), or the row max over both halves (every softmax warp reaches this
+    // barrier; finite: the first key of every tile is valid)
+    float mc;
+    if (pa == 0) {
+      mc = lse_in[(long long)(q0 + (valid ? row : 0)) * dm.H + h] * kLog2e;
+    } else {
+      red[half * BR + row] = m;
+      softmax_bar();
+      mc = fmaxf(m, red[(1 - half) * BR + row]) * c;
+    }
+    // ---- pass B: P = 2^(s c - mc) <= 1 (fp16) over S for O += P V; the row sum l
     float l = 0.f;
-    for (int s = nt; ok && s < nab; ++s) {
+    for (int s = pa; ok && s < nab; ++s) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + (s & 1)), (s >> 1) & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       int k0, kv;
-      tile_of(iv, s - nt, k0, kv);
+      tile_of(iv, s - pa, k0, kv);
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         const int q = 2 * half + qq;
@@ -772,7 +783,7 @@ cudaError_t launch_d(const Dims& d, const Inputs& in, const SmTcArgs& a, cudaStr
   auto kq = k_sbwd_q_tc<D, Ty>;
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem<D>())) != cudaSuccess)
     return e;
-  kq<<<(unsigned)items, kThr, q_smem<D>(), s>>>(d, in, a.dy, ws, a.dq, a.dgate, mq, mdo, mk, mv);
+  kq<<<(unsigned)items, kThr, q_smem<D>(), s>>>(d, in, a.dy, ws, a.dq, a.dgate, a.lse_in, mq, mdo, mk, mv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(k_sbwd_kv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv_smem<D>())) !=
       cudaSuccess)

@@ -510,6 +510,10 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       const bool valid = trow < tile.qrows;
       const long long tok = (long long)tile.q0 + trow;
       const long long gi = (tok * dm.H + tile.h) * D;
+      // the row's log-sum-exp, natural log (l_sum counts the row max at
+      // weight 2^(m - m_used) >= 1, so this bounds every scaled score)
+      if (!X && in.sm_lse != nullptr && valid)
+        in.sm_lse[tok * dm.H + tile.h] = (m_used * c + __log2f(l_sum)) * 0.6931471805599453f;
       To* y = static_cast<To*>(in.y) + ((!X && dm.out_mode == 0) ? 2 * gi : gi);
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
