@@ -86,6 +86,8 @@ CASES = [
     (Shape(B=1, T=12, N=40, H=2, d_k=128, d_v=128, L=8), "bf16", dict(y_dtype=L.VDN_BF16, fwd_init=True)),
     (Shape(B=2, T=15, N=33, H=3, d_k=64, d_v=64, L=4), "bf16", dict()),
     (Shape(B=1, T=10, N=20, H=1, d_k=128, d_v=128, L=0), "f32", dict(fwd_init=True)),
+    # bf16 d = 128 with a summed output: the tensor-core read backward reads dy itself
+    (Shape(B=1, T=16, N=150, H=2, d_k=128, d_v=128, L=6), "bf16", dict(out_mode=1)),
 ]
 
 
