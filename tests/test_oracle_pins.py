@@ -663,3 +663,16 @@ def test_softmax_lse_two_keys_closed_form():
         q = inp["q"][0, t, 0, 0]
         a, b = 3.0 * q @ inp["k"][0, 0, 0, 0], 3.0 * q @ inp["k"][0, 1, 0, 0]
         assert abs(lse[0, t, 0, 0] - np.log(np.exp(a) + np.exp(b))) < 1e-13
+
+
+@pytest.mark.parametrize("T", [2, 7, 10, 12, 23, 90, 102])
+@pytest.mark.parametrize("anchors", [0, 4])
+def test_frame_mask_is_symmetric(T, anchors):
+    """The window (chunks within one of each other) and the anchors (an anchor
+    frame sees and is seen by every frame) are symmetric relations: the query
+    frames that see key frame f are the frames f itself sees. The key-side
+    backward kernels of the softmax walk the query tiles of a key frame by
+    this."""
+    m = O.frame_mask(T, 5, anchors)
+    assert np.array_equal(m, m.T)
+    assert np.all(np.diag(m))
