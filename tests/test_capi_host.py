@@ -255,3 +255,16 @@ def test_sm_bwd_workspace_and_rejections():
     c = _cfg(update=2)
     assert L.vdn_hybrid_sm_bwd(c, _fake_args(c), L.make_sm_grads(**good), stream=0, check=False) == \
         L.VDN_ERR_UNSUPPORTED
+
+
+def test_sm_lse_pointers_validated_before_launch():
+    """The forward's optional log-sum-exp output and the softmax backward's
+    matching input: a misaligned pointer is refused before any launch."""
+    cfg = _cfg()
+    p = 1 << 26
+    assert L.vdn_hybrid_attn_fwd(cfg, _fake_args(cfg, sm_lse=(1 << 24) + 2), stream=0, check=False) == \
+        L.VDN_ERR_INVALID_ARG
+    good = dict(dy=p, dq=p, dk=p, dv=p, dgate_sm=p, workspace=p,
+                workspace_bytes=L.vdn_hybrid_sm_bwd_workspace_size(cfg))
+    g = L.make_sm_grads(**good, sm_lse=p + 2)
+    assert L.vdn_hybrid_sm_bwd(cfg, _fake_args(cfg), g, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
