@@ -59,3 +59,16 @@ def test_reference_arm_under_torchrun():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_backward_work_counts():
+    """The backward bench's pair count uses the mask density; it must be the
+    oracle's (19.975 % at T = 90), and the linear branch's algorithmic work
+    scales with the token-heads."""
+    import bench
+    from oracle import vdn_oracle as O
+    from video_diffusion_hybrid_b200.workloads import WORKLOADS
+    s = WORKLOADS["768p"].shape
+    assert abs(bench.O_density(s) - O.mask_density(s.T, 5, 4)) < 1e-15
+    f1, b1 = bench.bwd_work(s, True)
+    assert f1 > 4.5e11 and b1 == s.B * s.T * s.N * s.H * (4 * s.d_k * 2 + 4 + 4 * s.d_k + 16 * s.d_k + 4)
