@@ -254,7 +254,8 @@ const char *vdn_status_string(vdn_status s);
  * Precondition: args->workspace holds what vdn_hybrid_attn_fwd (or at least its
  * TEXT and SOLVE stages) wrote for the same cfg and the same inputs: M_t, the
  * write matrices and S_x / 2 are taken from there, not recomputed.
- * Reads cfg (update must be 0 and d_k 32, 64 or 128, else VDN_ERR_UNSUPPORTED)
+ * Reads cfg (update must be 0, d_k 32, 64 or 128 and T at most 65535, else
+ * VDN_ERR_UNSUPPORTED)
  * and args q, k, v, beta, alpha, gate_lin, rms_weight, fwd_init, workspace
  * (y, gate_sm and the text pointers are ignored).  Computes in fp32: SIMT
  * kernels, except the per-token products, which run on the tensor cores for
@@ -299,7 +300,8 @@ vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *
  * slot 0 of dy; out_mode 1: dy itself).  With vdn_hybrid_lin_bwd the two
  * branches' shares of dq, dk and dv add up to the whole core's gradient.
  * The exact derivative of the forward (the pages describe the forward only).
- * Reads cfg (update 0 and d_k 32, 64 or 128, else VDN_ERR_UNSUPPORTED) and
+ * Reads cfg (update 0, d_k 32, 64 or 128 and T at most 65535, else
+ * VDN_ERR_UNSUPPORTED) and
  * args q, k, v, gate_sm (the other pointers, the forward's workspace and its
  * output are not read: the softmax statistics and o are recomputed).  Two
  * implementations, chosen by cfg (vdn_hybrid_stage_impl(cfg,

@@ -198,8 +198,9 @@ def test_lin_bwd_workspace_size():
     dd = 128 * 128 * 4
     want = 2 * 24 * 91 * dd + 3 * 90 * 24 * dd + 90 * 24 * 128 * 4
     assert L.vdn_hybrid_lin_bwd_workspace_size(cfg) == want
-    for kw in (dict(update=1), dict(update=2), dict(d_k=256, d_v=256), dict(T=1)):
+    for kw in (dict(update=1), dict(update=2), dict(d_k=256, d_v=256), dict(T=1), dict(T=70000, N=8, H=2)):
         assert L.vdn_hybrid_lin_bwd_workspace_size(_cfg(**kw)) == 0
+        assert L.vdn_hybrid_sm_bwd_workspace_size(_cfg(**kw)) == 0
 
 
 def _fake_grads(cfg, **over):

@@ -150,6 +150,7 @@ vdn_status check_bwd_cfg(const vdn_hybrid_cfg* c) {
   vdn_status st = check_cfg(c);
   if (st != VDN_OK) return st;
   if (c->update != 0 || c->d_k > 128) return VDN_ERR_UNSUPPORTED;
+  if (c->T > 65535) return VDN_ERR_UNSUPPORTED;  // frames index a grid axis of the backward kernels
   return VDN_OK;
 }
 
