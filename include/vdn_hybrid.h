@@ -23,6 +23,10 @@
  *   c-1, c, c+1 (clipped at the ends), every query sees the anchor frames and
  *   anchor queries see every frame:  y_sm = sigmoid(g_sm) * softmax(s q K^T) V.
  *
+ *   The backward of both branches (vdn_hybrid_lin_bwd, vdn_hybrid_sm_bwd) is
+ *   the exact derivative of the forward above; the pages describe the forward
+ *   only.
+ *
  * Conventions for every entry point:
  *   - Ownership: the library allocates nothing.  The caller owns every input,
  *     the output and the workspace; all data pointers are DEVICE pointers on the
