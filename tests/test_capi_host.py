@@ -269,3 +269,31 @@ def test_sm_lse_pointers_validated_before_launch():
                 workspace_bytes=L.vdn_hybrid_sm_bwd_workspace_size(cfg))
     g = L.make_sm_grads(**good, sm_lse=p + 2)
     assert L.vdn_hybrid_sm_bwd(cfg, _fake_args(cfg), g, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+
+
+def _header_struct_fields(name):
+    """Field names, in order, of `typedef struct { ... } name;` in the header."""
+    src = open(os.path.join(ROOT, "include", "vdn_hybrid.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    m = re.search(r"typedef struct \{([^{}]*)\}\s*" + name + r"\s*;", src)
+    assert m, name
+    fields = []
+    for decl in m.group(1).split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        # "const void *q, *k, *v" -> q, k, v ; "size_t workspace_bytes" -> workspace_bytes
+        head, *rest = decl.split(",")
+        fields.append(re.findall(r"(\w+)\s*$", head)[0])
+        fields += [re.sub(r"[\s\*]", "", r) for r in rest]
+    return fields
+
+
+@pytest.mark.parametrize("cname,pystruct", [
+    ("vdn_hybrid_cfg", L.VdnCfg), ("vdn_hybrid_args", L.VdnArgs), ("vdn_lin_grads", L.VdnLinGrads),
+    ("vdn_sm_grads", L.VdnSmGrads), ("vdn_proj_cfg", L.ProjCfg), ("vdn_workspace_layout", L.VdnLayout),
+])
+def test_ctypes_mirrors_follow_the_header(cname, pystruct):
+    """The binding's structs list the header's fields in the same order (a
+    mismatch would hand the library wrong pointers)."""
+    assert [f for f, _ in pystruct._fields_] == _header_struct_fields(cname)
