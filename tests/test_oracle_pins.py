@@ -476,6 +476,80 @@ def test_quantize_e4m3_round_trip():
     assert O.quantize_e4m3(np.zeros(4))[1] == np.float32(1.0)
 
 
+def _e4m3_decode(codes):
+    """The value of each FP8 E4M3 byte from its bit fields, as the OCP 8-bit
+    floating point specification defines them: bit 7 the sign, bits 6..3 the
+    exponent with bias 7, bits 2..0 the mantissa; exponent 0 is subnormal
+    (m / 8 * 2^-6); there is no infinity, and S.1111.111 is NaN.  Written
+    from the format, not through any library conversion."""
+    out = np.empty(codes.shape, np.float64)
+    for idx, c in np.ndenumerate(np.asarray(codes, np.uint8)):
+        c = int(c)
+        sign = -1.0 if c & 0x80 else 1.0
+        e = (c >> 3) & 0xF
+        m = c & 0x7
+        if e == 0xF and m == 0x7:
+            out[idx] = np.nan
+        elif e == 0:
+            out[idx] = sign * (m / 8.0) * 2.0 ** -6
+        else:
+            out[idx] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return out
+
+
+def _e4m3_codes(byte_rows):
+    return torch.tensor(np.asarray(byte_rows, np.uint8)).view(torch.float8_e4m3fn)
+
+
+def test_e4m3_decoder_fixed_points():
+    """The bit-field decoder itself, on values the format fixes: the largest
+    finite code 0x7E = 448, the smallest normal 0x08 = 2^-6, the smallest
+    subnormal 0x01 = 2^-9, 1.0 = 0x38, -1.5 = 0xBC, and NaN at 0x7F."""
+    got = _e4m3_decode(np.array([0x7E, 0x08, 0x01, 0x38, 0xBC, 0x00, 0x80, 0x7F]))
+    np.testing.assert_array_equal(got[:7], [448.0, 2.0 ** -6, 2.0 ** -9, 1.0, -1.5, 0.0, -0.0])
+    assert np.isnan(got[7])
+
+
+def test_out_proj_fp8_hand_worked():
+    """A 2 x 3 by 3 x 2 product worked by hand.  y codes (row-major)
+    [1, 2, 0.5; -1, 1.5, 0] with s_y = 2, the transposed weight's codes
+    [1, 0, 2; 0.25, -1, 1] with s_w = 0.5.  Scaled: y = [2, 4, 1; -2, 3, 0],
+    w^T = [0.5, 0, 1; 0.125, -0.5, 0.5], so
+    out = [2*0.5 + 1*1, 2*0.125 - 4*0.5 + 1*0.5; -2*0.5, -2*0.125 - 3*0.5]
+        = [2, -1.25; -1, -1.75]."""
+    qy = _e4m3_codes([[0x38, 0x40, 0x30], [0xB8, 0x3C, 0x00]])
+    qw_t = _e4m3_codes([[0x38, 0x00, 0x40], [0x28, 0xB8, 0x38]])
+    got = O.out_proj_fp8(qy, np.float32(2.0), qw_t, np.float32(0.5))
+    np.testing.assert_array_equal(got, [[2.0, -1.25], [-1.0, -1.75]])
+
+
+def _out_proj_fp8_untransposed(qy, sy, qw_t, sw):
+    """A planted mistake: the weight codes taken as [K, N] (no transpose)."""
+    y = _e4m3_decode(qy.view(torch.uint8).numpy()) * float(sy)
+    w = _e4m3_decode(qw_t.view(torch.uint8).numpy()) * float(sw)
+    return y @ w
+
+
+@pytest.mark.parametrize("M,K,N", [(5, 7, 3), (9, 16, 16)])
+def test_out_proj_fp8_matches_bitfield_product(M, K, N):
+    """out_proj_fp8 equals the float64 product of the bit-field-decoded,
+    scaled codes, (s_y Y)(s_w W_t)^T, on random finite codes; non-square
+    shapes catch a transposed weight, and the square case shows that the
+    untransposed product differs."""
+    r = np.random.default_rng(M * 100 + K)
+    finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    cy = r.choice(finite, size=(M, K))
+    cw = r.choice(finite, size=(N, K))
+    sy, sw = np.float32(0.013), np.float32(3.25)
+    got = O.out_proj_fp8(_e4m3_codes(cy), sy, _e4m3_codes(cw), sw)
+    want = (_e4m3_decode(cy) * float(sy)) @ (_e4m3_decode(cw) * float(sw)).T
+    assert got.shape == (M, N)
+    np.testing.assert_allclose(got, want, rtol=1e-15, atol=1e-12 * np.abs(want).max())
+    if K == N:
+        wrong = _out_proj_fp8_untransposed(_e4m3_codes(cy), sy, _e4m3_codes(cw), sw)
+        assert np.abs(wrong - want).max() > 1e-3 * np.abs(want).max()
+
+
 # ----------------------------------------------------------- streaming ----
 def _tag_segment(frames, d, T):
     """One head, one token per frame: frame f (global index) carries the key
