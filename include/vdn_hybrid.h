@@ -213,12 +213,18 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg *cfg, const vdn_hybri
  * point; it is a deployment convenience of this library.
  * Scratch: a library-owned device array of VDN_NOALLOC_SCRATCH_BYTES (static
  * storage on every GPU that loads the library, held until the process exits).
+ * Those 16 MiB are reserved on each device where the library's module is
+ * loaded, whether or not this entry point is ever called; CUDA_MODULE_LOADING
+ * decides when that happens (at context creation when eager, at the library's
+ * first kernel launch or symbol lookup on that device when lazy).
  * Arguments are those of vdn_hybrid_attn_fwd, except that args->workspace must
  * be NULL and args->workspace_bytes 0 (else VDN_ERR_INVALID_ARG).  A cfg whose
  * workspace (vdn_hybrid_attn_workspace_size) exceeds VDN_NOALLOC_SCRATCH_BYTES
  * returns VDN_ERR_WORKSPACE and launches nothing.
- * Set-up: the first call on each device looks up the array's device address
- * with that device current; make that first call before any stream capture.
+ * Set-up: every call looks up the array's device address in the current
+ * device's context (so the address stays right after a device reset, which
+ * may move the array); the first call on a device may load the module, so
+ * make that first call before any stream capture.
  * Sharing: every call uses the same array, which keeps the last call's
  * contents (each call clears what must start at zero); calls whose work
  * overlaps on the GPU race on it and must be serialised by the caller.  The

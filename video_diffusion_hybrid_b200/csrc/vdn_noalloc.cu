@@ -13,8 +13,6 @@
 // every other scratch region is fully written before it is read.  Calls whose
 // kernels overlap on the GPU (two streams, two host threads, two devices'
 // worth of work aimed at one device) race on the array; serialise them.
-#include <mutex>
-
 #include "vdn_internal.h"
 
 namespace {
@@ -23,24 +21,16 @@ constexpr size_t kNoallocScratchBytes = VDN_NOALLOC_SCRATCH_BYTES;  // 16 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 128;
-void* g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mutex;
-
-// Device address of the array on the current device, looked up once per
-// device.  In host code `g_noalloc_scratch` names a host-side stand-in, not
-// device memory, so only this address may be given to a kernel.
+// Device address of the array in the current device's context.  In host code
+// `g_noalloc_scratch` names a host-side stand-in, not device memory, so only
+// this address may be given to a kernel.  It is looked up on every call
+// rather than cached: after a device reset (or any teardown of the primary
+// context) the module is loaded again and the array can move, and a cached
+// address would then point at memory the library no longer owns.
 vdn_status scratch_for_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return VDN_ERR_CUDA;
-  if (dev >= kMaxDevices) return VDN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return VDN_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return VDN_ERR_CUDA;
+  *out = p;
   return VDN_OK;
 }
 
