@@ -23,9 +23,9 @@
  *   c-1, c, c+1 (clipped at the ends), every query sees the anchor frames and
  *   anchor queries see every frame:  y_sm = sigmoid(g_sm) * softmax(s q K^T) V.
  *
- *   The backward of both branches (vdn_hybrid_lin_bwd, vdn_hybrid_sm_bwd) is
- *   the exact derivative of the forward above; the pages describe the forward
- *   only.
+ *   The backward of both branches (vdn_hybrid_lin_bwd, vdn_hybrid_sm_bwd, and
+ *   the two together, summed, in vdn_hybrid_bwd) is the exact derivative of
+ *   the forward above; the pages describe the forward only.
  *
  * Conventions for every entry point:
  *   - Ownership: the library allocates nothing.  The caller owns every input,
@@ -233,12 +233,38 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg *cfg, const vdn_hybri
 vdn_status vdn_hybrid_attn_fwd_noalloc(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
                                        vdn_stream_t stream);
 
+/* Kernel tags: which kernel's bounded wait gave up (vdn_hybrid_device_status). */
+enum {
+  VDN_TAG_NONE = 0,
+  VDN_TAG_SOFTMAX = 1,      /* windowed softmax (and the text cross-attention)  */
+  VDN_TAG_GRAM = 2,         /* per-frame and text Gram / write                  */
+  VDN_TAG_READ = 3,         /* state read + RMSNorm + gate                      */
+  VDN_TAG_SCAN = 4,         /* state scans                                      */
+  VDN_TAG_COMPOSE = 5,      /* chunk composition                                */
+  VDN_TAG_SOFTMAX_BWD = 6,  /* softmax branch backward                          */
+  VDN_TAG_LINEAR_BWD = 7    /* linear branch backward                           */
+};
+
 /* Reads the device status words left by the most recent call on this
  * workspace (every fwd / fwd_stages call clears them first; synchronises `stream`).
- * Returns VDN_OK or VDN_ERR_TIMEOUT; *where (if not NULL) gets the kernel tag
- * that gave up. */
+ * Returns VDN_OK or VDN_ERR_TIMEOUT; *where (if not NULL) gets the VDN_TAG_* of
+ * the kernel that gave up. */
 vdn_status vdn_hybrid_device_status(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
                                     vdn_stream_t stream, unsigned *where);
+
+/* Failure-path test hook (no counterpart on the pages).  Sets, on the current
+ * device, the wait limit in SM clock cycles of the state read's epilogue warps
+ * (the tensor-core read kernel at d = 64 or 128: the warps that wait for the
+ * tensor cores' products); 0 restores the default of every bounded wait
+ * (about one second).  With a limit shorter than the products take, those
+ * waits run out: the kernel records VDN_ERR_TIMEOUT and VDN_TAG_READ in the
+ * workspace status words, its producer and MMA roles stop issuing and drain
+ * what they issued, and the CTAs exit with their rows of y's linear slot
+ * unwritten (vdn_hybrid_device_status then reports the timeout; the context
+ * stays usable).  Synchronous and not stream-ordered: call it with no work of
+ * this library in flight on the device.  Errors: VDN_ERR_INVALID_ARG (cycles
+ * above the default limit), VDN_ERR_CUDA. */
+vdn_status vdn_debug_set_read_wait_limit(unsigned long long cycles);
 
 /* Which implementation a stage uses for cfg: 0 = SIMT fp32, 1 = tcgen05 tensor
  * cores (TMA + TMEM), 2 = the ablation variants' per-frame map kernel (SOLVE
@@ -351,6 +377,54 @@ size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg *cfg);
  * misaligned or too small); VDN_ERR_CUDA for a launch failure. */
 vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args, const vdn_sm_grads *grads,
                              vdn_stream_t stream);
+
+/* ------------------------------------------------------ backward of the core
+ * The whole core's gradient in one call: the exact derivative of the forward
+ * at the top of this header (both branches; the pages describe the forward
+ * only).  Given dy = dL/dy in y's shape and dtype, it writes dL/dq, dL/dk and
+ * dL/dv with the two branches' shares summed on the device, and the
+ * branch-specific gradients: dbeta, dalpha and dgate_lin (linear branch),
+ * dgate_sm (softmax branch), and drms_weight and dfwd_init where asked.
+ * Equivalent to vdn_hybrid_sm_bwd followed by vdn_hybrid_lin_bwd and a sum,
+ * without the extra buffers: the softmax branch runs first and writes dq, dk,
+ * dv; the linear branch then adds its share into them.
+ *
+ * Precondition, arguments and computation as for those two entry points (the
+ * forward's workspace in args->workspace for the linear branch; the forward's
+ * log-sum-exp in sm_lse, optional, for the softmax branch's tensor-core path).
+ * Scratch: one region of vdn_hybrid_bwd_workspace_size(cfg) bytes shared by the
+ * two branches in turn.  Status words of the bounded device waits: the
+ * softmax branch's in the first 256 bytes of grads->workspace, the linear
+ * branch's at the head of args->workspace; vdn_hybrid_device_status reads
+ * either (args->workspace set to the region in question).
+ * Errors (nothing enqueued): any error either branch's entry point reports
+ * for the same arguments, checked for both before the first launch;
+ * VDN_ERR_WORKSPACE for a missing, misaligned (256 bytes) or too small
+ * grads->workspace; VDN_ERR_CUDA for a launch failure. */
+typedef struct {
+  const void *dy;      /* dL/dy in y's shape (per cfg.out_mode) and cfg.y_dtype; 16-byte aligned      */
+  float *dq, *dk, *dv; /* [B,T,N,H,d] float32, overwritten with both branches' shares summed           */
+  float *dbeta;        /* [B,T,N,H] float32, overwritten                                             */
+  float *dalpha;       /* [B,T,H] float32, overwritten (zero at anchor frames)                        */
+  float *dgate_lin;    /* [B,T,N,H,d_v] float32, overwritten                                         */
+  float *dgate_sm;     /* [B,T,N,H,d_v] float32, overwritten                                         */
+  float *drms_weight;  /* [H,d_v] float32 or NULL (as in vdn_lin_grads)                               */
+  float *dfwd_init;    /* [B,H,d_v,d_k] float32 or NULL (as in vdn_lin_grads)                         */
+  void *workspace;     /* scratch shared by the two branches, 256-byte aligned, no overlap with anything
+                          else                                                                        */
+  size_t workspace_bytes; /* >= vdn_hybrid_bwd_workspace_size(cfg)                                     */
+  const float *sm_lse; /* [B,T,N,H] or NULL: the forward's args->sm_lse (as in vdn_sm_grads)           */
+} vdn_hybrid_grads;
+
+/* Bytes of scratch for vdn_hybrid_bwd: the larger of the softmax branch's scratch
+ * and 256 bytes plus the linear branch's; 0 if cfg is invalid or not
+ * supported by the backward. */
+size_t vdn_hybrid_bwd_workspace_size(const vdn_hybrid_cfg *cfg);
+
+/* Enqueue the whole core's backward on `stream` (no synchronisation, no
+ * allocation). */
+vdn_status vdn_hybrid_bwd(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args, const vdn_hybrid_grads *grads,
+                          vdn_stream_t stream);
 
 /* ------------------------------------------------------- text cross-attention
  * The DiT block's softmax cross-attention from the video tokens to the text

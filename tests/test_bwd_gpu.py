@@ -224,26 +224,50 @@ def test_sm_bwd_matches_oracle(shape, dtype, opts):
         assert e <= TOL[dtype], (n, e)
 
 
-def test_whole_core_backward_is_the_sum_of_the_branches():
-    """HybridAttention.backward: dq, dk, dv of the core equal the two oracles'
-    branch gradients added; the gate gradients are each branch's own."""
-    shape = Shape(B=1, T=12, N=30, H=2, d_k=64, d_v=64, L=4)
-    inp = make_inputs(shape, 71, "f32")
-    cfg = cfg_for(shape, "f32")
-    t = to_torch(inp, "f32", "cuda")
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128)])
+def test_whole_core_backward_is_the_sum_of_the_branches(dtype, d):
+    """vdn_hybrid_bwd (HybridAttention.backward, one library call): dq, dk, dv
+    of the core equal the two oracles' branch gradients added, the gate
+    gradients are each branch's own; and the one call equals the two branch
+    entry points' outputs added, bit for bit (the linear branch adds its share
+    in fp32 to what the softmax branch wrote).  fp32 d = 64 runs the SIMT
+    kernels, bf16 d = 128 the tensor-core ones (with an RMS weight and a
+    carried forward state)."""
+    shape = Shape(B=1, T=12, N=30, H=2, d_k=d, d_v=d, L=4)
+    inp = make_inputs(shape, 71, dtype)
+    if dtype == "bf16":
+        r = np.random.default_rng(73)
+        inp["rms_weight"] = (1 + 0.2 * r.standard_normal((2, d))).astype(np.float32)
+        inp["fwd_init"] = (0.1 * r.standard_normal((1, 2, d, d))).astype(np.float32)
+    cfg = cfg_for(shape, dtype)
+    t = to_torch(inp, dtype, "cuda")
+    for k in ("rms_weight", "fwd_init"):
+        if k in inp:
+            t[k] = torch.from_numpy(inp[k]).cuda()
     ha = HybridAttention(cfg)
     ha(t)
     dy = _dy(cfg, 72)
-    g = ha.backward(t, torch.from_numpy(dy.astype(np.float32)).cuda())
+    dyt = torch.from_numpy(dy.astype(np.float32)).cuda()
+    g = {k: v.clone() for k, v in ha.backward(t, dyt).items()}
     torch.cuda.synchronize()
+    assert ha.backward_status()[0] == L.VDN_OK
     oc = _ocfg(cfg)
     rl = OG.linear_branch_grads(inp, oc, dy[..., 1, :])
     rs = OG.softmax_branch_grads(inp, oc, dy[..., 0, :])
     for n in ("q", "k", "v"):
-        assert _rel(g["d" + n].cpu().numpy(), rl[n] + rs[n]) <= TOL["f32"], n
-    assert _rel(g["dgate_sm"].cpu().numpy(), rs["gate_sm"]) <= TOL["f32"]
-    assert _rel(g["dgate_lin"].cpu().numpy(), rl["gate_lin"]) <= TOL["f32"]
-    assert _rel(g["dbeta"].cpu().numpy(), rl["beta"]) <= TOL["f32"]
+        assert _rel(g["d" + n].cpu().numpy(), rl[n] + rs[n]) <= TOL[dtype], n
+    assert _rel(g["dgate_sm"].cpu().numpy(), rs["gate_sm"]) <= TOL[dtype]
+    assert _rel(g["dgate_lin"].cpu().numpy(), rl["gate_lin"]) <= TOL[dtype]
+    assert _rel(g["dbeta"].cpu().numpy(), rl["beta"]) <= TOL[dtype]
+    lin = ha.linear_backward(t, dyt, want_rms="rms_weight" in t, want_fwd_init="fwd_init" in t)
+    sm = ha.softmax_backward(t, dyt)
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv"):
+        assert torch.equal(g[n], lin[n] + sm[n]), n
+    for n in ("dbeta", "dalpha", "dgate_lin", "drms_weight", "dfwd_init"):
+        if n in lin:
+            assert torch.equal(g[n], lin[n]), n
+    assert torch.equal(g["dgate_sm"], sm["dgate_sm"])
 
 
 def test_sm_bwd_full_size_one_key_frame():

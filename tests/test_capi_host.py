@@ -271,6 +271,44 @@ def test_sm_lse_pointers_validated_before_launch():
     assert L.vdn_hybrid_sm_bwd(cfg, _fake_args(cfg), g, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
 
 
+def test_whole_bwd_workspace_and_rejections():
+    """vdn_hybrid_bwd: its scratch is the larger of the softmax branch's and
+    256 bytes plus the linear branch's; every check of either branch runs
+    before the first launch (a bad pointer of one branch stops the call)."""
+    cfg = _cfg()
+    sm, lin = L.vdn_hybrid_sm_bwd_workspace_size(cfg), L.vdn_hybrid_lin_bwd_workspace_size(cfg)
+    assert L.vdn_hybrid_bwd_workspace_size(cfg) == max(sm, 256 + lin)
+    for kw in (dict(update=1), dict(d_k=256, d_v=256), dict(T=1)):
+        assert L.vdn_hybrid_bwd_workspace_size(_cfg(**kw)) == 0
+    p = 1 << 26
+    good = dict(dy=p, dq=p, dk=p, dv=p, dbeta=p, dalpha=p, dgate_lin=p, dgate_sm=p, workspace=p,
+                workspace_bytes=L.vdn_hybrid_bwd_workspace_size(cfg))
+    for over, status in ((dict(dy=None), L.VDN_ERR_INVALID_ARG), (dict(dgate_sm=p + 8), L.VDN_ERR_INVALID_ARG),
+                         (dict(dgate_lin=None), L.VDN_ERR_INVALID_ARG), (dict(dalpha=p + 2), L.VDN_ERR_INVALID_ARG),
+                         (dict(dfwd_init=p + 4), L.VDN_ERR_INVALID_ARG), (dict(sm_lse=p + 2), L.VDN_ERR_INVALID_ARG),
+                         (dict(workspace=None), L.VDN_ERR_WORKSPACE), (dict(workspace=p + 128), L.VDN_ERR_WORKSPACE),
+                         (dict(workspace_bytes=max(sm, 256 + lin) - 1), L.VDN_ERR_WORKSPACE)):
+        g = L.make_grads(**{**good, **over})
+        assert L.vdn_hybrid_bwd(cfg, _fake_args(cfg), g, stream=0, check=False) == status, over
+    g = L.make_grads(**good)
+    assert L.vdn_hybrid_bwd(cfg, _fake_args(cfg, gate_sm=None), g, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.vdn_hybrid_bwd(cfg, _fake_args(cfg, gate_lin=None), g, stream=0, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.vdn_hybrid_bwd(cfg, _fake_args(cfg, workspace_bytes=1024), g, stream=0, check=False) == \
+        L.VDN_ERR_WORKSPACE
+    c = _cfg(update=2)
+    assert L.vdn_hybrid_bwd(c, _fake_args(c), g, stream=0, check=False) == L.VDN_ERR_UNSUPPORTED
+    lib = L.lib()
+    cc = cfg.c()
+    assert lib.vdn_hybrid_bwd(C.byref(cc), None, None, None) == L.VDN_ERR_INVALID_ARG
+
+
+def test_read_wait_limit_hook_rejects_out_of_range():
+    """The failure-path hook refuses a limit above the default (about one
+    second of clock cycles) before touching the device."""
+    assert L.vdn_debug_set_read_wait_limit(2_000_000_001, check=False) == L.VDN_ERR_INVALID_ARG
+    assert L.vdn_debug_set_read_wait_limit(2 ** 63, check=False) == L.VDN_ERR_INVALID_ARG
+
+
 def _header_struct_fields(name):
     """Field names, in order, of `typedef struct { ... } name;` in the header."""
     src = open(os.path.join(ROOT, "include", "vdn_hybrid.h")).read()
@@ -292,6 +330,7 @@ def _header_struct_fields(name):
 @pytest.mark.parametrize("cname,pystruct", [
     ("vdn_hybrid_cfg", L.VdnCfg), ("vdn_hybrid_args", L.VdnArgs), ("vdn_lin_grads", L.VdnLinGrads),
     ("vdn_sm_grads", L.VdnSmGrads), ("vdn_proj_cfg", L.ProjCfg), ("vdn_workspace_layout", L.VdnLayout),
+    ("vdn_hybrid_grads", L.VdnGrads),
 ])
 def test_ctypes_mirrors_follow_the_header(cname, pystruct):
     """The binding's structs list the header's fields in the same order (a

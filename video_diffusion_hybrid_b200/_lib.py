@@ -25,7 +25,8 @@ EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vd
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
             "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn",
             "vdn_quantize_fp8", "vdn_out_proj_fp8", "vdn_hybrid_lin_bwd_workspace_size", "vdn_hybrid_lin_bwd",
-            "vdn_hybrid_sm_bwd_workspace_size", "vdn_hybrid_sm_bwd")
+            "vdn_hybrid_sm_bwd_workspace_size", "vdn_hybrid_sm_bwd", "vdn_hybrid_bwd_workspace_size", "vdn_hybrid_bwd",
+            "vdn_debug_set_read_wait_limit")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -59,6 +60,14 @@ class VdnSmGrads(C.Structure):
     _fields_ = [("dy", C.c_void_p), ("dq", C.c_void_p), ("dk", C.c_void_p), ("dv", C.c_void_p),
                 ("dgate_sm", C.c_void_p), ("workspace", C.c_void_p), ("workspace_bytes", C.c_size_t),
                 ("sm_lse", C.c_void_p)]
+
+
+class VdnGrads(C.Structure):
+    """Mirror of ``vdn_hybrid_grads`` (the whole core's backward)."""
+    _fields_ = [("dy", C.c_void_p), ("dq", C.c_void_p), ("dk", C.c_void_p), ("dv", C.c_void_p),
+                ("dbeta", C.c_void_p), ("dalpha", C.c_void_p), ("dgate_lin", C.c_void_p), ("dgate_sm", C.c_void_p),
+                ("drms_weight", C.c_void_p), ("dfwd_init", C.c_void_p), ("workspace", C.c_void_p),
+                ("workspace_bytes", C.c_size_t), ("sm_lse", C.c_void_p)]
 
 
 class ProjCfg(C.Structure):
@@ -149,6 +158,12 @@ def lib() -> C.CDLL:
         L.vdn_hybrid_sm_bwd_workspace_size.argtypes = [C.POINTER(VdnCfg)]
         L.vdn_hybrid_sm_bwd.restype = C.c_int
         L.vdn_hybrid_sm_bwd.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.POINTER(VdnSmGrads), C.c_void_p]
+        L.vdn_hybrid_bwd_workspace_size.restype = C.c_size_t
+        L.vdn_hybrid_bwd_workspace_size.argtypes = [C.POINTER(VdnCfg)]
+        L.vdn_hybrid_bwd.restype = C.c_int
+        L.vdn_hybrid_bwd.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.POINTER(VdnGrads), C.c_void_p]
+        L.vdn_debug_set_read_wait_limit.restype = C.c_int
+        L.vdn_debug_set_read_wait_limit.argtypes = [C.c_ulonglong]
         L.vdn_status_string.restype = C.c_char_p
         L.vdn_status_string.argtypes = [C.c_int]
         _lib = L
@@ -316,4 +331,41 @@ def vdn_hybrid_sm_bwd(cfg: HybridCfg, args: VdnArgs, grads: VdnSmGrads, stream=N
     st = lib().vdn_hybrid_sm_bwd(C.byref(c), C.byref(args), C.byref(grads), _stream_handle(stream))
     if check and st != VDN_OK:
         raise VdnError(st, "vdn_hybrid_sm_bwd")
+    return st
+
+
+def vdn_hybrid_bwd_workspace_size(cfg: HybridCfg) -> int:
+    c = cfg.c()
+    return int(lib().vdn_hybrid_bwd_workspace_size(C.byref(c)))
+
+
+def make_grads(dy, dq, dk, dv, dbeta, dalpha, dgate_lin, dgate_sm, workspace, workspace_bytes=None, drms_weight=None,
+               dfwd_init=None, sm_lse=None) -> VdnGrads:
+    """Build a ``vdn_hybrid_grads`` from torch tensors (or raw device pointers)."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return VdnGrads(_ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dalpha), _ptr(dgate_lin),
+                    _ptr(dgate_sm), _ptr(drms_weight), _ptr(dfwd_init), _ptr(workspace), int(workspace_bytes),
+                    _ptr(sm_lse))
+
+
+def vdn_hybrid_bwd(cfg: HybridCfg, args: VdnArgs, grads: VdnGrads, stream=None, check: bool = True) -> int:
+    """The whole core's backward (both branches, dq / dk / dv summed on the
+    device); args.workspace holds the forward's."""
+    c = cfg.c()
+    st = lib().vdn_hybrid_bwd(C.byref(c), C.byref(args), C.byref(grads), _stream_handle(stream))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_hybrid_bwd")
+    return st
+
+
+TAG_READ = 3  # VDN_TAG_READ
+
+
+def vdn_debug_set_read_wait_limit(cycles: int, check: bool = True) -> int:
+    """Wait limit (SM clock cycles) of the state read's epilogue warps on the
+    current device; 0 = the default.  Failure-path tests only."""
+    st = lib().vdn_debug_set_read_wait_limit(int(cycles))
+    if check and st != VDN_OK:
+        raise VdnError(st, "vdn_debug_set_read_wait_limit")
     return st

@@ -128,17 +128,43 @@ class HybridAttention:
         return L.vdn_hybrid_device_status(self.cfg, a, stream)
 
     def backward(self, t: dict, dy: torch.Tensor, stream=None) -> dict:
-        """The whole core's gradients after a forward call on the same inputs:
-        both branches' shares of dq, dk, dv summed (one elementwise torch add
-        each, on the same stream), and the branch-specific gradients."""
-        lin = self.linear_backward(t, dy, want_rms=t.get("rms_weight") is not None,
-                                   want_fwd_init=t.get("fwd_init") is not None, stream=stream)
-        sm = self.softmax_backward(t, dy, stream=stream)
-        out = dict(lin)
-        for k in ("dq", "dk", "dv"):
-            out[k] = lin[k] + sm[k]
-        out["dgate_sm"] = sm["dgate_sm"]
-        return out
+        """The whole core's gradients after a forward call on the same inputs,
+        in one library call (``vdn_hybrid_bwd``): dq, dk, dv with both
+        branches' shares summed on the device, and the branch-specific
+        gradients (drms_weight / dfwd_init when those inputs are given)."""
+        c = self.cfg
+        if getattr(self, "whole_bwd_workspace", None) is None:
+            nb = L.vdn_hybrid_bwd_workspace_size(c)
+            if nb == 0:
+                raise L.VdnError(L.VDN_ERR_UNSUPPORTED, "vdn_hybrid_bwd_workspace_size")
+            self.whole_bwd_workspace = torch.empty(nb, dtype=torch.uint8, device=self.device)
+        f = lambda *shape: torch.empty(shape, dtype=torch.float32, device=self.device)
+        tok = (c.B, c.T, c.N, c.H)
+        g = {"dq": f(*tok, c.d_k), "dk": f(*tok, c.d_k), "dv": f(*tok, c.d_v), "dbeta": f(*tok),
+             "dalpha": f(c.B, c.T, c.H), "dgate_lin": f(*tok, c.d_v), "dgate_sm": f(*tok, c.d_v)}
+        if t.get("rms_weight") is not None:
+            g["drms_weight"] = f(c.H, c.d_v)
+        if t.get("fwd_init") is not None:
+            g["dfwd_init"] = f(c.B, c.H, c.d_v, c.d_k)
+        gr = L.make_grads(dy, g["dq"], g["dk"], g["dv"], g["dbeta"], g["dalpha"], g["dgate_lin"], g["dgate_sm"],
+                          self.whole_bwd_workspace, drms_weight=g.get("drms_weight"), dfwd_init=g.get("dfwd_init"),
+                          sm_lse=self.sm_lse)
+        L.vdn_hybrid_bwd(c, self.args(t), gr, stream)
+        return g
+
+    def backward_status(self, stream=None) -> tuple:
+        """(status, kernel tag) of the last whole-core backward: the softmax
+        branch's status words (head of the shared scratch), else the linear
+        branch's (head of the forward's workspace)."""
+        a = L.VdnArgs()
+        a.workspace = self.whole_bwd_workspace.data_ptr()
+        a.workspace_bytes = self.whole_bwd_workspace.numel()
+        st = L.vdn_hybrid_device_status(self.cfg, a, stream)
+        if st[0] != L.VDN_OK:
+            return st
+        a.workspace = self.workspace.data_ptr()
+        a.workspace_bytes = self.ws_bytes
+        return L.vdn_hybrid_device_status(self.cfg, a, stream)
 
     def intermediates(self) -> dict:
         """Views of the workspace's intermediate values (float32)."""

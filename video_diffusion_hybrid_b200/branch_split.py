@@ -31,7 +31,7 @@ import torch
 import torch.distributed as dist
 
 from . import _lib as L
-from .ulysses import REPLICATED_HEAD_AXIS, _world
+from .ulysses import REPLICATED_HEAD_AXIS, _world, to_device
 
 # per-token inputs [B, S/P, H, ...] and the branches that read them
 READ_BY = {"q": ("sm", "lin"), "k": ("sm", "lin"), "v": ("sm", "lin"), "gate_sm": ("sm",),
@@ -147,12 +147,20 @@ class BranchSplitHybridAttention:
         self.core = HybridAttention(self.local_cfg, device)
 
     def __call__(self, t_local: dict, stream=None) -> torch.Tensor:
-        t = split_inputs(t_local, self.cfg.T, self.cfg.N, self.lay, self.group)
+        # the exchange runs where the inputs are (GPU with NCCL, host copies
+        # with gloo); the core runs on its device
+        where = t_local["q"].device
+        t = to_device(split_inputs(t_local, self.cfg.T, self.cfg.N, self.lay, self.group), self.core.device)
         # the other branch's per-token inputs are not sent here; the core's
         # argument checks want every pointer, so they alias one that is
         # (their stages do not run)
         for name in ("gate_sm", "gate_lin"):
             t.setdefault(name, t["q"])
         t.setdefault("beta", torch.empty(t["q"].shape[:4], dtype=torch.float32, device=t["q"].device))
+        self._last = t  # the inputs of the last call, for device_status
         y = self.core(t, stages=STAGES[self.branch], stream=stream)
-        return merge_outputs(y, self.lay, self.group)
+        return merge_outputs(y.to(where), self.lay, self.group)
+
+    def device_status(self) -> tuple:
+        """(status, kernel tag) of this rank's last core call (synchronises)."""
+        return L.vdn_hybrid_device_status(self.local_cfg, self.core.args(self._last))

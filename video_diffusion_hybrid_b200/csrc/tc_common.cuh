@@ -56,6 +56,10 @@ struct Ctl {
   volatile int* abort;  // shared flag: some wait of this CTA gave up
   uint32_t* status;     // workspace status words
   unsigned tag;         // kernel tag recorded on a timeout
+  long long limit;      // wait limit in clock cycles; 0 = kWaitCycles (about one second).  A
+                        // shorter limit (the read's consumer roles can be given one, to test
+                        // the timeout path) polls without suspending and checks the clock on
+                        // every try, so that it runs out on time
 };
 
 // Non-suspending test of a phase.
@@ -74,6 +78,19 @@ static __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) 
 // Bounded wait, slow path: true when the phase completed; false after ~1 s
 // or when another role of the CTA already gave up.
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (c.limit > 0) {
+    const long long t0 = clock64();
+    for (;;) {
+      if (mbar_test(bar, parity)) return true;
+      if (*c.abort) return false;
+      if (clock64() - t0 > c.limit) {
+        *c.abort = 1;
+        atomicOr(c.status, 1u);
+        atomicExch(c.status + 1, c.tag);
+        return false;
+      }
+    }
+  }
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
@@ -94,6 +111,17 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
 // call and the suspending try_wait of the slow path.
 static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c) {
   return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, c);
+}
+
+// Bounded wait for this CTA's own copies or MMAs in flight (the phase a role
+// committed or expected itself), before the CTA frees its TMEM and exits.
+// Those end by themselves, so it ignores the abort flag of the other roles:
+// a CTA that gave up on some wait still drains what it issued.
+static __device__ __noinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
 }
 
 static __device__ __forceinline__ void fence_barrier_init() {

@@ -51,6 +51,7 @@ Dims make_dims(const vdn_hybrid_cfg* c) {
   d.out_bf16 = c->y_dtype == VDN_BF16;
   d.scan_mode = c->scan_mode;
   d.update = c->update;
+  d.grad_acc = 0;
   return d;
 }
 
@@ -302,8 +303,12 @@ size_t vdn_hybrid_lin_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {
   return lin_bwd_workspace(make_dims(cfg), nullptr);
 }
 
-vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_lin_grads* g,
-                              vdn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Everything vdn_hybrid_lin_bwd checks before launching.
+vdn_status lin_bwd_checks(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_lin_grads* g) {
   vdn_status st = check_bwd_cfg(cfg);
   if (st != VDN_OK) return st;
   if (!args || !g) return VDN_ERR_INVALID_ARG;
@@ -324,25 +329,31 @@ vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* 
   const Dims d = make_dims(cfg);
   if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < lin_bwd_workspace(d, nullptr))
     return VDN_ERR_WORKSPACE;
+  return VDN_OK;
+}
+
+// The linear branch's launches (arguments already checked); grad_acc adds its
+// dq, dk, dv into the outputs instead of overwriting them.
+vdn_status lin_bwd_launch(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_lin_grads* g,
+                          cudaStream_t s, bool grad_acc) {
+  Dims d = make_dims(cfg);
+  d.grad_acc = grad_acc ? 1 : 0;
   Work w = work_of(cfg, args);
   // the forward's choice of write form (B_t or C_t in the C_t slot)
   w.bform = (scan_tc_supported(d) && w.M16 != nullptr) ? 1 : 0;
   LinBwdArgs a{g->dy, g->dq, g->dk, g->dv, g->dbeta, g->dalpha, g->dgate_lin, g->drms_weight, g->dfwd_init,
                g->workspace, w.status};
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(w.status, 0, 256, s) != cudaSuccess) return VDN_ERR_CUDA;
   return launch_lin_bwd(d, inputs_of(args), w, a, s) == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
 }
 
-size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {
-  if (check_bwd_cfg(cfg) != VDN_OK) return 0;
-  const Dims d = make_dims(cfg);
+size_t sm_bwd_scratch(const Dims& d) {
   const size_t a = sm_bwd_workspace(d, nullptr), b = sm_bwd_tc_workspace(d, nullptr);
   return a > b ? a : b;
 }
 
-vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_sm_grads* g,
-                             vdn_stream_t stream) {
+// Everything vdn_hybrid_sm_bwd checks before launching.
+vdn_status sm_bwd_checks(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_sm_grads* g) {
   vdn_status st = check_bwd_cfg(cfg);
   if (st != VDN_OK) return st;
   if (!args || !g) return VDN_ERR_INVALID_ARG;
@@ -352,9 +363,14 @@ vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* a
   const Dims d = make_dims(cfg);
   if (g->sm_lse && !aligned(g->sm_lse, 4)) return VDN_ERR_INVALID_ARG;
   if ((long long)d.T * d.N > (1LL << 40)) return VDN_ERR_UNSUPPORTED;
-  if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < vdn_hybrid_sm_bwd_workspace_size(cfg))
+  if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < sm_bwd_scratch(d))
     return VDN_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return VDN_OK;
+}
+
+vdn_status sm_bwd_launch(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_sm_grads* g,
+                         cudaStream_t s) {
+  const Dims d = make_dims(cfg);
   char* base = static_cast<char*>(g->workspace);
   if (sm_bwd_tc_supported(d)) {
     size_t off[8];
@@ -370,6 +386,62 @@ vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* a
   if (cudaMemsetAsync(base, 0, kAlign, s) != cudaSuccess) return VDN_ERR_CUDA;  // no status on this path
   SmBwdArgs a{g->dy, g->dq, g->dk, g->dv, g->dgate_sm, base + kAlign};
   return launch_sm_bwd(d, inputs_of(args), a, s) == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
+// The whole-core backward shares one scratch region between the branches,
+// which run one after the other on the stream: the softmax branch's layout
+// from byte 0 (its status words in the first 256 bytes), the linear branch's
+// from byte 256, so that the softmax branch's status words survive it.
+size_t whole_bwd_scratch(const Dims& d) {
+  const size_t a = sm_bwd_scratch(d), b = kAlign + lin_bwd_workspace(d, nullptr);
+  return a > b ? a : b;
+}
+
+}  // namespace
+
+extern "C" {
+
+vdn_status vdn_hybrid_lin_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_lin_grads* g,
+                              vdn_stream_t stream) {
+  const vdn_status st = lin_bwd_checks(cfg, args, g);
+  if (st != VDN_OK) return st;
+  return lin_bwd_launch(cfg, args, g, reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+size_t vdn_hybrid_sm_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {
+  if (check_bwd_cfg(cfg) != VDN_OK) return 0;
+  return sm_bwd_scratch(make_dims(cfg));
+}
+
+vdn_status vdn_hybrid_sm_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_sm_grads* g,
+                             vdn_stream_t stream) {
+  const vdn_status st = sm_bwd_checks(cfg, args, g);
+  if (st != VDN_OK) return st;
+  return sm_bwd_launch(cfg, args, g, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t vdn_hybrid_bwd_workspace_size(const vdn_hybrid_cfg* cfg) {
+  if (check_bwd_cfg(cfg) != VDN_OK) return 0;
+  return whole_bwd_scratch(make_dims(cfg));
+}
+
+vdn_status vdn_hybrid_bwd(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, const vdn_hybrid_grads* g,
+                          vdn_stream_t stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!args || !g) return VDN_ERR_INVALID_ARG;
+  const Dims d = make_dims(cfg);
+  if (!g->workspace || !aligned(g->workspace, kAlign) || g->workspace_bytes < whole_bwd_scratch(d))
+    return VDN_ERR_WORKSPACE;
+  vdn_sm_grads sg{g->dy, g->dq, g->dk, g->dv, g->dgate_sm, g->workspace, g->workspace_bytes, g->sm_lse};
+  vdn_lin_grads lg{g->dy, g->dq, g->dk, g->dv, g->dbeta, g->dalpha, g->dgate_lin, g->drms_weight, g->dfwd_init,
+                   static_cast<char*>(g->workspace) + kAlign, g->workspace_bytes - kAlign};
+  if ((st = sm_bwd_checks(cfg, args, &sg)) != VDN_OK) return st;
+  if ((st = lin_bwd_checks(cfg, args, &lg)) != VDN_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the softmax branch writes dq, dk, dv; the linear branch adds its share
+  if ((st = sm_bwd_launch(cfg, args, &sg, s)) != VDN_OK) return st;
+  return lin_bwd_launch(cfg, args, &lg, s, true);
 }
 
 vdn_status vdn_text_cross_attn(const vdn_hybrid_cfg* cfg, const vdn_hybrid_args* args, vdn_stream_t stream) {

@@ -100,15 +100,6 @@ __device__ __forceinline__ void store_f32(float* dst, const float (&s)[32]) {
   for (int u = 0; u < 8; ++u) *reinterpret_cast<float4*>(dst + 4 * u) = make_float4(s[4 * u], s[4 * u + 1], s[4 * u + 2], s[4 * u + 3]);
 }
 
-// Bounded wait for this CTA's own copies or MMAs in flight, which end by
-// themselves: ignores the abort flag of the other roles.
-__device__ __noinline__ bool wait_own(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
-  return true;
-}
-
 __global__ void __launch_bounds__(kThreadsCmp, 1)
 k_compose_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -162,7 +153,7 @@ k_compose_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm
                         (int)((fh * 2 + part) * D));
         ++nb;
       }
-      if (nb > 0) wait_own(bar(B_BFULL), (nb - 1) & 1);
+      if (nb > 0) mbar_drain(bar(B_BFULL), (nb - 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -189,7 +180,7 @@ k_compose_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm
         mma_commit(bar(B_MDONE));
       }
       mma_commit(bar(B_DRAIN));
-      wait_own(bar(B_DRAIN), 0);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     const int quad = warp & 3, half = (warp - 4) >> 2, row = quad * 32 + lane;

@@ -121,7 +121,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
         last[s] = j;
       }
       for (int s = 0; s < ST; ++s)
-        if (last[s] >= 0) mbar_wait(bar(B_KVFULL + s), (last[s] / ST) & 1, ctl);
+        if (last[s] >= 0) mbar_drain(bar(B_KVFULL + s), (last[s] / ST) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -156,7 +156,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       }
       if (ok) mma_commit(bar(B_ACC));
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, ctl);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     const int quad = warp - 4;

@@ -18,10 +18,15 @@ struct Dims {
   int out_bf16;  // y stored as bf16
   int scan_mode;  // 0 auto, 1 frame steps, 2 chunk steps (tensor-core scan)
   int update;     // 0 joint solve, 1 frame-level independent writes (1/N), 2 token-wise delta rule
+  int grad_acc;   // linear-branch backward: add its dq, dk, dv into the outputs (the whole-core
+                  // backward, after the softmax branch wrote its share) instead of overwriting
 };
 
-// Device-side status words at the head of the workspace.
-enum : unsigned { TAG_NONE = 0, TAG_SOFTMAX_TC = 1, TAG_GRAM_TC = 2, TAG_READ_TC = 3, TAG_SCAN_TC = 4, TAG_COMPOSE_TC = 5, TAG_SMBWD_TC = 6, TAG_LINBWD_TC = 7 };
+// Device-side status words at the head of the workspace; the tags are the
+// header's VDN_TAG_* values.
+enum : unsigned { TAG_NONE = VDN_TAG_NONE, TAG_SOFTMAX_TC = VDN_TAG_SOFTMAX, TAG_GRAM_TC = VDN_TAG_GRAM,
+                  TAG_READ_TC = VDN_TAG_READ, TAG_SCAN_TC = VDN_TAG_SCAN, TAG_COMPOSE_TC = VDN_TAG_COMPOSE,
+                  TAG_SMBWD_TC = VDN_TAG_SOFTMAX_BWD, TAG_LINBWD_TC = VDN_TAG_LINEAR_BWD };
 
 struct Work {
   uint32_t* status;

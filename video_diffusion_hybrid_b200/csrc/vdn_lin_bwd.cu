@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(kBT, 1) k_bwd_read(Dims dm, Inputs in, Work w,
         if (n >= N) continue;
         float* dst = gr.dq + (tok(n) * H + h) * D;
 #pragma unroll
-        for (int m = 0; m < MI; ++m) dst[lane + 32 * m] = dq[p][m];
+        for (int m = 0; m < MI; ++m) dst[lane + 32 * m] = dm.grad_acc ? __fadd_rn(dst[lane + 32 * m], dq[p][m]) : dq[p][m];
       }
     }
     // ---- dR += do q^T over the tile's tokens
@@ -536,7 +536,8 @@ __global__ void __launch_bounds__(kBT, 1) k_bwd_tokens(Dims dm, Inputs in, BwdWo
   const long long DD = (long long)D * D, fh = ((long long)b * T + t) * H + h;
   auto row_of = [&](int n) { return (((long long)b * T + t) * N + n) * H + h; };
   if (is_anchor(dm, t)) {
-    for (long long e = tid; e < (long long)N * D; e += kBT) {
+    // not written: zero dk, dv (left as they are when adding to the softmax branch's share)
+    for (long long e = tid; !dm.grad_acc && e < (long long)N * D; e += kBT) {
       const long long row = row_of((int)(e / D));
       gr.dk[row * D + e % D] = 0.f;
       gr.dv[row * D + e % D] = 0.f;
@@ -601,8 +602,11 @@ __global__ void __launch_bounds__(kBT, 1) k_bwd_tokens(Dims dm, Inputs in, BwdWo
 #pragma unroll
       for (int m = 0; m < MI; ++m) {
         const int j = lane + 32 * m;
-        gr.dk[row * D + j] = be * (p1[p][m] + p2[p][m]);
-        gr.dv[row * D + j] = be * p3[p][m];
+        // the sum rounds the product first (no fused multiply-add), as adding
+        // the two branches' separate outputs would
+        const float gk = be * (p1[p][m] + p2[p][m]), gv = be * p3[p][m];
+        gr.dk[row * D + j] = dm.grad_acc ? __fadd_rn(gr.dk[row * D + j], gk) : gk;
+        gr.dv[row * D + j] = dm.grad_acc ? __fadd_rn(gr.dv[row * D + j], gv) : gv;
         db = fmaf(0.5f * Ks[r * QP + j], p1[p][m], fmaf(Vs[r * QP + j], p3[p][m], db));
       }
       db = warp_sum(db);

@@ -118,7 +118,7 @@ k_bwd_read_tc(Dims dm, Inputs in, const float* __restrict__ Fst, const float* __
         issued = j + 1;
       }
       for (int j = issued - STR < 0 ? 0 : issued - STR; j < issued; ++j)
-        mbar_wait(bar(B_FULL + j % STR), (j / STR) & 1, ctl);
+        mbar_drain(bar(B_FULL + j % STR), (j / STR) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -171,7 +171,7 @@ k_bwd_read_tc(Dims dm, Inputs in, const float* __restrict__ Fst, const float* __
       }
       if (ok) mma_commit(bar(B_DRDONE));
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, ctl);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     const int tid = threadIdx.x - 128, quad = warp - 4, row = quad * 32 + lane;
@@ -316,8 +316,15 @@ k_bwd_read_tc(Dims dm, Inputs in, const float* __restrict__ Fst, const float* __
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dq + grow * D + 32 * q + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          for (int i = 0; i < 32; i += 4) {
+            float4* p = reinterpret_cast<float4*>(dq + grow * D + 32 * q + i);
+            float4 x = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            if (dm.grad_acc) {
+              const float4 o = *p;
+              x = make_float4(__fadd_rn(o.x, x.x), __fadd_rn(o.y, x.y), __fadd_rn(o.z, x.z), __fadd_rn(o.w, x.w));
+            }
+            *p = x;
+          }
         }
       }
       tc_fence_before();

@@ -63,8 +63,9 @@ k_bwd_tokens_tc(Dims dm, Inputs in, const float* __restrict__ dAs, const float* 
   const int cb = blockIdx.x % (D / CW), t = blockIdx.x / (D / CW), h = blockIdx.y, b = blockIdx.z;
   const int N = dm.N, H = dm.H;
   const long long fh = ((long long)b * dm.T + t) * H + h, tok0 = ((long long)b * dm.T + t) * N;
-  if (is_anchor(dm, t)) {  // not written: zero dk, dv (dbeta is cleared by the launcher)
-    for (long long e = threadIdx.x; e < (long long)N * (CW / 4); e += kThrT) {
+  if (is_anchor(dm, t)) {  // not written: zero dk, dv (dbeta is cleared by the launcher);
+                           // left as they are when adding to the softmax branch's share
+    for (long long e = threadIdx.x; !dm.grad_acc && e < (long long)N * (CW / 4); e += kThrT) {
       const long long g = ((tok0 + e / (CW / 4)) * H + h) * D + cb * CW + (e % (CW / 4)) * 4;
       *reinterpret_cast<float4*>(dk + g) = make_float4(0.f, 0.f, 0.f, 0.f);
       *reinterpret_cast<float4*>(dv + g) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -104,7 +105,7 @@ k_bwd_tokens_tc(Dims dm, Inputs in, const float* __restrict__ dAs, const float* 
         issued = j + 1;
       }
       for (int j = issued - STT < 0 ? 0 : issued - STT; j < issued; ++j)
-        mbar_wait(bar(B_FULL + j % STT), (j / STT) & 1, ctl);
+        mbar_drain(bar(B_FULL + j % STT), (j / STT) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -138,7 +139,7 @@ k_bwd_tokens_tc(Dims dm, Inputs in, const float* __restrict__ dAs, const float* 
         mma_commit(bar(B_EMPTY + st));
       }
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, ctl);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     const int tid = threadIdx.x - 128, quad = warp - 4, row = quad * 32 + lane;
@@ -230,9 +231,16 @@ k_bwd_tokens_tc(Dims dm, Inputs in, const float* __restrict__ dAs, const float* 
           float* dvr = dv + grow * D + c0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            *reinterpret_cast<float4*>(dkr + i) = make_float4(be * (p1[i] + p2[i]), be * (p1[i + 1] + p2[i + 1]),
-                                                             be * (p1[i + 2] + p2[i + 2]), be * (p1[i + 3] + p2[i + 3]));
-            *reinterpret_cast<float4*>(dvr + i) = make_float4(be * p3[i], be * p3[i + 1], be * p3[i + 2], be * p3[i + 3]);
+            float4 gk = make_float4(be * (p1[i] + p2[i]), be * (p1[i + 1] + p2[i + 1]), be * (p1[i + 2] + p2[i + 2]),
+                                    be * (p1[i + 3] + p2[i + 3]));
+            float4 gv = make_float4(be * p3[i], be * p3[i + 1], be * p3[i + 2], be * p3[i + 3]);
+            if (dm.grad_acc) {  // products rounded first (no fused multiply-add)
+              const float4 pk = *reinterpret_cast<const float4*>(dkr + i), pv = *reinterpret_cast<const float4*>(dvr + i);
+              gk = make_float4(__fadd_rn(pk.x, gk.x), __fadd_rn(pk.y, gk.y), __fadd_rn(pk.z, gk.z), __fadd_rn(pk.w, gk.w));
+              gv = make_float4(__fadd_rn(pv.x, gv.x), __fadd_rn(pv.y, gv.y), __fadd_rn(pv.z, gv.z), __fadd_rn(pv.w, gv.w));
+            }
+            *reinterpret_cast<float4*>(dkr + i) = gk;
+            *reinterpret_cast<float4*>(dvr + i) = gv;
           }
         }
       }

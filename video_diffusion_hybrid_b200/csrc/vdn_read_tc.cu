@@ -27,6 +27,13 @@
 #include "tc_common.cuh"
 
 namespace vdn {
+
+// Wait limit, in clock cycles, of the epilogue warps' waits in k_read_tc (the
+// roles that wait for the tensor cores' products); 0 = the default of every
+// bounded wait (about one second).  vdn_debug_set_read_wait_limit sets it, so
+// that a test can make those waits run out and check the timeout path.
+__device__ long long g_read_epilogue_limit = 0;
+
 namespace {
 using namespace tc;
 
@@ -144,15 +151,6 @@ template <> __device__ __forceinline__ void put8<__nv_bfloat16>(__nv_bfloat16* p
       make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
 }
 
-// Bounded wait for this CTA's own copies or MMAs in flight, which end by
-// themselves: ignores the abort flag of the other roles.
-__device__ __noinline__ bool wait_landed(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
-  return true;
-}
-
 // sigmoid from the exponential and an approximate reciprocal (both a few ulp;
 // exp(-g) overflowing to inf gives 0, the limit)
 __device__ __forceinline__ float sigmoid_fast(float g) {
@@ -189,6 +187,9 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
   Run run;
   if (!decode_run(dm, blockIdx.x, run)) return;
   const Ctl ctl{abort_flag, w.status, (unsigned)TAG_READ_TC};
+  // the epilogue warps' waits: the settable limit (the producer and the MMA
+  // issuer keep the default, and drain what they issued whatever happens)
+  const Ctl ectl{abort_flag, w.status, (unsigned)TAG_READ_TC, g_read_epilogue_limit};
   auto bar = [&](int i) { return smem_u32(bars + i); };
 
   if (threadIdx.x == 0) {
@@ -228,11 +229,11 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
           tma_load_3d(smem_u32(sG + s * TBYTES + c * TQ * 128), &tmg, bar(B_GFULL + s), c * 64, run.h, tok);
         last[s] = t;
       }
-      mbar_wait(bar(B_R), 0, ctl);
+      mbar_drain(bar(B_R), 0);
       for (int s = 0; s < ST; ++s)
         if (last[s] >= 0) {
-          mbar_wait(bar(B_QFULL + s), (last[s] / ST) & 1, ctl);
-          mbar_wait(bar(B_GFULL + s), (last[s] / ST) & 1, ctl);
+          mbar_drain(bar(B_QFULL + s), (last[s] / ST) & 1);
+          mbar_drain(bar(B_GFULL + s), (last[s] / ST) & 1);
         }
     }
   } else if (warp == 1) {
@@ -257,7 +258,7 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
         mma_commit(bar(B_QEMPTY + s));
       }
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, ctl);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     const int quad = warp & 3, half = (warp - 4) >> 2;
@@ -266,8 +267,8 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
     const bool add = dm.out_mode != 0;
     for (int t = 0; t < run.ntiles; ++t) {
       const int s = t % ST;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + s), (t / ST) & 1, ctl))) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_GFULL + s), (t / ST) & 1, ctl))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + s), (t / ST) & 1, ectl))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_GFULL + s), (t / ST) & 1, ectl))) break;
       tc_fence_after();
       // own half of the row into o, the other half only for the sum of squares
       float o[HD];
@@ -396,8 +397,8 @@ k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         if (!ok) break;
       }
       // the last copies land before the CTA can exit (bounded, whatever the other roles do)
-      if (nq > 0) wait_landed(bar(B_QFULL), (nq - 1) & 1);
-      for (int u = nr - 2 < 0 ? 0 : nr - 2; u < nr; ++u) wait_landed(bar(B_RFULL + (u & 1)), (u >> 1) & 1);
+      if (nq > 0) mbar_drain(bar(B_QFULL), (nq - 1) & 1);
+      for (int u = nr - 2 < 0 ? 0 : nr - 2; u < nr; ++u) mbar_drain(bar(B_RFULL + (u & 1)), (u >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -425,7 +426,7 @@ k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         mma_commit(bar(B_QEMPTY));
       }
       mma_commit(bar(B_DRAIN));
-      wait_landed(bar(B_DRAIN), 0);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     const int quad = warp & 3, half = (warp - 4) >> 2;
@@ -567,3 +568,9 @@ cudaError_t launch_read_tc(const Dims& d, const Inputs& in, const Work& w, void*
 }
 
 }  // namespace vdn
+
+extern "C" vdn_status vdn_debug_set_read_wait_limit(unsigned long long cycles) {
+  if (cycles > (unsigned long long)vdn::tc::kWaitCycles) return VDN_ERR_INVALID_ARG;
+  const long long v = (long long)cycles;
+  return cudaMemcpyToSymbol(vdn::g_read_epilogue_limit, &v, sizeof(v)) == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}

@@ -75,15 +75,6 @@ __device__ __forceinline__ int snap_slot(const Dims& d, int dir, int st) {
   return (t % d.chunk == 0) ? t / d.chunk : -1;
 }
 
-// Bounded wait for this CTA's own copies or MMAs in flight, which end by
-// themselves: ignores the abort flag of the other roles.
-__device__ __noinline__ bool wait_own(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
-  return true;
-}
-
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -268,8 +259,8 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
       }
       // the last copies land before the pair can exit (the leader's B
       // barriers count both CTAs' bytes)
-      for (int n = nb - 2 < 0 ? 0 : nb - 2; lead && n < nb; ++n) wait_own(bar(B_BFULL + (n & 1)), (n >> 1) & 1);
-      for (int n = nc - 2 < 0 ? 0 : nc - 2; n < nc; ++n) wait_own(bar(B_CFULL + (n & 1)), (n >> 1) & 1);
+      for (int n = nb - 2 < 0 ? 0 : nb - 2; lead && n < nb; ++n) mbar_drain(bar(B_BFULL + (n & 1)), (n >> 1) & 1);
+      for (int n = nc - 2 < 0 ? 0 : nc - 2; n < nc; ++n) mbar_drain(bar(B_CFULL + (n & 1)), (n >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0 && lead) {
@@ -296,7 +287,7 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
         commit2(map_rank(bar(B_BEMPTY + slot), 1));
       }
       commit2(bar(B_DRAIN));
-      wait_own(bar(B_DRAIN), 0);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     const int quad = warp & 3, half = (warp - 4) >> 2;

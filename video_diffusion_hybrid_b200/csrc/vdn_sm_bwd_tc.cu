@@ -304,9 +304,9 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
         }
         issued = s + 1;
       }
-      mbar_wait(bar(B_QD), 0, ctl);
+      mbar_drain(bar(B_QD), 0);
       for (int s = issued - ST < 0 ? 0 : issued - ST; s < issued; ++s)
-        mbar_wait(bar(B_FULL + s % ST), (s / ST) & 1, ctl);
+        mbar_drain(bar(B_FULL + s % ST), (s / ST) & 1);
     }
   } else if (warp == 1) {
     // ---- MMA issuer
@@ -388,7 +388,7 @@ k_sbwd_q_tc(Dims dm, Inputs in, const void* dyp, SmTcWork ws, float* dq, float* 
       }
       mma_commit(bar(B_DQ));
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, ctl);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     // ---- softmax: two warps per TMEM lane quadrant, each with half the columns
@@ -638,9 +638,9 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
       issued = j + 1;
     }
     if (lane == 0) {
-      mbar_wait(bar(B_KV), 0, ctl);
+      mbar_drain(bar(B_KV), 0);
       for (int j = issued - ST < 0 ? 0 : issued - ST; j < issued; ++j)
-        mbar_wait(bar(B_FULL + j % ST), (j / ST) & 1, ctl);
+        mbar_drain(bar(B_FULL + j % ST), (j / ST) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -679,7 +679,7 @@ k_sbwd_kv_tc(Dims dm, SmTcWork ws, float* dk, float* dv, const __grid_constant__
       }
       mma_commit(bar(B_DONE));
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, ctl);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     // ---- softmax: two warps per TMEM lane quadrant, each with half the query columns

@@ -291,9 +291,9 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       }
       // drain: every copy issued into this CTA's shared memory has landed
       // (the last tile issued into each stage is one of the last KST)
-      mbar_wait(bar(B_Q), 0, ctl);
+      mbar_drain(bar(B_Q), 0);
       for (int jj = nk - KST < 0 ? 0 : nk - KST; jj < nk; ++jj)
-        mbar_wait(bar(B_KFULL + jj % KST), (jj / KST) & 1, ctl);
+        mbar_drain(bar(B_KFULL + jj % KST), (jj / KST) & 1);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ V producer
@@ -311,7 +311,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         nv = j + 1;
       }
       for (int jj = nv - VST < 0 ? 0 : nv - VST; jj < nv; ++jj)
-        mbar_wait(bar(B_VFULL + jj % VST), (jj / VST) & 1, ctl);
+        mbar_drain(bar(B_VFULL + jj % VST), (jj / VST) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -375,7 +375,7 @@ k_softmax_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
       }
       // drain: completion of every MMA issued by this thread
       mma_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, ctl);
+      mbar_drain(bar(B_DRAIN), 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax

@@ -100,6 +100,11 @@ def gather_output(y: torch.Tensor, group=None) -> torch.Tensor:
     return head_to_seq(y.flatten(1, 2), group, 2)
 
 
+def to_device(t: dict, device) -> dict:
+    """The tensors of t on `device` (no copy for those already there)."""
+    return {k: v.to(device, non_blocking=False) for k, v in t.items()}
+
+
 class UlyssesHybridAttention:
     """The hybrid attention core over P ranks (one per GPU): sequence-sharded
     inputs in, sequence-sharded output out, heads split over the ranks inside.
@@ -115,9 +120,12 @@ class UlyssesHybridAttention:
         self.core = HybridAttention(self.local_cfg, device)
 
     def __call__(self, t_local: dict, stream=None) -> torch.Tensor:
-        t = shard_inputs(t_local, self.cfg.T, self.cfg.N, self.cfg.H, self.group)
+        # the exchange runs where the inputs are: on the GPU with NCCL, or on
+        # host copies with a host backend (gloo), the core on the GPU either way
+        where = t_local["q"].device
+        t = to_device(shard_inputs(t_local, self.cfg.T, self.cfg.N, self.cfg.H, self.group), self.core.device)
         self._last = t  # the head-sharded inputs of the last call, for device_status
-        return gather_output(self.core(t, stream=stream), self.group)
+        return gather_output(self.core(t, stream=stream).to(where), self.group)
 
     def device_status(self) -> tuple:
         """(status, kernel tag) of this rank's last core call (synchronises)."""
