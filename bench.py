@@ -565,7 +565,7 @@ def run_proj(args):
         "metric": "layer output projection (one GEMM over the concat axis)", "value": tflops, "unit": "TFLOP/s",
         "ms_per_step": ms, "gemm_ms": gemm_ms, "steps": args.steps, "n_gpus": 1, "higher_is_better": True,
         "dtype": "fp8_e4m3" if args.fp8 else "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "library": "cuBLASLt",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "kernel": "k_gemm_tc (tcgen05, CTA pairs)",
                    "step": "quantise y + FP8 GEMM" if args.fp8 else "bf16 GEMM"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
                      "peak_source": f"bf16_tflops ({src})" + (" x 2 (nominal fp8 / bf16)" if args.fp8 else "")},

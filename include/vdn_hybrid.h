@@ -242,7 +242,8 @@ enum {
   VDN_TAG_SCAN = 4,         /* state scans                                      */
   VDN_TAG_COMPOSE = 5,      /* chunk composition                                */
   VDN_TAG_SOFTMAX_BWD = 6,  /* softmax branch backward                          */
-  VDN_TAG_LINEAR_BWD = 7    /* linear branch backward                           */
+  VDN_TAG_LINEAR_BWD = 7,   /* linear branch backward                           */
+  VDN_TAG_PROJ = 8          /* output projection (vdn_proj_device_status)       */
 };
 
 /* Reads the device status words left by the most recent call on this
@@ -459,10 +460,12 @@ typedef struct {
 /* out = y w on `stream`: y bfloat16 [M, K] row-major (the core's output with
  * y_dtype VDN_BF16), w bfloat16 [K, N] row-major, out [M, N] row-major in
  * out_dtype; fp32 accumulation.  Device pointers, 16-byte aligned, no overlap
- * of out with y or w.  A plain dense GEMM run by cuBLASLt without workspace
- * (a cuBLASLt handle is created on the first call of the process).  Errors:
- * VDN_ERR_INVALID_ARG (a NULL or misaligned pointer, sizes), VDN_ERR_UNSUPPORTED
- * (no GEMM algorithm for the sizes), VDN_ERR_CUDA. */
+ * of out with y or w.  On the tensor cores (tcgen05, pairs of CTAs on 256 x 256
+ * output tiles); no workspace, nothing allocated.  The bounded waits of its
+ * kernel record a timeout in library-owned status words (vdn_proj_device_status).
+ * Calls that overlap on the GPU share those words.  Errors: VDN_ERR_INVALID_ARG
+ * (a NULL or misaligned pointer, sizes), VDN_ERR_UNSUPPORTED (more than 2^30
+ * output tiles), VDN_ERR_CUDA. */
 vdn_status vdn_out_proj(const vdn_proj_cfg *cfg, const void *y, const void *w, void *out, vdn_stream_t stream);
 
 /* ------------------------------------------------------------ FP8 linear layers
@@ -482,10 +485,17 @@ vdn_status vdn_quantize_fp8(const void *x, int x_dtype, size_t n, void *q, float
  * e4m3 [M, K] row-major, the weight given TRANSPOSED as w_t e4m3 [N, K]
  * row-major (FP8 tensor-core GEMMs take both operands K-contiguous), scales =
  * {s_y, s_w} (two floats in device memory, e.g. as written by
- * vdn_quantize_fp8), out in cfg->out_dtype; fp32 accumulation, cuBLASLt, no
+ * vdn_quantize_fp8), out in cfg->out_dtype; fp32 accumulation on the tensor
+ * cores (tcgen05 kind::f8f6f4, the scales applied in the epilogue), no
  * workspace.  K and N multiples of 16.  Errors as vdn_out_proj. */
 vdn_status vdn_out_proj_fp8(const vdn_proj_cfg *cfg, const void *y, const void *w_t, const float *scales, void *out,
                             vdn_stream_t stream);
+
+/* Status of the last vdn_out_proj / vdn_out_proj_fp8 on the current device
+ * (synchronises `stream`): VDN_OK, or VDN_ERR_TIMEOUT when a bounded wait of its
+ * kernel gave up (the output is then incomplete); *where (if not NULL) gets
+ * VDN_TAG_PROJ or VDN_TAG_NONE.  Errors: VDN_ERR_CUDA. */
+vdn_status vdn_proj_device_status(vdn_stream_t stream, unsigned *where);
 
 #ifdef __cplusplus
 }

@@ -415,6 +415,27 @@ def test_out_proj_matches_oracle(out_dtype, M, H, dv, n):
     assert np.all(np.abs(got - ref) <= tol)
 
 
+@pytest.mark.parametrize("out_dtype", [L.VDN_F32, L.VDN_BF16])
+@pytest.mark.parametrize("M,K,N", [(2000, 144, 520), (4099, 1280, 768), (300, 6144, 3072)])
+def test_out_proj_tile_edges(out_dtype, M, K, N):
+    """The tensor-core projection at its tile edges: rows past M in the last
+    256-row tile, columns past N in the last 256-column tile, a last K block
+    of 16 of 64 values (K = 144), several tiles per CTA pair, and the layer's
+    K = 6,144; against the oracle's float64 product of the same bf16 values."""
+    r = np.random.default_rng(M + K + N)
+    yt = _bf16_tensor(r.standard_normal((M, K)))
+    wt = _bf16_tensor(r.standard_normal((K, N)) / np.sqrt(K))
+    out = torch.full((M, N), float("nan"), dtype=torch.float32 if out_dtype == L.VDN_F32 else torch.bfloat16,
+                     device="cuda")
+    L.vdn_out_proj(M, K, N, out_dtype, yt, wt, out)
+    torch.cuda.synchronize()
+    assert L.vdn_proj_device_status() == (L.VDN_OK, 0)
+    ref = O.out_proj(yt.float().cpu().numpy().reshape(M, 1, 1, K), wt.float().cpu().numpy())
+    got = out.float().cpu().numpy().astype(np.float64)
+    tol = 2e-5 * np.abs(ref).max() + (2.0 ** -8 * np.abs(ref) if out_dtype == L.VDN_BF16 else 0.0)
+    assert np.all(np.abs(got - ref) <= tol)
+
+
 def test_out_proj_on_core_output():
     """The projection of the core's own bf16 output (out_mode 0) matches the
     oracle's projection of the oracle's output within the bf16-mode tolerance."""
@@ -477,11 +498,12 @@ def test_quantize_fp8_matches_oracle(src):
 
 
 @pytest.mark.parametrize("out_dtype", [L.VDN_F32, L.VDN_BF16])
-def test_out_proj_fp8_matches_oracle(out_dtype):
+@pytest.mark.parametrize("M,K,N", [(777, 512, 256), (2000, 208, 528), (300, 6144, 3072)])
+def test_out_proj_fp8_matches_oracle(out_dtype, M, K, N):
     """The FP8 projection of quantised operands against the oracle's float64
-    product of the same dequantised values."""
-    r = np.random.default_rng(9)
-    M, K, N = 777, 512, 256
+    product of the same dequantised values (ragged M and N tiles, a last K
+    block of 80 of 128 values at K = 208, and the layer's K = 6,144)."""
+    r = np.random.default_rng(9 + M)
     y = torch.from_numpy(r.standard_normal((M, K)).astype(np.float32)).cuda().to(torch.bfloat16)
     w_t = torch.from_numpy((r.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32)).cuda().to(torch.bfloat16)
     qy = torch.empty((M, K), dtype=torch.uint8, device="cuda")
@@ -492,6 +514,7 @@ def test_out_proj_fp8_matches_oracle(out_dtype):
     out = torch.empty((M, N), dtype=torch.float32 if out_dtype == L.VDN_F32 else torch.bfloat16, device="cuda")
     L.vdn_out_proj_fp8(M, K, N, out_dtype, qy, qw, scales, out)
     torch.cuda.synchronize()
+    assert L.vdn_proj_device_status() == (L.VDN_OK, 0)
     sy, sw = scales.cpu().numpy()
     ref = O.out_proj_fp8(qy.cpu().view(torch.float8_e4m3fn), sy, qw.cpu().view(torch.float8_e4m3fn), sw)
     got = out.float().cpu().numpy().astype(np.float64)

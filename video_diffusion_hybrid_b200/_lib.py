@@ -26,7 +26,7 @@ EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vd
             "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn",
             "vdn_quantize_fp8", "vdn_out_proj_fp8", "vdn_hybrid_lin_bwd_workspace_size", "vdn_hybrid_lin_bwd",
             "vdn_hybrid_sm_bwd_workspace_size", "vdn_hybrid_sm_bwd", "vdn_hybrid_bwd_workspace_size", "vdn_hybrid_bwd",
-            "vdn_debug_set_read_wait_limit")
+            "vdn_debug_set_read_wait_limit", "vdn_proj_device_status")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -162,6 +162,8 @@ def lib() -> C.CDLL:
         L.vdn_hybrid_bwd_workspace_size.argtypes = [C.POINTER(VdnCfg)]
         L.vdn_hybrid_bwd.restype = C.c_int
         L.vdn_hybrid_bwd.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.POINTER(VdnGrads), C.c_void_p]
+        L.vdn_proj_device_status.restype = C.c_int
+        L.vdn_proj_device_status.argtypes = [C.c_void_p, C.POINTER(C.c_uint)]
         L.vdn_debug_set_read_wait_limit.restype = C.c_int
         L.vdn_debug_set_read_wait_limit.argtypes = [C.c_ulonglong]
         L.vdn_status_string.restype = C.c_char_p
@@ -369,3 +371,11 @@ def vdn_debug_set_read_wait_limit(cycles: int, check: bool = True) -> int:
     if check and st != VDN_OK:
         raise VdnError(st, "vdn_debug_set_read_wait_limit")
     return st
+
+
+def vdn_proj_device_status(stream=None) -> tuple:
+    """(status, kernel tag) of the last output projection on the current
+    device (synchronises the stream)."""
+    where = C.c_uint(0)
+    st = lib().vdn_proj_device_status(_stream_handle(stream), C.byref(where))
+    return st, where.value

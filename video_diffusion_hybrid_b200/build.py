@@ -57,11 +57,8 @@ def build(verbose_ptxas: bool = False) -> str:
         objs = list(ex.map(lambda s: _compile(s, extra), srcs))
     newest = max(os.path.getmtime(o) for o in objs)
     if not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
-        # cuBLASLt serves the layer's output projection (a plain GEMM); the
-        # toolkit's library directory is recorded so the .so loads on its own
-        cuda_lib = os.path.join(os.path.dirname(os.path.dirname(nvcc())), "lib64")
-        cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", LIB] + objs + \
-            ["-lcublasLt", "-Xlinker", "-rpath=" + cuda_lib]
+        # only the CUDA runtime (linked statically by nvcc): every kernel is the library's own
+        cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", LIB] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -410,6 +410,10 @@ bool make_token_map(CUtensorMap* m, const void* base, long long tokens, int H, i
 // `box_rows` rows, 128-byte swizzle.
 bool make_matrix_map(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows);
 
+// 2-D map over a row-major [rows][cols] byte matrix (e4m3 codes); box = 128
+// cols x `box_rows` rows, 128-byte swizzle.
+bool make_matrix_map_u8(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows);
+
 // 2-D map over a row-major [rows][cols] fp32 matrix; box = 32 cols x
 // `box_rows` rows, 128-byte swizzle.
 bool make_matrix_map_f32(CUtensorMap* m, const void* base, long long rows, int cols, int box_rows);

@@ -487,6 +487,17 @@ vdn_status vdn_out_proj_fp8(const vdn_proj_cfg* cfg, const void* y, const void* 
   return out_proj(cfg->M, cfg->K, cfg->N, cfg->out_dtype, y, w_t, out, reinterpret_cast<cudaStream_t>(stream), scales);
 }
 
+vdn_status vdn_proj_device_status(vdn_stream_t stream, unsigned* where) {
+  uint32_t* st = status_of_proj();
+  if (!st) return VDN_ERR_CUDA;
+  uint32_t host[2] = {0, 0};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host, st, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (where) *where = host[1];
+  return host[0] ? VDN_ERR_TIMEOUT : VDN_OK;
+}
+
 const char* vdn_status_string(vdn_status s) {
   switch (s) {
     case VDN_OK: return "ok";

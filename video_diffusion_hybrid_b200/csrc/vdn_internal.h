@@ -93,10 +93,12 @@ cudaError_t launch_read_big(const Dims& d, const Inputs& in, const Work& w, cuda
 // chunks = false: the frame-stepped scan; true: stepped by the chunk maps of launch_compose_tc
 cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s, bool chunks);
 cudaError_t launch_compose_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
-// out[M, N] = y[M, K] w[K, N] (bf16 operands, fp32 accumulation), cuBLASLt
+// out[M, N] = y[M, K] w[K, N] (bf16 operands, fp32 accumulation), tensor cores (vdn_gemm_tc.cu);
 // scales != nullptr: e4m3 y [M, K] and w [N, K], dequantisation scales {s_y, s_w} in device memory
 vdn_status out_proj(int M, int K, int N, int out_dtype, const void* y, const void* w, void* out, cudaStream_t s,
                     const float* scales = nullptr);
+// device address of the projection's status words (library-owned), or null
+uint32_t* status_of_proj();
 vdn_status quantize_fp8(const void* x, int dtype, long long n, void* q, float* scale, cudaStream_t s);
 // The chunk-composed scan where it helps: the compositions (one CTA per
 // chunk, batch-head and direction) take about one wave of the SMs, and then
