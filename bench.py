@@ -76,7 +76,7 @@ def oracle_prepare(workload, seed_offset=0):
     return inp, cfg
 
 
-def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
+def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None, vda_only=False):
     """Time the fp64 oracle on a bounded sample of head 0 of the workload: the
     full bidirectional VDA chain of the head (text solve, every frame's solve,
     both scans), both branches for every query of the non-anchor frames in
@@ -84,8 +84,9 @@ def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
     With `target_s`, further whole non-anchor frames (spread over the
     sequence) are added until the sample holds about that much CPU work.
     The per-frame costs are extrapolated to all frames of the head and the
-    head's cost to all B x H heads.  Returns (tokens/s, seconds of CPU work,
-    description)."""
+    head's cost to all B x H heads.  With `vda_only`, the frames' cost is the
+    linear branch alone (the read and its RMSNorm and gate).  Returns
+    (tokens/s, seconds of CPU work, description)."""
     from oracle import vdn_oracle as O
     inp, cfg = prep
     s = workload.shape
@@ -101,8 +102,9 @@ def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
         t1 = time.perf_counter()
         R = O.read_state(F, G, t, s.T, cfg.chunk, cfg.anchors)
         O.rms_gate(q[t, :n] @ R.T, inp["gate_lin"][0, t, :n, 0], cfg.rms_eps)
-        o = O.softmax_frame(q[t, :n], k, v, t, s.T, cfg.chunk, cfg.anchors, cfg.scale)
-        O.sigmoid(inp["gate_sm"][0, t, :n, 0]) * o
+        if not vda_only:
+            o = O.softmax_frame(q[t, :n], k, v, t, s.T, cfg.chunk, cfg.anchors, cfg.scale)
+            O.sigmoid(inp["gate_sm"][0, t, :n, 0]) * o
         return time.perf_counter() - t1
 
     frames = list(frames)
@@ -121,7 +123,8 @@ def oracle_sample(workload, prep, frames=None, n_anchor_q=None, target_s=None):
                 + n_anchor * c_anchor * s.N / n_anchor_q)
     layer = per_head * s.H * s.B
     work = t_chain + sum(c_frames) + c_anchor
-    desc = (f"head 0 of {workload.name}: the full VDA chain over {s.T} frames, both branches for all {s.N} "
+    what = "the linear branch" if vda_only else "both branches"
+    desc = (f"head 0 of {workload.name}: the full VDA chain over {s.T} frames, {what} for all {s.N} "
             f"queries of {len(frames)} non-anchor frames spread over the sequence and {n_anchor_q} queries of "
             f"anchor frame 0; costs extrapolated to {s.T} frames x {s.B * s.H} heads")
     return s.B * s.T * s.N / layer, work, desc
@@ -323,8 +326,8 @@ def run_ours(args):
     w = WORKLOADS[args.workload]
     s = w.shape
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.vda_only and args.update == 0:
-        val, work, desc = oracle_sample(w, oracle_prepare(w), target_s=12.0)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.update == 0:
+        val, work, desc = oracle_sample(w, oracle_prepare(w), target_s=12.0, vda_only=args.vda_only)
         cpu = {"value": val, "unit": UNIT, "cores": host_cores(), "kind": "oracle", "sample": desc,
                "sample_cpu_seconds": round(work, 2)}
 

@@ -9,13 +9,12 @@
 // eigenvalue >= 1, so symmetric Gauss-Jordan elimination (the sweep operator)
 // needs no pivoting: each pivot is a Schur complement of I + A_t and is >= 1.
 // Sweeping all d pivots turns G = I + A into -G^-1 in d^3 multiply-adds, the
-// same work as Cholesky + triangular inverse + W^T W, in one pass with one
-// barrier per two pivots (sweep.cuh) and every thread busy.
+// same work as Cholesky + triangular inverse + W^T W, in one pass: a panel of
+// d / 16 pivots per round, two barriers per round (sweep.cuh).
 //
 // Thread (ty, tx) of a 16 x 16 grid keeps the R x R block G[ty R + a][tx R + c]
-// (R = d / 16) in registers.  The only exchange per pivot is row p (column p
-// equals it by symmetry), and the pivot loop is unrolled by R so the owner
-// reads its row from a fixed register.  The sweep's special rules for row p,
+// (R = d / 16) in registers.  The only exchange per round is the panel's
+// rows (its columns equal them by symmetry).  The sweep's special rules for row p,
 // column p and the pivot itself are folded into the one rank-one update by
 // broadcasting g_pp - 1 in place of g_pp:
 //   g_ij - g_ip (g_pj / g_pp)              (i, j != p)  the ordinary update
@@ -54,11 +53,10 @@ __global__ void __launch_bounds__(kThreadsS, 2)
 k_solve_sweep(Dims dm, Work w) {
   constexpr int R = D / 16;   // register tile edge
   constexpr int P = D + 4;    // shared pitch (16-byte rows)
-  constexpr int BP = D + 4;   // pivot buffers: rows p and p + 1, then Z at [D], [D + 1]
   static_assert(R % 2 == 0, "pivot buffers alternate with the parity of p");
   extern __shared__ float sm[];
-  float* rowbuf = sm;         // [4][BP]
-  float* Ms = sm + 4 * BP;    // [D][P]
+  float* rowbuf = sm;                           // the sweep's rows, Z and V
+  float* Ms = sm + sweep_panel_floats<D>();     // [D][P]
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (!TEXT && is_anchor(dm, t)) return;
@@ -77,7 +75,7 @@ k_solve_sweep(Dims dm, Work w) {
     if (ty == tx) g[a][a] += 1.0f;
   }
 
-  sweep_regs<D>(g, rowbuf);  // g = -G^-1
+  sweep_panels<D>(g, rowbuf);  // g = -G^-1
 
   // the tensor-core scan forms (alpha S + B_t) M_t itself: no C_t
   const bool skip_c = !TEXT && w.bform;
@@ -134,7 +132,7 @@ k_solve_sweep(Dims dm, Work w) {
 
 template <int D, bool TEXT>
 cudaError_t launch(const Dims& d, const Work& w, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (size_t)(4 * (D + 4) + D * (D + 4));
+  const size_t smem = sizeof(float) * (size_t)(sweep_panel_floats<D>() + D * (D + 4));
   auto kern = k_solve_sweep<D, TEXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
