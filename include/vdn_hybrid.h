@@ -173,9 +173,9 @@ enum {
  *   text_gram  : [B,H,2,d,d]          A_x, B_x of the text tokens (tensor-core text
  *                                     path only)
  *   frame_M16  : [B,T,H,2,d,d]        bfloat16 hi/lo split of frame_M, the operand of the
- *                                     tensor-core scan (bf16 inputs with d = 128 only;
+ *                                     tensor-core scans (bf16 inputs with d = 128 or 256;
  *                                     an empty region otherwise)
- *   chunk_P16  : [B,C,H,2,d,d]        chunk maps (same condition): bfloat16 hi/lo split of
+ *   chunk_P16  : [B,C,H,2,d,d]        chunk maps (bf16, d = 128 only): bfloat16 hi/lo split of
  *                                     P_c = M_f1 ... M_fn over the chunk's written frames
  *   chunk_C    : [2,B,C,H,d_v,d_k]    the forward and backward constants Cf_c, Cb_c: the
  *                                     frames of chunk c map a state S to Lam_c S P_c + Cf_c

@@ -60,6 +60,12 @@ def test_workspace_size_and_layout():
                              "read_table_bf16", "text_gram", "frame_M16", "chunk_P16", "chunk_C", "chunk_lam",
                              "total")]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    # d = 256, bf16: M's split for the tensor-core scan, no chunk maps
+    big = L.vdn_hybrid_workspace_layout(_cfg(d_k=256, d_v=256))
+    assert big["chunk_P16"] - big["frame_M16"] >= 90 * 24 * 2 * 256 * 256 * 2
+    assert big["chunk_P16"] == big["chunk_C"] == big["chunk_lam"] == big["total"]
+    f32 = L.vdn_hybrid_workspace_layout(_cfg(dtype=L.VDN_F32))
+    assert f32["frame_M16"] == f32["total"]
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -176,7 +176,10 @@ def test_d256_vda_matches_oracle(shape):
                                   np.asarray(inp["v"][b, f, :, h], np.float64),
                                   np.asarray(inp["beta"][b, f, :, h], np.float64))[1]
                 np.testing.assert_allclose(it["C"][b, f, h], Bf, atol=2e-5 * np.abs(Bf).max())
-            np.testing.assert_allclose(it["R"][b, h], ref["R"], atol=1e-4 * np.sqrt(np.mean(ref["R"] ** 2)) + 1e-30)
+            # the tensor-core scan's three-term bf16 split leaves about 2^-18 relative per
+            # product term and a step sums d of them: the bar of the d = 128 read table,
+            # 1e-4 * RMS, scaled by d / 128
+            np.testing.assert_allclose(it["R"][b, h], ref["R"], atol=2e-4 * np.sqrt(np.mean(ref["R"] ** 2)) + 1e-30)
     ref_y = O.hybrid_attn(inp, ocfg(cfg))
     assert rel_err(y[..., 1, :], ref_y[..., 1, :]) <= TOL["bf16"]
     # the softmax stage has no kernel at this size: refused before any launch

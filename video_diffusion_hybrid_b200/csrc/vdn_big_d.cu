@@ -187,6 +187,25 @@ k_solve_block(Dims dm, Work w) {
   mm128<false, true, true>(g, T0, T2);
   tile_st(blk(gM, 0, 0), DB, g, 1.f);
   __syncthreads();  // M complete in global memory
+  if (!TEXT && w.M16 != nullptr) {
+    // operand of the tensor-core scan: M's bf16 [hi | lo] rows, 8 entries a thread per pass
+    __nv_bfloat16* mh = static_cast<__nv_bfloat16*>(w.M16) + fh * 2 * DD;
+    for (int e = threadIdx.x * 8; e < DD; e += kThreadsB * 8) {
+      const float4 x0 = *reinterpret_cast<const float4*>(gM + e), x1 = *reinterpret_cast<const float4*>(gM + e + 4);
+      const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      uint32_t hv[4], lv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat16 a = __float2bfloat16_rn(x[2 * j]), c = __float2bfloat16_rn(x[2 * j + 1]);
+        const __nv_bfloat16 ra = __float2bfloat16_rn(x[2 * j] - __bfloat162float(a));
+        const __nv_bfloat16 rc = __float2bfloat16_rn(x[2 * j + 1] - __bfloat162float(c));
+        hv[j] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(c) << 16);
+        lv[j] = (uint32_t)__bfloat16_as_ushort(ra) | ((uint32_t)__bfloat16_as_ushort(rc) << 16);
+      }
+      *reinterpret_cast<uint4*>(mh + e) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      *reinterpret_cast<uint4*>(mh + DD + e) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+    }
+  }
   // frames: the scan steps S <- (alpha S + B_t) M_t itself, B_t stays in the C_t slot
   if (!TEXT && w.bform) return;
 

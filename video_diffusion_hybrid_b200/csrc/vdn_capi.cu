@@ -71,8 +71,9 @@ void layout_of(const vdn_hybrid_cfg* c, vdn_workspace_layout* L) {
   L->text_gram = off;  off += up(bh * 2 * dd);
   const bool tc_scan = scan_tc_layout(c->dtype == VDN_BF16, c->d_k, c->d_v);
   const size_t kk2 = 2 * (size_t)c->d_k * c->d_k * sizeof(__nv_bfloat16);  // one hi/lo split
+  const bool m16 = tc_scan || scan256_layout(c->dtype == VDN_BF16, c->d_k, c->d_v);
   L->frame_M16 = off;
-  if (tc_scan) off += up(bh * (size_t)c->T * kk2);
+  if (m16) off += up(bh * (size_t)c->T * kk2);
   L->chunk_P16 = off;
   if (tc_scan) off += up(bh * C * kk2);
   L->chunk_C = off;
@@ -125,8 +126,9 @@ Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
   w.R = reinterpret_cast<float*>(base + L.read_table);
   w.R16 = base + L.read_table_bf16;
   w.text_gram = reinterpret_cast<float*>(base + L.text_gram);
-  const bool tc_scan = L.chunk_P16 > L.frame_M16;
-  w.M16 = tc_scan ? base + L.frame_M16 : nullptr;
+  // the chunk maps exist for the d = 128 tensor-core scan only, M's split for both
+  const bool tc_scan = scan_tc_layout(c->dtype == VDN_BF16, c->d_k, c->d_v);
+  w.M16 = L.chunk_P16 > L.frame_M16 ? base + L.frame_M16 : nullptr;
   w.P16 = tc_scan ? base + L.chunk_P16 : nullptr;
   w.Cf = tc_scan ? reinterpret_cast<float*>(base + L.chunk_C) : nullptr;
   w.Cb = tc_scan ? w.Cf + (size_t)c->B * c->H * ((c->T + c->chunk - 1) / c->chunk) * c->d_v * c->d_k
@@ -182,7 +184,7 @@ int vdn_hybrid_stage_impl(const vdn_hybrid_cfg* cfg, unsigned stage) {
   Dims d = make_dims(cfg);
   switch (stage) {
     case VDN_STAGE_SCAN:
-      return scan_tc_supported(d) ? 1 : 0;
+      return (scan_tc_supported(d) || scan256_tc_supported(d)) ? 1 : 0;
     case VDN_STAGE_SOLVE:
       if (d.update != 0) return 2;  // the variant-map kernel
       return gram_tc_supported(d) ? 1 : 0;
@@ -241,7 +243,8 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
     }
   }
   if (big && (stages & VDN_STAGE_SCAN)) {
-    if (launch_scan_big(d, in, w, s) != cudaSuccess) return VDN_ERR_CUDA;
+    e = (scan256_tc_supported(d) && w.M16 != nullptr) ? launch_scan256_tc(d, in, w, s) : launch_scan_big(d, in, w, s);
+    if (e != cudaSuccess) return VDN_ERR_CUDA;
   } else if (stages & VDN_STAGE_SCAN) {
     // the tensor-core scan reads the bf16 split of M that the sweep solve
     // writes; with enough chunks it first composes each chunk's frame maps

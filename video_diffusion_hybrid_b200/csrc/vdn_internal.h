@@ -38,7 +38,7 @@ struct Work {
   float* R;          // [B,H,C+1,dv,dk]
   void* R16;         // [B,H,C+1,2,dv,dk] bf16 (hi, lo)
   float* text_gram;  // [B,H,2,dk,dk] A_x, B_x
-  void* M16;         // [B,T,H,2,dk,dk] bf16 (hi, lo) of M; nullptr off the tensor-core scan
+  void* M16;         // [B,T,H,2,dk,dk] bf16 (hi, lo) of M; nullptr off the tensor-core scans
   // chunk maps (tensor-core scan only): P_c split, [Cf; Cb], Lam
   void* P16;         // [B,C,H,2,dk,dk] bf16 (hi, lo) of P_c
   float* Cf;         // [B,C,H,dv,dk]; Cb follows at Cf + B*C*H*dv*dk
@@ -93,6 +93,11 @@ cudaError_t launch_read_big(const Dims& d, const Inputs& in, const Work& w, cuda
 // chunks = false: the frame-stepped scan; true: stepped by the chunk maps of launch_compose_tc
 cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s, bool chunks);
 cudaError_t launch_compose_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+// d = 256, bf16: the frame scan on the tensor cores (a CTA pair per chain), from
+// the bf16 hi/lo split of M_t that the block solve writes
+__host__ __device__ inline bool scan256_layout(bool bf16, int dk, int dv) { return bf16 && dk == 256 && dv == 256; }
+bool scan256_tc_supported(const Dims& d);
+cudaError_t launch_scan256_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 // out[M, N] = y[M, K] w[K, N] (bf16 operands, fp32 accumulation), tensor cores (vdn_gemm_tc.cu);
 // scales != nullptr: e4m3 y [M, K] and w [N, K], dequantisation scales {s_y, s_w} in device memory
 vdn_status out_proj(int M, int K, int N, int out_dtype, const void* y, const void* w, void* out, cudaStream_t s,

@@ -400,6 +400,330 @@ k_scan_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm, c
   if (warp == 1) tmem_free2(tmem, kTmemScan);
 }
 
+// ----------------------------------------------------------- d = 256 --
+// The same frame scan at d = 256, S <- (alpha_t S + B_t) M_t.  The state
+// rows split over a CTA pair again, now 128 rows per CTA, and each step is
+// one tcgen05.mma.cta_group::2 product with M = 256 (the pair) and N = 256
+// (each CTA holds the 128 rows of M_t's split that are its half of B), K =
+// 256, over the same three bf16 hi/lo terms.  The A operand, this CTA's rows
+// of X = alpha S + B_t as hi | lo, lives in TMEM (columns 256..383 and
+// 384..511, two bf16 a column: the TS form), next to the accumulator
+// (columns 0..255: lane = row of this CTA's share, column = state column).
+// Shared memory holds a ring of three stages of M_t's split, each one
+// 64-wide K-chunk of both terms (32 KB; the product of a chunk's three terms
+// releases its stage), and the next frame's B_t rows as eight boxes of 32
+// columns (fp32, 16 KB each), loaded by TMA while the product runs.
+// Epilogue warps 4..11: warp w takes TMEM lanes 32 (w mod 4) .. + 31 and the
+// columns 128 ((w - 4) / 4) .. + 127 (boxes 4 ((w - 4) / 4) .. + 3), in four
+// groups of 32.
+namespace s256 {
+constexpr int D = 256;
+constexpr int R = 128;                   // state rows per CTA
+constexpr int kThreads = 384;
+constexpr uint32_t CHUNK = R * 128;      // 64 K-columns of a 128-row bf16 operand (SW128): 16 KB
+constexpr uint32_t STAGE = 2 * CHUNK;    // hi | lo of one K-chunk of this CTA's half of M_t: 32 KB
+constexpr int ST = 3;                    // ring stages
+constexpr int KCH = D / 64;              // K-chunks per step
+constexpr uint32_t CBOX = R * 128;       // 32 fp32 columns x 128 rows (SW128): 16 KB
+constexpr uint32_t kTmem = 512;
+constexpr uint32_t COL_AHI = 256, COL_ALO = 384;
+// FULL lives on the leader (both CTAs' bytes), EMPTY is committed by the
+// leader's MMAs to both CTAs, SREADY takes one arrival per epilogue warp of
+// the pair; CFULL / CEMPTY (one per column half) guard this CTA's B_t boxes.
+enum { B_FULL = 0, B_EMPTY = ST, B_CFULL = 2 * ST, B_CEMPTY = 2 * ST + 2, B_SREADY = 2 * ST + 4, B_MDONE, B_DRAIN,
+       NBARS };
+
+__host__ __device__ constexpr size_t smem_bytes() { return 1024 + ST * (size_t)STAGE + 8 * (size_t)CBOX + NBARS * 8 + 16; }
+
+// A operand from TMEM for the pair (bf16 pairs packed in 32-bit columns, lane = row)
+__device__ __forceinline__ void mma2_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// 32 values of X (K-columns col .. col + 31 of this lane's row) into the A
+// operand's hi and lo columns
+__device__ __forceinline__ void split_to_tmem(uint32_t lane_addr, int col, const float (&x)[32]) {
+  uint32_t hv[16], lv[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float x0 = x[2 * j], x1 = x[2 * j + 1];
+    hv[j] = pack_bf16(x0, x1);
+    lv[j] = pack_bf16(x0 - __uint_as_float(hv[j] << 16), x1 - __uint_as_float(hv[j] & 0xFFFF0000u));
+  }
+  tmem_st16(lane_addr + COL_AHI + col / 2, hv);
+  tmem_st16(lane_addr + COL_ALO + col / 2, lv);
+}
+
+// this lane's 32 values of box `box` (its row of the CTA's share)
+__device__ __forceinline__ void box32(const unsigned char* sC, int box, int srow, float (&v)[32]) {
+  const unsigned char* p = sC + box * CBOX + srow * 128;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const float4 a = *reinterpret_cast<const float4*>(p + ((u ^ (srow & 7)) << 4));
+    v[4 * u] = a.x; v[4 * u + 1] = a.y; v[4 * u + 2] = a.z; v[4 * u + 3] = a.w;
+  }
+}
+
+__device__ __forceinline__ void ld32(const float* src, float (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(src) + u);
+    v[4 * u] = a.x; v[4 * u + 1] = a.y; v[4 * u + 2] = a.z; v[4 * u + 3] = a.w;
+  }
+}
+
+__device__ __forceinline__ void snap32(const Dims& dm, int dir, const Slots& sl, float* snap_row, int col,
+                                       const float (&v)[32]) {
+  const long long DD = (long long)D * D;
+  if (sl.a >= 0) store_row32(snap_row + sl.a * DD + col, v);
+  if (sl.b >= 0) store_row32(snap_row + sl.b * DD + col, v);
+  for (int p = sl.p0; p < sl.p1; ++p) {
+    const int k = snap_slot(dm, dir, p);
+    if (k >= 0) store_row32(snap_row + k * DD + col, v);
+  }
+}
+}  // namespace s256
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(s256::kThreads, 1)
+k_scan256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmm,
+             const __grid_constant__ CUtensorMap tmc) {
+  constexpr int D = s256::D, R = s256::R, ST = s256::ST, KCH = s256::KCH;
+  constexpr uint32_t CHUNK = s256::CHUNK, STAGE = s256::STAGE, CBOX = s256::CBOX;
+  constexpr int B_FULL = s256::B_FULL, B_EMPTY = s256::B_EMPTY, B_CFULL = s256::B_CFULL, B_CEMPTY = s256::B_CEMPTY,
+                B_SREADY = s256::B_SREADY, B_MDONE = s256::B_MDONE, B_DRAIN = s256::B_DRAIN, NBARS = s256::NBARS;
+  using s256::box32;
+  using s256::ld32;
+  using s256::snap32;
+  using s256::split_to_tmem;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sB = sm;                // ST stages: a K-chunk of this CTA's half of M_t, hi | lo, K-major SW128
+  unsigned char* sC = sB + ST * STAGE;   // 8 boxes: this CTA's rows of the next B_t, fp32 SW128
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + 8 * CBOX);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // no early exit: both CTAs of the pair must reach the cluster barriers
+  const uint32_t rank = cta_rank();
+  const bool lead = rank == 0;
+  const int chain = blockIdx.x >> 1;
+  const int dir = chain & 1, bh = chain >> 1;
+  const int b = bh / dm.H, h = bh % dm.H;
+  const int row0 = R * (int)rank;
+  const Ctl ctl{abort_flag, w.status, (unsigned)TAG_SCAN_TC};
+  const long long DD = (long long)D * D;
+  auto bar = [&](int i) { return smem_u32(bars + i); };
+  auto lbar = [&](int i) { return map_rank(smem_u32(bars + i), 0); };
+  auto fh_of = [&](int t) { return ((long long)b * dm.T + t) * dm.H + h; };
+  int nw = 0;
+  for (int t = 0; t < dm.T; ++t) nw += is_anchor(dm, t) ? 0 : 1;
+
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < ST; ++k) {
+      mbar_init(bar(B_FULL + k), 1);
+      mbar_init(bar(B_EMPTY + k), 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(bar(B_CFULL + k), 1);
+      mbar_init(bar(B_CEMPTY + k), 4);  // the four epilogue warps of that column half
+    }
+    mbar_init(bar(B_SREADY), 16);
+    mbar_init(bar(B_MDONE), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc2(smem_u32(tmem_slot), s256::kTmem);
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Load g = i KCH + c (step i, K-chunk c) uses stage g mod ST, its
+  // (g / ST)-th use; FULL and EMPTY of a stage complete once per use.  B_t
+  // item k (the k-th written frame's rows, read by the epilogue that forms
+  // X_k) fills the boxes; CFULL / CEMPTY complete once per item.
+  if (warp == 0) {
+    if (lane == 0) {
+      const __nv_bfloat16* m16 = static_cast<const __nv_bfloat16*>(w.M16);
+      auto prefetch_step = [&](int pst) {
+        if (pst >= dm.T) return;
+        const long long pfh = fh_of(frame_at(dm, dir, pst));
+        prefetch_l2(m16 + ((pfh * 2) * D + row0) * D, R * D * 2);
+        prefetch_l2(m16 + ((pfh * 2 + 1) * D + row0) * D, R * D * 2);
+        prefetch_l2(w.Cm + (pfh * D + row0) * D, R * D * 4);
+      };
+      bool ok = true;
+      int nc[2] = {0, 0};  // items loaded, per column half
+      auto load_item = [&](int k, int kst) -> bool {
+        const long long crow = fh_of(frame_at(dm, dir, kst)) * D + row0;
+        for (int hf = 0; hf < 2; ++hf) {
+          if (k >= 1 && !mbar_wait_cl(bar(B_CEMPTY + hf), (k - 1) & 1, ctl)) return false;
+          mbar_expect_tx(bar(B_CFULL + hf), 4 * CBOX);
+          for (int x = 0; x < 4; ++x)
+            tma_load_2d(smem_u32(sC + (4 * hf + x) * CBOX), &tmc, bar(B_CFULL + hf), (4 * hf + x) * 32, (int)crow);
+          ++nc[hf];
+        }
+        return true;
+      };
+      int st = next_written(dm, dir, 0);
+      int pst = st;
+      prefetch_step(pst);
+      pst = next_written(dm, dir, pst + 1);
+      prefetch_step(pst);
+      if (nw > 0) ok = load_item(0, st);
+      int nl = 0;
+      for (int i = 0; ok && i < nw; ++i) {
+        const long long mrow = fh_of(frame_at(dm, dir, st));
+        const int st_next = next_written(dm, dir, st + 1);
+        pst = next_written(dm, dir, pst + 1);
+        prefetch_step(pst);
+        for (int c = 0; c < KCH; ++c) {
+          const int g = i * KCH + c, s = g % ST, u = g / ST;
+          if (u >= 1 && !mbar_wait_cl(bar(B_EMPTY + s), (u - 1) & 1, ctl)) { ok = false; break; }
+          if (lead) mbar_expect_tx(bar(B_FULL + s), 2 * STAGE);
+          for (int part = 0; part < 2; ++part)
+            tma_load_2d_pair(smem_u32(sB + s * STAGE + part * CHUNK), &tmm, lbar(B_FULL + s), c * 64,
+                             (int)((mrow * 2 + part) * D + row0));
+          ++nl;
+        }
+        // the next frame's B_t, once the epilogue has formed X_i from item i
+        if (ok && i + 1 < nw) ok = load_item(i + 1, st_next);
+        st = st_next;
+      }
+      // the last copies land before the pair can exit (the leader's FULL
+      // barriers count both CTAs' bytes); each is its stage's last use
+      for (int n = nl - ST < 0 ? 0 : nl - ST; lead && n < nl; ++n) mbar_drain(bar(B_FULL + n % ST), (n / ST) & 1);
+      for (int hf = 0; hf < 2; ++hf)
+        if (nc[hf] > 0) mbar_drain(bar(B_CFULL + hf), (nc[hf] - 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && lead) {
+      const uint32_t ID = idesc_bf16(2 * R, D, false);
+      const uint64_t b0 = sdesc(smem_u32(sB), 16, 1024);
+      bool ok = true;
+      for (int i = 0; ok && i < nw; ++i) {
+        if (!mbar_wait_cl(bar(B_SREADY), i & 1, ctl)) break;
+        tc_fence_after();
+        for (int c = 0; c < KCH; ++c) {
+          const int g = i * KCH + c, s = g % ST, u = g / ST;
+          if (!mbar_wait_cl(bar(B_FULL + s), u & 1, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t bs = dadd(b0, s * STAGE);
+#pragma unroll
+          for (int pass = 0; pass < 3; ++pass) {  // hi hi, hi lo, lo hi
+            const uint32_t acol = (pass == 2 ? s256::COL_ALO : s256::COL_AHI) + c * 32;
+            const uint32_t bo = pass == 1 ? CHUNK : 0u;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              s256::mma2_bf16_ts(tmem, tmem + acol + kk * 8, dadd(bs, bo + kk * 32), ID, (c | pass | kk) ? 1u : 0u);
+          }
+          commit2(bar(B_EMPTY + s));
+          commit2(map_rank(bar(B_EMPTY + s), 1));
+        }
+        if (!ok) break;
+        commit2(bar(B_MDONE));
+        commit2(map_rank(bar(B_MDONE), 1));
+      }
+      commit2(bar(B_DRAIN));
+      mbar_drain(bar(B_DRAIN), 0);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3, half = (warp - 4) >> 2;
+    const int srow = quad * 32 + lane;  // TMEM lane = row of this CTA's share
+    const int row = row0 + srow;        // state row
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    float* snap_row = (dir == 0 ? w.fsnap : w.bsnap) + (long long)bh * (dm.C + 1) * DD + (long long)row * D;
+    // item k's boxes of this column half, into X = a s + B_t and the A operand
+    // (s: four groups of 32 from `get`), then the half's boxes are released
+    int st = next_written(dm, dir, 0);
+    bool ok = true;
+    {
+      // start state: its own slot and those of leading unwritten frames; X_0
+      const float* start = (dir == 0 && in.fwd_init) ? in.fwd_init : w.half_text;
+      const float* src = start + (long long)bh * DD + (long long)row * D;
+      const int start_slot = dir == 0 ? 0 : dm.C;
+      const Slots sl = slots_of(dm, dir, 0, st);
+      const float a = nw > 0 ? __ldg(in.alpha + fh_of(frame_at(dm, dir, st))) : 0.f;
+      if (nw > 0) ok = __all_sync(0xffffffffu, mbar_wait_cl(bar(B_CFULL + half), 0, ctl));
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int col = 128 * half + 32 * j;
+        float sv[32];
+        ld32(src + col, sv);
+        store_row32(snap_row + start_slot * DD + col, sv);
+        snap32(dm, dir, sl, snap_row, col, sv);
+        if (nw > 0 && ok) {
+          float cv[32];
+          box32(sC, 4 * half + j, srow, cv);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) cv[u] = fmaf(a, sv[u], cv[u]);
+          split_to_tmem(lane_addr, col, cv);
+        }
+      }
+      if (nw > 0 && ok) {
+        mbar_arrive_warp(bar(B_CEMPTY + half));
+        tmem_wait_st();
+        tc_fence_before();
+        arrive_cluster_warp(lbar(B_SREADY));
+      }
+    }
+    for (int i = 0; ok && i < nw; ++i) {
+      const int st_next = next_written(dm, dir, st + 1);
+      const Slots sl = slots_of(dm, dir, st, st_next);
+      const bool more = i + 1 < nw;
+      const float a = more ? __ldg(in.alpha + fh_of(frame_at(dm, dir, st_next))) : 0.f;
+      if (!__all_sync(0xffffffffu, mbar_wait_cl(bar(B_MDONE), i & 1, ctl))) { ok = false; break; }
+      // item i + 1: the next frame's B_t
+      if (more && !__all_sync(0xffffffffu, mbar_wait_cl(bar(B_CFULL + half), (i + 1) & 1, ctl))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int col = 128 * half + 32 * j;
+        float v[32];
+        tmem_ld32(lane_addr + col, v);
+        tmem_wait_ld();
+        if (more) {
+          float cv[32];
+          box32(sC, 4 * half + j, srow, cv);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) cv[u] = fmaf(a, v[u], cv[u]);  // X = alpha_next S + B_next
+          split_to_tmem(lane_addr, col, cv);
+        }
+        snap32(dm, dir, sl, snap_row, col, v);
+      }
+      if (more) {
+        mbar_arrive_warp(bar(B_CEMPTY + half));
+        tmem_wait_st();
+      }
+      tc_fence_before();  // TMEM reads and writes done before the next product
+      if (more) arrive_cluster_warp(lbar(B_SREADY));
+      st = st_next;
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) tmem_free2(tmem, s256::kTmem);
+}
+
 }  // namespace
 
 bool scan_tc_supported(const Dims& d) {
@@ -430,6 +754,27 @@ cudaError_t launch_scan_tc(const Dims& d, const Inputs& in, const Work& w, cudaS
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)(2 * d.B * d.H * 2), kThreadsScan, smem, s>>>(d, in, w, mm, mc);  // a CTA pair per chain
+  return cudaGetLastError();
+}
+
+bool scan256_tc_supported(const Dims& d) {
+  if (d.update != 0 || !d.bf16 || d.dk != s256::D || d.dv != s256::D) return false;
+  if ((long long)d.B * d.T * d.H * 2 * s256::D >= (1LL << 31)) return false;  // TMA row coordinates
+  if ((long long)d.B * d.H * 4 > 0x7FFFFFFFLL) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_scan256_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
+  if (!scan256_tc_supported(d) || w.M16 == nullptr) return cudaErrorInvalidValue;
+  CUtensorMap mm, mc;
+  const long long fh = (long long)d.B * d.T * d.H;
+  if (!make_matrix_map(&mm, w.M16, fh * 2 * s256::D, s256::D, s256::R) ||
+      !make_matrix_map_f32(&mc, w.Cm, fh * s256::D, s256::D, s256::R))
+    return cudaErrorInvalidValue;
+  const size_t smem = s256::smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(k_scan256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k_scan256_tc<<<(unsigned)(2 * d.B * d.H * 2), s256::kThreads, smem, s>>>(d, in, w, mm, mc);  // a CTA pair per chain
   return cudaGetLastError();
 }
 
