@@ -14,16 +14,22 @@
 // so o = Q R_hi^T + Q R_lo^T carries R to about 16 significant bits (a single
 // bf16 R loses too much: o can be small next to |R| |q|, and the RMSNorm then
 // scales the rounding up).  k_read_tc then runs, per CTA, a run of up to kTilesPerCta
-// tiles of 128 query tokens of one (batch, head, query group):
-//   warp 0      TMA producer: R once (resident), then Q and gate tiles into a
-//               two-stage ring.
+// tiles of 128 query tokens of one (batch, head, query group); runs are
+// launched with the heads varying fastest:
+//   warp 0      TMA producer: R once (resident), then Q tiles into a
+//               three-stage ring that the products alone release.
+//   warp 3      TMA producer of the gate tiles (two-stage ring).
 //   warp 1      TMEM allocator; lane 0 issues O_t = Q_t R_hi^T + Q_t R_lo^T
 //               (M=128 tokens, N=d_v, K=d_k, both operands K-major in SMEM)
 //               into one of two TMEM accumulators.
 //   warps 4..11 epilogue, one token per thread (= TMEM lane) and half of d_v
 //               per warp (warps w and w + 4 share the TMEM lanes of one
 //               32-token quarter): sum of squares over all of d_v, rsqrt,
-//               gate from the SMEM tile, one 32-byte store per 8 outputs.
+//               gate from the SMEM tile.  bf16 y with both branch slots: a
+//               full tile's outputs overwrite its gates in shared memory (same
+//               swizzled layout) and
+//   warp 2      stores them with TMA, then returns the gate stage; other
+//               tiles and outputs go out as one 32-byte store per 8 outputs.
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -38,8 +44,10 @@ namespace {
 using namespace tc;
 
 constexpr int TQ = 128;          // tokens per tile
-constexpr int kTilesPerCta = 8;  // tiles of one query group handled by a CTA
+constexpr int kTilesPerCta = 32; // tiles of one query group handled by a CTA (amortises its R load)
 constexpr int kThreadsR = 384;
+constexpr int kQStages = 3;      // Q ring of k_read_tc (the gate ring has two)
+constexpr int kReadBars = 1 + 2 * kQStages + 2 * 2 + 2 * 2 + 2 + 1;
 
 // ------------------------------------------------------------ read table --
 __global__ void k_read_table(Dims dm, Work w, __nv_bfloat16* __restrict__ r16) {
@@ -96,9 +104,12 @@ __device__ bool decode_run(const Dims& d, long long item, Run& r) {
     if (f1 > f0) per_bh += runs_of_rows((long long)(f1 - f0) * d.N);
   }
   if (per_bh == 0) return false;
-  const long long bh = item / per_bh;
-  if (bh >= (long long)d.B * d.H) return false;
-  long long rem = item % per_bh;
+  // heads vary fastest: CTAs running at the same time read the same token rows
+  // (every head's q and gate of a token are one contiguous row)
+  const long long nbh = (long long)d.B * d.H;
+  const long long bh = item % nbh;
+  long long rem = item / nbh;
+  if (rem >= per_bh) return false;
   for (int g = 0; g < ngroups; ++g) {
     int f0, f1, ri;
     group_of(d, g, f0, f1, ri);
@@ -160,24 +171,38 @@ __device__ __forceinline__ float sigmoid_fast(float g) {
 }
 
 // ------------------------------------------------------------------ kernel --
+// TMA store of a tile from shared memory (bulk group of the issuing thread)
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+// TY: y is bf16 with the two branch slots side by side (out_mode 0): full
+// tiles go out through the gate tile's shared memory and TMA stores (tmy),
+// partial tiles (and every other y) through per-thread stores.
 template <int D, typename To>
 __global__ void __launch_bounds__(kThreadsR, 1)
 k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
-          const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmr) {
+          const __grid_constant__ CUtensorMap tmg, const __grid_constant__ CUtensorMap tmr,
+          const __grid_constant__ CUtensorMap tmy) {
   constexpr int NB = D / 64;
   constexpr uint32_t RBYTES = 2 * D * D * 2;  // hi and lo terms
   constexpr uint32_t TBYTES = TQ * D * 2;  // one Q or gate tile
-  constexpr int ST = 2;
+  constexpr int QS = kQStages, GS = 2;
   constexpr uint32_t kCols = 2 * D <= 128 ? 128 : 256;
   constexpr int HD = D / 2;  // columns per epilogue warp
-  enum { B_R = 0, B_QFULL = 1, B_QEMPTY = 3, B_GFULL = 5, B_GEMPTY = 7, B_AFULL = 9, B_AEMPTY = 11, B_DRAIN = 13,
-         NBARS = 14 };
+  enum { B_R = 0, B_QFULL = 1, B_QEMPTY = B_QFULL + QS, B_GFULL = B_QEMPTY + QS, B_GEMPTY = B_GFULL + GS,
+         B_AFULL = B_GEMPTY + GS, B_AEMPTY = B_AFULL + 2, B_YREADY = B_AEMPTY + 2, B_DRAIN = B_YREADY + GS,
+         NBARS = B_DRAIN + 1 };
+  static_assert(NBARS == kReadBars, "barrier count");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sR = sm;
   unsigned char* sQ = sR + RBYTES;
-  unsigned char* sG = sQ + ST * TBYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + ST * TBYTES);
+  unsigned char* sG = sQ + QS * TBYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sG + GS * TBYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sW = reinterpret_cast<float*>(tmem_slot + 4);  // [D] RMSNorm weight (ones if none)
@@ -187,14 +212,20 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
   Run run;
   if (!decode_run(dm, blockIdx.x, run)) return;
   const Ctl ctl{abort_flag, w.status, (unsigned)TAG_READ_TC};
-  // the epilogue warps' waits: the settable limit (the producer and the MMA
-  // issuer keep the default, and drain what they issued whatever happens)
+  // the epilogue warps' waits: the settable limit (the producers, the MMA
+  // issuer and the store issuer keep the default, and drain what they issued
+  // whatever happens)
   const Ctl ectl{abort_flag, w.status, (unsigned)TAG_READ_TC, g_read_epilogue_limit};
   auto bar = [&](int i) { return smem_u32(bars + i); };
+  constexpr bool TY = sizeof(To) == 2;
+  const bool ty = TY && dm.out_mode == 0;
+  auto full_tile = [&](int t) { return run.rows_left - t * TQ >= TQ; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), (i == B_GEMPTY || i == B_GEMPTY + 1 || i == B_AEMPTY ||
-                                                     i == B_AEMPTY + 1) ? 8 : 1);  // one arrival per epilogue warp
+    for (int i = 0; i < NBARS; ++i)
+      mbar_init(bar(i), (i == B_AEMPTY || i == B_AEMPTY + 1 || i == B_YREADY || i == B_YREADY + 1)
+                            ? 8    // one arrival per epilogue warp
+                            : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -207,34 +238,61 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // R once, then the Q ring (released by the products alone, so the
+    // products run up to QS tiles ahead of the epilogue)
     if (lane == 0) {
       const int rrow = ((run.b * dm.H + run.h) * (dm.C + 1) + run.ridx) * 2 * D;
       mbar_expect_tx(bar(B_R), RBYTES);
       for (int part = 0; part < 2; ++part)
         for (int c = 0; c < NB; ++c)
           tma_load_2d(smem_u32(sR + part * D * D * 2 + c * D * 128), &tmr, bar(B_R), c * 64, rrow + part * D);
-      int last[ST] = {-1, -1};
+      int last[QS];
+      for (int s = 0; s < QS; ++s) last[s] = -1;
       for (int t = 0; t < run.ntiles; ++t) {
-        const int s = t % ST;
+        const int s = t % QS;
         const int tok = (int)(run.tok0 + (long long)t * TQ);
-        if (t >= ST) {
-          if (!mbar_wait(bar(B_QEMPTY + s), (t / ST - 1) & 1, ctl)) break;
-          if (!mbar_wait(bar(B_GEMPTY + s), (t / ST - 1) & 1, ctl)) break;
-        }
+        if (t >= QS && !mbar_wait(bar(B_QEMPTY + s), (t / QS - 1) & 1, ctl)) break;
         mbar_expect_tx(bar(B_QFULL + s), TBYTES);
         for (int c = 0; c < NB; ++c)
           tma_load_3d(smem_u32(sQ + s * TBYTES + c * TQ * 128), &tmq, bar(B_QFULL + s), c * 64, run.h, tok);
+        last[s] = t;
+      }
+      mbar_drain(bar(B_R), 0);
+      for (int s = 0; s < QS; ++s)
+        if (last[s] >= 0) mbar_drain(bar(B_QFULL + s), (last[s] / QS) & 1);
+    }
+  } else if (warp == 3) {
+    // the gate ring (released once a tile's outputs have left its stage)
+    if (lane == 0) {
+      int last[GS] = {-1, -1};
+      for (int t = 0; t < run.ntiles; ++t) {
+        const int s = t % GS;
+        const int tok = (int)(run.tok0 + (long long)t * TQ);
+        if (t >= GS && !mbar_wait(bar(B_GEMPTY + s), (t / GS - 1) & 1, ctl)) break;
         mbar_expect_tx(bar(B_GFULL + s), TBYTES);
         for (int c = 0; c < NB; ++c)
           tma_load_3d(smem_u32(sG + s * TBYTES + c * TQ * 128), &tmg, bar(B_GFULL + s), c * 64, run.h, tok);
         last[s] = t;
       }
-      mbar_drain(bar(B_R), 0);
-      for (int s = 0; s < ST; ++s)
-        if (last[s] >= 0) {
-          mbar_drain(bar(B_QFULL + s), (last[s] / ST) & 1);
-          mbar_drain(bar(B_GFULL + s), (last[s] / ST) & 1);
+      for (int s = 0; s < GS; ++s)
+        if (last[s] >= 0) mbar_drain(bar(B_GFULL + s), (last[s] / GS) & 1);
+    }
+  } else if (warp == 2) {
+    // stores of full bf16 tiles from the gate stage the epilogue overwrote,
+    // then the stage goes back to the gate producer
+    if (lane == 0) {
+      for (int t = 0; t < run.ntiles; ++t) {
+        const int s = t % GS;
+        if (!mbar_wait(bar(B_YREADY + s), (t / GS) & 1, ctl)) break;
+        if (ty && full_tile(t)) {
+          const int tok = (int)(run.tok0 + (long long)t * TQ);
+          for (int c = 0; c < NB; ++c) tma_store_3d(&tmy, smem_u32(sG + s * TBYTES + c * TQ * 128), D + c * 64, run.h, tok);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
+        mbar_arrive(bar(B_GEMPTY + s));
+      }
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -242,19 +300,19 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
       const uint64_t rdesc = sdesc(smem_u32(sR), 16, 1024), qdesc0 = sdesc(smem_u32(sQ), 16, 1024);
       bool ok = mbar_wait(bar(B_R), 0, ctl);
       for (int t = 0; ok && t < run.ntiles; ++t) {
-        const int s = t % ST;
-        if (!mbar_wait(bar(B_QFULL + s), (t / ST) & 1, ctl)) break;
-        if (t >= ST && !mbar_wait(bar(B_AEMPTY + s), (t / ST - 1) & 1, ctl)) break;
+        const int s = t % QS, a = t & 1;
+        if (!mbar_wait(bar(B_QFULL + s), (t / QS) & 1, ctl)) break;
+        if (t >= 2 && !mbar_wait(bar(B_AEMPTY + a), (t / 2 - 1) & 1, ctl)) break;
         tc_fence_after();
         const uint64_t qd = dadd(qdesc0, s * TBYTES);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            mma_bf16(tmem + s * D, dadd(qd, (k >> 2) * (TQ * 128) + (k & 3) * 32),
+            mma_bf16(tmem + a * D, dadd(qd, (k >> 2) * (TQ * 128) + (k & 3) * 32),
                      dadd(rdesc, part * D * D * 2 + (k >> 2) * (D * 128) + (k & 3) * 32), ID, (part | k) ? 1u : 0u);
         }
-        mma_commit(bar(B_AFULL + s));
+        mma_commit(bar(B_AFULL + a));
         mma_commit(bar(B_QEMPTY + s));
       }
       mma_commit(bar(B_DRAIN));
@@ -266,9 +324,9 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const bool add = dm.out_mode != 0;
     for (int t = 0; t < run.ntiles; ++t) {
-      const int s = t % ST;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + s), (t / ST) & 1, ectl))) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_GFULL + s), (t / ST) & 1, ectl))) break;
+      const int s = t % GS, a = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_AFULL + a), (t / 2) & 1, ectl))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_GFULL + s), (t / GS) & 1, ectl))) break;
       tc_fence_after();
       // own half of the row into o, the other half only for the sum of squares
       float o[HD];
@@ -276,33 +334,34 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
 #pragma unroll
       for (int u = 0; u < 8; ++u) ss[u] = 0.f;
 #pragma unroll
-      for (int q = 0; q < HD / 32; ++q) tmem_ld32(lane_addr + s * D + half * HD + q * 32, *reinterpret_cast<float(*)[32]>(o + q * 32));
+      for (int q = 0; q < HD / 32; ++q) tmem_ld32(lane_addr + a * D + half * HD + q * 32, *reinterpret_cast<float(*)[32]>(o + q * 32));
 #pragma unroll
       for (int q = 0; q < HD / 32; ++q) {
         float v[32];
-        tmem_ld32(lane_addr + s * D + (1 - half) * HD + q * 32, v);
+        tmem_ld32(lane_addr + a * D + (1 - half) * HD + q * 32, v);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) ss[i & 7] = fmaf(v[i], v[i], ss[i & 7]);
       }
       tc_fence_before();
-      mbar_arrive_warp(bar(B_AEMPTY + s));  // accumulator free for tile t + ST
+      mbar_arrive_warp(bar(B_AEMPTY + a));  // accumulator free for tile t + 2
 #pragma unroll
       for (int i = 0; i < HD; ++i) ss[i & 7] = fmaf(o[i], o[i], ss[i & 7]);
       const float rs =
           rsqrtf((((ss[0] + ss[1]) + (ss[2] + ss[3])) + ((ss[4] + ss[5]) + (ss[6] + ss[7]))) / D + dm.eps);
       const int rows_valid = min(TQ, run.rows_left - t * TQ);
       const bool valid = row < rows_valid;
+      const bool via_smem = ty && rows_valid == TQ;  // uniform over the CTA
       const long long tok = run.tok0 + (long long)t * TQ + row;
       const long long gi = (tok * dm.H + run.h) * D;
       To* y = static_cast<To*>(in.y) + (dm.out_mode == 0 ? 2 * gi + D : gi) + half * HD;
-      const unsigned char* grow = sG + s * TBYTES + row * 128;
+      unsigned char* grow = sG + s * TBYTES + row * 128;
 #pragma unroll
       for (int ch = 0; ch < HD / 8; ++ch) {
         const int col0 = half * HD + ch * 8;
         // 8 gate values of this row from the 128B-swizzled tile (64 columns per slab)
-        const uint4 raw =
-            *reinterpret_cast<const uint4*>(grow + (col0 >> 6) * (TQ * 128) + ((((col0 & 63) >> 3) ^ (row & 7)) << 4));
+        uint4* gp = reinterpret_cast<uint4*>(grow + (col0 >> 6) * (TQ * 128) + ((((col0 & 63) >> 3) ^ (row & 7)) << 4));
+        const uint4 raw = *gp;
         const float4 w0 = *reinterpret_cast<const float4*>(sW + col0);
         const float4 w1 = *reinterpret_cast<const float4*>(sW + col0 + 4);
         const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
@@ -314,9 +373,16 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
           yv[2 * e] = o[ch * 8 + 2 * e] * rs * wv[2 * e] * sigmoid_fast(g0);
           yv[2 * e + 1] = o[ch * 8 + 2 * e + 1] * rs * wv[2 * e + 1] * sigmoid_fast(g1);
         }
-        if (valid) put8<To>(y + ch * 8, yv, add);
+        if (via_smem) {
+          // the outputs take the place of the gates they used (same layout as y's tile)
+          *gp = make_uint4(pack_bf16(yv[0], yv[1]), pack_bf16(yv[2], yv[3]), pack_bf16(yv[4], yv[5]),
+                           pack_bf16(yv[6], yv[7]));
+        } else if (valid) {
+          put8<To>(y + ch * 8, yv, add);
+        }
       }
-      mbar_arrive_warp(bar(B_GEMPTY + s));  // gate tile free
+      fence_proxy_async_smem();  // the outputs visible to the TMA store
+      mbar_arrive_warp(bar(B_YREADY + s));
     }
   }
 
@@ -515,18 +581,25 @@ cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, __nv_bfloat16
   k_read_table<<<dim3(d.C + 1, d.B * d.H), 256, 0, s>>>(d, w, r16);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap mq, mg, mr;
+  CUtensorMap mq, mg, mr, my;
   const long long tokens = (long long)d.B * d.T * d.N;
   if (!make_token_map(&mq, in.q, tokens, d.H, D, TQ) || !make_token_map(&mg, in.gate_lin, tokens, d.H, D, TQ) ||
       !make_matrix_map(&mr, r16, (long long)d.B * d.H * (d.C + 1) * 2 * D, D, D))
     return cudaErrorInvalidValue;
-  const size_t smem = 1024 + 2 * (size_t)D * D * 2 + 4 * (size_t)TQ * D * 2 + 14 * 8 + 16 + D * 4;
+  // bf16 y with both slots: the store map over [tokens, H, 2 D] (slot 1 = columns D..2D-1);
+  // otherwise unused (a copy of the gate map keeps the argument valid)
+  if (sizeof(To) == 2 && d.out_mode == 0) {
+    if (!make_token_map(&my, in.y, tokens, d.H, 2 * D, TQ)) return cudaErrorInvalidValue;
+  } else {
+    my = mg;
+  }
+  const size_t smem = 1024 + 2 * (size_t)D * D * 2 + (kQStages + 2) * (size_t)TQ * D * 2 + kReadBars * 8 + 16 + D * 4;
   auto kern = k_read_tc<D, To>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long items = num_runs(d);
   if (items <= 0 || items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  kern<<<(unsigned)items, kThreadsR, smem, s>>>(d, in, w, mq, mg, mr);
+  kern<<<(unsigned)items, kThreadsR, smem, s>>>(d, in, w, mq, mg, mr, my);
   return cudaGetLastError();
 }
 
