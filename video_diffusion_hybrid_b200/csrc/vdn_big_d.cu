@@ -129,7 +129,7 @@ __device__ __forceinline__ void add_identity(float (&g)[8][8]) {
 // block form of the sweep:
 //   X = G11^-1,  W = X G12,  Y = (G22 - G12^T W)^-1 (inverse of the Schur
 //   complement),  M22 = Y,  M12 = -W Y,  M21 = M12^T,  M11 = X - M12 W^T,
-// the two block inverses by the register sweep.  Then C = B M by blocks.
+// the two block inverses by the register sweep (panels of 8 pivots).  Then C = B M by blocks.
 // One CTA per frame-head; A_t (from the Gram) is overwritten by M_t in place,
 // each block only after it has been read.  TEXT: A_x, B_x of the text; writes
 // S_x / 2 = B_x M_x / 2 to the half-text state (the A_x slot is scratch).
@@ -140,7 +140,7 @@ k_solve_block(Dims dm, Work w) {
   float* T0 = smb;              // [128][PB] each
   float* T1 = T0 + TB * PB;
   float* T2 = T1 + TB * PB;
-  float* rowbuf = T2 + TB * PB;  // 4 (128 + 4) floats for the sweep
+  float* rowbuf = T2 + TB * PB;  // the panel sweep's rows, Z and V
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   if (!TEXT && is_anchor(dm, t)) return;
   const long long DD = (long long)DB * DB;
@@ -155,7 +155,7 @@ k_solve_block(Dims dm, Work w) {
   // X = G11^-1: kept in T0 and (as scratch until M11 replaces it) in M's block (0, 0)
   tile_ld(g, blk(gM, 0, 0), DB);
   add_identity(g);
-  sweep_regs<TB>(g, rowbuf);  // g = -X
+  sweep_panels<TB>(g, rowbuf);  // g = -X
   tile_st(T0, PB, g, -1.f);
   tile_st(blk(gM, 0, 0), DB, g, -1.f);
   tile_ld(acc, blk(gM, 0, 1), DB);  // G12
@@ -170,7 +170,7 @@ k_solve_block(Dims dm, Work w) {
   tile_ld(g, blk(gM, 1, 1), DB);
   add_identity(g);
   mm128<true, false, true>(g, T1, T2);
-  sweep_regs<TB>(g, rowbuf);  // g = -Y
+  sweep_panels<TB>(g, rowbuf);  // g = -Y
   __syncthreads();            // every read of T1 (G12) done
   tile_st(T1, PB, g, -1.f);
   tile_st(blk(gM, 1, 1), DB, g, -1.f);  // M22
@@ -538,7 +538,7 @@ bool big_d(const Dims& d) { return d.dk == DB && d.dv == DB; }
 
 cudaError_t launch_solve_big(const Dims& d, const Work& w, cudaStream_t s, bool text) {
   if (!big_d(d)) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(float) * (size_t)(3 * TB * PB + 4 * (TB + 4));
+  const size_t smem = sizeof(float) * (size_t)(3 * TB * PB + sweep_panel_floats<TB>());
   auto kern = text ? k_solve_block<true> : k_solve_block<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
