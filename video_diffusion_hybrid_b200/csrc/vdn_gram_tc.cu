@@ -23,15 +23,7 @@
 //               with both operands MN-major (d contiguous), so no repacking.
 //               For d = 64, K and V stack into one M = 128 operand and one
 //               accumulator [A; B] (64 columns).
-// d = 256 (block mode): A_t and B_t are 2 x 2 blocks of 128 x 128, and every
-// block is the second product of a CTA of the d = 128 form run on 128-column
-// views: with X = K[:, 128x : 128x + 128] for beta K and Y a 128-column view
-// of K or V, the CTA forms X^T (beta X) = A(x, x) and Y^T (beta X), which is
-// the block (y, x) of A (Y from K) or of B (Y from V).  Six CTAs per frame-head
-// cover the eight blocks: (x, Y) = (0, V0): A00 B00; (0, V1): B10; (1, V0):
-// A11 B01; (1, V1): B11; (0, K1): A10; (1, K0): A01.  The four CTAs that do
-// not write X^T (beta X) skip that product (16 MMAs per 16 tokens and
-// frame-head instead of 24), and the six are adjacent in the grid.
+// d = 256 runs as a CTA pair per frame-head (vdn_gram256_tc.cu).
 #include "tc_common.cuh"
 
 namespace vdn {
@@ -49,9 +41,8 @@ __device__ __forceinline__ void st_v8(float* p, const float* v) {
 }
 
 // TEXT: the L text tokens of (b, h) instead of one frame; A_x, B_x go to the
-// text_gram region of the workspace.  BLK: the d = 256 block mode above (D is
-// then the 128-column view width).
-template <int D, bool TEXT, bool BLK>
+// text_gram region of the workspace.
+template <int D, bool TEXT>
 __global__ void __launch_bounds__(kThreadsG, 2)
 k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
           const __grid_constant__ CUtensorMap tmv) {
@@ -70,16 +61,12 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  constexpr int DF = BLK ? 2 * D : D;  // row length of k, v and of A_t, B_t
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // block mode: the six CTAs of a frame-head are adjacent in launch order, so
   // five of them find the frame's k and v in L2
-  const int t = BLK ? blockIdx.x / 6 : blockIdx.x, b = blockIdx.z;
-  const int h = blockIdx.y, call = BLK ? blockIdx.x % 6 : 0;
+  const int t = blockIdx.x, b = blockIdx.z;
+  const int h = blockIdx.y;
   // block mode: view columns of X (beta K) and of Y, and where Y^T (beta X) goes
-  const int bx = (call == 2 || call == 3 || call == 5) ? 1 : 0;
-  const int by = (call == 1 || call == 3 || call == 4) ? 1 : 0;
-  const bool y_from_v = call < 4, write_a = call == 0 || call == 2;
   if (!TEXT && is_anchor(dm, t)) return;
   if (*reinterpret_cast<volatile uint32_t*>(w.status) != 0u) return;
   const int ntok = TEXT ? dm.L : dm.N;
@@ -87,7 +74,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
   // first token of the frame (or of batch b's text)
   const long long tok0 = TEXT ? (long long)b * dm.L : ((long long)b * dm.T + t) * dm.N;
   const float* betap = TEXT ? in.text_beta : in.beta;
-  const long long DDg = (long long)DF * DF;
+  const long long DDg = (long long)D * D;
   float* outA = TEXT ? w.text_gram + ((long long)b * dm.H + h) * 2 * DDg
                      : w.M + (((long long)b * dm.T + t) * dm.H + h) * DDg;
   float* outB = TEXT ? outA + DDg : w.Cm + (((long long)b * dm.T + t) * dm.H + h) * DDg;
@@ -114,9 +101,8 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
         const int tok = (int)(tok0 + (long long)j * TT);
         mbar_expect_tx(bar(B_KVFULL + s), STAGE);
         for (int c = 0; c < NB; ++c) {
-          tma_load_3d(smem_u32(sKV + s * STAGE + c * TT * 128), &tmk, bar(B_KVFULL + s), c * 64 + bx * D, h, tok);
-          tma_load_3d(smem_u32(sKV + s * STAGE + TB + c * TT * 128), (!BLK || y_from_v) ? &tmv : &tmk,
-                      bar(B_KVFULL + s), c * 64 + by * D, h, tok);
+          tma_load_3d(smem_u32(sKV + s * STAGE + c * TT * 128), &tmk, bar(B_KVFULL + s), c * 64, h, tok);
+          tma_load_3d(smem_u32(sKV + s * STAGE + TB + c * TT * 128), &tmv, bar(B_KVFULL + s), c * 64, h, tok);
         }
         last[s] = j;
       }
@@ -131,7 +117,6 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       const uint64_t hidesc = sdesc(smem_u32(sHi), TT * 128, 1024), lodesc = sdesc(smem_u32(sLo), TT * 128, 1024);
       const uint64_t kvdesc0 = sdesc(smem_u32(sKV), TT * 128, 1024);
       // block mode: X^T (beta X) only where the CTA writes it
-      const bool first = !BLK || write_a;
       bool ok = true;
       for (int j = 0; ok && j < ntiles; ++j) {
         const int s = j % ST;
@@ -147,7 +132,7 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
 #pragma unroll
           for (int k = 0; k < TT / 16; ++k) {
             const uint32_t acc = (j | part | k) ? 1u : 0u;
-            if (first) mma_bf16(tmem, dadd(kd, k * 2048), dadd(bd, k * 2048), ID, acc);
+            mma_bf16(tmem, dadd(kd, k * 2048), dadd(bd, k * 2048), ID, acc);
             if (D == 128) mma_bf16(tmem + 128, dadd(vd, k * 2048), dadd(bd, k * 2048), ID, acc);
           }
         }
@@ -204,14 +189,11 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
       tc_fence_after();
       const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
       if (D == 128) {
-        // rows of X^T (beta X) and Y^T (beta X); in block mode placed as the
-        // blocks (bx, bx) and (by, bx) of the d = 256 matrices
-        float* Ag = outA + (long long)(bx * D + row) * DF + bx * D;
-        float* Bg = (!BLK || y_from_v ? outB : outA) + (long long)(by * D + row) * DF + bx * D;
-        const bool wa = !BLK || write_a;
+        // rows of K^T (beta K) and V^T (beta K)
+        float* Ag = outA + (long long)row * D;
+        float* Bg = outB + (long long)row * D;
 #pragma unroll
         for (int q = 0; q < 2 * D / 32; ++q) {
-          if (q < D / 32 && !wa) continue;
           float v[32];
           tmem_ld32(lane_addr + q * 32, v);
           tmem_wait_ld();
@@ -241,19 +223,18 @@ k_gram_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk,
   if (warp == 1) tmem_free(tmem, kCols);
 }
 
-template <int D, bool TEXT, bool BLK = false>
+template <int D, bool TEXT>
 cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
-  constexpr int DF = BLK ? 2 * D : D;
   CUtensorMap mk, mv;
   const long long tokens = TEXT ? (long long)d.B * d.L : (long long)d.B * d.T * d.N;
-  if (!make_token_map(&mk, TEXT ? in.text_k : in.k, tokens, d.H, DF, TT) ||
-      !make_token_map(&mv, TEXT ? in.text_v : in.v, tokens, d.H, DF, TT))
+  if (!make_token_map(&mk, TEXT ? in.text_k : in.k, tokens, d.H, D, TT) ||
+      !make_token_map(&mv, TEXT ? in.text_v : in.v, tokens, d.H, D, TT))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 2 * (2 * (size_t)TT * D * 2) + 2 * (size_t)TT * D * 2 + 8 * 8 + 16;
-  auto kern = k_gram_tc<D, TEXT, BLK>;
+  auto kern = k_gram_tc<D, TEXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3((TEXT ? 1 : d.T) * (BLK ? 6 : 1), d.H, d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
+  kern<<<dim3(TEXT ? 1 : d.T, d.H, d.B), kThreadsG, smem, s>>>(d, in, w, mk, mv);
   return cudaGetLastError();
 }
 
@@ -262,12 +243,12 @@ cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t 
 bool gram_tc_supported(const Dims& d) {
   if (!d.bf16 || d.dk != d.dv || (d.dk != 64 && d.dk != 128 && d.dk != 256)) return false;
   if ((long long)d.B * d.T * d.N >= (1LL << 31)) return false;
-  if ((long long)d.T * 6 > 0x7FFFFFFFLL) return false;
+  if (2LL * d.B * d.H * d.T > 0x7FFFFFFFLL) return false;  // the d = 256 pair grid
   return encode_fn() != nullptr;
 }
 
 cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
-  if (d.dk == 256) return launch<128, false, true>(d, in, w, s);
+  if (d.dk == 256) return launch_gram256_tc(d, in, w, s, false);
   if (d.dk == 128) return launch<128, false>(d, in, w, s);
   if (d.dk == 64) return launch<64, false>(d, in, w, s);
   return cudaErrorInvalidValue;
@@ -275,7 +256,7 @@ cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaS
 
 cudaError_t launch_text_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s) {
   if (d.L <= 0 || (long long)d.B * d.L >= (1LL << 31)) return cudaErrorInvalidValue;
-  if (d.dk == 256) return launch<128, true, true>(d, in, w, s);
+  if (d.dk == 256) return launch_gram256_tc(d, in, w, s, true);
   if (d.dk == 128) return launch<128, true>(d, in, w, s);
   if (d.dk == 64) return launch<64, true>(d, in, w, s);
   return cudaErrorInvalidValue;

@@ -72,6 +72,8 @@ cudaError_t launch_text_solve_sweep(const Dims& d, const Work& w, cudaStream_t s
 cudaError_t launch_text_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 bool gram_tc_supported(const Dims& d);
 cudaError_t launch_gram_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
+// d = 256: a CTA pair per frame-head (text = true: per batch-head, over the text tokens)
+cudaError_t launch_gram256_tc(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s, bool text);
 cudaError_t launch_scan_simt(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
 // the ablation variants' per-frame maps (M'_t, C'_t) into the M_t, C_t slots
 cudaError_t launch_variant_maps(const Dims& d, const Inputs& in, const Work& w, cudaStream_t s);
