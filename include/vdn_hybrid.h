@@ -33,7 +33,11 @@
  *     current CUDA device, all struct pointers are HOST pointers read during the
  *     call only.
  *   - Asynchrony: work is enqueued on `stream` (NULL = legacy default stream)
- *     and the call returns without synchronising.
+ *     and the call returns without synchronising.  A forward call that runs the
+ *     text and frame-write stages together on a large problem (B*T*H >= 1024,
+ *     text tokens present, `stream` not capturing) runs the text stage on a
+ *     stream it creates for that call, which first waits for `stream` and which
+ *     `stream` waits for before the scans: the work stays ordered on `stream`.
  *   - Errors: arguments are validated before any launch; a status other than
  *     VDN_OK from validation means nothing was enqueued.  A launch failure is
  *     VDN_ERR_CUDA (the CUDA error is left for cudaGetLastError).
@@ -228,10 +232,19 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg *cfg, const vdn_hybri
  * Sharing: every call uses the same array, which keeps the last call's
  * contents (each call clears what must start at zero); calls whose work
  * overlaps on the GPU race on it and must be serialised by the caller.  The
- * device status words of these calls are not readable by the caller. */
+ * device status words of the last call on the current device are read by
+ * vdn_hybrid_noalloc_device_status. */
 #define VDN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 vdn_status vdn_hybrid_attn_fwd_noalloc(const vdn_hybrid_cfg *cfg, const vdn_hybrid_args *args,
                                        vdn_stream_t stream);
+
+/* Device status of the last vdn_hybrid_attn_fwd_noalloc call on the current
+ * device (the first words of the library-owned array): VDN_OK, or
+ * VDN_ERR_TIMEOUT if a bounded wait of one of its kernels gave up (its output
+ * is then incomplete), with the kernel's VDN_TAG_* in *where (if not NULL).
+ * Synchronises `stream` (give the stream of that call); VDN_ERR_CUDA if the
+ * read fails. */
+vdn_status vdn_hybrid_noalloc_device_status(vdn_stream_t stream, unsigned *where);
 
 /* Kernel tags: which kernel's bounded wait gave up (vdn_hybrid_device_status). */
 enum {

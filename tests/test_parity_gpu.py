@@ -186,6 +186,34 @@ def test_d256_vda_matches_oracle(shape):
     assert L.vdn_hybrid_attn_fwd(cfg, ha.args(t), check=False) == L.VDN_ERR_UNSUPPORTED
 
 
+D256_EDGE = {
+    # anchors at both ends: no written frame (the scans only copy the start state)
+    "T2": (Shape(1, 2, 24, 1, 256, 256, 8), {}),
+    # one written frame between the anchors
+    "T3": (Shape(1, 3, 24, 1, 256, 256, 0), {}),
+    # no anchors: every frame written, a ragged last chunk
+    "T7_no_anchors": (Shape(1, 7, 16, 2, 256, 256, 8), {"anchors": 0}),
+    # two batch elements: chains of both in one launch
+    "B2": (Shape(2, 11, 20, 1, 256, 256, 8), {}),
+}
+
+
+@pytest.mark.parametrize("case", sorted(D256_EDGE))
+def test_d256_edge_cases(case):
+    """d = 256 with few or no written frames, no anchors and two batch
+    elements (the tensor-core scan's empty, single-step and multi-chain
+    forms): the read table and the linear slot against the oracle."""
+    shape, kw = D256_EDGE[case]
+    inp, cfg, ha, t, y = run(shape, "bf16", 29, drop_text=shape.L == 0, stages=VDA, **kw)
+    it = {k: v.double().cpu().numpy() for k, v in ha.intermediates().items()}
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            ref = O.vda_intermediates(inp, ocfg(cfg), b, h)
+            np.testing.assert_allclose(it["R"][b, h], ref["R"], atol=2e-4 * np.sqrt(np.mean(ref["R"] ** 2)) + 1e-30)
+    ref_y = O.hybrid_attn(inp, ocfg(cfg))
+    assert rel_err(y[..., 1, :], ref_y[..., 1, :]) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("y_bf16,out_mode", [(False, 1), (True, 0), (True, 1)])
 def test_d256_output_options(y_bf16, out_mode):
     """d = 256 with a caller-given text state, an RMSNorm weight, bf16 y and

@@ -54,6 +54,8 @@ def test_noalloc_matches_regular_entry_point_twice(cuda_ok, name, shape, kw):
         y.fill_(float("nan"))
         L.vdn_hybrid_attn_fwd_noalloc(cfg, _noalloc_args(t, y))
         torch.cuda.synchronize()
+        # the no-alloc call's own status words (every bounded wait completed)
+        assert L.vdn_hybrid_noalloc_device_status() == (L.VDN_OK, 0)
         if not torch.equal(y, ref):
             got, want = y.double().cpu().numpy(), ref.double().cpu().numpy()
             errs = [np.nanmax(np.abs(got[..., s, :] - want[..., s, :])) / np.sqrt(np.mean(want[..., s, :] ** 2))

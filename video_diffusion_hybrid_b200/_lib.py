@@ -23,7 +23,7 @@ STAGE_SOFTMAX_BWD = 32  # vdn_hybrid_stage_impl key of the softmax branch's back
 
 EXPORTED = ("vdn_hybrid_attn_workspace_size", "vdn_hybrid_workspace_layout", "vdn_hybrid_attn_fwd",
             "vdn_hybrid_attn_fwd_stages", "vdn_hybrid_device_status", "vdn_hybrid_stage_impl",
-            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_out_proj", "vdn_text_cross_attn",
+            "vdn_status_string", "vdn_hybrid_attn_fwd_noalloc", "vdn_hybrid_noalloc_device_status", "vdn_out_proj", "vdn_text_cross_attn",
             "vdn_quantize_fp8", "vdn_out_proj_fp8", "vdn_hybrid_lin_bwd_workspace_size", "vdn_hybrid_lin_bwd",
             "vdn_hybrid_sm_bwd_workspace_size", "vdn_hybrid_sm_bwd", "vdn_hybrid_bwd_workspace_size", "vdn_hybrid_bwd",
             "vdn_debug_set_read_wait_limit", "vdn_proj_device_status")
@@ -141,6 +141,8 @@ def lib() -> C.CDLL:
         L.vdn_hybrid_stage_impl.argtypes = [C.POINTER(VdnCfg), C.c_uint]
         L.vdn_hybrid_attn_fwd_noalloc.restype = C.c_int
         L.vdn_hybrid_attn_fwd_noalloc.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
+        L.vdn_hybrid_noalloc_device_status.restype = C.c_int
+        L.vdn_hybrid_noalloc_device_status.argtypes = [C.c_void_p, C.POINTER(C.c_uint)]
         L.vdn_text_cross_attn.restype = C.c_int
         L.vdn_text_cross_attn.argtypes = [C.POINTER(VdnCfg), C.POINTER(VdnArgs), C.c_void_p]
         L.vdn_quantize_fp8.restype = C.c_int
@@ -278,6 +280,14 @@ def vdn_hybrid_attn_fwd_stages(cfg: HybridCfg, args: VdnArgs, stages: int, strea
 def vdn_hybrid_device_status(cfg: HybridCfg, args: VdnArgs, stream=None) -> tuple:
     c, where = cfg.c(), C.c_uint(0)
     st = lib().vdn_hybrid_device_status(C.byref(c), C.byref(args), _stream_handle(stream), C.byref(where))
+    return st, int(where.value)
+
+
+def vdn_hybrid_noalloc_device_status(stream=None) -> tuple:
+    """(status, kernel tag) of the last no-alloc call on the current device
+    (synchronises the stream)."""
+    where = C.c_uint(0)
+    st = lib().vdn_hybrid_noalloc_device_status(_stream_handle(stream), C.byref(where))
     return st, int(where.value)
 
 

@@ -137,6 +137,55 @@ Work work_of(const vdn_hybrid_cfg* c, const vdn_hybrid_args* a) {
   return w;
 }
 
+// The text stage beside the frame write.  With text tokens, the text Gram
+// and solve are a few dozen CTAs that the frame Gram and solve do not depend
+// on (nor the reverse), so when one call runs both they go on a side stream
+// (created for the call, highest priority) that waits for `s` first and that
+// `s` waits for when the guard ends: the stage stays ordered on `s` like any
+// other.  Not under stream capture, and not for problems too small to fill the
+// GPU with the frame write.
+struct TextFork {
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev[2] = {nullptr, nullptr};
+  cudaStream_t main = nullptr;
+  bool forked = false;
+  cudaError_t err = cudaSuccess;
+  bool open(const Dims& d, cudaStream_t s) {
+    if (d.L <= 0 || (long long)d.B * d.T * d.H < 1024) return false;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&side, cudaStreamNonBlocking, hi) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev[1], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventRecord(ev[0], s) != cudaSuccess || cudaStreamWaitEvent(side, ev[0], 0) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return false;  // the destructor releases what was created; nothing was enqueued on the side
+    }
+    main = s;
+    forked = true;
+    return true;
+  }
+  // `s` waits for everything enqueued on the side stream
+  cudaError_t join() {
+    if (!forked) return err;
+    forked = false;
+    if (err == cudaSuccess) err = cudaEventRecord(ev[1], side);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(main, ev[1], 0);
+    return err;
+  }
+  ~TextFork() {
+    join();
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);  // released once complete
+    if (side) cudaStreamDestroy(side);  // likewise
+  }
+};
+
 Inputs inputs_of(const vdn_hybrid_args* a) {
   Inputs in;
   in.q = a->q; in.k = a->k; in.v = a->v; in.beta = a->beta; in.alpha = a->alpha;
@@ -222,12 +271,15 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
   if (big && ((stages & VDN_STAGE_SOFTMAX) || !gram_tc_supported(d))) return VDN_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
   if (cudaMemsetAsync(w.status, 0, 256, s) != cudaSuccess) return VDN_ERR_CUDA;
+  TextFork fork;
   if (stages & VDN_STAGE_TEXT) {
+    cudaStream_t ts = s;
+    if ((stages & VDN_STAGE_SOLVE) && d.update == 0 && gram_tc_supported(d) && fork.open(d, s)) ts = fork.side;
     if (d.L > 0 && gram_tc_supported(d)) {
-      if ((e = launch_text_gram_tc(d, in, w, s)) != cudaSuccess) return VDN_ERR_CUDA;
-      e = big ? launch_solve_big(d, w, s, true) : launch_text_solve_sweep(d, w, s);
+      if ((e = launch_text_gram_tc(d, in, w, ts)) != cudaSuccess) return VDN_ERR_CUDA;
+      e = big ? launch_solve_big(d, w, ts, true) : launch_text_solve_sweep(d, w, ts);
       if (e != cudaSuccess) return VDN_ERR_CUDA;
-    } else if ((e = launch_text(d, in, w, s)) != cudaSuccess) {
+    } else if ((e = launch_text(d, in, w, ts)) != cudaSuccess) {
       return VDN_ERR_CUDA;
     }
   }
@@ -242,6 +294,7 @@ vdn_status vdn_hybrid_attn_fwd_stages(const vdn_hybrid_cfg* cfg, const vdn_hybri
       return VDN_ERR_CUDA;
     }
   }
+  if (fork.join() != cudaSuccess) return VDN_ERR_CUDA;  // the scans start from the text state
   if (big && (stages & VDN_STAGE_SCAN)) {
     e = (scan256_tc_supported(d) && w.M16 != nullptr) ? launch_scan256_tc(d, in, w, s) : launch_scan_big(d, in, w, s);
     if (e != cudaSuccess) return VDN_ERR_CUDA;

@@ -54,3 +54,16 @@ extern "C" vdn_status vdn_hybrid_attn_fwd_noalloc(const vdn_hybrid_cfg* cfg, con
   a.workspace_bytes = kNoallocScratchBytes;
   return vdn_hybrid_attn_fwd(cfg, &a, stream);
 }
+
+extern "C" vdn_status vdn_hybrid_noalloc_device_status(vdn_stream_t stream, unsigned* where) {
+  void* scratch = nullptr;
+  vdn_status st = scratch_for_current_device(&scratch);
+  if (st != VDN_OK) return st;
+  // the status words lead the workspace layout of every configuration
+  uint32_t host[2] = {0, 0};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host, scratch, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (where) *where = host[1];
+  return host[0] ? VDN_ERR_TIMEOUT : VDN_OK;
+}
