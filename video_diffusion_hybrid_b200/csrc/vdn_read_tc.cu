@@ -162,6 +162,41 @@ template <> __device__ __forceinline__ void put8<__nv_bfloat16>(__nv_bfloat16* p
       make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
 }
 
+// y[0..16) (+)= v as whole 32-byte sectors: bf16 rows as one 256-bit store,
+// fp32 rows as two (dst 32-byte aligned).
+template <typename To> __device__ __forceinline__ void put16(To* p, float (&v)[16], bool add);
+template <> __device__ __forceinline__ void put16<float>(float* p, float (&v)[16], bool add) {
+  put8<float>(p, *reinterpret_cast<float(*)[8]>(v), add);
+  put8<float>(p + 8, *reinterpret_cast<float(*)[8]>(v + 8), add);
+}
+template <> __device__ __forceinline__ void put16<__nv_bfloat16>(__nv_bfloat16* p, float (&v)[16], bool add) {
+  if (add) {
+    uint32_t o[8];
+    asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7])
+                 : "l"(p));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      v[2 * e] += __uint_as_float(o[e] << 16);
+      v[2 * e + 1] += __uint_as_float(o[e] & 0xFFFF0000u);
+    }
+  }
+  uint32_t u[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) u[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(u[0]), "r"(u[1]), "r"(u[2]),
+               "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+               : "memory");
+}
+
+// L2 prefetch of a tensor-map box (no shared memory, no barrier)
+__device__ __forceinline__ void prefetch_box_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // sigmoid from the exponential and an approximate reciprocal (both a few ulp;
 // exp(-g) overflowing to inf gives 0, the limit)
 __device__ __forceinline__ float sigmoid_fast(float g) {
@@ -400,13 +435,15 @@ k_read_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
 // M = 128, N = 256, K = 16 accumulate O = Q R_hi^T + Q R_lo^T into one of two
 // 256-column TMEM accumulators.  Epilogue: eight warps, each owning 128 of the
 // 256 columns of its 32 rows; a first pass over all 256 TMEM columns forms the
-// sum of squares, a second pass its own outputs (gates read from global).
+// sum of squares, a second pass its own outputs (gates read from global after
+// the producer prefetched the tile's gate boxes into L2 with its Q tile; y
+// written in whole 32-byte sectors).
 constexpr int D2 = 256;
 
 template <typename To>
 __global__ void __launch_bounds__(kThreadsR, 1)
 k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq,
-             const __grid_constant__ CUtensorMap tmr) {
+             const __grid_constant__ CUtensorMap tmr, const __grid_constant__ CUtensorMap tmg) {
   constexpr uint32_t QCH = TQ * 128;        // one 64-column chunk of the Q tile: 16 KB
   constexpr uint32_t QBYTES = 4 * QCH;      // the Q tile
   constexpr uint32_t RHALF = D2 * 128;      // 64 columns of all 256 rows of R_hi (or R_lo): 32 KB
@@ -445,9 +482,18 @@ k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
     if (lane == 0) {
       const int rrow = ((run.b * dm.H + run.h) * (dm.C + 1) + run.ridx) * 2 * D2;
       int nq = 0, nr = 0;
+      // the gates of a tile go to L2 with its Q tile: the epilogue reads them
+      // with plain loads one product later
+      auto prefetch_gates = [&](int j) {
+        if (j >= run.ntiles) return;
+        const int tok = (int)(run.tok0 + (long long)j * TQ);
+        for (int c = 0; c < 4; ++c) prefetch_box_3d(&tmg, c * 64, run.h, tok);
+      };
+      prefetch_gates(0);
       for (int j = 0; j < run.ntiles; ++j) {
         const int tok = (int)(run.tok0 + (long long)j * TQ);
         if (j > 0 && !mbar_wait(bar(B_QEMPTY), (j - 1) & 1, ctl)) break;
+        prefetch_gates(j + 1);
         mbar_expect_tx(bar(B_QFULL), QBYTES);
         for (int c = 0; c < 4; ++c) tma_load_3d(smem_u32(sQ + c * QCH), &tmq, bar(B_QFULL), c * 64, run.h, tok);
         ++nq;
@@ -530,17 +576,18 @@ k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         tmem_wait_ld();
         if (valid) {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4*>(grow + col0 + ch * 8));
-            const uint32_t gu[4] = {raw.x, raw.y, raw.z, raw.w};
-            float yv[8];
+          for (int ch = 0; ch < 2; ++ch) {
+            const uint4 r0 = __ldg(reinterpret_cast<const uint4*>(grow + col0 + ch * 16));
+            const uint4 r1 = __ldg(reinterpret_cast<const uint4*>(grow + col0 + ch * 16 + 8));
+            const uint32_t gu[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            float yv[16];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i0 = ch * 8 + 2 * e;
+            for (int e = 0; e < 8; ++e) {
+              const int i0 = ch * 16 + 2 * e;
               yv[2 * e] = v[i0] * rs * sW[col0 + i0] * sigmoid_fast(__uint_as_float(gu[e] << 16));
               yv[2 * e + 1] = v[i0 + 1] * rs * sW[col0 + i0 + 1] * sigmoid_fast(__uint_as_float(gu[e] & 0xFFFF0000u));
             }
-            put8<To>(y + col0 + ch * 8, yv, add);
+            put16<To>(y + col0 + ch * 16, yv, add);
           }
         }
       }
@@ -608,9 +655,9 @@ cudaError_t launch256(const Dims& d, const Inputs& in, const Work& w, __nv_bfloa
   k_read_table<<<dim3(d.C + 1, d.B * d.H), 256, 0, s>>>(d, w, r16);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap mq, mr;
+  CUtensorMap mq, mr, mg;
   const long long tokens = (long long)d.B * d.T * d.N;
-  if (!make_token_map(&mq, in.q, tokens, d.H, D2, TQ) ||
+  if (!make_token_map(&mq, in.q, tokens, d.H, D2, TQ) || !make_token_map(&mg, in.gate_lin, tokens, d.H, D2, TQ) ||
       !make_matrix_map(&mr, r16, (long long)d.B * d.H * (d.C + 1) * 2 * D2, D2, D2))
     return cudaErrorInvalidValue;
   const size_t smem = 1024 + 4 * (size_t)TQ * 128 + 2 * 2 * (size_t)D2 * 128 + 11 * 8 + 16 + D2 * 4;
@@ -619,7 +666,7 @@ cudaError_t launch256(const Dims& d, const Inputs& in, const Work& w, __nv_bfloa
   if (e != cudaSuccess) return e;
   const long long items = num_runs(d);
   if (items <= 0 || items > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-  kern<<<(unsigned)items, kThreadsR, smem, s>>>(d, in, w, mq, mr);
+  kern<<<(unsigned)items, kThreadsR, smem, s>>>(d, in, w, mq, mr, mg);
   return cudaGetLastError();
 }
 
