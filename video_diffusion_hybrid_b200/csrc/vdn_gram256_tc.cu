@@ -12,7 +12,8 @@
 // The pair splits the 256 columns of k and v: CTA r streams columns
 // 128 r .. 128 r + 127 of K and V (64-token tiles, two-stage ring) and forms
 // its half of beta K as two bf16 terms (hi = bf16(beta k), lo = bf16(beta k -
-// hi)).  The leader issues, per 16 tokens, the pair products
+// hi)), double-buffered so that scaling and products overlap.  The leader
+// issues, per 16 tokens, the pair products
 //   A += K^T (beta K)_hi + K^T (beta K)_lo,   B += V^T (beta K)_hi + V^T (beta K)_lo
 // with M = 256 (each CTA's half of K^T or V^T: its 128 rows of A or B) and N =
 // 256 (each CTA's half of beta K), both operands MN-major straight from the
@@ -42,7 +43,9 @@ constexpr uint32_t STAGE = 2 * TB;      // K then V
 constexpr int ST = 2;
 constexpr int kThreads = 256;
 constexpr uint32_t kCols = 512;       // A (0..255) and B (256..511)
-enum { B_KVFULL = 0, B_KVEMPTY = 2, B_KBFULL = 4, B_KBEMPTY = 5, B_ACC = 6, B_DRAIN = 7, NBARS = 8 };
+// beta K is double-buffered too (slot j & 1 for tile j), so the scaling of
+// tile j + 1 runs while the pair's products of tile j do
+enum { B_KVFULL = 0, B_KVEMPTY = 2, B_KBFULL = 4, B_KBEMPTY = 6, B_ACC = 8, B_DRAIN = 9, NBARS = 10 };
 
 __device__ __forceinline__ void st_v8(float* p, const float* v) {
   asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
@@ -57,9 +60,8 @@ k_gram256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sKV = sm;                // ST stages of [K half | V half]
-  unsigned char* sHi = sKV + ST * STAGE;  // this CTA's half of beta K, high term
-  unsigned char* sLo = sHi + TB;          // low term
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sLo + TB);
+  unsigned char* sKB = sKV + ST * STAGE;  // 2 slots of this CTA's half of beta K: high term, low term
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKB + 2 * 2 * TB);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -86,7 +88,8 @@ k_gram256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk
   auto lbar = [&](int i) { return map_rank(smem_u32(bars + i), 0); };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), i == B_KBFULL ? 8 : 1);  // KBFULL: 4 warps x 2 CTAs
+    for (int i = 0; i < NBARS; ++i)
+      mbar_init(bar(i), (i == B_KBFULL || i == B_KBFULL + 1) ? 8 : 1);  // KBFULL: 4 warps x 2 CTAs
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -120,13 +123,14 @@ k_gram256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk
       // chunks TT*128 bytes apart, 8-token groups 1024 bytes apart, 16 tokens
       // (2048 bytes) per K-step; M = N = 256 over the pair
       constexpr uint32_t ID = idesc_bf16(2 * HALF, D, true) | (1u << 15);
-      const uint64_t hidesc = sdesc(smem_u32(sHi), TT * 128, 1024), lodesc = sdesc(smem_u32(sLo), TT * 128, 1024);
+      const uint64_t kbdesc0 = sdesc(smem_u32(sKB), TT * 128, 1024);
       const uint64_t kvdesc0 = sdesc(smem_u32(sKV), TT * 128, 1024);
       bool ok = true;
       for (int j = 0; ok && j < ntiles; ++j) {
         const int s = j % ST;
         // both CTAs' tiles landed and their halves of beta K written
-        if (!mbar_wait_cl(bar(B_KBFULL), j & 1, ctl)) {
+        const int kb = j & 1;
+        if (!mbar_wait_cl(bar(B_KBFULL + kb), (j >> 1) & 1, ctl)) {
           ok = false;
           break;
         }
@@ -134,7 +138,7 @@ k_gram256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk
         const uint64_t kd = dadd(kvdesc0, s * STAGE), vd = dadd(kd, TB);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint64_t bd = part ? lodesc : hidesc;
+          const uint64_t bd = dadd(kbdesc0, (2 * kb + part) * TB);
 #pragma unroll
           for (int k = 0; k < TT / 16; ++k) {
             const uint32_t acc = (j | part | k) ? 1u : 0u;
@@ -144,8 +148,8 @@ k_gram256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk
         }
         commit2(bar(B_KVEMPTY + s));
         commit2(map_rank(bar(B_KVEMPTY + s), 1));
-        commit2(bar(B_KBEMPTY));
-        commit2(map_rank(bar(B_KBEMPTY), 1));
+        commit2(bar(B_KBEMPTY + kb));
+        commit2(map_rank(bar(B_KBEMPTY + kb), 1));
       }
       if (ok) {
         commit2(bar(B_ACC));
@@ -171,8 +175,14 @@ k_gram256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk
       const float beta = beta_next;
       if (j + 1 < ntiles) beta_next = beta_of(j + 1);
       if (!__all_sync(0xffffffffu, mbar_wait(bar(B_KVFULL + s), (j / ST) & 1, ctl))) { ok = false; break; }
-      // the scaled copy is single-buffered: the pair's products of tile j - 1 are done with it
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait_cl(bar(B_KBEMPTY), (j - 1) & 1, ctl))) { ok = false; break; }
+      // slot j & 1 of the scaled copy: the pair's products of tile j - 2 are done with it
+      const int kb = j & 1;
+      unsigned char* sHi = sKB + 2 * kb * TB;
+      unsigned char* sLo = sHi + TB;
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_cl(bar(B_KBEMPTY + kb), ((j >> 1) - 1) & 1, ctl))) {
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int uu = 0; uu < NB * 4; ++uu) {
         const int unit = shalf * NB * 4 + uu, c = unit >> 3, q = unit & 7;
@@ -191,7 +201,7 @@ k_gram256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmk
         *reinterpret_cast<uint4*>(sLo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
       }
       fence_proxy_async_smem();
-      arrive_cluster_warp(lbar(B_KBFULL));
+      arrive_cluster_warp(lbar(B_KBFULL + kb));
     }
     // ---- epilogue: this CTA's rows of A_t and B_t (fp32, row-major)
     if (__all_sync(0xffffffffu, ok && mbar_wait_cl(bar(B_ACC), 0, ctl))) {
@@ -225,7 +235,7 @@ cudaError_t launch(const Dims& d, const Inputs& in, const Work& w, cudaStream_t 
       !make_token_map(&mv, TEXT ? in.text_v : in.v, tokens, d.H, D, TT))
     return cudaErrorInvalidValue;
   // one CTA per SM (the 512 TMEM columns; the two CTAs of a pair on two SMs)
-  const size_t need = 1024 + ST * (size_t)STAGE + 2 * (size_t)TB + NBARS * 8 + 16;
+  const size_t need = 1024 + ST * (size_t)STAGE + 4 * (size_t)TB + NBARS * 8 + 16;
   const size_t smem = need < 120 * 1024 ? 120 * 1024 : need;
   auto kern = k_gram256_tc<TEXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
