@@ -189,6 +189,36 @@ template <> __device__ __forceinline__ void put16<__nv_bfloat16>(__nv_bfloat16* 
                : "memory");
 }
 
+// TMA loads with an L2 eviction-priority policy (createpolicy): R's split,
+// re-read by every tile of a run, is kept (evict_last); the streaming Q tiles
+// go first (evict_first)
+__device__ __forceinline__ uint64_t l2_policy_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_load_2d_pol(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                                uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+      "%4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pol(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                                int z, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+      "%4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "l"(pol)
+      : "memory");
+}
+
 // L2 prefetch of a tensor-map box (no shared memory, no barrier)
 __device__ __forceinline__ void prefetch_box_3d(const CUtensorMap* map, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
@@ -481,6 +511,7 @@ k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
   if (warp == 0) {
     if (lane == 0) {
       const int rrow = ((run.b * dm.H + run.h) * (dm.C + 1) + run.ridx) * 2 * D2;
+      const uint64_t pol_last = l2_policy_last(), pol_first = l2_policy_first();
       int nq = 0, nr = 0;
       // the gates of a tile go to L2 with its Q tile: the epilogue reads them
       // with plain loads one product later
@@ -495,15 +526,16 @@ k_read256_tc(Dims dm, Inputs in, Work w, const __grid_constant__ CUtensorMap tmq
         if (j > 0 && !mbar_wait(bar(B_QEMPTY), (j - 1) & 1, ctl)) break;
         prefetch_gates(j + 1);
         mbar_expect_tx(bar(B_QFULL), QBYTES);
-        for (int c = 0; c < 4; ++c) tma_load_3d(smem_u32(sQ + c * QCH), &tmq, bar(B_QFULL), c * 64, run.h, tok);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d_pol(smem_u32(sQ + c * QCH), &tmq, bar(B_QFULL), c * 64, run.h, tok, pol_first);
         ++nq;
         bool ok = true;
         for (int kc = 0; kc < 4; ++kc) {
           const int u = j * 4 + kc, s = u & 1;
           if (u >= 2 && !mbar_wait(bar(B_REMPTY + s), ((u >> 1) - 1) & 1, ctl)) { ok = false; break; }
           mbar_expect_tx(bar(B_RFULL + s), RST);
-          tma_load_2d(smem_u32(sR + s * RST), &tmr, bar(B_RFULL + s), kc * 64, rrow);
-          tma_load_2d(smem_u32(sR + s * RST + RHALF), &tmr, bar(B_RFULL + s), kc * 64, rrow + D2);
+          tma_load_2d_pol(smem_u32(sR + s * RST), &tmr, bar(B_RFULL + s), kc * 64, rrow, pol_last);
+          tma_load_2d_pol(smem_u32(sR + s * RST + RHALF), &tmr, bar(B_RFULL + s), kc * 64, rrow + D2, pol_last);
           ++nr;
         }
         if (!ok) break;
