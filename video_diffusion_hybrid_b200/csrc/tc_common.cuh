@@ -362,7 +362,7 @@ static __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // TMA into this CTA's shared memory, bytes counted on a barrier of either
-// CTA of the pair (no multicast)
+// CTA of the pair (the data lands in this CTA only)
 static __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cl, int x,
                                                         int y) {
   asm volatile(

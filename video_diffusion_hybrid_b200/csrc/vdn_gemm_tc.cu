@@ -29,7 +29,7 @@
 // The two accumulators let one tile's epilogue run under the next tile's
 // products.  Tiles go to the pairs round robin, columns fastest, so the pairs
 // running at one time share A row blocks and the whole weight in L2.
-// No load uses multicast: each CTA loads its own half.
+// Every load lands in the issuing CTA alone: each CTA loads its own half.
 //
 // Every wait is bounded; on expiry the CTA records VDN_ERR_TIMEOUT and
 // VDN_TAG_PROJ in the projection's status words (a library-owned device array,
