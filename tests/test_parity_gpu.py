@@ -347,6 +347,33 @@ def test_stages_compose_to_full_call_and_are_deterministic():
     assert np.array_equal(y, ha.y.float().cpu().numpy())
 
 
+@pytest.mark.parametrize("d", [128, 256])
+def test_text_stage_beside_frame_write_is_exact(d):
+    """A problem large enough (B*T*H >= 1024, text tokens present) that one
+    call runs the text stage on a stream of its own beside the frame write:
+    the result must equal, bit for bit, the stages called one at a time (the
+    text stage alone never forks), over the VDA stages and at d = 128 the
+    whole core too."""
+    shape = Shape(1, 45, 16, 24, d, d, 8)
+    assert shape.B * shape.T * shape.H >= 1024
+    stages = L.STAGE_ALL if d == 128 else VDA
+    inp, cfg, ha, t, y = run(shape, "bf16", 41, stages=stages)
+    ha.y.zero_()
+    for st in (L.STAGE_TEXT, L.STAGE_SOLVE, L.STAGE_SCAN, L.STAGE_SOFTMAX, L.STAGE_READ):
+        if st & stages:
+            ha(t, stages=st)
+    torch.cuda.synchronize()
+    y2 = ha.y.float().cpu().numpy()
+    if d == 128:
+        assert np.array_equal(y, y2)
+    else:
+        # the VDA stages write the linear slot only (slot 0 is left as it was)
+        assert np.array_equal(y[..., 1, :], y2[..., 1, :])
+    # and the linear slot against the oracle
+    ref = O.hybrid_attn(inp, ocfg(cfg))
+    assert rel_err(y[..., 1, :], ref[..., 1, :]) <= TOL["bf16"]
+
+
 def _sample_rows(cfg, heads, per_head, rng):
     T, N = cfg.T, cfg.N
     rows = []
